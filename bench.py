@@ -1,0 +1,427 @@
+#!/usr/bin/env python
+"""Benchmark of the QLoRA NF4 linear layer on B200.
+
+One step = forward + backward of the Llama-7B-shaped q_proj workload
+(X [4096 tokens, 4096] bf16, W 4096x4096 in NF4 with double quantization,
+LoRA r = 16, alpha = 32): qlora_linear_fwd then qlora_linear_bwd through the
+C ABI, all inputs resident in HBM.  The metric is algorithmic TFLOP/s
+(4MNK + 6Mr(K+N) per step; no gradient for W).  L2 is flushed (a 256 MB write)
+between timed steps; each step is timed with CUDA events on the launching
+stream and the per-step times are summed.
+
+Also reported: the fused dequant-GEMM kernel against the tensor-core roofline
+(events around each launch), the decode GEMV weight stream (70B-shaped up
+projection, 1/4/16 tokens) and nf4_quantize against HBM bandwidth, an
+end-to-end number with host buffers (pinned host -> device copies of X and dY,
+device -> host copies of Y, dX, dA, dB inside the timed region), SM clocks
+sampled through NVML during the timed region, and the CPU oracle timed on the
+host cores on a bounded sample.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun, one rank per GPU) every rank runs the same step on its
+own tokens (weak scaling) and the adapter gradients dA, dB are all-reduced
+over NCCL each step, as data-parallel training of the adapters requires.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s and NF4 weight-stream GB/s on 1 B200; % roofline"
+WORKLOAD = "qproj_7b"
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def step_flops(M, N, K, r):
+    return 4 * M * N * K + 6 * M * r * (K + N)
+
+
+# ------------------------------------------------------------------ clocks
+
+
+class ClockSampler:
+    """Polls SM clock and throttle reasons of one GPU through NVML (read only)."""
+
+    def __init__(self, torch_device_index: int, period_s: float = 0.005):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self.ok = False
+        self.period = period_s
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(torch_device_index).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode() if isinstance(uuid, str) else uuid)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.err = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        names = {
+            "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+            "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+            "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for n, bit in names.items():
+                    if mask & bit and n not in ("gpu_idle",):
+                        self.reasons.add(n)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._stop = threading.Event()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+        return False
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# -------------------------------------------------------------- CPU oracle
+
+
+def oracle_sample(rows_sample: int = 48):
+    """Times the CPU oracle on a bounded sample of the workload: Y and dX for
+    `rows_sample` token rows, H, dH, dA, dB in full.  Returns (TFLOP/s, cores,
+    sample description, seconds)."""
+    import numpy as np
+
+    import oracle
+    from bit_nf4_quantized_24_b200 import workloads as wl
+    w = wl.WORKLOADS[WORKLOAD]
+    p = wl.draw_linear(w)
+    M, N, K, r = p["M"], p["N"], p["K"], p["r"]
+    oc, oa, od, _ = oracle.nf4_quantize(p["W"].numpy())
+    _, Wp = oracle.nf4_dequantize(oc, oa, od, N, K)
+    bits = wl.bf16_bits
+    X, A, B, dY = bits(p["X"]), bits(p["A"]), bits(p["B"]), bits(p["dY"])
+    rows = np.linspace(0, M - 1, rows_sample).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.linear_fwd(X, Wp, A, B, p["scale"], rows=rows)
+    oracle.linear_bwd(X, dY, Wp, A, B, p["scale"], rows=rows)
+    dt = time.perf_counter() - t0
+    S = len(rows)
+    flops = S * (2 * K * r + 2 * N * K + 2 * N * r)          # forward rows
+    flops += 2 * M * K * r + 2 * M * N * r                    # H, dH
+    flops += S * (2 * N * K + 2 * r * K)                      # dX rows
+    flops += 2 * r * K * M + 2 * N * r * M                    # dA, dB
+    desc = (f"{WORKLOAD} (M={M}, N={N}, K={K}, r={r}): Y and dX for {S} of {M} token rows, "
+            f"H, dH, dA, dB in full; fp64 oracle")
+    return flops / dt / 1e12, oracle.num_threads(), desc, dt
+
+
+# -------------------------------------------------------------- our arm
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from bit_nf4_quantized_24_b200 import build as qbuild
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    if rank == 0:
+        qbuild.build()
+    if world > 1:
+        dist.barrier()
+    from bit_nf4_quantized_24_b200 import binding as qb
+    from bit_nf4_quantized_24_b200 import workloads as wl
+
+    pk = peaks()
+    w = wl.WORKLOADS[WORKLOAD]
+    p = wl.draw_linear(w)
+    M, N, K, r, s = p["M"], p["N"], p["K"], p["r"], p["scale"]
+    dev = torch.device("cuda", local_rank)
+    q = qb.nf4_quantize(p["W"].to(dev))
+    X, A, B, dY = (p[k].to(dev) for k in ("X", "A", "B", "dY"))
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    dA = torch.empty(r, K, dtype=torch.bfloat16, device=dev)
+    dB = torch.empty(N, r, dtype=torch.bfloat16, device=dev)
+    H = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
+    wsf = torch.empty(qb.fwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+    wsb = torch.empty(qb.bwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    L = qb.lib()
+    import ctypes
+    f32 = ctypes.c_float
+    P = qb._ptr
+
+    def step():
+        st = qb._stream()
+        e = L.qlora_linear_fwd(P(q.codes), P(q.absmax_q), P(q.dq_scale), N, K, P(X), M, P(A), P(B), r, f32(s), P(Y),
+                               P(H), P(wsf), wsf.numel(), st)
+        if e:
+            raise qb.QloraError(e, "fwd")
+        e = L.qlora_linear_bwd(P(q.codes), P(q.absmax_q), P(q.dq_scale), N, K, P(X), P(dY), M, P(A), P(B), r, f32(s),
+                               P(H), P(dX), P(dA), P(dB), P(wsb), wsb.numel(), st)
+        if e:
+            raise qb.QloraError(e, "bwd")
+        if world > 1:
+            dist.all_reduce(dA)
+            dist.all_reduce(dB)
+
+    launches_per_step = 2 + 7  # fwd: rowdot, gemm; bwd: transpose, rowdot, gemm, 2x(coldot partial + reduce)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    K_steps = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K_steps)]
+    sampler = ClockSampler(local_rank)
+    trace = qb.GemmTrace(2 * K_steps)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with sampler, trace:
+        for i in range(K_steps):
+            flush.zero_()
+            ev[i][0].record()
+            step()
+            ev[i][1].record()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = sum(step_ms)
+    gemm_ms = trace.times_ms()
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    flops = step_flops(M, N, K, r)
+    value = flops * world * K_steps / (total_ms / 1e3) / 1e12
+
+    # dominant kernel: the fused dequant-GEMM, launched twice per step (forward, dX)
+    fwd_ms = gemm_ms[0::2]
+    bwd_ms = gemm_ms[1::2]
+    gemm_flops_fwd = 2 * M * N * K + 2 * M * N * r
+    gemm_flops_bwd = 2 * M * N * K + 2 * M * K * r
+    avg_ms = statistics.mean(gemm_ms) if gemm_ms else float("nan")
+    achieved = ((gemm_flops_fwd + gemm_flops_bwd) / 2) / (avg_ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(achieved / pk["bf16_tflops"], 4), "traffic": None,
+                "kernel": "k_nf4_gemm (fused NF4 dequant + tcgen05 GEMM, forward and dX launches)",
+                "peak_source": f"{pk['source']} bf16 burst (MEASURED_PEAKS.json)",
+                "fwd_ms": round(statistics.mean(fwd_ms), 4) if fwd_ms else None,
+                "dx_ms": round(statistics.mean(bwd_ms), 4) if bwd_ms else None}
+
+    # end to end through the C ABI with host buffers
+    Xh = p["X"].pin_memory()
+    dYh = p["dY"].pin_memory()
+    Yh = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
+    dXh = torch.empty(M, K, dtype=torch.bfloat16).pin_memory()
+    dAh = torch.empty(r, K, dtype=torch.bfloat16).pin_memory()
+    dBh = torch.empty(N, r, dtype=torch.bfloat16).pin_memory()
+
+    def e2e_step():
+        X.copy_(Xh, non_blocking=True)
+        dY.copy_(dYh, non_blocking=True)
+        step()
+        Yh.copy_(Y, non_blocking=True)
+        dXh.copy_(dX, non_blocking=True)
+        dAh.copy_(dA, non_blocking=True)
+        dBh.copy_(dB, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    n_e2e = max(3, min(K_steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e0.record()
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": round(flops * world * n_e2e / (e2e_ms / 1e3) / 1e12, 3), "unit": "TFLOP/s",
+           "h2d_bytes_per_step": Xh.numel() * 2 + dYh.numel() * 2,
+           "d2h_bytes_per_step": (Yh.numel() + dXh.numel() + dAh.numel() + dBh.numel()) * 2,
+           "steps": n_e2e}
+
+    extra = {}
+    if not args.no_extras:
+        extra = run_extras(qb, wl, dev, pk, flush)
+
+    status = qb.device_status()
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": K_steps,
+        "warmup": args.warmup, "ms_per_step": round(total_ms / K_steps, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; see workloads.py)",
+        "config": {"workload": f"{WORKLOAD}: Llama-7B q_proj fwd+bwd, M=4096 tokens (4x1024), N=K=4096, "
+                               f"NF4 block 64 + 8-bit double quant (group 256), LoRA r=16 alpha=32",
+                   "M": M, "N": N, "K": K, "r": r, "global_batch_tokens": M * world,
+                   "parallelism": f"dp{world} (adapter grads all-reduced)" if world > 1 else "single GPU",
+                   "l2": "flushed between timed steps (256 MB write)"},
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * K_steps,
+        "clocks": sampler.summary(),
+        "extra": extra,
+        "device_status": status,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu:
+        tf, cores, desc, dt = oracle_sample()
+        out["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc,
+                               "seconds": round(dt, 2)}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_extras(qb, wl, dev, pk, flush):
+    """Decode GEMV weight stream, quantize and dequantize bandwidth."""
+    import torch
+    res = {}
+
+    def timed(fn, n=20, flush_between=True):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(n):
+            if flush_between:
+                flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        return statistics.median([a.elapsed_time(b) for a, b in ts])
+
+    # decode: 70B-shaped up projection, 1 / 4 / 16 tokens
+    w = wl.WORKLOADS["decode_70b_up"]
+    p = wl.draw_linear(w, M=16)
+    Wd = p["W"].to(dev)
+    q = qb.nf4_quantize(Wd)
+    N, K, r, s = p["N"], p["K"], p["r"], p["scale"]
+    weight_bytes = q.codes.numel() + q.absmax_q.numel() + 4 * q.dq_scale.numel()
+    A, B = p["A"].to(dev), p["B"].to(dev)
+    dec = {}
+    for M in (1, 4, 16):
+        X = p["X"][:M].contiguous().to(dev)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(qb.fwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+        ms = timed(lambda: qb.qlora_linear_fwd(q, X, A, B, s, save_h=False, out=Y, workspace=ws))
+        total_bytes = weight_bytes + 2 * r * (K + N) + 2 * M * (K + N)
+        dec[f"M{M}"] = {"us": round(ms * 1e3, 2), "weight_stream_gbs": round(weight_bytes / ms / 1e6, 1),
+                        "total_gbs": round(total_bytes / ms / 1e6, 1),
+                        "frac_hbm": round(total_bytes / ms / 1e6 / pk["hbm_gbs"], 4)}
+    res["decode_70b_up"] = dec
+    # quantize of the same weight (4 B read + 0.516 B written per weight)
+    numel = N * K
+    qbytes = 4 * numel + numel // 2 + numel // 64 + 4 * ((numel // 64 + 255) // 256)
+    ms = timed(lambda: qb.nf4_quantize(Wd), n=5)
+    res["nf4_quantize"] = {"ms": round(ms, 4), "gbs": round(qbytes / ms / 1e6, 1),
+                           "frac_hbm": round(qbytes / ms / 1e6 / pk["hbm_gbs"], 4),
+                           "note": "includes the call's stream synchronization (non-finite check)"}
+    out = torch.empty(N, K, dtype=torch.bfloat16, device=dev)
+    dbytes = numel // 2 + numel // 64 + 4 * ((numel // 64 + 255) // 256) + 2 * numel
+    ms = timed(lambda: qb.nf4_dequantize(q, out=out), n=10)
+    res["nf4_dequantize"] = {"ms": round(ms, 4), "gbs": round(dbytes / ms / 1e6, 1),
+                             "frac_hbm": round(dbytes / ms / 1e6 / pk["hbm_gbs"], 4)}
+    del Wd, out
+    torch.cuda.empty_cache()
+    return res
+
+
+# -------------------------------------------------------- reference arm
+
+
+def run_reference(args, rank, world):
+    """The reference arm is the CPU oracle (this method has no runnable
+    reference implementation): it is timed as it stands on the host cores."""
+    if rank != 0:
+        return
+    vals = []
+    cores = desc = None
+    for _ in range(max(1, args.steps if args.steps <= 3 else 3)):
+        tf, cores, desc, dt = oracle_sample(rows_sample=16)
+        vals.append(tf)
+    v = statistics.median(vals)
+    out = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
+           "steps": len(vals), "warmup": 0, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": "f64", "data": "synthetic (seeded; see workloads.py)",
+           "config": {"workload": f"{WORKLOAD} (bounded sample, see cpu_baseline.sample)"},
+           "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
+           "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extras", action="store_true", help="skip decode/quantize measurements")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,330 @@
+// The C ABI (include/qlora_nf4.h): argument checks, workspace layout, the
+// sequence of kernel launches for each call, device status and tracing.
+#include <climits>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+#include "qlora_nf4.h"
+
+namespace qn {
+
+// File-scope device words: the status of bounded waits, and nf4_quantize's
+// non-finite flag.  Every device that loads the library holds its own copy.
+__device__ int g_device_status;
+__device__ int g_nonfinite;
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+std::mutex g_quantize_mutex;
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices];
+int* g_nonfinite_ptr[kMaxDevices];
+std::mutex g_symbol_mutex;
+
+void** g_trace_events = nullptr;
+int g_trace_pairs = 0;
+int g_trace_count = 0;
+
+int current_device() {
+  int d = 0;
+  cudaGetDevice(&d);
+  return d;
+}
+
+template <typename T>
+T* symbol_ptr(T** cache, const void* symbol) {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_symbol_mutex);
+  if (!cache[d]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, symbol) != cudaSuccess) return nullptr;
+    cache[d] = static_cast<T*>(p);
+  }
+  return cache[d];
+}
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return QLORA_OK;
+  t_last_cuda_error = static_cast<int>(e);
+  return QLORA_ERR_CUDA;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Shape rules shared by the layer entry points.
+int check_layer_shapes(int64_t M, int64_t N, int64_t K, int r) {
+  if (M < 0 || N <= 0 || K <= 0) return QLORA_ERR_ARG;
+  if (r < 8 || r > 64 || r % 8) return r <= 0 ? QLORA_ERR_ARG : QLORA_ERR_UNSUPPORTED;
+  if (K % 64 || N % 8) return QLORA_ERR_SHAPE;
+  if (M > (1 << 24) || N > (1 << 24) || K > (1 << 24) || N * K / 2 > (int64_t(1) << 40)) return QLORA_ERR_SHAPE;
+  return QLORA_OK;
+}
+
+struct FwdWorkspace {
+  uint16_t* Hs;  // bf16(scale * X A^T) [M, r]
+  size_t bytes;
+};
+FwdWorkspace fwd_layout(void* ws, int64_t M, int r) {
+  FwdWorkspace w{};
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  w.Hs = reinterpret_cast<uint16_t*>(p);
+  w.bytes = align256(static_cast<size_t>(M) * r * 2);
+  if (w.bytes == 0) w.bytes = 256;
+  return w;
+}
+
+struct BwdWorkspace {
+  uint16_t* dH16;   // bf16(scale * dY B) [M, r]
+  uint16_t* Bt;     // lora_B transposed [r, N]
+  uint16_t* H16;    // bf16(X A^T) [M, r] when recomputed
+  float* partial;   // split partial sums of the column reductions
+  size_t bytes;
+};
+BwdWorkspace bwd_layout(void* ws, int64_t M, int64_t N, int64_t K, int r) {
+  BwdWorkspace w{};
+  size_t off = 0;
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  auto take = [&](size_t n) {
+    uint8_t* q = p ? p + off : nullptr;
+    off += align256(n);
+    return q;
+  };
+  w.dH16 = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(M) * r * 2));
+  w.Bt = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(N) * r * 2));
+  w.H16 = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(M) * r * 2));
+  const size_t pf = std::max(coldot_partial_floats(M, K, r), coldot_partial_floats(M, N, r));
+  w.partial = reinterpret_cast<float*>(take(std::max<size_t>(pf, static_cast<size_t>(r) * std::max(N, K)) * 4));
+  w.bytes = off;
+  return w;
+}
+
+}  // namespace
+
+int* device_status_ptr() { return symbol_ptr(g_status_ptr, &g_device_status); }
+int* device_nonfinite_ptr() { return symbol_ptr(g_nonfinite_ptr, &g_nonfinite); }
+
+void trace_before(cudaStream_t st) {
+  if (g_trace_events && g_trace_count < g_trace_pairs)
+    cudaEventRecord(static_cast<cudaEvent_t>(g_trace_events[2 * g_trace_count]), st);
+}
+void trace_after(cudaStream_t st) {
+  if (g_trace_events && g_trace_count < g_trace_pairs) {
+    cudaEventRecord(static_cast<cudaEvent_t>(g_trace_events[2 * g_trace_count + 1]), st);
+    ++g_trace_count;
+  }
+}
+
+}  // namespace qn
+
+using namespace qn;
+
+extern "C" {
+
+const char* qlora_status_string(int status) {
+  switch (status) {
+    case QLORA_OK: return "QLORA_OK";
+    case QLORA_ERR_ARG: return "QLORA_ERR_ARG: null pointer or invalid argument";
+    case QLORA_ERR_SHAPE: return "QLORA_ERR_SHAPE: unsupported or misaligned shape";
+    case QLORA_ERR_NONFINITE: return "QLORA_ERR_NONFINITE: the weight holds NaN or infinity";
+    case QLORA_ERR_WORKSPACE: return "QLORA_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case QLORA_ERR_CUDA: return "QLORA_ERR_CUDA: a CUDA call failed";
+    case QLORA_ERR_TIMEOUT: return "QLORA_ERR_TIMEOUT: a bounded device wait ran out";
+    case QLORA_ERR_UNSUPPORTED: return "QLORA_ERR_UNSUPPORTED: parameter outside this build's set";
+    default: return "QLORA_ERR_UNKNOWN";
+  }
+}
+
+int qlora_last_cuda_error(void) { return t_last_cuda_error; }
+
+int qlora_version(void) { return (1 << 16) | 0; }
+
+int nf4_quantized_sizes(int64_t N, int64_t K, int block, int dq_block, size_t* codes_bytes, size_t* absmax_bytes,
+                        size_t* dq_scale_bytes) {
+  if (N < 0 || K < 0 || !codes_bytes || !absmax_bytes || !dq_scale_bytes) return QLORA_ERR_ARG;
+  if (block != 64 || dq_block != 256) return QLORA_ERR_UNSUPPORTED;
+  if (K % block) return QLORA_ERR_SHAPE;
+  const int64_t numel = N * K, nblocks = numel / block;
+  *codes_bytes = static_cast<size_t>(numel / 2);
+  *absmax_bytes = static_cast<size_t>(nblocks);
+  *dq_scale_bytes = static_cast<size_t>((nblocks + dq_block - 1) / dq_block) * 4;
+  return QLORA_OK;
+}
+
+int nf4_codebook(float* levels_out) {
+  if (!levels_out) return QLORA_ERR_ARG;
+  std::memcpy(levels_out, host_codebook().levels.v, sizeof(float) * 16);
+  return QLORA_OK;
+}
+
+int nf4_quantize(const float* W, int64_t N, int64_t K, int block, int dq_block, uint8_t* codes,
+                 uint8_t* absmax_q, float* dq_scale, void* stream) {
+  size_t cb, ab, db;
+  int st = nf4_quantized_sizes(N, K, block, dq_block, &cb, &ab, &db);
+  if (st) return st;
+  if (N * K == 0) return QLORA_OK;
+  if (!W || !codes || !absmax_q || !dq_scale) return QLORA_ERR_ARG;
+  if (!aligned(W, 16) || !aligned(codes, 4)) return QLORA_ERR_SHAPE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(g_quantize_mutex);
+  int* flag = device_nonfinite_ptr();
+  if (!flag) return cuda_status(cudaErrorInvalidSymbol);
+  cudaError_t e = cudaMemsetAsync(flag, 0, sizeof(int), s);
+  if (e == cudaSuccess) e = launch_quantize(W, N * K, codes, absmax_q, dq_scale, flag, s);
+  int host_flag = 0;
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&host_flag, flag, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_status(e);
+  return host_flag ? QLORA_ERR_NONFINITE : QLORA_OK;
+}
+
+int nf4_dequantize(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale, int64_t N, int64_t K,
+                   int block, int dq_block, qlora_bf16_t* W_out, void* stream) {
+  size_t cb, ab, db;
+  int st = nf4_quantized_sizes(N, K, block, dq_block, &cb, &ab, &db);
+  if (st) return st;
+  if (N * K == 0) return QLORA_OK;
+  if (!codes || !absmax_q || !dq_scale || !W_out) return QLORA_ERR_ARG;
+  if (!aligned(codes, 16) || !aligned(W_out, 16)) return QLORA_ERR_SHAPE;
+  return cuda_status(launch_dequantize(codes, absmax_q, dq_scale, N * K, W_out, static_cast<cudaStream_t>(stream)));
+}
+
+int qlora_linear_fwd_workspace(int64_t M, int64_t N, int64_t K, int r, size_t* bytes) {
+  if (!bytes) return QLORA_ERR_ARG;
+  int st = check_layer_shapes(M, N, K, r);
+  if (st) return st;
+  *bytes = fwd_layout(nullptr, M, r).bytes;
+  return QLORA_OK;
+}
+
+int qlora_linear_bwd_workspace(int64_t M, int64_t N, int64_t K, int r, size_t* bytes) {
+  if (!bytes) return QLORA_ERR_ARG;
+  int st = check_layer_shapes(M, N, K, r);
+  if (st) return st;
+  *bytes = bwd_layout(nullptr, M, N, K, r).bytes;
+  return QLORA_OK;
+}
+
+int qlora_linear_fwd(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale, int64_t N, int64_t K,
+                     const qlora_bf16_t* X, int64_t M, const qlora_bf16_t* A, const qlora_bf16_t* B, int r,
+                     float scale, qlora_bf16_t* Y, qlora_bf16_t* H_save, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  int st = check_layer_shapes(M, N, K, r);
+  if (st) return st;
+  if (!codes || !absmax_q || !dq_scale || !A || !B || (M > 0 && (!X || !Y))) return QLORA_ERR_ARG;
+  if (!std::isfinite(scale)) return QLORA_ERR_ARG;
+  if (M == 0) return QLORA_OK;
+  const void* ptrs[] = {codes, X, A, B, Y};
+  for (const void* p : ptrs)
+    if (!aligned(p, 16)) return QLORA_ERR_SHAPE;
+  if (H_save && !aligned(H_save, 16)) return QLORA_ERR_SHAPE;
+  FwdWorkspace w = fwd_layout(workspace, M, r);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < w.bytes) return QLORA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  cudaError_t e = launch_rowdot(X, A, M, K, r, scale, w.Hs, 1.0f, H_save, nullptr, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (M <= 16) {
+    e = launch_gemv(X, M, codes, absmax_q, dq_scale, N, K, w.Hs, B, r, Y, s);
+  } else {
+    GemmArgs a{};
+    a.mode = 0;
+    a.act = X;
+    a.tail_a = w.Hs;
+    a.tail_b = B;
+    a.codes = codes;
+    a.absmax_q = absmax_q;
+    a.dq_scale = dq_scale;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.r = r;
+    a.out = Y;
+    e = launch_nf4_gemm(a, s);
+  }
+  return cuda_status(e);
+}
+
+int qlora_linear_bwd(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale, int64_t N, int64_t K,
+                     const qlora_bf16_t* X, const qlora_bf16_t* dY, int64_t M, const qlora_bf16_t* A,
+                     const qlora_bf16_t* B, int r, float scale, const qlora_bf16_t* H, qlora_bf16_t* dX,
+                     qlora_bf16_t* dA, qlora_bf16_t* dB, void* workspace, size_t workspace_bytes, void* stream) {
+  int st = check_layer_shapes(M, N, K, r);
+  if (st) return st;
+  if (!codes || !absmax_q || !dq_scale || !A || !B || !dA || !dB || (M > 0 && (!X || !dY)))
+    return QLORA_ERR_ARG;
+  if (!std::isfinite(scale)) return QLORA_ERR_ARG;
+  const void* ptrs[] = {codes, A, B, dA, dB};
+  for (const void* p : ptrs)
+    if (!aligned(p, 16)) return QLORA_ERR_SHAPE;
+  if ((X && !aligned(X, 16)) || (dY && !aligned(dY, 16)) || (dX && !aligned(dX, 16)) || (H && !aligned(H, 16)))
+    return QLORA_ERR_SHAPE;
+  BwdWorkspace w = bwd_layout(workspace, M, N, K, r);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < w.bytes) return QLORA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  cudaError_t e = cudaSuccess;
+  if (M == 0) {  // no tokens: zero adapter gradients
+    e = cudaMemsetAsync(dA, 0, static_cast<size_t>(r) * K * 2, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dB, 0, static_cast<size_t>(N) * r * 2, s);
+    return cuda_status(e);
+  }
+  // dH = scale * dY B  (B^T staged so the contraction dim is contiguous)
+  e = launch_transpose_bf16(B, N, r, w.Bt, s);
+  if (e == cudaSuccess) e = launch_rowdot(dY, w.Bt, M, N, r, scale, w.dH16, scale, nullptr, nullptr, s);
+  const uint16_t* Huse = H;
+  if (e == cudaSuccess && !H) {
+    e = launch_rowdot(X, A, M, K, r, 1.0f, w.H16, 1.0f, nullptr, nullptr, s);
+    Huse = w.H16;
+  }
+  // dX = dY deq(W) + dH A
+  if (e == cudaSuccess && dX) {
+    GemmArgs a{};
+    a.mode = 1;
+    a.act = dY;
+    a.tail_a = w.dH16;
+    a.tail_b = A;
+    a.codes = codes;
+    a.absmax_q = absmax_q;
+    a.dq_scale = dq_scale;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.r = r;
+    a.out = dX;
+    e = launch_nf4_gemm(a, s);
+  }
+  // dA = dH^T X ;  dB = scale * dY^T H
+  if (e == cudaSuccess) e = launch_coldot(w.dH16, X, M, K, r, 1.0f, 0, w.partial, dA, s);
+  if (e == cudaSuccess) e = launch_coldot(Huse, dY, M, N, r, scale, 1, w.partial, dB, s);
+  return cuda_status(e);
+}
+
+int qlora_device_status(void) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_status(e);
+  int* p = device_status_ptr();
+  if (!p) return cuda_status(cudaErrorInvalidSymbol);
+  int v = 0;
+  e = cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(p, 0, sizeof(int));
+  if (e != cudaSuccess) return cuda_status(e);
+  return v == kDevTimeout ? QLORA_ERR_TIMEOUT : QLORA_OK;
+}
+
+int qlora_trace_gemm_events(void** events, int n_pairs) {
+  if (n_pairs < 0 || (n_pairs > 0 && !events)) return QLORA_ERR_ARG;
+  g_trace_events = n_pairs > 0 ? events : nullptr;
+  g_trace_pairs = n_pairs;
+  g_trace_count = 0;
+  return QLORA_OK;
+}
+
+int qlora_trace_gemm_count(void) { return g_trace_count; }
+
+}  // extern "C"

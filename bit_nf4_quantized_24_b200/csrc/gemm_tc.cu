@@ -1,0 +1,355 @@
+// Fused NF4-dequant GEMM on the sm_100a tensor cores (tcgen05 + TMEM).
+//
+// "At runtime, the kernel dequantizes a block back to the compute dtype, does
+// the matmul, and discards the dequantized copy" -- katajob, "NF4: 4-bit
+// NormalFloat".  Here the dequantized weight tile exists only in shared
+// memory, one pipeline stage at a time, as the B operand of tcgen05.mma.
+//
+// Tile: 128 tokens (M) x 256 outputs (N) x 64 contraction (K) per stage.
+//   mode 0, forward:  D[m, n] = sum_k X[m,k] W'[n,k]       (W' K-major)
+//   mode 1, dX:       D[m, k] = sum_n dY[m,n] W'[n,k]      (W' MN-major)
+// followed by one tail stage that adds the LoRA product from bf16 operands
+// loaded by TMA: Hs B^T (forward, Hs = s*H) or dH A (dX).
+//
+// Warp roles (320 threads):
+//   warp 0      TMA producer: activation tile + NF4 code tile per stage
+//   warp 1      TMEM allocator and single-thread MMA issuer
+//   warps 2..9  dequantizers (one 64-weight block per thread per stage:
+//               register lookup table -> 128 B of swizzled bf16 in smem),
+//               then the epilogue (TMEM -> registers -> bf16 -> global)
+// Every wait is bounded (kWaitLimitNs); on expiry the kernel records
+// kDevTimeout, drains its in-flight copies and MMAs, frees TMEM and exits.
+#include <mutex>
+
+#include "internal.h"
+
+namespace qn {
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;     // 16 KB
+constexpr int B_BYTES = BN * BK * 2;     // 32 KB
+constexpr int C_BYTES = BN * BK / 2;     // 8 KB of packed codes
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+constexpr int OFF_C = OFF_B + STAGES * B_BYTES;
+constexpr int OFF_BAR = OFF_C + STAGES * C_BYTES;
+constexpr int SMEM_USED = OFF_BAR + 256;
+constexpr int SMEM_ALLOC = SMEM_USED + 1024;  // slack for 1024-byte alignment
+constexpr int NUM_THREADS = 320;
+constexpr int TMEM_COLS = 256;
+
+static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+
+struct Bars {
+  uint64_t full_tma[STAGES];  // activation + code tiles landed (tx bytes)
+  uint64_t full_deq[STAGES];  // 8 dequant warps finished the B tile
+  uint64_t empty[STAGES];     // MMAs of the stage completed
+  uint64_t accum;             // all MMAs completed
+  uint64_t drain;             // used only when aborting
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    k_nf4_gemm(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_codes,
+               const __grid_constant__ CUtensorMap tm_tail_a, const __grid_constant__ CUtensorMap tm_tail_b,
+               const uint8_t* __restrict__ absmax_q, const float* __restrict__ dq_scale, Nf4Levels lv, int M, int N,
+               int K, int r, __nv_bfloat16* __restrict__ out, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  Bars* bars = reinterpret_cast<Bars*>(base_ptr + OFF_BAR);
+  const uint32_t bar0 = base + OFF_BAR;
+  auto full_tma = [&](int s) { return bar0 + 8u * s; };
+  auto full_deq = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto empty = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
+  const uint32_t accum_bar = bar0 + 8u * (3 * STAGES);
+  const uint32_t drain_bar = bar0 + 8u * (3 * STAGES + 1);
+  volatile int* abort = &bars->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // mode 0: contraction K, outputs N.  mode 1: contraction N, outputs K.
+  const int Kc = MODE == 0 ? K : N;
+  const int Nout = MODE == 0 ? N : K;
+  const int numK = (Kc + BK - 1) / BK;
+  const int n0 = blockIdx.x * BN;  // first output column of the tile
+  const int m0 = blockIdx.y * BM;  // first token of the tile
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_tma(s), 1);
+      mbar_init(full_deq(s), 8);
+      mbar_init(empty(s), 1);
+    }
+    mbar_init(accum_bar, 1);
+    mbar_init(drain_bar, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_act);
+    tma_prefetch_desc(&tm_codes);
+    tma_prefetch_desc(&tm_tail_a);
+    tma_prefetch_desc(&tm_tail_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(base + OFF_BAR + static_cast<uint32_t>(offsetof(Bars, tmem_base)), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      bool ok = true;
+      for (int it = 0; it < numK && ok; ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!(ok = wait_bounded(empty(s), ph ^ 1, abort, status))) break;
+        mbar_arrive_expect_tx(full_tma(s), A_BYTES + C_BYTES);
+        tma_load_2d(base + OFF_A + s * A_BYTES, &tm_act, full_tma(s), it * BK, m0);
+        if (MODE == 0)
+          tma_load_2d(base + OFF_C + s * C_BYTES, &tm_codes, full_tma(s), it * (BK / 2), n0);
+        else
+          tma_load_2d(base + OFF_C + s * C_BYTES, &tm_codes, full_tma(s), n0 / 2, it * BK);
+        ++issued;
+      }
+      if (ok) {  // tail stage: LoRA operands
+        const int it = numK, s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if ((ok = wait_bounded(empty(s), ph ^ 1, abort, status))) {
+          mbar_arrive_expect_tx(full_tma(s), A_BYTES + B_BYTES);
+          tma_load_2d(base + OFF_A + s * A_BYTES, &tm_tail_a, full_tma(s), 0, m0);
+          if (MODE == 0) {
+            tma_load_2d(base + OFF_B + s * B_BYTES, &tm_tail_b, full_tma(s), 0, n0);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_2d(base + OFF_B + s * B_BYTES + j * 8192, &tm_tail_b, full_tma(s), n0 + 64 * j, 0);
+          }
+          ++issued;
+        }
+      }
+      if (!ok) {  // let the copies already issued land before the CTA exits
+        for (int it = (issued > STAGES ? issued - STAGES : 0); it < issued; ++it)
+          wait_drain(full_tma(it % STAGES), (it / STAGES) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(BM, BN, false, MODE == 1);
+      bool ok = true;
+      int committed = 0;
+      for (int it = 0; it <= numK; ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        const bool tail = (it == numK);
+        if (!(ok = wait_bounded(full_tma(s), ph, abort, status))) break;
+        if (!tail && !(ok = wait_bounded(full_deq(s), ph, abort, status))) break;
+        tc_fence_after();
+        const uint32_t a_s = base + OFF_A + s * A_BYTES;
+        const uint32_t b_s = base + OFF_B + s * B_BYTES;
+        const int nk = tail ? (r + 15) / 16 : BK / 16;
+        for (int kk = 0; kk < nk; ++kk) {
+          const uint64_t ad = desc_sw128(a_s + kk * 32, 16, 1024);
+          const uint64_t bd = MODE == 0 ? desc_sw128(b_s + kk * 32, 16, 1024)
+                                        : desc_sw128(b_s + kk * 2048, 8192, 1024);
+          tc_mma_f16(tmem, ad, bd, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(empty(s));
+        committed = 1;
+      }
+      if (ok) {
+        tc_commit(accum_bar);
+      } else if (committed) {  // wait for MMAs in flight before TMEM is freed
+        tc_commit(drain_bar);
+        wait_drain(drain_bar, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------- dequantizers, then epilogue
+    const int t = threadIdx.x - 64;  // 0..255
+    bool ok = true;
+    const int KB = K / 64;           // 64-blocks per weight row
+    for (int it = 0; it < numK; ++it) {
+      const int s = it % STAGES;
+      const uint32_t ph = (it / STAGES) & 1;
+      // which (row, 64-block) of W this thread expands, and where it goes
+      int wrow, kcol0, srow;
+      if (MODE == 0) {
+        wrow = n0 + t;
+        kcol0 = it * BK;
+        srow = t;
+      } else {
+        wrow = it * BK + (t & 63);
+        kcol0 = n0 + 64 * (t >> 6);
+        srow = t;  // = 64 * (t >> 6) + (t & 63): sub-tile j holds outputs n0+64j..
+      }
+      const bool valid = (wrow < N) && (kcol0 < K);
+      float ap = 0.0f;
+      if (valid) {
+        const int64_t blk = static_cast<int64_t>(wrow) * KB + (kcol0 >> 6);
+        ap = __fmul_rn(static_cast<float>(__ldg(absmax_q + blk)), __ldg(dq_scale + (blk >> 8)));
+      }
+      if (!(ok = wait_bounded(full_tma(s), ph, abort, status))) break;
+      const uint32_t c_s = base + OFF_C + s * C_BYTES;
+      uint4 q0, q1;
+      if (MODE == 0) {  // code tile [256 rows][32 B], 32-byte swizzle
+        const uint32_t sw = (static_cast<uint32_t>(t) >> 2) & 1u;
+        q0 = ld_shared_v4(c_s + t * 32 + ((0u ^ sw) << 4));
+        q1 = ld_shared_v4(c_s + t * 32 + ((1u ^ sw) << 4));
+      } else {          // code tile [64 rows][128 B], 128-byte swizzle
+        const uint32_t row = t & 63, j = t >> 6;
+        q0 = ld_shared_v4(c_s + row * 128 + (((2 * j) ^ (row & 7)) << 4));
+        q1 = ld_shared_v4(c_s + row * 128 + (((2 * j + 1) ^ (row & 7)) << 4));
+      }
+      const uint32_t b_row = base + OFF_B + s * B_BYTES + srow * 128;
+      const uint32_t sw = srow & 7;
+      if (valid) {
+        const Nf4Lut lut = make_lut(lv, ap);
+        const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t o0, o1, o2, o3;
+          deq8(w[c], lut, o0, o1, o2, o3);
+          st_shared_v4(b_row + ((c ^ sw) << 4), o0, o1, o2, o3);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) st_shared_v4(b_row + (c << 4), 0u, 0u, 0u, 0u);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(full_deq(s));
+    }
+
+    // -------------------------------------------------------- epilogue
+    if (ok) ok = wait_bounded(accum_bar, 0, abort, status);
+    if (ok) {
+      tc_fence_after();
+      const int quad = warp & 3;                 // TMEM lanes 32*quad .. +31
+      const int colh = (warp - 2) >> 2;          // column half: 0 or 1
+      const int m = m0 + quad * 32 + lane;
+#pragma unroll 1
+      for (int cc = 0; cc < BN / 2; cc += 32) {
+        const int col = colh * (BN / 2) + cc;
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(col), v);
+        tmem_ld_wait();
+        const int n = n0 + col;
+        if (m < M && n < Nout) {
+          uint4* dst = reinterpret_cast<uint4*>(out + static_cast<int64_t>(m) * Nout + n);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (n + 8 * q < Nout) {
+              uint4 o;
+              o.x = bf16x2_bits(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
+              o.y = bf16x2_bits(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
+              o.z = bf16x2_bits(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
+              o.w = bf16x2_bits(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
+              dst[q] = o;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------ host side
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2D row-major map: inner dimension `inner` elements, `outer` rows, row
+// pitch `pitch_bytes`; box {box_inner, box_outer}.
+bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* ptr, uint64_t inner, uint64_t outer,
+              uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {pitch_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE>
+cudaError_t launch_mode(const GemmArgs& a, cudaStream_t st) {
+  const int64_t Kc = MODE == 0 ? a.K : a.N;
+  const int64_t Nout = MODE == 0 ? a.N : a.K;
+  CUtensorMap tm_act, tm_codes, tm_ta, tm_tb;
+  const auto BF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  bool ok = make_map(&tm_act, BF16, a.act, Kc, a.M, Kc * 2, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (MODE == 0)
+    ok = ok && make_map(&tm_codes, U8, a.codes, a.K / 2, a.N, a.K / 2, BK / 2, BN, CU_TENSOR_MAP_SWIZZLE_32B);
+  else
+    ok = ok && make_map(&tm_codes, U8, a.codes, a.K / 2, a.N, a.K / 2, BN / 2, BK, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok = ok && make_map(&tm_ta, BF16, a.tail_a, a.r, a.M, a.r * 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (MODE == 0)
+    ok = ok && make_map(&tm_tb, BF16, a.tail_b, a.r, a.N, a.r * 2, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+  else
+    ok = ok && make_map(&tm_tb, BF16, a.tail_b, a.K, a.r, a.K * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return cudaErrorInvalidValue;
+
+  static std::once_flag attr_once[2];
+  cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once[MODE], [&] {
+    attr_err = cudaFuncSetAttribute(k_nf4_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  // The attribute is per device; set it again cheaply on every launch so a
+  // second device is covered too.
+  cudaError_t e = cudaFuncSetAttribute(k_nf4_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+  if (e != cudaSuccess) return e;
+
+  const dim3 grid(static_cast<unsigned>((Nout + BN - 1) / BN), static_cast<unsigned>((a.M + BM - 1) / BM));
+  trace_before(st);
+  k_nf4_gemm<MODE><<<grid, NUM_THREADS, SMEM_ALLOC, st>>>(
+      tm_act, tm_codes, tm_ta, tm_tb, a.absmax_q, a.dq_scale, host_codebook().levels, static_cast<int>(a.M),
+      static_cast<int>(a.N), static_cast<int>(a.K), a.r, reinterpret_cast<__nv_bfloat16*>(a.out),
+      device_status_ptr());
+  e = cudaGetLastError();
+  trace_after(st);
+  return e;
+}
+
+}  // namespace
+
+cudaError_t launch_nf4_gemm(const GemmArgs& a, cudaStream_t st) {
+  return a.mode == 0 ? launch_mode<0>(a, st) : launch_mode<1>(a, st);
+}
+
+}  // namespace qn

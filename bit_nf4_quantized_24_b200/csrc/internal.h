@@ -1,0 +1,72 @@
+// Launchers shared between the translation units of libqlora_nf4.so.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace qn {
+
+// Host-side NF4 table (computed once by codebook.cu).
+struct HostCodebook {
+  Nf4Levels levels;
+  Nf4Mids mids;
+};
+const HostCodebook& host_codebook();
+
+// Per-device status word (timeouts of bounded waits) and the non-finite
+// flag of nf4_quantize; both live in file-scope device memory.
+int* device_status_ptr();      // device address of the status word
+int* device_nonfinite_ptr();   // device address of the non-finite flag
+
+// ----- quantize / dequantize (HBM-bound)
+cudaError_t launch_quantize(const float* W, int64_t numel, uint8_t* codes, uint8_t* absmax_q,
+                            float* dq_scale, int* nonfinite, cudaStream_t st);
+cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale,
+                              int64_t numel, uint16_t* out, cudaStream_t st);
+
+// ----- fused dequant-GEMM on tcgen05 (tensor cores)
+// mode 0 (forward):  Y[M,N]  = X[M,K]  deq(W)^T + Ht[M,r] Bt^T, Bt = lora_B [N,r]
+// mode 1 (dX):       dX[M,K] = dY[M,N] deq(W)   + Ht[M,r] A,   A  = lora_A [r,K]
+// Ht is the bf16 tail operand (s*H for the forward, dH for dX).
+struct GemmArgs {
+  int mode;
+  const uint16_t* act;     // X or dY, bf16 [M, Kc]
+  const uint16_t* tail_a;  // bf16 [M, r]
+  const uint16_t* tail_b;  // lora_B [N, r] (mode 0) or lora_A [r, K] (mode 1)
+  const uint8_t* codes;
+  const uint8_t* absmax_q;
+  const float* dq_scale;
+  int64_t M, N, K;
+  int r;
+  uint16_t* out;  // Y [M, N] or dX [M, K]
+};
+cudaError_t launch_nf4_gemm(const GemmArgs& a, cudaStream_t st);
+
+// ----- adapter kernels
+// out[m, j] = sum_k P[m,k] Q[j,k]  (P bf16 [M, Kc], Q bf16 [R, Kc]); writes
+// out16a = bf16(sa * acc) [M,R], out16b = bf16(sb * acc) (nullable),
+// out32 = sb * acc fp32 (nullable).
+cudaError_t launch_rowdot(const uint16_t* P, const uint16_t* Q, int64_t M, int64_t Kc, int R, float sa,
+                          uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st);
+// out[j, c] = sum_m G[m, j] P[m, c] over all m (G bf16 [M, R], P bf16 [M, C]),
+// written as bf16(scale * out) either [R, C] (transpose = 0) or [C, R]
+// (transpose = 1).  partial: fp32 scratch of coldot_partial_floats(...) floats.
+size_t coldot_partial_floats(int64_t M, int64_t C, int R);
+cudaError_t launch_coldot(const uint16_t* G, const uint16_t* P, int64_t M, int64_t C, int R, float scale,
+                          int transpose, float* partial, uint16_t* out, cudaStream_t st);
+// dst[c, r] = src[r, c] for a bf16 [R, C] matrix.
+cudaError_t launch_transpose_bf16(const uint16_t* src, int64_t R, int64_t C, uint16_t* dst, cudaStream_t st);
+
+// ----- decode GEMV (M <= 16): Y = X deq(W)^T + Hs B^T, Hs = bf16(s X A^T)
+cudaError_t launch_gemv(const uint16_t* X, int64_t M, const uint8_t* codes, const uint8_t* absmax_q,
+                        const float* dq_scale, int64_t N, int64_t K, const uint16_t* Hs, const uint16_t* B, int r,
+                        uint16_t* Y, cudaStream_t st);
+
+// ----- tracing of the fused GEMM launches
+void trace_before(cudaStream_t st);
+void trace_after(cudaStream_t st);
+
+}  // namespace qn

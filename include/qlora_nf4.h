@@ -1,0 +1,171 @@
+/*
+ * qlora_nf4.h -- C ABI of the B200 (sm_100a) QLoRA frozen-NF4 linear layer.
+ *
+ * The operations follow the QLoRA pages (cited by title and section):
+ *  - "What does QLoRA change compared with plain LoRA when fine-tuning Llama?"
+ *    (katajob): "NF4: 4-bit NormalFloat" (16-level type for normally
+ *    distributed weights; per-block scaling over small groups of contiguous
+ *    weights, commonly 64; dequantized block by block to bf16 inside the
+ *    matmul and discarded), "Double quantization" (the per-block scales are
+ *    themselves quantized to 8 bits with a second-level scale over groups),
+ *    "What stays in full precision" (A, B are bf16; gradients reach them
+ *    through the dequantized base; the base gets no update).
+ *  - "QLoRA: fine-tuning a large model on one GPU" (pranaymahendrakar),
+ *    "LoRA, stated once": h = W0 x + (alpha/r) B A x with B in R^{d x r},
+ *    A in R^{r x k}.
+ *  - "QLoRA and Quantized Fine-Tuning" (quantmemo), "The two mechanisms
+ *    combined": W' = W_4bit + BA, only B and A are trained.
+ *
+ * Conventions shared by every entry point
+ *  - Types: bf16 tensors are passed as raw bit patterns (qlora_bf16_t =
+ *    uint16_t); fp32 as float; NF4 codes, absmax codes as uint8_t.
+ *  - Layout: every matrix is row-major and contiguous.  Weights are [N, K]
+ *    (out_features x in_features, the nn.Linear layout); X is [M, K];
+ *    Y and dY are [M, N]; LoRA A is [r, K] and B is [N, r].
+ *  - NF4 format (produced by nf4_quantize, consumed by everything else):
+ *      codes     uint8 [N*K/2]   element 2j in the low nibble of byte j,
+ *                                element 2j+1 in the high nibble; the code is
+ *                                the index (0..15) of the ascending level.
+ *      absmax_q  uint8 [N*K/block]      8-bit code of each block's absmax.
+ *      dq_scale  fp32  [ceil(N*K/block/dq_block)]  second-level scale of each
+ *                                group of dq_block consecutive blocks.
+ *    Blocks are `block` consecutive elements of the flattened weight (they
+ *    never straddle a row: K % block == 0).  This build supports
+ *    block == 64 and dq_block == 256 (other values: QLORA_ERR_UNSUPPORTED).
+ *  - Pointers: every tensor pointer is a DEVICE pointer of the current CUDA
+ *    device unless stated otherwise; the caller owns all memory.  The library
+ *    never frees or retains caller memory.
+ *  - Streams: `stream` is a cudaStream_t (NULL = legacy default stream).  All
+ *    device work is enqueued asynchronously on it; argument errors are
+ *    returned synchronously before anything is enqueued.
+ *  - Status: every function returns QLORA_OK (0) or a negative QLORA_ERR_*.
+ *    A launch failure returns QLORA_ERR_CUDA (the CUDA error is readable via
+ *    qlora_last_cuda_error()).
+ *  - Device-side waits inside the tensor-core kernels are bounded; a wait
+ *    that runs out records QLORA_ERR_TIMEOUT in a device status word that
+ *    qlora_device_status() reads (it synchronizes the device).
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t qlora_bf16_t;
+
+#define QLORA_OK 0
+#define QLORA_ERR_ARG (-1)         /* null pointer, negative size, bad r or scale */
+#define QLORA_ERR_SHAPE (-2)       /* K % block != 0, misaligned sizes */
+#define QLORA_ERR_NONFINITE (-3)   /* the weight holds a NaN or an infinity */
+#define QLORA_ERR_WORKSPACE (-4)   /* workspace null or smaller than required */
+#define QLORA_ERR_CUDA (-5)        /* a CUDA runtime call or launch failed */
+#define QLORA_ERR_TIMEOUT (-6)     /* a bounded device-side wait ran out */
+#define QLORA_ERR_UNSUPPORTED (-7) /* block/dq_block/r outside this build's set */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* qlora_status_string(int status);
+
+/* Last CUDA error code seen by the library on this host thread (0 if none). */
+int qlora_last_cuda_error(void);
+
+/* ABI version: (major << 16) | minor. */
+int qlora_version(void);
+
+/* Byte sizes of the three NF4 buffers of an [N, K] weight.
+ * Errors: QLORA_ERR_ARG (negative sizes, null outputs),
+ * QLORA_ERR_SHAPE (K % block != 0), QLORA_ERR_UNSUPPORTED. */
+int nf4_quantized_sizes(int64_t N, int64_t K, int block, int dq_block,
+                        size_t* codes_bytes, size_t* absmax_bytes, size_t* dq_scale_bytes);
+
+/* The 16 NF4 levels (fp32, ascending, HOST memory) this library encodes with.
+ * They are equal-probability quantiles of the standard normal on each side of
+ * an exact zero (8 positive, 7 negative), scaled to [-1, 1] (katajob,
+ * "NF4: 4-bit NormalFloat": levels optimal for a zero-centred normal).
+ * levels_out: host pointer to 16 floats.  Errors: QLORA_ERR_ARG. */
+int nf4_codebook(float* levels_out);
+
+/* Quantize an fp32 weight [N, K] to NF4 with double quantization (katajob,
+ * "NF4: 4-bit NormalFloat" and "Double quantization").  Per block b:
+ * a_b = max |w|; code = index of the nearest level to fl32(w / a_b) (ties at
+ * a midpoint take the lower code; an all-zero block encodes the zero level).
+ * Per group g of dq_block blocks: s2_g = fl32(max_b a_b / 255);
+ * absmax_q[b] = min(255, round_half_even(fl32(a_b / s2_g))) (0 if s2_g == 0).
+ * W: device fp32 [N, K]; codes, absmax_q, dq_scale: device outputs sized by
+ * nf4_quantized_sizes.  Synchronizes `stream` to report non-finite input:
+ * returns QLORA_ERR_NONFINITE if W holds a NaN or an infinity (the outputs are
+ * then unspecified).  Other errors: ARG, SHAPE, UNSUPPORTED, CUDA. */
+int nf4_quantize(const float* W, int64_t N, int64_t K, int block, int dq_block,
+                 uint8_t* codes, uint8_t* absmax_q, float* dq_scale, void* stream);
+
+/* Dequantize NF4 to bf16 (katajob, "NF4: 4-bit NormalFloat": the block is
+ * expanded to the compute dtype).  w' = bf16_rne(fl32(level[code] *
+ * fl32(absmax_q[b] * dq_scale[g]))).  W_out: device bf16 [N, K].
+ * Errors: ARG, SHAPE, UNSUPPORTED, CUDA. */
+int nf4_dequantize(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale,
+                   int64_t N, int64_t K, int block, int dq_block,
+                   qlora_bf16_t* W_out, void* stream);
+
+/* Workspace bytes needed by qlora_linear_fwd / qlora_linear_bwd for these
+ * shapes (the caller allocates it, 256-byte aligned, device memory). */
+int qlora_linear_fwd_workspace(int64_t M, int64_t N, int64_t K, int r, size_t* bytes);
+int qlora_linear_bwd_workspace(int64_t M, int64_t N, int64_t K, int r, size_t* bytes);
+
+/* Forward of the QLoRA linear ("QLoRA: fine-tuning a large model on one GPU",
+ * "LoRA, stated once"):
+ *     Y = X deq(W)^T + scale * (X A^T) B^T
+ * with deq(W) expanded to bf16 on the fly inside the tensor-core GEMM and
+ * never written to memory.  Accumulation is fp32; Y is rounded to bf16.
+ * X: bf16 [M, K]; A: bf16 [r, K]; B: bf16 [N, r]; Y: bf16 [M, N] output.
+ * H_save (nullable): bf16 [M, r] output receiving H = X A^T for the backward.
+ * scale = alpha / r.  1 <= r <= 64, r % 8 == 0; K % 64 == 0; N % 8 == 0.
+ * M <= 16 runs the bandwidth-bound decode kernel; larger M the tensor-core
+ * GEMM (one selection by shape, both exact to the same tolerance).
+ * workspace: device scratch of qlora_linear_fwd_workspace bytes.
+ * Errors: ARG, SHAPE, UNSUPPORTED, WORKSPACE, CUDA. */
+int qlora_linear_fwd(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale,
+                     int64_t N, int64_t K, const qlora_bf16_t* X, int64_t M,
+                     const qlora_bf16_t* A, const qlora_bf16_t* B, int r, float scale,
+                     qlora_bf16_t* Y, qlora_bf16_t* H_save,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward of the QLoRA linear: gradients flow through deq(W) to the
+ * adapters and to the input; the frozen base gets none (katajob, "What stays
+ * in full precision"):
+ *     dH = scale * dY B                 [M, r]
+ *     dX = dY deq(W) + dH A             [M, K]
+ *     dA = dH^T X                       [r, K]
+ *     dB = scale * dY^T H,  H = X A^T   [N, r]
+ * dY: bf16 [M, N].  H: bf16 [M, r] from qlora_linear_fwd's H_save, or NULL to
+ * recompute it.  dX, dA, dB: bf16 outputs (dX may be NULL to skip it).
+ * Same shape rules and errors as qlora_linear_fwd. */
+int qlora_linear_bwd(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale,
+                     int64_t N, int64_t K, const qlora_bf16_t* X, const qlora_bf16_t* dY,
+                     int64_t M, const qlora_bf16_t* A, const qlora_bf16_t* B, int r,
+                     float scale, const qlora_bf16_t* H,
+                     qlora_bf16_t* dX, qlora_bf16_t* dA, qlora_bf16_t* dB,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* Reads and clears the device status word of the current device (a
+ * QLORA_ERR_TIMEOUT left by a bounded wait, else QLORA_OK).  Synchronizes the
+ * device. */
+int qlora_device_status(void);
+
+/* Kernel-level tracing for profiling.  While enabled, each launch of the
+ * fused dequant-GEMM kernel (forward or dX) records events[2i] before and
+ * events[2i+1] after it on the launching stream, for i = 0, 1, ... up to
+ * n_pairs - 1 (later launches are not recorded).  `events` is a host array of
+ * cudaEvent_t owned by the caller; n_pairs = 0 disables tracing.  Not
+ * thread-safe: set it from one host thread.  Errors: ARG. */
+int qlora_trace_gemm_events(void** events, int n_pairs);
+
+/* Number of event pairs recorded since the last qlora_trace_gemm_events. */
+int qlora_trace_gemm_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QLORA_NF4_H */

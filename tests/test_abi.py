@@ -1,0 +1,70 @@
+"""The C-ABI library loads, exports every function the header declares, and
+rejects bad arguments before touching the GPU.  Runs without a GPU."""
+import ctypes
+
+import numpy as np
+import pytest
+
+from bit_nf4_quantized_24_b200 import binding as qb
+
+
+@pytest.fixture(scope="module")
+def L():
+    from bit_nf4_quantized_24_b200 import build
+    build.build()
+    return qb.lib()
+
+
+def test_exports_every_declared_function(L):
+    names = qb.header_functions()
+    for must in ["nf4_quantize", "nf4_dequantize", "qlora_linear_fwd", "qlora_linear_bwd", "nf4_quantized_sizes",
+                 "nf4_codebook", "qlora_linear_fwd_workspace", "qlora_linear_bwd_workspace"]:
+        assert must in names
+    for n in names:
+        assert hasattr(L, n), f"library does not export {n}"
+
+
+def test_status_strings_and_version(L):
+    for code in range(0, -8, -1):
+        assert qb.status_string(code).startswith(qb.STATUS[code])
+    assert qb.version() >> 16 == 1
+
+
+def test_codebook_matches_oracle_bit_for_bit(L, oracle):
+    """The library computes its table with its own code (Newton on erfc); the
+    oracle with bisection.  Both must round to the same fp32 levels."""
+    lib_levels = np.array(qb.nf4_codebook(), np.float32)
+    _, o32, _ = oracle.nf4_codebook()
+    assert lib_levels.tobytes() == o32.tobytes()
+
+
+def test_sizes_match_oracle_format(L, oracle):
+    for N, K in [(1, 64), (3, 192), (4096, 4096), (28672, 8192), (11008, 4096)]:
+        cb, ab, db = qb.nf4_quantized_sizes(N, K)
+        ocb, oab, odc = oracle.nf4_sizes(N, K)
+        assert (cb, ab, db) == (ocb, oab, 4 * odc)
+
+
+def test_argument_errors_return_before_any_device_work(L):
+    i = ctypes.c_size_t()
+    assert L.nf4_quantized_sizes(4, 96, 64, 256, ctypes.byref(i), ctypes.byref(i), ctypes.byref(i)) == -2
+    assert L.nf4_quantized_sizes(4, 128, 32, 256, ctypes.byref(i), ctypes.byref(i), ctypes.byref(i)) == -7
+    assert L.nf4_quantized_sizes(-1, 64, 64, 256, ctypes.byref(i), ctypes.byref(i), ctypes.byref(i)) == -1
+    assert L.nf4_codebook(None) == -1
+    assert L.qlora_linear_fwd_workspace(16, 64, 64, 12, ctypes.byref(i)) == -7
+    assert L.qlora_linear_fwd_workspace(16, 64, 64, 0, ctypes.byref(i)) == -1
+    assert L.qlora_linear_fwd_workspace(16, 64, 96, 16, ctypes.byref(i)) == -2
+    assert L.qlora_linear_bwd_workspace(16, 60, 64, 16, ctypes.byref(i)) == -2
+    # null tensors are rejected before any launch
+    assert L.qlora_linear_fwd(None, None, None, 64, 64, None, 16, None, None, 16, ctypes.c_float(2.0), None, None,
+                              None, 0, None) == -1
+    assert L.qlora_linear_bwd(None, None, None, 64, 64, None, None, 16, None, None, 16, ctypes.c_float(2.0), None,
+                              None, None, None, None, 0, None) == -1
+    assert L.qlora_trace_gemm_events(None, -1) == -1
+
+
+def test_workspace_sizes_grow_with_shape(L):
+    a = qb.fwd_workspace_bytes(128, 2048, 2048, 8)
+    b = qb.fwd_workspace_bytes(4096, 4096, 4096, 16)
+    assert 0 < a < b and a % 256 == 0 and b % 256 == 0
+    assert qb.bwd_workspace_bytes(4096, 4096, 4096, 16) > qb.bwd_workspace_bytes(128, 2048, 2048, 8)

@@ -1,0 +1,295 @@
+"""Parity of the CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+Bars: NF4 codes, absmax codes and double-quant scales bit-exact; dequantized
+bf16 weights bit-exact; Y, dX, dA, dB within a relative Frobenius error of 1e-2
+(the layer's stated tolerance; the expected error is the bf16 rounding of the
+outputs, ~3e-3).  Small cases span several tiles with ragged tails and are
+checked in full; the five workloads are checked at full size on sampled rows of
+Y and dX plus all of dA and dB, with the same launches the benchmark times.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from bit_nf4_quantized_24_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-2
+
+
+@pytest.fixture(scope="module")
+def qb():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from bit_nf4_quantized_24_b200 import binding, build
+    build.build()
+    binding.lib()
+    return binding
+
+
+def relfro(got, ref):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    d = np.linalg.norm(got - ref)
+    n = np.linalg.norm(ref)
+    return d / n if n > 0 else d
+
+
+def bits(t):
+    return wl.bf16_bits(t.cpu())
+
+
+def quantize_both(qb, oracle, W):
+    """GPU and oracle quantization of the same fp32 weight; asserts bit-exact."""
+    q = qb.nf4_quantize(W.cuda())
+    oc, oa, od, _ = oracle.nf4_quantize(W.numpy())
+    assert np.array_equal(q.codes.cpu().numpy(), oc), "NF4 codes differ"
+    assert np.array_equal(q.absmax_q.cpu().numpy(), oa), "absmax codes differ"
+    assert q.dq_scale.cpu().numpy().tobytes() == od.tobytes(), "double-quant scales differ"
+    _, Wp = oracle.nf4_dequantize(oc, oa, od, W.shape[0], W.shape[1])
+    return q, Wp
+
+
+def run_fwd_check(qb, oracle, p, rows=None, q=None, Wp=None):
+    if q is None:
+        q, Wp = quantize_both(qb, oracle, p["W"])
+    X, A, B = p["X"].cuda(), p["A"].cuda(), p["B"].cuda()
+    Y, H = qb.qlora_linear_fwd(q, X, A, B, p["scale"])
+    torch.cuda.synchronize()
+    Yref = oracle.linear_fwd(bits(p["X"]), Wp, bits(p["A"]), bits(p["B"]), p["scale"], rows=rows)
+    Yg = Y.float().cpu().numpy()
+    if rows is not None:
+        Yg = Yg[rows]
+    e = relfro(Yg, Yref)
+    assert e <= TOL, f"Y rel err {e}"
+    Href = oracle.lora_h(bits(p["X"][rows] if rows is not None else p["X"]), bits(p["A"]))
+    Hg = H.float().cpu().numpy()
+    eh = relfro(Hg[rows] if rows is not None else Hg, Href)
+    assert eh <= TOL, f"H rel err {eh}"
+    return e, q, Wp
+
+
+def run_bwd_check(qb, oracle, p, rows=None, q=None, Wp=None, use_saved_h=True):
+    if q is None:
+        q, Wp = quantize_both(qb, oracle, p["W"])
+    X, A, B, dY = p["X"].cuda(), p["A"].cuda(), p["B"].cuda(), p["dY"].cuda()
+    H = None
+    if use_saved_h:
+        _, H = qb.qlora_linear_fwd(q, X, A, B, p["scale"])
+    dX, dA, dB = qb.qlora_linear_bwd(q, X, dY, A, B, p["scale"], H=H)
+    torch.cuda.synchronize()
+    dXr, dAr, dBr, _ = oracle.linear_bwd(bits(p["X"]), bits(p["dY"]), Wp, bits(p["A"]), bits(p["B"]), p["scale"],
+                                         rows=rows)
+    dXg = dX.float().cpu().numpy()
+    if rows is not None:
+        dXg = dXg[rows]
+    errs = (relfro(dXg, dXr), relfro(dA.float().cpu().numpy(), dAr), relfro(dB.float().cpu().numpy(), dBr))
+    assert max(errs) <= TOL, f"dX/dA/dB rel err {errs}"
+    return errs
+
+
+# ------------------------------------------------------------------ codec
+
+
+@pytest.mark.parametrize("N,K,seed", [(1, 64, 0), (3, 192, 1), (5, 320, 2), (37, 4160, 3), (300, 1024, 4)])
+def test_quantize_bit_exact(qb, oracle, N, K, seed):
+    W = wl.draw_weight(wl.generator(seed), N, K, 0.02, 0.02)
+    W[0, :64] = 0.0                      # an all-zero block
+    if N > 2:
+        W[2, :] *= 1e-30                 # tiny magnitudes
+    quantize_both(qb, oracle, W)
+
+
+def test_quantize_codebook_values_and_ties(qb, oracle):
+    _, l32, m32 = oracle.nf4_codebook()
+    rows = []
+    for e in (-7, 0, 3):
+        idx = np.arange(64) % 16
+        rows.append(l32[idx] * np.float32(2.0 ** e))
+    for i in range(15):
+        r = np.zeros(64, np.float32)
+        r[0] = 1.0
+        r[1] = m32[i]
+        r[2] = np.nextafter(m32[i], np.float32(2))
+        r[3] = np.nextafter(m32[i], np.float32(-2))
+        r[4:] = np.float32(-1.0)
+        rows.append(r)
+    W = torch.from_numpy(np.stack(rows).astype(np.float32))
+    quantize_both(qb, oracle, W)
+
+
+def test_quantize_rejects_nonfinite(qb):
+    for bad in (float("nan"), float("inf"), -float("inf")):
+        W = torch.zeros(4, 128, device="cuda")
+        W[2, 77] = bad
+        with pytest.raises(qb.QloraError) as ei:
+            qb.nf4_quantize(W)
+        assert ei.value.status == -3
+
+
+@pytest.mark.parametrize("N,K,seed", [(7, 192, 5), (64, 4096, 6)])
+def test_dequantize_bit_exact(qb, oracle, N, K, seed):
+    W = wl.draw_weight(wl.generator(seed), N, K, 0.02, 0.01)
+    q, _ = quantize_both(qb, oracle, W)
+    Wd = qb.nf4_dequantize(q)
+    torch.cuda.synchronize()
+    o16, _ = oracle.nf4_dequantize(q.codes.cpu().numpy(), q.absmax_q.cpu().numpy(), q.dq_scale.cpu().numpy(), N, K)
+    assert np.array_equal(bits(Wd), o16)
+
+
+# ----------------------------------------------------------- layer, small
+
+
+SMALL = [
+    # M, N, K, r        (GEMM path: M > 16)
+    (17, 64, 64, 8),
+    (128, 256, 128, 16),
+    (200, 264, 320, 16),
+    (300, 520, 1024, 64),
+    (257, 1000, 192, 24),
+]
+
+
+@pytest.mark.parametrize("M,N,K,r", SMALL)
+def test_forward_small(qb, oracle, M, N, K, r):
+    p = wl.draw_small(1000 + M + N + K, M, N, K, r, 2.0 * r, with_dy=False)
+    run_fwd_check(qb, oracle, p)
+
+
+@pytest.mark.parametrize("M,N,K,r", [(1, 64, 64, 8), (4, 264, 320, 16), (16, 1000, 1024, 64), (9, 72, 4096, 8)])
+def test_forward_decode_small(qb, oracle, M, N, K, r):
+    p = wl.draw_small(2000 + M + N, M, N, K, r, 2.0 * r, with_dy=False)
+    run_fwd_check(qb, oracle, p)
+
+
+@pytest.mark.parametrize("M,N,K,r", SMALL)
+def test_backward_small(qb, oracle, M, N, K, r):
+    p = wl.draw_small(3000 + M + N + K, M, N, K, r, 2.0 * r)
+    run_bwd_check(qb, oracle, p)
+    run_bwd_check(qb, oracle, p, use_saved_h=False)
+
+
+def test_adapter_isolating_cases(qb, oracle):
+    """W = 0 makes Y and dX pure LoRA; a large B makes the adapter dominate."""
+    M, N, K, r = 150, 320, 256, 16
+    p = wl.draw_small(77, M, N, K, r, 32.0)
+    p["W"] = torch.zeros(N, K)
+    run_fwd_check(qb, oracle, p)
+    run_bwd_check(qb, oracle, p)
+    p = wl.draw_small(78, M, N, K, r, 32.0, b_std=1.0)
+    run_fwd_check(qb, oracle, p)
+    run_bwd_check(qb, oracle, p)
+    p = wl.draw_small(79, 12, N, K, r, 32.0, b_std=1.0, with_dy=False)  # decode path
+    p["W"] = torch.zeros(N, K)
+    run_fwd_check(qb, oracle, p)
+
+
+def test_zero_B_gives_base_and_zero_dA(qb, oracle):
+    M, N, K, r = 130, 256, 256, 16
+    p = wl.draw_small(81, M, N, K, r, 32.0)
+    p["B"] = torch.zeros(N, r, dtype=torch.bfloat16)
+    q, Wp = quantize_both(qb, oracle, p["W"])
+    X, A, B, dY = p["X"].cuda(), p["A"].cuda(), p["B"].cuda(), p["dY"].cuda()
+    Y1, _ = qb.qlora_linear_fwd(q, X, A, B, p["scale"])
+    Y2, _ = qb.qlora_linear_fwd(q, X, A, B, p["scale"])
+    assert torch.equal(Y1, Y2)
+    Yb = oracle.linear_fwd(bits(p["X"]), Wp, bits(p["A"]), bits(p["B"]), p["scale"])
+    assert relfro(Y1.float().cpu().numpy(), Yb) <= TOL
+    _, dA, dB = qb.qlora_linear_bwd(q, X, dY, A, B, p["scale"])
+    assert torch.count_nonzero(dA).item() == 0
+    assert torch.count_nonzero(dB).item() > 0
+
+
+def test_no_tokens(qb):
+    N, K, r = 128, 128, 16
+    q = qb.nf4_quantize(torch.randn(N, K, device="cuda") * 0.02)
+    X = torch.empty(0, K, dtype=torch.bfloat16, device="cuda")
+    A = torch.randn(r, K, device="cuda").bfloat16()
+    B = torch.randn(N, r, device="cuda").bfloat16()
+    Y, _ = qb.qlora_linear_fwd(q, X, A, B, 2.0)
+    assert Y.shape == (0, N)
+    dX, dA, dB = qb.qlora_linear_bwd(q, X, torch.empty(0, N, dtype=torch.bfloat16, device="cuda"), A, B, 2.0)
+    assert torch.count_nonzero(dA).item() == 0 and torch.count_nonzero(dB).item() == 0
+
+
+def test_decode_and_gemm_paths_agree(qb):
+    """M <= 16 runs the decode kernel, M > 16 the tensor-core GEMM; the same
+    rows must agree within tolerance."""
+    N, K, r = 1024, 2048, 16
+    p = wl.draw_small(91, 17, N, K, r, 32.0, with_dy=False)
+    q = qb.nf4_quantize(p["W"].cuda())
+    X, A, B = p["X"].cuda(), p["A"].cuda(), p["B"].cuda()
+    Yg, _ = qb.qlora_linear_fwd(q, X, A, B, p["scale"])          # GEMM
+    Yd, _ = qb.qlora_linear_fwd(q, X[:16].contiguous(), A, B, p["scale"])  # decode
+    assert relfro(Yd.float().cpu().numpy(), Yg[:16].float().cpu().numpy()) <= 5e-3
+
+
+def test_argument_errors_on_device(qb):
+    q = qb.nf4_quantize(torch.randn(64, 128, device="cuda") * 0.02)
+    X = torch.randn(32, 128, device="cuda").bfloat16()
+    A = torch.randn(16, 128, device="cuda").bfloat16()
+    B = torch.randn(64, 16, device="cuda").bfloat16()
+    L = qb.lib()
+    import ctypes
+    Y = torch.empty(32, 64, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(64, dtype=torch.uint8, device="cuda")
+    st = L.qlora_linear_fwd(qb._ptr(q.codes), qb._ptr(q.absmax_q), qb._ptr(q.dq_scale), 64, 128, qb._ptr(X), 32,
+                            qb._ptr(A), qb._ptr(B), 16, ctypes.c_float(2.0), qb._ptr(Y), None, qb._ptr(ws), 64,
+                            qb._stream())
+    assert st == -4  # workspace too small
+    assert qb.device_status() == 0
+
+
+# ---------------------------------------------------- workloads, full size
+
+
+def _rows(M, n, seed):
+    g = np.random.default_rng(seed)
+    rows = np.sort(g.choice(M, size=min(n, M), replace=False))
+    rows[0], rows[-1] = 0, M - 1  # first and last (ragged) rows included
+    return np.unique(rows)
+
+
+def test_workload_fwd_2048(qb, oracle):
+    p = wl.draw_linear(wl.WORKLOADS["fwd_2048"])
+    run_fwd_check(qb, oracle, p)
+
+
+def test_workload_qproj_7b(qb, oracle):
+    w = wl.WORKLOADS["qproj_7b"]
+    p = wl.draw_linear(w)
+    rows = _rows(p["M"], 48, 1)
+    _, q, Wp = run_fwd_check(qb, oracle, p, rows=rows)
+    run_bwd_check(qb, oracle, p, rows=rows, q=q, Wp=Wp)
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_workload_decode_70b_up(qb, oracle, M):
+    w = wl.WORKLOADS["decode_70b_up"]
+    p = wl.draw_linear(w, M=M)
+    run_fwd_check(qb, oracle, p)
+
+
+@pytest.mark.parametrize("proj", [0, 1, 2])
+def test_workload_mlp_7b(qb, oracle, proj):
+    w = wl.WORKLOADS["mlp_7b"]
+    p = wl.draw_linear(w, proj)
+    rows = _rows(p["M"], 16, 10 + proj)
+    _, q, Wp = run_fwd_check(qb, oracle, p, rows=rows)
+    run_bwd_check(qb, oracle, p, rows=rows, q=q, Wp=Wp)
+
+
+@pytest.mark.parametrize("proj", range(7))
+def test_workload_layer_70b(qb, oracle, proj):
+    w = wl.WORKLOADS["layer_70b"]
+    p = wl.draw_linear(w, proj)
+    rows = _rows(p["M"], 8, 20 + proj)
+    _, q, Wp = run_fwd_check(qb, oracle, p, rows=rows)
+    run_bwd_check(qb, oracle, p, rows=rows, q=q, Wp=Wp)
+
+
+def test_device_status_clean(qb):
+    assert qb.device_status() == 0
