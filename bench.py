@@ -123,7 +123,7 @@ class ClockSampler:
 # -------------------------------------------------------------- CPU oracle
 
 
-def oracle_sample(rows_sample: int = 48):
+def oracle_sample(rows_sample: int | None = None):
     """Times the CPU oracle on a bounded sample of the workload: Y and dX for
     `rows_sample` token rows, H, dH, dA, dB in full.  Returns (TFLOP/s, cores,
     sample description, seconds)."""
@@ -138,7 +138,7 @@ def oracle_sample(rows_sample: int = 48):
     _, Wp = oracle.nf4_dequantize(oc, oa, od, N, K)
     bits = wl.bf16_bits
     X, A, B, dY = bits(p["X"]), bits(p["A"]), bits(p["B"]), bits(p["dY"])
-    rows = np.linspace(0, M - 1, rows_sample).astype(np.int64)
+    rows = np.arange(M, dtype=np.int64) if rows_sample is None else np.linspace(0, M - 1, rows_sample).astype(np.int64)
     t0 = time.perf_counter()
     oracle.linear_fwd(X, Wp, A, B, p["scale"], rows=rows)
     oracle.linear_bwd(X, dY, Wp, A, B, p["scale"], rows=rows)
@@ -149,7 +149,7 @@ def oracle_sample(rows_sample: int = 48):
     flops += S * (2 * N * K + 2 * r * K)                      # dX rows
     flops += 2 * r * K * M + 2 * N * r * M                    # dA, dB
     desc = (f"{WORKLOAD} (M={M}, N={N}, K={K}, r={r}): Y and dX for {S} of {M} token rows, "
-            f"H, dH, dA, dB in full; fp64 oracle")
+            f"H, dH, dA, dB in full; one fwd+bwd pass of the fp64 oracle")
     return flops / dt / 1e12, oracle.num_threads(), desc, dt
 
 
@@ -391,7 +391,7 @@ def run_reference(args, rank, world):
     vals = []
     cores = desc = None
     for _ in range(max(1, args.steps if args.steps <= 3 else 3)):
-        tf, cores, desc, dt = oracle_sample(rows_sample=16)
+        tf, cores, desc, dt = oracle_sample(rows_sample=512)
         vals.append(tf)
     v = statistics.median(vals)
     out = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
@@ -403,6 +403,35 @@ def run_reference(args, rank, world):
     print(json.dumps(out), flush=True)
 
 
+def run_profile(args):
+    """A few launches of one kernel on one workload, for ncu captures."""
+    import torch
+
+    from bit_nf4_quantized_24_b200 import binding as qb
+    from bit_nf4_quantized_24_b200 import build as qbuild
+    from bit_nf4_quantized_24_b200 import workloads as wl
+    qbuild.build()
+    dev = torch.device("cuda", 0)
+    w = wl.WORKLOADS[args.workload]
+    M = args.tokens if args.tokens else None
+    p = wl.draw_linear(w, 0, M=M, with_dy=args.profile in ("bwd", "step"))
+    q = qb.nf4_quantize(p["W"].to(dev))
+    X, A, B = p["X"].to(dev), p["A"].to(dev), p["B"].to(dev)
+    dY = p["dY"].to(dev) if "dY" in p else None
+    for _ in range(args.warmup + args.steps):
+        if args.profile in ("fwd", "step"):
+            _, H = qb.qlora_linear_fwd(q, X, A, B, p["scale"])
+        if args.profile in ("bwd", "step"):
+            qb.qlora_linear_bwd(q, X, dY, A, B, p["scale"])
+        if args.profile == "quantize":
+            qb.nf4_quantize(p["W"].to(dev))
+        if args.profile == "dequantize":
+            qb.nf4_dequantize(q)
+    torch.cuda.synchronize()
+    assert qb.device_status() == 0
+    print(f"profile {args.profile} {args.workload} M={p['M']} N={p['N']} K={p['K']} done")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -411,7 +440,14 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true", help="skip decode/quantize measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--profile", choices=["fwd", "bwd", "step", "quantize", "dequantize"],
+                    help="run only warmup+steps launches of one entry point (for ncu)")
+    ap.add_argument("--workload", default=WORKLOAD, help="workload for --profile")
+    ap.add_argument("--tokens", type=int, default=0, help="token count for --profile (default: the workload's)")
     args = ap.parse_args()
+    if args.profile:
+        run_profile(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     world = int(os.environ.get("WORLD_SIZE", "1"))
