@@ -28,7 +28,8 @@ __device__ __forceinline__ uint4 ldg_v4_or_zero(const uint16_t* p, bool ok) {
 // Inside a chunk, thread t (= lane & 3) owns the 8 consecutive k's 8t..8t+7;
 // they fill the fragment slots {2t, 2t+1, 2t+8, 2t+9} of two m16n8k16 steps.
 // The same k permutation is used for both operands, so the sum is unchanged.
-template <int NT>  // NT = ceil(R / 8) n8 tiles
+// U chunks are loaded before any is used, to keep enough bytes in flight.
+template <int NT, int U>  // NT = ceil(R / 8) n8 tiles
 __global__ void __launch_bounds__(256) k_rowdot(const uint16_t* __restrict__ P, const uint16_t* __restrict__ Q,
                                                 int M, int Kc, int R, float sa, uint16_t* __restrict__ out16a,
                                                 float sb, uint16_t* __restrict__ out16b, float* __restrict__ out32) {
@@ -41,17 +42,27 @@ __global__ void __launch_bounds__(256) k_rowdot(const uint16_t* __restrict__ P, 
   for (int i = 0; i < NT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
   const int nchunks = (Kc + 31) / 32;
   const bool row_lo = m0 + g < M, row_hi = m0 + g + 8 < M;
-  for (int c = warp; c < nchunks; c += 8) {
-    const int k = c * 32 + 8 * t;
-    const bool kin = k < Kc;
-    const uint4 alo = ldg_v4_or_zero(P + static_cast<int64_t>(m0 + g) * Kc + k, kin && row_lo);
-    const uint4 ahi = ldg_v4_or_zero(P + static_cast<int64_t>(m0 + g + 8) * Kc + k, kin && row_hi);
+  for (int c0 = warp; c0 < nchunks; c0 += 8 * U) {
+    uint4 alo[U], ahi[U], b[U][NT];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int j = nt * 8 + g;
-      const uint4 b = ldg_v4_or_zero(Q + static_cast<int64_t>(j) * Kc + k, kin && j < R);
-      mma_bf16_16816(acc[nt], alo.x, ahi.x, alo.y, ahi.y, b.x, b.y);
-      mma_bf16_16816(acc[nt], alo.z, ahi.z, alo.w, ahi.w, b.z, b.w);
+    for (int u = 0; u < U; ++u) {
+      const int k = (c0 + 8 * u) * 32 + 8 * t;
+      const bool kin = (c0 + 8 * u < nchunks) && k < Kc;
+      alo[u] = ldg_v4_or_zero(P + static_cast<int64_t>(m0 + g) * Kc + k, kin && row_lo);
+      ahi[u] = ldg_v4_or_zero(P + static_cast<int64_t>(m0 + g + 8) * Kc + k, kin && row_hi);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int j = nt * 8 + g;
+        b[u][nt] = ldg_v4_or_zero(Q + static_cast<int64_t>(j) * Kc + k, kin && j < R);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        mma_bf16_16816(acc[nt], alo[u].x, ahi[u].x, alo[u].y, ahi[u].y, b[u][nt].x, b[u][nt].y);
+        mma_bf16_16816(acc[nt], alo[u].z, ahi[u].z, alo[u].w, ahi[u].w, b[u][nt].z, b[u][nt].w);
+      }
     }
   }
 #pragma unroll
@@ -79,56 +90,114 @@ __global__ void __launch_bounds__(256) k_rowdot(const uint16_t* __restrict__ P, 
   }
 }
 
-// partial[split][j][c] = sum over this split's rows m of G[m, j] P[m, c].
-// Thread = 2 adjacent columns c; the split's G rows are staged in shared
-// memory (fp32) 64 rows at a time and read as broadcasts.
-template <int RP>  // R rounded up to 8, 16, 32 or 64
-__global__ void __launch_bounds__(128) k_coldot_partial(const uint16_t* __restrict__ G,
-                                                        const uint16_t* __restrict__ P, int M, int C, int R,
-                                                        int rows_per_split, float* __restrict__ partial) {
-  __shared__ __align__(16) float sG[64][RP];
-  const int c = (blockIdx.x * 128 + threadIdx.x) * 2;
+__device__ __forceinline__ void cp_async_16z(uint32_t dst, const void* src, bool valid) {
+  const int n = valid ? 16 : 0;  // 0 source bytes -> 16 zero bytes
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                              uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// partial[split][j][c] = sum over this split's tokens m of G[m, j] P[m, c],
+// on the tensor cores: D[c, j] = sum_m P^T[c, m] G[m, j] with m16n8k16 tiles.
+// Both operands are row-major with the contraction (m) as the row index, so
+// 32-token slabs are staged in shared memory (cp.async, double-buffered,
+// rows padded by 16 B so the 8 rows of an ldmatrix phase hit distinct banks)
+// and read with ldmatrix.trans.  CTA = 128 columns x all R; warp w owns
+// columns 32w..32w+31.
+constexpr int CD_COLS = 128, CD_SLAB = 32, CD_PPITCH = CD_COLS + 8, CD_GPITCH = 64 + 8;
+
+template <int NT>  // NT = ceil(R / 8) rounded up to even (ldmatrix.x4 feeds two n8 tiles)
+__global__ void __launch_bounds__(128) k_coldot_mma(const uint16_t* __restrict__ G, const uint16_t* __restrict__ P,
+                                                    int M, int C, int R, int rows_per_split,
+                                                    float* __restrict__ partial) {
+  __shared__ __align__(16) uint16_t sP[2][CD_SLAB][CD_PPITCH];
+  __shared__ __align__(16) uint16_t sG[2][CD_SLAB][CD_GPITCH];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int c0 = blockIdx.x * CD_COLS;
   const int split = blockIdx.y;
   const int mb0 = split * rows_per_split;
   const int mb1 = min(M, mb0 + rows_per_split);
-  float acc[RP][2];
-#pragma unroll
-  for (int j = 0; j < RP; ++j) acc[j][0] = acc[j][1] = 0.f;
-  for (int mb = mb0; mb < mb1; mb += 64) {
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < 64 * RP; idx += 128) {
-      const int i = idx / RP, j = idx % RP;
-      const int m = mb + i;
-      float v = 0.f;
-      if (m < mb1 && j < R) v = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(G)[static_cast<int64_t>(m) * R + j]);
-      sG[i][j] = v;
+  const int nslab = mb1 > mb0 ? (mb1 - mb0 + CD_SLAB - 1) / CD_SLAB : 0;
+  const int gchunks = (R + 7) / 8;  // 16-byte chunks per G row
+
+  auto stage = [&](int sl, int buf) {
+    const int mb = mb0 + sl * CD_SLAB;
+    for (int u = tid; u < CD_SLAB * (CD_COLS / 8); u += 128) {
+      const int i = u / (CD_COLS / 8), cc = (u % (CD_COLS / 8)) * 8;
+      const bool ok = (mb + i < mb1) && (c0 + cc < C);
+      const uint16_t* src = ok ? P + static_cast<int64_t>(mb + i) * C + c0 + cc : P;
+      cp_async_16z(smem_u32(&sP[buf][i][cc]), src, ok);
     }
-    __syncthreads();
-    const int iend = min(64, mb1 - mb);
-    if (c < C) {
-      for (int i = 0; i < iend; ++i) {
-        const uint32_t pv = __ldg(reinterpret_cast<const uint32_t*>(P + static_cast<int64_t>(mb + i) * C + c));
-        const float p0 = __uint_as_float(pv << 16), p1 = __uint_as_float(pv & 0xffff0000u);
+    for (int u = tid; u < CD_SLAB * 8; u += 128) {
+      const int i = u / 8, cc = (u % 8) * 8;
+      const bool ok = (mb + i < mb1) && (u % 8) < gchunks;
+      const uint16_t* src = ok ? G + static_cast<int64_t>(mb + i) * R + cc : G;
+      cp_async_16z(smem_u32(&sG[buf][i][cc]), src, ok);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+
+  float acc[2][NT][4];
 #pragma unroll
-        for (int j = 0; j < RP; j += 4) {
-          const float4 gv = *reinterpret_cast<const float4*>(&sG[i][j]);
-          acc[j][0] = fmaf(gv.x, p0, acc[j][0]);
-          acc[j][1] = fmaf(gv.x, p1, acc[j][1]);
-          acc[j + 1][0] = fmaf(gv.y, p0, acc[j + 1][0]);
-          acc[j + 1][1] = fmaf(gv.y, p1, acc[j + 1][1]);
-          acc[j + 2][0] = fmaf(gv.z, p0, acc[j + 2][0]);
-          acc[j + 2][1] = fmaf(gv.z, p1, acc[j + 2][1]);
-          acc[j + 3][0] = fmaf(gv.w, p0, acc[j + 3][0]);
-          acc[j + 3][1] = fmaf(gv.w, p1, acc[j + 3][1]);
+  for (int a = 0; a < 2; ++a)
+#pragma unroll
+    for (int n = 0; n < NT; ++n) acc[a][n][0] = acc[a][n][1] = acc[a][n][2] = acc[a][n][3] = 0.f;
+
+  if (nslab > 0) stage(0, 0);
+  for (int sl = 0; sl < nslab; ++sl) {
+    const int buf = sl & 1;
+    if (sl + 1 < nslab) stage(sl + 1, buf ^ 1);
+    else asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+    __syncthreads();
+    const int q = lane >> 3, rr = lane & 7;
+#pragma unroll
+    for (int ks = 0; ks < CD_SLAB / 16; ++ks) {
+      uint32_t a[2][4];
+#pragma unroll
+      for (int ct = 0; ct < 2; ++ct) {
+        // matrices: (m 0-7, c 0-7), (m 0-7, c 8-15), (m 8-15, c 0-7), (m 8-15, c 8-15)
+        const int m = ks * 16 + (q >> 1) * 8 + rr;
+        const int c = warp * 32 + ct * 16 + (q & 1) * 8;
+        ldsm_x4_trans(smem_u32(&sP[buf][m][c]), a[ct][0], a[ct][1], a[ct][2], a[ct][3]);
+      }
+#pragma unroll
+      for (int np = 0; np < NT / 2; ++np) {
+        // matrices: (m 0-7, tile 2np), (m 8-15, tile 2np), (m 0-7, tile 2np+1), (m 8-15, tile 2np+1)
+        const int m = ks * 16 + (q & 1) * 8 + rr;
+        const int j = (2 * np + (q >> 1)) * 8;
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_trans(smem_u32(&sG[buf][m][j]), b0, b1, b2, b3);
+#pragma unroll
+        for (int ct = 0; ct < 2; ++ct) {
+          mma_bf16_16816(acc[ct][2 * np], a[ct][0], a[ct][1], a[ct][2], a[ct][3], b0, b1);
+          mma_bf16_16816(acc[ct][2 * np + 1], a[ct][0], a[ct][1], a[ct][2], a[ct][3], b2, b3);
         }
       }
     }
+    __syncthreads();
   }
-  if (c < C) {
-    float* dst = partial + static_cast<int64_t>(split) * R * C;
+  float* dst = partial + static_cast<int64_t>(split) * R * C;
 #pragma unroll
-    for (int j = 0; j < RP; ++j)
-      if (j < R) *reinterpret_cast<float2*>(dst + static_cast<int64_t>(j) * C + c) = make_float2(acc[j][0], acc[j][1]);
+  for (int ct = 0; ct < 2; ++ct) {
+    const int cbase = c0 + warp * 32 + ct * 16 + g;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int j = nt * 8 + 2 * t;
+      if (cbase < C) {
+        if (j < R) dst[static_cast<int64_t>(j) * C + cbase] = acc[ct][nt][0];
+        if (j + 1 < R) dst[static_cast<int64_t>(j + 1) * C + cbase] = acc[ct][nt][1];
+      }
+      if (cbase + 8 < C) {
+        if (j < R) dst[static_cast<int64_t>(j) * C + cbase + 8] = acc[ct][nt][2];
+        if (j + 1 < R) dst[static_cast<int64_t>(j + 1) * C + cbase + 8] = acc[ct][nt][3];
+      }
+    }
   }
 }
 
@@ -168,9 +237,9 @@ __global__ void k_transpose_bf16(const uint16_t* __restrict__ src, int R, int C,
 }
 
 int coldot_splits(int64_t M, int64_t C) {
-  const int64_t col_tiles = (C + 255) / 256;
-  int64_t s = (4 * 148 + col_tiles - 1) / col_tiles;  // aim for ~4 CTAs per SM
-  s = std::max<int64_t>(1, std::min<int64_t>(s, (M + 63) / 64));
+  const int64_t col_tiles = (C + CD_COLS - 1) / CD_COLS;
+  int64_t s = (6 * 148 + col_tiles - 1) / col_tiles;  // aim for ~6 CTAs per SM
+  s = std::max<int64_t>(1, std::min<int64_t>(s, (M + 127) / 128));
   return static_cast<int>(s);
 }
 
@@ -181,10 +250,11 @@ cudaError_t launch_rowdot(const uint16_t* P, const uint16_t* Q, int64_t M, int64
   if (M == 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>((M + 15) / 16);
   const int nt = (R + 7) / 8;
-#define QN_ROWDOT(NTV)                                                                                   \
-  case NTV:                                                                                              \
-    k_rowdot<NTV><<<grid, 256, 0, st>>>(P, Q, static_cast<int>(M), static_cast<int>(Kc), R, sa, out16a, \
-                                         sb, out16b, out32);                                             \
+#define QN_ROWDOT(NTV)                                                                            \
+  case NTV:                                                                                       \
+    k_rowdot<NTV, (NTV <= 2 ? 4 : 2)><<<grid, 256, 0, st>>>(P, Q, static_cast<int>(M),             \
+                                                           static_cast<int>(Kc), R, sa, out16a,   \
+                                                           sb, out16b, out32);                    \
     break;
   switch (nt) {
     QN_ROWDOT(1) QN_ROWDOT(2) QN_ROWDOT(3) QN_ROWDOT(4) QN_ROWDOT(5) QN_ROWDOT(6) QN_ROWDOT(7) QN_ROWDOT(8)
@@ -203,16 +273,17 @@ cudaError_t launch_coldot(const uint16_t* G, const uint16_t* P, int64_t M, int64
                           int transpose, float* partial, uint16_t* out, cudaStream_t st) {
   const int splits = coldot_splits(M, C);
   const int rows_per_split = static_cast<int>((M + splits - 1) / splits);
-  const dim3 grid(static_cast<unsigned>((C + 255) / 256), static_cast<unsigned>(splits));
+  const dim3 grid(static_cast<unsigned>((C + CD_COLS - 1) / CD_COLS), static_cast<unsigned>(splits));
   if (M > 0) {
-    if (R <= 8)
-      k_coldot_partial<8><<<grid, 128, 0, st>>>(G, P, int(M), int(C), R, rows_per_split, partial);
-    else if (R <= 16)
-      k_coldot_partial<16><<<grid, 128, 0, st>>>(G, P, int(M), int(C), R, rows_per_split, partial);
-    else if (R <= 32)
-      k_coldot_partial<32><<<grid, 128, 0, st>>>(G, P, int(M), int(C), R, rows_per_split, partial);
-    else if (R <= 64)
-      k_coldot_partial<64><<<grid, 128, 0, st>>>(G, P, int(M), int(C), R, rows_per_split, partial);
+    const int nt = (R + 7) / 8;
+    if (nt <= 2)
+      k_coldot_mma<2><<<grid, 128, 0, st>>>(G, P, int(M), int(C), R, rows_per_split, partial);
+    else if (nt <= 4)
+      k_coldot_mma<4><<<grid, 128, 0, st>>>(G, P, int(M), int(C), R, rows_per_split, partial);
+    else if (nt <= 6)
+      k_coldot_mma<6><<<grid, 128, 0, st>>>(G, P, int(M), int(C), R, rows_per_split, partial);
+    else if (nt <= 8)
+      k_coldot_mma<8><<<grid, 128, 0, st>>>(G, P, int(M), int(C), R, rows_per_split, partial);
     else
       return cudaErrorInvalidValue;
   } else {

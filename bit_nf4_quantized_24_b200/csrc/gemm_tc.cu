@@ -5,7 +5,9 @@
 // NormalFloat".  Here the dequantized weight tile exists only in shared
 // memory, one pipeline stage at a time, as the B operand of tcgen05.mma.
 //
-// Tile: 128 tokens (M) x 256 outputs (N) x 64 contraction (K) per stage.
+// Tile: 256 tokens (M) x 256 outputs (N) x 64 contraction (K) per stage, as
+// two 128 x 256 fp32 accumulators in TMEM (all 512 columns) that share every
+// dequantized weight tile, so each expanded weight feeds 256 tokens.
 //   mode 0, forward:  D[m, n] = sum_k X[m,k] W'[n,k]       (W' K-major)
 //   mode 1, dX:       D[m, k] = sum_n dY[m,n] W'[n,k]      (W' MN-major)
 // followed by one tail stage that adds the LoRA product from bf16 operands
@@ -27,8 +29,8 @@ namespace qn {
 
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;     // 16 KB
+constexpr int BM = 256, UM = 128, BN = 256, BK = 64, STAGES = 3;
+constexpr int A_BYTES = BM * BK * 2;     // 32 KB (two 128-row halves)
 constexpr int B_BYTES = BN * BK * 2;     // 32 KB
 constexpr int C_BYTES = BN * BK / 2;     // 8 KB of packed codes
 constexpr int OFF_A = 0;
@@ -38,7 +40,7 @@ constexpr int OFF_BAR = OFF_C + STAGES * C_BYTES;
 constexpr int SMEM_USED = OFF_BAR + 256;
 constexpr int SMEM_ALLOC = SMEM_USED + 1024;  // slack for 1024-byte alignment
 constexpr int NUM_THREADS = 320;
-constexpr int TMEM_COLS = 256;
+constexpr int TMEM_COLS = 512;  // accumulator h at columns 256h .. 256h+255
 
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 
@@ -146,7 +148,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(BM, BN, false, MODE == 1);
+      constexpr uint32_t idesc = idesc_bf16(UM, BN, false, MODE == 1);
       bool ok = true;
       int committed = 0;
       for (int it = 0; it <= numK; ++it) {
@@ -160,10 +162,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t b_s = base + OFF_B + s * B_BYTES;
         const int nk = tail ? (r + 15) / 16 : BK / 16;
         for (int kk = 0; kk < nk; ++kk) {
-          const uint64_t ad = desc_sw128(a_s + kk * 32, 16, 1024);
           const uint64_t bd = MODE == 0 ? desc_sw128(b_s + kk * 32, 16, 1024)
                                         : desc_sw128(b_s + kk * 2048, 8192, 1024);
-          tc_mma_f16(tmem, ad, bd, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+          tc_mma_f16(tmem, desc_sw128(a_s + kk * 32, 16, 1024), bd, idesc, acc);
+          tc_mma_f16(tmem + 256, desc_sw128(a_s + UM * 128 + kk * 32, 16, 1024), bd, idesc, acc);
         }
         tc_commit(empty(s));
         committed = 1;
@@ -237,13 +240,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (ok) {
       tc_fence_after();
       const int quad = warp & 3;                 // TMEM lanes 32*quad .. +31
-      const int colh = (warp - 2) >> 2;          // column half: 0 or 1
-      const int m = m0 + quad * 32 + lane;
+      const int h = (warp - 2) >> 2;             // accumulator: tokens 128h .. 128h+127
+      const int m = m0 + h * UM + quad * 32 + lane;
 #pragma unroll 1
-      for (int cc = 0; cc < BN / 2; cc += 32) {
-        const int col = colh * (BN / 2) + cc;
+      for (int col = 0; col < BN; col += 32) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(col), v);
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(h * 256 + col),
+                           v);
         tmem_ld_wait();
         const int n = n0 + col;
         if (m < M && n < Nout) {
