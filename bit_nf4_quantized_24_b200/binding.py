@@ -60,6 +60,7 @@ def lib():
     L.qlora_linear_bwd_workspace.argtypes = [i64, i64, i64, i32, P]
     L.qlora_linear_fwd.argtypes = [P, P, P, i64, i64, P, i64, P, P, i32, f32, P, P, P, sz, P]
     L.qlora_linear_bwd.argtypes = [P, P, P, i64, i64, P, P, i64, P, P, i32, f32, P, P, P, P, P, sz, P]
+    L.qlora_linear_fwd_noalloc.argtypes = [P, P, P, i64, i64, P, i64, P, P, i32, f32, P, P, P]
     L.qlora_device_status.restype = i32
     L.qlora_trace_gemm_events.argtypes = [P, i32]
     L.qlora_trace_gemm_count.restype = i32
@@ -220,6 +221,25 @@ def qlora_linear_bwd(w: NF4Weight, X: torch.Tensor, dY: torch.Tensor, A: torch.T
                                   M, _ptr(A), _ptr(B), r, float(scale), _ptr(H), _ptr(dX), _ptr(dA), _ptr(dB),
                                   _ptr(ws), ws.numel(), _stream(stream)), "qlora_linear_bwd")
     return dX, dA, dB
+
+
+def qlora_linear_fwd_noalloc(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, scale: float,
+                             save_h: bool = True, out: torch.Tensor | None = None, stream=None):
+    """qlora_linear_fwd without a workspace: the library's fixed device scratch
+    is used instead (M * r <= QLORA_NOALLOC_MAX_TOKENS_X_RANK).  Returns (Y, H)."""
+    M = X.shape[0]
+    r = A.shape[0]
+    _req(X, torch.bfloat16, "X", (M, w.K))
+    _req(A, torch.bfloat16, "A", (r, w.K))
+    _req(B, torch.bfloat16, "B", (w.N, r))
+    if out is None:
+        out = torch.empty(M, w.N, dtype=torch.bfloat16, device=X.device)
+    _req(out, torch.bfloat16, "Y", (M, w.N))
+    H = torch.empty(M, r, dtype=torch.bfloat16, device=X.device) if save_h else None
+    _check(lib().qlora_linear_fwd_noalloc(_ptr(w.codes), _ptr(w.absmax_q), _ptr(w.dq_scale), w.N, w.K, _ptr(X), M,
+                                          _ptr(A), _ptr(B), r, float(scale), _ptr(out), _ptr(H), _stream(stream)),
+           "qlora_linear_fwd_noalloc")
+    return out, H
 
 
 def device_status() -> int:

@@ -149,6 +149,32 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* absmax_q, const float*
                      qlora_bf16_t* dX, qlora_bf16_t* dA, qlora_bf16_t* dB,
                      void* workspace, size_t workspace_bytes, void* stream);
 
+/* Largest M * r that qlora_linear_fwd_noalloc accepts: its fixed device
+ * scratch holds this many bf16 values (2 MiB on every device that loads the
+ * library, held until the process exits). */
+#define QLORA_NOALLOC_MAX_TOKENS_X_RANK (1 << 20)
+
+/* qlora_linear_fwd for callers that cannot allocate device memory -- for
+ * example a plugin inside a framework that owns all device memory and gives
+ * the plugin no allocator, a service that reserves its memory up front and
+ * forbids later allocations, or a latency-critical thread that cannot take
+ * cudaMalloc's implicit device synchronization.  The QLoRA pages have no
+ * counterpart to this entry point; it exists only for such callers.
+ * Same arguments, result and errors as qlora_linear_fwd, minus the workspace:
+ * the scratch lives in a fixed array in device memory inside the library, and
+ * no cudaMalloc, cudaFree or other allocating routine is called.
+ * Limits: M * r <= QLORA_NOALLOC_MAX_TOKENS_X_RANK, else QLORA_ERR_WORKSPACE
+ * (returned before anything is enqueued).
+ * Sharing: all calls on a device share the one scratch array, which keeps the
+ * last call's contents; calls that overlap on the GPU (streams without
+ * ordering between them) race on it.
+ * Set-up: the first call on each device looks up the array's device address
+ * with that device current; make that first call before any stream capture. */
+int qlora_linear_fwd_noalloc(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale,
+                             int64_t N, int64_t K, const qlora_bf16_t* X, int64_t M,
+                             const qlora_bf16_t* A, const qlora_bf16_t* B, int r, float scale,
+                             qlora_bf16_t* Y, qlora_bf16_t* H_save, void* stream);
+
 /* Reads and clears the device status word of the current device (a
  * QLORA_ERR_TIMEOUT left by a bounded wait, else QLORA_OK).  Synchronizes the
  * device. */
