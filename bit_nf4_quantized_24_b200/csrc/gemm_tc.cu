@@ -1,9 +1,9 @@
 // Fused NF4-dequant GEMM on the sm_100a tensor cores (tcgen05 + TMEM).
 //
-// "At runtime, the kernel dequantizes a block back to the compute dtype, does
-// the matmul, and discards the dequantized copy" -- katajob, "NF4: 4-bit
-// NormalFloat".  Here the dequantized weight tile exists only in shared
-// memory, one pipeline stage at a time, as the B operand of tcgen05.mma.
+// katajob, "NF4: 4-bit NormalFloat": the 4-bit weight is expanded block by
+// block to bf16 only for the product and thrown away afterwards.  Here the
+// expanded weight tile exists only in shared memory, one pipeline stage at a
+// time, as the B operand of tcgen05.mma.
 //
 // Tile: 256 tokens (M) x 256 outputs (N) x 64 contraction (K) per stage, as
 // two 128 x 256 fp32 accumulators in TMEM (all 512 columns) that share every

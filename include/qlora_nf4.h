@@ -5,8 +5,8 @@
  *  - "What does QLoRA change compared with plain LoRA when fine-tuning Llama?"
  *    (katajob): "NF4: 4-bit NormalFloat" (16-level type for normally
  *    distributed weights; per-block scaling over small groups of contiguous
- *    weights, commonly 64; dequantized block by block to bf16 inside the
- *    matmul and discarded), "Double quantization" (the per-block scales are
+ *    weights, 64 being the usual size; expanded block by block to bf16 for
+ *    the matmul only), "Double quantization" (the per-block scales are
  *    themselves quantized to 8 bits with a second-level scale over groups),
  *    "What stays in full precision" (A, B are bf16; gradients reach them
  *    through the dequantized base; the base gets no update).

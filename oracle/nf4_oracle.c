@@ -99,9 +99,9 @@ static double phi_inv(double p) {
     return 0.5 * (lo + hi);
 }
 
-/* The top probability used for the outermost levels.  Reading: the pages give
- * only "16 levels ... information-theoretically optimal for a zero-centred
- * normal" with an exact zero; the plainest construction uses equal-probability
+/* The top probability used for the outermost levels.  Reading: the pages say
+ * only that the 16 levels suit zero-centred normal weights (and the layer needs
+ * an exact zero); the plainest construction uses equal-probability
  * quantiles on each side of zero, and delta is taken as the mean of the centres
  * of the top equal-mass bins of a 16-bin and a 15-bin split of the line:
  * delta = 1 - (1/32 + 1/30) / 2. */
