@@ -170,6 +170,7 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         dist.barrier()
     from bit_nf4_quantized_24_b200 import binding as qb
+    from bit_nf4_quantized_24_b200 import dp
     from bit_nf4_quantized_24_b200 import workloads as wl
 
     pk = peaks()
@@ -203,8 +204,7 @@ def run_ours(args, rank, world, local_rank):
         if e:
             raise qb.QloraError(e, "bwd")
         if world > 1:
-            dist.all_reduce(dA)
-            dist.all_reduce(dB)
+            dp.allreduce_adapter_grads(dA, dB)
 
     launches_per_step = 2 + 7  # fwd: rowdot, gemm; bwd: transpose, rowdot, gemm, 2x(coldot partial + reduce)
 
