@@ -202,24 +202,38 @@ __global__ void __launch_bounds__(128) k_coldot_mma(const uint16_t* __restrict__
 }
 
 // out = bf16(scale * sum_split partial[split]), as [R, C] or transposed [C, R].
-__global__ void k_coldot_reduce(const float* __restrict__ partial, int splits, int R, int C, float scale,
-                                int transpose, uint16_t* __restrict__ out) {
-  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t total = static_cast<int64_t>(R) * C;
-  if (idx >= total) return;
-  // idx enumerates the output in its own row-major order
-  int j, c;
-  if (transpose) {
-    c = static_cast<int>(idx / R);
-    j = static_cast<int>(idx % R);
-  } else {
-    j = static_cast<int>(idx / C);
-    c = static_cast<int>(idx % C);
+// Thread = one column c and 8 consecutive j (blockIdx.y picks the 8): every
+// partial read is coalesced across the warp, and a transposed output row
+// segment of 8 values is one 16-byte store.
+__global__ void __launch_bounds__(64) k_coldot_reduce(const float* __restrict__ partial, int splits, int R, int C,
+                                                      float scale, int transpose, uint16_t* __restrict__ out) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  const int j0 = blockIdx.y * 8;
+  if (c >= C) return;
+  const int64_t plane = static_cast<int64_t>(R) * C;
+  float acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+#pragma unroll 4
+  for (int sp = 0; sp < splits; ++sp) {
+    const float* src = partial + sp * plane + static_cast<int64_t>(j0) * C + c;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] += __ldcs(src + static_cast<int64_t>(j) * C);
   }
-  float v = 0.f;
-  for (int s = 0; s < splits; ++s) v += partial[static_cast<int64_t>(s) * total + static_cast<int64_t>(j) * C + c];
-  const __nv_bfloat16 h = __float2bfloat16_rn(scale * v);
-  out[idx] = *reinterpret_cast<const uint16_t*>(&h);
+  if (transpose) {
+    uint4 v;
+    v.x = bf16x2_bits(scale * acc[0], scale * acc[1]);
+    v.y = bf16x2_bits(scale * acc[2], scale * acc[3]);
+    v.z = bf16x2_bits(scale * acc[4], scale * acc[5]);
+    v.w = bf16x2_bits(scale * acc[6], scale * acc[7]);
+    *reinterpret_cast<uint4*>(out + static_cast<int64_t>(c) * R + j0) = v;
+  } else {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const __nv_bfloat16 h = __float2bfloat16_rn(scale * acc[j]);
+      out[static_cast<int64_t>(j0 + j) * C + c] = *reinterpret_cast<const uint16_t*>(&h);
+    }
+  }
 }
 
 __global__ void k_transpose_bf16(const uint16_t* __restrict__ src, int R, int C, uint16_t* __restrict__ dst) {
@@ -238,8 +252,8 @@ __global__ void k_transpose_bf16(const uint16_t* __restrict__ src, int R, int C,
 
 int coldot_splits(int64_t M, int64_t C) {
   const int64_t col_tiles = (C + CD_COLS - 1) / CD_COLS;
-  int64_t s = (6 * 148 + col_tiles - 1) / col_tiles;  // aim for ~6 CTAs per SM
-  s = std::max<int64_t>(1, std::min<int64_t>(s, (M + 127) / 128));
+  int64_t s = (2 * 148 + col_tiles - 1) / col_tiles;  // ~2 CTAs per SM, long token slabs
+  s = std::max<int64_t>(1, std::min<int64_t>(s, (M + 255) / 256));
   return static_cast<int>(s);
 }
 
@@ -292,9 +306,9 @@ cudaError_t launch_coldot(const uint16_t* G, const uint16_t* P, int64_t M, int64
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int64_t total = static_cast<int64_t>(R) * C;
-  k_coldot_reduce<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(partial, M > 0 ? splits : 1, R,
-                                                                                int(C), scale, transpose, out);
+  const int sp = M > 0 ? splits : 1;
+  const dim3 rgrid(static_cast<unsigned>((C + 63) / 64), static_cast<unsigned>(R / 8));
+  k_coldot_reduce<<<rgrid, 64, 0, st>>>(partial, sp, R, int(C), scale, transpose, out);
   return cudaGetLastError();
 }
 

@@ -13,12 +13,14 @@
 // followed by one tail stage that adds the LoRA product from bf16 operands
 // loaded by TMA: Hs B^T (forward, Hs = s*H) or dH A (dX).
 //
-// Warp roles (320 threads):
-//   warp 0      TMA producer: activation tile + NF4 code tile per stage
-//   warp 1      TMEM allocator and single-thread MMA issuer
-//   warps 2..9  dequantizers (one 64-weight block per thread per stage:
-//               register lookup table -> 128 B of swizzled bf16 in smem),
-//               then the epilogue (TMEM -> registers -> bf16 -> global)
+// Warp roles (576 threads):
+//   warp 0       TMA producer: activation tile + NF4 code tile per stage
+//   warp 1       TMEM allocator and single-thread MMA issuer
+//   warps 2..17  dequantizers in two groups of 8 that take alternate stages
+//                (one 64-weight block per thread per stage: register lookup
+//                table -> 128 B of swizzled bf16 in smem); each thread loads
+//                its blocks' absmax code and group scale four stages ahead.
+//                Then all 16 run the epilogue (TMEM -> bf16 -> global).
 // Every wait is bounded (kWaitLimitNs); on expiry the kernel records
 // kDevTimeout, drains its in-flight copies and MMAs, frees TMEM and exits.
 #include <mutex>
@@ -39,7 +41,8 @@ constexpr int OFF_C = OFF_B + STAGES * B_BYTES;
 constexpr int OFF_BAR = OFF_C + STAGES * C_BYTES;
 constexpr int SMEM_USED = OFF_BAR + 256;
 constexpr int SMEM_ALLOC = SMEM_USED + 1024;  // slack for 1024-byte alignment
-constexpr int NUM_THREADS = 320;
+constexpr int DQ_GROUPS = 2;                       // dequant groups of 8 warps
+constexpr int NUM_THREADS = 64 + DQ_GROUPS * 256;
 constexpr int TMEM_COLS = 512;  // accumulator h at columns 256h .. 256h+255
 
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
@@ -180,29 +183,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ------------------------------------------- dequantizers, then epilogue
-    const int t = threadIdx.x - 64;  // 0..255
+    const int e = warp - 2;            // 0..15
+    const int grp = e >> 3;            // stages it = grp, grp + 2, ...
+    const int t = (e & 7) * 32 + lane; // item of the stage: 0..255
     bool ok = true;
-    const int KB = K / 64;           // 64-blocks per weight row
-    for (int it = 0; it < numK; ++it) {
-      const int s = it % STAGES;
-      const uint32_t ph = (it / STAGES) & 1;
-      // which (row, 64-block) of W this thread expands, and where it goes
-      int wrow, kcol0, srow;
+    const int KB = K / 64;             // 64-blocks per weight row
+    // which (row, 64-block) of W this thread expands at iteration it
+    auto item_of = [&](int it, int& wrow, int& kcol0) {
       if (MODE == 0) {
         wrow = n0 + t;
         kcol0 = it * BK;
-        srow = t;
       } else {
         wrow = it * BK + (t & 63);
-        kcol0 = n0 + 64 * (t >> 6);
-        srow = t;  // = 64 * (t >> 6) + (t & 63): sub-tile j holds outputs n0+64j..
+        kcol0 = n0 + 64 * (t >> 6);  // smem row t = 64 * (t >> 6) + (t & 63)
       }
-      const bool valid = (wrow < N) && (kcol0 < K);
-      float ap = 0.0f;
-      if (valid) {
-        const int64_t blk = static_cast<int64_t>(wrow) * KB + (kcol0 >> 6);
-        ap = __fmul_rn(static_cast<float>(__ldg(absmax_q + blk)), __ldg(dq_scale + (blk >> 8)));
+    };
+    struct Scale {
+      uint32_t q;
+      float s2;
+      bool valid;
+    };
+    auto fetch = [&](int it) {
+      Scale sc{0u, 0.0f, false};
+      if (it < numK) {
+        int wrow, kcol0;
+        item_of(it, wrow, kcol0);
+        if (wrow < N && kcol0 < K) {
+          const int64_t blk = static_cast<int64_t>(wrow) * KB + (kcol0 >> 6);
+          sc.q = __ldg(absmax_q + blk);
+          sc.s2 = __ldg(dq_scale + (blk >> 8));
+          sc.valid = true;
+        }
       }
+      return sc;
+    };
+    Scale p0 = fetch(grp), p1 = fetch(grp + DQ_GROUPS);
+    for (int it = grp; it < numK; it += DQ_GROUPS) {
+      const Scale p2 = fetch(it + 2 * DQ_GROUPS);
+      const int s = it % STAGES;
+      const uint32_t ph = (it / STAGES) & 1;
       if (!(ok = wait_bounded(full_tma(s), ph, abort, status))) break;
       const uint32_t c_s = base + OFF_C + s * C_BYTES;
       uint4 q0, q1;
@@ -215,10 +234,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         q0 = ld_shared_v4(c_s + row * 128 + (((2 * j) ^ (row & 7)) << 4));
         q1 = ld_shared_v4(c_s + row * 128 + (((2 * j + 1) ^ (row & 7)) << 4));
       }
-      const uint32_t b_row = base + OFF_B + s * B_BYTES + srow * 128;
-      const uint32_t sw = srow & 7;
-      if (valid) {
-        const Nf4Lut lut = make_lut(lv, ap);
+      const uint32_t b_row = base + OFF_B + s * B_BYTES + t * 128;
+      const uint32_t sw = t & 7;
+      if (p0.valid) {
+        const Nf4Lut lut = make_lut(lv, __fmul_rn(static_cast<float>(p0.q), p0.s2));
         const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
@@ -233,6 +252,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(full_deq(s));
+      p0 = p1;
+      p1 = p2;
     }
 
     // -------------------------------------------------------- epilogue
@@ -240,10 +261,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (ok) {
       tc_fence_after();
       const int quad = warp & 3;                 // TMEM lanes 32*quad .. +31
-      const int h = (warp - 2) >> 2;             // accumulator: tokens 128h .. 128h+127
+      const int h = (e >> 2) & 1;                // accumulator: tokens 128h .. 128h+127
+      const int ch = e >> 3;                     // column half of the accumulator
       const int m = m0 + h * UM + quad * 32 + lane;
 #pragma unroll 1
-      for (int col = 0; col < BN; col += 32) {
+      for (int col = ch * (BN / 2); col < (ch + 1) * (BN / 2); col += 32) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(h * 256 + col),
                            v);
