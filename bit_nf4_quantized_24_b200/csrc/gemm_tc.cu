@@ -1,28 +1,35 @@
-// Fused NF4-dequant GEMM on the sm_100a tensor cores (tcgen05 + TMEM).
+// Fused NF4-dequant GEMM on the sm_100a tensor cores (tcgen05 + TMEM), run by
+// pairs of CTAs on two SMs (cta_group::2).
 //
 // katajob, "NF4: 4-bit NormalFloat": the 4-bit weight is expanded block by
 // block to bf16 only for the product and thrown away afterwards.  Here the
 // expanded weight tile exists only in shared memory, one pipeline stage at a
 // time, as the B operand of tcgen05.mma.
 //
-// Tile: 256 tokens (M) x 256 outputs (N) x 64 contraction (K) per stage, as
-// two 128 x 256 fp32 accumulators in TMEM (all 512 columns) that share every
-// dequantized weight tile, so each expanded weight feeds 256 tokens.
 //   mode 0, forward:  D[m, n] = sum_k X[m,k] W'[n,k]       (W' K-major)
 //   mode 1, dX:       D[m, k] = sum_n dY[m,n] W'[n,k]      (W' MN-major)
 // followed by one tail stage that adds the LoRA product from bf16 operands
 // loaded by TMA: Hs B^T (forward, Hs = s*H) or dH A (dX).
 //
-// Warp roles (576 threads):
+// Tiling.  A cluster of 2 CTAs (one per SM) computes 512 tokens x 256 outputs.
+// Each CTA owns 256 tokens (its A tile, two 128-row halves) and expands half of
+// the 256-row weight tile (128 rows) into its own shared memory.  The leader
+// CTA issues tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16): the MMA
+// reads the A rows and the B half of both CTAs and writes 128 x 256 fp32 into
+// each CTA's TMEM.  Two such MMAs per k16 step (one per A half) fill all 512
+// TMEM columns of both SMs.  Per SM this halves the dequantization work and
+// the B-operand shared-memory traffic of a single-CTA tile of the same size.
+//
+// Warp roles (576 threads per CTA):
 //   warp 0       TMA producer: activation tile + NF4 code tile per stage
-//   warp 1       TMEM allocator and single-thread MMA issuer
-//   warps 2..17  dequantizers in two groups of 8 that take alternate stages
-//                (one 64-weight block per thread per stage: register lookup
-//                table -> 128 B of swizzled bf16 in smem); each thread loads
-//                its blocks' absmax code and group scale four stages ahead.
-//                Then all 16 run the epilogue (TMEM -> bf16 -> global).
+//   warp 1       TMEM allocation (both CTAs); MMA issue (leader only)
+//   warps 2..17  dequantizers in four groups of four that take every fourth
+//                stage (one 64-weight block per thread per stage: register
+//                lookup table -> 128 B of swizzled bf16 in smem); the scale
+//                of each block is loaded eight stages ahead.  They signal the
+//                leader's barrier (the peer remotely), then run the epilogue.
 // Every wait is bounded (kWaitLimitNs); on expiry the kernel records
-// kDevTimeout, drains its in-flight copies and MMAs, frees TMEM and exits.
+// kDevTimeout, drains what it issued, frees TMEM and exits.
 #include <mutex>
 
 #include "internal.h"
@@ -31,34 +38,40 @@ namespace qn {
 
 namespace {
 
-constexpr int BM = 256, UM = 128, BN = 256, BK = 64, STAGES = 3;
-constexpr int A_BYTES = BM * BK * 2;     // 32 KB (two 128-row halves)
-constexpr int B_BYTES = BN * BK * 2;     // 32 KB
-constexpr int C_BYTES = BN * BK / 2;     // 8 KB of packed codes
+constexpr int BM = 256;              // tokens per CTA (two MMA halves of 128)
+constexpr int UM = 128;              // rows of A each CTA gives one pair MMA
+constexpr int BN = 256;              // outputs per pair (N of the MMA)
+constexpr int BNL = BN / 2;          // outputs expanded by each CTA
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+constexpr int DQ_GROUPS = 4;         // dequant groups of 4 warps (128 threads)
+constexpr int A_BYTES = BM * BK * 2;     // 32 KB
+constexpr int B_BYTES = BNL * BK * 2;    // 16 KB
+constexpr int C_BYTES = BNL * BK / 2;    // 4 KB of packed codes
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
 constexpr int OFF_C = OFF_B + STAGES * B_BYTES;
 constexpr int OFF_BAR = OFF_C + STAGES * C_BYTES;
 constexpr int SMEM_USED = OFF_BAR + 256;
 constexpr int SMEM_ALLOC = SMEM_USED + 1024;  // slack for 1024-byte alignment
-constexpr int DQ_GROUPS = 2;                       // dequant groups of 8 warps
-constexpr int NUM_THREADS = 64 + DQ_GROUPS * 256;
+constexpr int NUM_THREADS = 64 + DQ_GROUPS * 128;
 constexpr int TMEM_COLS = 512;  // accumulator h at columns 256h .. 256h+255
 
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 
 struct Bars {
-  uint64_t full_tma[STAGES];  // activation + code tiles landed (tx bytes)
-  uint64_t full_deq[STAGES];  // 8 dequant warps finished the B tile
-  uint64_t empty[STAGES];     // MMAs of the stage completed
-  uint64_t accum;             // all MMAs completed
-  uint64_t drain;             // used only when aborting
+  uint64_t full_tma[STAGES];  // this CTA's activation + code tiles landed
+  uint64_t full_deq[STAGES];  // leader: both CTAs' B halves (and tail tiles) ready
+  uint64_t empty[STAGES];     // MMAs of the stage completed (multicast by the leader)
+  uint64_t accum;             // all MMAs completed (multicast by the leader)
+  uint64_t drain;             // leader: used only when aborting
+  uint64_t dealloc;           // the other CTA finished with the pair's TMEM
   uint32_t tmem_base;
   int abort;
 };
 
 template <int MODE>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(NUM_THREADS, 1)
     k_nf4_gemm(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_codes,
                const __grid_constant__ CUtensorMap tm_tail_a, const __grid_constant__ CUtensorMap tm_tail_b,
                const uint8_t* __restrict__ absmax_q, const float* __restrict__ dq_scale, Nf4Levels lv, int M, int N,
@@ -74,24 +87,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   auto empty = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
   const uint32_t accum_bar = bar0 + 8u * (3 * STAGES);
   const uint32_t drain_bar = bar0 + 8u * (3 * STAGES + 1);
+  const uint32_t dealloc_bar = bar0 + 8u * (3 * STAGES + 2);
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0 = leader, 1 = peer
+  const bool leader = rank == 0;
   // mode 0: contraction K, outputs N.  mode 1: contraction N, outputs K.
   const int Kc = MODE == 0 ? K : N;
   const int Nout = MODE == 0 ? N : K;
   const int numK = (Kc + BK - 1) / BK;
-  const int n0 = blockIdx.x * BN;  // first output column of the tile
-  const int m0 = blockIdx.y * BM;  // first token of the tile
+  const int n0 = blockIdx.x * BN;                       // first output of the pair's tile
+  const int nl0 = n0 + BNL * static_cast<int>(rank);    // first output this CTA expands
+  const int m0 = blockIdx.y * BM;                       // first token of this CTA
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full_tma(s), 1);
-      mbar_init(full_deq(s), 8);
+      mbar_init(full_deq(s), 2 * 4);  // the stage group's 4 warps in each CTA
       mbar_init(empty(s), 1);
     }
     mbar_init(accum_bar, 1);
     mbar_init(drain_bar, 1);
+    mbar_init(dealloc_bar, 1);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -102,11 +120,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tm_tail_b);
   }
   if (warp == 1) {
-    tmem_alloc(base + OFF_BAR + static_cast<uint32_t>(offsetof(Bars, tmem_base)), TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(base + OFF_BAR + static_cast<uint32_t>(offsetof(Bars, tmem_base)), TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
@@ -122,9 +140,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mbar_arrive_expect_tx(full_tma(s), A_BYTES + C_BYTES);
         tma_load_2d(base + OFF_A + s * A_BYTES, &tm_act, full_tma(s), it * BK, m0);
         if (MODE == 0)
-          tma_load_2d(base + OFF_C + s * C_BYTES, &tm_codes, full_tma(s), it * (BK / 2), n0);
+          tma_load_2d(base + OFF_C + s * C_BYTES, &tm_codes, full_tma(s), it * (BK / 2), nl0);
         else
-          tma_load_2d(base + OFF_C + s * C_BYTES, &tm_codes, full_tma(s), n0 / 2, it * BK);
+          tma_load_2d(base + OFF_C + s * C_BYTES, &tm_codes, full_tma(s), nl0 / 2, it * BK);
         ++issued;
       }
       if (ok) {  // tail stage: LoRA operands
@@ -134,11 +152,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           mbar_arrive_expect_tx(full_tma(s), A_BYTES + B_BYTES);
           tma_load_2d(base + OFF_A + s * A_BYTES, &tm_tail_a, full_tma(s), 0, m0);
           if (MODE == 0) {
-            tma_load_2d(base + OFF_B + s * B_BYTES, &tm_tail_b, full_tma(s), 0, n0);
+            tma_load_2d(base + OFF_B + s * B_BYTES, &tm_tail_b, full_tma(s), 0, nl0);
           } else {
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j)
-              tma_load_2d(base + OFF_B + s * B_BYTES + j * 8192, &tm_tail_b, full_tma(s), n0 + 64 * j, 0);
+            for (int j = 0; j < BNL / 64; ++j)
+              tma_load_2d(base + OFF_B + s * B_BYTES + j * 8192, &tm_tail_b, full_tma(s), nl0 + 64 * j, 0);
           }
           ++issued;
         }
@@ -150,16 +168,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(UM, BN, false, MODE == 1);
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(2 * UM, BN, false, MODE == 1);
       bool ok = true;
       int committed = 0;
       for (int it = 0; it <= numK; ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
         const bool tail = (it == numK);
-        if (!(ok = wait_bounded(full_tma(s), ph, abort, status))) break;
-        if (!tail && !(ok = wait_bounded(full_deq(s), ph, abort, status))) break;
+        // full_deq gathers both CTAs: their tiles landed and their B halves are written
+        if (!(ok = wait_bounded_cluster(full_deq(s), ph, abort, status))) break;
         tc_fence_after();
         const uint32_t a_s = base + OFF_A + s * A_BYTES;
         const uint32_t b_s = base + OFF_B + s * B_BYTES;
@@ -168,34 +186,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint64_t bd = MODE == 0 ? desc_sw128(b_s + kk * 32, 16, 1024)
                                         : desc_sw128(b_s + kk * 2048, 8192, 1024);
           const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-          tc_mma_f16(tmem, desc_sw128(a_s + kk * 32, 16, 1024), bd, idesc, acc);
-          tc_mma_f16(tmem + 256, desc_sw128(a_s + UM * 128 + kk * 32, 16, 1024), bd, idesc, acc);
+          tc_mma_f16_pair(tmem, desc_sw128(a_s + kk * 32, 16, 1024), bd, idesc, acc);
+          tc_mma_f16_pair(tmem + 256, desc_sw128(a_s + UM * 128 + kk * 32, 16, 1024), bd, idesc, acc);
         }
-        tc_commit(empty(s));
+        tc_commit_pair(empty(s));
         committed = 1;
       }
       if (ok) {
-        tc_commit(accum_bar);
+        tc_commit_pair(accum_bar);
       } else if (committed) {  // wait for MMAs in flight before TMEM is freed
-        tc_commit(drain_bar);
+        tc_commit_pair(drain_bar);
         wait_drain(drain_bar, 0);
       }
     }
   } else {
     // ------------------------------------------- dequantizers, then epilogue
-    const int e = warp - 2;            // 0..15
-    const int grp = e >> 3;            // stages it = grp, grp + 2, ...
-    const int t = (e & 7) * 32 + lane; // item of the stage: 0..255
+    const int e = warp - 2;             // 0..15
+    const int grp = e >> 2;             // stages it = grp, grp + 4, ...
+    const int t = (e & 3) * 32 + lane;  // item of the stage: 0..127
+    const uint32_t deq_bar_leader0 = mapa_shared(full_deq(0), 0);
     bool ok = true;
-    const int KB = K / 64;             // 64-blocks per weight row
-    // which (row, 64-block) of W this thread expands at iteration it
+    const int KB = K / 64;              // 64-blocks per weight row
+    // which (row, 64-block) of W this thread expands at iteration it; its
+    // expansion goes to row t of this CTA's B stage
     auto item_of = [&](int it, int& wrow, int& kcol0) {
       if (MODE == 0) {
-        wrow = n0 + t;
+        wrow = nl0 + t;
         kcol0 = it * BK;
       } else {
         wrow = it * BK + (t & 63);
-        kcol0 = n0 + 64 * (t >> 6);  // smem row t = 64 * (t >> 6) + (t & 63)
+        kcol0 = nl0 + 64 * (t >> 6);  // smem row t = 64 * (t >> 6) + (t & 63)
       }
     };
     struct Scale {
@@ -218,40 +238,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       return sc;
     };
     Scale p0 = fetch(grp), p1 = fetch(grp + DQ_GROUPS);
-    for (int it = grp; it < numK; it += DQ_GROUPS) {
+    for (int it = grp; it <= numK; it += DQ_GROUPS) {  // it == numK: the tail stage
       const Scale p2 = fetch(it + 2 * DQ_GROUPS);
       const int s = it % STAGES;
       const uint32_t ph = (it / STAGES) & 1;
       if (!(ok = wait_bounded(full_tma(s), ph, abort, status))) break;
-      const uint32_t c_s = base + OFF_C + s * C_BYTES;
-      uint4 q0, q1;
-      if (MODE == 0) {  // code tile [256 rows][32 B], 32-byte swizzle
-        const uint32_t sw = (static_cast<uint32_t>(t) >> 2) & 1u;
-        q0 = ld_shared_v4(c_s + t * 32 + ((0u ^ sw) << 4));
-        q1 = ld_shared_v4(c_s + t * 32 + ((1u ^ sw) << 4));
-      } else {          // code tile [64 rows][128 B], 128-byte swizzle
-        const uint32_t row = t & 63, j = t >> 6;
-        q0 = ld_shared_v4(c_s + row * 128 + (((2 * j) ^ (row & 7)) << 4));
-        q1 = ld_shared_v4(c_s + row * 128 + (((2 * j + 1) ^ (row & 7)) << 4));
-      }
-      const uint32_t b_row = base + OFF_B + s * B_BYTES + t * 128;
-      const uint32_t sw = t & 7;
-      if (p0.valid) {
-        const Nf4Lut lut = make_lut(lv, __fmul_rn(static_cast<float>(p0.q), p0.s2));
-        const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint32_t o0, o1, o2, o3;
-          deq8(w[c], lut, o0, o1, o2, o3);
-          st_shared_v4(b_row + ((c ^ sw) << 4), o0, o1, o2, o3);
+      if (it < numK) {
+        const uint32_t c_s = base + OFF_C + s * C_BYTES;
+        uint4 q0, q1;
+        if (MODE == 0) {  // code tile [128 rows][32 B], 32-byte swizzle
+          const uint32_t sw = (static_cast<uint32_t>(t) >> 2) & 1u;
+          q0 = ld_shared_v4(c_s + t * 32 + ((0u ^ sw) << 4));
+          q1 = ld_shared_v4(c_s + t * 32 + ((1u ^ sw) << 4));
+        } else {          // code tile [64 rows][64 B], 64-byte swizzle
+          const uint32_t row = t & 63, j = t >> 6, sw = (row >> 1) & 3u;
+          q0 = ld_shared_v4(c_s + row * 64 + (((2 * j) ^ sw) << 4));
+          q1 = ld_shared_v4(c_s + row * 64 + (((2 * j + 1) ^ sw) << 4));
         }
-      } else {
+        const uint32_t b_row = base + OFF_B + s * B_BYTES + t * 128;
+        const uint32_t sw = t & 7;
+        if (p0.valid) {
+          const Nf4Lut lut = make_lut(lv, __fmul_rn(static_cast<float>(p0.q), p0.s2));
+          const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
-        for (int c = 0; c < 8; ++c) st_shared_v4(b_row + (c << 4), 0u, 0u, 0u, 0u);
+          for (int c = 0; c < 8; ++c) {
+            uint32_t o0, o1, o2, o3;
+            deq8(w[c], lut, o0, o1, o2, o3);
+            st_shared_v4(b_row + ((c ^ sw) << 4), o0, o1, o2, o3);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) st_shared_v4(b_row + (c << 4), 0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(full_deq(s));
+      if (lane == 0) {
+        if (leader) mbar_arrive(full_deq(s));
+        else mbar_arrive_remote(deq_bar_leader0 + 8u * s);
+      }
       p0 = p1;
       p1 = p2;
     }
@@ -289,11 +314,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   }
 
+  // Both CTAs must be done with the pair's TMEM before it is freed: each tells
+  // the other (remote arrive) and waits for the other's word (bounded).
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    if (lane == 0) {
+      mbar_arrive_remote(mapa_shared(dealloc_bar, rank ^ 1u));
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait_cluster(dealloc_bar, 0)) {
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+          atomicExch(status, kDevTimeout);
+          break;
+        }
+      }
+    }
+    __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    tmem_dealloc_pair(tmem, TMEM_COLS);
   }
 }
 
@@ -339,28 +377,24 @@ cudaError_t launch_mode(const GemmArgs& a, cudaStream_t st) {
   const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
   bool ok = make_map(&tm_act, BF16, a.act, Kc, a.M, Kc * 2, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B);
   if (MODE == 0)
-    ok = ok && make_map(&tm_codes, U8, a.codes, a.K / 2, a.N, a.K / 2, BK / 2, BN, CU_TENSOR_MAP_SWIZZLE_32B);
+    ok = ok && make_map(&tm_codes, U8, a.codes, a.K / 2, a.N, a.K / 2, BK / 2, BNL, CU_TENSOR_MAP_SWIZZLE_32B);
   else
-    ok = ok && make_map(&tm_codes, U8, a.codes, a.K / 2, a.N, a.K / 2, BN / 2, BK, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && make_map(&tm_codes, U8, a.codes, a.K / 2, a.N, a.K / 2, BNL / 2, BK, CU_TENSOR_MAP_SWIZZLE_64B);
   ok = ok && make_map(&tm_ta, BF16, a.tail_a, a.r, a.M, a.r * 2, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B);
   if (MODE == 0)
-    ok = ok && make_map(&tm_tb, BF16, a.tail_b, a.r, a.N, a.r * 2, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok = ok && make_map(&tm_tb, BF16, a.tail_b, a.r, a.N, a.r * 2, 64, BNL, CU_TENSOR_MAP_SWIZZLE_128B);
   else
     ok = ok && make_map(&tm_tb, BF16, a.tail_b, a.K, a.r, a.K * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return cudaErrorInvalidValue;
 
-  static std::once_flag attr_once[2];
-  cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once[MODE], [&] {
-    attr_err = cudaFuncSetAttribute(k_nf4_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
-  });
-  if (attr_err != cudaSuccess) return attr_err;
-  // The attribute is per device; set it again cheaply on every launch so a
-  // second device is covered too.
+  // The attribute is per device; setting it on every launch covers every device.
   cudaError_t e = cudaFuncSetAttribute(k_nf4_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
   if (e != cudaSuccess) return e;
 
-  const dim3 grid(static_cast<unsigned>((Nout + BN - 1) / BN), static_cast<unsigned>((a.M + BM - 1) / BM));
+  // Token tiles are rounded up to whole pairs: a CTA past the last token
+  // feeds zeros (TMA fills out-of-range rows) to its half and stores nothing.
+  const int64_t mt = (a.M + BM - 1) / BM;
+  const dim3 grid(static_cast<unsigned>((Nout + BN - 1) / BN), static_cast<unsigned>((mt + 1) / 2 * 2));
   trace_before(st);
   k_nf4_gemm<MODE><<<grid, NUM_THREADS, SMEM_ALLOC, st>>>(
       tm_act, tm_codes, tm_ta, tm_tb, a.absmax_q, a.dq_scale, host_codebook().levels, static_cast<int>(a.M),
