@@ -64,6 +64,8 @@ def lib():
     L.qlora_device_status.restype = i32
     L.qlora_trace_gemm_events.argtypes = [P, i32]
     L.qlora_trace_gemm_count.restype = i32
+    L.qlora_gemm_resident_pairs.argtypes = [i32]
+    L.qlora_gemm_resident_pairs.restype = i32
     _lib = L
     return L
 
@@ -240,6 +242,11 @@ def qlora_linear_fwd_noalloc(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: 
                                           _ptr(A), _ptr(B), r, float(scale), _ptr(out), _ptr(H), _stream(stream)),
            "qlora_linear_fwd_noalloc")
     return out, H
+
+
+def gemm_resident_pairs(mode: int = 0) -> int:
+    """CTA pairs of the fused GEMM that fit on the current device at once."""
+    return lib().qlora_gemm_resident_pairs(mode)
 
 
 def device_status() -> int:

@@ -327,4 +327,10 @@ int qlora_trace_gemm_events(void** events, int n_pairs) {
 
 int qlora_trace_gemm_count(void) { return g_trace_count; }
 
+int qlora_gemm_resident_pairs(int mode) {
+  if (mode != 0 && mode != 1) return QLORA_ERR_ARG;
+  const int n = nf4_gemm_max_active_pairs(mode);
+  return n < 0 ? QLORA_ERR_CUDA : n;
+}
+
 }  // extern "C"

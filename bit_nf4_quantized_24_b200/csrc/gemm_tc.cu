@@ -71,7 +71,7 @@ struct Bars {
 };
 
 template <int MODE>
-__global__ void __cluster_dims__(1, 2, 1) __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(NUM_THREADS, 1)
     k_nf4_gemm(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_codes,
                const __grid_constant__ CUtensorMap tm_tail_a, const __grid_constant__ CUtensorMap tm_tail_b,
                const uint8_t* __restrict__ absmax_q, const float* __restrict__ dq_scale, Nf4Levels lv, int M, int N,
@@ -395,14 +395,44 @@ cudaError_t launch_mode(const GemmArgs& a, cudaStream_t st) {
   // feeds zeros (TMA fills out-of-range rows) to its half and stores nothing.
   const int64_t mt = (a.M + BM - 1) / BM;
   const dim3 grid(static_cast<unsigned>((Nout + BN - 1) / BN), static_cast<unsigned>((mt + 1) / 2 * 2));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_ALLOC;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 2;  // the two CTAs of a pair hold consecutive token tiles
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   trace_before(st);
-  k_nf4_gemm<MODE><<<grid, NUM_THREADS, SMEM_ALLOC, st>>>(
-      tm_act, tm_codes, tm_ta, tm_tb, a.absmax_q, a.dq_scale, host_codebook().levels, static_cast<int>(a.M),
-      static_cast<int>(a.N), static_cast<int>(a.K), a.r, reinterpret_cast<__nv_bfloat16*>(a.out),
-      device_status_ptr());
-  e = cudaGetLastError();
+  e = cudaLaunchKernelEx(&cfg, k_nf4_gemm<MODE>, tm_act, tm_codes, tm_ta, tm_tb, a.absmax_q, a.dq_scale,
+                         host_codebook().levels, static_cast<int>(a.M), static_cast<int>(a.N), static_cast<int>(a.K),
+                         a.r, reinterpret_cast<__nv_bfloat16*>(a.out), device_status_ptr());
   trace_after(st);
   return e;
+}
+
+template <int MODE>
+int max_active_pairs() {
+  if (cudaFuncSetAttribute(k_nf4_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC) != cudaSuccess)
+    return -1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1, 2, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_ALLOC;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 2;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, k_nf4_gemm<MODE>, &cfg) != cudaSuccess) return -2;
+  return n;
 }
 
 }  // namespace
@@ -410,5 +440,7 @@ cudaError_t launch_mode(const GemmArgs& a, cudaStream_t st) {
 cudaError_t launch_nf4_gemm(const GemmArgs& a, cudaStream_t st) {
   return a.mode == 0 ? launch_mode<0>(a, st) : launch_mode<1>(a, st);
 }
+
+int nf4_gemm_max_active_pairs(int mode) { return mode == 0 ? max_active_pairs<0>() : max_active_pairs<1>(); }
 
 }  // namespace qn

@@ -44,6 +44,9 @@ struct GemmArgs {
   uint16_t* out;  // Y [M, N] or dX [M, K]
 };
 cudaError_t launch_nf4_gemm(const GemmArgs& a, cudaStream_t st);
+// CTA pairs of the fused GEMM that fit on the current device at once
+// (negative: the occupancy query failed).
+int nf4_gemm_max_active_pairs(int mode);
 
 // ----- adapter kernels
 // out[m, j] = sum_k P[m,k] Q[j,k]  (P bf16 [M, Kc], Q bf16 [R, Kc]); writes

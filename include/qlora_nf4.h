@@ -191,6 +191,11 @@ int qlora_trace_gemm_events(void** events, int n_pairs);
 /* Number of event pairs recorded since the last qlora_trace_gemm_events. */
 int qlora_trace_gemm_count(void);
 
+/* How many CTA pairs (2-SM clusters) of the fused dequant-GEMM kernel can be
+ * resident at once on the current device; mode 0 = forward, 1 = dX.  A value
+ * of 0 means the kernel cannot launch on this device.  Errors: ARG, CUDA. */
+int qlora_gemm_resident_pairs(int mode);
+
 #ifdef __cplusplus
 }
 #endif
