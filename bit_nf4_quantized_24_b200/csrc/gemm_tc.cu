@@ -97,9 +97,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int Kc = MODE == 0 ? K : N;
   const int Nout = MODE == 0 ? N : K;
   const int numK = (Kc + BK - 1) / BK;
-  const int n0 = blockIdx.x * BN;                       // first output of the pair's tile
+  const int n0 = blockIdx.y * BN;                       // first output of the pair's tile
   const int nl0 = n0 + BNL * static_cast<int>(rank);    // first output this CTA expands
-  const int m0 = blockIdx.y * BM;                       // first token of this CTA
+  const int m0 = blockIdx.x * BM;                       // first token of this CTA (pairs along x)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -394,7 +394,7 @@ cudaError_t launch_mode(const GemmArgs& a, cudaStream_t st) {
   // Token tiles are rounded up to whole pairs: a CTA past the last token
   // feeds zeros (TMA fills out-of-range rows) to its half and stores nothing.
   const int64_t mt = (a.M + BM - 1) / BM;
-  const dim3 grid(static_cast<unsigned>((Nout + BN - 1) / BN), static_cast<unsigned>((mt + 1) / 2 * 2));
+  const dim3 grid(static_cast<unsigned>((mt + 1) / 2 * 2), static_cast<unsigned>((Nout + BN - 1) / BN));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
@@ -402,8 +402,8 @@ cudaError_t launch_mode(const GemmArgs& a, cudaStream_t st) {
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = 2;  // the two CTAs of a pair hold consecutive token tiles
+  attr[0].val.clusterDim.x = 2;  // the two CTAs of a pair hold consecutive token tiles
+  attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
@@ -420,13 +420,13 @@ int max_active_pairs() {
   if (cudaFuncSetAttribute(k_nf4_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC) != cudaSuccess)
     return -1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(1, 2, 1);
+  cfg.gridDim = dim3(2, 1, 1);
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = SMEM_ALLOC;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = 2;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
