@@ -21,7 +21,8 @@
 // the B-operand shared-memory traffic of a single-CTA tile of the same size.
 //
 // Warp roles (576 threads per CTA):
-//   warp 0       TMA producer: activation tile + NF4 code tile per stage
+//   warp 0       TMA producer: NF4 code tiles into an 8-deep ring, CAHEAD
+//                stages ahead of the activation tiles (4-deep ring)
 //   warp 1       TMEM allocation (both CTAs); MMA issue (leader only)
 //   warps 2..17  dequantizers in four groups of four that take every fourth
 //                stage (one 64-weight block per thread per stage: register
@@ -30,6 +31,7 @@
 //                leader's barrier (the peer remotely), then run the epilogue.
 // Every wait is bounded (kWaitLimitNs); on expiry the kernel records
 // kDevTimeout, drains what it issued, frees TMEM and exits.
+#include <algorithm>
 #include <mutex>
 
 #include "internal.h"
@@ -43,7 +45,9 @@ constexpr int UM = 128;              // rows of A each CTA gives one pair MMA
 constexpr int BN = 256;              // outputs per pair (N of the MMA)
 constexpr int BNL = BN / 2;          // outputs expanded by each CTA
 constexpr int BK = 64;
-constexpr int STAGES = 4;
+constexpr int STAGES = 4;             // activation (A) and expanded-weight (B) ring
+constexpr int CSTAGES = 8;            // NF4 code ring: codes run CAHEAD stages ahead of A
+constexpr int CAHEAD = 4;
 constexpr int DQ_GROUPS = 4;         // dequant groups of 4 warps (128 threads)
 constexpr int A_BYTES = BM * BK * 2;     // 32 KB
 constexpr int B_BYTES = BNL * BK * 2;    // 16 KB
@@ -51,7 +55,7 @@ constexpr int C_BYTES = BNL * BK / 2;    // 4 KB of packed codes
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
 constexpr int OFF_C = OFF_B + STAGES * B_BYTES;
-constexpr int OFF_BAR = OFF_C + STAGES * C_BYTES;
+constexpr int OFF_BAR = OFF_C + CSTAGES * C_BYTES;
 constexpr int SMEM_USED = OFF_BAR + 256;
 constexpr int SMEM_ALLOC = SMEM_USED + 1024;  // slack for 1024-byte alignment
 constexpr int NUM_THREADS = 64 + DQ_GROUPS * 128;
@@ -60,9 +64,11 @@ constexpr int TMEM_COLS = 512;  // accumulator h at columns 256h .. 256h+255
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 
 struct Bars {
-  uint64_t full_tma[STAGES];  // this CTA's activation + code tiles landed
-  uint64_t full_deq[STAGES];  // leader: both CTAs' B halves (and tail tiles) ready
+  uint64_t full_tma[STAGES];  // this CTA's activation tile (or tail tiles) landed
+  uint64_t full_deq[STAGES];  // leader: both CTAs' A tiles landed and B halves written
   uint64_t empty[STAGES];     // MMAs of the stage completed (multicast by the leader)
+  uint64_t full_c[CSTAGES];   // this CTA's code tile landed
+  uint64_t empty_c[CSTAGES];  // this CTA's dequantizers finished with a code tile
   uint64_t accum;             // all MMAs completed (multicast by the leader)
   uint64_t drain;             // leader: used only when aborting
   uint64_t dealloc;           // the other CTA finished with the pair's TMEM
@@ -75,7 +81,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_nf4_gemm(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_codes,
                const __grid_constant__ CUtensorMap tm_tail_a, const __grid_constant__ CUtensorMap tm_tail_b,
                const uint8_t* __restrict__ absmax_q, const float* __restrict__ dq_scale, Nf4Levels lv, int M, int N,
-               int K, int r, __nv_bfloat16* __restrict__ out, int* status) {
+               int K, int r, int band_pairs, __nv_bfloat16* __restrict__ out, int* status) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -85,9 +91,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   auto full_tma = [&](int s) { return bar0 + 8u * s; };
   auto full_deq = [&](int s) { return bar0 + 8u * (STAGES + s); };
   auto empty = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
-  const uint32_t accum_bar = bar0 + 8u * (3 * STAGES);
-  const uint32_t drain_bar = bar0 + 8u * (3 * STAGES + 1);
-  const uint32_t dealloc_bar = bar0 + 8u * (3 * STAGES + 2);
+  auto full_c = [&](int c) { return bar0 + 8u * (3 * STAGES + c); };
+  auto empty_c = [&](int c) { return bar0 + 8u * (3 * STAGES + CSTAGES + c); };
+  const uint32_t accum_bar = bar0 + 8u * (3 * STAGES + 2 * CSTAGES);
+  const uint32_t drain_bar = accum_bar + 8u;
+  const uint32_t dealloc_bar = accum_bar + 16u;
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -97,15 +105,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int Kc = MODE == 0 ? K : N;
   const int Nout = MODE == 0 ? N : K;
   const int numK = (Kc + BK - 1) / BK;
-  const int n0 = blockIdx.y * BN;                       // first output of the pair's tile
+  // Pairs are handed out band by band: a band of `band_pairs` token pairs
+  // sweeps every output tile before the next band starts, so the band's
+  // activations stay in L2 while the weight tiles stream past them.
+  int pair, otile;
+  {
+    const int npx = gridDim.x >> 1, nout = gridDim.y;
+    const int L = blockIdx.y * npx + (blockIdx.x >> 1);  // launch order of the pair
+    const int per_band = band_pairs * nout;
+    const int band = L / per_band, rem = L - band * per_band;
+    const int in_band = min(band_pairs, npx - band * band_pairs);
+    otile = rem / in_band;
+    pair = band * band_pairs + (rem - otile * in_band);
+  }
+  const int n0 = otile * BN;                            // first output of the pair's tile
   const int nl0 = n0 + BNL * static_cast<int>(rank);    // first output this CTA expands
-  const int m0 = blockIdx.x * BM;                       // first token of this CTA (pairs along x)
+  const int m0 = (2 * pair + static_cast<int>(rank)) * BM;  // first token of this CTA
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full_tma(s), 1);
       mbar_init(full_deq(s), 2 * 4);  // the stage group's 4 warps in each CTA
       mbar_init(empty(s), 1);
+    }
+    for (int c = 0; c < CSTAGES; ++c) {
+      mbar_init(full_c(c), 1);
+      mbar_init(empty_c(c), 4);  // the 4 warps of the iteration's dequant group
     }
     mbar_init(accum_bar, 1);
     mbar_init(drain_bar, 1);
@@ -130,20 +155,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer
+    // Code tiles run CAHEAD iterations ahead of the activation tiles, so the
+    // expansion of a stage overlaps the latency of its activation tile.
     if (lane == 0) {
-      int issued = 0;
+      int a_issued = 0, c_issued = 0;
       bool ok = true;
+      auto issue_codes = [&](int it) {
+        const int c = it % CSTAGES;
+        if (!(ok = wait_bounded(empty_c(c), ((it / CSTAGES) & 1) ^ 1, abort, status))) return;
+        mbar_arrive_expect_tx(full_c(c), C_BYTES);
+        if (MODE == 0)
+          tma_load_2d(base + OFF_C + c * C_BYTES, &tm_codes, full_c(c), it * (BK / 2), nl0);
+        else
+          tma_load_2d(base + OFF_C + c * C_BYTES, &tm_codes, full_c(c), nl0 / 2, it * BK);
+        ++c_issued;
+      };
+      for (int it = 0; it < CAHEAD && it < numK && ok; ++it) issue_codes(it);
       for (int it = 0; it < numK && ok; ++it) {
+        if (it + CAHEAD < numK) {
+          issue_codes(it + CAHEAD);
+          if (!ok) break;
+        }
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
         if (!(ok = wait_bounded(empty(s), ph ^ 1, abort, status))) break;
-        mbar_arrive_expect_tx(full_tma(s), A_BYTES + C_BYTES);
+        mbar_arrive_expect_tx(full_tma(s), A_BYTES);
         tma_load_2d(base + OFF_A + s * A_BYTES, &tm_act, full_tma(s), it * BK, m0);
-        if (MODE == 0)
-          tma_load_2d(base + OFF_C + s * C_BYTES, &tm_codes, full_tma(s), it * (BK / 2), nl0);
-        else
-          tma_load_2d(base + OFF_C + s * C_BYTES, &tm_codes, full_tma(s), nl0 / 2, it * BK);
-        ++issued;
+        ++a_issued;
       }
       if (ok) {  // tail stage: LoRA operands
         const int it = numK, s = it % STAGES;
@@ -158,12 +196,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int j = 0; j < BNL / 64; ++j)
               tma_load_2d(base + OFF_B + s * B_BYTES + j * 8192, &tm_tail_b, full_tma(s), nl0 + 64 * j, 0);
           }
-          ++issued;
+          ++a_issued;
         }
       }
       if (!ok) {  // let the copies already issued land before the CTA exits
-        for (int it = (issued > STAGES ? issued - STAGES : 0); it < issued; ++it)
+        for (int it = (a_issued > STAGES ? a_issued - STAGES : 0); it < a_issued; ++it)
           wait_drain(full_tma(it % STAGES), (it / STAGES) & 1);
+        for (int it = (c_issued > CSTAGES ? c_issued - CSTAGES : 0); it < c_issued; ++it)
+          wait_drain(full_c(it % CSTAGES), (it / CSTAGES) & 1);
       }
     }
   } else if (warp == 1) {
@@ -242,9 +282,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const Scale p2 = fetch(it + 2 * DQ_GROUPS);
       const int s = it % STAGES;
       const uint32_t ph = (it / STAGES) & 1;
-      if (!(ok = wait_bounded(full_tma(s), ph, abort, status))) break;
       if (it < numK) {
-        const uint32_t c_s = base + OFF_C + s * C_BYTES;
+        const int cs = it % CSTAGES;
+        if (!(ok = wait_bounded(full_c(cs), (it / CSTAGES) & 1, abort, status))) break;
+        const uint32_t c_s = base + OFF_C + cs * C_BYTES;
         uint4 q0, q1;
         if (MODE == 0) {  // code tile [128 rows][32 B], 32-byte swizzle
           const uint32_t sw = (static_cast<uint32_t>(t) >> 2) & 1u;
@@ -255,6 +296,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           q0 = ld_shared_v4(c_s + row * 64 + (((2 * j) ^ sw) << 4));
           q1 = ld_shared_v4(c_s + row * 64 + (((2 * j + 1) ^ sw) << 4));
         }
+        // the B slot is free once the MMAs of iteration it - STAGES completed
+        if (!(ok = wait_bounded(empty(s), ph ^ 1, abort, status))) break;
         const uint32_t b_row = base + OFF_B + s * B_BYTES + t * 128;
         const uint32_t sw = t & 7;
         if (p0.valid) {
@@ -271,7 +314,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int c = 0; c < 8; ++c) st_shared_v4(b_row + (c << 4), 0u, 0u, 0u, 0u);
         }
         fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_c(cs));  // code tile consumed (values are in registers)
       }
+      // the stage's activation tile (or the tail tiles) must have landed too
+      if (!(ok = wait_bounded(full_tma(s), ph, abort, status))) break;
       __syncwarp();
       if (lane == 0) {
         if (leader) mbar_arrive(full_deq(s));
@@ -394,7 +441,11 @@ cudaError_t launch_mode(const GemmArgs& a, cudaStream_t st) {
   // Token tiles are rounded up to whole pairs: a CTA past the last token
   // feeds zeros (TMA fills out-of-range rows) to its half and stores nothing.
   const int64_t mt = (a.M + BM - 1) / BM;
-  const dim3 grid(static_cast<unsigned>((mt + 1) / 2 * 2), static_cast<unsigned>((Nout + BN - 1) / BN));
+  const int64_t npairs = (mt + 1) / 2;
+  const dim3 grid(static_cast<unsigned>(2 * npairs), static_cast<unsigned>((Nout + BN - 1) / BN));
+  // token pairs per band: keep a band's activations (512 tokens x Kc per pair) near 48 MB
+  const int64_t pair_bytes = int64_t(2) * BM * Kc * 2;
+  const int band_pairs = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(npairs, (48ll << 20) / pair_bytes)));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
@@ -410,7 +461,7 @@ cudaError_t launch_mode(const GemmArgs& a, cudaStream_t st) {
   trace_before(st);
   e = cudaLaunchKernelEx(&cfg, k_nf4_gemm<MODE>, tm_act, tm_codes, tm_ta, tm_tb, a.absmax_q, a.dq_scale,
                          host_codebook().levels, static_cast<int>(a.M), static_cast<int>(a.N), static_cast<int>(a.K),
-                         a.r, reinterpret_cast<__nv_bfloat16*>(a.out), device_status_ptr());
+                         a.r, band_pairs, reinterpret_cast<__nv_bfloat16*>(a.out), device_status_ptr());
   trace_after(st);
   return e;
 }
