@@ -206,7 +206,7 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             dp.allreduce_adapter_grads(dA, dB)
 
-    launches_per_step = 2 + 7  # fwd: rowdot, gemm; bwd: transpose, rowdot, gemm, 2x(coldot partial + reduce)
+    launches_per_step = 2 + 6  # fwd: rows, gemm; bwd: rows, gemm, 2x(cols partial + reduce)
 
     for _ in range(args.warmup):
         step()

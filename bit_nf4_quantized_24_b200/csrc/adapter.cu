@@ -1,9 +1,14 @@
 // LoRA adapter kernels ("QLoRA: fine-tuning a large model on one GPU",
 // "LoRA, stated once": h = W0 x + (alpha/r) B A x).  With H = X A^T:
 //   forward     H = X A^T                   (rowdot, contraction over K)
-//   backward    dH = s dY B                 (rowdot over N, with B^T)
+//   backward    dH = s dY B                 (rowdot over N, B read in place)
 //               dA = dH^T X, dB = s dY^T H  (coldot, contraction over tokens)
-// These are skinny (r <= 64 outputs per token) and bound by reading X / dY.
+// These are skinny (r <= 64 outputs per token) and bound by reading X or dY
+// once: a single thread streams tiles with TMA through a deep shared-memory
+// ring and the consumer warps run ldmatrix + mma.sync on swizzled tiles
+// (r is too narrow for a full tcgen05 tile).
+#include <algorithm>
+
 #include "internal.h"
 
 namespace qn {
@@ -19,80 +24,10 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint4 ldg_v4_or_zero(const uint16_t* p, bool ok) {
-  return ok ? __ldg(reinterpret_cast<const uint4*>(p)) : make_uint4(0u, 0u, 0u, 0u);
-}
-
-// out[m, j] = sum_k P[m,k] Q[j,k].  One CTA = 16 rows of P; its 8 warps split
-// the contraction into interleaved 32-wide chunks and meet in shared memory.
-// Inside a chunk, thread t (= lane & 3) owns the 8 consecutive k's 8t..8t+7;
-// they fill the fragment slots {2t, 2t+1, 2t+8, 2t+9} of two m16n8k16 steps.
-// The same k permutation is used for both operands, so the sum is unchanged.
-// U chunks are loaded before any is used, to keep enough bytes in flight.
-template <int NT, int U>  // NT = ceil(R / 8) n8 tiles
-__global__ void __launch_bounds__(256) k_rowdot(const uint16_t* __restrict__ P, const uint16_t* __restrict__ Q,
-                                                int M, int Kc, int R, float sa, uint16_t* __restrict__ out16a,
-                                                float sb, uint16_t* __restrict__ out16b, float* __restrict__ out32) {
-  __shared__ float red[8][16][NT * 8];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, t = lane & 3;
-  const int m0 = blockIdx.x * 16;
-  float acc[NT][4];
-#pragma unroll
-  for (int i = 0; i < NT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-  const int nchunks = (Kc + 31) / 32;
-  const bool row_lo = m0 + g < M, row_hi = m0 + g + 8 < M;
-  for (int c0 = warp; c0 < nchunks; c0 += 8 * U) {
-    uint4 alo[U], ahi[U], b[U][NT];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int k = (c0 + 8 * u) * 32 + 8 * t;
-      const bool kin = (c0 + 8 * u < nchunks) && k < Kc;
-      alo[u] = ldg_v4_or_zero(P + static_cast<int64_t>(m0 + g) * Kc + k, kin && row_lo);
-      ahi[u] = ldg_v4_or_zero(P + static_cast<int64_t>(m0 + g + 8) * Kc + k, kin && row_hi);
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int j = nt * 8 + g;
-        b[u][nt] = ldg_v4_or_zero(Q + static_cast<int64_t>(j) * Kc + k, kin && j < R);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        mma_bf16_16816(acc[nt], alo[u].x, ahi[u].x, alo[u].y, ahi[u].y, b[u][nt].x, b[u][nt].y);
-        mma_bf16_16816(acc[nt], alo[u].z, ahi[u].z, alo[u].w, ahi[u].w, b[u][nt].z, b[u][nt].w);
-      }
-    }
-  }
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    red[warp][g][nt * 8 + 2 * t] = acc[nt][0];
-    red[warp][g][nt * 8 + 2 * t + 1] = acc[nt][1];
-    red[warp][g + 8][nt * 8 + 2 * t] = acc[nt][2];
-    red[warp][g + 8][nt * 8 + 2 * t + 1] = acc[nt][3];
-  }
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < 16 * R; idx += blockDim.x) {
-    const int row = idx / R, j = idx % R;
-    const int m = m0 + row;
-    if (m >= M) continue;
-    float v = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) v += red[w][row][j];
-    const __nv_bfloat16 ha = __float2bfloat16_rn(sa * v);
-    out16a[static_cast<int64_t>(m) * R + j] = *reinterpret_cast<const uint16_t*>(&ha);
-    if (out16b) {
-      const __nv_bfloat16 hb = __float2bfloat16_rn(sb * v);
-      out16b[static_cast<int64_t>(m) * R + j] = *reinterpret_cast<const uint16_t*>(&hb);
-    }
-    if (out32) out32[static_cast<int64_t>(m) * R + j] = sb * v;
-  }
-}
-
-__device__ __forceinline__ void cp_async_16z(uint32_t dst, const void* src, bool valid) {
-  const int n = valid ? 16 : 0;  // 0 source bytes -> 16 zero bytes
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
 }
 __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
                                               uint32_t& r3) {
@@ -101,102 +36,240 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint3
                : "r"(addr));
 }
 
-// partial[split][j][c] = sum over this split's tokens m of G[m, j] P[m, c],
-// on the tensor cores: D[c, j] = sum_m P^T[c, m] G[m, j] with m16n8k16 tiles.
-// Both operands are row-major with the contraction (m) as the row index, so
-// 32-token slabs are staged in shared memory (cp.async, double-buffered,
-// rows padded by 16 B so the 8 rows of an ldmatrix phase hit distinct banks)
-// and read with ldmatrix.trans.  CTA = 128 columns x all R; warp w owns
-// columns 32w..32w+31.
-constexpr int CD_COLS = 128, CD_SLAB = 32, CD_PPITCH = CD_COLS + 8, CD_GPITCH = 64 + 8;
+// A narrow tile [rows][NT * 8] bf16 loaded by TMA with the swizzle that
+// matches its row pitch (NT = 2, 4, 8 -> 32, 64, 128 bytes).  Byte address of
+// the 16-byte chunk holding columns j .. j+7 of row `row`.
+template <int NT>
+__device__ __forceinline__ uint32_t narrow_addr(uint32_t tile, int row, int j) {
+  constexpr int PITCH = NT * 16;
+  const int chunk = j >> 3;
+  const int sw = ((row * PITCH) >> 7) & (PITCH / 16 - 1);
+  return tile + row * PITCH + ((chunk ^ sw) << 4);
+}
+template <int NT>
+constexpr CUtensorMapSwizzle narrow_swizzle() {
+  return NT == 2 ? CU_TENSOR_MAP_SWIZZLE_32B : NT == 4 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+}
 
-template <int NT>  // NT = ceil(R / 8) rounded up to even (ldmatrix.x4 feeds two n8 tiles)
-__global__ void __launch_bounds__(128) k_coldot_mma(const uint16_t* __restrict__ G, const uint16_t* __restrict__ P,
-                                                    int M, int C, int R, int rows_per_split,
-                                                    float* __restrict__ partial) {
-  __shared__ __align__(16) uint16_t sP[2][CD_SLAB][CD_PPITCH];
-  __shared__ __align__(16) uint16_t sG[2][CD_SLAB][CD_GPITCH];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, t = lane & 3;
-  const int c0 = blockIdx.x * CD_COLS;
-  const int split = blockIdx.y;
-  const int mb0 = split * rows_per_split;
-  const int mb1 = min(M, mb0 + rows_per_split);
-  const int nslab = mb1 > mb0 ? (mb1 - mb0 + CD_SLAB - 1) / CD_SLAB : 0;
-  const int gchunks = (R + 7) / 8;  // 16-byte chunks per G row
+// ------------------------------------------------------------------ rows
+//
+// out[m, j] = sum_k P[m, k] Q(j, k) for 16 * CW tokens per CTA over the whole
+// contraction.  P is bf16 [M, Kc]; Q is either [R, Kc] (QT = false: A) or
+// [Kc, R] (QT = true: lora_B, read in place for dH = dY B).  CW = NT / 2
+// consumer warps (16 tokens each) run ldmatrix + m16n8k16, the last warp's
+// lane 0 produces: per stage a (16 CW) x 64 tile of P (128-byte swizzle) and
+// the 64-wide slice of Q (as many bytes as the P tile, so Q costs no more L2
+// traffic than P), RW_ST stages in flight.
+constexpr int RW_ST = 8;
 
-  auto stage = [&](int sl, int buf) {
-    const int mb = mb0 + sl * CD_SLAB;
-    for (int u = tid; u < CD_SLAB * (CD_COLS / 8); u += 128) {
-      const int i = u / (CD_COLS / 8), cc = (u % (CD_COLS / 8)) * 8;
-      const bool ok = (mb + i < mb1) && (c0 + cc < C);
-      const uint16_t* src = ok ? P + static_cast<int64_t>(mb + i) * C + c0 + cc : P;
-      cp_async_16z(smem_u32(&sP[buf][i][cc]), src, ok);
+template <int NT>
+struct RowsSmem {
+  static constexpr int CW = NT / 2;
+  static constexpr int P_BYTES = 16 * CW * 64 * 2;
+  static constexpr int Q_BYTES = NT * 8 * 64 * 2;
+  static constexpr int OFF_Q = RW_ST * P_BYTES;
+  static constexpr int OFF_BAR = OFF_Q + RW_ST * Q_BYTES;
+  static constexpr int BYTES = OFF_BAR + 2 * RW_ST * 8 + 1024;
+};
+
+template <int NT, bool QT>
+__global__ void __launch_bounds__(32 * (NT / 2 + 1)) k_rows(const __grid_constant__ CUtensorMap tmP,
+                                                            const __grid_constant__ CUtensorMap tmQ, int M, int Kc,
+                                                            int R, float sa, uint16_t* __restrict__ out16a, float sb,
+                                                            uint16_t* __restrict__ out16b, float* __restrict__ out32,
+                                                            int* status) {
+  using S = RowsSmem<NT>;
+  constexpr int CW = S::CW;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const uint32_t full0 = base + S::OFF_BAR, empty0 = full0 + 8u * RW_ST;
+  __shared__ int abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * 16 * CW;
+  const int nk = (Kc + 63) / 64;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < RW_ST; ++s) {
+      mbar_init(full0 + 8u * s, 1);
+      mbar_init(empty0 + 8u * s, CW);
     }
-    for (int u = tid; u < CD_SLAB * 8; u += 128) {
-      const int i = u / 8, cc = (u % 8) * 8;
-      const bool ok = (mb + i < mb1) && (u % 8) < gchunks;
-      const uint16_t* src = ok ? G + static_cast<int64_t>(mb + i) * R + cc : G;
-      cp_async_16z(smem_u32(&sG[buf][i][cc]), src, ok);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == CW) {  // producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int it = 0; it < nk; ++it) {
+        const int s = it % RW_ST;
+        if (!wait_bounded(empty0 + 8u * s, ((it / RW_ST) & 1) ^ 1, &abort_flag, status)) break;
+        mbar_arrive_expect_tx(full0 + 8u * s, S::P_BYTES + S::Q_BYTES);
+        tma_load_2d(base + s * S::P_BYTES, &tmP, full0 + 8u * s, it * 64, m0);
+        if (QT)
+          tma_load_2d(base + S::OFF_Q + s * S::Q_BYTES, &tmQ, full0 + 8u * s, 0, it * 64);
+        else
+          tma_load_2d(base + S::OFF_Q + s * S::Q_BYTES, &tmQ, full0 + 8u * s, it * 64, 0);
+        ++issued;
+      }
+      for (int it = (issued > RW_ST ? issued - RW_ST : 0); it < issued; ++it)  // all copies land before exit
+        wait_drain(full0 + 8u * (it % RW_ST), (it / RW_ST) & 1);
     }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-  };
+    return;
+  }
 
-  float acc[2][NT][4];
+  float acc[NT][4];
 #pragma unroll
-  for (int a = 0; a < 2; ++a)
+  for (int i = 0; i < NT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+  const int q = lane >> 3, l7 = lane & 7;
+  for (int it = 0; it < nk; ++it) {
+    const int s = it % RW_ST;
+    if (!wait_bounded(full0 + 8u * s, (it / RW_ST) & 1, &abort_flag, status)) break;
+    const uint32_t pt = base + s * S::P_BYTES;
+    const uint32_t qt = base + S::OFF_Q + s * S::Q_BYTES;
 #pragma unroll
-    for (int n = 0; n < NT; ++n) acc[a][n][0] = acc[a][n][1] = acc[a][n][2] = acc[a][n][3] = 0.f;
-
-  if (nslab > 0) stage(0, 0);
-  for (int sl = 0; sl < nslab; ++sl) {
-    const int buf = sl & 1;
-    if (sl + 1 < nslab) stage(sl + 1, buf ^ 1);
-    else asm volatile("cp.async.commit_group;" ::: "memory");
-    asm volatile("cp.async.wait_group 1;" ::: "memory");
-    __syncthreads();
-    const int q = lane >> 3, rr = lane & 7;
-#pragma unroll
-    for (int ks = 0; ks < CD_SLAB / 16; ++ks) {
-      uint32_t a[2][4];
-#pragma unroll
-      for (int ct = 0; ct < 2; ++ct) {
-        // matrices: (m 0-7, c 0-7), (m 0-7, c 8-15), (m 8-15, c 0-7), (m 8-15, c 8-15)
-        const int m = ks * 16 + (q >> 1) * 8 + rr;
-        const int c = warp * 32 + ct * 16 + (q & 1) * 8;
-        ldsm_x4_trans(smem_u32(&sP[buf][m][c]), a[ct][0], a[ct][1], a[ct][2], a[ct][3]);
+    for (int k16 = 0; k16 < 4; ++k16) {
+      // A: (rows 0-7, k 0-7), (rows 8-15, k 0-7), (rows 0-7, k 8-15), (rows 8-15, k 8-15)
+      uint32_t a0, a1, a2, a3;
+      {
+        const int row = 16 * warp + l7 + (q & 1) * 8, chunk = 2 * k16 + (q >> 1);
+        ldsm_x4(pt + row * 128 + ((chunk ^ (row & 7)) << 4), a0, a1, a2, a3);
       }
 #pragma unroll
       for (int np = 0; np < NT / 2; ++np) {
-        // matrices: (m 0-7, tile 2np), (m 8-15, tile 2np), (m 0-7, tile 2np+1), (m 8-15, tile 2np+1)
-        const int m = ks * 16 + (q & 1) * 8 + rr;
-        const int j = (2 * np + (q >> 1)) * 8;
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_trans(smem_u32(&sG[buf][m][j]), b0, b1, b2, b3);
-#pragma unroll
-        for (int ct = 0; ct < 2; ++ct) {
-          mma_bf16_16816(acc[ct][2 * np], a[ct][0], a[ct][1], a[ct][2], a[ct][3], b0, b1);
-          mma_bf16_16816(acc[ct][2 * np + 1], a[ct][0], a[ct][1], a[ct][2], a[ct][3], b2, b3);
+        uint32_t b0, b1, b2, b3;  // (tile 2np: k 0-7, k 8-15), (tile 2np+1: k 0-7, k 8-15)
+        if (QT) {  // Q tile [64 k][NT*8 j], rows = contraction
+          const int kr = 16 * k16 + l7 + (q & 1) * 8, j = (2 * np + (q >> 1)) * 8;
+          ldsm_x4_trans(narrow_addr<NT>(qt, kr, j), b0, b1, b2, b3);
+        } else {   // Q tile [NT*8 j][64 k], 128-byte swizzle
+          const int j = (2 * np + (q >> 1)) * 8 + l7, chunk = 2 * k16 + (q & 1);
+          ldsm_x4(qt + j * 128 + ((chunk ^ (j & 7)) << 4), b0, b1, b2, b3);
         }
+        mma_bf16_16816(acc[2 * np], a0, a1, a2, a3, b0, b1);
+        mma_bf16_16816(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
       }
     }
-    __syncthreads();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty0 + 8u * s);
   }
+
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int m = m0 + 16 * warp + g + 8 * h;
+      const int j = nt * 8 + 2 * t;
+      if (m >= M || j >= R) continue;
+      const float v0 = acc[nt][2 * h], v1 = acc[nt][2 * h + 1];
+      const int64_t o = static_cast<int64_t>(m) * R + j;
+      *reinterpret_cast<uint32_t*>(out16a + o) = bf16x2_bits(sa * v0, sa * v1);
+      if (out16b) *reinterpret_cast<uint32_t*>(out16b + o) = bf16x2_bits(sb * v0, sb * v1);
+      if (out32) *reinterpret_cast<float2*>(out32 + o) = make_float2(sb * v0, sb * v1);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ cols
+//
+// partial[split][j][c] = sum over this split's tokens m of G[m, j] P[m, c]:
+// D[c, j] = sum_m P^T[c, m] G[m, j].  CTA = 64 columns c (4 consumer warps of
+// 16) x all R, over one token range (a multiple of 32 tokens); warp 4 lane 0
+// streams 32-token slabs of P (32 x 64, 128-byte swizzle) and G (32 x NT*8)
+// through CL_ST stages.  Both operands have the contraction as their row and
+// are read with ldmatrix.trans.  Rows past M arrive as zeros from TMA.
+constexpr int CL_ST = 8;
+
+template <int NT>
+struct ColsSmem {
+  static constexpr int P_BYTES = 32 * 64 * 2;
+  static constexpr int G_BYTES = 32 * NT * 8 * 2;
+  static constexpr int OFF_G = CL_ST * P_BYTES;
+  static constexpr int OFF_BAR = OFF_G + CL_ST * G_BYTES;
+  static constexpr int BYTES = OFF_BAR + 2 * CL_ST * 8 + 1024;
+};
+
+template <int NT>
+__global__ void __launch_bounds__(160) k_cols(const __grid_constant__ CUtensorMap tmP,
+                                              const __grid_constant__ CUtensorMap tmG, int M, int C, int R,
+                                              int rows_per_split, float* __restrict__ partial, int* status) {
+  using S = ColsSmem<NT>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const uint32_t full0 = base + S::OFF_BAR, empty0 = full0 + 8u * CL_ST;
+  __shared__ int abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c0 = blockIdx.x * 64;
+  const int split = blockIdx.y;
+  const int mb0 = split * rows_per_split;
+  const int mb1 = min(M, mb0 + rows_per_split);
+  const int nslab = mb1 > mb0 ? (mb1 - mb0 + 31) / 32 : 0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < CL_ST; ++s) {
+      mbar_init(full0 + 8u * s, 1);
+      mbar_init(empty0 + 8u * s, 4);
+    }
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == 4) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int it = 0; it < nslab; ++it) {
+        const int s = it % CL_ST;
+        if (!wait_bounded(empty0 + 8u * s, ((it / CL_ST) & 1) ^ 1, &abort_flag, status)) break;
+        mbar_arrive_expect_tx(full0 + 8u * s, S::P_BYTES + S::G_BYTES);
+        tma_load_2d(base + s * S::P_BYTES, &tmP, full0 + 8u * s, c0, mb0 + 32 * it);
+        tma_load_2d(base + S::OFF_G + s * S::G_BYTES, &tmG, full0 + 8u * s, 0, mb0 + 32 * it);
+        ++issued;
+      }
+      for (int it = (issued > CL_ST ? issued - CL_ST : 0); it < issued; ++it)
+        wait_drain(full0 + 8u * (it % CL_ST), (it / CL_ST) & 1);
+    }
+    return;
+  }
+
+  float acc[NT][4];
+#pragma unroll
+  for (int i = 0; i < NT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+  const int q = lane >> 3, l7 = lane & 7;
+  for (int it = 0; it < nslab; ++it) {
+    const int s = it % CL_ST;
+    if (!wait_bounded(full0 + 8u * s, (it / CL_ST) & 1, &abort_flag, status)) break;
+    const uint32_t pt = base + s * S::P_BYTES;
+    const uint32_t gt = base + S::OFF_G + s * S::G_BYTES;
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+      uint32_t a0, a1, a2, a3;  // P^T: (c 0-7, m 0-7), (c 8-15, m 0-7), (c 0-7, m 8-15), (c 8-15, m 8-15)
+      {
+        const int m = 16 * ks + (q >> 1) * 8 + l7, chunk = 2 * warp + (q & 1);
+        ldsm_x4_trans(pt + m * 128 + ((chunk ^ (m & 7)) << 4), a0, a1, a2, a3);
+      }
+#pragma unroll
+      for (int np = 0; np < NT / 2; ++np) {
+        uint32_t b0, b1, b2, b3;  // G: (m 0-7, tile 2np), (m 8-15, tile 2np), (m 0-7, tile 2np+1), (m 8-15, ...)
+        const int m = 16 * ks + (q & 1) * 8 + l7, j = (2 * np + (q >> 1)) * 8;
+        ldsm_x4_trans(narrow_addr<NT>(gt, m, j), b0, b1, b2, b3);
+        mma_bf16_16816(acc[2 * np], a0, a1, a2, a3, b0, b1);
+        mma_bf16_16816(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty0 + 8u * s);
+  }
+
+  const int g = lane >> 2, t = lane & 3;
   float* dst = partial + static_cast<int64_t>(split) * R * C;
 #pragma unroll
-  for (int ct = 0; ct < 2; ++ct) {
-    const int cbase = c0 + warp * 32 + ct * 16 + g;
+  for (int nt = 0; nt < NT; ++nt) {
+    const int j = nt * 8 + 2 * t;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int j = nt * 8 + 2 * t;
-      if (cbase < C) {
-        if (j < R) dst[static_cast<int64_t>(j) * C + cbase] = acc[ct][nt][0];
-        if (j + 1 < R) dst[static_cast<int64_t>(j + 1) * C + cbase] = acc[ct][nt][1];
-      }
-      if (cbase + 8 < C) {
-        if (j < R) dst[static_cast<int64_t>(j) * C + cbase + 8] = acc[ct][nt][2];
-        if (j + 1 < R) dst[static_cast<int64_t>(j + 1) * C + cbase + 8] = acc[ct][nt][3];
-      }
+    for (int h = 0; h < 2; ++h) {
+      const int c = c0 + 16 * warp + g + 8 * h;
+      if (c >= C) continue;
+      if (j < R) dst[static_cast<int64_t>(j) * C + c] = acc[nt][2 * h];
+      if (j + 1 < R) dst[static_cast<int64_t>(j + 1) * C + c] = acc[nt][2 * h + 1];
     }
   }
 }
@@ -236,25 +309,59 @@ __global__ void __launch_bounds__(64) k_coldot_reduce(const float* __restrict__ 
   }
 }
 
-__global__ void k_transpose_bf16(const uint16_t* __restrict__ src, int R, int C, uint16_t* __restrict__ dst) {
-  __shared__ uint16_t tile[32][33];
-  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int rr = r0 + i, cc = c0 + threadIdx.x;
-    if (rr < R && cc < C) tile[i][threadIdx.x] = src[static_cast<int64_t>(rr) * C + cc];
-  }
-  __syncthreads();
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int cc = c0 + i, rr = r0 + threadIdx.x;
-    if (rr < R && cc < C) dst[static_cast<int64_t>(cc) * R + rr] = tile[threadIdx.x][i];
+int nt_for(int R) { return R <= 16 ? 2 : R <= 32 ? 4 : 8; }
+
+int coldot_splits(int64_t M, int64_t C) {
+  const int64_t col_tiles = (C + 63) / 64;
+  int64_t s = (3 * 148 + col_tiles - 1) / col_tiles;  // ~3 CTAs per SM
+  s = std::max<int64_t>(1, std::min<int64_t>(s, (M + 255) / 256));
+  return static_cast<int>(s);
+}
+
+template <int NT, bool QT>
+cudaError_t rows_launch(const uint16_t* P, const uint16_t* Q, int64_t M, int64_t Kc, int R, float sa,
+                        uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st) {
+  using S = RowsSmem<NT>;
+  CUtensorMap tmP, tmQ;
+  const auto BF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  bool ok = make_map(&tmP, BF16, P, Kc, M, Kc * 2, 64, 16 * S::CW, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (QT)
+    ok = ok && make_map(&tmQ, BF16, Q, R, Kc, R * 2, NT * 8, 64, narrow_swizzle<NT>());
+  else
+    ok = ok && make_map(&tmQ, BF16, Q, Kc, R, Kc * 2, 64, NT * 8, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(k_rows<NT, QT>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>((M + 16 * S::CW - 1) / (16 * S::CW));
+  k_rows<NT, QT><<<grid, 32 * (S::CW + 1), S::BYTES, st>>>(tmP, tmQ, int(M), int(Kc), R, sa, out16a, sb, out16b,
+                                                           out32, device_status_ptr());
+  return cudaGetLastError();
+}
+
+template <bool QT>
+cudaError_t rows_dispatch(const uint16_t* P, const uint16_t* Q, int64_t M, int64_t Kc, int R, float sa,
+                          uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st) {
+  switch (nt_for(R)) {
+    case 2: return rows_launch<2, QT>(P, Q, M, Kc, R, sa, out16a, sb, out16b, out32, st);
+    case 4: return rows_launch<4, QT>(P, Q, M, Kc, R, sa, out16a, sb, out16b, out32, st);
+    default: return rows_launch<8, QT>(P, Q, M, Kc, R, sa, out16a, sb, out16b, out32, st);
   }
 }
 
-int coldot_splits(int64_t M, int64_t C) {
-  const int64_t col_tiles = (C + CD_COLS - 1) / CD_COLS;
-  int64_t s = (2 * 148 + col_tiles - 1) / col_tiles;  // ~2 CTAs per SM, long token slabs
-  s = std::max<int64_t>(1, std::min<int64_t>(s, (M + 255) / 256));
-  return static_cast<int>(s);
+template <int NT>
+cudaError_t cols_launch(const uint16_t* G, const uint16_t* P, int64_t M, int64_t C, int R, int splits,
+                        int rows_per_split, float* partial, cudaStream_t st) {
+  using S = ColsSmem<NT>;
+  CUtensorMap tmP, tmG;
+  const auto BF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  bool ok = make_map(&tmP, BF16, P, C, M, C * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok = ok && make_map(&tmG, BF16, G, R, M, R * 2, NT * 8, 32, narrow_swizzle<NT>());
+  if (!ok) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(k_cols<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(static_cast<unsigned>((C + 63) / 64), static_cast<unsigned>(splits));
+  k_cols<NT><<<grid, 160, S::BYTES, st>>>(tmP, tmG, int(M), int(C), R, rows_per_split, partial, device_status_ptr());
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -262,21 +369,13 @@ int coldot_splits(int64_t M, int64_t C) {
 cudaError_t launch_rowdot(const uint16_t* P, const uint16_t* Q, int64_t M, int64_t Kc, int R, float sa,
                           uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st) {
   if (M == 0) return cudaSuccess;
-  const unsigned grid = static_cast<unsigned>((M + 15) / 16);
-  const int nt = (R + 7) / 8;
-#define QN_ROWDOT(NTV)                                                                            \
-  case NTV:                                                                                       \
-    k_rowdot<NTV, (NTV <= 2 ? 4 : 2)><<<grid, 256, 0, st>>>(P, Q, static_cast<int>(M),             \
-                                                           static_cast<int>(Kc), R, sa, out16a,   \
-                                                           sb, out16b, out32);                    \
-    break;
-  switch (nt) {
-    QN_ROWDOT(1) QN_ROWDOT(2) QN_ROWDOT(3) QN_ROWDOT(4) QN_ROWDOT(5) QN_ROWDOT(6) QN_ROWDOT(7) QN_ROWDOT(8)
-    default:
-      return cudaErrorInvalidValue;
-  }
-#undef QN_ROWDOT
-  return cudaGetLastError();
+  return rows_dispatch<false>(P, Q, M, Kc, R, sa, out16a, sb, out16b, out32, st);
+}
+
+cudaError_t launch_rowdot_qt(const uint16_t* P, const uint16_t* Qt, int64_t M, int64_t Kc, int R, float sa,
+                             uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  return rows_dispatch<true>(P, Qt, M, Kc, R, sa, out16a, sb, out16b, out32, st);
 }
 
 size_t coldot_partial_floats(int64_t M, int64_t C, int R) {
@@ -286,35 +385,22 @@ size_t coldot_partial_floats(int64_t M, int64_t C, int R) {
 cudaError_t launch_coldot(const uint16_t* G, const uint16_t* P, int64_t M, int64_t C, int R, float scale,
                           int transpose, float* partial, uint16_t* out, cudaStream_t st) {
   const int splits = coldot_splits(M, C);
-  const int rows_per_split = static_cast<int>((M + splits - 1) / splits);
-  const dim3 grid(static_cast<unsigned>((C + CD_COLS - 1) / CD_COLS), static_cast<unsigned>(splits));
+  // token ranges are whole 32-token slabs, so a slab never straddles two splits
+  const int rows_per_split = static_cast<int>(((M + splits - 1) / splits + 31) / 32 * 32);
+  cudaError_t e = cudaSuccess;
   if (M > 0) {
-    const int nt = (R + 7) / 8;
-    if (nt <= 2)
-      k_coldot_mma<2><<<grid, 128, 0, st>>>(G, P, int(M), int(C), R, rows_per_split, partial);
-    else if (nt <= 4)
-      k_coldot_mma<4><<<grid, 128, 0, st>>>(G, P, int(M), int(C), R, rows_per_split, partial);
-    else if (nt <= 6)
-      k_coldot_mma<6><<<grid, 128, 0, st>>>(G, P, int(M), int(C), R, rows_per_split, partial);
-    else if (nt <= 8)
-      k_coldot_mma<8><<<grid, 128, 0, st>>>(G, P, int(M), int(C), R, rows_per_split, partial);
-    else
-      return cudaErrorInvalidValue;
+    switch (nt_for(R)) {
+      case 2: e = cols_launch<2>(G, P, M, C, R, splits, rows_per_split, partial, st); break;
+      case 4: e = cols_launch<4>(G, P, M, C, R, splits, rows_per_split, partial, st); break;
+      default: e = cols_launch<8>(G, P, M, C, R, splits, rows_per_split, partial, st); break;
+    }
   } else {
-    cudaError_t e = cudaMemsetAsync(partial, 0, sizeof(float) * R * C, st);
-    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(partial, 0, sizeof(float) * R * C, st);
   }
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int sp = M > 0 ? splits : 1;
   const dim3 rgrid(static_cast<unsigned>((C + 63) / 64), static_cast<unsigned>(R / 8));
   k_coldot_reduce<<<rgrid, 64, 0, st>>>(partial, sp, R, int(C), scale, transpose, out);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_transpose_bf16(const uint16_t* src, int64_t R, int64_t C, uint16_t* dst, cudaStream_t st) {
-  const dim3 grid(static_cast<unsigned>((C + 31) / 32), static_cast<unsigned>((R + 31) / 32));
-  k_transpose_bf16<<<grid, dim3(32, 8), 0, st>>>(src, int(R), int(C), dst);
   return cudaGetLastError();
 }
 

@@ -81,7 +81,6 @@ FwdWorkspace fwd_layout(void* ws, int64_t M, int r) {
 
 struct BwdWorkspace {
   uint16_t* dH16;   // bf16(scale * dY B) [M, r]
-  uint16_t* Bt;     // lora_B transposed [r, N]
   uint16_t* H16;    // bf16(X A^T) [M, r] when recomputed
   float* partial;   // split partial sums of the column reductions
   size_t bytes;
@@ -96,7 +95,6 @@ BwdWorkspace bwd_layout(void* ws, int64_t M, int64_t N, int64_t K, int r) {
     return q;
   };
   w.dH16 = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(M) * r * 2));
-  w.Bt = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(N) * r * 2));
   w.H16 = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(M) * r * 2));
   const size_t pf = std::max(coldot_partial_floats(M, K, r), coldot_partial_floats(M, N, r));
   w.partial = reinterpret_cast<float*>(take(std::max<size_t>(pf, static_cast<size_t>(r) * std::max(N, K)) * 4));
@@ -274,9 +272,8 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* absmax_q, const float*
     if (e == cudaSuccess) e = cudaMemsetAsync(dB, 0, static_cast<size_t>(N) * r * 2, s);
     return cuda_status(e);
   }
-  // dH = scale * dY B  (B^T staged so the contraction dim is contiguous)
-  e = launch_transpose_bf16(B, N, r, w.Bt, s);
-  if (e == cudaSuccess) e = launch_rowdot(dY, w.Bt, M, N, r, scale, w.dH16, scale, nullptr, nullptr, s);
+  // dH = scale * dY B  (B [N, r] read in place: its rows are the contraction)
+  e = launch_rowdot_qt(dY, B, M, N, r, scale, w.dH16, scale, nullptr, nullptr, s);
   const uint16_t* Huse = H;
   if (e == cudaSuccess && !H) {
     e = launch_rowdot(X, A, M, K, r, 1.0f, w.H16, 1.0f, nullptr, nullptr, s);

@@ -9,6 +9,12 @@
 
 namespace qn {
 
+// 2D row-major TMA tensor map: `inner` elements per row, `outer` rows, row
+// pitch `pitch_bytes`, box {box_inner, box_outer}; out-of-range elements read
+// as zero.  Returns false if the driver rejects the description.
+bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* ptr, uint64_t inner, uint64_t outer,
+              uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz);
+
 // Host-side NF4 table (computed once by codebook.cu).
 struct HostCodebook {
   Nf4Levels levels;
@@ -60,8 +66,9 @@ cudaError_t launch_rowdot(const uint16_t* P, const uint16_t* Q, int64_t M, int64
 size_t coldot_partial_floats(int64_t M, int64_t C, int R);
 cudaError_t launch_coldot(const uint16_t* G, const uint16_t* P, int64_t M, int64_t C, int R, float scale,
                           int transpose, float* partial, uint16_t* out, cudaStream_t st);
-// dst[c, r] = src[r, c] for a bf16 [R, C] matrix.
-cudaError_t launch_transpose_bf16(const uint16_t* src, int64_t R, int64_t C, uint16_t* dst, cudaStream_t st);
+// The same with Q given transposed, Qt bf16 [Kc, R] (lora_B read in place).
+cudaError_t launch_rowdot_qt(const uint16_t* P, const uint16_t* Qt, int64_t M, int64_t Kc, int R, float sa,
+                             uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st);
 
 // ----- decode GEMV (M <= 16): Y = X deq(W)^T + Hs B^T, Hs = bf16(s X A^T)
 cudaError_t launch_gemv(const uint16_t* X, int64_t M, const uint8_t* codes, const uint8_t* absmax_q,
