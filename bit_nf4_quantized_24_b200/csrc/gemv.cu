@@ -2,23 +2,27 @@
 // Bound by streaming the NF4 weight once (katajob, "NF4: 4-bit NormalFloat":
 // the weight is read in 4-bit and expanded per block only inside the product).
 //
-// Expansion.  A code byte holds two weights; a 256-entry table maps it to the
-// two levels as a bf16 pair.  The table lives in shared memory replicated
-// once per lane (entry e of lane l at T + 256 e + 4 l), so every lookup of a
-// warp is conflict-free, and T is 64 KB aligned, so one prmt assembles the
-// address from the code byte and the lane's base: 1 prmt + 1 ld.shared per two
-// weights, with no per-block table to build.  The per-block scale is applied
-// afterwards: the four m16n8k16 steps of one 64-weight block accumulate into a
-// fresh fragment, which is then added with the block's scale.  For this each
-// MMA step must stay inside one block: lane t contributes k = 16t + 4s + 0..3
-// at step s (its 8 code bytes 8t .. 8t+7 of the block), and the activation
-// fragments are read in the same permuted order.
+// Data movement.  One persistent CTA per SM owns a contiguous run of 16-row
+// weight tiles.  A producer thread streams each tile's code bytes through a
+// ring in shared memory with 2D TMA copies (16 rows x 128 bytes per box,
+// 128-byte swizzle), one stage = 16 rows x 32 blocks of 64 weights.
 //
-// Schedule.  One persistent CTA per SM, 8 warps.  A task is 32 weight rows:
-// the 8 warps split the task's blocks along K, each warp handles the 32 rows
-// as four n8 tiles with its code blocks (and scales) loaded G_DEPTH blocks
-// ahead into a register ring, and the partial sums meet in shared memory
-// (fixed order, so the result is deterministic).
+// Expansion.  A code byte holds two weights; a 256-entry table maps it to the
+// two levels as a bf16 pair.  The table is replicated once per lane (entry e
+// of lane l at T + 256 e + 4 l, T aligned to 64 KB), so a warp's lookups never
+// share a bank and one prmt builds the lookup address from the code byte and
+// the lane's base.  The weights are the A operand of m16n8k16 (16 rows x 16
+// k per step, tokens in n), and the four steps of one 64-weight block
+// accumulate into a fresh fragment that is then added with the block's scale
+// absmax(q) * dq_scale.  Each step stays inside one block: lane t holds the
+// block's code bytes 8t .. 8t+7 and covers k = 16t + 4s + 0..3 at step s; the
+// activation fragments are read in the same order.
+//
+// Work split.  16 consumer warps take two blocks of every stage each (a
+// K-split), keep per-row partial sums in registers across the tile, and hand
+// them to an epilogue warp through a double-buffered shared array.  The
+// epilogue warp adds the 16 partials in a fixed order (deterministic), adds
+// the LoRA term with one more MMA over r, and stores bf16 Y.
 #include <algorithm>
 
 #include "internal.h"
@@ -27,13 +31,25 @@ namespace qn {
 
 namespace {
 
-constexpr int G_WARPS = 8;
-constexpr int G_DEPTH = 6;                        // code blocks in flight per warp
-constexpr int G_THREADS = G_WARPS * 32;
-constexpr int G_ROWS = 32;                        // weight rows per task (4 n8 tiles)
-constexpr int G_RED_BYTES = G_WARPS * 4 * 4 * 32 * 4;  // partial sums of one task
-constexpr int G_TABLE_BYTES = 256 * 256;          // 256 entries x 256 B (128 B used)
-constexpr int G_SMEM = G_TABLE_BYTES + 65536 + G_RED_BYTES;  // room to align the table to 64 KB
+constexpr int G_CW = 16;                            // consumer warps
+constexpr int G_THREADS = (G_CW + 2) * 32;          // + TMA producer warp + epilogue warp
+constexpr int G_ROWS = 16;                          // weight rows per tile
+constexpr int G_SBLK = 2 * G_CW;                    // 64-weight blocks per stage
+constexpr int G_BOX = 128 * G_ROWS;                 // one TMA box: 16 rows x 128 code bytes
+constexpr int G_STAGE = (G_SBLK / 4) * G_BOX;       // 16 KB of codes per stage
+constexpr int G_TABLE = 65536;                      // 256 entries x 256 B (128 B used)
+
+template <int NTILE>
+struct GemvSmem {  // offsets from the 64 KB-aligned table
+  static constexpr int NS = NTILE == 1 ? 5 : 4;                       // ring stages
+  static constexpr int RED_FLOATS = G_CW * NTILE * 4 * 32;             // one partial-sum buffer
+  static constexpr int OFF_RING = G_TABLE;
+  static constexpr int OFF_RED = OFF_RING + NS * G_STAGE;
+  static constexpr int OFF_BAR = OFF_RED + 2 * RED_FLOATS * 4;
+  static constexpr int USED = OFF_BAR + 8 * (2 * NS + 4);
+  static constexpr int BYTES = USED + 65536;                          // room to align the table
+};
+static_assert(GemvSmem<1>::BYTES <= 232448 && GemvSmem<2>::BYTES <= 232448, "shared memory");
 
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
@@ -50,9 +66,9 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   return v;
 }
 
-__device__ __forceinline__ uint2 ldg_nc_v2(const void* p) {
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
   uint2 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
   return v;
 }
 
@@ -63,25 +79,100 @@ __device__ __forceinline__ uint32_t lut_pair(uint32_t word, uint32_t lane_base) 
   return lds32(prmt(word, lane_base, 0x7604u | (BYTE << 4)));
 }
 
-struct RowScale {
-  float ap0, ap1;  // block scales of W rows 2t and 2t+1 of an n8 tile
+// What one consumer lane preloads for one block: its activation fragment
+// (X[8nt + g][64b + 16t .. +15]) and the two row scales (rows g, g + 8).
+template <int NTILE>
+struct BlockIn {
+  uint32_t x[NTILE][8];
+  uint32_t q[2];
+  float d[2];
 };
 
-__global__ void __launch_bounds__(G_THREADS, 1) k_gemv(const uint16_t* __restrict__ X, int M,
-                                                        const uint8_t* __restrict__ codes,
-                                                        const uint8_t* __restrict__ absmax_q,
-                                                        const float* __restrict__ dq_scale, int N, int K,
-                                                        const uint16_t* __restrict__ Hs,
-                                                        const uint16_t* __restrict__ Bl, int r, Nf4Levels lv,
-                                                        uint16_t* __restrict__ Y, int* status) {
+template <int NTILE>
+__device__ __forceinline__ void load_block(BlockIn<NTILE>& in, const uint16_t* __restrict__ X, int M, int K,
+                                           const uint8_t* __restrict__ absmax_q,
+                                           const float* __restrict__ dq_scale, int N, int KB, int n0, int b,
+                                           int g, int t) {
+  const bool bok = b < KB;
+#pragma unroll
+  for (int nt = 0; nt < NTILE; ++nt) {
+    const int m = 8 * nt + g;
+    uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
+    if (bok && m < M) {
+      const uint4* p = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(m) * K + 64 * b + 16 * t);
+      lo = __ldg(p);
+      hi = __ldg(p + 1);
+    }
+    in.x[nt][0] = lo.x; in.x[nt][1] = lo.y; in.x[nt][2] = lo.z; in.x[nt][3] = lo.w;
+    in.x[nt][4] = hi.x; in.x[nt][5] = hi.y; in.x[nt][6] = hi.z; in.x[nt][7] = hi.w;
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int row = n0 + g + 8 * h;
+    in.q[h] = 0u;
+    in.d[h] = 0.f;
+    if (bok && row < N) {
+      const int64_t blk = static_cast<int64_t>(row) * KB + b;
+      in.q[h] = __ldg(absmax_q + blk);
+      in.d[h] = __ldg(dq_scale + (blk >> 8));
+    }
+  }
+}
+
+// One 64-weight block of a 16-row tile: codes of rows g and g + 8 from the
+// staged box, four MMA steps, then the scaled add into acc.
+template <int NTILE>
+__device__ __forceinline__ void block_mma(float (&acc)[NTILE][4], const BlockIn<NTILE>& in, uint32_t code_addr,
+                                          uint32_t lane_base) {
+  const uint2 cg = lds64(code_addr), ch = lds64(code_addr + 1024u);  // row g + 8 is 8 box rows further
+  float p[NTILE][4];
+#pragma unroll
+  for (int nt = 0; nt < NTILE; ++nt) p[nt][0] = p[nt][1] = p[nt][2] = p[nt][3] = 0.f;
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    const uint32_t wg = s < 2 ? cg.x : cg.y, wh = s < 2 ? ch.x : ch.y;
+    uint32_t a0, a1, a2, a3;
+    if ((s & 1) == 0) {
+      a0 = lut_pair<0>(wg, lane_base); a2 = lut_pair<1>(wg, lane_base);
+      a1 = lut_pair<0>(wh, lane_base); a3 = lut_pair<1>(wh, lane_base);
+    } else {
+      a0 = lut_pair<2>(wg, lane_base); a2 = lut_pair<3>(wg, lane_base);
+      a1 = lut_pair<2>(wh, lane_base); a3 = lut_pair<3>(wh, lane_base);
+    }
+#pragma unroll
+    for (int nt = 0; nt < NTILE; ++nt) mma16816(p[nt], a0, a1, a2, a3, in.x[nt][2 * s], in.x[nt][2 * s + 1]);
+  }
+  const float sg = __fmul_rn(static_cast<float>(in.q[0]), in.d[0]);
+  const float sh = __fmul_rn(static_cast<float>(in.q[1]), in.d[1]);
+#pragma unroll
+  for (int nt = 0; nt < NTILE; ++nt) {
+    acc[nt][0] = fmaf(sg, p[nt][0], acc[nt][0]);
+    acc[nt][1] = fmaf(sg, p[nt][1], acc[nt][1]);
+    acc[nt][2] = fmaf(sh, p[nt][2], acc[nt][2]);
+    acc[nt][3] = fmaf(sh, p[nt][3], acc[nt][3]);
+  }
+}
+
+template <int NTILE>
+__global__ void __launch_bounds__(G_THREADS, 1)
+    k_gemv(const __grid_constant__ CUtensorMap tm_codes, const uint16_t* __restrict__ X, int M,
+           const uint8_t* __restrict__ absmax_q, const float* __restrict__ dq_scale, int N, int K,
+           const uint16_t* __restrict__ Hs, const uint16_t* __restrict__ Bl, int r, Nf4Levels lv,
+           uint16_t* __restrict__ Y, int* status) {
+  using S = GemvSmem<NTILE>;
+  constexpr int NS = S::NS;
   extern __shared__ uint8_t smem_raw[];
+  __shared__ int abort_flag;
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t table = (raw + 65535u) & ~65535u;
-  if (table + G_TABLE_BYTES + G_RED_BYTES > raw + G_SMEM) {  // cannot happen with G_SMEM; never index past it
+  if (table + S::USED > raw + S::BYTES) {  // cannot happen with S::BYTES; never index past it
     if (threadIdx.x == 0) atomicExch(status, kDevTimeout);
     return;
   }
-  float* red = reinterpret_cast<float*>(smem_raw + (table - raw) + G_TABLE_BYTES);
+  const uint32_t ring = table + S::OFF_RING;
+  float* red = reinterpret_cast<float*>(smem_raw + (table - raw) + S::OFF_RED);
+  const uint32_t full0 = table + S::OFF_BAR, empty0 = full0 + 8u * NS;
+  const uint32_t rfull0 = empty0 + 8u * NS, rempty0 = rfull0 + 16u;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
 
@@ -91,126 +182,175 @@ __global__ void __launch_bounds__(G_THREADS, 1) k_gemv(const uint16_t* __restric
     const uint32_t v = bf16x2_bits(lv.v[e & 15], lv.v[e >> 4]);
     asm volatile("st.shared.b32 [%0], %1;" ::"r"(table + e * 256 + l * 4), "r"(v) : "memory");
   }
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(full0 + 8u * s, 1);
+      mbar_init(empty0 + 8u * s, G_CW);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(rfull0 + 8u * b, G_CW);
+      mbar_init(rempty0 + 8u * b, 1);
+    }
+    abort_flag = 0;
+    fence_mbar_init();
+  }
   __syncthreads();
-  const uint32_t lane_base = table + lane * 4;
 
   const int KB = K / 64;
-  const int b_lo = (warp * KB) / G_WARPS, b_hi = ((warp + 1) * KB) / G_WARPS;  // this warp's blocks
-  const bool lo_ok = g < M, hi_ok = g + 8 < M;
-  const int ntasks = (N + G_ROWS - 1) / G_ROWS;
+  const int spt = (KB + G_SBLK - 1) / G_SBLK;  // stages per tile
+  const int ntiles = (N + G_ROWS - 1) / G_ROWS;
+  const int t0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * ntiles / gridDim.x);
+  const int t1 = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * ntiles / gridDim.x);
+  const int nit = (t1 - t0) * spt;
 
-  for (int task = blockIdx.x; task < ntasks; task += gridDim.x) {
-    const int n0 = task * G_ROWS;
-    float acc[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+  if (warp == G_CW) {  // producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_codes);
+      int issued = 0, s = 0, tile = t0;
+      for (int it = 0; it < nit; ++it) {
+        const int slot = it % NS;
+        if (!wait_bounded(empty0 + 8u * slot, ((it / NS) & 1) ^ 1, &abort_flag, status)) break;
+        const int b0 = s * G_SBLK;
+        const int nbox = min(G_SBLK / 4, (KB - b0 + 3) / 4);  // boxes that start inside the row
+        mbar_arrive_expect_tx(full0 + 8u * slot, nbox * G_BOX);
+        for (int bx = 0; bx < nbox; ++bx)
+          tma_load_2d(ring + slot * G_STAGE + bx * G_BOX, &tm_codes, full0 + 8u * slot, (b0 + 4 * bx) * 32,
+                      tile * G_ROWS);
+        ++issued;
+        if (++s == spt) { s = 0; ++tile; }
+      }
+      for (int it = (issued > NS ? issued - NS : 0); it < issued; ++it)  // all copies land before exit
+        wait_drain(full0 + 8u * (it % NS), (it / NS) & 1);
+    }
+    return;
+  }
 
-    // per tile: this lane's code row and the two rows whose scales it applies
-    const int crow[4] = {n0 + g, n0 + 8 + g, n0 + 16 + g, n0 + 24 + g};
-    auto load_codes = [&](int b, uint2 (&cw)[4]) {
+  if (warp == G_CW + 1) {  // epilogue: sum the K-split partials, add the LoRA term, store
+    for (int ti = 0; ti < t1 - t0; ++ti) {
+      const int n0 = (t0 + ti) * G_ROWS;
+      const int buf = ti & 1;
+      // LoRA operands first; their latency hides behind the wait
+      auto ld2 = [&](const uint16_t* p, int row, int rows, int j) -> uint32_t {
+        if (row >= rows || j >= r) return 0u;
+        return __ldg(reinterpret_cast<const uint32_t*>(p + static_cast<int64_t>(row) * r + j));
+      };
+      uint32_t la[4][4], lb[4][NTILE][2];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        cw[i] = (crow[i] < N && b < b_hi)
-                    ? ldg_nc_v2(codes + (static_cast<int64_t>(crow[i]) * KB + b) * 32 + 8 * t)
-                    : make_uint2(0u, 0u);
-    };
-    auto load_scales = [&](int b, RowScale (&sc)[4]) {
+      for (int k = 0; k < 4; ++k) {
+        const int j0 = 16 * k;
+        la[k][0] = ld2(Bl, n0 + g, N, j0 + 2 * t);
+        la[k][1] = ld2(Bl, n0 + g + 8, N, j0 + 2 * t);
+        la[k][2] = ld2(Bl, n0 + g, N, j0 + 2 * t + 8);
+        la[k][3] = ld2(Bl, n0 + g + 8, N, j0 + 2 * t + 8);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r0 = n0 + 8 * i + 2 * t;
-        float a[2];
+        for (int nt = 0; nt < NTILE; ++nt) {
+          lb[k][nt][0] = ld2(Hs, 8 * nt + g, M, j0 + 2 * t);
+          lb[k][nt][1] = ld2(Hs, 8 * nt + g, M, j0 + 2 * t + 8);
+        }
+      }
+      if (!wait_bounded(rfull0 + 8u * buf, (ti >> 1) & 1, &abort_flag, status)) break;
+      float v[NTILE][4];
+      const float* rb = red + buf * S::RED_FLOATS;
+#pragma unroll
+      for (int nt = 0; nt < NTILE; ++nt)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float sum = 0.f;
+#pragma unroll 4
+          for (int w = 0; w < G_CW; ++w) sum += rb[((w * NTILE + nt) * 4 + c) * 32 + lane];
+          v[nt][c] = sum;
+        }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(rempty0 + 8u * buf);  // partial sums read: the buffer is free
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (16 * k >= r) break;
+#pragma unroll
+        for (int nt = 0; nt < NTILE; ++nt)
+          mma16816(v[nt], la[k][0], la[k][1], la[k][2], la[k][3], lb[k][nt][0], lb[k][nt][1]);
+      }
+#pragma unroll
+      for (int nt = 0; nt < NTILE; ++nt) {
+        const int m = 8 * nt + 2 * t;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          a[h] = 0.0f;
-          if (r0 + h < N && b < b_hi) {
-            const int64_t blk = static_cast<int64_t>(r0 + h) * KB + b;
-            a[h] = __fmul_rn(static_cast<float>(__ldg(absmax_q + blk)), __ldg(dq_scale + (blk >> 8)));
-          }
+          const int n = n0 + g + 8 * h;
+          if (n >= N) continue;
+          if (m < M) Y[static_cast<int64_t>(m) * N + n] = static_cast<uint16_t>(bf16x2_bits(v[nt][2 * h], 0.f));
+          if (m + 1 < M)
+            Y[static_cast<int64_t>(m + 1) * N + n] = static_cast<uint16_t>(bf16x2_bits(v[nt][2 * h + 1], 0.f));
         }
-        sc[i].ap0 = a[0];
-        sc[i].ap1 = a[1];
-      }
-    };
-
-    // register ring of G_DEPTH blocks: slot j holds block b_lo + j (mod G_DEPTH)
-    uint2 cw[G_DEPTH][4];
-    RowScale sc[G_DEPTH][4];
-#pragma unroll
-    for (int j = 0; j < G_DEPTH; ++j) {
-      load_codes(b_lo + j, cw[j]);
-      load_scales(b_lo + j, sc[j]);
-    }
-    for (int b0 = b_lo; b0 < b_hi; b0 += G_DEPTH) {
-#pragma unroll
-      for (int j = 0; j < G_DEPTH; ++j) {
-        const int b = b0 + j;
-        if (b >= b_hi) break;
-        // activation fragments of this block: X[row][64b + 16t .. +15]
-        uint4 x0 = make_uint4(0, 0, 0, 0), x1 = x0, y0 = x0, y1 = x0;
-        if (lo_ok) {
-          const uint4* p = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(g) * K + 64 * b + 16 * t);
-          x0 = __ldg(p);
-          x1 = __ldg(p + 1);
-        }
-        if (hi_ok) {
-          const uint4* p = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(g + 8) * K + 64 * b + 16 * t);
-          y0 = __ldg(p);
-          y1 = __ldg(p + 1);
-        }
-        const uint32_t xg[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-        const uint32_t xh[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint2 c = cw[j][i];
-          float tmp[4] = {0.f, 0.f, 0.f, 0.f};
-          mma16816(tmp, xg[0], xh[0], xg[1], xh[1], lut_pair<0>(c.x, lane_base), lut_pair<1>(c.x, lane_base));
-          mma16816(tmp, xg[2], xh[2], xg[3], xh[3], lut_pair<2>(c.x, lane_base), lut_pair<3>(c.x, lane_base));
-          mma16816(tmp, xg[4], xh[4], xg[5], xh[5], lut_pair<0>(c.y, lane_base), lut_pair<1>(c.y, lane_base));
-          mma16816(tmp, xg[6], xh[6], xg[7], xh[7], lut_pair<2>(c.y, lane_base), lut_pair<3>(c.y, lane_base));
-          acc[i][0] = fmaf(sc[j][i].ap0, tmp[0], acc[i][0]);
-          acc[i][1] = fmaf(sc[j][i].ap1, tmp[1], acc[i][1]);
-          acc[i][2] = fmaf(sc[j][i].ap0, tmp[2], acc[i][2]);
-          acc[i][3] = fmaf(sc[j][i].ap1, tmp[3], acc[i][3]);
-        }
-        load_codes(b + G_DEPTH, cw[j]);  // refill the slot G_DEPTH blocks ahead
-        load_scales(b + G_DEPTH, sc[j]);
       }
     }
-
-    // K-split partial sums meet in shared memory
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) red[((warp * 4 + i) * 4 + c) * 32 + lane] = acc[i][c];
-    __syncthreads();
-    if (warp < 4) {  // warp i finishes tile i: sum, LoRA term, store
-      const int i = warp;
-      float v[4];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float s = 0.f;
-        for (int w = 0; w < G_WARPS; ++w) s += red[((w * 4 + i) * 4 + c) * 32 + lane];
-        v[c] = s;
-      }
-      // + Hs[m, :] . B[n, :] in k16 steps over r (standard fragment order)
-      for (int j0 = 0; j0 < r; j0 += 16) {
-        auto ld2 = [&](const uint16_t* base_p, int row, int rows, int j) -> uint32_t {
-          if (row >= rows || j >= r) return 0u;
-          return __ldg(reinterpret_cast<const uint32_t*>(base_p + static_cast<int64_t>(row) * r + j));
-        };
-        const int n = n0 + 8 * i + g;
-        mma16816(v, ld2(Hs, g, M, j0 + 2 * t), ld2(Hs, g + 8, M, j0 + 2 * t), ld2(Hs, g, M, j0 + 2 * t + 8),
-                 ld2(Hs, g + 8, M, j0 + 2 * t + 8), ld2(Bl, n, N, j0 + 2 * t), ld2(Bl, n, N, j0 + 2 * t + 8));
-      }
-      const int n = n0 + 8 * i + 2 * t;
-      if (n < N) {
-        if (g < M) *reinterpret_cast<uint32_t*>(Y + static_cast<int64_t>(g) * N + n) = bf16x2_bits(v[0], v[1]);
-        if (g + 8 < M)
-          *reinterpret_cast<uint32_t*>(Y + static_cast<int64_t>(g + 8) * N + n) = bf16x2_bits(v[2], v[3]);
-      }
-    }
-    __syncthreads();  // red is reused by the next task
+    return;
   }
+
+  // consumers: warp w takes blocks 2w and 2w + 1 of every stage
+  const uint32_t lane_base = table + lane * 4;
+  uint32_t coff[2];  // byte offset of this lane's 8 code bytes (row g) inside a stage
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const int bb = 2 * warp + q;
+    const int chunk = 2 * (bb & 3) + (t >> 1);
+    coff[q] = (bb >> 2) * G_BOX + g * 128 + ((chunk ^ g) << 4) + ((t & 1) << 3);
+  }
+  float acc[NTILE][4];
+#pragma unroll
+  for (int nt = 0; nt < NTILE; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+
+  BlockIn<NTILE> in[2];
+  int s = 0, ti = 0;
+#pragma unroll
+  for (int q = 0; q < 2; ++q)
+    load_block(in[q], X, M, K, absmax_q, dq_scale, N, KB, t0 * G_ROWS, 2 * warp + q, g, t);
+  for (int it = 0; it < nit; ++it) {
+    const int slot = it % NS;
+    if (!wait_bounded(full0 + 8u * slot, (it / NS) & 1, &abort_flag, status)) break;
+    // the block this slot refills with: same position, next stage
+    const int ns = s + 1 == spt ? 0 : s + 1;
+    const int nn0 = (t0 + ti + (s + 1 == spt ? 1 : 0)) * G_ROWS;
+    const bool more = it + 1 < nit;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      if (s * G_SBLK + 2 * warp + q < KB) block_mma(acc, in[q], ring + slot * G_STAGE + coff[q], lane_base);
+      if (more) load_block(in[q], X, M, K, absmax_q, dq_scale, N, KB, nn0, ns * G_SBLK + 2 * warp + q, g, t);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty0 + 8u * slot);
+    if (++s == spt) {  // tile done: hand the partial sums to the epilogue warp
+      const int buf = ti & 1;
+      if (!wait_bounded(rempty0 + 8u * buf, ((ti >> 1) & 1) ^ 1, &abort_flag, status)) break;
+      float* rb = red + buf * S::RED_FLOATS;
+#pragma unroll
+      for (int nt = 0; nt < NTILE; ++nt)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          rb[((warp * NTILE + nt) * 4 + c) * 32 + lane] = acc[nt][c];
+          acc[nt][c] = 0.f;
+        }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(rfull0 + 8u * buf);
+      s = 0;
+      ++ti;
+    }
+  }
+}
+
+template <int NTILE>
+cudaError_t gemv_launch(const CUtensorMap& tm, const uint16_t* X, int64_t M, const uint8_t* absmax_q,
+                        const float* dq_scale, int64_t N, int64_t K, const uint16_t* Hs, const uint16_t* B, int r,
+                        uint16_t* Y, cudaStream_t st) {
+  using S = GemvSmem<NTILE>;
+  cudaError_t e = cudaFuncSetAttribute(k_gemv<NTILE>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t ntiles = (N + G_ROWS - 1) / G_ROWS;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ntiles, sms));
+  k_gemv<NTILE><<<grid, G_THREADS, S::BYTES, st>>>(tm, X, int(M), absmax_q, dq_scale, int(N), int(K), Hs, B, r,
+                                                   host_codebook().levels, Y, device_status_ptr());
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -219,16 +359,13 @@ cudaError_t launch_gemv(const uint16_t* X, int64_t M, const uint8_t* codes, cons
                         const float* dq_scale, int64_t N, int64_t K, const uint16_t* Hs, const uint16_t* B, int r,
                         uint16_t* Y, cudaStream_t st) {
   if (M == 0 || N == 0) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(k_gemv, cudaFuncAttributeMaxDynamicSharedMemorySize, G_SMEM);
-  if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t ntasks = (N + G_ROWS - 1) / G_ROWS;
-  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ntasks, sms));
-  k_gemv<<<grid, G_THREADS, G_SMEM, st>>>(X, int(M), codes, absmax_q, dq_scale, int(N), int(K), Hs, B, r,
-                                           host_codebook().levels, Y, device_status_ptr());
-  return cudaGetLastError();
+  if (M > 16 || r > 64) return cudaErrorInvalidValue;
+  CUtensorMap tm;
+  if (!make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, 128, G_ROWS,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  return M <= 8 ? gemv_launch<1>(tm, X, M, absmax_q, dq_scale, N, K, Hs, B, r, Y, st)
+                : gemv_launch<2>(tm, X, M, absmax_q, dq_scale, N, K, Hs, B, r, Y, st);
 }
 
 }  // namespace qn
