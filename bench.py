@@ -5,8 +5,9 @@ One step = forward + backward of the Llama-7B-shaped q_proj workload
 (X [4096 tokens, 4096] bf16, W 4096x4096 in NF4 with double quantization,
 LoRA r = 16, alpha = 32): qlora_linear_fwd then qlora_linear_bwd through the
 C ABI, all inputs resident in HBM.  The metric is algorithmic TFLOP/s
-(4MNK + 6Mr(K+N) per step; no gradient for W).  L2 is flushed (a 256 MB write)
-between timed steps; each step is timed with CUDA events on the launching
+(4MNK + 6Mr(K+N) per step; no gradient for W).  L2 is flushed between timed
+steps (a 256 MB write, then a 256 MB read so that no dirty lines are left to
+be written back inside the timed region); each step is timed with CUDA events on the launching
 stream and the per-step times are summed.
 
 Also reported: the fused dequant-GEMM kernel against the tensor-core roofline
@@ -39,6 +40,24 @@ sys.path.insert(0, ROOT)
 
 METRIC = "QLoRA linear fwd+bwd TFLOP/s and NF4 weight-stream GB/s on 1 B200; % roofline"
 WORKLOAD = "qproj_7b"
+
+
+class L2Flush:
+    """Evicts L2 (126 MB on B200) between timed steps: writes one 256 MB
+    buffer, then reads another, so the timed step starts with a cold L2 that
+    holds no dirty lines (a write-only flush leaves ~126 MB of dirty lines,
+    whose write-back would land inside the timed region)."""
+
+    def __init__(self, dev):
+        import torch
+        self.w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.r = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+        self.out = torch.empty((), dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        import torch
+        self.w.zero_()
+        torch.sum(self.r, 0, out=self.out)
 
 
 def peaks():
@@ -187,7 +206,7 @@ def run_ours(args, rank, world, local_rank):
     H = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
     wsf = torch.empty(qb.fwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
     wsb = torch.empty(qb.bwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     L = qb.lib()
     import ctypes
     f32 = ctypes.c_float
@@ -221,7 +240,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     with sampler, trace:
         for i in range(K_steps):
-            flush.zero_()
+            flush()
             ev[i][0].record()
             step()
             ev[i][1].record()
@@ -304,7 +323,7 @@ def run_ours(args, rank, world, local_rank):
                                f"NF4 block 64 + 8-bit double quant (group 256), LoRA r=16 alpha=32",
                    "M": M, "N": N, "K": K, "r": r, "global_batch_tokens": M * world,
                    "parallelism": f"dp{world} (adapter grads all-reduced)" if world > 1 else "single GPU",
-                   "l2": "flushed between timed steps (256 MB write)"},
+                   "l2": "flushed between timed steps (256 MB write, then 256 MB read: cold and clean)"},
         "roofline": roofline,
         "e2e": e2e,
         "gpu_launches": launches_per_step * K_steps,
@@ -335,7 +354,7 @@ def run_extras(qb, wl, dev, pk, flush):
         ts = []
         for _ in range(n):
             if flush_between:
-                flush.zero_()
+                flush()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
             fn()
@@ -357,9 +376,21 @@ def run_extras(qb, wl, dev, pk, flush):
         X = p["X"][:M].contiguous().to(dev)
         Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
         ws = torch.empty(qb.fwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
-        ms = timed(lambda: qb.qlora_linear_fwd(q, X, A, B, s, save_h=False, out=Y, workspace=ws))
+        # a decode loop issues the call from a CUDA graph: time the replay
+        call = lambda: qb.qlora_linear_fwd(q, X, A, B, s, save_h=False, out=Y, workspace=ws)
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            call()
+        torch.cuda.current_stream().wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            call()
+        ms = timed(graph.replay)
+        ms_eager = timed(call)
         total_bytes = weight_bytes + 2 * r * (K + N) + 2 * M * (K + N)
-        dec[f"M{M}"] = {"us": round(ms * 1e3, 2), "weight_stream_gbs": round(weight_bytes / ms / 1e6, 1),
+        dec[f"M{M}"] = {"us": round(ms * 1e3, 2), "us_eager_call": round(ms_eager * 1e3, 2),
+                        "weight_stream_gbs": round(weight_bytes / ms / 1e6, 1),
                         "total_gbs": round(total_bytes / ms / 1e6, 1),
                         "frac_hbm": round(total_bytes / ms / 1e6 / pk["hbm_gbs"], 4)}
     res["decode_70b_up"] = dec

@@ -51,6 +51,86 @@ constexpr CUtensorMapSwizzle narrow_swizzle() {
   return NT == 2 ? CU_TENSOR_MAP_SWIZZLE_32B : NT == 4 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
 }
 
+// ------------------------------------------------------------- rows, M <= 16
+//
+// The same product for at most 16 tokens (decode).  There is a single token
+// tile, so the contraction is split instead: RS_CTAS CTAs of one cluster x
+// RS_WARPS warps each take whole 64-wide k groups.  The warps of a CTA meet
+// in shared memory, the CTAs through distributed shared memory, where CTA 0
+// adds the cluster's partials in a fixed order and writes the outputs.  Each
+// CTA lets the next kernel of the stream launch at once (programmatic
+// dependent launch); that kernel waits for this grid to finish before it
+// reads the outputs.
+constexpr int RS_CTAS = 8, RS_WARPS = 8;
+
+__device__ __forceinline__ uint32_t ldg32(const uint16_t* p) {
+  return __ldg(reinterpret_cast<const uint32_t*>(p));
+}
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t cluster_addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+
+template <int NT>
+__global__ void __cluster_dims__(RS_CTAS, 1, 1) __launch_bounds__(RS_WARPS * 32)
+    k_rows_small(const uint16_t* __restrict__ P, const uint16_t* __restrict__ Q, int M, int Kc, int R, float sa,
+                 uint16_t* __restrict__ out16a, float sb, uint16_t* __restrict__ out16b,
+                 float* __restrict__ out32) {
+  __shared__ float wpart[RS_WARPS][16 * 64];
+  __shared__ float cpart[16 * 64];
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int rank = static_cast<int>(cluster_ctarank());
+  const int worker = rank * RS_WARPS + warp;
+  const int ngroups = Kc / 64;
+  const int gl = static_cast<int>(static_cast<int64_t>(worker) * ngroups / (RS_CTAS * RS_WARPS));
+  const int gh = static_cast<int>(static_cast<int64_t>(worker + 1) * ngroups / (RS_CTAS * RS_WARPS));
+  // token rows >= M and output columns >= R read clamped rows; those results are never stored
+  const uint16_t* p0 = P + static_cast<int64_t>(min(g, M - 1)) * Kc + 2 * t;
+  const uint16_t* p1 = P + static_cast<int64_t>(min(g + 8, M - 1)) * Kc + 2 * t;
+  const uint16_t* qr[NT];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) qr[nt] = Q + static_cast<int64_t>(min(8 * nt + g, R - 1)) * Kc + 2 * t;
+  float acc[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+  for (int grp = gl; grp < gh; ++grp) {
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const int k = grp * 64 + 16 * s;
+      const uint32_t a0 = ldg32(p0 + k), a1 = ldg32(p1 + k), a2 = ldg32(p0 + k + 8), a3 = ldg32(p1 + k + 8);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(acc[nt], a0, a1, a2, a3, ldg32(qr[nt] + k), ldg32(qr[nt] + k + 8));
+    }
+  }
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) wpart[warp][(g + 8 * (c >> 1)) * 64 + 8 * nt + 2 * t + (c & 1)] = acc[nt][c];
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < 16 * 64; idx += RS_WARPS * 32) {
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < RS_WARPS; ++w) v += wpart[w][idx];
+    cpart[idx] = v;
+  }
+  cluster_sync_all();  // every CTA's partial is in its shared memory
+  if (rank == 0) {
+    const uint32_t base = smem_u32(cpart);
+    for (int idx = threadIdx.x; idx < M * R; idx += RS_WARPS * 32) {
+      const int m = idx / R, j = idx - m * R;
+      float v = 0.f;
+#pragma unroll
+      for (int c = 0; c < RS_CTAS; ++c) v += ld_dsmem_f32(mapa_shared(base + 4u * (m * 64 + j), c));
+      out16a[idx] = static_cast<uint16_t>(bf16x2_bits(sa * v, 0.f));
+      if (out16b) out16b[idx] = static_cast<uint16_t>(bf16x2_bits(sb * v, 0.f));
+      if (out32) out32[idx] = sb * v;
+    }
+  }
+  cluster_sync_all();  // peers keep their shared memory until CTA 0 has read it
+}
+
 // ------------------------------------------------------------------ rows
 //
 // out[m, j] = sum_k P[m, k] Q(j, k) for 16 * CW tokens per CTA over the whole
@@ -330,7 +410,7 @@ cudaError_t rows_launch(const uint16_t* P, const uint16_t* Q, int64_t M, int64_t
   else
     ok = ok && make_map(&tmQ, BF16, Q, Kc, R, Kc * 2, 64, NT * 8, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(k_rows<NT, QT>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES);
+  cudaError_t e = smem_limit_once<k_rows<NT, QT>>(S::BYTES);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>((M + 16 * S::CW - 1) / (16 * S::CW));
   k_rows<NT, QT><<<grid, 32 * (S::CW + 1), S::BYTES, st>>>(tmP, tmQ, int(M), int(Kc), R, sa, out16a, sb, out16b,
@@ -357,7 +437,7 @@ cudaError_t cols_launch(const uint16_t* G, const uint16_t* P, int64_t M, int64_t
   bool ok = make_map(&tmP, BF16, P, C, M, C * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
   ok = ok && make_map(&tmG, BF16, G, R, M, R * 2, NT * 8, 32, narrow_swizzle<NT>());
   if (!ok) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(k_cols<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES);
+  cudaError_t e = smem_limit_once<k_cols<NT>>(S::BYTES);
   if (e != cudaSuccess) return e;
   const dim3 grid(static_cast<unsigned>((C + 63) / 64), static_cast<unsigned>(splits));
   k_cols<NT><<<grid, 160, S::BYTES, st>>>(tmP, tmG, int(M), int(C), R, rows_per_split, partial, device_status_ptr());
@@ -369,6 +449,15 @@ cudaError_t cols_launch(const uint16_t* G, const uint16_t* P, int64_t M, int64_t
 cudaError_t launch_rowdot(const uint16_t* P, const uint16_t* Q, int64_t M, int64_t Kc, int R, float sa,
                           uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st) {
   if (M == 0) return cudaSuccess;
+  if (M <= 16) {
+    const int iM = static_cast<int>(M), iK = static_cast<int>(Kc);
+    switch (nt_for(R)) {
+      case 2: k_rows_small<2><<<RS_CTAS, RS_WARPS * 32, 0, st>>>(P, Q, iM, iK, R, sa, out16a, sb, out16b, out32); break;
+      case 4: k_rows_small<4><<<RS_CTAS, RS_WARPS * 32, 0, st>>>(P, Q, iM, iK, R, sa, out16a, sb, out16b, out32); break;
+      default: k_rows_small<8><<<RS_CTAS, RS_WARPS * 32, 0, st>>>(P, Q, iM, iK, R, sa, out16a, sb, out16b, out32); break;
+    }
+    return cudaGetLastError();
+  }
   return rows_dispatch<false>(P, Q, M, Kc, R, sa, out16a, sb, out16b, out32, st);
 }
 

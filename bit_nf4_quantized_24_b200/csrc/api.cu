@@ -34,6 +34,22 @@ int current_device() {
   return d;
 }
 
+}  // namespace
+
+int device_sm_count() {
+  static std::atomic<int> cache[kMaxDevices] = {};
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return 148;
+  int v = cache[d].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || v <= 0) return 148;
+  cache[d].store(v, std::memory_order_relaxed);
+  return v;
+}
+
+namespace {
+
+
 template <typename T>
 T* symbol_ptr(T** cache, const void* symbol) {
   const int d = current_device();

@@ -403,8 +403,7 @@ cudaError_t launch_mode(const GemmArgs& a, cudaStream_t st) {
     ok = ok && make_map(&tm_tb, BF16, a.tail_b, a.K, a.r, a.K * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return cudaErrorInvalidValue;
 
-  // The attribute is per device; setting it on every launch covers every device.
-  cudaError_t e = cudaFuncSetAttribute(k_nf4_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
+  cudaError_t e = smem_limit_once<k_nf4_gemm<MODE>>(SMEM_ALLOC);
   if (e != cudaSuccess) return e;
 
   // Token tiles are rounded up to whole pairs: a CTA past the last token
@@ -437,8 +436,7 @@ cudaError_t launch_mode(const GemmArgs& a, cudaStream_t st) {
 
 template <int MODE>
 int max_active_pairs() {
-  if (cudaFuncSetAttribute(k_nf4_gemm<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC) != cudaSuccess)
-    return -1;
+  if (smem_limit_once<k_nf4_gemm<MODE>>(SMEM_ALLOC) != cudaSuccess) return -1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2, 1, 1);
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);

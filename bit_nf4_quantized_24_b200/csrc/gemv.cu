@@ -38,31 +38,56 @@ constexpr int G_SBLK = 2 * G_CW;                    // 64-weight blocks per stag
 constexpr int G_BOX = 128 * G_ROWS;                 // one TMA box: 16 rows x 128 code bytes
 constexpr int G_STAGE = (G_SBLK / 4) * G_BOX;       // 16 KB of codes per stage
 constexpr int G_TABLE = 65536;                      // 256 entries x 256 B (128 B used)
+constexpr int G_SDEPTH = 4;                         // stages the block-scale loads run ahead
 
+// Shared memory, from the 64 KB-aligned table T: the table (entry e of lane
+// l at T + 256 e + 4 l) fills the lower half of each 256-byte row; the upper
+// halves (T + 256 e + 128) are 32-float rows that hold the partial sums
+// handed to the epilogue warp.  The code ring, the warps' scale buffers and
+// the barriers follow the table.
 template <int NTILE>
-struct GemvSmem {  // offsets from the 64 KB-aligned table
-  static constexpr int NS = NTILE == 1 ? 5 : 4;                       // ring stages
-  static constexpr int RED_FLOATS = G_CW * NTILE * 4 * 32;             // one partial-sum buffer
+struct GemvSmem {
+  static constexpr int NS = 5;                                        // ring stages
+  static constexpr int RED_ROWS = G_CW * NTILE * 4;                   // 32-float rows per partial-sum buffer
   static constexpr int OFF_RING = G_TABLE;
-  static constexpr int OFF_RED = OFF_RING + NS * G_STAGE;
-  static constexpr int OFF_BAR = OFF_RED + 2 * RED_FLOATS * 4;
+  static constexpr int OFF_SCALE = OFF_RING + NS * G_STAGE;           // [warp][2][32] fp32 block scales
+  static constexpr int OFF_BAR = OFF_SCALE + G_CW * 2 * 32 * 4;
   static constexpr int USED = OFF_BAR + 8 * (2 * NS + 4);
   static constexpr int BYTES = USED + 65536;                          // room to align the table
 };
+static_assert(2 * GemvSmem<2>::RED_ROWS <= 256, "partial sums fit the table rows");
 static_assert(GemvSmem<1>::BYTES <= 232448 && GemvSmem<2>::BYTES <= 232448, "shared memory");
 
+// The MMA and the table loads are plain register functions for the compiler
+// (no volatile), so it can schedule the lookups of a block ahead of its MMAs.
+// Loads from the TMA ring stay volatile: they must not move above the wait.
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
       "{%0, %1, %2, %3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {  // the level table: written once, before any use
   uint32_t v;
-  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  asm("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void sts_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ float2 lds_f2(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
   return v;
 }
 
@@ -80,77 +105,54 @@ __device__ __forceinline__ uint32_t lut_pair(uint32_t word, uint32_t lane_base) 
 }
 
 // What one consumer lane preloads for one block: its activation fragment
-// (X[8nt + g][64b + 16t .. +15]) and the two row scales (rows g, g + 8).
+// X[8nt + g][64b + 16t .. +15].
 template <int NTILE>
 struct BlockIn {
   uint32_t x[NTILE][8];
-  uint32_t q[2];
-  float d[2];
 };
 
-template <int NTILE>
-__device__ __forceinline__ void load_block(BlockIn<NTILE>& in, const uint16_t* __restrict__ X, int M, int K,
-                                           const uint8_t* __restrict__ absmax_q,
-                                           const float* __restrict__ dq_scale, int N, int KB, int n0, int b,
-                                           int g, int t) {
-  const bool bok = b < KB;
+// NB (1 or 2) consecutive 64-weight blocks of a 16-row tile, as one
+// straight-line sequence so that the lookups and the two MMA chains of the
+// blocks interleave: the lane's code bytes of its two rows (8 box rows apart)
+// from the staged boxes, all table lookups, four MMA steps per block into a
+// fresh fragment, then the scaled add into acc.
+template <int NTILE, int NB>
+__device__ __forceinline__ void blocks_mma(float (&acc)[NTILE][4], const BlockIn<NTILE> (&in)[2],
+                                           const uint32_t (&code_addr)[2], uint32_t lane_base,
+                                           const float2 (&sc)[2]) {
+  uint2 cg[NB], ch[NB];
 #pragma unroll
-  for (int nt = 0; nt < NTILE; ++nt) {
-    const int m = 8 * nt + g;
-    uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
-    if (bok && m < M) {
-      const uint4* p = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(m) * K + 64 * b + 16 * t);
-      lo = __ldg(p);
-      hi = __ldg(p + 1);
-    }
-    in.x[nt][0] = lo.x; in.x[nt][1] = lo.y; in.x[nt][2] = lo.z; in.x[nt][3] = lo.w;
-    in.x[nt][4] = hi.x; in.x[nt][5] = hi.y; in.x[nt][6] = hi.z; in.x[nt][7] = hi.w;
+  for (int b = 0; b < NB; ++b) {
+    cg[b] = lds64(code_addr[b]);
+    ch[b] = lds64(code_addr[b] + 1024u);
   }
+  uint32_t a[NB][4][4];  // A fragments of the four k16 steps of each block
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int row = n0 + g + 8 * h;
-    in.q[h] = 0u;
-    in.d[h] = 0.f;
-    if (bok && row < N) {
-      const int64_t blk = static_cast<int64_t>(row) * KB + b;
-      in.q[h] = __ldg(absmax_q + blk);
-      in.d[h] = __ldg(dq_scale + (blk >> 8));
-    }
-  }
-}
-
-// One 64-weight block of a 16-row tile: codes of rows g and g + 8 from the
-// staged box, four MMA steps, then the scaled add into acc.
-template <int NTILE>
-__device__ __forceinline__ void block_mma(float (&acc)[NTILE][4], const BlockIn<NTILE>& in, uint32_t code_addr,
-                                          uint32_t lane_base) {
-  const uint2 cg = lds64(code_addr), ch = lds64(code_addr + 1024u);  // row g + 8 is 8 box rows further
-  float p[NTILE][4];
+  for (int b = 0; b < NB; ++b)
 #pragma unroll
-  for (int nt = 0; nt < NTILE; ++nt) p[nt][0] = p[nt][1] = p[nt][2] = p[nt][3] = 0.f;
-#pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    const uint32_t wg = s < 2 ? cg.x : cg.y, wh = s < 2 ? ch.x : ch.y;
-    uint32_t a0, a1, a2, a3;
-    if ((s & 1) == 0) {
-      a0 = lut_pair<0>(wg, lane_base); a2 = lut_pair<1>(wg, lane_base);
-      a1 = lut_pair<0>(wh, lane_base); a3 = lut_pair<1>(wh, lane_base);
-    } else {
-      a0 = lut_pair<2>(wg, lane_base); a2 = lut_pair<3>(wg, lane_base);
-      a1 = lut_pair<2>(wh, lane_base); a3 = lut_pair<3>(wh, lane_base);
+    for (int s = 0; s < 4; ++s) {
+      const uint32_t wg = s < 2 ? cg[b].x : cg[b].y, wh = s < 2 ? ch[b].x : ch[b].y;
+      if ((s & 1) == 0) {
+        a[b][s][0] = lut_pair<0>(wg, lane_base); a[b][s][2] = lut_pair<1>(wg, lane_base);
+        a[b][s][1] = lut_pair<0>(wh, lane_base); a[b][s][3] = lut_pair<1>(wh, lane_base);
+      } else {
+        a[b][s][0] = lut_pair<2>(wg, lane_base); a[b][s][2] = lut_pair<3>(wg, lane_base);
+        a[b][s][1] = lut_pair<2>(wh, lane_base); a[b][s][3] = lut_pair<3>(wh, lane_base);
+      }
     }
 #pragma unroll
-    for (int nt = 0; nt < NTILE; ++nt) mma16816(p[nt], a0, a1, a2, a3, in.x[nt][2 * s], in.x[nt][2 * s + 1]);
-  }
-  const float sg = __fmul_rn(static_cast<float>(in.q[0]), in.d[0]);
-  const float sh = __fmul_rn(static_cast<float>(in.q[1]), in.d[1]);
+  for (int b = 0; b < NB; ++b)
 #pragma unroll
-  for (int nt = 0; nt < NTILE; ++nt) {
-    acc[nt][0] = fmaf(sg, p[nt][0], acc[nt][0]);
-    acc[nt][1] = fmaf(sg, p[nt][1], acc[nt][1]);
-    acc[nt][2] = fmaf(sh, p[nt][2], acc[nt][2]);
-    acc[nt][3] = fmaf(sh, p[nt][3], acc[nt][3]);
-  }
+    for (int nt = 0; nt < NTILE; ++nt) {
+      float p[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int s = 0; s < 4; ++s)
+        mma16816(p, a[b][s][0], a[b][s][1], a[b][s][2], a[b][s][3], in[b].x[nt][2 * s], in[b].x[nt][2 * s + 1]);
+      acc[nt][0] = fmaf(sc[b].x, p[0], acc[nt][0]);
+      acc[nt][1] = fmaf(sc[b].x, p[1], acc[nt][1]);
+      acc[nt][2] = fmaf(sc[b].y, p[2], acc[nt][2]);
+      acc[nt][3] = fmaf(sc[b].y, p[3], acc[nt][3]);
+    }
 }
 
 template <int NTILE>
@@ -170,11 +172,15 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     return;
   }
   const uint32_t ring = table + S::OFF_RING;
-  float* red = reinterpret_cast<float*>(smem_raw + (table - raw) + S::OFF_RED);
+  // partial-sum row `row` of buffer `buf`, lane l: upper half of table row buf * RED_ROWS + row
+  auto red_addr = [&](int buf, int row, int l) -> uint32_t {
+    return table + (buf * S::RED_ROWS + row) * 256 + 128 + l * 4;
+  };
   const uint32_t full0 = table + S::OFF_BAR, empty0 = full0 + 8u * NS;
   const uint32_t rfull0 = empty0 + 8u * NS, rempty0 = rfull0 + 16u;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
+  const int pg = ((g & 3) << 1) | (g >> 2);  // tile row of MMA row g
 
   // table: entry e -> {bf16(L[e & 15]), bf16(L[e >> 4])}, one copy per lane
   for (int idx = tid; idx < 256 * 32; idx += G_THREADS) {
@@ -226,6 +232,9 @@ __global__ void __launch_bounds__(G_THREADS, 1)
   }
 
   if (warp == G_CW + 1) {  // epilogue: sum the K-split partials, add the LoRA term, store
+    // Hs comes from the previous kernel of the stream, which may still be
+    // running (programmatic dependent launch): wait for it to complete
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     for (int ti = 0; ti < t1 - t0; ++ti) {
       const int n0 = (t0 + ti) * G_ROWS;
       const int buf = ti & 1;
@@ -238,10 +247,10 @@ __global__ void __launch_bounds__(G_THREADS, 1)
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int j0 = 16 * k;
-        la[k][0] = ld2(Bl, n0 + g, N, j0 + 2 * t);
-        la[k][1] = ld2(Bl, n0 + g + 8, N, j0 + 2 * t);
-        la[k][2] = ld2(Bl, n0 + g, N, j0 + 2 * t + 8);
-        la[k][3] = ld2(Bl, n0 + g + 8, N, j0 + 2 * t + 8);
+        la[k][0] = ld2(Bl, n0 + pg, N, j0 + 2 * t);
+        la[k][1] = ld2(Bl, n0 + pg + 8, N, j0 + 2 * t);
+        la[k][2] = ld2(Bl, n0 + pg, N, j0 + 2 * t + 8);
+        la[k][3] = ld2(Bl, n0 + pg + 8, N, j0 + 2 * t + 8);
 #pragma unroll
         for (int nt = 0; nt < NTILE; ++nt) {
           lb[k][nt][0] = ld2(Hs, 8 * nt + g, M, j0 + 2 * t);
@@ -250,14 +259,13 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       }
       if (!wait_bounded(rfull0 + 8u * buf, (ti >> 1) & 1, &abort_flag, status)) break;
       float v[NTILE][4];
-      const float* rb = red + buf * S::RED_FLOATS;
 #pragma unroll
       for (int nt = 0; nt < NTILE; ++nt)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           float sum = 0.f;
 #pragma unroll 4
-          for (int w = 0; w < G_CW; ++w) sum += rb[((w * NTILE + nt) * 4 + c) * 32 + lane];
+          for (int w = 0; w < G_CW; ++w) sum += lds_f32(red_addr(buf, (w * NTILE + nt) * 4 + c, lane));
           v[nt][c] = sum;
         }
       __syncwarp();
@@ -274,7 +282,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         const int m = 8 * nt + 2 * t;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const int n = n0 + g + 8 * h;
+          const int n = n0 + pg + 8 * h;
           if (n >= N) continue;
           if (m < M) Y[static_cast<int64_t>(m) * N + n] = static_cast<uint16_t>(bf16x2_bits(v[nt][2 * h], 0.f));
           if (m + 1 < M)
@@ -285,47 +293,120 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     return;
   }
 
-  // consumers: warp w takes blocks 2w and 2w + 1 of every stage
+  // consumers: warp w takes blocks 2w and 2w + 1 of every stage.  MMA row g
+  // is tile row pg (and g + 8 is pg + 8): with this order the 16 lanes of a
+  // half-warp read 8 different 16-byte chunks of the swizzled box, so the
+  // 64-bit code loads are conflict-free.
   const uint32_t lane_base = table + lane * 4;
-  uint32_t coff[2];  // byte offset of this lane's 8 code bytes (row g) inside a stage
+  uint32_t coff[2];  // byte offset of this lane's 8 code bytes (row pg) inside a stage
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
     const int bb = 2 * warp + q;
     const int chunk = 2 * (bb & 3) + (t >> 1);
-    coff[q] = (bb >> 2) * G_BOX + g * 128 + ((chunk ^ g) << 4) + ((t & 1) << 3);
+    coff[q] = (bb >> 2) * G_BOX + pg * 128 + ((chunk ^ pg) << 4) + ((t & 1) << 3);
   }
+  // Token rows >= M read row M - 1 and weight rows >= N read row N - 1: those
+  // columns and rows of the product are computed but never stored.
+  const uint16_t* xrow[NTILE];
+#pragma unroll
+  for (int nt = 0; nt < NTILE; ++nt)
+    xrow[nt] = X + static_cast<int64_t>(min(8 * nt + g, M - 1)) * K + 16 * t + 128 * warp;
   float acc[NTILE][4];
 #pragma unroll
   for (int nt = 0; nt < NTILE; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
 
+  // Activation fragments are loaded one stage ahead of the MMAs into
+  // registers (ls: the stage they fetch; they do not depend on the tile).  The block
+  // scales come from HBM, so they run G_SDEPTH stages ahead in a register
+  // shift ring: one per lane (tile row lane & 15, block 2w + (lane >> 4));
+  // at its stage the lane stores absmax * dq_scale to the warp's scale
+  // buffer, where rows pg and pg + 8 of a block sit side by side.
+  const uint32_t wscale = table + S::OFF_SCALE + warp * (2 * 32 * 4);
+  const int srow = lane & 15, sq = lane >> 4;
+  const uint32_t sput = ((sq * 16 + (srow & 7) * 2 + (srow >> 3)) << 2);
+  const uint32_t sget = pg * 8;  // + q * 64 for block q
   BlockIn<NTILE> in[2];
-  int s = 0, ti = 0;
+  int ls = 0;
+  auto load_q = [&](int q) {
 #pragma unroll
-  for (int q = 0; q < 2; ++q)
-    load_block(in[q], X, M, K, absmax_q, dq_scale, N, KB, t0 * G_ROWS, 2 * warp + q, g, t);
-  for (int it = 0; it < nit; ++it) {
-    const int slot = it % NS;
-    if (!wait_bounded(full0 + 8u * slot, (it / NS) & 1, &abort_flag, status)) break;
-    // the block this slot refills with: same position, next stage
-    const int ns = s + 1 == spt ? 0 : s + 1;
-    const int nn0 = (t0 + ti + (s + 1 == spt ? 1 : 0)) * G_ROWS;
-    const bool more = it + 1 < nit;
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      if (s * G_SBLK + 2 * warp + q < KB) block_mma(acc, in[q], ring + slot * G_STAGE + coff[q], lane_base);
-      if (more) load_block(in[q], X, M, K, absmax_q, dq_scale, N, KB, nn0, ns * G_SBLK + 2 * warp + q, g, t);
+    for (int nt = 0; nt < NTILE; ++nt) {
+      const uint4* p = reinterpret_cast<const uint4*>(xrow[nt] + ls * (64 * G_SBLK) + 64 * q);
+      const uint4 lo = __ldg(p), hi = __ldg(p + 1);
+      in[q].x[nt][0] = lo.x; in[q].x[nt][1] = lo.y; in[q].x[nt][2] = lo.z; in[q].x[nt][3] = lo.w;
+      in[q].x[nt][4] = hi.x; in[q].x[nt][5] = hi.y; in[q].x[nt][6] = hi.z; in[q].x[nt][7] = hi.w;
     }
+  };
+  auto load_next = [&]() {  // both blocks of stage ls, or the one inside the row (warp-uniform)
+    const int nv = KB - ls * G_SBLK - 2 * warp;
+    if (nv >= 2) {
+      load_q(0);
+      load_q(1);
+    } else if (nv == 1) {
+      load_q(0);
+    }
+    if (++ls == spt) ls = 0;
+  };
+  uint32_t rq[G_SDEPTH];
+  float rd[G_SDEPTH];
+  int ss = 0, sn0 = t0 * G_ROWS;  // stage and tile row of the next scale load
+  int sidx = min(sn0 + srow, N - 1) * KB + 2 * warp + sq;
+  auto load_scale = [&](uint32_t& q, float& d) {
+    q = 0u;
+    d = 0.f;
+    if (ss * G_SBLK + 2 * warp + sq < KB) {
+      const int j = sidx + ss * G_SBLK;
+      q = __ldg(absmax_q + j);
+      d = __ldg(dq_scale + (j >> 8));
+    }
+    if (++ss == spt) {
+      ss = 0;
+      sn0 += G_ROWS;
+      sidx = min(sn0 + srow, N - 1) * KB + 2 * warp + sq;
+    }
+  };
+  load_next();
+#pragma unroll
+  for (int i = 0; i < G_SDEPTH; ++i) load_scale(rq[i], rd[i]);  // loads past the last stage read clamped rows
+
+  int s = 0, ti = 0, slot = 0;
+  uint32_t ph = 0;
+  for (int it = 0; it < nit; ++it) {
+    if (!wait_bounded(full0 + 8u * slot, ph, &abort_flag, status)) break;
+    const bool more = it + 1 < nit;
+    const int nvalid = KB - s * G_SBLK - 2 * warp;  // blocks of this warp inside the row
+    const uint32_t sbuf = wscale + ((it & 1) << 7);
+    sts_f32(sbuf + sput, __fmul_rn(static_cast<float>(rq[0]), rd[0]));
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i + 1 < G_SDEPTH; ++i) {
+      rq[i] = rq[i + 1];
+      rd[i] = rd[i + 1];
+    }
+    load_scale(rq[G_SDEPTH - 1], rd[G_SDEPTH - 1]);
+    {
+      const uint32_t sb = ring + slot * G_STAGE;
+      const uint32_t ca[2] = {sb + coff[0], sb + coff[1]};
+      const float2 sc[2] = {lds_f2(sbuf + sget), lds_f2(sbuf + sget + 64)};
+      if (nvalid >= 2)
+        blocks_mma<NTILE, 2>(acc, in, ca, lane_base, sc);
+      else if (nvalid == 1)
+        blocks_mma<NTILE, 1>(acc, in, ca, lane_base, sc);
+    }
+    if (more) load_next();
     __syncwarp();
     if (lane == 0) mbar_arrive(empty0 + 8u * slot);
+    if (++slot == NS) {
+      slot = 0;
+      ph ^= 1u;
+    }
     if (++s == spt) {  // tile done: hand the partial sums to the epilogue warp
       const int buf = ti & 1;
       if (!wait_bounded(rempty0 + 8u * buf, ((ti >> 1) & 1) ^ 1, &abort_flag, status)) break;
-      float* rb = red + buf * S::RED_FLOATS;
 #pragma unroll
       for (int nt = 0; nt < NTILE; ++nt)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          rb[((warp * NTILE + nt) * 4 + c) * 32 + lane] = acc[nt][c];
+          sts_f32(red_addr(buf, (warp * NTILE + nt) * 4 + c, lane), acc[nt][c]);
           acc[nt][c] = 0.f;
         }
       __syncwarp();
@@ -341,16 +422,25 @@ cudaError_t gemv_launch(const CUtensorMap& tm, const uint16_t* X, int64_t M, con
                         const float* dq_scale, int64_t N, int64_t K, const uint16_t* Hs, const uint16_t* B, int r,
                         uint16_t* Y, cudaStream_t st) {
   using S = GemvSmem<NTILE>;
-  cudaError_t e = cudaFuncSetAttribute(k_gemv<NTILE>, cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES);
+  cudaError_t e = smem_limit_once<k_gemv<NTILE>>(S::BYTES);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = device_sm_count();
   const int64_t ntiles = (N + G_ROWS - 1) / G_ROWS;
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ntiles, sms));
-  k_gemv<NTILE><<<grid, G_THREADS, S::BYTES, st>>>(tm, X, int(M), absmax_q, dq_scale, int(N), int(K), Hs, B, r,
-                                                   host_codebook().levels, Y, device_status_ptr());
-  return cudaGetLastError();
+  // Programmatic dependent launch: the weight stream starts while the kernel
+  // that computes Hs finishes; only the epilogue warp waits for it.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(G_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = S::BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_gemv<NTILE>, tm, static_cast<const uint16_t*>(X), int(M), absmax_q, dq_scale,
+                            int(N), int(K), Hs, B, r, host_codebook().levels, Y, device_status_ptr());
 }
 
 }  // namespace
@@ -359,7 +449,7 @@ cudaError_t launch_gemv(const uint16_t* X, int64_t M, const uint8_t* codes, cons
                         const float* dq_scale, int64_t N, int64_t K, const uint16_t* Hs, const uint16_t* B, int r,
                         uint16_t* Y, cudaStream_t st) {
   if (M == 0 || N == 0) return cudaSuccess;
-  if (M > 16 || r > 64) return cudaErrorInvalidValue;
+  if (M > 16 || r > 64 || N * (K / 64) >= (int64_t(1) << 31)) return cudaErrorInvalidValue;  // 32-bit block index
   CUtensorMap tm;
   if (!make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, 128, G_ROWS,
                 CU_TENSOR_MAP_SWIZZLE_128B))

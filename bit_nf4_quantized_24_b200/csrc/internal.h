@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "common.cuh"
 
 namespace qn {
@@ -57,7 +59,8 @@ int nf4_gemm_max_active_pairs(int mode);
 // ----- adapter kernels
 // out[m, j] = sum_k P[m,k] Q[j,k]  (P bf16 [M, Kc], Q bf16 [R, Kc]); writes
 // out16a = bf16(sa * acc) [M,R], out16b = bf16(sb * acc) (nullable),
-// out32 = sb * acc fp32 (nullable).
+// out32 = sb * acc fp32 (nullable).  M <= 16 runs a split-contraction kernel
+// that allows the next kernel of the stream an early (programmatic) launch.
 cudaError_t launch_rowdot(const uint16_t* P, const uint16_t* Q, int64_t M, int64_t Kc, int R, float sa,
                           uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st);
 // out[j, c] = sum_m G[m, j] P[m, c] over all m (G bf16 [M, R], P bf16 [M, C]),
@@ -74,6 +77,25 @@ cudaError_t launch_rowdot_qt(const uint16_t* P, const uint16_t* Qt, int64_t M, i
 cudaError_t launch_gemv(const uint16_t* X, int64_t M, const uint8_t* codes, const uint8_t* absmax_q,
                         const float* dq_scale, int64_t N, int64_t K, const uint16_t* Hs, const uint16_t* B, int r,
                         uint16_t* Y, cudaStream_t st);
+
+// ----- per-device launch setup, done once per device and kernel
+
+// Raises the dynamic shared-memory limit of kernel KERN to `bytes` on the
+// current device the first time it is asked for that device.
+template <auto KERN>
+cudaError_t smem_limit_once(int bytes) {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(KERN, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
+// Streaming multiprocessors of the current device (cached per device).
+int device_sm_count();
 
 // ----- tracing of the fused GEMM launches
 void trace_before(cudaStream_t st);

@@ -159,10 +159,32 @@ def test_forward_small(qb, oracle, M, N, K, r):
     run_fwd_check(qb, oracle, p)
 
 
-@pytest.mark.parametrize("M,N,K,r", [(1, 64, 64, 8), (4, 264, 320, 16), (16, 1000, 1024, 64), (9, 72, 4096, 8)])
+DECODE = [
+    (1, 64, 64, 8),
+    (4, 264, 320, 16),
+    (16, 1000, 1024, 64),
+    (9, 72, 4096, 8),
+    (8, 136, 2112, 24),    # 33 blocks per row: the last stage holds one block
+    (13, 520, 11008, 40),  # 172 blocks per row, r not a multiple of 16
+    (2, 8, 64, 8),         # a single half tile
+]
+
+
+@pytest.mark.parametrize("M,N,K,r", DECODE)
 def test_forward_decode_small(qb, oracle, M, N, K, r):
     p = wl.draw_small(2000 + M + N, M, N, K, r, 2.0 * r, with_dy=False)
     run_fwd_check(qb, oracle, p)
+
+
+def test_decode_repeatable(qb):
+    """The decode kernel sums its K-split partials in a fixed order: two calls
+    give the same bits."""
+    p = wl.draw_small(2100, 5, 2056, 4160, 16, 32.0, with_dy=False)
+    q = qb.nf4_quantize(p["W"].cuda())
+    X, A, B = p["X"].cuda(), p["A"].cuda(), p["B"].cuda()
+    Y1, _ = qb.qlora_linear_fwd(q, X, A, B, p["scale"])
+    Y2, _ = qb.qlora_linear_fwd(q, X, A, B, p["scale"])
+    assert torch.equal(Y1, Y2)
 
 
 @pytest.mark.parametrize("M,N,K,r", SMALL)
