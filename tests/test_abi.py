@@ -68,3 +68,18 @@ def test_workspace_sizes_grow_with_shape(L):
     b = qb.fwd_workspace_bytes(4096, 4096, 4096, 16)
     assert 0 < a < b and a % 256 == 0 and b % 256 == 0
     assert qb.bwd_workspace_bytes(4096, 4096, 4096, 16) > qb.bwd_workspace_bytes(128, 2048, 2048, 8)
+
+
+def test_midpoints_avoid_the_quantizer_cell_edges(L):
+    """The GPU quantizer finds a code from the 1/64-wide cell that holds
+    t = w / absmax (cell edges at odd multiples of 1/128) plus one compare with
+    the single midpoint inside the cell.  That is exact only if cells are
+    narrower than the midpoint spacing and no midpoint sits on a cell edge."""
+    lv = (ctypes.c_float * 16)()
+    assert L.nf4_codebook(lv) == 0
+    levels = np.array(list(lv), dtype=np.float32)
+    mids = ((levels[:-1] + levels[1:]) * np.float32(0.5)).astype(np.float32)
+    assert np.all(np.diff(mids.astype(np.float64)) > 1.0 / 64)
+    scaled = mids.astype(np.float64) * 128.0
+    on_edge = (scaled == np.round(scaled)) & (np.round(scaled) % 2 == 1)
+    assert not on_edge.any()

@@ -121,6 +121,30 @@ def test_quantize_codebook_values_and_ties(qb, oracle):
     quantize_both(qb, oracle, W)
 
 
+def test_quantize_near_midpoints_any_scale(qb, oracle):
+    """Weights within a few ulps of m * midpoint for block absmax m of every
+    size (not powers of two), so that the quotient w / m lands next to a
+    midpoint: the GPU's division and code lookup must match the oracle's
+    IEEE division and midpoint count bit for bit."""
+    _, _, m32 = oracle.nf4_codebook()
+    g = np.random.default_rng(123)
+    rows = []
+    for e in (-110, -60, -20, -7, -1, 0, 3, 40, 90, 110):
+        for _ in range(40):
+            m = np.float32(g.uniform(1.0, 2.0) * 2.0 ** e)
+            r = np.empty(64, np.float32)
+            r[0] = m
+            for j in range(1, 64):
+                mid = m32[g.integers(0, 15)]
+                w = np.float32(np.float64(mid) * np.float64(m))
+                for _ in range(int(g.integers(-3, 4))):
+                    w = np.nextafter(w, np.float32(np.inf) if g.random() < 0.5 else np.float32(-np.inf))
+                r[j] = np.clip(w, -m, m)
+            rows.append(r)
+    W = torch.from_numpy(np.stack(rows).astype(np.float32))
+    quantize_both(qb, oracle, W)
+
+
 def test_quantize_rejects_nonfinite(qb):
     for bad in (float("nan"), float("inf"), -float("inf")):
         W = torch.zeros(4, 128, device="cuda")
