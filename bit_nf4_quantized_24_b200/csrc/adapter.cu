@@ -79,7 +79,8 @@ __global__ void __cluster_dims__(RS_CTAS, 1, 1) __launch_bounds__(RS_WARPS * 32)
                  float* __restrict__ out32) {
   __shared__ float wpart[RS_WARPS][16 * 64];
   __shared__ float cpart[16 * 64];
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  pdl_trigger();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const int rank = static_cast<int>(cluster_ctarank());
   const int worker = rank * RS_WARPS + warp;
@@ -160,6 +161,8 @@ __global__ void __launch_bounds__(32 * (NT / 2 + 1)) k_rows(const __grid_constan
                                                             int* status) {
   using S = RowsSmem<NT>;
   constexpr int CW = S::CW;
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t full0 = base + S::OFF_BAR, empty0 = full0 + 8u * RW_ST;
@@ -273,6 +276,8 @@ __global__ void __launch_bounds__(160) k_cols(const __grid_constant__ CUtensorMa
                                               const __grid_constant__ CUtensorMap tmG, int M, int C, int R,
                                               int rows_per_split, float* __restrict__ partial, int* status) {
   using S = ColsSmem<NT>;
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t full0 = base + S::OFF_BAR, empty0 = full0 + 8u * CL_ST;
@@ -360,6 +365,8 @@ __global__ void __launch_bounds__(160) k_cols(const __grid_constant__ CUtensorMa
 // segment of 8 values is one 16-byte store.
 __global__ void __launch_bounds__(64) k_coldot_reduce(const float* __restrict__ partial, int splits, int R, int C,
                                                       float scale, int transpose, uint16_t* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   const int j0 = blockIdx.y * 8;
   if (c >= C) return;
@@ -400,7 +407,7 @@ int coldot_splits(int64_t M, int64_t C) {
 
 template <int NT, bool QT>
 cudaError_t rows_launch(const uint16_t* P, const uint16_t* Q, int64_t M, int64_t Kc, int R, float sa,
-                        uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st) {
+                        uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st, bool pdl) {
   using S = RowsSmem<NT>;
   CUtensorMap tmP, tmQ;
   const auto BF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -413,24 +420,23 @@ cudaError_t rows_launch(const uint16_t* P, const uint16_t* Q, int64_t M, int64_t
   cudaError_t e = smem_limit_once<k_rows<NT, QT>>(S::BYTES);
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>((M + 16 * S::CW - 1) / (16 * S::CW));
-  k_rows<NT, QT><<<grid, 32 * (S::CW + 1), S::BYTES, st>>>(tmP, tmQ, int(M), int(Kc), R, sa, out16a, sb, out16b,
-                                                           out32, device_status_ptr());
-  return cudaGetLastError();
+  return launch_ex(k_rows<NT, QT>, dim3(grid), dim3(32 * (S::CW + 1)), S::BYTES, st, pdl, tmP, tmQ, int(M), int(Kc),
+                   R, sa, out16a, sb, out16b, out32, device_status_ptr());
 }
 
 template <bool QT>
 cudaError_t rows_dispatch(const uint16_t* P, const uint16_t* Q, int64_t M, int64_t Kc, int R, float sa,
-                          uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st) {
+                          uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st, bool pdl) {
   switch (nt_for(R)) {
-    case 2: return rows_launch<2, QT>(P, Q, M, Kc, R, sa, out16a, sb, out16b, out32, st);
-    case 4: return rows_launch<4, QT>(P, Q, M, Kc, R, sa, out16a, sb, out16b, out32, st);
-    default: return rows_launch<8, QT>(P, Q, M, Kc, R, sa, out16a, sb, out16b, out32, st);
+    case 2: return rows_launch<2, QT>(P, Q, M, Kc, R, sa, out16a, sb, out16b, out32, st, pdl);
+    case 4: return rows_launch<4, QT>(P, Q, M, Kc, R, sa, out16a, sb, out16b, out32, st, pdl);
+    default: return rows_launch<8, QT>(P, Q, M, Kc, R, sa, out16a, sb, out16b, out32, st, pdl);
   }
 }
 
 template <int NT>
 cudaError_t cols_launch(const uint16_t* G, const uint16_t* P, int64_t M, int64_t C, int R, int splits,
-                        int rows_per_split, float* partial, cudaStream_t st) {
+                        int rows_per_split, float* partial, cudaStream_t st, bool pdl) {
   using S = ColsSmem<NT>;
   CUtensorMap tmP, tmG;
   const auto BF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -440,31 +446,31 @@ cudaError_t cols_launch(const uint16_t* G, const uint16_t* P, int64_t M, int64_t
   cudaError_t e = smem_limit_once<k_cols<NT>>(S::BYTES);
   if (e != cudaSuccess) return e;
   const dim3 grid(static_cast<unsigned>((C + 63) / 64), static_cast<unsigned>(splits));
-  k_cols<NT><<<grid, 160, S::BYTES, st>>>(tmP, tmG, int(M), int(C), R, rows_per_split, partial, device_status_ptr());
-  return cudaGetLastError();
+  return launch_ex(k_cols<NT>, grid, dim3(160), S::BYTES, st, pdl, tmP, tmG, int(M), int(C), R, rows_per_split,
+                   partial, device_status_ptr());
 }
 
 }  // namespace
 
 cudaError_t launch_rowdot(const uint16_t* P, const uint16_t* Q, int64_t M, int64_t Kc, int R, float sa,
-                          uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st) {
+                          uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st, bool pdl) {
   if (M == 0) return cudaSuccess;
   if (M <= 16) {
     const int iM = static_cast<int>(M), iK = static_cast<int>(Kc);
+    const dim3 g(RS_CTAS), b(RS_WARPS * 32);
     switch (nt_for(R)) {
-      case 2: k_rows_small<2><<<RS_CTAS, RS_WARPS * 32, 0, st>>>(P, Q, iM, iK, R, sa, out16a, sb, out16b, out32); break;
-      case 4: k_rows_small<4><<<RS_CTAS, RS_WARPS * 32, 0, st>>>(P, Q, iM, iK, R, sa, out16a, sb, out16b, out32); break;
-      default: k_rows_small<8><<<RS_CTAS, RS_WARPS * 32, 0, st>>>(P, Q, iM, iK, R, sa, out16a, sb, out16b, out32); break;
+      case 2: return launch_ex(k_rows_small<2>, g, b, 0, st, pdl, P, Q, iM, iK, R, sa, out16a, sb, out16b, out32);
+      case 4: return launch_ex(k_rows_small<4>, g, b, 0, st, pdl, P, Q, iM, iK, R, sa, out16a, sb, out16b, out32);
+      default: return launch_ex(k_rows_small<8>, g, b, 0, st, pdl, P, Q, iM, iK, R, sa, out16a, sb, out16b, out32);
     }
-    return cudaGetLastError();
   }
-  return rows_dispatch<false>(P, Q, M, Kc, R, sa, out16a, sb, out16b, out32, st);
+  return rows_dispatch<false>(P, Q, M, Kc, R, sa, out16a, sb, out16b, out32, st, pdl);
 }
 
 cudaError_t launch_rowdot_qt(const uint16_t* P, const uint16_t* Qt, int64_t M, int64_t Kc, int R, float sa,
-                             uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st) {
+                             uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st, bool pdl) {
   if (M == 0) return cudaSuccess;
-  return rows_dispatch<true>(P, Qt, M, Kc, R, sa, out16a, sb, out16b, out32, st);
+  return rows_dispatch<true>(P, Qt, M, Kc, R, sa, out16a, sb, out16b, out32, st, pdl);
 }
 
 size_t coldot_partial_floats(int64_t M, int64_t C, int R) {
@@ -472,16 +478,16 @@ size_t coldot_partial_floats(int64_t M, int64_t C, int R) {
 }
 
 cudaError_t launch_coldot(const uint16_t* G, const uint16_t* P, int64_t M, int64_t C, int R, float scale,
-                          int transpose, float* partial, uint16_t* out, cudaStream_t st) {
+                          int transpose, float* partial, uint16_t* out, cudaStream_t st, bool pdl) {
   const int splits = coldot_splits(M, C);
   // token ranges are whole 32-token slabs, so a slab never straddles two splits
   const int rows_per_split = static_cast<int>(((M + splits - 1) / splits + 31) / 32 * 32);
   cudaError_t e = cudaSuccess;
   if (M > 0) {
     switch (nt_for(R)) {
-      case 2: e = cols_launch<2>(G, P, M, C, R, splits, rows_per_split, partial, st); break;
-      case 4: e = cols_launch<4>(G, P, M, C, R, splits, rows_per_split, partial, st); break;
-      default: e = cols_launch<8>(G, P, M, C, R, splits, rows_per_split, partial, st); break;
+      case 2: e = cols_launch<2>(G, P, M, C, R, splits, rows_per_split, partial, st, pdl); break;
+      case 4: e = cols_launch<4>(G, P, M, C, R, splits, rows_per_split, partial, st, pdl); break;
+      default: e = cols_launch<8>(G, P, M, C, R, splits, rows_per_split, partial, st, pdl); break;
     }
   } else {
     e = cudaMemsetAsync(partial, 0, sizeof(float) * R * C, st);
@@ -489,8 +495,9 @@ cudaError_t launch_coldot(const uint16_t* G, const uint16_t* P, int64_t M, int64
   if (e != cudaSuccess) return e;
   const int sp = M > 0 ? splits : 1;
   const dim3 rgrid(static_cast<unsigned>((C + 63) / 64), static_cast<unsigned>(R / 8));
-  k_coldot_reduce<<<rgrid, 64, 0, st>>>(partial, sp, R, int(C), scale, transpose, out);
-  return cudaGetLastError();
+  // the reduce follows the partial kernel directly (or a memset when M == 0)
+  return launch_ex(k_coldot_reduce, rgrid, dim3(64), 0, st, M > 0, static_cast<const float*>(partial), sp, R,
+                   int(C), scale, transpose, out);
 }
 
 }  // namespace qn

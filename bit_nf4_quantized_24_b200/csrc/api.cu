@@ -259,6 +259,7 @@ int qlora_linear_fwd(const uint8_t* codes, const uint8_t* absmax_q, const float*
     a.K = K;
     a.r = r;
     a.out = Y;
+    a.pdl = true;  // its main loop runs while the H kernel finishes; the LoRA tail waits
     e = launch_nf4_gemm(a, s);
   }
   return cuda_status(e);
@@ -288,13 +289,20 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* absmax_q, const float*
     if (e == cudaSuccess) e = cudaMemsetAsync(dB, 0, static_cast<size_t>(N) * r * 2, s);
     return cuda_status(e);
   }
+  // Kernel order: dH, (H), dA, dB, then the dX GEMM.  Each kernel after the
+  // first is a programmatic dependent launch that waits for its predecessor
+  // before touching shared data; putting the large GEMM last lets its main
+  // loop start while the adapter kernels finish (only its LoRA tail reads dH).
   // dH = scale * dY B  (B [N, r] read in place: its rows are the contraction)
-  e = launch_rowdot_qt(dY, B, M, N, r, scale, w.dH16, scale, nullptr, nullptr, s);
+  e = launch_rowdot_qt(dY, B, M, N, r, scale, w.dH16, scale, nullptr, nullptr, s, false);
   const uint16_t* Huse = H;
   if (e == cudaSuccess && !H) {
-    e = launch_rowdot(X, A, M, K, r, 1.0f, w.H16, 1.0f, nullptr, nullptr, s);
+    e = launch_rowdot(X, A, M, K, r, 1.0f, w.H16, 1.0f, nullptr, nullptr, s, true);
     Huse = w.H16;
   }
+  // dA = dH^T X ;  dB = scale * dY^T H
+  if (e == cudaSuccess) e = launch_coldot(w.dH16, X, M, K, r, 1.0f, 0, w.partial, dA, s, true);
+  if (e == cudaSuccess) e = launch_coldot(Huse, dY, M, N, r, scale, 1, w.partial, dB, s, true);
   // dX = dY deq(W) + dH A
   if (e == cudaSuccess && dX) {
     GemmArgs a{};
@@ -310,11 +318,9 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* absmax_q, const float*
     a.K = K;
     a.r = r;
     a.out = dX;
+    a.pdl = true;
     e = launch_nf4_gemm(a, s);
   }
-  // dA = dH^T X ;  dB = scale * dY^T H
-  if (e == cudaSuccess) e = launch_coldot(w.dH16, X, M, K, r, 1.0f, 0, w.partial, dA, s);
-  if (e == cudaSuccess) e = launch_coldot(Huse, dY, M, N, r, scale, 1, w.partial, dB, s);
   return cuda_status(e);
 }
 

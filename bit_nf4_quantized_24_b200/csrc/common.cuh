@@ -216,6 +216,19 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
   }
 }
 
+// ------------------------------------------------ programmatic dependent launch
+//
+// pdl_trigger lets the next kernel of the stream begin launching once every
+// CTA of this grid has called it (or exited).  pdl_wait blocks the calling
+// thread until the previous kernel of the stream has completed and its writes
+// are visible; it returns at once when this kernel was launched without the
+// programmatic-serialization attribute.  Every kernel that is launched with the
+// attribute calls pdl_wait (at least in one thread of each CTA) before it
+// reads or overwrites anything an earlier kernel of the layer touches, and
+// before it exits, so that its completion implies that of all earlier kernels.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // -------------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

@@ -82,6 +82,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                const __grid_constant__ CUtensorMap tm_tail_a, const __grid_constant__ CUtensorMap tm_tail_b,
                const uint8_t* __restrict__ absmax_q, const float* __restrict__ dq_scale, Nf4Levels lv, int M, int N,
                int K, int r, int band_pairs, __nv_bfloat16* __restrict__ out, int* status) {
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -183,6 +184,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tma_load_2d(base + OFF_A + s * A_BYTES, &tm_act, full_tma(s), it * BK, m0);
         ++a_issued;
       }
+      // The tail operands come from the previous kernel of the stream, which
+      // may still be running (programmatic dependent launch); every other
+      // input of this kernel predates it.  Waited for on every path, so that
+      // this grid completes only after its predecessor.
+      pdl_wait();
       if (ok) {  // tail stage: LoRA operands
         const int it = numK, s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
@@ -419,13 +425,15 @@ cudaError_t launch_mode(const GemmArgs& a, cudaStream_t st) {
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = SMEM_ALLOC;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;  // the two CTAs of a pair hold consecutive token tiles
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = a.pdl ? 2 : 1;
   trace_before(st);
   e = cudaLaunchKernelEx(&cfg, k_nf4_gemm<MODE>, tm_act, tm_codes, tm_ta, tm_tb, a.absmax_q, a.dq_scale,
                          host_codebook().levels, static_cast<int>(a.M), static_cast<int>(a.N), static_cast<int>(a.K),

@@ -163,6 +163,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
            uint16_t* __restrict__ Y, int* status) {
   using S = GemvSmem<NTILE>;
   constexpr int NS = S::NS;
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   __shared__ int abort_flag;
   const uint32_t raw = smem_u32(smem_raw);
@@ -234,7 +235,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
   if (warp == G_CW + 1) {  // epilogue: sum the K-split partials, add the LoRA term, store
     // Hs comes from the previous kernel of the stream, which may still be
     // running (programmatic dependent launch): wait for it to complete
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    pdl_wait();
     for (int ti = 0; ti < t1 - t0; ++ti) {
       const int n0 = (t0 + ti) * G_ROWS;
       const int buf = ti & 1;

@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <utility>
 
 #include "common.cuh"
 
@@ -50,6 +51,7 @@ struct GemmArgs {
   int64_t M, N, K;
   int r;
   uint16_t* out;  // Y [M, N] or dX [M, K]
+  bool pdl;       // launched right after another kernel of the layer (programmatic dependent launch)
 };
 cudaError_t launch_nf4_gemm(const GemmArgs& a, cudaStream_t st);
 // CTA pairs of the fused GEMM that fit on the current device at once
@@ -62,16 +64,18 @@ int nf4_gemm_max_active_pairs(int mode);
 // out32 = sb * acc fp32 (nullable).  M <= 16 runs a split-contraction kernel
 // that allows the next kernel of the stream an early (programmatic) launch.
 cudaError_t launch_rowdot(const uint16_t* P, const uint16_t* Q, int64_t M, int64_t Kc, int R, float sa,
-                          uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st);
+                          uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st,
+                          bool pdl = false);
 // out[j, c] = sum_m G[m, j] P[m, c] over all m (G bf16 [M, R], P bf16 [M, C]),
 // written as bf16(scale * out) either [R, C] (transpose = 0) or [C, R]
 // (transpose = 1).  partial: fp32 scratch of coldot_partial_floats(...) floats.
 size_t coldot_partial_floats(int64_t M, int64_t C, int R);
 cudaError_t launch_coldot(const uint16_t* G, const uint16_t* P, int64_t M, int64_t C, int R, float scale,
-                          int transpose, float* partial, uint16_t* out, cudaStream_t st);
+                          int transpose, float* partial, uint16_t* out, cudaStream_t st, bool pdl = false);
 // The same with Q given transposed, Qt bf16 [Kc, R] (lora_B read in place).
 cudaError_t launch_rowdot_qt(const uint16_t* P, const uint16_t* Qt, int64_t M, int64_t Kc, int R, float sa,
-                             uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st);
+                             uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st,
+                             bool pdl = false);
 
 // ----- decode GEMV (M <= 16): Y = X deq(W)^T + Hs B^T, Hs = bf16(s X A^T)
 cudaError_t launch_gemv(const uint16_t* X, int64_t M, const uint8_t* codes, const uint8_t* absmax_q,
@@ -96,6 +100,25 @@ cudaError_t smem_limit_once(int bytes) {
 }
 // Streaming multiprocessors of the current device (cached per device).
 int device_sm_count();
+
+// Launches `kern` on `st`; with pdl the launch may begin while the previous
+// kernel of the stream is still running (the kernel synchronises with
+// pdl_wait, see common.cuh).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                      Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // ----- tracing of the fused GEMM launches
 void trace_before(cudaStream_t st);

@@ -117,6 +117,7 @@ extern "C" int qlora_linear_fwd_noalloc(const uint8_t* codes, const uint8_t* abs
       a.K = K;
       a.r = r;
       a.out = Y;
+      a.pdl = true;
       e = launch_nf4_gemm(a, s);
     }
   }
