@@ -254,37 +254,49 @@ __global__ void __launch_bounds__(32 * (NT / 2 + 1)) k_rows(const __grid_constan
 
 // ------------------------------------------------------------------ cols
 //
-// partial[split][j][c] = sum over this split's tokens m of G[m, j] P[m, c]:
-// D[c, j] = sum_m P^T[c, m] G[m, j].  CTA = 64 columns c (4 consumer warps of
-// 16) x all R, over one token range (a multiple of 32 tokens); warp 4 lane 0
-// streams 32-token slabs of P (32 x 64, 128-byte swizzle) and G (32 x NT*8)
-// through CL_ST stages.  Both operands have the contraction as their row and
-// are read with ldmatrix.trans.  Rows past M arrive as zeros from TMA.
+// out = bf16(scale * D), D[c, j] = sum_m P[m, c] G[m, j] (contraction over
+// tokens), written as [R, C] or transposed [C, R].  A cluster of CL_SPLIT CTAs
+// (consecutive along grid x) owns 64 columns c x all R; its CTAs split the
+// tokens into ranges of whole 32-token slabs.  In a CTA, warp 4 lane 0 streams
+// 32-token slabs of P (32 x 64, 128-byte swizzle) and G (32 x NT*8) through
+// CL_ST stages and 4 consumer warps (16 columns each) run ldmatrix.trans +
+// mma.sync.  The CTAs then leave their fp32 partial sums in shared memory and,
+// after a cluster barrier, each CTA adds one share of the outputs over the
+// cluster's partials (distributed shared memory, fixed order) and stores it:
+// no global scratch, no second kernel, deterministic.  Rows past M arrive as
+// zeros from TMA.
 constexpr int CL_ST = 8;
+constexpr int CL_SPLIT_MAX = 8;  // portable cluster size
 
 template <int NT>
 struct ColsSmem {
   static constexpr int P_BYTES = 32 * 64 * 2;
   static constexpr int G_BYTES = 32 * NT * 8 * 2;
   static constexpr int OFF_G = CL_ST * P_BYTES;
-  static constexpr int OFF_BAR = OFF_G + CL_ST * G_BYTES;
+  static constexpr int OFF_PART = OFF_G + CL_ST * G_BYTES;      // fp32 [64 c][NT * 8 j]
+  static constexpr int OFF_BAR = OFF_PART + 64 * NT * 8 * 4;
   static constexpr int BYTES = OFF_BAR + 2 * CL_ST * 8 + 1024;
 };
 
 template <int NT>
 __global__ void __launch_bounds__(160) k_cols(const __grid_constant__ CUtensorMap tmP,
                                               const __grid_constant__ CUtensorMap tmG, int M, int C, int R,
-                                              int rows_per_split, float* __restrict__ partial, int* status) {
+                                              int rows_per_split, float scale, int transpose,
+                                              uint16_t* __restrict__ out, int* status) {
   using S = ColsSmem<NT>;
+  constexpr int RJ = NT * 8;  // j extent of the partial buffer
   pdl_trigger();
   pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t full0 = base + S::OFF_BAR, empty0 = full0 + 8u * CL_ST;
+  const uint32_t part = base + S::OFF_PART;
   __shared__ int abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int c0 = blockIdx.x * 64;
-  const int split = blockIdx.y;
+  uint32_t nsplit;
+  asm("mov.u32 %0, %%cluster_nctarank;" : "=r"(nsplit));
+  const int split = static_cast<int>(cluster_ctarank());
+  const int c0 = (blockIdx.x / nsplit) * 64;
   const int mb0 = split * rows_per_split;
   const int mb1 = min(M, mb0 + rows_per_split);
   const int nslab = mb1 > mb0 ? (mb1 - mb0 + 31) / 32 : 0;
@@ -312,97 +324,86 @@ __global__ void __launch_bounds__(160) k_cols(const __grid_constant__ CUtensorMa
       for (int it = (issued > CL_ST ? issued - CL_ST : 0); it < issued; ++it)
         wait_drain(full0 + 8u * (it % CL_ST), (it / CL_ST) & 1);
     }
-    return;
-  }
-
-  float acc[NT][4];
-#pragma unroll
-  for (int i = 0; i < NT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-  const int q = lane >> 3, l7 = lane & 7;
-  for (int it = 0; it < nslab; ++it) {
-    const int s = it % CL_ST;
-    if (!wait_bounded(full0 + 8u * s, (it / CL_ST) & 1, &abort_flag, status)) break;
-    const uint32_t pt = base + s * S::P_BYTES;
-    const uint32_t gt = base + S::OFF_G + s * S::G_BYTES;
-#pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-      uint32_t a0, a1, a2, a3;  // P^T: (c 0-7, m 0-7), (c 8-15, m 0-7), (c 0-7, m 8-15), (c 8-15, m 8-15)
-      {
-        const int m = 16 * ks + (q >> 1) * 8 + l7, chunk = 2 * warp + (q & 1);
-        ldsm_x4_trans(pt + m * 128 + ((chunk ^ (m & 7)) << 4), a0, a1, a2, a3);
-      }
-#pragma unroll
-      for (int np = 0; np < NT / 2; ++np) {
-        uint32_t b0, b1, b2, b3;  // G: (m 0-7, tile 2np), (m 8-15, tile 2np), (m 0-7, tile 2np+1), (m 8-15, ...)
-        const int m = 16 * ks + (q & 1) * 8 + l7, j = (2 * np + (q >> 1)) * 8;
-        ldsm_x4_trans(narrow_addr<NT>(gt, m, j), b0, b1, b2, b3);
-        mma_bf16_16816(acc[2 * np], a0, a1, a2, a3, b0, b1);
-        mma_bf16_16816(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
-      }
-    }
     __syncwarp();
-    if (lane == 0) mbar_arrive(empty0 + 8u * s);
-  }
-
-  const int g = lane >> 2, t = lane & 3;
-  float* dst = partial + static_cast<int64_t>(split) * R * C;
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const int j = nt * 8 + 2 * t;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int c = c0 + 16 * warp + g + 8 * h;
-      if (c >= C) continue;
-      if (j < R) dst[static_cast<int64_t>(j) * C + c] = acc[nt][2 * h];
-      if (j + 1 < R) dst[static_cast<int64_t>(j + 1) * C + c] = acc[nt][2 * h + 1];
-    }
-  }
-}
-
-// out = bf16(scale * sum_split partial[split]), as [R, C] or transposed [C, R].
-// Thread = one column c and 8 consecutive j (blockIdx.y picks the 8): every
-// partial read is coalesced across the warp, and a transposed output row
-// segment of 8 values is one 16-byte store.
-__global__ void __launch_bounds__(64) k_coldot_reduce(const float* __restrict__ partial, int splits, int R, int C,
-                                                      float scale, int transpose, uint16_t* __restrict__ out) {
-  pdl_trigger();
-  pdl_wait();
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  const int j0 = blockIdx.y * 8;
-  if (c >= C) return;
-  const int64_t plane = static_cast<int64_t>(R) * C;
-  float acc[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-#pragma unroll 4
-  for (int sp = 0; sp < splits; ++sp) {
-    const float* src = partial + sp * plane + static_cast<int64_t>(j0) * C + c;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] += __ldcs(src + static_cast<int64_t>(j) * C);
-  }
-  if (transpose) {
-    uint4 v;
-    v.x = bf16x2_bits(scale * acc[0], scale * acc[1]);
-    v.y = bf16x2_bits(scale * acc[2], scale * acc[3]);
-    v.z = bf16x2_bits(scale * acc[4], scale * acc[5]);
-    v.w = bf16x2_bits(scale * acc[6], scale * acc[7]);
-    *reinterpret_cast<uint4*>(out + static_cast<int64_t>(c) * R + j0) = v;
   } else {
+    float acc[NT][4];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const __nv_bfloat16 h = __float2bfloat16_rn(scale * acc[j]);
-      out[static_cast<int64_t>(j0 + j) * C + c] = *reinterpret_cast<const uint16_t*>(&h);
+    for (int i = 0; i < NT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+    const int q = lane >> 3, l7 = lane & 7;
+    for (int it = 0; it < nslab; ++it) {
+      const int s = it % CL_ST;
+      if (!wait_bounded(full0 + 8u * s, (it / CL_ST) & 1, &abort_flag, status)) break;
+      const uint32_t pt = base + s * S::P_BYTES;
+      const uint32_t gt = base + S::OFF_G + s * S::G_BYTES;
+#pragma unroll
+      for (int ks = 0; ks < 2; ++ks) {
+        uint32_t a0, a1, a2, a3;  // P^T: (c 0-7, m 0-7), (c 8-15, m 0-7), (c 0-7, m 8-15), (c 8-15, m 8-15)
+        {
+          const int m = 16 * ks + (q >> 1) * 8 + l7, chunk = 2 * warp + (q & 1);
+          ldsm_x4_trans(pt + m * 128 + ((chunk ^ (m & 7)) << 4), a0, a1, a2, a3);
+        }
+#pragma unroll
+        for (int np = 0; np < NT / 2; ++np) {
+          uint32_t b0, b1, b2, b3;  // G: (m 0-7, tile 2np), (m 8-15, tile 2np), (m 0-7, tile 2np+1), (m 8-15, ...)
+          const int m = 16 * ks + (q & 1) * 8 + l7, j = (2 * np + (q >> 1)) * 8;
+          ldsm_x4_trans(narrow_addr<NT>(gt, m, j), b0, b1, b2, b3);
+          mma_bf16_16816(acc[2 * np], a0, a1, a2, a3, b0, b1);
+          mma_bf16_16816(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty0 + 8u * s);
     }
+    // this CTA's partial sums: part[c_local][j]
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int cl = 16 * warp + g + 8 * h, j = nt * 8 + 2 * t;
+        asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(part + (cl * RJ + j) * 4), "f"(acc[nt][2 * h]),
+                     "f"(acc[nt][2 * h + 1])
+                     : "memory");
+      }
   }
+  cluster_sync_all();  // every CTA's partial sums are in its shared memory
+
+  // This CTA's share of the 64 x R outputs, each the sum of the cluster's
+  // partials in rank order.  Consecutive threads take consecutive output
+  // addresses (c for [R, C], j for [C, R]).
+  const int V = 64 * R;
+  const int v0 = static_cast<int>((static_cast<int64_t>(V) * split) / nsplit);
+  const int v1 = static_cast<int>((static_cast<int64_t>(V) * (split + 1)) / nsplit);
+  for (int v = v0 + static_cast<int>(threadIdx.x); v < v1; v += blockDim.x) {
+    int cl, j;
+    if (transpose) {
+      cl = v / R;
+      j = v - cl * R;
+    } else {
+      j = v >> 6;
+      cl = v & 63;
+    }
+    const int c = c0 + cl;
+    if (c >= C) continue;
+    const uint32_t off = part + (cl * RJ + j) * 4;
+    float sum = 0.f;
+    for (uint32_t rk = 0; rk < nsplit; ++rk) {
+      float x;
+      asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(x) : "r"(mapa_shared(off, rk)) : "memory");
+      sum += x;
+    }
+    const int64_t o = transpose ? static_cast<int64_t>(c) * R + j : static_cast<int64_t>(j) * C + c;
+    out[o] = static_cast<uint16_t>(bf16x2_bits(scale * sum, 0.f));
+  }
+  cluster_sync_all();  // peers keep their shared memory until every read is done
 }
 
 int nt_for(int R) { return R <= 16 ? 2 : R <= 32 ? 4 : 8; }
 
-int coldot_splits(int64_t M, int64_t C) {
-  const int64_t col_tiles = (C + 63) / 64;
-  int64_t s = (3 * 148 + col_tiles - 1) / col_tiles;  // ~3 CTAs per SM
-  s = std::max<int64_t>(1, std::min<int64_t>(s, (M + 255) / 256));
-  return static_cast<int>(s);
+// Token splits per column tile: one cluster of up to CL_SPLIT_MAX CTAs, at
+// least 256 tokens each.
+int cols_splits(int64_t M) {
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(CL_SPLIT_MAX, (M + 255) / 256)));
 }
 
 template <int NT, bool QT>
@@ -435,8 +436,8 @@ cudaError_t rows_dispatch(const uint16_t* P, const uint16_t* Q, int64_t M, int64
 }
 
 template <int NT>
-cudaError_t cols_launch(const uint16_t* G, const uint16_t* P, int64_t M, int64_t C, int R, int splits,
-                        int rows_per_split, float* partial, cudaStream_t st, bool pdl) {
+cudaError_t cols_launch(const uint16_t* G, const uint16_t* P, int64_t M, int64_t C, int R, float scale,
+                        int transpose, uint16_t* out, cudaStream_t st, bool pdl) {
   using S = ColsSmem<NT>;
   CUtensorMap tmP, tmG;
   const auto BF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -445,9 +446,25 @@ cudaError_t cols_launch(const uint16_t* G, const uint16_t* P, int64_t M, int64_t
   if (!ok) return cudaErrorInvalidValue;
   cudaError_t e = smem_limit_once<k_cols<NT>>(S::BYTES);
   if (e != cudaSuccess) return e;
-  const dim3 grid(static_cast<unsigned>((C + 63) / 64), static_cast<unsigned>(splits));
-  return launch_ex(k_cols<NT>, grid, dim3(160), S::BYTES, st, pdl, tmP, tmG, int(M), int(C), R, rows_per_split,
-                   partial, device_status_ptr());
+  const int splits = cols_splits(M);
+  // token ranges are whole 32-token slabs, so a slab never straddles two splits
+  const int rows_per_split = static_cast<int>(((M + splits - 1) / splits + 31) / 32 * 32);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((C + 63) / 64 * splits), 1, 1);
+  cfg.blockDim = dim3(160, 1, 1);
+  cfg.dynamicSmemBytes = S::BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(splits);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, k_cols<NT>, tmP, tmG, int(M), int(C), R, rows_per_split, scale, transpose, out,
+                            device_status_ptr());
 }
 
 }  // namespace
@@ -473,31 +490,14 @@ cudaError_t launch_rowdot_qt(const uint16_t* P, const uint16_t* Qt, int64_t M, i
   return rows_dispatch<true>(P, Qt, M, Kc, R, sa, out16a, sb, out16b, out32, st, pdl);
 }
 
-size_t coldot_partial_floats(int64_t M, int64_t C, int R) {
-  return static_cast<size_t>(coldot_splits(M, C)) * static_cast<size_t>(R) * static_cast<size_t>(C);
-}
-
 cudaError_t launch_coldot(const uint16_t* G, const uint16_t* P, int64_t M, int64_t C, int R, float scale,
-                          int transpose, float* partial, uint16_t* out, cudaStream_t st, bool pdl) {
-  const int splits = coldot_splits(M, C);
-  // token ranges are whole 32-token slabs, so a slab never straddles two splits
-  const int rows_per_split = static_cast<int>(((M + splits - 1) / splits + 31) / 32 * 32);
-  cudaError_t e = cudaSuccess;
-  if (M > 0) {
-    switch (nt_for(R)) {
-      case 2: e = cols_launch<2>(G, P, M, C, R, splits, rows_per_split, partial, st, pdl); break;
-      case 4: e = cols_launch<4>(G, P, M, C, R, splits, rows_per_split, partial, st, pdl); break;
-      default: e = cols_launch<8>(G, P, M, C, R, splits, rows_per_split, partial, st, pdl); break;
-    }
-  } else {
-    e = cudaMemsetAsync(partial, 0, sizeof(float) * R * C, st);
+                          int transpose, uint16_t* out, cudaStream_t st, bool pdl) {
+  if (M == 0) return cudaMemsetAsync(out, 0, sizeof(uint16_t) * static_cast<size_t>(R) * C, st);
+  switch (nt_for(R)) {
+    case 2: return cols_launch<2>(G, P, M, C, R, scale, transpose, out, st, pdl);
+    case 4: return cols_launch<4>(G, P, M, C, R, scale, transpose, out, st, pdl);
+    default: return cols_launch<8>(G, P, M, C, R, scale, transpose, out, st, pdl);
   }
-  if (e != cudaSuccess) return e;
-  const int sp = M > 0 ? splits : 1;
-  const dim3 rgrid(static_cast<unsigned>((C + 63) / 64), static_cast<unsigned>(R / 8));
-  // the reduce follows the partial kernel directly (or a memset when M == 0)
-  return launch_ex(k_coldot_reduce, rgrid, dim3(64), 0, st, M > 0, static_cast<const float*>(partial), sp, R,
-                   int(C), scale, transpose, out);
 }
 
 }  // namespace qn

@@ -98,7 +98,6 @@ FwdWorkspace fwd_layout(void* ws, int64_t M, int r) {
 struct BwdWorkspace {
   uint16_t* dH16;   // bf16(scale * dY B) [M, r]
   uint16_t* H16;    // bf16(X A^T) [M, r] when recomputed
-  float* partial;   // split partial sums of the column reductions
   size_t bytes;
 };
 BwdWorkspace bwd_layout(void* ws, int64_t M, int64_t N, int64_t K, int r) {
@@ -112,8 +111,6 @@ BwdWorkspace bwd_layout(void* ws, int64_t M, int64_t N, int64_t K, int r) {
   };
   w.dH16 = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(M) * r * 2));
   w.H16 = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(M) * r * 2));
-  const size_t pf = std::max(coldot_partial_floats(M, K, r), coldot_partial_floats(M, N, r));
-  w.partial = reinterpret_cast<float*>(take(std::max<size_t>(pf, static_cast<size_t>(r) * std::max(N, K)) * 4));
   w.bytes = off;
   return w;
 }
@@ -301,8 +298,8 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* absmax_q, const float*
     Huse = w.H16;
   }
   // dA = dH^T X ;  dB = scale * dY^T H
-  if (e == cudaSuccess) e = launch_coldot(w.dH16, X, M, K, r, 1.0f, 0, w.partial, dA, s, true);
-  if (e == cudaSuccess) e = launch_coldot(Huse, dY, M, N, r, scale, 1, w.partial, dB, s, true);
+  if (e == cudaSuccess) e = launch_coldot(w.dH16, X, M, K, r, 1.0f, 0, dA, s, true);
+  if (e == cudaSuccess) e = launch_coldot(Huse, dY, M, N, r, scale, 1, dB, s, true);
   // dX = dY deq(W) + dH A
   if (e == cudaSuccess && dX) {
     GemmArgs a{};

@@ -68,10 +68,10 @@ cudaError_t launch_rowdot(const uint16_t* P, const uint16_t* Q, int64_t M, int64
                           bool pdl = false);
 // out[j, c] = sum_m G[m, j] P[m, c] over all m (G bf16 [M, R], P bf16 [M, C]),
 // written as bf16(scale * out) either [R, C] (transpose = 0) or [C, R]
-// (transpose = 1).  partial: fp32 scratch of coldot_partial_floats(...) floats.
-size_t coldot_partial_floats(int64_t M, int64_t C, int R);
+// (transpose = 1).  One kernel; the token splits meet in a thread-block
+// cluster, so no scratch is needed.
 cudaError_t launch_coldot(const uint16_t* G, const uint16_t* P, int64_t M, int64_t C, int R, float scale,
-                          int transpose, float* partial, uint16_t* out, cudaStream_t st, bool pdl = false);
+                          int transpose, uint16_t* out, cudaStream_t st, bool pdl = false);
 // The same with Q given transposed, Qt bf16 [Kc, R] (lora_B read in place).
 cudaError_t launch_rowdot_qt(const uint16_t* P, const uint16_t* Qt, int64_t M, int64_t Kc, int R, float sa,
                              uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st,
