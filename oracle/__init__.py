@@ -114,15 +114,17 @@ def nf4_sizes(N: int, K: int, block: int = 64, dq_block: int = 256):
 
 def nf4_quantize(W: np.ndarray, block: int = 64, dq_block: int = 256):
     """W fp32 [N, K] -> (codes u8 [N*K/2], absmax_q u8 [N*K/block],
-    dq_scale f32 [groups], absmax f32 [N*K/block] (exact first-level scales))."""
+    dq_scale f32 [groups], absmax f32 [N*K/block] (exact first-level scales)).
+    dq_block = 0: no double quantization; absmax_q is empty and dq_scale holds
+    the exact fp32 absmax of every block."""
     lib = _load()
     W = _c(W, np.float32)
     N, K = W.shape
     cb, ab, dc = nf4_sizes(N, K, block, dq_block)
     codes = np.zeros(cb, np.uint8)
-    aq = np.zeros(ab, np.uint8)
+    aq = np.zeros(max(ab, 1), np.uint8)[:ab]
     dq = np.zeros(dc, np.float32)
-    a = np.zeros(ab, np.float32)
+    a = np.zeros(N * K // block, np.float32)
     _check(lib.or_nf4_quantize(_p(W), N, K, block, dq_block, _p(codes), _p(aq), _p(dq), _p(a)),
            "quantize")
     return codes, aq, dq, a

@@ -141,14 +141,17 @@ int or_nf4_codebook(double* levels64, float* levels32, float* mids32) {
 
 /* codes: two 4-bit codes per byte; absmax_q: one byte per block; dq_scale:
  * one fp32 per group of dq_block consecutive blocks (last group may be short). */
+/* dq_block == 0 means no double quantization: the exact fp32 absmax of every
+ * block is stored (dq_count = number of blocks, in the fp32 array) and the
+ * 8-bit array is empty. */
 int or_nf4_sizes(int64_t N, int64_t K, int block, int dq_block,
                  int64_t* codes_bytes, int64_t* absmax_bytes, int64_t* dq_count) {
-    if (N < 0 || K < 0 || block <= 0 || dq_block <= 0) return OR_ERR_ARG;
+    if (N < 0 || K < 0 || block <= 0 || dq_block < 0) return OR_ERR_ARG;
     if (block % 2 || K % block) return OR_ERR_SHAPE;
     int64_t numel = N * K, nblocks = numel / block;
     if (codes_bytes) *codes_bytes = numel / 2;
-    if (absmax_bytes) *absmax_bytes = nblocks;
-    if (dq_count) *dq_count = (nblocks + dq_block - 1) / dq_block;
+    if (absmax_bytes) *absmax_bytes = dq_block ? nblocks : 0;
+    if (dq_count) *dq_count = dq_block ? (nblocks + dq_block - 1) / dq_block : nblocks;
     return OR_OK;
 }
 
@@ -164,15 +167,17 @@ int or_nf4_sizes(int64_t N, int64_t K, int block, int dq_block,
  *  a4: groups of dq_block consecutive blocks; c2 = max a_b over the group;
  *      s2 = fl32(c2 / 255) (0 when c2 == 0); q_b = min(255, rne(fl32(a_b/s2)))
  *      (0 when s2 == 0): an unsigned linear 8-bit code of the non-negative
- *      absmax values.
+ *      absmax values.  With dq_block == 0 (no double quantization) dq_scale
+ *      receives a_b itself and absmax_q is not used.
  * absmax_out (nullable) receives the exact a_b. */
 int or_nf4_quantize(const float* W, int64_t N, int64_t K, int block, int dq_block,
                     uint8_t* codes, uint8_t* absmax_q, float* dq_scale, float* absmax_out) {
-    if (!W || !codes || !absmax_q || !dq_scale) return OR_ERR_ARG;
+    if (!W || !codes || (dq_block && !absmax_q) || !dq_scale) return OR_ERR_ARG;
     int64_t cb, ab, dc;
     int st = or_nf4_sizes(N, K, block, dq_block, &cb, &ab, &dc);
     if (st) return st;
-    const int64_t numel = N * K, nblocks = ab;
+    const int64_t numel = N * K, nblocks = numel / block;
+    (void)ab;
     for (int64_t i = 0; i < numel; ++i)
         if (!isfinite(W[i])) return OR_ERR_NONFINITE;
 
@@ -204,6 +209,10 @@ int or_nf4_quantize(const float* W, int64_t N, int64_t K, int block, int dq_bloc
         }
     }
 
+    if (dq_block == 0) {
+        for (int64_t b = 0; b < nblocks; ++b) dq_scale[b] = a[b];
+        dc = 0;  /* no groups */
+    }
     for (int64_t g = 0; g < dc; ++g) {
         int64_t b0 = g * dq_block, b1 = b0 + dq_block;
         if (b1 > nblocks) b1 = nblocks;
@@ -231,7 +240,7 @@ int or_nf4_quantize(const float* W, int64_t N, int64_t K, int block, int dq_bloc
 int or_nf4_dequantize(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale,
                       int64_t N, int64_t K, int block, int dq_block,
                       uint16_t* out_bf16, float* out_f32) {
-    if (!codes || !absmax_q || !dq_scale || (!out_bf16 && !out_f32)) return OR_ERR_ARG;
+    if (!codes || (dq_block && !absmax_q) || !dq_scale || (!out_bf16 && !out_f32)) return OR_ERR_ARG;
     int64_t cb, ab, dc;
     int st = or_nf4_sizes(N, K, block, dq_block, &cb, &ab, &dc);
     if (st) return st;
@@ -240,10 +249,11 @@ int or_nf4_dequantize(const uint8_t* codes, const uint8_t* absmax_q, const float
     const int64_t numel = N * K;
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < numel; ++i) {
-        int64_t b = i / block, g = b / dq_block;
+        int64_t b = i / block;
         uint8_t byte = codes[i / 2];
         int code = (i % 2 == 0) ? (byte & 0xf) : (byte >> 4);
-        float ap = r32((double)absmax_q[b] * (double)dq_scale[g]);
+        /* the block scale: q_b * s2 of its group, or the stored fp32 absmax */
+        float ap = dq_block ? r32((double)absmax_q[b] * (double)dq_scale[b / dq_block]) : dq_scale[b];
         float w = r32((double)L[code] * (double)ap);
         uint16_t h = f32_to_bf16_rne(w);
         if (out_bf16) out_bf16[i] = h;

@@ -311,3 +311,77 @@ def test_zero_adapter_B_gives_base_output_and_zero_dA(oracle):
     _, dA, dB, _ = oracle.linear_bwd(_bits(p["X"]), _bits(p["dY"]), Wp, _bits(p["A"]), B0, p["scale"])
     assert np.all(dA == 0.0)
     assert np.any(dB != 0.0)
+
+
+# --------------------------------------- other block sizes, double quant off
+
+
+@pytest.mark.parametrize("block", [32, 64, 128, 256])
+@pytest.mark.parametrize("dq_block", [256, 0])
+def test_levels_round_trip_any_block(oracle, block, dq_block):
+    """Blocks made of the levels times a power-of-two absmax encode to the level
+    indices whatever the block size; with double quantization off the stored
+    scale is that absmax exactly and each weight dequantizes to its own bf16
+    rounding."""
+    _, l32, _ = oracle.nf4_codebook()
+    rows = 3
+    idx = (np.arange(rows * block) * 7 + 3) % 16
+    idx[::block] = 15  # each block holds level 1 (its absmax) once
+    e = np.repeat(np.array([-6, 0, 5])[: rows], block)
+    W = (l32[idx] * (2.0 ** e)).astype(np.float32).reshape(rows, block)
+    codes, aq, dq, absmax = oracle.nf4_quantize(W, block=block, dq_block=dq_block)
+    assert np.array_equal(unpack(codes), idx)
+    assert np.array_equal(absmax, (2.0 ** np.array([-6, 0, 5])).astype(np.float32))
+    if dq_block == 0:
+        assert aq.size == 0 and np.array_equal(dq, absmax)
+        w16, w32 = oracle.nf4_dequantize(codes, aq, dq, rows, block, block=block, dq_block=0)
+        # L * 2^e is exact in fp32, so the dequantized value is bf16(W) itself
+        assert np.array_equal(w32, torch.from_numpy(W).to(torch.bfloat16).float().numpy())
+    else:
+        assert aq.size == rows
+
+
+@pytest.mark.parametrize("block", [32, 128, 256])
+def test_brute_force_nearest_level_any_block(oracle, block):
+    """The nearest-level rule holds with the block's own absmax for every block
+    size (exhaustive fp64 search on t = fl32(x / a))."""
+    W = wl.draw_weight(wl.generator(300 + block), 6, 512, 0.02, 0.05).numpy()
+    _, l32, _ = oracle.nf4_codebook()
+    codes, _, _, absmax = oracle.nf4_quantize(W, block=block)
+    blocks = W.reshape(-1, block)
+    a = np.abs(blocks).max(axis=1)
+    assert np.array_equal(a, absmax)
+    t = (blocks / a[:, None]).astype(np.float32).reshape(-1)
+    brute = np.argmin(np.abs(t.astype(np.float64)[:, None] - l32.astype(np.float64)[None, :]), axis=1)
+    assert np.array_equal(brute, unpack(codes))
+
+
+def test_double_quant_off_stores_exact_scales(oracle):
+    """Without double quantization the block scale is the exact absmax: the
+    element of largest magnitude dequantizes to +-bf16(absmax), and the whole
+    block's error is bounded by half the widest level gap times absmax plus
+    the bf16 rounding -- with no second-level term."""
+    W = wl.draw_weight(wl.generator(77), 8, 256, 0.02, 0.05).numpy()
+    _, l32, _ = oracle.nf4_codebook()
+    codes, aq, dq, a = oracle.nf4_quantize(W, block=64, dq_block=0)
+    assert aq.size == 0 and np.array_equal(dq, a)
+    w16, w32 = oracle.nf4_dequantize(codes, aq, dq, 8, 256, block=64, dq_block=0)
+    blocks = W.reshape(-1, 64)
+    i = np.abs(blocks).argmax(axis=1)
+    top = w32.reshape(-1, 64)[np.arange(blocks.shape[0]), i]
+    want = torch.from_numpy(np.sign(blocks[np.arange(blocks.shape[0]), i]) * a).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(top, want)
+    half_gap = np.max(np.diff(l32.astype(np.float64))) / 2
+    bound = np.repeat(a.astype(np.float64), 64).reshape(8, 256) * half_gap + np.abs(W) * 2 ** -8 + 1e-30
+    assert np.all(np.abs(w32.astype(np.float64) - W) <= bound)
+
+
+@pytest.mark.parametrize("block,dq_block,bits", [(64, 256, 4 + 8 / 64 + 32 / (64 * 256)), (64, 0, 4.5),
+                                                  (32, 0, 5.0), (128, 256, 4 + 8 / 128 + 32 / (128 * 256)),
+                                                  (256, 0, 4.125)])
+def test_format_bits_per_parameter(oracle, block, dq_block, bits):
+    """Storage per weight: 4 code bits + the block's scale (8 bits, or 32 bits
+    without double quantization) / block + 32 bits per group of 256 blocks."""
+    N, K = 64, 4096
+    cb, ab, dc = oracle.nf4_sizes(N, K, block, dq_block)
+    assert (8 * (cb + ab) + 32 * dc) / (N * K) == pytest.approx(bits, rel=1e-12)
