@@ -127,11 +127,20 @@ def nf4_codebook():
 
 
 class NF4Weight:
-    """The three buffers of a quantized [N, K] weight (device tensors)."""
+    """The three buffers of a quantized [N, K] weight (device tensors) and its
+    format: `block` weights per absmax, `dq_block` blocks per second-level
+    scale (0: no double quantization; dq_scale then holds each block's fp32
+    absmax and absmax_q is empty)."""
 
-    def __init__(self, codes, absmax_q, dq_scale, N, K):
+    def __init__(self, codes, absmax_q, dq_scale, N, K, block=BLOCK, dq_block=DQ_BLOCK):
         self.codes, self.absmax_q, self.dq_scale = codes, absmax_q, dq_scale
         self.N, self.K = int(N), int(K)
+        self.block, self.dq_block = int(block), int(dq_block)
+
+    def _layer_format(self):
+        if (self.block, self.dq_block) != (BLOCK, DQ_BLOCK):
+            raise QloraError(-7, f"the layer entry points read the default NF4 format "
+                                 f"(block {BLOCK}, dq_block {DQ_BLOCK}), not ({self.block}, {self.dq_block})")
 
     @property
     def nbytes(self):
@@ -146,17 +155,17 @@ def nf4_quantize(W: torch.Tensor, block: int = BLOCK, dq_block: int = DQ_BLOCK, 
     codes = torch.empty(cb, dtype=torch.uint8, device=dev)
     absmax_q = torch.empty(ab, dtype=torch.uint8, device=dev)
     dq_scale = torch.empty(db // 4, dtype=torch.float32, device=dev)
-    _check(lib().nf4_quantize(_ptr(W), N, K, block, dq_block, _ptr(codes), _ptr(absmax_q), _ptr(dq_scale),
-                              _stream(stream)), "nf4_quantize")
-    return NF4Weight(codes, absmax_q, dq_scale, N, K)
+    _check(lib().nf4_quantize(_ptr(W), N, K, block, dq_block, _ptr(codes), _ptr(absmax_q) if ab else None,
+                              _ptr(dq_scale), _stream(stream)), "nf4_quantize")
+    return NF4Weight(codes, absmax_q, dq_scale, N, K, block, dq_block)
 
 
 def nf4_dequantize(w: NF4Weight, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     if out is None:
         out = torch.empty(w.N, w.K, dtype=torch.bfloat16, device=w.codes.device)
     _req(out, torch.bfloat16, "out", (w.N, w.K))
-    _check(lib().nf4_dequantize(_ptr(w.codes), _ptr(w.absmax_q), _ptr(w.dq_scale), w.N, w.K, BLOCK, DQ_BLOCK,
-                                _ptr(out), _stream(stream)), "nf4_dequantize")
+    _check(lib().nf4_dequantize(_ptr(w.codes), _ptr(w.absmax_q) if w.absmax_q.numel() else None, _ptr(w.dq_scale),
+                                w.N, w.K, w.block, w.dq_block, _ptr(out), _stream(stream)), "nf4_dequantize")
     return out
 
 
@@ -182,6 +191,7 @@ def qlora_linear_fwd(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Te
                      save_h: bool = True, out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
                      stream=None):
     """Y = X deq(W)^T + scale (X A^T) B^T.  Returns (Y, H) with H = X A^T (bf16) or None."""
+    w._layer_format()
     M = X.shape[0]
     r = A.shape[0]
     _req(X, torch.bfloat16, "X", (M, w.K))
@@ -203,6 +213,7 @@ def qlora_linear_bwd(w: NF4Weight, X: torch.Tensor, dY: torch.Tensor, A: torch.T
                      scale: float, H: torch.Tensor | None = None, want_dx: bool = True,
                      outs=None, workspace: torch.Tensor | None = None, stream=None):
     """Returns (dX or None, dA, dB) for Y = X deq(W)^T + scale (X A^T) B^T."""
+    w._layer_format()
     M = X.shape[0]
     r = A.shape[0]
     _req(X, torch.bfloat16, "X", (M, w.K))
@@ -229,6 +240,7 @@ def qlora_linear_fwd_noalloc(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: 
                              save_h: bool = True, out: torch.Tensor | None = None, stream=None):
     """qlora_linear_fwd without a workspace: the library's fixed device scratch
     is used instead (M * r <= QLORA_NOALLOC_MAX_TOKENS_X_RANK).  Returns (Y, H)."""
+    w._layer_format()
     M = X.shape[0]
     r = A.shape[0]
     _req(X, torch.bfloat16, "X", (M, w.K))

@@ -158,12 +158,13 @@ int qlora_version(void) { return (1 << 16) | 0; }
 int nf4_quantized_sizes(int64_t N, int64_t K, int block, int dq_block, size_t* codes_bytes, size_t* absmax_bytes,
                         size_t* dq_scale_bytes) {
   if (N < 0 || K < 0 || !codes_bytes || !absmax_bytes || !dq_scale_bytes) return QLORA_ERR_ARG;
-  if (block != 64 || dq_block != 256) return QLORA_ERR_UNSUPPORTED;
+  if ((block != 32 && block != 64 && block != 128 && block != 256) || (dq_block != 256 && dq_block != 0))
+    return QLORA_ERR_UNSUPPORTED;
   if (K % block) return QLORA_ERR_SHAPE;
   const int64_t numel = N * K, nblocks = numel / block;
   *codes_bytes = static_cast<size_t>(numel / 2);
-  *absmax_bytes = static_cast<size_t>(nblocks);
-  *dq_scale_bytes = static_cast<size_t>((nblocks + dq_block - 1) / dq_block) * 4;
+  *absmax_bytes = dq_block ? static_cast<size_t>(nblocks) : 0;
+  *dq_scale_bytes = static_cast<size_t>(dq_block ? (nblocks + dq_block - 1) / dq_block : nblocks) * 4;
   return QLORA_OK;
 }
 
@@ -179,14 +180,14 @@ int nf4_quantize(const float* W, int64_t N, int64_t K, int block, int dq_block, 
   int st = nf4_quantized_sizes(N, K, block, dq_block, &cb, &ab, &db);
   if (st) return st;
   if (N * K == 0) return QLORA_OK;
-  if (!W || !codes || !absmax_q || !dq_scale) return QLORA_ERR_ARG;
+  if (!W || !codes || (dq_block && !absmax_q) || !dq_scale) return QLORA_ERR_ARG;
   if (!aligned(W, 16) || !aligned(codes, 4)) return QLORA_ERR_SHAPE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   std::lock_guard<std::mutex> lock(g_quantize_mutex);
   int* flag = device_nonfinite_ptr();
   if (!flag) return cuda_status(cudaErrorInvalidSymbol);
   cudaError_t e = cudaMemsetAsync(flag, 0, sizeof(int), s);
-  if (e == cudaSuccess) e = launch_quantize(W, N * K, codes, absmax_q, dq_scale, flag, s);
+  if (e == cudaSuccess) e = launch_quantize(W, N * K, block, dq_block, codes, absmax_q, dq_scale, flag, s);
   int host_flag = 0;
   if (e == cudaSuccess) e = cudaMemcpyAsync(&host_flag, flag, sizeof(int), cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
@@ -200,9 +201,10 @@ int nf4_dequantize(const uint8_t* codes, const uint8_t* absmax_q, const float* d
   int st = nf4_quantized_sizes(N, K, block, dq_block, &cb, &ab, &db);
   if (st) return st;
   if (N * K == 0) return QLORA_OK;
-  if (!codes || !absmax_q || !dq_scale || !W_out) return QLORA_ERR_ARG;
+  if (!codes || (dq_block && !absmax_q) || !dq_scale || !W_out) return QLORA_ERR_ARG;
   if (!aligned(codes, 16) || !aligned(W_out, 16)) return QLORA_ERR_SHAPE;
-  return cuda_status(launch_dequantize(codes, absmax_q, dq_scale, N * K, W_out, static_cast<cudaStream_t>(stream)));
+  return cuda_status(
+      launch_dequantize(codes, absmax_q, dq_scale, N * K, block, dq_block, W_out, static_cast<cudaStream_t>(stream)));
 }
 
 int qlora_linear_fwd_workspace(int64_t M, int64_t N, int64_t K, int r, size_t* bytes) {

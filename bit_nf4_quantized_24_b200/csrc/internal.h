@@ -31,10 +31,12 @@ int* device_status_ptr();      // device address of the status word
 int* device_nonfinite_ptr();   // device address of the non-finite flag
 
 // ----- quantize / dequantize (HBM-bound)
-cudaError_t launch_quantize(const float* W, int64_t numel, uint8_t* codes, uint8_t* absmax_q,
-                            float* dq_scale, int* nonfinite, cudaStream_t st);
+// block in {32, 64, 128, 256}; dq_block 256 or 0 (no double quantization:
+// dq_scale then holds each block's fp32 absmax and absmax_q is unused).
+cudaError_t launch_quantize(const float* W, int64_t numel, int block, int dq_block, uint8_t* codes,
+                            uint8_t* absmax_q, float* dq_scale, int* nonfinite, cudaStream_t st);
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale,
-                              int64_t numel, uint16_t* out, cudaStream_t st);
+                              int64_t numel, int block, int dq_block, uint16_t* out, cudaStream_t st);
 
 // ----- fused dequant-GEMM on tcgen05 (tensor cores)
 // mode 0 (forward):  Y[M,N]  = X[M,K]  deq(W)^T + Ht[M,r] Bt^T, Bt = lora_B [N,r]

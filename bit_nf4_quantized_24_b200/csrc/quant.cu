@@ -15,8 +15,7 @@ namespace qn {
 
 namespace {
 
-constexpr int kBlock = 64;
-constexpr int kGroup = 256;  // blocks per double-quant group
+constexpr int kGroup = 256;  // blocks per double-quant group (and per quantize CTA)
 
 // Code of t = fl32(w / a) in [-1, 1]: the number of midpoints strictly below
 // t.  t is placed exactly on a grid of 129 cells of width 1/64 (cell j holds
@@ -51,17 +50,23 @@ __device__ __forceinline__ float div_by_absmax(float w, float a, float r) {
   return __fmaf_rn(e, r, q0);
 }
 
-// One CTA per double-quant group (256 blocks = 16384 weights, 64 KB of fp32).
-// A warp covers two blocks per step: 16 lanes per block, one float4 per lane.
-// Four steps' loads are issued before any is used, to keep HBM busy.
+// One CTA per group of 256 blocks (the double-quant group).  A block of B
+// weights is spread over LP = min(32, B / 4) lanes, F = B / (4 LP) float4s per
+// lane; a warp covers 32 / LP blocks per step, and four steps' loads are
+// issued before any is used, to keep HBM busy.  DQ: double quantization of the
+// group's absmax values (else each block's fp32 absmax is stored as is).
+template <int B, bool DQ>
 __global__ void __launch_bounds__(256) k_quantize(const float* __restrict__ W, int64_t nblocks, Nf4Mids mids,
                                                   uint8_t* __restrict__ codes, uint8_t* __restrict__ absmax_q,
                                                   float* __restrict__ dq_scale, int* nonfinite) {
+  constexpr int LP = B / 4 < 32 ? B / 4 : 32;
+  constexpr int F = B / (4 * LP);
+  constexpr int BPW = 32 / LP;  // blocks per warp step
   __shared__ Cell s_cell[kCells];
   __shared__ float s_amax[kGroup];
   __shared__ float s_red[8];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int half = lane >> 4, sl = lane & 15;
+  const int sub = lane / LP, sl = lane % LP;
   const int64_t g = blockIdx.x;
   const int64_t b0 = g * kGroup;
   const int64_t rem = nblocks - b0;
@@ -78,45 +83,66 @@ __global__ void __launch_bounds__(256) k_quantize(const float* __restrict__ W, i
   }
   __syncthreads();
 
-  const int npairs = (nb + 1) >> 1;
+  const int nsteps = (nb + BPW - 1) / BPW;
   float nan_probe = 0.0f;  // becomes NaN if any weight is NaN or infinite (x * 0)
-  for (int p0 = warp; p0 < npairs; p0 += 32) {
-    float4 x[4];
+  for (int p0 = warp; p0 < nsteps; p0 += 32) {
+    float4 x[4][F];
     bool ok[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int i = 2 * (p0 + 8 * u) + half;
-      ok[u] = (p0 + 8 * u < npairs) && (i < nb);
-      x[u] = ok[u] ? __ldcs(reinterpret_cast<const float4*>(W + (b0 + i) * kBlock) + sl)
-                   : make_float4(0.f, 0.f, 0.f, 0.f);
+      const int i = BPW * (p0 + 8 * u) + sub;
+      ok[u] = (p0 + 8 * u < nsteps) && (i < nb);
+#pragma unroll
+      for (int f = 0; f < F; ++f)
+        x[u][f] = ok[u] ? __ldcs(reinterpret_cast<const float4*>(W + (b0 + i) * B) + f * LP + sl)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      if (p0 + 8 * u >= npairs) break;  // warp-uniform
-      const int i = 2 * (p0 + 8 * u) + half;
-      nan_probe = __fmaf_rn(x[u].x, 0.0f, __fmaf_rn(x[u].y, 0.0f, __fmaf_rn(x[u].z, 0.0f, __fmaf_rn(x[u].w, 0.0f, nan_probe))));
-      float m = fmaxf(fmaxf(fabsf(x[u].x), fabsf(x[u].y)), fmaxf(fabsf(x[u].z), fabsf(x[u].w)));
+      if (p0 + 8 * u >= nsteps) break;  // warp-uniform
+      const int i = BPW * (p0 + 8 * u) + sub;
+      float m = 0.0f;
 #pragma unroll
-      for (int off = 8; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      for (int f = 0; f < F; ++f) {
+        const float4 v = x[u][f];
+        nan_probe = __fmaf_rn(v.x, 0.0f, __fmaf_rn(v.y, 0.0f, __fmaf_rn(v.z, 0.0f, __fmaf_rn(v.w, 0.0f, nan_probe))));
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+      }
+#pragma unroll
+      for (int off = LP / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
       if (ok[u]) {
-        uint32_t c;
-        if (m == 0.0f) {
-          c = 0x7777u;  // an all-zero block encodes the zero level
-        } else if (m >= 0x1p-100f && m <= 0x1p100f) {
-          const float r = __frcp_rn(m);
-          c = nf4_code(div_by_absmax(x[u].x, m, r), s_cell) | (nf4_code(div_by_absmax(x[u].y, m, r), s_cell) << 4) |
-              (nf4_code(div_by_absmax(x[u].z, m, r), s_cell) << 8) |
-              (nf4_code(div_by_absmax(x[u].w, m, r), s_cell) << 12);
-        } else {
-          c = nf4_code(__fdiv_rn(x[u].x, m), s_cell) | (nf4_code(__fdiv_rn(x[u].y, m), s_cell) << 4) |
-              (nf4_code(__fdiv_rn(x[u].z, m), s_cell) << 8) | (nf4_code(__fdiv_rn(x[u].w, m), s_cell) << 12);
+        const bool fast = m >= 0x1p-100f && m <= 0x1p100f;
+        const float r = fast ? __frcp_rn(m) : 0.0f;
+#pragma unroll
+        for (int f = 0; f < F; ++f) {
+          const float4 v = x[u][f];
+          uint32_t c;
+          if (m == 0.0f) {
+            c = 0x7777u;  // an all-zero block encodes the zero level
+          } else if (fast) {
+            c = nf4_code(div_by_absmax(v.x, m, r), s_cell) | (nf4_code(div_by_absmax(v.y, m, r), s_cell) << 4) |
+                (nf4_code(div_by_absmax(v.z, m, r), s_cell) << 8) |
+                (nf4_code(div_by_absmax(v.w, m, r), s_cell) << 12);
+          } else {
+            c = nf4_code(__fdiv_rn(v.x, m), s_cell) | (nf4_code(__fdiv_rn(v.y, m), s_cell) << 4) |
+                (nf4_code(__fdiv_rn(v.z, m), s_cell) << 8) | (nf4_code(__fdiv_rn(v.w, m), s_cell) << 12);
+          }
+          reinterpret_cast<uint16_t*>(codes + (b0 + i) * (B / 2))[f * LP + sl] = static_cast<uint16_t>(c);
         }
-        reinterpret_cast<uint16_t*>(codes + (b0 + i) * (kBlock / 2))[sl] = static_cast<uint16_t>(c);
-        if (sl == 0) s_amax[i] = m;
+        if (sl == 0) {
+          if (DQ)
+            s_amax[i] = m;
+          else
+            dq_scale[b0 + i] = m;
+        }
       }
     }
   }
   const bool bad = !(nan_probe == 0.0f);
+  if (!DQ) {
+    if (__syncthreads_or(bad) && tid == 0) atomicExch(nonfinite, 1);
+    return;
+  }
   __syncthreads();
 
   // double quantization of the group's absmax values
@@ -138,61 +164,108 @@ __global__ void __launch_bounds__(256) k_quantize(const float* __restrict__ W, i
   if (__syncthreads_or(bad) && tid == 0) atomicExch(nonfinite, 1);
 }
 
-// One thread expands one 64-weight block (one register table, 32 code bytes
-// in, 128 bytes of bf16 out); a warp's 32 blocks pass through shared memory
+// One thread expands 64 consecutive weights (one register table per block
+// of B weights it touches: two for B = 32, one otherwise; 32 code bytes in,
+// 128 bytes of bf16 out); a warp's 32 x 64 weights pass through shared memory
 // (16-byte chunks XOR-swizzled by lane) so that the global stores are 512
-// contiguous bytes per instruction.
+// contiguous bytes per instruction.  DQ: block scale = absmax_q * dq_scale of
+// its group; else the stored fp32 absmax.
+template <int B, bool DQ>
 __global__ void __launch_bounds__(256) k_dequantize(const uint8_t* __restrict__ codes,
                                                     const uint8_t* __restrict__ absmax_q,
-                                                    const float* __restrict__ dq_scale, int64_t nblocks,
+                                                    const float* __restrict__ dq_scale, int64_t nchunks64,
                                                     Nf4Levels L, uint16_t* __restrict__ out) {
   __shared__ uint4 s_out[8][32 * 8];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t wb0 = (static_cast<int64_t>(blockIdx.x) * 8 + warp) * 32;  // first block of this warp
-  const int64_t b = wb0 + lane;
-  if (wb0 >= nblocks) return;  // warp-uniform
-  if (b < nblocks) {
-    const uint4 c0 = ldg_nc_v4(codes + b * 32);
-    const uint4 c1 = ldg_nc_v4(codes + b * 32 + 16);
-    const float ap = __fmul_rn(static_cast<float>(absmax_q[b]), dq_scale[b / kGroup]);
-    const Nf4Lut t = make_lut(L, ap);
+  const int64_t wc0 = (static_cast<int64_t>(blockIdx.x) * 8 + warp) * 32;  // first 64-weight chunk of this warp
+  const int64_t c = wc0 + lane;
+  if (wc0 >= nchunks64) return;  // warp-uniform
+  auto scale = [&](int64_t b) -> float {
+    return DQ ? __fmul_rn(static_cast<float>(absmax_q[b]), dq_scale[b / kGroup]) : dq_scale[b];
+  };
+  if (c < nchunks64) {
+    const uint4 c0 = ldg_nc_v4(codes + c * 32);
+    const uint4 c1 = ldg_nc_v4(codes + c * 32 + 16);
     const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+    if (B == 32) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      uint4 o;
-      deq8(w[i], t, o.x, o.y, o.z, o.w);
-      s_out[warp][lane * 8 + (i ^ (lane & 7))] = o;
+      for (int h = 0; h < 2; ++h) {
+        const Nf4Lut t = make_lut(L, scale(2 * c + h));
+#pragma unroll
+        for (int i = 4 * h; i < 4 * h + 4; ++i) {
+          uint4 o;
+          deq8(w[i], t, o.x, o.y, o.z, o.w);
+          s_out[warp][lane * 8 + (i ^ (lane & 7))] = o;
+        }
+      }
+    } else {
+      const Nf4Lut t = make_lut(L, scale(c * 64 / B));
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        uint4 o;
+        deq8(w[i], t, o.x, o.y, o.z, o.w);
+        s_out[warp][lane * 8 + (i ^ (lane & 7))] = o;
+      }
     }
   }
   __syncwarp();
-  const int64_t nchunks = (nblocks - wb0 < 32 ? nblocks - wb0 : 32) * 8;
-  uint4* dst = reinterpret_cast<uint4*>(out + wb0 * kBlock);
+  const int64_t nout = (nchunks64 - wc0 < 32 ? nchunks64 - wc0 : 32) * 8;
+  uint4* dst = reinterpret_cast<uint4*>(out + wc0 * 64);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int q = i * 32 + lane;  // chunk q of the warp's 32 x 128 bytes
-    if (q < nchunks) __stcs(dst + q, s_out[warp][(q >> 3) * 8 + ((q & 7) ^ ((q >> 3) & 7))]);
+    const int q = i * 32 + lane;  // 16-byte chunk q of the warp's 32 x 128 bytes
+    if (q < nout) __stcs(dst + q, s_out[warp][(q >> 3) * 8 + ((q & 7) ^ ((q >> 3) & 7))]);
   }
+}
+
+template <int B, bool DQ>
+cudaError_t quantize_launch(const float* W, int64_t numel, uint8_t* codes, uint8_t* absmax_q, float* dq_scale,
+                            int* nonfinite, cudaStream_t st) {
+  const int64_t nblocks = numel / B;
+  const int64_t ngroups = (nblocks + kGroup - 1) / kGroup;
+  if (ngroups == 0) return cudaSuccess;
+  k_quantize<B, DQ><<<static_cast<unsigned>(ngroups), 256, 0, st>>>(W, nblocks, host_codebook().mids, codes,
+                                                                    absmax_q, dq_scale, nonfinite);
+  return cudaGetLastError();
+}
+
+template <int B, bool DQ>
+cudaError_t dequantize_launch(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale, int64_t numel,
+                              uint16_t* out, cudaStream_t st) {
+  const int64_t nchunks = numel / 64;
+  if (nchunks == 0) return cudaSuccess;
+  const unsigned grid = static_cast<unsigned>((nchunks + 255) / 256);  // 8 warps x 32 chunks per CTA
+  k_dequantize<B, DQ><<<grid, 256, 0, st>>>(codes, absmax_q, dq_scale, nchunks, host_codebook().levels, out);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_quantize(const float* W, int64_t numel, uint8_t* codes, uint8_t* absmax_q, float* dq_scale,
-                            int* nonfinite, cudaStream_t st) {
-  const int64_t nblocks = numel / kBlock;
-  const int64_t ngroups = (nblocks + kGroup - 1) / kGroup;
-  if (ngroups == 0) return cudaSuccess;
-  k_quantize<<<static_cast<unsigned>(ngroups), 256, 0, st>>>(W, nblocks, host_codebook().mids, codes, absmax_q,
-                                                            dq_scale, nonfinite);
-  return cudaGetLastError();
+// Formats: block in {32, 64, 128, 256}; dq_block 256 (double quantization) or
+// 0 (none).  The caller has validated them.
+#define QN_CODEC_DISPATCH(FN, ...)                                                  \
+  switch (block * 2 + (dq_block ? 1 : 0)) {                                        \
+    case 64 * 2 + 1: return FN<64, true>(__VA_ARGS__);                              \
+    case 64 * 2: return FN<64, false>(__VA_ARGS__);                                 \
+    case 32 * 2 + 1: return FN<32, true>(__VA_ARGS__);                              \
+    case 32 * 2: return FN<32, false>(__VA_ARGS__);                                 \
+    case 128 * 2 + 1: return FN<128, true>(__VA_ARGS__);                            \
+    case 128 * 2: return FN<128, false>(__VA_ARGS__);                               \
+    case 256 * 2 + 1: return FN<256, true>(__VA_ARGS__);                            \
+    case 256 * 2: return FN<256, false>(__VA_ARGS__);                               \
+    default: return cudaErrorInvalidValue;                                         \
+  }
+
+cudaError_t launch_quantize(const float* W, int64_t numel, int block, int dq_block, uint8_t* codes,
+                            uint8_t* absmax_q, float* dq_scale, int* nonfinite, cudaStream_t st) {
+  QN_CODEC_DISPATCH(quantize_launch, W, numel, codes, absmax_q, dq_scale, nonfinite, st)
 }
 
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale, int64_t numel,
-                              uint16_t* out, cudaStream_t st) {
-  const int64_t nblocks = numel / kBlock;
-  if (nblocks == 0) return cudaSuccess;
-  const unsigned grid = static_cast<unsigned>((nblocks + 255) / 256);  // 8 warps x 32 blocks per CTA
-  k_dequantize<<<grid, 256, 0, st>>>(codes, absmax_q, dq_scale, nblocks, host_codebook().levels, out);
-  return cudaGetLastError();
+                              int block, int dq_block, uint16_t* out, cudaStream_t st) {
+  QN_CODEC_DISPATCH(dequantize_launch, codes, absmax_q, dq_scale, numel, out, st)
 }
+
+#undef QN_CODEC_DISPATCH
 
 }  // namespace qn

@@ -30,8 +30,13 @@
  *      dq_scale  fp32  [ceil(N*K/block/dq_block)]  second-level scale of each
  *                                group of dq_block consecutive blocks.
  *    Blocks are `block` consecutive elements of the flattened weight (they
- *    never straddle a row: K % block == 0).  This build supports
- *    block == 64 and dq_block == 256 (other values: QLORA_ERR_UNSUPPORTED).
+ *    never straddle a row: K % block == 0).  The codec entry points
+ *    (nf4_quantized_sizes, nf4_quantize, nf4_dequantize) accept block in
+ *    {32, 64, 128, 256} and dq_block 256 or 0.  dq_block == 0 turns double
+ *    quantization off: absmax_q is then empty (NULL allowed) and dq_scale holds
+ *    the exact fp32 absmax of every block ([N*K/block]).  The layer entry
+ *    points (qlora_linear_*) read the default format, block 64 with
+ *    dq_block 256.  Other values: QLORA_ERR_UNSUPPORTED.
  *  - Pointers: every tensor pointer is a DEVICE pointer of the current CUDA
  *    device unless stated otherwise; the caller owns all memory.  The library
  *    never frees or retains caller memory.
@@ -93,7 +98,8 @@ int nf4_codebook(float* levels_out);
  * a_b = max |w|; code = index of the nearest level to fl32(w / a_b) (ties at
  * a midpoint take the lower code; an all-zero block encodes the zero level).
  * Per group g of dq_block blocks: s2_g = fl32(max_b a_b / 255);
- * absmax_q[b] = min(255, round_half_even(fl32(a_b / s2_g))) (0 if s2_g == 0).
+ * absmax_q[b] = min(255, round_half_even(fl32(a_b / s2_g))) (0 if s2_g == 0);
+ * with dq_block == 0, dq_scale[b] = a_b instead.
  * W: device fp32 [N, K]; codes, absmax_q, dq_scale: device outputs sized by
  * nf4_quantized_sizes.  Synchronizes `stream` to report non-finite input:
  * returns QLORA_ERR_NONFINITE if W holds a NaN or an infinity (the outputs are
@@ -102,8 +108,9 @@ int nf4_quantize(const float* W, int64_t N, int64_t K, int block, int dq_block,
                  uint8_t* codes, uint8_t* absmax_q, float* dq_scale, void* stream);
 
 /* Dequantize NF4 to bf16 (katajob, "NF4: 4-bit NormalFloat": the block is
- * expanded to the compute dtype).  w' = bf16_rne(fl32(level[code] *
- * fl32(absmax_q[b] * dq_scale[g]))).  W_out: device bf16 [N, K].
+ * expanded to the compute dtype).  w' = bf16_rne(fl32(level[code] * a')) with
+ * a' = fl32(absmax_q[b] * dq_scale[g]) (or a' = dq_scale[b] when dq_block is
+ * 0).  W_out: device bf16 [N, K].
  * Errors: ARG, SHAPE, UNSUPPORTED, CUDA. */
 int nf4_dequantize(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale,
                    int64_t N, int64_t K, int block, int dq_block,

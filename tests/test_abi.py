@@ -43,12 +43,18 @@ def test_sizes_match_oracle_format(L, oracle):
         cb, ab, db = qb.nf4_quantized_sizes(N, K)
         ocb, oab, odc = oracle.nf4_sizes(N, K)
         assert (cb, ab, db) == (ocb, oab, 4 * odc)
+    for block in (32, 64, 128, 256):
+        for dq in (256, 0):
+            cb, ab, db = qb.nf4_quantized_sizes(7, 1024, block, dq)
+            assert (cb, ab, db) == tuple(v * (4 if k == 2 else 1)
+                                         for k, v in enumerate(oracle.nf4_sizes(7, 1024, block, dq)))
 
 
 def test_argument_errors_return_before_any_device_work(L):
     i = ctypes.c_size_t()
     assert L.nf4_quantized_sizes(4, 96, 64, 256, ctypes.byref(i), ctypes.byref(i), ctypes.byref(i)) == -2
-    assert L.nf4_quantized_sizes(4, 128, 32, 256, ctypes.byref(i), ctypes.byref(i), ctypes.byref(i)) == -7
+    assert L.nf4_quantized_sizes(4, 192, 48, 256, ctypes.byref(i), ctypes.byref(i), ctypes.byref(i)) == -7
+    assert L.nf4_quantized_sizes(4, 128, 64, 128, ctypes.byref(i), ctypes.byref(i), ctypes.byref(i)) == -7
     assert L.nf4_quantized_sizes(-1, 64, 64, 256, ctypes.byref(i), ctypes.byref(i), ctypes.byref(i)) == -1
     assert L.nf4_codebook(None) == -1
     assert L.qlora_linear_fwd_workspace(16, 64, 64, 12, ctypes.byref(i)) == -7

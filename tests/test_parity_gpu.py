@@ -42,14 +42,14 @@ def bits(t):
     return wl.bf16_bits(t.cpu())
 
 
-def quantize_both(qb, oracle, W):
+def quantize_both(qb, oracle, W, block=64, dq_block=256):
     """GPU and oracle quantization of the same fp32 weight; asserts bit-exact."""
-    q = qb.nf4_quantize(W.cuda())
-    oc, oa, od, _ = oracle.nf4_quantize(W.numpy())
+    q = qb.nf4_quantize(W.cuda(), block, dq_block)
+    oc, oa, od, _ = oracle.nf4_quantize(W.numpy(), block=block, dq_block=dq_block)
     assert np.array_equal(q.codes.cpu().numpy(), oc), "NF4 codes differ"
     assert np.array_equal(q.absmax_q.cpu().numpy(), oa), "absmax codes differ"
-    assert q.dq_scale.cpu().numpy().tobytes() == od.tobytes(), "double-quant scales differ"
-    _, Wp = oracle.nf4_dequantize(oc, oa, od, W.shape[0], W.shape[1])
+    assert q.dq_scale.cpu().numpy().tobytes() == od.tobytes(), "scales differ"
+    _, Wp = oracle.nf4_dequantize(oc, oa, od, W.shape[0], W.shape[1], block=block, dq_block=dq_block)
     return q, Wp
 
 
@@ -143,6 +143,34 @@ def test_quantize_near_midpoints_any_scale(qb, oracle):
             rows.append(r)
     W = torch.from_numpy(np.stack(rows).astype(np.float32))
     quantize_both(qb, oracle, W)
+
+
+@pytest.mark.parametrize("block", [32, 64, 128, 256])
+@pytest.mark.parametrize("dq_block", [256, 0])
+def test_codec_other_formats_bit_exact(qb, oracle, block, dq_block):
+    """Every block size with and without double quantization: codes, absmax
+    codes and scales bit-exact; the dequantized weight bit-exact.  37 rows of
+    2048 make the last group of 256 blocks ragged for every block size."""
+    N, K = 37, 2048
+    W = wl.draw_weight(wl.generator(500 + block + dq_block), N, K, 0.02, 0.02)
+    W[0, :block] = 0.0  # an all-zero block
+    W[3, :] *= 1e-30    # tiny magnitudes
+    q, Wp = quantize_both(qb, oracle, W, block, dq_block)
+    assert (q.block, q.dq_block) == (block, dq_block)
+    Wd = qb.nf4_dequantize(q)
+    o16, _ = oracle.nf4_dequantize(q.codes.cpu().numpy(), q.absmax_q.cpu().numpy(), q.dq_scale.cpu().numpy(),
+                                   N, K, block=block, dq_block=dq_block)
+    assert np.array_equal(Wd.view(torch.int16).cpu().numpy().view(np.uint16), o16)
+
+
+def test_layer_rejects_other_formats(qb):
+    q = qb.nf4_quantize(torch.randn(64, 256, device="cuda") * 0.02, 128, 0)
+    X = torch.randn(32, 256, device="cuda").bfloat16()
+    A = torch.randn(16, 256, device="cuda").bfloat16()
+    B = torch.randn(64, 16, device="cuda").bfloat16()
+    with pytest.raises(qb.QloraError) as ei:
+        qb.qlora_linear_fwd(q, X, A, B, 2.0)
+    assert ei.value.status == -7
 
 
 def test_quantize_rejects_nonfinite(qb):
