@@ -61,6 +61,9 @@ def lib():
     L.qlora_linear_fwd.argtypes = [P, P, P, i64, i64, P, i64, P, P, i32, f32, P, P, P, sz, P]
     L.qlora_linear_bwd.argtypes = [P, P, P, i64, i64, P, P, i64, P, P, i32, f32, P, P, P, P, P, sz, P]
     L.qlora_linear_fwd_noalloc.argtypes = [P, P, P, i64, i64, P, i64, P, P, i32, f32, P, P, P]
+    L.qlora_linear_fwd_fmt.argtypes = [P, P, P, i32, i32, i64, i64, P, i64, P, P, i32, f32, P, P, P, sz, P]
+    L.qlora_linear_bwd_fmt.argtypes = [P, P, P, i32, i32, i64, i64, P, P, i64, P, P, i32, f32, P, P, P, P, P, sz,
+                                       P]
     L.qlora_device_status.restype = i32
     L.qlora_trace_gemm_events.argtypes = [P, i32]
     L.qlora_trace_gemm_count.restype = i32
@@ -139,7 +142,7 @@ class NF4Weight:
 
     def _layer_format(self):
         if (self.block, self.dq_block) != (BLOCK, DQ_BLOCK):
-            raise QloraError(-7, f"the layer entry points read the default NF4 format "
+            raise QloraError(-7, f"this entry point reads the default NF4 format "
                                  f"(block {BLOCK}, dq_block {DQ_BLOCK}), not ({self.block}, {self.dq_block})")
 
     @property
@@ -191,7 +194,6 @@ def qlora_linear_fwd(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Te
                      save_h: bool = True, out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
                      stream=None):
     """Y = X deq(W)^T + scale (X A^T) B^T.  Returns (Y, H) with H = X A^T (bf16) or None."""
-    w._layer_format()
     M = X.shape[0]
     r = A.shape[0]
     _req(X, torch.bfloat16, "X", (M, w.K))
@@ -203,9 +205,10 @@ def qlora_linear_fwd(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Te
     H = torch.empty(M, r, dtype=torch.bfloat16, device=X.device) if save_h else None
     nbytes = fwd_workspace_bytes(M, w.N, w.K, r)
     ws = _workspace(nbytes, X.device, workspace)
-    _check(lib().qlora_linear_fwd(_ptr(w.codes), _ptr(w.absmax_q), _ptr(w.dq_scale), w.N, w.K, _ptr(X), M, _ptr(A),
-                                  _ptr(B), r, float(scale), _ptr(out), _ptr(H), _ptr(ws), ws.numel(),
-                                  _stream(stream)), "qlora_linear_fwd")
+    _check(lib().qlora_linear_fwd_fmt(_ptr(w.codes), _ptr(w.absmax_q) if w.absmax_q.numel() else None,
+                                      _ptr(w.dq_scale), w.block, w.dq_block, w.N, w.K, _ptr(X), M, _ptr(A), _ptr(B),
+                                      r, float(scale), _ptr(out), _ptr(H), _ptr(ws), ws.numel(), _stream(stream)),
+           "qlora_linear_fwd")
     return out, H
 
 
@@ -213,7 +216,6 @@ def qlora_linear_bwd(w: NF4Weight, X: torch.Tensor, dY: torch.Tensor, A: torch.T
                      scale: float, H: torch.Tensor | None = None, want_dx: bool = True,
                      outs=None, workspace: torch.Tensor | None = None, stream=None):
     """Returns (dX or None, dA, dB) for Y = X deq(W)^T + scale (X A^T) B^T."""
-    w._layer_format()
     M = X.shape[0]
     r = A.shape[0]
     _req(X, torch.bfloat16, "X", (M, w.K))
@@ -230,9 +232,10 @@ def qlora_linear_bwd(w: NF4Weight, X: torch.Tensor, dY: torch.Tensor, A: torch.T
         dX, dA, dB = outs
     nbytes = bwd_workspace_bytes(M, w.N, w.K, r)
     ws = _workspace(nbytes, X.device, workspace)
-    _check(lib().qlora_linear_bwd(_ptr(w.codes), _ptr(w.absmax_q), _ptr(w.dq_scale), w.N, w.K, _ptr(X), _ptr(dY),
-                                  M, _ptr(A), _ptr(B), r, float(scale), _ptr(H), _ptr(dX), _ptr(dA), _ptr(dB),
-                                  _ptr(ws), ws.numel(), _stream(stream)), "qlora_linear_bwd")
+    _check(lib().qlora_linear_bwd_fmt(_ptr(w.codes), _ptr(w.absmax_q) if w.absmax_q.numel() else None,
+                                      _ptr(w.dq_scale), w.block, w.dq_block, w.N, w.K, _ptr(X), _ptr(dY), M, _ptr(A),
+                                      _ptr(B), r, float(scale), _ptr(H), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws),
+                                      ws.numel(), _stream(stream)), "qlora_linear_bwd")
     return dX, dA, dB
 
 

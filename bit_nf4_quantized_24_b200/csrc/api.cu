@@ -82,6 +82,13 @@ int check_layer_shapes(int64_t M, int64_t N, int64_t K, int r) {
   return QLORA_OK;
 }
 
+// The NF4 formats the layer reads: block in {32, 64, 128, 256}, dq_block 256 or 0.
+int check_format(int64_t K, int block, int dq_block) {
+  if ((block != 32 && block != 64 && block != 128 && block != 256) || (dq_block != 256 && dq_block != 0))
+    return QLORA_ERR_UNSUPPORTED;
+  return K % block ? QLORA_ERR_SHAPE : QLORA_OK;
+}
+
 struct FwdWorkspace {
   uint16_t* Hs;  // bf16(scale * X A^T) [M, r]
   size_t bytes;
@@ -223,13 +230,15 @@ int qlora_linear_bwd_workspace(int64_t M, int64_t N, int64_t K, int r, size_t* b
   return QLORA_OK;
 }
 
-int qlora_linear_fwd(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale, int64_t N, int64_t K,
-                     const qlora_bf16_t* X, int64_t M, const qlora_bf16_t* A, const qlora_bf16_t* B, int r,
-                     float scale, qlora_bf16_t* Y, qlora_bf16_t* H_save, void* workspace, size_t workspace_bytes,
-                     void* stream) {
+int qlora_linear_fwd_fmt(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale, int block,
+                         int dq_block, int64_t N, int64_t K, const qlora_bf16_t* X, int64_t M, const qlora_bf16_t* A,
+                         const qlora_bf16_t* B, int r, float scale, qlora_bf16_t* Y, qlora_bf16_t* H_save,
+                         void* workspace, size_t workspace_bytes, void* stream) {
   int st = check_layer_shapes(M, N, K, r);
   if (st) return st;
-  if (!codes || !absmax_q || !dq_scale || !A || !B || (M > 0 && (!X || !Y))) return QLORA_ERR_ARG;
+  st = check_format(K, block, dq_block);
+  if (st) return st;
+  if (!codes || (dq_block && !absmax_q) || !dq_scale || !A || !B || (M > 0 && (!X || !Y))) return QLORA_ERR_ARG;
   if (!std::isfinite(scale)) return QLORA_ERR_ARG;
   if (M == 0) return QLORA_OK;
   const void* ptrs[] = {codes, X, A, B, Y};
@@ -242,7 +251,7 @@ int qlora_linear_fwd(const uint8_t* codes, const uint8_t* absmax_q, const float*
 
   cudaError_t e = launch_rowdot(X, A, M, K, r, scale, w.Hs, 1.0f, H_save, nullptr, s);
   if (e != cudaSuccess) return cuda_status(e);
-  if (M <= 16) {
+  if (M <= 16 && block == 64 && dq_block == 256) {  // the decode kernel reads the default format
     e = launch_gemv(X, M, codes, absmax_q, dq_scale, N, K, w.Hs, B, r, Y, s);
   } else {
     GemmArgs a{};
@@ -259,18 +268,31 @@ int qlora_linear_fwd(const uint8_t* codes, const uint8_t* absmax_q, const float*
     a.r = r;
     a.out = Y;
     a.pdl = true;  // its main loop runs while the H kernel finishes; the LoRA tail waits
+    a.block = block;
+    a.dq_block = dq_block;
     e = launch_nf4_gemm(a, s);
   }
   return cuda_status(e);
 }
 
-int qlora_linear_bwd(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale, int64_t N, int64_t K,
-                     const qlora_bf16_t* X, const qlora_bf16_t* dY, int64_t M, const qlora_bf16_t* A,
-                     const qlora_bf16_t* B, int r, float scale, const qlora_bf16_t* H, qlora_bf16_t* dX,
-                     qlora_bf16_t* dA, qlora_bf16_t* dB, void* workspace, size_t workspace_bytes, void* stream) {
+int qlora_linear_fwd(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale, int64_t N, int64_t K,
+                     const qlora_bf16_t* X, int64_t M, const qlora_bf16_t* A, const qlora_bf16_t* B, int r,
+                     float scale, qlora_bf16_t* Y, qlora_bf16_t* H_save, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  return qlora_linear_fwd_fmt(codes, absmax_q, dq_scale, 64, 256, N, K, X, M, A, B, r, scale, Y, H_save, workspace,
+                              workspace_bytes, stream);
+}
+
+int qlora_linear_bwd_fmt(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale, int block,
+                         int dq_block, int64_t N, int64_t K, const qlora_bf16_t* X, const qlora_bf16_t* dY, int64_t M,
+                         const qlora_bf16_t* A, const qlora_bf16_t* B, int r, float scale, const qlora_bf16_t* H,
+                         qlora_bf16_t* dX, qlora_bf16_t* dA, qlora_bf16_t* dB, void* workspace, size_t workspace_bytes,
+                         void* stream) {
   int st = check_layer_shapes(M, N, K, r);
   if (st) return st;
-  if (!codes || !absmax_q || !dq_scale || !A || !B || !dA || !dB || (M > 0 && (!X || !dY)))
+  st = check_format(K, block, dq_block);
+  if (st) return st;
+  if (!codes || (dq_block && !absmax_q) || !dq_scale || !A || !B || !dA || !dB || (M > 0 && (!X || !dY)))
     return QLORA_ERR_ARG;
   if (!std::isfinite(scale)) return QLORA_ERR_ARG;
   const void* ptrs[] = {codes, A, B, dA, dB};
@@ -318,9 +340,19 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* absmax_q, const float*
     a.r = r;
     a.out = dX;
     a.pdl = true;
+    a.block = block;
+    a.dq_block = dq_block;
     e = launch_nf4_gemm(a, s);
   }
   return cuda_status(e);
+}
+
+int qlora_linear_bwd(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale, int64_t N, int64_t K,
+                     const qlora_bf16_t* X, const qlora_bf16_t* dY, int64_t M, const qlora_bf16_t* A,
+                     const qlora_bf16_t* B, int r, float scale, const qlora_bf16_t* H, qlora_bf16_t* dX,
+                     qlora_bf16_t* dA, qlora_bf16_t* dB, void* workspace, size_t workspace_bytes, void* stream) {
+  return qlora_linear_bwd_fmt(codes, absmax_q, dq_scale, 64, 256, N, K, X, dY, M, A, B, r, scale, H, dX, dA, dB,
+                              workspace, workspace_bytes, stream);
 }
 
 int qlora_device_status(void) {

@@ -76,12 +76,16 @@ struct Bars {
   int abort;
 };
 
-template <int MODE>
+// GEN = false: the default NF4 format (64-weight blocks, double quantization
+// over groups of 256 blocks).  GEN = true: 2^lg-weight blocks (lg = 5..8),
+// double quantization on or off (dq), chosen at run time; a thread's 64
+// consecutive weights then lie in one block, or in two when blocks hold 32.
+template <int MODE, bool GEN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_nf4_gemm(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_codes,
                const __grid_constant__ CUtensorMap tm_tail_a, const __grid_constant__ CUtensorMap tm_tail_b,
                const uint8_t* __restrict__ absmax_q, const float* __restrict__ dq_scale, Nf4Levels lv, int M, int N,
-               int K, int r, int band_pairs, __nv_bfloat16* __restrict__ out, int* status) {
+               int K, int r, int band_pairs, int lg, int dq, __nv_bfloat16* __restrict__ out, int* status) {
   pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -264,20 +268,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         kcol0 = nl0 + 64 * (t >> 6);  // smem row t = 64 * (t >> 6) + (t & 63)
       }
     };
+    // Raw scale parts of the (one or two) blocks of a thread's 64 weights,
+    // loaded two iterations ahead and combined only when used.
     struct Scale {
-      uint32_t q;
-      float s2;
+      uint32_t q0, q1;
+      float s0, s1;
       bool valid;
     };
     auto fetch = [&](int it) {
-      Scale sc{0u, 0.0f, false};
+      Scale sc{0u, 0u, 0.0f, 0.0f, false};
       if (it < numK) {
         int wrow, kcol0;
         item_of(it, wrow, kcol0);
         if (wrow < N && kcol0 < K) {
-          const int64_t blk = static_cast<int64_t>(wrow) * KB + (kcol0 >> 6);
-          sc.q = __ldg(absmax_q + blk);
-          sc.s2 = __ldg(dq_scale + (blk >> 8));
+          if (!GEN) {
+            const int64_t blk = static_cast<int64_t>(wrow) * KB + (kcol0 >> 6);
+            sc.q0 = __ldg(absmax_q + blk);
+            sc.s0 = __ldg(dq_scale + (blk >> 8));
+          } else {
+            const int64_t blk = (static_cast<int64_t>(wrow) * K + kcol0) >> lg;
+            if (dq) {
+              sc.q0 = __ldg(absmax_q + blk);
+              sc.s0 = __ldg(dq_scale + (blk >> 8));
+              if (lg == 5) {
+                sc.q1 = __ldg(absmax_q + blk + 1);
+                sc.s1 = __ldg(dq_scale + ((blk + 1) >> 8));
+              }
+            } else {
+              sc.s0 = __ldg(dq_scale + blk);
+              if (lg == 5) sc.s1 = __ldg(dq_scale + blk + 1);
+            }
+          }
           sc.valid = true;
         }
       }
@@ -307,13 +328,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t b_row = base + OFF_B + s * B_BYTES + t * 128;
         const uint32_t sw = t & 7;
         if (p0.valid) {
-          const Nf4Lut lut = make_lut(lv, __fmul_rn(static_cast<float>(p0.q), p0.s2));
+          const float a0 = (GEN && !dq) ? p0.s0 : __fmul_rn(static_cast<float>(p0.q0), p0.s0);
+          const Nf4Lut lut = make_lut(lv, a0);
           const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+          if (GEN && lg == 5) {  // two 32-weight blocks: words 0-3 and 4-7
+            const float a1 = dq ? __fmul_rn(static_cast<float>(p0.q1), p0.s1) : p0.s1;
+            const Nf4Lut lut1 = make_lut(lv, a1);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint32_t o0, o1, o2, o3;
-            deq8(w[c], lut, o0, o1, o2, o3);
-            st_shared_v4(b_row + ((c ^ sw) << 4), o0, o1, o2, o3);
+            for (int c = 0; c < 8; ++c) {
+              uint32_t o0, o1, o2, o3;
+              deq8(w[c], c < 4 ? lut : lut1, o0, o1, o2, o3);
+              st_shared_v4(b_row + ((c ^ sw) << 4), o0, o1, o2, o3);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              uint32_t o0, o1, o2, o3;
+              deq8(w[c], lut, o0, o1, o2, o3);
+              st_shared_v4(b_row + ((c ^ sw) << 4), o0, o1, o2, o3);
+            }
           }
         } else {
 #pragma unroll
@@ -390,8 +423,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 // ------------------------------------------------------------ host side
 
-template <int MODE>
+template <int MODE, bool GEN>
 cudaError_t launch_mode(const GemmArgs& a, cudaStream_t st) {
+  int lg = 0;
+  while ((1 << lg) < a.block) ++lg;
   const int64_t Kc = MODE == 0 ? a.K : a.N;
   const int64_t Nout = MODE == 0 ? a.N : a.K;
   CUtensorMap tm_act, tm_codes, tm_ta, tm_tb;
@@ -409,7 +444,7 @@ cudaError_t launch_mode(const GemmArgs& a, cudaStream_t st) {
     ok = ok && make_map(&tm_tb, BF16, a.tail_b, a.K, a.r, a.K * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return cudaErrorInvalidValue;
 
-  cudaError_t e = smem_limit_once<k_nf4_gemm<MODE>>(SMEM_ALLOC);
+  cudaError_t e = smem_limit_once<k_nf4_gemm<MODE, GEN>>(SMEM_ALLOC);
   if (e != cudaSuccess) return e;
 
   // Token tiles are rounded up to whole pairs: a CTA past the last token
@@ -435,16 +470,16 @@ cudaError_t launch_mode(const GemmArgs& a, cudaStream_t st) {
   cfg.attrs = attr;
   cfg.numAttrs = a.pdl ? 2 : 1;
   trace_before(st);
-  e = cudaLaunchKernelEx(&cfg, k_nf4_gemm<MODE>, tm_act, tm_codes, tm_ta, tm_tb, a.absmax_q, a.dq_scale,
+  e = cudaLaunchKernelEx(&cfg, k_nf4_gemm<MODE, GEN>, tm_act, tm_codes, tm_ta, tm_tb, a.absmax_q, a.dq_scale,
                          host_codebook().levels, static_cast<int>(a.M), static_cast<int>(a.N), static_cast<int>(a.K),
-                         a.r, band_pairs, reinterpret_cast<__nv_bfloat16*>(a.out), device_status_ptr());
+                         a.r, band_pairs, lg, a.dq_block ? 1 : 0, reinterpret_cast<__nv_bfloat16*>(a.out), device_status_ptr());
   trace_after(st);
   return e;
 }
 
 template <int MODE>
 int max_active_pairs() {
-  if (smem_limit_once<k_nf4_gemm<MODE>>(SMEM_ALLOC) != cudaSuccess) return -1;
+  if (smem_limit_once<k_nf4_gemm<MODE, false>>(SMEM_ALLOC) != cudaSuccess) return -1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2, 1, 1);
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
@@ -457,7 +492,7 @@ int max_active_pairs() {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, k_nf4_gemm<MODE>, &cfg) != cudaSuccess) return -2;
+  if (cudaOccupancyMaxActiveClusters(&n, k_nf4_gemm<MODE, false>, &cfg) != cudaSuccess) return -2;
   return n;
 }
 
@@ -495,7 +530,9 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* ptr, uint64_
 }
 
 cudaError_t launch_nf4_gemm(const GemmArgs& a, cudaStream_t st) {
-  return a.mode == 0 ? launch_mode<0>(a, st) : launch_mode<1>(a, st);
+  const bool gen = !(a.block == 64 && a.dq_block == 256);
+  if (a.mode == 0) return gen ? launch_mode<0, true>(a, st) : launch_mode<0, false>(a, st);
+  return gen ? launch_mode<1, true>(a, st) : launch_mode<1, false>(a, st);
 }
 
 int nf4_gemm_max_active_pairs(int mode) { return mode == 0 ? max_active_pairs<0>() : max_active_pairs<1>(); }

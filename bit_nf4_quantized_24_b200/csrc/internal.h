@@ -54,6 +54,8 @@ struct GemmArgs {
   int r;
   uint16_t* out;  // Y [M, N] or dX [M, K]
   bool pdl;       // launched right after another kernel of the layer (programmatic dependent launch)
+  int block = 64;       // NF4 format: weights per block (32, 64, 128, 256)
+  int dq_block = 256;   // 256: double quantization; 0: fp32 absmax per block in dq_scale
 };
 cudaError_t launch_nf4_gemm(const GemmArgs& a, cudaStream_t st);
 // CTA pairs of the fused GEMM that fit on the current device at once

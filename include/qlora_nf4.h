@@ -139,6 +139,18 @@ int qlora_linear_fwd(const uint8_t* codes, const uint8_t* absmax_q, const float*
                      qlora_bf16_t* Y, qlora_bf16_t* H_save,
                      void* workspace, size_t workspace_bytes, void* stream);
 
+/* qlora_linear_fwd for an NF4 weight in any format the codec writes: block
+ * in {32, 64, 128, 256}, dq_block 256 or 0 (absmax_q may then be NULL; see
+ * the NF4 format above; K % block == 0).  qlora_linear_fwd is this call with
+ * block 64, dq_block 256.  The bandwidth-bound decode kernel reads the default
+ * format only: other formats run the tensor-core GEMM for every M. */
+int qlora_linear_fwd_fmt(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale,
+                         int block, int dq_block, int64_t N, int64_t K,
+                         const qlora_bf16_t* X, int64_t M, const qlora_bf16_t* A,
+                         const qlora_bf16_t* B, int r, float scale, qlora_bf16_t* Y,
+                         qlora_bf16_t* H_save, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
 /* Backward of the QLoRA linear: gradients flow through deq(W) to the
  * adapters and to the input; the frozen base gets none (katajob, "What stays
  * in full precision"):
@@ -155,6 +167,16 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* absmax_q, const float*
                      float scale, const qlora_bf16_t* H,
                      qlora_bf16_t* dX, qlora_bf16_t* dA, qlora_bf16_t* dB,
                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* qlora_linear_bwd for an NF4 weight in any codec format (as
+ * qlora_linear_fwd_fmt); qlora_linear_bwd is this call with block 64,
+ * dq_block 256. */
+int qlora_linear_bwd_fmt(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale,
+                         int block, int dq_block, int64_t N, int64_t K,
+                         const qlora_bf16_t* X, const qlora_bf16_t* dY, int64_t M,
+                         const qlora_bf16_t* A, const qlora_bf16_t* B, int r, float scale,
+                         const qlora_bf16_t* H, qlora_bf16_t* dX, qlora_bf16_t* dA,
+                         qlora_bf16_t* dB, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Largest M * r that qlora_linear_fwd_noalloc accepts: its fixed device
  * scratch holds this many bf16 values (2 MiB on every device that loads the

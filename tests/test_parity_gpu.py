@@ -163,13 +163,28 @@ def test_codec_other_formats_bit_exact(qb, oracle, block, dq_block):
     assert np.array_equal(Wd.view(torch.int16).cpu().numpy().view(np.uint16), o16)
 
 
-def test_layer_rejects_other_formats(qb):
+@pytest.mark.parametrize("block,dq_block", [(32, 256), (128, 0), (256, 256), (64, 0)])
+def test_layer_other_formats(qb, oracle, block, dq_block):
+    """The fused GEMM reads every codec format: forward at a GEMM size and at a
+    decode size (both through the GEMM for non-default formats) and backward,
+    against the oracle's dequantized weight of the same format."""
+    M, N, K, r = 150, 264, 1024, 16
+    p = wl.draw_small(600 + block + dq_block, M, N, K, r, 2.0 * r)
+    q, Wp = quantize_both(qb, oracle, p["W"], block, dq_block)
+    run_fwd_check(qb, oracle, p, q=q, Wp=Wp)
+    run_bwd_check(qb, oracle, p, q=q, Wp=Wp)
+    p2 = dict(p)
+    p2["X"] = p["X"][:5].contiguous()
+    run_fwd_check(qb, oracle, p2, q=q, Wp=Wp)
+
+
+def test_noalloc_entry_reads_default_format_only(qb):
     q = qb.nf4_quantize(torch.randn(64, 256, device="cuda") * 0.02, 128, 0)
     X = torch.randn(32, 256, device="cuda").bfloat16()
     A = torch.randn(16, 256, device="cuda").bfloat16()
     B = torch.randn(64, 16, device="cuda").bfloat16()
     with pytest.raises(qb.QloraError) as ei:
-        qb.qlora_linear_fwd(q, X, A, B, 2.0)
+        qb.qlora_linear_fwd_noalloc(q, X, A, B, 2.0)
     assert ei.value.status == -7
 
 
