@@ -63,6 +63,8 @@ def _load():
     lib.or_linear_bwd.argtypes = [P, P, i64, i64, P, i64, P, P, ctypes.c_int, ctypes.c_double,
                                   P, i64, P, P, P, P]
     lib.or_num_threads.restype = ctypes.c_int
+    lib.or_nf4_merge_lora.argtypes = [P, P, P, ctypes.c_int, ctypes.c_int, i64, i64, P, P, ctypes.c_int,
+                                      ctypes.c_float, ctypes.c_int, ctypes.c_int, P, P, P, P]
     _lib = lib
     return lib
 
@@ -142,6 +144,26 @@ def nf4_dequantize(codes, absmax_q, dq_scale, N: int, K: int, block: int = 64,
     _check(lib.or_nf4_dequantize(_p(codes), _p(absmax_q), _p(dq_scale), N, K, block, dq_block,
                                  _p(out16), _p(out32)), "dequantize")
     return out16, out32
+
+
+def nf4_merge_lora(codes, absmax_q, dq_scale, N: int, K: int, A16, B16, scale: float, block: int = 64,
+                   dq_block: int = 256, out_block: int = 64, out_dq_block: int = 256):
+    """Merge s * B A into the NF4 weight and quantize the sum again.
+    A16: bf16 bits u16 [r, K]; B16: bf16 bits u16 [N, r].  Returns
+    (codes, absmax_q, dq_scale, merged fp32 [N, K]) in the output format."""
+    lib = _load()
+    A16 = _c(A16, np.uint16)
+    B16 = _c(B16, np.uint16)
+    r = A16.shape[0]
+    cb, ab, dc = nf4_sizes(N, K, out_block, out_dq_block)
+    oc = np.zeros(cb, np.uint8)
+    oa = np.zeros(max(ab, 1), np.uint8)[:ab]
+    od = np.zeros(dc, np.float32)
+    merged = np.zeros((N, K), np.float32)
+    _check(lib.or_nf4_merge_lora(_p(_c(codes, np.uint8)), _p(_c(absmax_q, np.uint8)), _p(_c(dq_scale, np.float32)),
+                                 block, dq_block, N, K, _p(A16), _p(B16), r, float(scale), out_block, out_dq_block,
+                                 _p(oc), _p(oa), _p(od), _p(merged)), "merge_lora")
+    return oc, oa, od, merged
 
 
 def f32_to_bf16_bits(x: float) -> int:

@@ -262,6 +262,42 @@ int or_nf4_dequantize(const uint8_t* codes, const uint8_t* absmax_q, const float
     return OR_OK;
 }
 
+/* ------------------------------------------- merge and re-quantize (f2) */
+
+/* After training the adapter is folded into the frozen weight ("QLoRA and
+ * Quantized Fine-Tuning", "The two mechanisms combined": the model computes
+ * with W' + BA) and the sum is stored as NF4 again:
+ *   w'[n,k]    = the dequantized weight the layer uses (bf16 value, in fp32)
+ *   delta[n,k] = sum_j B[n,j] A[j,k], accumulated in fp32 in the order
+ *                j = 0 .. r-1 (each product of two bf16 values is exact in fp32)
+ *   merged     = fl32(w' + fl32(s * delta))
+ * then quantized with or_nf4_quantize in the output format.  The sum order is
+ * fixed so that the fp32 value, and hence every code, is reproducible. */
+int or_nf4_merge_lora(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale,
+                      int block, int dq_block, int64_t N, int64_t K,
+                      const uint16_t* A, const uint16_t* B, int r, float s,
+                      int out_block, int out_dq_block, uint8_t* out_codes, uint8_t* out_absmax_q,
+                      float* out_dq_scale, float* merged_out) {
+    if (!A || !B || r <= 0 || !out_codes || !out_dq_scale) return OR_ERR_ARG;
+    const int64_t numel = N * K;
+    float* wp = (float*)malloc(sizeof(float) * (size_t)(numel ? numel : 1));
+    if (!wp) return OR_ERR_ARG;
+    int st = or_nf4_dequantize(codes, absmax_q, dq_scale, N, K, block, dq_block, NULL, wp);
+    if (st) { free(wp); return st; }
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            float acc = 0.0f;
+            for (int j = 0; j < r; ++j)
+                acc = r32((double)acc + bf16_to_f64(B[n * r + j]) * bf16_to_f64(A[(int64_t)j * K + k]));
+            wp[n * K + k] = r32((double)wp[n * K + k] + (double)r32((double)s * (double)acc));
+        }
+    if (merged_out) memcpy(merged_out, wp, sizeof(float) * (size_t)numel);
+    st = or_nf4_quantize(wp, N, K, out_block, out_dq_block, out_codes, out_absmax_q, out_dq_scale, NULL);
+    free(wp);
+    return st;
+}
+
 /* bf16 rounding exposed for the tests that pin it against textbook values. */
 uint16_t or_f32_to_bf16(float f) { return f32_to_bf16_rne(f); }
 

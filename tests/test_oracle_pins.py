@@ -385,3 +385,62 @@ def test_format_bits_per_parameter(oracle, block, dq_block, bits):
     N, K = 64, 4096
     cb, ab, dc = oracle.nf4_sizes(N, K, block, dq_block)
     assert (8 * (cb + ab) + 32 * dc) / (N * K) == pytest.approx(bits, rel=1e-12)
+
+
+# ------------------------------------------------- merge and re-quantize (f2)
+
+
+def _quantized(oracle, seed, N=12, K=512, block=64, dq_block=256):
+    W = wl.draw_weight(wl.generator(seed), N, K, 0.02, 0.05).numpy()
+    W[1, :block] = 0.0  # an all-zero block
+    codes, aq, dq, _ = oracle.nf4_quantize(W, block=block, dq_block=dq_block)
+    _, wp = oracle.nf4_dequantize(codes, aq, dq, N, K, block=block, dq_block=dq_block)
+    return codes, aq, dq, wp
+
+
+@pytest.mark.parametrize("block,dq_block", [(64, 256), (32, 0), (256, 256)])
+def test_merge_with_zero_adapter_is_idempotent(oracle, block, dq_block):
+    """B = 0: the merged weight is the dequantized weight itself, and quantizing
+    it again returns the same codes (each block's largest weight sits on level
+    +-1, and bf16 rounding moves w'/a far less than the level spacing)."""
+    N, K, r = 12, 512, 8
+    codes, aq, dq, wp = _quantized(oracle, 31, N, K, block, dq_block)
+    A = wl.bf16_bits(torch.randn(r, K).bfloat16())
+    B = np.zeros((N, r), np.uint16)
+    oc, oa, od, merged = oracle.nf4_merge_lora(codes, aq, dq, N, K, A, B, 2.0, block, dq_block, block, dq_block)
+    assert np.array_equal(merged, wp)
+    assert np.array_equal(oc, codes)
+
+
+def test_merge_closed_form_shift(oracle):
+    """r = 1, A = 1, B = 0.25, s = 2: every weight moves by exactly 0.5."""
+    N, K = 4, 128
+    codes, aq, dq, wp = _quantized(oracle, 32, N, K)
+    one = np.uint16(0x3F80)      # bf16 1.0
+    quarter = np.uint16(0x3E80)  # bf16 0.25
+    A = np.full((1, K), one, np.uint16)
+    B = np.full((N, 1), quarter, np.uint16)
+    _, _, _, merged = oracle.nf4_merge_lora(codes, aq, dq, N, K, A, B, 2.0)
+    assert np.array_equal(merged.astype(np.float64) - wp.astype(np.float64), np.full((N, K), 0.5))
+
+
+@pytest.mark.parametrize("out_block,out_dq", [(64, 256), (128, 0)])
+def test_merge_matches_real_sum_within_quantization_error(oracle, out_block, out_dq):
+    """The re-quantized merge dequantizes to w' + s B A (fp64) within the NF4
+    error of its own blocks: half the widest level gap times the block absmax,
+    plus the scale coding and bf16 rounding."""
+    N, K, r, s = 16, 512, 16, 0.25
+    codes, aq, dq, wp = _quantized(oracle, 33, N, K)
+    g = wl.generator(34)
+    A = (torch.rand(r, K, generator=g) * 2 - 1) / np.sqrt(K)
+    B = torch.randn(N, r, generator=g) * 0.05
+    A16, B16 = wl.bf16_bits(A.bfloat16()), wl.bf16_bits(B.bfloat16())
+    oc, oa, od, merged = oracle.nf4_merge_lora(codes, aq, dq, N, K, A16, B16, s, 64, 256, out_block, out_dq)
+    exact = wp.astype(np.float64) + s * (B.bfloat16().double().numpy() @ A.bfloat16().double().numpy())
+    assert np.max(np.abs(merged - exact)) <= 1e-6 * np.max(np.abs(exact))
+    _, back = oracle.nf4_dequantize(oc, oa, od, N, K, block=out_block, dq_block=out_dq)
+    _, l32, _ = oracle.nf4_codebook()
+    half_gap = np.max(np.diff(l32.astype(np.float64))) / 2
+    amax = np.repeat(np.abs(merged.reshape(-1, out_block)).max(axis=1), out_block).reshape(N, K).astype(np.float64)
+    bound = amax * (half_gap + 1.0 / 255) + np.abs(exact) * 2 ** -8 + 1e-30
+    assert np.all(np.abs(back - exact) <= bound)
