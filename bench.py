@@ -425,7 +425,40 @@ def run_extras(qb, wl, dev, pk, flush):
     ms = timed(lambda: qb.nf4_dequantize(q, out=out), n=10)
     res["nf4_dequantize"] = {"ms": round(ms, 4), "gbs": round(dbytes / ms / 1e6, 1),
                              "frac_hbm": round(dbytes / ms / 1e6 / pk["hbm_gbs"], 4)}
-    del Wd, out
+    # other NF4 formats (block size, double quantization on/off): the codec on
+    # the same weight, and the forward of the q_proj workload through the GEMM
+    fmts = {}
+    for block, dq in ((32, 256), (128, 0), (256, 256)):
+        cb, ab, db = qb.nf4_quantized_sizes(N, K, block, dq)
+        qf = qb.nf4_quantize(Wd, block, dq)
+        ms_q = timed(lambda: qb.nf4_quantize(Wd, block, dq), n=5)
+        ms_d = timed(lambda: qb.nf4_dequantize(qf, out=out), n=10)
+        fmts[f"b{block}_dq{dq}"] = {
+            "quantize_gbs": round((4 * numel + cb + ab + db) / ms_q / 1e6, 1),
+            "dequantize_gbs": round((cb + ab + db + 2 * numel) / ms_d / 1e6, 1)}
+        del qf
+    w2 = wl.WORKLOADS[WORKLOAD]
+    p2 = wl.draw_linear(w2)
+    W2, X2, A2, B2 = p2["W"].to(dev), p2["X"].to(dev), p2["A"].to(dev), p2["B"].to(dev)
+    M2, N2, K2, r2 = p2["M"], p2["N"], p2["K"], p2["r"]
+    Y2 = torch.empty(M2, N2, dtype=torch.bfloat16, device=dev)
+    ws2 = torch.empty(qb.fwd_workspace_bytes(M2, N2, K2, r2), dtype=torch.uint8, device=dev)
+    flops = 2 * M2 * N2 * K2 + 2 * M2 * r2 * (K2 + N2)
+    for block, dq in ((64, 256), (32, 256), (128, 0), (256, 256)):
+        qf = qb.nf4_quantize(W2, block, dq)
+        ms_f = timed(lambda: qb.qlora_linear_fwd(qf, X2, A2, B2, p2["scale"], save_h=False, out=Y2, workspace=ws2),
+                     n=10)
+        fmts.setdefault(f"b{block}_dq{dq}", {})["qproj_fwd_tflops"] = round(flops / ms_f / 1e9, 1)
+        del qf
+    res["formats"] = fmts
+    # merge of the decode weight with its r = 16 adapter, quantized again
+    # (reads codes + scales + A + B, writes codes + scales)
+    mbytes = weight_bytes * 2 + 2 * r * (K + N)
+    ms_m = timed(lambda: qb.nf4_merge_lora(q, A, B, s), n=5)
+    res["nf4_merge_lora"] = {"ms": round(ms_m, 4), "gbs": round(mbytes / ms_m / 1e6, 1),
+                             "frac_hbm": round(mbytes / ms_m / 1e6 / pk["hbm_gbs"], 4),
+                             "note": "includes the call's stream synchronization (non-finite check)"}
+    del Wd, out, W2, X2, Y2
     torch.cuda.empty_cache()
     return res
 

@@ -62,6 +62,7 @@ def lib():
     L.qlora_linear_bwd.argtypes = [P, P, P, i64, i64, P, P, i64, P, P, i32, f32, P, P, P, P, P, sz, P]
     L.qlora_linear_fwd_noalloc.argtypes = [P, P, P, i64, i64, P, i64, P, P, i32, f32, P, P, P]
     L.qlora_linear_fwd_fmt.argtypes = [P, P, P, i32, i32, i64, i64, P, i64, P, P, i32, f32, P, P, P, sz, P]
+    L.nf4_merge_lora.argtypes = [P, P, P, i32, i32, i64, i64, P, P, i32, f32, i32, i32, P, P, P, P]
     L.qlora_linear_bwd_fmt.argtypes = [P, P, P, i32, i32, i64, i64, P, P, i64, P, P, i32, f32, P, P, P, P, P, sz,
                                        P]
     L.qlora_device_status.restype = i32
@@ -170,6 +171,27 @@ def nf4_dequantize(w: NF4Weight, out: torch.Tensor | None = None, stream=None) -
     _check(lib().nf4_dequantize(_ptr(w.codes), _ptr(w.absmax_q) if w.absmax_q.numel() else None, _ptr(w.dq_scale),
                                 w.N, w.K, w.block, w.dq_block, _ptr(out), _stream(stream)), "nf4_dequantize")
     return out
+
+
+def nf4_merge_lora(w: NF4Weight, A: torch.Tensor, B: torch.Tensor, scale: float, block: int | None = None,
+                   dq_block: int | None = None, stream=None) -> NF4Weight:
+    """A new NF4 weight holding deq(W) + scale * B A, quantized again (in w's
+    format unless block / dq_block are given)."""
+    r = A.shape[0]
+    _req(A, torch.bfloat16, "A", (r, w.K))
+    _req(B, torch.bfloat16, "B", (w.N, r))
+    block = w.block if block is None else block
+    dq_block = w.dq_block if dq_block is None else dq_block
+    cb, ab, db = nf4_quantized_sizes(w.N, w.K, block, dq_block)
+    dev = w.codes.device
+    codes = torch.empty(cb, dtype=torch.uint8, device=dev)
+    absmax_q = torch.empty(ab, dtype=torch.uint8, device=dev)
+    dq_scale = torch.empty(db // 4, dtype=torch.float32, device=dev)
+    _check(lib().nf4_merge_lora(_ptr(w.codes), _ptr(w.absmax_q) if w.absmax_q.numel() else None, _ptr(w.dq_scale),
+                                w.block, w.dq_block, w.N, w.K, _ptr(A), _ptr(B), r, float(scale), block, dq_block,
+                                _ptr(codes), _ptr(absmax_q) if ab else None, _ptr(dq_scale), _stream(stream)),
+           "nf4_merge_lora")
+    return NF4Weight(codes, absmax_q, dq_scale, w.N, w.K, block, dq_block)
 
 
 def fwd_workspace_bytes(M, N, K, r) -> int:

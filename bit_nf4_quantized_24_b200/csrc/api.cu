@@ -214,6 +214,36 @@ int nf4_dequantize(const uint8_t* codes, const uint8_t* absmax_q, const float* d
       launch_dequantize(codes, absmax_q, dq_scale, N * K, block, dq_block, W_out, static_cast<cudaStream_t>(stream)));
 }
 
+int nf4_merge_lora(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale, int block, int dq_block,
+                   int64_t N, int64_t K, const qlora_bf16_t* A, const qlora_bf16_t* B, int r, float scale,
+                   int out_block, int out_dq_block, uint8_t* out_codes, uint8_t* out_absmax_q, float* out_dq_scale,
+                   void* stream) {
+  size_t cb, ab, db;
+  int st = nf4_quantized_sizes(N, K, block, dq_block, &cb, &ab, &db);
+  if (st) return st;
+  st = nf4_quantized_sizes(N, K, out_block, out_dq_block, &cb, &ab, &db);
+  if (st) return st;
+  if (r < 1 || r > 64 || !std::isfinite(scale)) return r < 1 ? QLORA_ERR_ARG : QLORA_ERR_UNSUPPORTED;
+  if (N * K == 0) return QLORA_OK;
+  if (!codes || (dq_block && !absmax_q) || !dq_scale || !A || !B || !out_codes || (out_dq_block && !out_absmax_q) ||
+      !out_dq_scale)
+    return QLORA_ERR_ARG;
+  if (!aligned(codes, 4) || !aligned(A, 16) || !aligned(out_codes, 4)) return QLORA_ERR_SHAPE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(g_quantize_mutex);
+  int* flag = device_nonfinite_ptr();
+  if (!flag) return cuda_status(cudaErrorInvalidSymbol);
+  cudaError_t e = cudaMemsetAsync(flag, 0, sizeof(int), s);
+  if (e == cudaSuccess)
+    e = launch_merge_quantize(codes, absmax_q, dq_scale, block, dq_block, N, K, A, B, r, scale, out_block,
+                              out_dq_block, out_codes, out_absmax_q, out_dq_scale, flag, s);
+  int host_flag = 0;
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&host_flag, flag, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_status(e);
+  return host_flag ? QLORA_ERR_NONFINITE : QLORA_OK;
+}
+
 int qlora_linear_fwd_workspace(int64_t M, int64_t N, int64_t K, int r, size_t* bytes) {
   if (!bytes) return QLORA_ERR_ARG;
   int st = check_layer_shapes(M, N, K, r);

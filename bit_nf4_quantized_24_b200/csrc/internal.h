@@ -37,6 +37,12 @@ cudaError_t launch_quantize(const float* W, int64_t numel, int block, int dq_blo
                             uint8_t* absmax_q, float* dq_scale, int* nonfinite, cudaStream_t st);
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale,
                               int64_t numel, int block, int dq_block, uint16_t* out, cudaStream_t st);
+// Quantize (into block / dq_block) the merge of an NF4 weight (block_in /
+// dq_block_in) with the adapter: fl32(w' + fl32(scale * sum_j B[n,j] A[j,k])).
+cudaError_t launch_merge_quantize(const uint8_t* codes_in, const uint8_t* absmax_in, const float* dq_in, int block_in,
+                                  int dq_block_in, int64_t N, int64_t K, const uint16_t* A, const uint16_t* Bl, int r,
+                                  float scale, int block, int dq_block, uint8_t* codes, uint8_t* absmax_q,
+                                  float* dq_scale, int* nonfinite, cudaStream_t st);
 
 // ----- fused dequant-GEMM on tcgen05 (tensor cores)
 // mode 0 (forward):  Y[M,N]  = X[M,K]  deq(W)^T + Ht[M,r] Bt^T, Bt = lora_B [N,r]

@@ -50,23 +50,72 @@ __device__ __forceinline__ float div_by_absmax(float w, float a, float r) {
   return __fmaf_rn(e, r, q0);
 }
 
+// Source of the values to quantize: an fp32 weight, or (merge) the NF4 weight
+// the layer uses plus the folded adapter ("QLoRA and Quantized Fine-Tuning",
+// "The two mechanisms combined": the merged model computes with W' + BA):
+//   merged[n, k] = fl32(w'[n, k] + fl32(s * sum_j B[n, j] A[j, k])),
+// w' = bf16(L[code] * a') as dequantized for the layer, the sum in fp32 in the
+// order j = 0 .. r-1 (every product of two bf16 values is exact in fp32, so
+// each FMA adds one exact product).
+struct MergeSrc {
+  const uint8_t* codes;
+  const uint8_t* absmax_q;
+  const float* dq_scale;
+  int lg;  // log2 of the input block size
+  int dq;  // input has double quantization
+  const uint16_t* A;  // bf16 [r, K]
+  const uint16_t* B;  // bf16 [N, r]
+  int r;
+  float s;
+  int64_t K;
+};
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as_float(h << 16); }
+
+// merged values of elements e .. e+3 (one row, one input block); lv: the 16
+// levels in shared memory
+__device__ __forceinline__ float4 merged4(const MergeSrc& m, const float* lv, int64_t e) {
+  const int64_t n = e / m.K, k = e - n * m.K;
+  const uint32_t c = *reinterpret_cast<const uint16_t*>(m.codes + e / 2);
+  const int64_t b = e >> m.lg;
+  const float a = m.dq ? __fmul_rn(static_cast<float>(m.absmax_q[b]), m.dq_scale[b >> 8]) : m.dq_scale[b];
+  float w[4], acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) w[i] = __bfloat162float(__float2bfloat16_rn(__fmul_rn(lv[(c >> (4 * i)) & 15u], a)));
+  const uint16_t* arow = m.A + k;
+  const uint16_t* brow = m.B + n * m.r;
+  for (int j = 0; j < m.r; ++j) {
+    const float bj = bf16_bits_to_f32(brow[j]);
+    const uint2 a4 = *reinterpret_cast<const uint2*>(arow + static_cast<int64_t>(j) * m.K);
+    acc[0] = __fmaf_rn(bj, bf16_bits_to_f32(a4.x & 0xffffu), acc[0]);
+    acc[1] = __fmaf_rn(bj, bf16_bits_to_f32(a4.x >> 16), acc[1]);
+    acc[2] = __fmaf_rn(bj, bf16_bits_to_f32(a4.y & 0xffffu), acc[2]);
+    acc[3] = __fmaf_rn(bj, bf16_bits_to_f32(a4.y >> 16), acc[3]);
+  }
+  return make_float4(__fadd_rn(w[0], __fmul_rn(m.s, acc[0])), __fadd_rn(w[1], __fmul_rn(m.s, acc[1])),
+                     __fadd_rn(w[2], __fmul_rn(m.s, acc[2])), __fadd_rn(w[3], __fmul_rn(m.s, acc[3])));
+}
+
 // One CTA per group of 256 blocks (the double-quant group).  A block of B
 // weights is spread over LP = min(32, B / 4) lanes, F = B / (4 LP) float4s per
 // lane; a warp covers 32 / LP blocks per step, and four steps' loads are
 // issued before any is used, to keep HBM busy.  DQ: double quantization of the
 // group's absmax values (else each block's fp32 absmax is stored as is).
-template <int B, bool DQ>
-__global__ void __launch_bounds__(256) k_quantize(const float* __restrict__ W, int64_t nblocks, Nf4Mids mids,
-                                                  uint8_t* __restrict__ codes, uint8_t* __restrict__ absmax_q,
-                                                  float* __restrict__ dq_scale, int* nonfinite) {
+template <int B, bool DQ, bool MERGE>
+__global__ void __launch_bounds__(256) k_quantize(const float* __restrict__ W, MergeSrc msrc, Nf4Levels levels,
+                                                  int64_t nblocks, Nf4Mids mids, uint8_t* __restrict__ codes,
+                                                  uint8_t* __restrict__ absmax_q, float* __restrict__ dq_scale,
+                                                  int* nonfinite) {
   constexpr int LP = B / 4 < 32 ? B / 4 : 32;
   constexpr int F = B / (4 * LP);
   constexpr int BPW = 32 / LP;  // blocks per warp step
   __shared__ Cell s_cell[kCells];
   __shared__ float s_amax[kGroup];
   __shared__ float s_red[8];
+  __shared__ float s_lv[16];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int sub = lane / LP, sl = lane % LP;
+  if (MERGE && tid < 16) s_lv[tid] = levels.v[tid];
   const int64_t g = blockIdx.x;
   const int64_t b0 = g * kGroup;
   const int64_t rem = nblocks - b0;
@@ -93,9 +142,13 @@ __global__ void __launch_bounds__(256) k_quantize(const float* __restrict__ W, i
       const int i = BPW * (p0 + 8 * u) + sub;
       ok[u] = (p0 + 8 * u < nsteps) && (i < nb);
 #pragma unroll
-      for (int f = 0; f < F; ++f)
-        x[u][f] = ok[u] ? __ldcs(reinterpret_cast<const float4*>(W + (b0 + i) * B) + f * LP + sl)
-                        : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int f = 0; f < F; ++f) {
+        if (MERGE)
+          x[u][f] = ok[u] ? merged4(msrc, s_lv, (b0 + i) * B + (f * LP + sl) * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        else
+          x[u][f] = ok[u] ? __ldcs(reinterpret_cast<const float4*>(W + (b0 + i) * B) + f * LP + sl)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -219,13 +272,18 @@ __global__ void __launch_bounds__(256) k_dequantize(const uint8_t* __restrict__ 
 }
 
 template <int B, bool DQ>
-cudaError_t quantize_launch(const float* W, int64_t numel, uint8_t* codes, uint8_t* absmax_q, float* dq_scale,
-                            int* nonfinite, cudaStream_t st) {
+cudaError_t quantize_launch(const float* W, const MergeSrc* merge, int64_t numel, uint8_t* codes,
+                            uint8_t* absmax_q, float* dq_scale, int* nonfinite, cudaStream_t st) {
   const int64_t nblocks = numel / B;
   const int64_t ngroups = (nblocks + kGroup - 1) / kGroup;
   if (ngroups == 0) return cudaSuccess;
-  k_quantize<B, DQ><<<static_cast<unsigned>(ngroups), 256, 0, st>>>(W, nblocks, host_codebook().mids, codes,
-                                                                    absmax_q, dq_scale, nonfinite);
+  const HostCodebook& cb = host_codebook();
+  if (merge)
+    k_quantize<B, DQ, true><<<static_cast<unsigned>(ngroups), 256, 0, st>>>(
+        nullptr, *merge, cb.levels, nblocks, cb.mids, codes, absmax_q, dq_scale, nonfinite);
+  else
+    k_quantize<B, DQ, false><<<static_cast<unsigned>(ngroups), 256, 0, st>>>(
+        W, MergeSrc{}, cb.levels, nblocks, cb.mids, codes, absmax_q, dq_scale, nonfinite);
   return cudaGetLastError();
 }
 
@@ -258,7 +316,20 @@ cudaError_t dequantize_launch(const uint8_t* codes, const uint8_t* absmax_q, con
 
 cudaError_t launch_quantize(const float* W, int64_t numel, int block, int dq_block, uint8_t* codes,
                             uint8_t* absmax_q, float* dq_scale, int* nonfinite, cudaStream_t st) {
-  QN_CODEC_DISPATCH(quantize_launch, W, numel, codes, absmax_q, dq_scale, nonfinite, st)
+  QN_CODEC_DISPATCH(quantize_launch, W, nullptr, numel, codes, absmax_q, dq_scale, nonfinite, st)
+}
+
+cudaError_t launch_merge_quantize(const uint8_t* codes_in, const uint8_t* absmax_in, const float* dq_in, int block_in,
+                                  int dq_block_in, int64_t N, int64_t K, const uint16_t* A, const uint16_t* Bl, int r,
+                                  float scale, int block, int dq_block, uint8_t* codes, uint8_t* absmax_q,
+                                  float* dq_scale, int* nonfinite, cudaStream_t st) {
+  int lg = 0;
+  while ((1 << lg) < block_in) ++lg;
+  const MergeSrc m{codes_in, absmax_in, dq_in, lg, dq_block_in ? 1 : 0, A, Bl, r, scale, K};
+  const MergeSrc* mp = &m;
+  const int64_t numel = N * K;
+  const float* W = nullptr;
+  QN_CODEC_DISPATCH(quantize_launch, W, mp, numel, codes, absmax_q, dq_scale, nonfinite, st)
 }
 
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale, int64_t numel,

@@ -116,6 +116,26 @@ int nf4_dequantize(const uint8_t* codes, const uint8_t* absmax_q, const float* d
                    int64_t N, int64_t K, int block, int dq_block,
                    qlora_bf16_t* W_out, void* stream);
 
+/* Merge the trained adapter into the frozen weight and store the sum as NF4
+ * again ("QLoRA and Quantized Fine-Tuning", "The two mechanisms combined": the
+ * merged model computes with W' + BA):
+ *     merged[n, k] = fl32(w'[n, k] + fl32(scale * sum_j B[n, j] A[j, k]))
+ * where w' is the bf16 weight the layer dequantizes (format block / dq_block)
+ * and the sum runs in fp32 in the order j = 0 .. r-1 (each product of two
+ * bf16 values is exact in fp32); merged is then quantized exactly as
+ * nf4_quantize does, into the format out_block / out_dq_block.
+ * codes, absmax_q, dq_scale: the input weight (device); A: bf16 [r, K];
+ * B: bf16 [N, r]; 1 <= r <= 64; out_*: device outputs sized by
+ * nf4_quantized_sizes(N, K, out_block, out_dq_block).  The input is only read,
+ * so the outputs must not alias it.  Synchronizes `stream` like nf4_quantize
+ * and returns QLORA_ERR_NONFINITE if a merged value is not finite.
+ * Errors: ARG, SHAPE, UNSUPPORTED, NONFINITE, CUDA. */
+int nf4_merge_lora(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale,
+                   int block, int dq_block, int64_t N, int64_t K,
+                   const qlora_bf16_t* A, const qlora_bf16_t* B, int r, float scale,
+                   int out_block, int out_dq_block, uint8_t* out_codes,
+                   uint8_t* out_absmax_q, float* out_dq_scale, void* stream);
+
 /* Workspace bytes needed by qlora_linear_fwd / qlora_linear_bwd for these
  * shapes (the caller allocates it, 256-byte aligned, device memory). */
 int qlora_linear_fwd_workspace(int64_t M, int64_t N, int64_t K, int r, size_t* bytes);

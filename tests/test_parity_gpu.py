@@ -178,6 +178,48 @@ def test_layer_other_formats(qb, oracle, block, dq_block):
     run_fwd_check(qb, oracle, p2, q=q, Wp=Wp)
 
 
+@pytest.mark.parametrize("fmt_in,fmt_out,r", [((64, 256), (64, 256), 16), ((32, 0), (128, 256), 8),
+                                               ((256, 256), (64, 0), 64), ((64, 256), (64, 256), 3)])
+def test_merge_lora_bit_exact(qb, oracle, fmt_in, fmt_out, r):
+    """Merge-and-requantize on the GPU equals the oracle bit for bit (codes,
+    absmax codes, scales), for changes of format and any r."""
+    N, K = 37, 1024
+    W = wl.draw_weight(wl.generator(700 + r), N, K, 0.02, 0.02)
+    W[2, :256] = 0.0
+    q, _ = quantize_both(qb, oracle, W, *fmt_in)
+    g = wl.generator(800 + r)
+    A = ((torch.rand(r, K, generator=g) * 2 - 1) / np.sqrt(K)).bfloat16()
+    B = (torch.randn(N, r, generator=g) * 0.05).bfloat16()
+    m = qb.nf4_merge_lora(q, A.cuda(), B.cuda(), 0.5, *fmt_out)
+    oc, oa, od, _ = oracle.nf4_merge_lora(q.codes.cpu().numpy(), q.absmax_q.cpu().numpy(), q.dq_scale.cpu().numpy(),
+                                          N, K, bits(A), bits(B), 0.5, *fmt_in, *fmt_out)
+    assert np.array_equal(m.codes.cpu().numpy(), oc), "codes differ"
+    assert np.array_equal(m.absmax_q.cpu().numpy(), oa), "absmax codes differ"
+    assert m.dq_scale.cpu().numpy().tobytes() == od.tobytes(), "scales differ"
+
+
+def test_merge_lora_at_decode_scale(qb, oracle):
+    """The 70B-shaped up projection merged with its r = 16 adapter: sampled
+    rows against the oracle (the merge of a row depends only on that row)."""
+    w = wl.WORKLOADS["decode_70b_up"]
+    p = wl.draw_linear(w, M=1)
+    q = qb.nf4_quantize(p["W"].cuda())
+    m = qb.nf4_merge_lora(q, p["A"].cuda(), p["B"].cuda(), p["scale"])
+    N, K = p["N"], p["K"]
+    rows = np.array([0, 1, 4097, N - 2, N - 1])
+    bpr = K // 64  # blocks per row; 128 per row -> whole double-quant groups are 2 rows
+    for n in rows:
+        n0 = n - n % 2  # the pair of rows that shares a group of 256 blocks
+        sl = slice(n0 * K // 2, (n0 + 2) * K // 2)
+        bs = slice(n0 * bpr, (n0 + 2) * bpr)
+        oc, oa, od, _ = oracle.nf4_merge_lora(q.codes[sl].cpu().numpy(), q.absmax_q[bs].cpu().numpy(),
+                                              q.dq_scale[n0 // 2: n0 // 2 + 1].cpu().numpy(), 2, K,
+                                              bits(p["A"]), bits(p["B"][n0:n0 + 2]), p["scale"])
+        assert np.array_equal(m.codes[sl].cpu().numpy(), oc)
+        assert np.array_equal(m.absmax_q[bs].cpu().numpy(), oa)
+        assert m.dq_scale[n0 // 2: n0 // 2 + 1].cpu().numpy().tobytes() == od.tobytes()
+
+
 def test_noalloc_entry_reads_default_format_only(qb):
     q = qb.nf4_quantize(torch.randn(64, 256, device="cuda") * 0.02, 128, 0)
     X = torch.randn(32, 256, device="cuda").bfloat16()
