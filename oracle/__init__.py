@@ -63,6 +63,7 @@ def _load():
     lib.or_linear_bwd.argtypes = [P, P, i64, i64, P, i64, P, P, ctypes.c_int, ctypes.c_double,
                                   P, i64, P, P, P, P]
     lib.or_num_threads.restype = ctypes.c_int
+    lib.or_linear_fwd_multi.argtypes = [P, i64, i64, P, i64, P, P, ctypes.c_int, ctypes.c_int, P, P, P]
     lib.or_nf4_merge_lora.argtypes = [P, P, P, ctypes.c_int, ctypes.c_int, i64, i64, P, P, ctypes.c_int,
                                       ctypes.c_float, ctypes.c_int, ctypes.c_int, P, P, P, P]
     _lib = lib
@@ -201,6 +202,25 @@ def linear_fwd(X16, Wp32, A16, B16, scale: float, rows=None):
     Y = np.zeros((nrows, N), np.float64)
     _check(lib.or_linear_fwd(_p(X16), M, K, _p(Wp32), N, _p(A16), _p(B16), r, float(scale),
                              _p(rows_a), nrows, _p(Y)), "linear_fwd")
+    return Y
+
+
+def linear_fwd_multi(X16, Wp32, A16_all, B16_all, scales, idx):
+    """Y [M, N] (fp64) of the multi-adapter forward: token m uses adapter
+    idx[m] of A16_all [na, r, K], B16_all [na, N, r] with scale scales[na]."""
+    lib = _load()
+    X16 = _c(X16, np.uint16)
+    Wp32 = _c(Wp32, np.float32)
+    A16_all = _c(A16_all, np.uint16)
+    B16_all = _c(B16_all, np.uint16)
+    sc = _c(np.asarray(scales, np.float64), np.float64)
+    ix = _c(np.asarray(idx, np.int32), np.int32)
+    M, K = X16.shape
+    N = Wp32.shape[0]
+    na, r = A16_all.shape[0], A16_all.shape[1]
+    Y = np.zeros((M, N), np.float64)
+    _check(lib.or_linear_fwd_multi(_p(X16), M, K, _p(Wp32), N, _p(A16_all), _p(B16_all), na, r, _p(sc), _p(ix),
+                                   _p(Y)), "linear_fwd_multi")
     return Y
 
 

@@ -353,6 +353,26 @@ int or_linear_fwd(const uint16_t* X, int64_t M, int64_t K, const float* Wp, int6
     return bad ? OR_ERR_ARG : OR_OK;
 }
 
+/* Multi-adapter forward (f3; "QLoRA and Quantized Fine-Tuning": one frozen
+ * base, many small adapters): token m uses adapter a = idx[m] of a stack,
+ *   Y[m, n] = sum_k X[m,k] Wp[n,k] + s_a * sum_j H[m,j] B_a[n,j],  H = X A_a^T,
+ * A_all bf16 [na, r, K], B_all bf16 [na, N, r], scales fp64 [na], idx [M].
+ * Y is [M, N] fp64.  An index outside [0, na) is an argument error. */
+int or_linear_fwd_multi(const uint16_t* X, int64_t M, int64_t K, const float* Wp, int64_t N,
+                        const uint16_t* A_all, const uint16_t* B_all, int na, int r, const double* scales,
+                        const int32_t* idx, double* Y) {
+    if (!X || !Wp || !A_all || !B_all || !scales || !idx || !Y || r <= 0 || na <= 0) return OR_ERR_ARG;
+    for (int64_t m = 0; m < M; ++m)
+        if (idx[m] < 0 || idx[m] >= na) return OR_ERR_ARG;
+    for (int64_t m = 0; m < M; ++m) {
+        const int a = idx[m];
+        int st = or_linear_fwd(X, M, K, Wp, N, A_all + (int64_t)a * r * K, B_all + (int64_t)a * N * r, r,
+                               scales[a], &m, 1, Y + m * N);
+        if (st) return st;
+    }
+    return OR_OK;
+}
+
 /* Backward (a8 + a9).  With upstream gradient dY [M,N]:
  *   dH[m,j] = s * sum_n dY[m,n] B[n,j]                       [M, r]
  *   dX[m,k] = sum_n dY[m,n] Wp[n,k] + sum_j dH[m,j] A[j,k]   rows listed

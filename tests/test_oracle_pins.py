@@ -444,3 +444,31 @@ def test_merge_matches_real_sum_within_quantization_error(oracle, out_block, out
     amax = np.repeat(np.abs(merged.reshape(-1, out_block)).max(axis=1), out_block).reshape(N, K).astype(np.float64)
     bound = amax * (half_gap + 1.0 / 255) + np.abs(exact) * 2 ** -8 + 1e-30
     assert np.all(np.abs(back - exact) <= bound)
+
+
+# ------------------------------------------------- multi-adapter decode (f3)
+
+
+def test_multi_adapter_forward_reduces_to_single_adapter(oracle):
+    """A stack of adapters with a per-token index: every token's output row is
+    the single-adapter forward with its own adapter and scale, and a uniform
+    index is the single-adapter forward itself."""
+    M, N, K, r, na = 6, 40, 256, 8, 3
+    p = wl.draw_small(41, M, N, K, r, 16.0)
+    codes, aq, dq, _ = oracle.nf4_quantize(p["W"].numpy())
+    _, Wp = oracle.nf4_dequantize(codes, aq, dq, N, K)
+    g = wl.generator(42)
+    A_all = np.stack([wl.bf16_bits((torch.rand(r, K, generator=g) - 0.5).bfloat16()) for _ in range(na)])
+    B_all = np.stack([wl.bf16_bits((torch.randn(N, r, generator=g) * 0.1).bfloat16()) for _ in range(na)])
+    scales = [2.0, 0.5, 4.0]
+    idx = np.array([2, 0, 1, 1, 2, 0], np.int32)
+    X16 = _bits(p["X"])
+    Y = oracle.linear_fwd_multi(X16, Wp, A_all, B_all, scales, idx)
+    for m in range(M):
+        a = idx[m]
+        ref = oracle.linear_fwd(X16, Wp, A_all[a], B_all[a], scales[a], rows=np.array([m]))
+        assert np.array_equal(Y[m], ref[0])
+    Y1 = oracle.linear_fwd_multi(X16, Wp, A_all, B_all, scales, np.ones(M, np.int32))
+    assert np.array_equal(Y1, oracle.linear_fwd(X16, Wp, A_all[1], B_all[1], scales[1]))
+    with pytest.raises(RuntimeError):
+        oracle.linear_fwd_multi(X16, Wp, A_all, B_all, scales, np.array([0, 1, 3, 0, 0, 0], np.int32))
