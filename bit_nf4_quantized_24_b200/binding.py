@@ -63,6 +63,7 @@ def lib():
     L.qlora_linear_fwd_noalloc.argtypes = [P, P, P, i64, i64, P, i64, P, P, i32, f32, P, P, P]
     L.qlora_linear_fwd_fmt.argtypes = [P, P, P, i32, i32, i64, i64, P, i64, P, P, i32, f32, P, P, P, sz, P]
     L.nf4_merge_lora.argtypes = [P, P, P, i32, i32, i64, i64, P, P, i32, f32, i32, i32, P, P, P, P]
+    L.qlora_linear_fwd_multi.argtypes = [P, P, P, i64, i64, P, i64, P, P, i32, i32, P, P, P, P, sz, P]
     L.qlora_linear_bwd_fmt.argtypes = [P, P, P, i32, i32, i64, i64, P, P, i64, P, P, i32, f32, P, P, P, P, P, sz,
                                        P]
     L.qlora_device_status.restype = i32
@@ -232,6 +233,29 @@ def qlora_linear_fwd(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Te
                                       r, float(scale), _ptr(out), _ptr(H), _ptr(ws), ws.numel(), _stream(stream)),
            "qlora_linear_fwd")
     return out, H
+
+
+def qlora_linear_fwd_multi(w: NF4Weight, X: torch.Tensor, A_all: torch.Tensor, B_all: torch.Tensor,
+                           scales: torch.Tensor, adapter_idx: torch.Tensor, out: torch.Tensor | None = None,
+                           workspace: torch.Tensor | None = None, stream=None):
+    """Decode with one adapter per token: Y[m] = X[m] deq(W)^T +
+    scales[a] (X[m] A_a^T) B_a^T, a = adapter_idx[m] (M <= 16)."""
+    w._layer_format()
+    M = X.shape[0]
+    na, r = A_all.shape[0], A_all.shape[1]
+    _req(X, torch.bfloat16, "X", (M, w.K))
+    _req(A_all, torch.bfloat16, "A_all", (na, r, w.K))
+    _req(B_all, torch.bfloat16, "B_all", (na, w.N, r))
+    _req(scales, torch.float32, "scales", (na,))
+    _req(adapter_idx, torch.int32, "adapter_idx", (M,))
+    if out is None:
+        out = torch.empty(M, w.N, dtype=torch.bfloat16, device=X.device)
+    _req(out, torch.bfloat16, "Y", (M, w.N))
+    ws = _workspace(fwd_workspace_bytes(M, w.N, w.K, r), X.device, workspace)
+    _check(lib().qlora_linear_fwd_multi(_ptr(w.codes), _ptr(w.absmax_q), _ptr(w.dq_scale), w.N, w.K, _ptr(X), M,
+                                        _ptr(A_all), _ptr(B_all), na, r, _ptr(scales), _ptr(adapter_idx), _ptr(out),
+                                        _ptr(ws), ws.numel(), _stream(stream)), "qlora_linear_fwd_multi")
+    return out
 
 
 def qlora_linear_bwd(w: NF4Weight, X: torch.Tensor, dY: torch.Tensor, A: torch.Tensor, B: torch.Tensor,

@@ -132,6 +132,61 @@ __global__ void __cluster_dims__(RS_CTAS, 1, 1) __launch_bounds__(RS_WARPS * 32)
   cluster_sync_all();  // peers keep their shared memory until CTA 0 has read it
 }
 
+// ------------------------------------------------ rows, one adapter per token
+//
+// Hs[m, j] = bf16(scales[a] * sum_k X[m, k] A_all[a, j, k]), a = aidx[m], for
+// the multi-adapter decode: every token may use a different A, so there is no
+// shared operand for an MMA.  CTA (m, 8 consecutive j): its 256 threads split
+// the contraction in 8-wide chunks (16-byte loads), then the CTA adds the
+// threads' sums in a fixed order.  An index outside [0, na) gives zeros.
+__global__ void __launch_bounds__(256) k_rows_multi(const uint16_t* __restrict__ X, int K,
+                                                    const uint16_t* __restrict__ A_all, int na, int r,
+                                                    const float* __restrict__ scales,
+                                                    const int32_t* __restrict__ aidx, uint16_t* __restrict__ Hs) {
+  __shared__ float red[8][8];
+  pdl_trigger();
+  pdl_wait();
+  const int m = blockIdx.x, j0 = blockIdx.y * 8;
+  const int a = aidx[m];
+  const bool ok = a >= 0 && a < na;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if (ok) {
+    const uint4* xr = reinterpret_cast<const uint4*>(X + static_cast<int64_t>(m) * K);
+    const uint16_t* ab = A_all + static_cast<int64_t>(a) * r * K;
+    for (int c = threadIdx.x; c < K / 8; c += 256) {
+      const uint4 x = __ldg(xr + c);
+      const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        if (j0 + jj >= r) break;
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(ab + static_cast<int64_t>(j0 + jj) * K) + c);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          acc[jj] = fmaf(__uint_as_float(xw[q] << 16), __uint_as_float(ww[q] << 16), acc[jj]);
+          acc[jj] = fmaf(__uint_as_float(xw[q] & 0xffff0000u), __uint_as_float(ww[q] & 0xffff0000u), acc[jj]);
+        }
+      }
+    }
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc[jj] += __shfl_xor_sync(0xffffffffu, acc[jj], off);
+  if (lane == 0)
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) red[warp][jj] = acc[jj];
+  __syncthreads();
+  if (threadIdx.x < 8 && j0 + static_cast<int>(threadIdx.x) < r) {
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) v += red[w][threadIdx.x];
+    const float sc = ok ? scales[a] : 0.f;
+    Hs[static_cast<int64_t>(m) * r + j0 + threadIdx.x] = static_cast<uint16_t>(bf16x2_bits(sc * v, 0.f));
+  }
+}
+
 // ------------------------------------------------------------------ rows
 //
 // out[m, j] = sum_k P[m, k] Q(j, k) for 16 * CW tokens per CTA over the whole
@@ -482,6 +537,13 @@ cudaError_t launch_rowdot(const uint16_t* P, const uint16_t* Q, int64_t M, int64
     }
   }
   return rows_dispatch<false>(P, Q, M, Kc, R, sa, out16a, sb, out16b, out32, st, pdl);
+}
+
+cudaError_t launch_rows_multi(const uint16_t* X, int64_t M, int64_t K, const uint16_t* A_all, int na, int r,
+                              const float* scales, const int32_t* aidx, uint16_t* Hs, cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  return launch_ex(k_rows_multi, dim3(static_cast<unsigned>(M), static_cast<unsigned>((r + 7) / 8)), dim3(256), 0,
+                   st, false, X, static_cast<int>(K), A_all, na, r, scales, aidx, Hs);
 }
 
 cudaError_t launch_rowdot_qt(const uint16_t* P, const uint16_t* Qt, int64_t M, int64_t Kc, int R, float sa,

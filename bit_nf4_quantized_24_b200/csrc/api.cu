@@ -305,6 +305,28 @@ int qlora_linear_fwd_fmt(const uint8_t* codes, const uint8_t* absmax_q, const fl
   return cuda_status(e);
 }
 
+int qlora_linear_fwd_multi(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale, int64_t N, int64_t K,
+                           const qlora_bf16_t* X, int64_t M, const qlora_bf16_t* A_all, const qlora_bf16_t* B_all,
+                           int n_adapters, int r, const float* scales, const int32_t* adapter_idx, qlora_bf16_t* Y,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  int st = check_layer_shapes(M, N, K, r);
+  if (st) return st;
+  if (M > 16 || n_adapters < 1) return n_adapters < 1 ? QLORA_ERR_ARG : QLORA_ERR_UNSUPPORTED;
+  if (!codes || !absmax_q || !dq_scale || !A_all || !B_all || !scales || (M > 0 && (!X || !Y || !adapter_idx)))
+    return QLORA_ERR_ARG;
+  if (M == 0) return QLORA_OK;
+  const void* ptrs[] = {codes, X, A_all, B_all, Y};
+  for (const void* p : ptrs)
+    if (!aligned(p, 16)) return QLORA_ERR_SHAPE;
+  FwdWorkspace w = fwd_layout(workspace, M, r);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < w.bytes) return QLORA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_rows_multi(X, M, K, A_all, n_adapters, r, scales, adapter_idx, w.Hs, s);
+  if (e == cudaSuccess)
+    e = launch_gemv(X, M, codes, absmax_q, dq_scale, N, K, w.Hs, B_all, r, Y, s, adapter_idx, n_adapters);
+  return cuda_status(e);
+}
+
 int qlora_linear_fwd(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale, int64_t N, int64_t K,
                      const qlora_bf16_t* X, int64_t M, const qlora_bf16_t* A, const qlora_bf16_t* B, int r,
                      float scale, qlora_bf16_t* Y, qlora_bf16_t* H_save, void* workspace, size_t workspace_bytes,

@@ -155,12 +155,16 @@ __device__ __forceinline__ void blocks_mma(float (&acc)[NTILE][4], const BlockIn
     }
 }
 
-template <int NTILE>
+// MULTI: token m uses adapter aidx[m] of a stack (Bl = B_all [na, N, r]; Hs
+// already holds that adapter's scaled H); the epilogue then adds the LoRA
+// term per output with FMAs instead of one MMA shared by all tokens.  A
+// token whose index is outside [0, na) gets no LoRA term.
+template <int NTILE, bool MULTI>
 __global__ void __launch_bounds__(G_THREADS, 1)
     k_gemv(const __grid_constant__ CUtensorMap tm_codes, const uint16_t* __restrict__ X, int M,
            const uint8_t* __restrict__ absmax_q, const float* __restrict__ dq_scale, int N, int K,
            const uint16_t* __restrict__ Hs, const uint16_t* __restrict__ Bl, int r, Nf4Levels lv,
-           uint16_t* __restrict__ Y, int* status) {
+           const int32_t* __restrict__ aidx, int na, uint16_t* __restrict__ Y, int* status) {
   using S = GemvSmem<NTILE>;
   constexpr int NS = S::NS;
   pdl_trigger();
@@ -247,6 +251,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       uint32_t la[4][4], lb[4][NTILE][2];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
+        if (MULTI) break;
         const int j0 = 16 * k;
         la[k][0] = ld2(Bl, n0 + pg, N, j0 + 2 * t);
         la[k][1] = ld2(Bl, n0 + pg + 8, N, j0 + 2 * t);
@@ -271,12 +276,37 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         }
       __syncwarp();
       if (lane == 0) mbar_arrive(rempty0 + 8u * buf);  // partial sums read: the buffer is free
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        if (16 * k >= r) break;
+      if (MULTI) {  // per-token adapters: sum_j Hs[m, j] B_a[n, j] with 8-wide loads
 #pragma unroll
         for (int nt = 0; nt < NTILE; ++nt)
-          mma16816(v[nt], la[k][0], la[k][1], la[k][2], la[k][3], lb[k][nt][0], lb[k][nt][1]);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int m = 8 * nt + 2 * t + (c & 1), n = n0 + pg + 8 * (c >> 1);
+            if (m >= M || n >= N) continue;
+            const int a = __ldg(aidx + m);
+            if (a < 0 || a >= na) continue;
+            const uint4* hp = reinterpret_cast<const uint4*>(Hs + static_cast<int64_t>(m) * r);
+            const uint4* bp = reinterpret_cast<const uint4*>(Bl + (static_cast<int64_t>(a) * N + n) * r);
+            float lora = 0.f;
+            for (int j8 = 0; j8 < r / 8; ++j8) {
+              const uint4 h = __ldg(hp + j8), b = __ldg(bp + j8);
+              const uint32_t hw[4] = {h.x, h.y, h.z, h.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                lora = fmaf(__uint_as_float(hw[q] << 16), __uint_as_float(bw[q] << 16), lora);
+                lora = fmaf(__uint_as_float(hw[q] & 0xffff0000u), __uint_as_float(bw[q] & 0xffff0000u), lora);
+              }
+            }
+            v[nt][c] += lora;
+          }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if (16 * k >= r) break;
+#pragma unroll
+          for (int nt = 0; nt < NTILE; ++nt)
+            mma16816(v[nt], la[k][0], la[k][1], la[k][2], la[k][3], lb[k][nt][0], lb[k][nt][1]);
+        }
       }
 #pragma unroll
       for (int nt = 0; nt < NTILE; ++nt) {
@@ -418,12 +448,12 @@ __global__ void __launch_bounds__(G_THREADS, 1)
   }
 }
 
-template <int NTILE>
+template <int NTILE, bool MULTI>
 cudaError_t gemv_launch(const CUtensorMap& tm, const uint16_t* X, int64_t M, const uint8_t* absmax_q,
                         const float* dq_scale, int64_t N, int64_t K, const uint16_t* Hs, const uint16_t* B, int r,
-                        uint16_t* Y, cudaStream_t st) {
+                        const int32_t* aidx, int na, uint16_t* Y, cudaStream_t st) {
   using S = GemvSmem<NTILE>;
-  cudaError_t e = smem_limit_once<k_gemv<NTILE>>(S::BYTES);
+  cudaError_t e = smem_limit_once<k_gemv<NTILE, MULTI>>(S::BYTES);
   if (e != cudaSuccess) return e;
   const int sms = device_sm_count();
   const int64_t ntiles = (N + G_ROWS - 1) / G_ROWS;
@@ -440,23 +470,27 @@ cudaError_t gemv_launch(const CUtensorMap& tm, const uint16_t* X, int64_t M, con
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_gemv<NTILE>, tm, static_cast<const uint16_t*>(X), int(M), absmax_q, dq_scale,
-                            int(N), int(K), Hs, B, r, host_codebook().levels, Y, device_status_ptr());
+  return cudaLaunchKernelEx(&cfg, k_gemv<NTILE, MULTI>, tm, static_cast<const uint16_t*>(X), int(M), absmax_q,
+                            dq_scale, int(N), int(K), Hs, B, r, host_codebook().levels, aidx, na, Y,
+                            device_status_ptr());
 }
 
 }  // namespace
 
 cudaError_t launch_gemv(const uint16_t* X, int64_t M, const uint8_t* codes, const uint8_t* absmax_q,
                         const float* dq_scale, int64_t N, int64_t K, const uint16_t* Hs, const uint16_t* B, int r,
-                        uint16_t* Y, cudaStream_t st) {
+                        uint16_t* Y, cudaStream_t st, const int32_t* aidx, int na) {
   if (M == 0 || N == 0) return cudaSuccess;
   if (M > 16 || r > 64 || N * (K / 64) >= (int64_t(1) << 31)) return cudaErrorInvalidValue;  // 32-bit block index
   CUtensorMap tm;
   if (!make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, 128, G_ROWS,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  return M <= 8 ? gemv_launch<1>(tm, X, M, absmax_q, dq_scale, N, K, Hs, B, r, Y, st)
-                : gemv_launch<2>(tm, X, M, absmax_q, dq_scale, N, K, Hs, B, r, Y, st);
+  if (aidx)
+    return M <= 8 ? gemv_launch<1, true>(tm, X, M, absmax_q, dq_scale, N, K, Hs, B, r, aidx, na, Y, st)
+                  : gemv_launch<2, true>(tm, X, M, absmax_q, dq_scale, N, K, Hs, B, r, aidx, na, Y, st);
+  return M <= 8 ? gemv_launch<1, false>(tm, X, M, absmax_q, dq_scale, N, K, Hs, B, r, nullptr, 0, Y, st)
+                : gemv_launch<2, false>(tm, X, M, absmax_q, dq_scale, N, K, Hs, B, r, nullptr, 0, Y, st);
 }
 
 }  // namespace qn

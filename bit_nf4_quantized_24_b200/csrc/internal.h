@@ -90,7 +90,11 @@ cudaError_t launch_rowdot_qt(const uint16_t* P, const uint16_t* Qt, int64_t M, i
 // ----- decode GEMV (M <= 16): Y = X deq(W)^T + Hs B^T, Hs = bf16(s X A^T)
 cudaError_t launch_gemv(const uint16_t* X, int64_t M, const uint8_t* codes, const uint8_t* absmax_q,
                         const float* dq_scale, int64_t N, int64_t K, const uint16_t* Hs, const uint16_t* B, int r,
-                        uint16_t* Y, cudaStream_t st);
+                        uint16_t* Y, cudaStream_t st, const int32_t* aidx = nullptr, int na = 0);
+// Multi-adapter Hs for the decode kernel: Hs[m, j] = bf16(scales[a] *
+// sum_k X[m, k] A_all[a, j, k]) with a = aidx[m] (0 when a is outside [0, na)).
+cudaError_t launch_rows_multi(const uint16_t* X, int64_t M, int64_t K, const uint16_t* A_all, int na, int r,
+                              const float* scales, const int32_t* aidx, uint16_t* Hs, cudaStream_t st);
 
 // ----- per-device launch setup, done once per device and kernel
 

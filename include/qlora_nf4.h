@@ -171,6 +171,22 @@ int qlora_linear_fwd_fmt(const uint8_t* codes, const uint8_t* absmax_q, const fl
                          qlora_bf16_t* H_save, void* workspace, size_t workspace_bytes,
                          void* stream);
 
+/* Multi-adapter decode (one frozen NF4 base serving many adapters;
+ * "QLoRA and Quantized Fine-Tuning", "The two mechanisms combined"): token m
+ * uses adapter a = adapter_idx[m] of a stack,
+ *     Y[m] = X[m] deq(W)^T + scales[a] * (X[m] A_a^T) B_a^T.
+ * A_all: bf16 [n_adapters, r, K]; B_all: bf16 [n_adapters, N, r];
+ * scales: device fp32 [n_adapters]; adapter_idx: device int32 [M].  A token
+ * whose index is outside [0, n_adapters) gets no LoRA term.  M <= 16 (the
+ * decode kernel; larger M: QLORA_ERR_UNSUPPORTED); the default NF4 format.
+ * workspace: qlora_linear_fwd_workspace(M, N, K, r) bytes.  Same shape rules
+ * and errors as qlora_linear_fwd. */
+int qlora_linear_fwd_multi(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale,
+                           int64_t N, int64_t K, const qlora_bf16_t* X, int64_t M,
+                           const qlora_bf16_t* A_all, const qlora_bf16_t* B_all, int n_adapters,
+                           int r, const float* scales, const int32_t* adapter_idx, qlora_bf16_t* Y,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
 /* Backward of the QLoRA linear: gradients flow through deq(W) to the
  * adapters and to the input; the frozen base gets none (katajob, "What stays
  * in full precision"):

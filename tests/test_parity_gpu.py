@@ -220,6 +220,36 @@ def test_merge_lora_at_decode_scale(qb, oracle):
         assert m.dq_scale[n0 // 2: n0 // 2 + 1].cpu().numpy().tobytes() == od.tobytes()
 
 
+@pytest.mark.parametrize("M,r", [(1, 16), (5, 64), (12, 16), (16, 64)])
+def test_multi_adapter_decode(qb, oracle, M, r):
+    """Decode with a stack of 3 adapters and a per-token index against the
+    oracle's multi-adapter forward; a token with an index outside the stack
+    gets the base output only."""
+    N, K, na = 1000, 2048, 3
+    p = wl.draw_small(900 + M + r, M, N, K, r, 2.0 * r, with_dy=False)
+    q, Wp = quantize_both(qb, oracle, p["W"])
+    g = wl.generator(950 + M)
+    A_all = ((torch.rand(na, r, K, generator=g) * 2 - 1) / np.sqrt(K)).bfloat16()
+    B_all = (torch.randn(na, N, r, generator=g) * 0.5).bfloat16()
+    scales = torch.tensor([2.0, 0.5, 4.0], dtype=torch.float32)
+    idx = torch.tensor([(3 * m + 1) % na for m in range(M)], dtype=torch.int32)
+    bad = M > 3
+    if bad:
+        idx[3] = 7  # outside the stack: no LoRA term
+    Y = qb.qlora_linear_fwd_multi(q, p["X"].cuda(), A_all.cuda(), B_all.cuda(), scales.cuda(), idx.cuda())
+    torch.cuda.synchronize()
+    X16 = bits(p["X"])
+    ref_idx = idx.numpy().copy()
+    if bad:
+        ref_idx[3] = 0
+    Yref = oracle.linear_fwd_multi(X16, Wp, bits(A_all), bits(B_all), scales.double().numpy(), ref_idx)
+    if bad:
+        zeroB = np.zeros((N, r), np.uint16)
+        Yref[3] = oracle.linear_fwd(X16, Wp, bits(A_all[0]), zeroB, 1.0, rows=np.array([3]))[0]
+    e = relfro(Y.float().cpu().numpy(), Yref)
+    assert e <= TOL, f"Y rel err {e}"
+
+
 def test_noalloc_entry_reads_default_format_only(qb):
     q = qb.nf4_quantize(torch.randn(64, 256, device="cuda") * 0.02, 128, 0)
     X = torch.randn(32, 256, device="cuda").bfloat16()
