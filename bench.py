@@ -413,6 +413,31 @@ def run_extras(qb, wl, dev, pk, flush):
                         "total_gbs": round(total_bytes / ms / 1e6, 1),
                         "frac_hbm": round(total_bytes / ms / 1e6 / pk["hbm_gbs"], 4)}
     res["decode_70b_up"] = dec
+    # multi-adapter decode: 16 tokens spread over 4 adapters (r = 16), graph replay
+    na, Mm = 4, 16
+    g = torch.Generator().manual_seed(77)
+    A_all = ((torch.rand(na, r, K, generator=g) * 2 - 1) / K ** 0.5).bfloat16().to(dev)
+    B_all = (torch.randn(na, N, r, generator=g) * 0.01).bfloat16().to(dev)
+    sc_all = torch.full((na,), float(s), dtype=torch.float32, device=dev)
+    idx = (torch.arange(Mm, dtype=torch.int32) % na).to(dev)
+    Xm = p["X"][:Mm].contiguous().to(dev)
+    Ym = torch.empty(Mm, N, dtype=torch.bfloat16, device=dev)
+    wsm = torch.empty(qb.fwd_workspace_bytes(Mm, N, K, r), dtype=torch.uint8, device=dev)
+    callm = lambda: qb.qlora_linear_fwd_multi(q, Xm, A_all, B_all, sc_all, idx, out=Ym, workspace=wsm)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        callm()
+    torch.cuda.current_stream().wait_stream(side)
+    graph_m = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_m):
+        callm()
+    ms = timed(graph_m.replay)
+    mbytes = weight_bytes + 2 * na * r * (K + N) + 2 * Mm * (K + N)
+    res["decode_70b_up_multi_adapter"] = {"tokens": Mm, "adapters": na, "us": round(ms * 1e3, 2),
+                                          "total_gbs": round(mbytes / ms / 1e6, 1),
+                                          "frac_hbm": round(mbytes / ms / 1e6 / pk["hbm_gbs"], 4)}
+    del graph_m
     # quantize of the same weight (4 B read + 0.516 B written per weight)
     numel = N * K
     qbytes = 4 * numel + numel // 2 + numel // 64 + 4 * ((numel // 64 + 255) // 256)
