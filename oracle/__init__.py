@@ -63,6 +63,7 @@ def _load():
     lib.or_linear_bwd.argtypes = [P, P, i64, i64, P, i64, P, P, ctypes.c_int, ctypes.c_double,
                                   P, i64, P, P, P, P]
     lib.or_num_threads.restype = ctypes.c_int
+    lib.or_dropout_input.argtypes = [P, P, ctypes.c_float, i64, P]
     lib.or_linear_fwd_multi.argtypes = [P, i64, i64, P, i64, P, P, ctypes.c_int, ctypes.c_int, P, P, P]
     lib.or_nf4_merge_lora.argtypes = [P, P, P, ctypes.c_int, ctypes.c_int, i64, i64, P, P, ctypes.c_int,
                                       ctypes.c_float, ctypes.c_int, ctypes.c_int, P, P, P, P]
@@ -203,6 +204,47 @@ def linear_fwd(X16, Wp32, A16, B16, scale: float, rows=None):
     _check(lib.or_linear_fwd(_p(X16), M, K, _p(Wp32), N, _p(A16), _p(B16), r, float(scale),
                              _p(rows_a), nrows, _p(Y)), "linear_fwd")
     return Y
+
+
+def dropout_input(X16, mask, keep: float):
+    """Xd = mask ? bf16(fl32(X * keep)) : 0, as bf16 bits (mask: 1 = keep)."""
+    lib = _load()
+    X16 = _c(X16, np.uint16)
+    mask = _c(mask, np.uint8)
+    Xd = np.zeros(X16.shape, np.uint16)
+    _check(lib.or_dropout_input(_p(X16), _p(mask), float(keep), X16.size, _p(Xd)), "dropout_input")
+    return Xd
+
+
+def _bf16_to_f64(b):
+    return (np.asarray(b, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def linear_fwd_dropout(X16, mask, keep, Wp32, A16, B16, scale: float, rows=None):
+    """Y with LoRA dropout on the adapter input: the base product uses X, the
+    adapter uses Xd = dropout_input(X) (fp64, library matmuls as steps)."""
+    B0 = np.zeros_like(_c(B16, np.uint16))
+    Y = linear_fwd(X16, Wp32, A16, B0, scale, rows=rows)        # base only
+    Xd = _bf16_to_f64(dropout_input(X16, mask, keep))
+    if rows is not None:
+        Xd = Xd[rows]
+    H = Xd @ _bf16_to_f64(A16).T
+    return Y + scale * (H @ _bf16_to_f64(B16).T)
+
+
+def linear_bwd_dropout(X16, mask, keep, dY16, Wp32, A16, B16, scale: float):
+    """(dX, dA, dB) with LoRA dropout: dH = s dY B, H = Xd A^T,
+    dX = dY Wp + (dH A) * mask * keep, dA = dH^T Xd, dB = s dY^T H."""
+    B0 = np.zeros_like(_c(B16, np.uint16))
+    dX, _, _, _ = linear_bwd(X16, dY16, Wp32, A16, B0, scale)   # dY Wp (the adapter term is added below)
+    Xd = _bf16_to_f64(dropout_input(X16, mask, keep))
+    A = _bf16_to_f64(A16)
+    B = _bf16_to_f64(B16)
+    dY = _bf16_to_f64(dY16)
+    dH = scale * (dY @ B)
+    dX = dX + (dH @ A) * (np.asarray(mask, np.float64) * float(np.float32(keep)))
+    H = Xd @ A.T
+    return dX, dH.T @ Xd, scale * (dY.T @ H)
 
 
 def linear_fwd_multi(X16, Wp32, A16_all, B16_all, scales, idx):

@@ -298,6 +298,21 @@ int or_nf4_merge_lora(const uint8_t* codes, const uint8_t* absmax_q, const float
     return st;
 }
 
+/* ------------------------------------------------ LoRA dropout input (f4) */
+
+/* The adapter branch sees dropout(X) ("QLoRA: fine-tuning a large model on
+ * one GPU": lora_dropout in the LoraConfig): Xd = X * keep where the mask
+ * keeps the element, else 0, rounded to bf16 like any bf16 product:
+ *   Xd[i] = mask[i] ? bf16_rne(fl32(X[i] * keep)) : 0.
+ * The random draw is an input (mask, 1 = keep); keep = 1 / (1 - p). */
+int or_dropout_input(const uint16_t* X, const uint8_t* mask, float keep, int64_t n, uint16_t* Xd) {
+    if (!X || !mask || !Xd || n < 0) return OR_ERR_ARG;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i)
+        Xd[i] = mask[i] ? f32_to_bf16_rne(r32(bf16_to_f64(X[i]) * (double)keep)) : (uint16_t)0;
+    return OR_OK;
+}
+
 /* bf16 rounding exposed for the tests that pin it against textbook values. */
 uint16_t or_f32_to_bf16(float f) { return f32_to_bf16_rne(f); }
 

@@ -472,3 +472,71 @@ def test_multi_adapter_forward_reduces_to_single_adapter(oracle):
     assert np.array_equal(Y1, oracle.linear_fwd(X16, Wp, A_all[1], B_all[1], scales[1]))
     with pytest.raises(RuntimeError):
         oracle.linear_fwd_multi(X16, Wp, A_all, B_all, scales, np.array([0, 1, 3, 0, 0, 0], np.int32))
+
+
+# ------------------------------------------------------ LoRA dropout (f4)
+
+
+def _dropout_case(oracle, seed=51, M=10, N=24, K=128, r=8):
+    p = _small(seed, M, N, K, r)
+    codes, aq, dq, _ = oracle.nf4_quantize(p["W"].numpy())
+    _, Wp = oracle.nf4_dequantize(codes, aq, dq, N, K)
+    return p, Wp
+
+
+def test_dropout_input_rounding(oracle):
+    """Xd = mask ? bf16(fl32(x * keep)) : 0: keep = 2 scales exactly, a kept
+    element of 1.0 times 1/(1-0.1) rounds to the bf16 nearest fl32(1/0.9)."""
+    X = np.array([0x3F80, 0xC040, 0x3F80, 0x0000], np.uint16)  # 1, -3, 1, 0
+    m = np.array([1, 1, 0, 1], np.uint8)
+    Xd = oracle.dropout_input(X, m, 2.0)
+    assert list(Xd) == [0x4000, 0xC0C0, 0, 0]                  # 2, -6, 0, 0
+    keep = float(np.float32(1.0 / 0.9))
+    Xd = oracle.dropout_input(X[:1], np.ones(1, np.uint8), keep)
+    want = torch.tensor([np.float32(keep)]).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert Xd[0] == want[0]
+
+
+def test_dropout_keep_all_is_the_plain_layer(oracle):
+    p, Wp = _dropout_case(oracle)
+    X16, A16, B16, dY16 = _bits(p["X"]), _bits(p["A"]), _bits(p["B"]), _bits(p["dY"])
+    ones = np.ones(X16.shape, np.uint8)
+    Y = oracle.linear_fwd_dropout(X16, ones, 1.0, Wp, A16, B16, p["scale"])
+    assert np.allclose(Y, oracle.linear_fwd(X16, Wp, A16, B16, p["scale"]), rtol=1e-12, atol=1e-12)
+    dX, dA, dB = oracle.linear_bwd_dropout(X16, ones, 1.0, dY16, Wp, A16, B16, p["scale"])
+    rX, rA, rB, _ = oracle.linear_bwd(X16, dY16, Wp, A16, B16, p["scale"])
+    for a, b in ((dX, rX), (dA, rA), (dB, rB)):
+        assert np.allclose(a, b, rtol=1e-12, atol=1e-12)
+
+
+def test_dropout_drop_all_removes_the_adapter(oracle):
+    p, Wp = _dropout_case(oracle)
+    X16, A16, B16, dY16 = _bits(p["X"]), _bits(p["A"]), _bits(p["B"]), _bits(p["dY"])
+    zeros = np.zeros(X16.shape, np.uint8)
+    B0 = np.zeros_like(B16)
+    Y = oracle.linear_fwd_dropout(X16, zeros, 1.25, Wp, A16, B16, p["scale"])
+    assert np.allclose(Y, oracle.linear_fwd(X16, Wp, A16, B0, p["scale"]), rtol=1e-12, atol=1e-12)
+    dX, dA, dB = oracle.linear_bwd_dropout(X16, zeros, 1.25, dY16, Wp, A16, B16, p["scale"])
+    rX, _, _, _ = oracle.linear_bwd(X16, dY16, Wp, A16, B0, p["scale"])
+    assert np.allclose(dX, rX, rtol=1e-12, atol=1e-12)
+    assert not dA.any() and not dB.any()
+
+
+def test_dropout_backward_is_adjoint_of_forward(oracle):
+    """keep = 2 makes Xd = 2 * mask * X exact, so the layer is linear in X and
+    in A; the backward must be its adjoint: <dY, J V> = <dX, V>."""
+    p, Wp = _dropout_case(oracle)
+    M, K = p["X"].shape
+    X16, A16, B16, dY16 = _bits(p["X"]), _bits(p["A"]), _bits(p["B"]), _bits(p["dY"])
+    g = np.random.default_rng(52)
+    mask = (g.random((M, K)) < 0.5).astype(np.uint8)
+    s = p["scale"]
+    dX, dA, dB = oracle.linear_bwd_dropout(X16, mask, 2.0, dY16, Wp, A16, B16, s)
+    dY = oracle._bf16_to_f64(dY16)
+    A, B = oracle._bf16_to_f64(A16), oracle._bf16_to_f64(B16)
+    V = g.standard_normal((M, K))
+    JV = V @ Wp.astype(np.float64).T + s * ((2.0 * mask * V) @ A.T) @ B.T
+    assert np.isclose(np.sum(dY * JV), np.sum(dX * V), rtol=1e-10)
+    Xd = oracle._bf16_to_f64(oracle.dropout_input(X16, mask, 2.0))
+    VA = g.standard_normal(A.shape)
+    assert np.isclose(np.sum(dY * (s * (Xd @ VA.T) @ B.T)), np.sum(dA * VA), rtol=1e-10)
