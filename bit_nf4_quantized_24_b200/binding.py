@@ -64,6 +64,10 @@ def lib():
     L.qlora_linear_fwd_fmt.argtypes = [P, P, P, i32, i32, i64, i64, P, i64, P, P, i32, f32, P, P, P, sz, P]
     L.nf4_merge_lora.argtypes = [P, P, P, i32, i32, i64, i64, P, P, i32, f32, i32, i32, P, P, P, P]
     L.qlora_linear_fwd_multi.argtypes = [P, P, P, i64, i64, P, i64, P, P, i32, i32, P, P, P, P, sz, P]
+    L.qlora_linear_dropout_workspace.argtypes = [i64, i64, i64, i32, P]
+    L.qlora_linear_fwd_dropout.argtypes = [P, P, P, i64, i64, P, i64, P, P, i32, f32, P, f32, P, P, P, sz, P]
+    L.qlora_linear_bwd_dropout.argtypes = [P, P, P, i64, i64, P, P, i64, P, P, i32, f32, P, f32, P, P, P, P, P, sz,
+                                           P]
     L.qlora_linear_bwd_fmt.argtypes = [P, P, P, i32, i32, i64, i64, P, P, i64, P, P, i32, f32, P, P, P, P, P, sz,
                                        P]
     L.qlora_device_status.restype = i32
@@ -233,6 +237,56 @@ def qlora_linear_fwd(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Te
                                       r, float(scale), _ptr(out), _ptr(H), _ptr(ws), ws.numel(), _stream(stream)),
            "qlora_linear_fwd")
     return out, H
+
+
+def dropout_workspace_bytes(M, N, K, r) -> int:
+    b = ctypes.c_size_t()
+    _check(lib().qlora_linear_dropout_workspace(M, N, K, r, ctypes.byref(b)), "qlora_linear_dropout_workspace")
+    return b.value
+
+
+def qlora_linear_fwd_dropout(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, scale: float,
+                             keep_mask: torch.Tensor, keep_scale: float, save_h: bool = True, out=None,
+                             workspace=None, stream=None):
+    """Forward with LoRA dropout on the adapter input (keep_mask uint8 [M, K],
+    1 = keep; keep_scale = 1 / (1 - p)).  Returns (Y, H) with H = Xd A^T."""
+    w._layer_format()
+    M = X.shape[0]
+    r = A.shape[0]
+    _req(X, torch.bfloat16, "X", (M, w.K))
+    _req(A, torch.bfloat16, "A", (r, w.K))
+    _req(B, torch.bfloat16, "B", (w.N, r))
+    _req(keep_mask, torch.uint8, "keep_mask", (M, w.K))
+    if out is None:
+        out = torch.empty(M, w.N, dtype=torch.bfloat16, device=X.device)
+    H = torch.empty(M, r, dtype=torch.bfloat16, device=X.device) if save_h else None
+    ws = _workspace(dropout_workspace_bytes(M, w.N, w.K, r), X.device, workspace)
+    _check(lib().qlora_linear_fwd_dropout(_ptr(w.codes), _ptr(w.absmax_q), _ptr(w.dq_scale), w.N, w.K, _ptr(X), M,
+                                          _ptr(A), _ptr(B), r, float(scale), _ptr(keep_mask), float(keep_scale),
+                                          _ptr(out), _ptr(H), _ptr(ws), ws.numel(), _stream(stream)),
+           "qlora_linear_fwd_dropout")
+    return out, H
+
+
+def qlora_linear_bwd_dropout(w: NF4Weight, X: torch.Tensor, dY: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
+                             scale: float, keep_mask: torch.Tensor, keep_scale: float, H=None, want_dx=True,
+                             workspace=None, stream=None):
+    """Backward with LoRA dropout; returns (dX or None, dA, dB)."""
+    w._layer_format()
+    M = X.shape[0]
+    r = A.shape[0]
+    _req(X, torch.bfloat16, "X", (M, w.K))
+    _req(dY, torch.bfloat16, "dY", (M, w.N))
+    _req(keep_mask, torch.uint8, "keep_mask", (M, w.K))
+    dX = torch.empty(M, w.K, dtype=torch.bfloat16, device=X.device) if want_dx else None
+    dA = torch.empty(r, w.K, dtype=torch.bfloat16, device=X.device)
+    dB = torch.empty(w.N, r, dtype=torch.bfloat16, device=X.device)
+    ws = _workspace(dropout_workspace_bytes(M, w.N, w.K, r), X.device, workspace)
+    _check(lib().qlora_linear_bwd_dropout(_ptr(w.codes), _ptr(w.absmax_q), _ptr(w.dq_scale), w.N, w.K, _ptr(X),
+                                          _ptr(dY), M, _ptr(A), _ptr(B), r, float(scale), _ptr(keep_mask),
+                                          float(keep_scale), _ptr(H), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws),
+                                          ws.numel(), _stream(stream)), "qlora_linear_bwd_dropout")
+    return dX, dA, dB
 
 
 def qlora_linear_fwd_multi(w: NF4Weight, X: torch.Tensor, A_all: torch.Tensor, B_all: torch.Tensor,

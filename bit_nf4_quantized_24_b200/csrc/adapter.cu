@@ -132,6 +132,74 @@ __global__ void __cluster_dims__(RS_CTAS, 1, 1) __launch_bounds__(RS_WARPS * 32)
   cluster_sync_all();  // peers keep their shared memory until CTA 0 has read it
 }
 
+// ------------------------------------------------------------ LoRA dropout
+//
+// The adapter branch reads dropout(X) (the random draw is an input: mask,
+// 1 = keep, and keep = 1 / (1 - p)):  Xd = mask ? bf16(fl32(x * keep)) : 0.
+// Eight elements per thread (16-byte loads).
+__global__ void __launch_bounds__(256) k_dropout_input(const uint16_t* __restrict__ X,
+                                                       const uint8_t* __restrict__ mask, float keep, int64_t n8,
+                                                       uint16_t* __restrict__ Xd) {
+  pdl_trigger();
+  pdl_wait();
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const uint4 x = __ldg(reinterpret_cast<const uint4*>(X) + i);
+  const uint2 mk = __ldg(reinterpret_cast<const uint2*>(mask) + i);
+  const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t mw = q < 2 ? mk.x : mk.y;
+    const int sh = 16 * (q & 1);
+    const float lo = ((mw >> sh) & 0xffu) ? __fmul_rn(__uint_as_float(xw[q] << 16), keep) : 0.f;
+    const float hi = ((mw >> (sh + 8)) & 0xffu) ? __fmul_rn(__uint_as_float(xw[q] & 0xffff0000u), keep) : 0.f;
+    o[q] = bf16x2_bits(lo, hi);
+  }
+  reinterpret_cast<uint4*>(Xd)[i] = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// dX += mask * keep * (dH A): the adapter's part of the input gradient under
+// dropout, added to the base gradient dY deq(W) the GEMM left in dX.  Per
+// element: t = fl32(sum_j dH[m, j] A[j, k]) (j in order), then
+// dX = bf16(fl32(dX) + fl32(t * keep)) where the mask keeps k.  Eight
+// consecutive k of one row per thread.
+__global__ void __launch_bounds__(256) k_dx_add_masked(uint16_t* __restrict__ dX, const uint16_t* __restrict__ dH,
+                                                       const uint16_t* __restrict__ A,
+                                                       const uint8_t* __restrict__ mask, float keep, int64_t M,
+                                                       int64_t K, int r) {
+  pdl_trigger();
+  pdl_wait();
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // 8-element chunk
+  if (i >= M * K / 8) return;
+  const int64_t m = (8 * i) / K, k0 = 8 * i - m * K;
+  float t[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  const uint16_t* hr = dH + m * r;
+  for (int j = 0; j < r; ++j) {
+    const float h = __uint_as_float(static_cast<uint32_t>(hr[j]) << 16);
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(A + static_cast<int64_t>(j) * K + k0));
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      t[2 * q] = fmaf(h, __uint_as_float(aw[q] << 16), t[2 * q]);
+      t[2 * q + 1] = fmaf(h, __uint_as_float(aw[q] & 0xffff0000u), t[2 * q + 1]);
+    }
+  }
+  uint4 d = reinterpret_cast<const uint4*>(dX)[i];
+  const uint2 mk = __ldg(reinterpret_cast<const uint2*>(mask) + i);
+  uint32_t dw[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t mw = q < 2 ? mk.x : mk.y;
+    const int sh = 16 * (q & 1);
+    float lo = __uint_as_float(dw[q] << 16), hi = __uint_as_float(dw[q] & 0xffff0000u);
+    if ((mw >> sh) & 0xffu) lo = __fadd_rn(lo, __fmul_rn(t[2 * q], keep));
+    if ((mw >> (sh + 8)) & 0xffu) hi = __fadd_rn(hi, __fmul_rn(t[2 * q + 1], keep));
+    dw[q] = bf16x2_bits(lo, hi);
+  }
+  reinterpret_cast<uint4*>(dX)[i] = make_uint4(dw[0], dw[1], dw[2], dw[3]);
+}
+
 // ------------------------------------------------ rows, one adapter per token
 //
 // Hs[m, j] = bf16(scales[a] * sum_k X[m, k] A_all[a, j, k]), a = aidx[m], for
@@ -537,6 +605,22 @@ cudaError_t launch_rowdot(const uint16_t* P, const uint16_t* Q, int64_t M, int64
     }
   }
   return rows_dispatch<false>(P, Q, M, Kc, R, sa, out16a, sb, out16b, out32, st, pdl);
+}
+
+cudaError_t launch_dropout_input(const uint16_t* X, const uint8_t* mask, float keep, int64_t n, uint16_t* Xd,
+                                 cudaStream_t st, bool pdl) {
+  const int64_t n8 = n / 8;
+  if (n8 == 0) return cudaSuccess;
+  return launch_ex(k_dropout_input, dim3(static_cast<unsigned>((n8 + 255) / 256)), dim3(256), 0, st, pdl, X, mask,
+                   keep, n8, Xd);
+}
+
+cudaError_t launch_dx_add_masked(uint16_t* dX, const uint16_t* dH, const uint16_t* A, const uint8_t* mask, float keep,
+                                 int64_t M, int64_t K, int r, cudaStream_t st, bool pdl) {
+  const int64_t n8 = M * K / 8;
+  if (n8 == 0) return cudaSuccess;
+  return launch_ex(k_dx_add_masked, dim3(static_cast<unsigned>((n8 + 255) / 256)), dim3(256), 0, st, pdl, dX, dH, A,
+                   mask, keep, M, K, r);
 }
 
 cudaError_t launch_rows_multi(const uint16_t* X, int64_t M, int64_t K, const uint16_t* A_all, int na, int r,

@@ -82,6 +82,25 @@ int check_layer_shapes(int64_t M, int64_t N, int64_t K, int r) {
   return QLORA_OK;
 }
 
+// Scratch of the dropout variants: Xd [M, K] bf16 and a zero [M, r] bf16
+// tail (the dX GEMM then adds no adapter term; k_dx_add_masked does, masked).
+struct DropWorkspace {
+  uint16_t* Xd;
+  uint16_t* zero_tail;
+  size_t bytes;
+};
+DropWorkspace drop_layout(void* ws, size_t off0, int64_t M, int64_t K, int r) {
+  DropWorkspace w{};
+  size_t off = (off0 + 255) & ~size_t(255);
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  w.Xd = p ? reinterpret_cast<uint16_t*>(p + off) : nullptr;
+  off += (static_cast<size_t>(M) * K * 2 + 255) & ~size_t(255);
+  w.zero_tail = p ? reinterpret_cast<uint16_t*>(p + off) : nullptr;
+  off += (static_cast<size_t>(M) * r * 2 + 255) & ~size_t(255);
+  w.bytes = off;
+  return w;
+}
+
 // The NF4 formats the layer reads: block in {32, 64, 128, 256}, dq_block 256 or 0.
 int check_format(int64_t K, int block, int dq_block) {
   if ((block != 32 && block != 64 && block != 128 && block != 256) || (dq_block != 256 && dq_block != 0))
@@ -324,6 +343,117 @@ int qlora_linear_fwd_multi(const uint8_t* codes, const uint8_t* absmax_q, const 
   cudaError_t e = launch_rows_multi(X, M, K, A_all, n_adapters, r, scales, adapter_idx, w.Hs, s);
   if (e == cudaSuccess)
     e = launch_gemv(X, M, codes, absmax_q, dq_scale, N, K, w.Hs, B_all, r, Y, s, adapter_idx, n_adapters);
+  return cuda_status(e);
+}
+
+int qlora_linear_dropout_workspace(int64_t M, int64_t N, int64_t K, int r, size_t* bytes) {
+  if (!bytes) return QLORA_ERR_ARG;
+  int st = check_layer_shapes(M, N, K, r);
+  if (st) return st;
+  const size_t base = std::max(fwd_layout(nullptr, M, r).bytes, bwd_layout(nullptr, M, N, K, r).bytes);
+  *bytes = drop_layout(nullptr, base, M, K, r).bytes;
+  return QLORA_OK;
+}
+
+int qlora_linear_fwd_dropout(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale, int64_t N,
+                             int64_t K, const qlora_bf16_t* X, int64_t M, const qlora_bf16_t* A, const qlora_bf16_t* B,
+                             int r, float scale, const uint8_t* keep_mask, float keep_scale, qlora_bf16_t* Y,
+                             qlora_bf16_t* H_save, void* workspace, size_t workspace_bytes, void* stream) {
+  int st = check_layer_shapes(M, N, K, r);
+  if (st) return st;
+  if (!codes || !absmax_q || !dq_scale || !A || !B || (M > 0 && (!X || !Y || !keep_mask))) return QLORA_ERR_ARG;
+  if (!std::isfinite(scale) || !std::isfinite(keep_scale)) return QLORA_ERR_ARG;
+  if (M == 0) return QLORA_OK;
+  const void* ptrs[] = {codes, X, A, B, Y, keep_mask};
+  for (const void* p : ptrs)
+    if (!aligned(p, 16)) return QLORA_ERR_SHAPE;
+  if (H_save && !aligned(H_save, 16)) return QLORA_ERR_SHAPE;
+  FwdWorkspace w = fwd_layout(workspace, M, r);
+  const size_t base = std::max(w.bytes, bwd_layout(nullptr, M, N, K, r).bytes);
+  DropWorkspace d = drop_layout(workspace, base, M, K, r);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < d.bytes) return QLORA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // H from the dropped-out input; the base product from X itself
+  cudaError_t e = launch_dropout_input(X, keep_mask, keep_scale, M * K, d.Xd, s, false);
+  if (e == cudaSuccess) e = launch_rowdot(d.Xd, A, M, K, r, scale, w.Hs, 1.0f, H_save, nullptr, s, true);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (M <= 16) {
+    e = launch_gemv(X, M, codes, absmax_q, dq_scale, N, K, w.Hs, B, r, Y, s);
+  } else {
+    GemmArgs a{};
+    a.mode = 0;
+    a.act = X;
+    a.tail_a = w.Hs;
+    a.tail_b = B;
+    a.codes = codes;
+    a.absmax_q = absmax_q;
+    a.dq_scale = dq_scale;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.r = r;
+    a.out = Y;
+    a.pdl = true;
+    e = launch_nf4_gemm(a, s);
+  }
+  return cuda_status(e);
+}
+
+int qlora_linear_bwd_dropout(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale, int64_t N,
+                             int64_t K, const qlora_bf16_t* X, const qlora_bf16_t* dY, int64_t M, const qlora_bf16_t* A,
+                             const qlora_bf16_t* B, int r, float scale, const uint8_t* keep_mask, float keep_scale,
+                             const qlora_bf16_t* H, qlora_bf16_t* dX, qlora_bf16_t* dA, qlora_bf16_t* dB,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  int st = check_layer_shapes(M, N, K, r);
+  if (st) return st;
+  if (!codes || !absmax_q || !dq_scale || !A || !B || !dA || !dB || (M > 0 && (!X || !dY || !keep_mask)))
+    return QLORA_ERR_ARG;
+  if (!std::isfinite(scale) || !std::isfinite(keep_scale)) return QLORA_ERR_ARG;
+  const void* ptrs[] = {codes, A, B, dA, dB};
+  for (const void* p : ptrs)
+    if (!aligned(p, 16)) return QLORA_ERR_SHAPE;
+  if ((X && !aligned(X, 16)) || (dY && !aligned(dY, 16)) || (dX && !aligned(dX, 16)) || (H && !aligned(H, 16)) ||
+      (keep_mask && !aligned(keep_mask, 16)))
+    return QLORA_ERR_SHAPE;
+  BwdWorkspace w = bwd_layout(workspace, M, N, K, r);
+  const size_t base = std::max(fwd_layout(nullptr, M, r).bytes, w.bytes);
+  DropWorkspace d = drop_layout(workspace, base, M, K, r);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < d.bytes) return QLORA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  if (M == 0) {
+    e = cudaMemsetAsync(dA, 0, static_cast<size_t>(r) * K * 2, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dB, 0, static_cast<size_t>(N) * r * 2, s);
+    return cuda_status(e);
+  }
+  if (dX) e = cudaMemsetAsync(d.zero_tail, 0, static_cast<size_t>(M) * r * 2, s);
+  if (e == cudaSuccess) e = launch_dropout_input(X, keep_mask, keep_scale, M * K, d.Xd, s, false);
+  if (e == cudaSuccess) e = launch_rowdot_qt(dY, B, M, N, r, scale, w.dH16, scale, nullptr, nullptr, s, true);
+  const uint16_t* Huse = H;
+  if (e == cudaSuccess && !H) {
+    e = launch_rowdot(d.Xd, A, M, K, r, 1.0f, w.H16, 1.0f, nullptr, nullptr, s, true);
+    Huse = w.H16;
+  }
+  if (e == cudaSuccess) e = launch_coldot(w.dH16, d.Xd, M, K, r, 1.0f, 0, dA, s, true);
+  if (e == cudaSuccess) e = launch_coldot(Huse, dY, M, N, r, scale, 1, dB, s, true);
+  if (e == cudaSuccess && dX) {  // dY deq(W) with a zero adapter tail, then the masked adapter term
+    GemmArgs a{};
+    a.mode = 1;
+    a.act = dY;
+    a.tail_a = d.zero_tail;
+    a.tail_b = A;
+    a.codes = codes;
+    a.absmax_q = absmax_q;
+    a.dq_scale = dq_scale;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.r = r;
+    a.out = dX;
+    a.pdl = true;
+    e = launch_nf4_gemm(a, s);
+    if (e == cudaSuccess) e = launch_dx_add_masked(dX, w.dH16, A, keep_mask, keep_scale, M, K, r, s, true);
+  }
   return cuda_status(e);
 }
 

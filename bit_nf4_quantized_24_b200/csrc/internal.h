@@ -91,6 +91,12 @@ cudaError_t launch_rowdot_qt(const uint16_t* P, const uint16_t* Qt, int64_t M, i
 cudaError_t launch_gemv(const uint16_t* X, int64_t M, const uint8_t* codes, const uint8_t* absmax_q,
                         const float* dq_scale, int64_t N, int64_t K, const uint16_t* Hs, const uint16_t* B, int r,
                         uint16_t* Y, cudaStream_t st, const int32_t* aidx = nullptr, int na = 0);
+// LoRA dropout: Xd = mask ? bf16(fl32(X * keep)) : 0 over n elements (n % 8 == 0,
+// 16-byte aligned); dX += mask * keep * (dH A) (see adapter.cu).
+cudaError_t launch_dropout_input(const uint16_t* X, const uint8_t* mask, float keep, int64_t n, uint16_t* Xd,
+                                 cudaStream_t st, bool pdl);
+cudaError_t launch_dx_add_masked(uint16_t* dX, const uint16_t* dH, const uint16_t* A, const uint8_t* mask, float keep,
+                                 int64_t M, int64_t K, int r, cudaStream_t st, bool pdl);
 // Multi-adapter Hs for the decode kernel: Hs[m, j] = bf16(scales[a] *
 // sum_k X[m, k] A_all[a, j, k]) with a = aidx[m] (0 when a is outside [0, na)).
 cudaError_t launch_rows_multi(const uint16_t* X, int64_t M, int64_t K, const uint16_t* A_all, int na, int r,

@@ -214,6 +214,31 @@ int qlora_linear_bwd_fmt(const uint8_t* codes, const uint8_t* absmax_q, const fl
                          const qlora_bf16_t* H, qlora_bf16_t* dX, qlora_bf16_t* dA,
                          qlora_bf16_t* dB, void* workspace, size_t workspace_bytes, void* stream);
 
+/* LoRA dropout on the adapter input ("QLoRA: fine-tuning a large model on one
+ * GPU": lora_dropout in the LoraConfig).  The adapter branch reads
+ *     Xd = keep_mask ? bf16(fl32(X * keep_scale)) : 0
+ * (keep_mask: device uint8 [M, K], 1 = keep, the caller's random draw;
+ * keep_scale = 1 / (1 - p)); the base product reads X itself:
+ *     Y  = X deq(W)^T + scale * (Xd A^T) B^T
+ *     dX = dY deq(W) + keep_mask * keep_scale * (dH A),  dH = scale * dY B
+ *     dA = dH^T Xd,  dB = scale * dY^T H,  H = Xd A^T  (H_save / H hold it).
+ * workspace: qlora_linear_dropout_workspace bytes (shared by both calls).
+ * Shapes, format and errors as qlora_linear_fwd / qlora_linear_bwd; keep_mask
+ * 16-byte aligned. */
+int qlora_linear_dropout_workspace(int64_t M, int64_t N, int64_t K, int r, size_t* bytes);
+int qlora_linear_fwd_dropout(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale,
+                             int64_t N, int64_t K, const qlora_bf16_t* X, int64_t M,
+                             const qlora_bf16_t* A, const qlora_bf16_t* B, int r, float scale,
+                             const uint8_t* keep_mask, float keep_scale, qlora_bf16_t* Y,
+                             qlora_bf16_t* H_save, void* workspace, size_t workspace_bytes,
+                             void* stream);
+int qlora_linear_bwd_dropout(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale,
+                             int64_t N, int64_t K, const qlora_bf16_t* X, const qlora_bf16_t* dY,
+                             int64_t M, const qlora_bf16_t* A, const qlora_bf16_t* B, int r,
+                             float scale, const uint8_t* keep_mask, float keep_scale,
+                             const qlora_bf16_t* H, qlora_bf16_t* dX, qlora_bf16_t* dA,
+                             qlora_bf16_t* dB, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Largest M * r that qlora_linear_fwd_noalloc accepts: its fixed device
  * scratch holds this many bf16 values (2 MiB on every device that loads the
  * library, held until the process exits). */

@@ -250,6 +250,34 @@ def test_multi_adapter_decode(qb, oracle, M, r):
     assert e <= TOL, f"Y rel err {e}"
 
 
+@pytest.mark.parametrize("M", [200, 5])
+def test_lora_dropout(qb, oracle, M):
+    """LoRA dropout on the adapter input (p = 0.1, mask drawn on the host):
+    forward through the GEMM (M = 200) or the decode kernel (M = 5), and the
+    backward, against the oracle."""
+    N, K, r = 264, 1024, 16
+    p = wl.draw_small(1100 + M, M, N, K, r, 32.0, b_std=0.5)
+    q, Wp = quantize_both(qb, oracle, p["W"])
+    g = np.random.default_rng(1200 + M)
+    mask = (g.random((M, K)) >= 0.1).astype(np.uint8)
+    keep = float(np.float32(1.0 / 0.9))
+    X, A, B, dY = p["X"].cuda(), p["A"].cuda(), p["B"].cuda(), p["dY"].cuda()
+    mk = torch.from_numpy(mask).cuda()
+    Y, H = qb.qlora_linear_fwd_dropout(q, X, A, B, p["scale"], mk, keep)
+    X16, A16, B16, dY16 = bits(p["X"]), bits(p["A"]), bits(p["B"]), bits(p["dY"])
+    Yref = oracle.linear_fwd_dropout(X16, mask, keep, Wp, A16, B16, p["scale"])
+    assert relfro(Y.float().cpu().numpy(), Yref) <= TOL
+    Href = oracle._bf16_to_f64(oracle.dropout_input(X16, mask, keep)) @ oracle._bf16_to_f64(A16).T
+    assert relfro(H.float().cpu().numpy(), Href) <= TOL
+    dX, dA, dB = qb.qlora_linear_bwd_dropout(q, X, dY, A, B, p["scale"], mk, keep, H=H)
+    rX, rA, rB = oracle.linear_bwd_dropout(X16, mask, keep, dY16, Wp, A16, B16, p["scale"])
+    errs = (relfro(dX.float().cpu().numpy(), rX), relfro(dA.float().cpu().numpy(), rA),
+            relfro(dB.float().cpu().numpy(), rB))
+    assert max(errs) <= TOL, f"dX/dA/dB rel err {errs}"
+    _, dA2, _ = qb.qlora_linear_bwd_dropout(q, X, dY, A, B, p["scale"], mk, keep, want_dx=False)  # H recomputed
+    assert relfro(dA2.float().cpu().numpy(), rA) <= TOL
+
+
 def test_noalloc_entry_reads_default_format_only(qb):
     q = qb.nf4_quantize(torch.randn(64, 256, device="cuda") * 0.02, 128, 0)
     X = torch.randn(32, 256, device="cuda").bfloat16()
