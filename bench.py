@@ -476,6 +476,21 @@ def run_extras(qb, wl, dev, pk, flush):
         fmts.setdefault(f"b{block}_dq{dq}", {})["qproj_fwd_tflops"] = round(flops / ms_f / 1e9, 1)
         del qf
     res["formats"] = fmts
+    # q_proj fwd + bwd with LoRA dropout (p = 0.1, mask drawn once on the host)
+    dY2 = torch.randn(M2, N2, generator=torch.Generator().manual_seed(5)).bfloat16().to(dev)
+    q2 = qb.nf4_quantize(W2)
+    mk = (torch.rand(M2, K2, generator=torch.Generator().manual_seed(6)) >= 0.1).to(torch.uint8).to(dev)
+    keep = 1.0 / 0.9
+    wsd = torch.empty(qb.dropout_workspace_bytes(M2, N2, K2, r2), dtype=torch.uint8, device=dev)
+
+    def drop_step():
+        _, Hd = qb.qlora_linear_fwd_dropout(q2, X2, A2, B2, p2["scale"], mk, keep, out=Y2, workspace=wsd)
+        qb.qlora_linear_bwd_dropout(q2, X2, dY2, A2, B2, p2["scale"], mk, keep, H=Hd, workspace=wsd)
+
+    ms_d = timed(drop_step, n=10)
+    res["qproj_fwd_bwd_lora_dropout"] = {"ms": round(ms_d, 4),
+                                         "tflops": round((4 * M2 * N2 * K2 + 6 * M2 * r2 * (K2 + N2)) / ms_d / 1e9, 1)}
+    del q2, dY2, mk, wsd
     # merge of the decode weight with its r = 16 adapter, quantized again
     # (reads codes + scales + A + B, writes codes + scales)
     mbytes = weight_bytes * 2 + 2 * r * (K + N)
