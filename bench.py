@@ -390,13 +390,8 @@ def run_extras(qb, wl, dev, pk, flush):
     N, K, r, s = p["N"], p["K"], p["r"], p["scale"]
     weight_bytes = q.codes.numel() + q.absmax_q.numel() + 4 * q.dq_scale.numel()
     A, B = p["A"].to(dev), p["B"].to(dev)
-    dec = {}
-    for M in (1, 4, 16):
-        X = p["X"][:M].contiguous().to(dev)
-        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-        ws = torch.empty(qb.fwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
-        # a decode loop issues the call from a CUDA graph: time the replay
-        call = lambda: qb.qlora_linear_fwd(q, X, A, B, s, save_h=False, out=Y, workspace=ws)
+    def graph_time(call):
+        """A decode loop issues the call from a CUDA graph: time the replay."""
         side = torch.cuda.Stream()
         side.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(side):
@@ -406,13 +401,36 @@ def run_extras(qb, wl, dev, pk, flush):
         with torch.cuda.graph(graph):
             call()
         ms = timed(graph.replay)
-        ms_eager = timed(call)
+        del graph
+        return ms
+
+    tiles = qb.nf4_decode_tiles(q)
+    ms_pack = timed(lambda: qb.nf4_decode_tiles(q, out=tiles), n=10)
+    res["nf4_decode_tiles"] = {"ms": round(ms_pack, 4),
+                               "gbs": round(2 * q.codes.numel() / ms_pack / 1e6, 1),
+                               "note": "one-time rearrangement of the codes for the decode calls"}
+    dec, dec_t = {}, {}
+    for M in (1, 4, 16):
+        X = p["X"][:M].contiguous().to(dev)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(qb.fwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
         total_bytes = weight_bytes + 2 * r * (K + N) + 2 * M * (K + N)
+        call = lambda: qb.qlora_linear_fwd(q, X, A, B, s, save_h=False, out=Y, workspace=ws)
+        ms = graph_time(call)
+        ms_eager = timed(call)
         dec[f"M{M}"] = {"us": round(ms * 1e3, 2), "us_eager_call": round(ms_eager * 1e3, 2),
                         "weight_stream_gbs": round(weight_bytes / ms / 1e6, 1),
                         "total_gbs": round(total_bytes / ms / 1e6, 1),
                         "frac_hbm": round(total_bytes / ms / 1e6 / pk["hbm_gbs"], 4)}
+        call_t = lambda: qb.qlora_linear_fwd_tiles(q, tiles, X, A, B, s, save_h=False, out=Y, workspace=ws)
+        ms = graph_time(call_t)
+        ms_eager = timed(call_t)
+        dec_t[f"M{M}"] = {"us": round(ms * 1e3, 2), "us_eager_call": round(ms_eager * 1e3, 2),
+                          "weight_stream_gbs": round(weight_bytes / ms / 1e6, 1),
+                          "total_gbs": round(total_bytes / ms / 1e6, 1),
+                          "frac_hbm": round(total_bytes / ms / 1e6 / pk["hbm_gbs"], 4)}
     res["decode_70b_up"] = dec
+    res["decode_70b_up_tiles"] = dec_t
     # multi-adapter decode: 16 tokens spread over 4 adapters (r = 16), graph replay
     na, Mm = 4, 16
     g = torch.Generator().manual_seed(77)
@@ -423,21 +441,16 @@ def run_extras(qb, wl, dev, pk, flush):
     Xm = p["X"][:Mm].contiguous().to(dev)
     Ym = torch.empty(Mm, N, dtype=torch.bfloat16, device=dev)
     wsm = torch.empty(qb.fwd_workspace_bytes(Mm, N, K, r), dtype=torch.uint8, device=dev)
-    callm = lambda: qb.qlora_linear_fwd_multi(q, Xm, A_all, B_all, sc_all, idx, out=Ym, workspace=wsm)
-    side = torch.cuda.Stream()
-    side.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(side):
-        callm()
-    torch.cuda.current_stream().wait_stream(side)
-    graph_m = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_m):
-        callm()
-    ms = timed(graph_m.replay)
     mbytes = weight_bytes + 2 * na * r * (K + N) + 2 * Mm * (K + N)
+    ms = graph_time(lambda: qb.qlora_linear_fwd_multi(q, Xm, A_all, B_all, sc_all, idx, out=Ym, workspace=wsm))
     res["decode_70b_up_multi_adapter"] = {"tokens": Mm, "adapters": na, "us": round(ms * 1e3, 2),
                                           "total_gbs": round(mbytes / ms / 1e6, 1),
                                           "frac_hbm": round(mbytes / ms / 1e6 / pk["hbm_gbs"], 4)}
-    del graph_m
+    ms = graph_time(lambda: qb.qlora_linear_fwd_multi_tiles(q, tiles, Xm, A_all, B_all, sc_all, idx, out=Ym,
+                                                            workspace=wsm))
+    res["decode_70b_up_multi_adapter_tiles"] = {"tokens": Mm, "adapters": na, "us": round(ms * 1e3, 2),
+                                                "total_gbs": round(mbytes / ms / 1e6, 1),
+                                                "frac_hbm": round(mbytes / ms / 1e6 / pk["hbm_gbs"], 4)}
     # quantize of the same weight (4 B read + 0.516 B written per weight)
     numel = N * K
     qbytes = 4 * numel + numel // 2 + numel // 64 + 4 * ((numel // 64 + 255) // 256)
@@ -541,7 +554,10 @@ def run_profile(args):
     q = qb.nf4_quantize(p["W"].to(dev))
     X, A, B = p["X"].to(dev), p["A"].to(dev), p["B"].to(dev)
     dY = p["dY"].to(dev) if "dY" in p else None
+    tiles = qb.nf4_decode_tiles(q) if args.profile == "fwd_tiles" else None
     for _ in range(args.warmup + args.steps):
+        if args.profile == "fwd_tiles":
+            qb.qlora_linear_fwd_tiles(q, tiles, X, A, B, p["scale"])
         if args.profile in ("fwd", "step"):
             _, H = qb.qlora_linear_fwd(q, X, A, B, p["scale"])
         if args.profile in ("bwd", "step"):
@@ -563,7 +579,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true", help="skip decode/quantize measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--profile", choices=["fwd", "bwd", "step", "quantize", "dequantize"],
+    ap.add_argument("--profile", choices=["fwd", "fwd_tiles", "bwd", "step", "quantize", "dequantize"],
                     help="run only warmup+steps launches of one entry point (for ncu)")
     ap.add_argument("--workload", default=WORKLOAD, help="workload for --profile")
     ap.add_argument("--tokens", type=int, default=0, help="token count for --profile (default: the workload's)")

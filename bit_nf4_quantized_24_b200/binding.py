@@ -65,6 +65,10 @@ def lib():
     L.nf4_merge_lora.argtypes = [P, P, P, i32, i32, i64, i64, P, P, i32, f32, i32, i32, P, P, P, P]
     L.qlora_linear_fwd_multi.argtypes = [P, P, P, i64, i64, P, i64, P, P, i32, i32, P, P, P, P, sz, P]
     L.qlora_linear_dropout_workspace.argtypes = [i64, i64, i64, i32, P]
+    L.nf4_decode_tiles_bytes.argtypes = [i64, i64, P]
+    L.nf4_decode_tiles.argtypes = [P, i64, i64, P, P]
+    L.qlora_linear_fwd_tiles.argtypes = [P, P, P, i64, i64, P, i64, P, P, i32, f32, P, P, P, sz, P]
+    L.qlora_linear_fwd_multi_tiles.argtypes = [P, P, P, i64, i64, P, i64, P, P, i32, i32, P, P, P, P, sz, P]
     L.qlora_linear_fwd_dropout.argtypes = [P, P, P, i64, i64, P, i64, P, P, i32, f32, P, f32, P, P, P, sz, P]
     L.qlora_linear_bwd_dropout.argtypes = [P, P, P, i64, i64, P, P, i64, P, P, i32, f32, P, f32, P, P, P, P, P, sz,
                                            P]
@@ -309,6 +313,71 @@ def qlora_linear_fwd_multi(w: NF4Weight, X: torch.Tensor, A_all: torch.Tensor, B
     _check(lib().qlora_linear_fwd_multi(_ptr(w.codes), _ptr(w.absmax_q), _ptr(w.dq_scale), w.N, w.K, _ptr(X), M,
                                         _ptr(A_all), _ptr(B_all), na, r, _ptr(scales), _ptr(adapter_idx), _ptr(out),
                                         _ptr(ws), ws.numel(), _stream(stream)), "qlora_linear_fwd_multi")
+    return out
+
+
+def nf4_decode_tiles_bytes(N: int, K: int) -> int:
+    b = ctypes.c_size_t()
+    _check(lib().nf4_decode_tiles_bytes(N, K, ctypes.byref(b)), "nf4_decode_tiles_bytes")
+    return b.value
+
+
+def nf4_decode_tiles(w: NF4Weight, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The decode-tile copy of w's codes (uint8, nf4_decode_tiles_bytes(N, K)
+    bytes) for qlora_linear_fwd_tiles / qlora_linear_fwd_multi_tiles."""
+    w._layer_format()
+    nbytes = nf4_decode_tiles_bytes(w.N, w.K)
+    if out is None:
+        out = torch.empty(nbytes, dtype=torch.uint8, device=w.codes.device)
+    _req(out, torch.uint8, "tiles", (nbytes,))
+    _check(lib().nf4_decode_tiles(_ptr(w.codes), w.N, w.K, _ptr(out), _stream(stream)), "nf4_decode_tiles")
+    return out
+
+
+def qlora_linear_fwd_tiles(w: NF4Weight, tiles: torch.Tensor, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
+                           scale: float, save_h: bool = True, out: torch.Tensor | None = None,
+                           workspace: torch.Tensor | None = None, stream=None):
+    """qlora_linear_fwd for M <= 16 tokens reading the decode tiles of w's
+    codes (w supplies absmax_q, dq_scale and the shape).  Returns (Y, H)."""
+    w._layer_format()
+    M = X.shape[0]
+    r = A.shape[0]
+    _req(tiles, torch.uint8, "tiles", (nf4_decode_tiles_bytes(w.N, w.K),))
+    _req(X, torch.bfloat16, "X", (M, w.K))
+    _req(A, torch.bfloat16, "A", (r, w.K))
+    _req(B, torch.bfloat16, "B", (w.N, r))
+    if out is None:
+        out = torch.empty(M, w.N, dtype=torch.bfloat16, device=X.device)
+    _req(out, torch.bfloat16, "Y", (M, w.N))
+    H = torch.empty(M, r, dtype=torch.bfloat16, device=X.device) if save_h else None
+    ws = _workspace(fwd_workspace_bytes(M, w.N, w.K, r), X.device, workspace)
+    _check(lib().qlora_linear_fwd_tiles(_ptr(tiles), _ptr(w.absmax_q), _ptr(w.dq_scale), w.N, w.K, _ptr(X), M,
+                                        _ptr(A), _ptr(B), r, float(scale), _ptr(out), _ptr(H), _ptr(ws), ws.numel(),
+                                        _stream(stream)), "qlora_linear_fwd_tiles")
+    return out, H
+
+
+def qlora_linear_fwd_multi_tiles(w: NF4Weight, tiles: torch.Tensor, X: torch.Tensor, A_all: torch.Tensor,
+                                 B_all: torch.Tensor, scales: torch.Tensor, adapter_idx: torch.Tensor,
+                                 out: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None):
+    """qlora_linear_fwd_multi reading the decode tiles of w's codes."""
+    w._layer_format()
+    M = X.shape[0]
+    na, r = A_all.shape[0], A_all.shape[1]
+    _req(tiles, torch.uint8, "tiles", (nf4_decode_tiles_bytes(w.N, w.K),))
+    _req(X, torch.bfloat16, "X", (M, w.K))
+    _req(A_all, torch.bfloat16, "A_all", (na, r, w.K))
+    _req(B_all, torch.bfloat16, "B_all", (na, w.N, r))
+    _req(scales, torch.float32, "scales", (na,))
+    _req(adapter_idx, torch.int32, "adapter_idx", (M,))
+    if out is None:
+        out = torch.empty(M, w.N, dtype=torch.bfloat16, device=X.device)
+    _req(out, torch.bfloat16, "Y", (M, w.N))
+    ws = _workspace(fwd_workspace_bytes(M, w.N, w.K, r), X.device, workspace)
+    _check(lib().qlora_linear_fwd_multi_tiles(_ptr(tiles), _ptr(w.absmax_q), _ptr(w.dq_scale), w.N, w.K, _ptr(X), M,
+                                              _ptr(A_all), _ptr(B_all), na, r, _ptr(scales), _ptr(adapter_idx),
+                                              _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
+           "qlora_linear_fwd_multi_tiles")
     return out
 
 

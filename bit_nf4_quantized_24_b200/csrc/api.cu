@@ -346,6 +346,69 @@ int qlora_linear_fwd_multi(const uint8_t* codes, const uint8_t* absmax_q, const 
   return cuda_status(e);
 }
 
+int nf4_decode_tiles_bytes(int64_t N, int64_t K, size_t* bytes) {
+  if (!bytes || N <= 0 || K <= 0) return QLORA_ERR_ARG;
+  if (K % 1024 || N > (1 << 24) || K > (1 << 24)) return QLORA_ERR_SHAPE;
+  *bytes = static_cast<size_t>(decode_tiles_bytes(N, K));
+  return QLORA_OK;
+}
+
+int nf4_decode_tiles(const uint8_t* codes, int64_t N, int64_t K, uint8_t* tiles, void* stream) {
+  size_t bytes = 0;
+  int st = nf4_decode_tiles_bytes(N, K, &bytes);
+  if (st) return st;
+  if (!codes || !tiles) return QLORA_ERR_ARG;
+  if (!aligned(codes, 16) || !aligned(tiles, 16)) return QLORA_ERR_SHAPE;
+  return cuda_status(launch_pack_tiles(codes, N, K, tiles, static_cast<cudaStream_t>(stream)));
+}
+
+int qlora_linear_fwd_tiles(const uint8_t* tiles, const uint8_t* absmax_q, const float* dq_scale, int64_t N, int64_t K,
+                           const qlora_bf16_t* X, int64_t M, const qlora_bf16_t* A, const qlora_bf16_t* B, int r,
+                           float scale, qlora_bf16_t* Y, qlora_bf16_t* H_save, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  int st = check_layer_shapes(M, N, K, r);
+  if (st) return st;
+  if (K % 1024) return QLORA_ERR_SHAPE;
+  if (M > 16) return QLORA_ERR_UNSUPPORTED;
+  if (!tiles || !absmax_q || !dq_scale || !A || !B || (M > 0 && (!X || !Y))) return QLORA_ERR_ARG;
+  if (!std::isfinite(scale)) return QLORA_ERR_ARG;
+  if (M == 0) return QLORA_OK;
+  const void* ptrs[] = {tiles, absmax_q, X, A, B, Y};
+  for (const void* p : ptrs)
+    if (!aligned(p, 16)) return QLORA_ERR_SHAPE;
+  if (H_save && !aligned(H_save, 16)) return QLORA_ERR_SHAPE;
+  FwdWorkspace w = fwd_layout(workspace, M, r);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < w.bytes) return QLORA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_rowdot(X, A, M, K, r, scale, w.Hs, 1.0f, H_save, nullptr, s);
+  if (e == cudaSuccess) e = launch_gemv_tiles(X, M, tiles, absmax_q, dq_scale, N, K, w.Hs, B, r, Y, s);
+  return cuda_status(e);
+}
+
+int qlora_linear_fwd_multi_tiles(const uint8_t* tiles, const uint8_t* absmax_q, const float* dq_scale, int64_t N,
+                                 int64_t K, const qlora_bf16_t* X, int64_t M, const qlora_bf16_t* A_all,
+                                 const qlora_bf16_t* B_all, int n_adapters, int r, const float* scales,
+                                 const int32_t* adapter_idx, qlora_bf16_t* Y, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+  int st = check_layer_shapes(M, N, K, r);
+  if (st) return st;
+  if (K % 1024) return QLORA_ERR_SHAPE;
+  if (M > 16 || n_adapters < 1) return n_adapters < 1 ? QLORA_ERR_ARG : QLORA_ERR_UNSUPPORTED;
+  if (!tiles || !absmax_q || !dq_scale || !A_all || !B_all || !scales || (M > 0 && (!X || !Y || !adapter_idx)))
+    return QLORA_ERR_ARG;
+  if (M == 0) return QLORA_OK;
+  const void* ptrs[] = {tiles, absmax_q, X, A_all, B_all, Y};
+  for (const void* p : ptrs)
+    if (!aligned(p, 16)) return QLORA_ERR_SHAPE;
+  FwdWorkspace w = fwd_layout(workspace, M, r);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < w.bytes) return QLORA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_rows_multi(X, M, K, A_all, n_adapters, r, scales, adapter_idx, w.Hs, s);
+  if (e == cudaSuccess)
+    e = launch_gemv_tiles(X, M, tiles, absmax_q, dq_scale, N, K, w.Hs, B_all, r, Y, s, adapter_idx, n_adapters);
+  return cuda_status(e);
+}
+
 int qlora_linear_dropout_workspace(int64_t M, int64_t N, int64_t K, int r, size_t* bytes) {
   if (!bytes) return QLORA_ERR_ARG;
   int st = check_layer_shapes(M, N, K, r);

@@ -493,4 +493,413 @@ cudaError_t launch_gemv(const uint16_t* X, int64_t M, const uint8_t* codes, cons
                 : gemv_launch<2, false>(tm, X, M, absmax_q, dq_scale, N, K, Hs, B, r, nullptr, 0, Y, st);
 }
 
+namespace {
+
+// ---------------------------------------------------------------------------
+// Decode tiles: a serving layout of the codes, made once when the weight is
+// loaded.  Unit (tile tau, block kb) is 512 contiguous bytes in which lane
+// L = 4g + t of a warp owns bytes 16L .. 16L+15: the code bytes 8t .. 8t+7 of
+// block kb in row 16 tau + g, then the same bytes of row 16 tau + g + 8 (rows
+// past N hold zeros).  The units of a tile follow in kb order, so a tile is
+// one contiguous run of 8 K bytes, a warp reads a unit with one 128-bit load
+// per lane, and the bytes land in exactly the registers the lookups of the
+// row-major kernel above build from shared memory.
+//
+// Work split.  A CTA owns a run of tiles; a work item is 16 blocks (8 KB) of
+// one tile, and consumer warp w takes items w, w + 15, w + 30, ... of the
+// CTA's run, so the 15 warps read 120 KB of consecutive codes at a time.
+// Each warp prefetches its next item into L2 with a bulk prefetch and keeps
+// four units of loads in flight in registers.  A warp hands the item's
+// per-row partial sums to the epilogue warp through a slot of shared memory;
+// the epilogue adds a tile's items in item order (deterministic), adds the
+// LoRA term and stores Y.
+//
+// Block scales.  With K % 1024 == 0 the 16 blocks of an item lie in one
+// double-quantization group for every row, so a lane loads its two rows' 16
+// absmax bytes and group scales once per item; the scale of unit u is then
+// fl32(q * d) = fma(2^23 + q, d, -2^23 d) with 2^23 + q built by one prmt.
+
+constexpr int T_CW = 15;                      // consumer warps (+ 1: four warps per SM sub-partition)
+constexpr int T_THREADS = (T_CW + 1) * 32;    // + epilogue warp
+constexpr int T_UNIT = 512;                   // bytes of one (tile, block) unit
+constexpr int T_ITEM = 16;                    // blocks per work item
+constexpr int T_GU = 4;                       // units per group of code loads (two groups in flight)
+constexpr int T_SLOTS_MAX = 4;                // tiles whose partial sums can wait for the epilogue
+constexpr int T_SMEM_LIMIT = 231424;          // dynamic shared memory cap (227 KB less 1 KB of static)
+
+__host__ __device__ constexpr int tiles_slot_bytes(int nch, int ntile) { return nch * ntile * 4 * 32 * 4; }
+__host__ __device__ constexpr int tiles_smem_bytes(int nch, int ntile, int ts) {
+  return 65536 /* table alignment */ + G_TABLE + ts * tiles_slot_bytes(nch, ntile) + 16 * ts + 64;
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+
+__device__ __forceinline__ uint4 ldg_v4(const void* p) {  // activations and absmax bytes: keep them in L1
+  return __ldg(reinterpret_cast<const uint4*>(p));
+}
+// The same load issued only by lanes with `on` set (others get zeros): the
+// predicate is explicit so the compiler cannot turn it into a load by every
+// lane, and the L1 returns only the active lanes' bytes.
+__device__ __forceinline__ uint4 ldg_v4_if(const void* p, bool on) {
+  uint4 v;
+  asm volatile(
+      "{\n\t.reg .pred q;\n\t"
+      "setp.ne.b32 q, %5, 0;\n\t"
+      "mov.b32 %0, 0;\n\tmov.b32 %1, 0;\n\tmov.b32 %2, 0;\n\tmov.b32 %3, 0;\n\t"
+      "@q ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];\n\t}"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p), "r"(static_cast<int>(on)));
+  return v;
+}
+
+// fl32(q * d) for the absmax byte at byte position `byte` of `word`: 2^23 + q
+// is exact in fp32, so one fused multiply-add with c = -2^23 d rounds q * d once.
+__device__ __forceinline__ float block_scale(uint32_t word, int byte, float d, float c) {
+  return fmaf(__uint_as_float(prmt(word, 0x4B000000u, 0x7540u | byte)), d, c);
+}
+
+template <int NTILE>
+struct UnitX {
+  uint32_t x[NTILE][8];
+};
+
+// One unit: 16 lookups, four MMA steps into a fresh fragment per token tile,
+// then the scaled add (rows g: sa, rows g + 8: sb).
+template <int NTILE>
+__device__ __forceinline__ void unit_mma(float (&acc)[NTILE][4], const uint4& cw, const UnitX<NTILE>& in,
+                                         uint32_t lane_base, float sa, float sb) {
+  uint32_t a[4][4];
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    const uint32_t wg = s < 2 ? cw.x : cw.y, wh = s < 2 ? cw.z : cw.w;
+    if ((s & 1) == 0) {
+      a[s][0] = lut_pair<0>(wg, lane_base); a[s][2] = lut_pair<1>(wg, lane_base);
+      a[s][1] = lut_pair<0>(wh, lane_base); a[s][3] = lut_pair<1>(wh, lane_base);
+    } else {
+      a[s][0] = lut_pair<2>(wg, lane_base); a[s][2] = lut_pair<3>(wg, lane_base);
+      a[s][1] = lut_pair<2>(wh, lane_base); a[s][3] = lut_pair<3>(wh, lane_base);
+    }
+  }
+#pragma unroll
+  for (int nt = 0; nt < NTILE; ++nt) {
+    float p[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int s = 0; s < 4; ++s) mma16816(p, a[s][0], a[s][1], a[s][2], a[s][3], in.x[nt][2 * s], in.x[nt][2 * s + 1]);
+    acc[nt][0] = fmaf(sa, p[0], acc[nt][0]);
+    acc[nt][1] = fmaf(sa, p[1], acc[nt][1]);
+    acc[nt][2] = fmaf(sb, p[2], acc[nt][2]);
+    acc[nt][3] = fmaf(sb, p[3], acc[nt][3]);
+  }
+}
+
+template <int NTILE, bool MULTI>
+__global__ void __launch_bounds__(T_THREADS, 1)
+    k_gemv_tiles(const uint8_t* __restrict__ tiles, const uint16_t* __restrict__ X, int M,
+                 const uint8_t* __restrict__ absmax_q, const float* __restrict__ dq_scale, int N, int K,
+                 const uint16_t* __restrict__ Hs, const uint16_t* __restrict__ Bl, int r, Nf4Levels lv,
+                 const int32_t* __restrict__ aidx, int na, int ts, int pf, uint16_t* __restrict__ Y, int* status) {
+  pdl_trigger();
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ int abort_flag;
+  const int KB = K / 64, NCH = KB / T_ITEM;
+  const int bytes = tiles_smem_bytes(NCH, NTILE, ts);
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t table = (raw + 65535u) & ~65535u;
+  const uint32_t part0 = table + G_TABLE;
+  const uint32_t slot_bytes = tiles_slot_bytes(NCH, NTILE);
+  const uint32_t full0 = part0 + ts * slot_bytes, empty0 = full0 + 8u * ts;
+  if (empty0 + 8u * ts > raw + bytes) {  // cannot happen with the launch's size; never index past it
+    if (threadIdx.x == 0) atomicExch(status, kDevTimeout);
+    return;
+  }
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
+
+  for (int idx = tid; idx < 256 * 32; idx += T_THREADS) {
+    const int e = idx >> 5, l = idx & 31;
+    const uint32_t v = bf16x2_bits(lv.v[e & 15], lv.v[e >> 4]);
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(table + e * 256 + l * 4), "r"(v) : "memory");
+  }
+  if (tid == 0) {
+    for (int s = 0; s < ts; ++s) {
+      mbar_init(full0 + 8u * s, NCH);
+      mbar_init(empty0 + 8u * s, 1);
+    }
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const int ntiles = (N + G_ROWS - 1) / G_ROWS;
+  const int t0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * ntiles / gridDim.x);
+  const int t1 = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * ntiles / gridDim.x);
+  const int nitems = (t1 - t0) * NCH;
+  // partial-sum word (chunk ch, tile nt, element c) of slot `slot`, lane l
+  auto part_addr = [&](int slot, int ch, int nt, int c, int l) -> uint32_t {
+    return part0 + slot * slot_bytes + ((((ch * NTILE + nt) * 4 + c) * 32 + l) << 2);
+  };
+
+  if (warp == T_CW) {  // epilogue: sum the items of each tile in order, add the LoRA term, store
+    pdl_wait();  // Hs comes from the previous kernel of the stream
+    for (int ti = 0; ti < t1 - t0; ++ti) {
+      const int n0 = (t0 + ti) * G_ROWS;
+      const int slot = ti % ts, use = ti / ts;
+      auto ld2 = [&](const uint16_t* p, int row, int rows, int j) -> uint32_t {
+        if (row >= rows || j >= r) return 0u;
+        return __ldg(reinterpret_cast<const uint32_t*>(p + static_cast<int64_t>(row) * r + j));
+      };
+      uint32_t la[4][4], lb[4][NTILE][2];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (MULTI) break;
+        const int j0 = 16 * k;
+        la[k][0] = ld2(Bl, n0 + g, N, j0 + 2 * t);
+        la[k][1] = ld2(Bl, n0 + g + 8, N, j0 + 2 * t);
+        la[k][2] = ld2(Bl, n0 + g, N, j0 + 2 * t + 8);
+        la[k][3] = ld2(Bl, n0 + g + 8, N, j0 + 2 * t + 8);
+#pragma unroll
+        for (int nt = 0; nt < NTILE; ++nt) {
+          lb[k][nt][0] = ld2(Hs, 8 * nt + g, M, j0 + 2 * t);
+          lb[k][nt][1] = ld2(Hs, 8 * nt + g, M, j0 + 2 * t + 8);
+        }
+      }
+      if (!wait_bounded(full0 + 8u * slot, use & 1, &abort_flag, status)) break;
+      float v[NTILE][4];
+#pragma unroll
+      for (int nt = 0; nt < NTILE; ++nt)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) v[nt][c] = 0.f;
+      for (int ch = 0; ch < NCH; ++ch)
+#pragma unroll
+        for (int nt = 0; nt < NTILE; ++nt)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) v[nt][c] += lds_f32(part_addr(slot, ch, nt, c, lane));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty0 + 8u * slot);  // partial sums read: the slot is free
+      if (MULTI) {
+#pragma unroll
+        for (int nt = 0; nt < NTILE; ++nt)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int m = 8 * nt + 2 * t + (c & 1), n = n0 + g + 8 * (c >> 1);
+            if (m >= M || n >= N) continue;
+            const int a = __ldg(aidx + m);
+            if (a < 0 || a >= na) continue;
+            const uint4* hp = reinterpret_cast<const uint4*>(Hs + static_cast<int64_t>(m) * r);
+            const uint4* bp = reinterpret_cast<const uint4*>(Bl + (static_cast<int64_t>(a) * N + n) * r);
+            float lora = 0.f;
+            for (int j8 = 0; j8 < r / 8; ++j8) {
+              const uint4 h = __ldg(hp + j8), b = __ldg(bp + j8);
+              const uint32_t hw[4] = {h.x, h.y, h.z, h.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                lora = fmaf(__uint_as_float(hw[q] << 16), __uint_as_float(bw[q] << 16), lora);
+                lora = fmaf(__uint_as_float(hw[q] & 0xffff0000u), __uint_as_float(bw[q] & 0xffff0000u), lora);
+              }
+            }
+            v[nt][c] += lora;
+          }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if (16 * k >= r) break;
+#pragma unroll
+          for (int nt = 0; nt < NTILE; ++nt)
+            mma16816(v[nt], la[k][0], la[k][1], la[k][2], la[k][3], lb[k][nt][0], lb[k][nt][1]);
+        }
+      }
+#pragma unroll
+      for (int nt = 0; nt < NTILE; ++nt) {
+        const int m = 8 * nt + 2 * t;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int n = n0 + g + 8 * h;
+          if (n >= N) continue;
+          if (m < M) Y[static_cast<int64_t>(m) * N + n] = static_cast<uint16_t>(bf16x2_bits(v[nt][2 * h], 0.f));
+          if (m + 1 < M)
+            Y[static_cast<int64_t>(m + 1) * N + n] = static_cast<uint16_t>(bf16x2_bits(v[nt][2 * h + 1], 0.f));
+        }
+      }
+    }
+    return;
+  }
+
+  // consumers
+  const uint32_t lane_base = table + lane * 4;
+  const int64_t tile_bytes = static_cast<int64_t>(KB) * T_UNIT;
+  auto item_codes = [&](int j) -> const uint8_t* {  // this lane's 16 bytes of the item's first unit
+    const int ti = j / NCH, ch = j - ti * NCH;
+    return tiles + static_cast<int64_t>(t0 + ti) * tile_bytes + static_cast<int64_t>(ch) * (T_ITEM * T_UNIT) + lane * 16;
+  };
+  // Lanes of token rows >= M load nothing and hold zeros (those columns are
+  // never stored): the loads return only the bytes of real tokens, which
+  // matters because every byte a load returns costs the same L1 bandwidth
+  // as the table lookups.
+  const uint16_t* xrow[NTILE];
+  bool xon[NTILE];
+#pragma unroll
+  for (int nt = 0; nt < NTILE; ++nt) {
+    xon[nt] = 8 * nt + g < M;
+    xrow[nt] = X + static_cast<int64_t>(min(8 * nt + g, M - 1)) * K + 16 * t;
+  }
+  auto load_x = [&](UnitX<NTILE>& in, int kb) {
+#pragma unroll
+    for (int nt = 0; nt < NTILE; ++nt) {
+      const uint16_t* p = xrow[nt] + kb * 64;
+      const uint4 lo = ldg_v4_if(p, xon[nt]), hi = ldg_v4_if(p + 8, xon[nt]);
+      in.x[nt][0] = lo.x; in.x[nt][1] = lo.y; in.x[nt][2] = lo.z; in.x[nt][3] = lo.w;
+      in.x[nt][4] = hi.x; in.x[nt][5] = hi.y; in.x[nt][6] = hi.z; in.x[nt][7] = hi.w;
+    }
+  };
+  // the two rows' absmax bytes of item j start at this lane's index (dq group: index >> 8)
+  auto absmax_index = [&](int j, int h) -> int64_t {
+    const int ti = j / NCH, ch = j - ti * NCH;
+    return static_cast<int64_t>(min((t0 + ti) * G_ROWS + g + 8 * h, N - 1)) * KB + ch * T_ITEM;
+  };
+
+  if (lane == 0)
+    for (int q = 0; q < pf; ++q) {
+      const int j = warp + q * T_CW;
+      if (j < nitems) prefetch_l2(item_codes(j), T_ITEM * T_UNIT);
+    }
+  constexpr int NG = T_ITEM / T_GU;  // code groups per item (even: the next item's first group goes to cw[0])
+  static_assert(NG % 2 == 0, "group count");
+  uint4 cw[2][T_GU];  // codes of the current and the next group of units
+  if (warp < nitems) {
+    const uint8_t* c0 = item_codes(warp);
+#pragma unroll
+    for (int u = 0; u < T_GU; ++u) cw[0][u] = ldg_nc_v4(c0 + u * T_UNIT);
+  }
+  float acc[NTILE][4];
+#pragma unroll
+  for (int nt = 0; nt < NTILE; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+
+  for (int j = warp; j < nitems; j += T_CW) {
+    const int ti = j / NCH, ch = j - ti * NCH;
+    const uint8_t* cbase = item_codes(j);
+    if (lane == 0 && pf > 0) {
+      const int jp = j + pf * T_CW;
+      if (jp < nitems) prefetch_l2(item_codes(jp), T_ITEM * T_UNIT);
+    }
+    // the two rows' absmax bytes and group scales of the item; the next
+    // item's lines go to L1 now, so its loads do not wait on L2
+    const int kb0 = ch * T_ITEM;
+    const int64_t ia = absmax_index(j, 0), ib = absmax_index(j, 1);
+    const uint4 qa = ldg_v4(absmax_q + ia), qb = ldg_v4(absmax_q + ib);
+    const float da = __ldg(dq_scale + (ia >> 8)), db = __ldg(dq_scale + (ib >> 8));
+    if (j + T_CW < nitems) {
+      const int64_t pa = absmax_index(j + T_CW, 0), pb = absmax_index(j + T_CW, 1);
+      prefetch_l1(absmax_q + pa);
+      prefetch_l1(absmax_q + pb);
+      prefetch_l1(dq_scale + (pa >> 8));
+      prefetch_l1(dq_scale + (pb >> 8));
+    }
+    const float ca = -8388608.0f * da, cb = -8388608.0f * db;
+    const uint32_t qaw[4] = {qa.x, qa.y, qa.z, qa.w}, qbw[4] = {qb.x, qb.y, qb.z, qb.w};
+    UnitX<NTILE> xin[2];
+    load_x(xin[0], kb0);
+#pragma unroll
+    for (int grp = 0; grp < NG; ++grp) {
+      // loads of the next group: this item's, or the first of the next item
+      if (grp + 1 < NG) {
+#pragma unroll
+        for (int u = 0; u < T_GU; ++u)
+          cw[(grp + 1) & 1][u] = ldg_nc_v4(cbase + (T_GU * (grp + 1) + u) * T_UNIT);
+      } else if (j + T_CW < nitems) {
+        const uint8_t* cn = item_codes(j + T_CW);
+#pragma unroll
+        for (int u = 0; u < T_GU; ++u) cw[0][u] = ldg_nc_v4(cn + u * T_UNIT);
+      }
+#pragma unroll
+      for (int u = 0; u < T_GU; ++u) {
+        const int uu = T_GU * grp + u;
+        if (uu + 1 < T_ITEM) load_x(xin[(uu + 1) & 1], kb0 + uu + 1);
+        const float sa = block_scale(qaw[uu >> 2], uu & 3, da, ca);
+        const float sb = block_scale(qbw[uu >> 2], uu & 3, db, cb);
+        unit_mma<NTILE>(acc, cw[grp & 1][u], xin[uu & 1], lane_base, sa, sb);
+      }
+    }
+    // hand the item's partial sums to the epilogue warp
+    const int slot = ti % ts, use = ti / ts;
+    if (!wait_bounded(empty0 + 8u * slot, (use & 1) ^ 1, &abort_flag, status)) break;
+#pragma unroll
+    for (int nt = 0; nt < NTILE; ++nt)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        sts_f32(part_addr(slot, ch, nt, c, lane), acc[nt][c]);
+        acc[nt][c] = 0.f;
+      }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(full0 + 8u * slot);
+  }
+}
+
+// one thread per 16-byte chunk of the tiles: chunk (tau * KB + kb) * 32 + L
+__global__ void k_pack_tiles(const uint8_t* __restrict__ codes, int N, int K, uint8_t* __restrict__ tiles,
+                             int64_t nchunks) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= nchunks) return;
+  const int KB = K / 64;
+  const int L = static_cast<int>(idx & 31);
+  const int64_t rest = idx >> 5;
+  const int kb = static_cast<int>(rest % KB);
+  const int64_t tau = rest / KB;
+  const int g = L >> 2, t = L & 3;
+  const int64_t ra = tau * G_ROWS + g, rb = ra + 8;
+  const int64_t off = static_cast<int64_t>(kb) * 32 + 8 * t;
+  uint2 a = make_uint2(0u, 0u), b = make_uint2(0u, 0u);
+  if (ra < N) a = __ldg(reinterpret_cast<const uint2*>(codes + ra * (K / 2) + off));
+  if (rb < N) b = __ldg(reinterpret_cast<const uint2*>(codes + rb * (K / 2) + off));
+  reinterpret_cast<uint4*>(tiles)[idx] = make_uint4(a.x, a.y, b.x, b.y);
+}
+
+template <int NTILE, bool MULTI>
+cudaError_t gemv_tiles_launch(const uint8_t* tiles, const uint16_t* X, int64_t M, const uint8_t* absmax_q,
+                              const float* dq_scale, int64_t N, int64_t K, const uint16_t* Hs, const uint16_t* B,
+                              int r, const int32_t* aidx, int na, uint16_t* Y, cudaStream_t st) {
+  const int nch = static_cast<int>(K / 64 / T_ITEM);
+  const int avail = T_SMEM_LIMIT - tiles_smem_bytes(nch, NTILE, 0);
+  const int ts = std::min(T_SLOTS_MAX, avail / (tiles_slot_bytes(nch, NTILE) + 16));
+  if (ts < 1) return cudaErrorInvalidValue;  // K too large for one slot of partial sums
+  cudaError_t e = smem_limit_once<k_gemv_tiles<NTILE, MULTI>>(T_SMEM_LIMIT);
+  if (e != cudaSuccess) return e;
+  const int sms = device_sm_count();
+  const int64_t ntiles = (N + G_ROWS - 1) / G_ROWS;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ntiles, sms));
+  return launch_ex(k_gemv_tiles<NTILE, MULTI>, dim3(grid), dim3(T_THREADS), tiles_smem_bytes(nch, NTILE, ts), st,
+                   true, tiles, X, int(M), absmax_q, dq_scale, int(N), int(K), Hs, B, r, host_codebook().levels,
+                   aidx, na, ts, 1, Y, device_status_ptr());
+}
+
+}  // namespace
+
+int64_t decode_tiles_bytes(int64_t N, int64_t K) { return (N + G_ROWS - 1) / G_ROWS * (K / 64) * T_UNIT; }
+
+cudaError_t launch_pack_tiles(const uint8_t* codes, int64_t N, int64_t K, uint8_t* tiles, cudaStream_t st) {
+  if (N == 0) return cudaSuccess;
+  if (K % 1024 || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+  const int64_t nchunks = decode_tiles_bytes(N, K) / 16;
+  const unsigned grid = static_cast<unsigned>((nchunks + 255) / 256);
+  k_pack_tiles<<<grid, 256, 0, st>>>(codes, int(N), int(K), tiles, nchunks);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemv_tiles(const uint16_t* X, int64_t M, const uint8_t* tiles, const uint8_t* absmax_q,
+                              const float* dq_scale, int64_t N, int64_t K, const uint16_t* Hs, const uint16_t* B,
+                              int r, uint16_t* Y, cudaStream_t st, const int32_t* aidx, int na) {
+  if (M == 0 || N == 0) return cudaSuccess;
+  if (M > 16 || r > 64 || K % 1024 || N * (K / 64) >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+  if (aidx)
+    return M <= 8 ? gemv_tiles_launch<1, true>(tiles, X, M, absmax_q, dq_scale, N, K, Hs, B, r, aidx, na, Y, st)
+                  : gemv_tiles_launch<2, true>(tiles, X, M, absmax_q, dq_scale, N, K, Hs, B, r, aidx, na, Y, st);
+  return M <= 8 ? gemv_tiles_launch<1, false>(tiles, X, M, absmax_q, dq_scale, N, K, Hs, B, r, nullptr, 0, Y, st)
+                : gemv_tiles_launch<2, false>(tiles, X, M, absmax_q, dq_scale, N, K, Hs, B, r, nullptr, 0, Y, st);
+}
+
 }  // namespace qn

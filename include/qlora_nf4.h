@@ -187,6 +187,41 @@ int qlora_linear_fwd_multi(const uint8_t* codes, const uint8_t* absmax_q, const 
                            int r, const float* scales, const int32_t* adapter_idx, qlora_bf16_t* Y,
                            void* workspace, size_t workspace_bytes, void* stream);
 
+/* Decode tiles: a serving layout of an NF4 weight's codes for the decode
+ * calls below (M <= 16), made once when the weight is loaded.  It holds the
+ * same code bytes as the row-major codes (the NF4 format above, "NF4: 4-bit
+ * NormalFloat": two 4-bit codes per byte, first element in the low nibble),
+ * rearranged so that every 16-row x 64-column unit is 512 contiguous bytes:
+ * for tile tau (rows 16 tau .. 16 tau + 15), block kb and i = 4g + t
+ * (g < 8, t < 4), bytes [16 i, 16 i + 16) of unit (tau, kb) at offset
+ * (tau * K/64 + kb) * 512 are codes[16 tau + g][32 kb + 8t .. + 7] followed by
+ * codes[16 tau + g + 8][32 kb + 8t .. + 7]; rows past N hold zeros.  absmax_q
+ * and dq_scale keep their layout.  K % 1024 == 0 (QLORA_ERR_SHAPE otherwise).
+ * nf4_decode_tiles_bytes: size of the tiles, ceil(N / 16) * K / 64 * 512.
+ * nf4_decode_tiles: codes (device, row-major [N, K/2], 16-byte aligned) ->
+ * tiles (device, caller-owned, 16-byte aligned), asynchronous on `stream`.
+ * Errors: ARG, SHAPE, CUDA. */
+int nf4_decode_tiles_bytes(int64_t N, int64_t K, size_t* bytes);
+int nf4_decode_tiles(const uint8_t* codes, int64_t N, int64_t K, uint8_t* tiles, void* stream);
+
+/* qlora_linear_fwd and qlora_linear_fwd_multi for M <= 16 tokens with the
+ * codes given as decode tiles (default NF4 format: block 64, double
+ * quantization over 256 blocks).  The result is the same sum in the same fp32
+ * order per 16-block item, so it equals the row-major decode call to within
+ * rounding of the per-item partial sums.  M > 16: QLORA_ERR_UNSUPPORTED.
+ * Same shape rules, workspace and errors as the row-major calls, plus
+ * K % 1024 == 0. */
+int qlora_linear_fwd_tiles(const uint8_t* tiles, const uint8_t* absmax_q, const float* dq_scale,
+                           int64_t N, int64_t K, const qlora_bf16_t* X, int64_t M,
+                           const qlora_bf16_t* A, const qlora_bf16_t* B, int r, float scale,
+                           qlora_bf16_t* Y, qlora_bf16_t* H_save,
+                           void* workspace, size_t workspace_bytes, void* stream);
+int qlora_linear_fwd_multi_tiles(const uint8_t* tiles, const uint8_t* absmax_q, const float* dq_scale,
+                                 int64_t N, int64_t K, const qlora_bf16_t* X, int64_t M,
+                                 const qlora_bf16_t* A_all, const qlora_bf16_t* B_all, int n_adapters,
+                                 int r, const float* scales, const int32_t* adapter_idx, qlora_bf16_t* Y,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
 /* Backward of the QLoRA linear: gradients flow through deq(W) to the
  * adapters and to the input; the frozen base gets none (katajob, "What stays
  * in full precision"):

@@ -67,6 +67,20 @@ def test_argument_errors_return_before_any_device_work(L):
     assert L.qlora_linear_bwd(None, None, None, 64, 64, None, None, 16, None, None, 16, ctypes.c_float(2.0), None,
                               None, None, None, None, 0, None) == -1
     assert L.qlora_trace_gemm_events(None, -1) == -1
+    # decode tiles: K % 1024 == 0, M <= 16
+    assert L.nf4_decode_tiles_bytes(40, 1088, ctypes.byref(i)) == -2
+    assert L.nf4_decode_tiles_bytes(0, 1024, ctypes.byref(i)) == -1
+    assert L.nf4_decode_tiles_bytes(40, 1024, ctypes.byref(i)) == 0 and i.value == 3 * 16 * 512
+    assert L.nf4_decode_tiles(None, 40, 1024, None, None) == -1
+    f2 = ctypes.c_float(2.0)
+    assert L.qlora_linear_fwd_tiles(None, None, None, 64, 1024, None, 17, None, None, 16, f2, None, None, None, 0,
+                                    None) == -7
+    assert L.qlora_linear_fwd_tiles(None, None, None, 64, 1088, None, 4, None, None, 16, f2, None, None, None, 0,
+                                    None) == -2
+    assert L.qlora_linear_fwd_tiles(None, None, None, 64, 1024, None, 4, None, None, 16, f2, None, None, None, 0,
+                                    None) == -1
+    assert L.qlora_linear_fwd_multi_tiles(None, None, None, 64, 1024, None, 4, None, None, 2, 16, None, None, None,
+                                          None, 0, None) == -1
 
 
 def test_workspace_sizes_grow_with_shape(L):

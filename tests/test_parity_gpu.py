@@ -343,6 +343,112 @@ def test_forward_decode_small(qb, oracle, M, N, K, r):
     run_fwd_check(qb, oracle, p)
 
 
+# ------------------------------------------------------------ decode tiles
+
+
+def tiles_from_codes(codes, N, K):
+    """The decode-tile arrangement of row-major codes as the header states it,
+    restated by index arithmetic: unit (tau, kb) at (tau * K/64 + kb) * 512,
+    lane i = 4g + t at 16 i holding row 16 tau + g bytes 32 kb + 8t .. +7, then
+    row 16 tau + g + 8; rows past N are zeros."""
+    c = np.asarray(codes, np.uint8).reshape(N, K // 2)
+    T = -(-N // 16)
+    pad = np.zeros((T * 16, K // 2), np.uint8)
+    pad[:N] = c
+    v = pad.reshape(T, 2, 8, K // 64, 4, 8)  # [tau][row half h][g][kb][t][byte]
+    return np.ascontiguousarray(v.transpose(0, 3, 2, 4, 1, 5)).reshape(-1)
+
+
+@pytest.mark.parametrize("N,K", [(8, 1024), (40, 1024), (1000, 2048), (64, 3072)])
+def test_decode_tiles_layout(qb, N, K):
+    W = torch.randn(N, K, generator=wl.generator(N + K)) * 0.05
+    q = qb.nf4_quantize(W.cuda())
+    T = qb.nf4_decode_tiles(q)
+    torch.cuda.synchronize()
+    assert T.numel() == qb.nf4_decode_tiles_bytes(N, K) == -(-N // 16) * (K // 64) * 512
+    assert np.array_equal(T.cpu().numpy(), tiles_from_codes(q.codes.cpu().numpy(), N, K))
+
+
+def run_fwd_tiles_check(qb, oracle, p, rows=None):
+    q, Wp = quantize_both(qb, oracle, p["W"])
+    T = qb.nf4_decode_tiles(q)
+    X, A, B = p["X"].cuda(), p["A"].cuda(), p["B"].cuda()
+    Y, H = qb.qlora_linear_fwd_tiles(q, T, X, A, B, p["scale"])
+    Yrow, _ = qb.qlora_linear_fwd(q, X, A, B, p["scale"])  # row-major decode kernel
+    torch.cuda.synchronize()
+    Yref = oracle.linear_fwd(bits(p["X"]), Wp, bits(p["A"]), bits(p["B"]), p["scale"], rows=rows)
+    Yg, Yr = Y.float().cpu().numpy(), Yrow.float().cpu().numpy()
+    if rows is not None:
+        Yg, Yr = Yg[rows], Yr[rows]
+    e = relfro(Yg, Yref)
+    assert e <= TOL, f"Y rel err {e}"
+    assert relfro(Yg, Yr) <= 5e-3, "tiles and row-major decode disagree"
+    Href = oracle.lora_h(bits(p["X"]), bits(p["A"]))
+    assert relfro(H.float().cpu().numpy(), Href) <= TOL
+    return e
+
+
+DECODE_TILES = [
+    (1, 40, 1024, 8),      # one item per tile, a ragged last tile
+    (4, 264, 2048, 16),
+    (8, 1000, 4096, 64),   # ragged last tile (1000 = 62 * 16 + 8)
+    (9, 72, 1024, 8),      # two token tiles
+    (16, 520, 3072, 40),   # three items per tile, r not a multiple of 16
+    (3, 8, 1024, 24),      # a single half tile
+    (2, 4096, 5120, 16),   # more tiles than SMs
+]
+
+
+@pytest.mark.parametrize("M,N,K,r", DECODE_TILES)
+def test_forward_decode_tiles(qb, oracle, M, N, K, r):
+    p = wl.draw_small(2500 + M + N, M, N, K, r, 2.0 * r, with_dy=False)
+    run_fwd_tiles_check(qb, oracle, p)
+
+
+def test_decode_tiles_repeatable(qb):
+    """Items of a tile are added in item order: two calls give the same bits."""
+    p = wl.draw_small(2600, 7, 2056, 4096, 16, 32.0, with_dy=False)
+    q = qb.nf4_quantize(p["W"].cuda())
+    T = qb.nf4_decode_tiles(q)
+    X, A, B = p["X"].cuda(), p["A"].cuda(), p["B"].cuda()
+    Y1, _ = qb.qlora_linear_fwd_tiles(q, T, X, A, B, p["scale"])
+    Y2, _ = qb.qlora_linear_fwd_tiles(q, T, X, A, B, p["scale"])
+    assert torch.equal(Y1, Y2)
+
+
+@pytest.mark.parametrize("M,r", [(1, 16), (12, 64)])
+def test_multi_adapter_decode_tiles(qb, oracle, M, r):
+    N, K, na = 1000, 2048, 3
+    p = wl.draw_small(960 + M + r, M, N, K, r, 2.0 * r, with_dy=False)
+    q, Wp = quantize_both(qb, oracle, p["W"])
+    T = qb.nf4_decode_tiles(q)
+    g = wl.generator(970 + M)
+    A_all = ((torch.rand(na, r, K, generator=g) * 2 - 1) / np.sqrt(K)).bfloat16()
+    B_all = (torch.randn(na, N, r, generator=g) * 0.5).bfloat16()
+    scales = torch.tensor([2.0, 0.5, 4.0], dtype=torch.float32)
+    idx = torch.tensor([(2 * m + 1) % na for m in range(M)], dtype=torch.int32)
+    Y = qb.qlora_linear_fwd_multi_tiles(q, T, p["X"].cuda(), A_all.cuda(), B_all.cuda(), scales.cuda(), idx.cuda())
+    torch.cuda.synchronize()
+    Yref = oracle.linear_fwd_multi(bits(p["X"]), Wp, bits(A_all), bits(B_all), scales.double().numpy(),
+                                   idx.numpy().copy())
+    e = relfro(Y.float().cpu().numpy(), Yref)
+    assert e <= TOL, f"Y rel err {e}"
+
+
+def test_decode_tiles_rejects_shapes(qb):
+    q = qb.nf4_quantize(torch.randn(64, 1088, device="cuda") * 0.02)
+    with pytest.raises(qb.QloraError):
+        qb.nf4_decode_tiles(q)  # K % 1024 != 0
+    q = qb.nf4_quantize(torch.randn(64, 1024, device="cuda") * 0.02)
+    T = qb.nf4_decode_tiles(q)
+    X = torch.randn(17, 1024, device="cuda").bfloat16()
+    A = torch.randn(16, 1024, device="cuda").bfloat16()
+    B = torch.randn(64, 16, device="cuda").bfloat16()
+    with pytest.raises(qb.QloraError):
+        qb.qlora_linear_fwd_tiles(q, T, X, A, B, 2.0)  # M > 16
+    assert qb.device_status() == 0
+
+
 def test_decode_repeatable(qb):
     """The decode kernel sums its K-split partials in a fixed order: two calls
     give the same bits."""
@@ -460,6 +566,14 @@ def test_workload_decode_70b_up(qb, oracle, M):
     w = wl.WORKLOADS["decode_70b_up"]
     p = wl.draw_linear(w, M=M)
     run_fwd_check(qb, oracle, p)
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_workload_decode_70b_up_tiles(qb, oracle, M):
+    """The decode workload through the decode tiles, the launch the benchmark times."""
+    w = wl.WORKLOADS["decode_70b_up"]
+    p = wl.draw_linear(w, M=M)
+    run_fwd_tiles_check(qb, oracle, p)
 
 
 @pytest.mark.parametrize("proj", [0, 1, 2])
