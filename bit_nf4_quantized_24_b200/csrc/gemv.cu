@@ -569,22 +569,23 @@ struct UnitX {
   uint32_t x[NTILE][8];
 };
 
-// One unit: 16 lookups, four MMA steps into a fresh fragment per token tile,
-// then the scaled add (rows g: sa, rows g + 8: sb).
+// One unit: the A fragments of four MMA steps from the lane's four code
+// words by 16 lookups (word i = cw.x, .y: row g bytes 0-3, 4-7; cw.z, .w:
+// row g + 8; it fills steps 2(i & 1) and 2(i & 1) + 1), four MMA steps into a
+// fresh fragment per token tile, then the scaled add (rows g: sa, rows g + 8:
+// sb).
 template <int NTILE>
 __device__ __forceinline__ void unit_mma(float (&acc)[NTILE][4], const uint4& cw, const UnitX<NTILE>& in,
                                          uint32_t lane_base, float sa, float sb) {
   uint32_t a[4][4];
+  const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    const uint32_t wg = s < 2 ? cw.x : cw.y, wh = s < 2 ? cw.z : cw.w;
-    if ((s & 1) == 0) {
-      a[s][0] = lut_pair<0>(wg, lane_base); a[s][2] = lut_pair<1>(wg, lane_base);
-      a[s][1] = lut_pair<0>(wh, lane_base); a[s][3] = lut_pair<1>(wh, lane_base);
-    } else {
-      a[s][0] = lut_pair<2>(wg, lane_base); a[s][2] = lut_pair<3>(wg, lane_base);
-      a[s][1] = lut_pair<2>(wh, lane_base); a[s][3] = lut_pair<3>(wh, lane_base);
-    }
+  for (int i = 0; i < 4; ++i) {
+    const int s0 = 2 * (i & 1), h = i >> 1;
+    a[s0][h] = lut_pair<0>(w[i], lane_base);
+    a[s0][h + 2] = lut_pair<1>(w[i], lane_base);
+    a[s0 + 1][h] = lut_pair<2>(w[i], lane_base);
+    a[s0 + 1][h + 2] = lut_pair<3>(w[i], lane_base);
   }
 #pragma unroll
   for (int nt = 0; nt < NTILE; ++nt) {
