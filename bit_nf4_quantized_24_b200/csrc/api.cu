@@ -28,6 +28,16 @@ void** g_trace_events = nullptr;
 int g_trace_pairs = 0;
 int g_trace_count = 0;
 
+// Per-device side stream of the backward: dA and dB run on it while the dX
+// GEMM runs on the caller's stream (fork and join through two events).  The
+// mutex keeps each call's record/wait pairs together.
+struct SideStream {
+  cudaStream_t st = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+SideStream g_side[kMaxDevices];
+std::mutex g_side_mutex;
+
 int current_device() {
   int d = 0;
   cudaGetDevice(&d);
@@ -139,6 +149,29 @@ BwdWorkspace bwd_layout(void* ws, int64_t M, int64_t N, int64_t K, int r) {
   w.H16 = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(M) * r * 2));
   w.bytes = off;
   return w;
+}
+
+// The current device's side stream, created on first use (nullptr if that fails).
+// Call with g_side_mutex held.
+SideStream* side_stream() {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return nullptr;
+  SideStream& ss = g_side[d];
+  if (!ss.st) {
+    cudaStream_t st = nullptr;
+    cudaEvent_t f = nullptr, j = nullptr;
+    if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (cudaEventCreateWithFlags(&f, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&j, cudaEventDisableTiming) != cudaSuccess) {
+      if (f) cudaEventDestroy(f);
+      cudaStreamDestroy(st);
+      return nullptr;
+    }
+    ss.st = st;
+    ss.fork = f;
+    ss.join = j;
+  }
+  return &ss;
 }
 
 }  // namespace
@@ -528,6 +561,34 @@ int qlora_linear_fwd(const uint8_t* codes, const uint8_t* absmax_q, const float*
                               workspace_bytes, stream);
 }
 
+namespace qn {
+namespace {
+// dX = dY deq(W) + dH A: the fused GEMM in its MN-major mode with the LoRA
+// tail (dH, A); a programmatic dependent launch (it waits before the tail).
+cudaError_t launch_dx_gemm(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale, int block,
+                           int dq_block, int64_t N, int64_t K, const uint16_t* dY, int64_t M, const uint16_t* A, int r,
+                           const uint16_t* dH, uint16_t* dX, cudaStream_t s) {
+  GemmArgs a{};
+  a.mode = 1;
+  a.act = dY;
+  a.tail_a = dH;
+  a.tail_b = A;
+  a.codes = codes;
+  a.absmax_q = absmax_q;
+  a.dq_scale = dq_scale;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.r = r;
+  a.out = dX;
+  a.pdl = true;
+  a.block = block;
+  a.dq_block = dq_block;
+  return launch_nf4_gemm(a, s);
+}
+}  // namespace
+}  // namespace qn
+
 int qlora_linear_bwd_fmt(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale, int block,
                          int dq_block, int64_t N, int64_t K, const qlora_bf16_t* X, const qlora_bf16_t* dY, int64_t M,
                          const qlora_bf16_t* A, const qlora_bf16_t* B, int r, float scale, const qlora_bf16_t* H,
@@ -555,40 +616,41 @@ int qlora_linear_bwd_fmt(const uint8_t* codes, const uint8_t* absmax_q, const fl
     if (e == cudaSuccess) e = cudaMemsetAsync(dB, 0, static_cast<size_t>(N) * r * 2, s);
     return cuda_status(e);
   }
-  // Kernel order: dH, (H), dA, dB, then the dX GEMM.  Each kernel after the
-  // first is a programmatic dependent launch that waits for its predecessor
-  // before touching shared data; putting the large GEMM last lets its main
-  // loop start while the adapter kernels finish (only its LoRA tail reads dH).
-  // dH = scale * dY B  (B [N, r] read in place: its rows are the contraction)
+  // dH = scale * dY B  (B [N, r] read in place: its rows are the contraction),
+  // then H if the caller did not keep it.  The second is a programmatic
+  // dependent launch that waits for the first before touching shared data.
   e = launch_rowdot_qt(dY, B, M, N, r, scale, w.dH16, scale, nullptr, nullptr, s, false);
   const uint16_t* Huse = H;
   if (e == cudaSuccess && !H) {
     e = launch_rowdot(X, A, M, K, r, 1.0f, w.H16, 1.0f, nullptr, nullptr, s, true);
     Huse = w.H16;
   }
-  // dA = dH^T X ;  dB = scale * dY^T H
-  if (e == cudaSuccess) e = launch_coldot(w.dH16, X, M, K, r, 1.0f, 0, dA, s, true);
-  if (e == cudaSuccess) e = launch_coldot(Huse, dY, M, N, r, scale, 1, dB, s, true);
-  // dX = dY deq(W) + dH A
-  if (e == cudaSuccess && dX) {
-    GemmArgs a{};
-    a.mode = 1;
-    a.act = dY;
-    a.tail_a = w.dH16;
-    a.tail_b = A;
-    a.codes = codes;
-    a.absmax_q = absmax_q;
-    a.dq_scale = dq_scale;
-    a.M = M;
-    a.N = N;
-    a.K = K;
-    a.r = r;
-    a.out = dX;
-    a.pdl = true;
-    a.block = block;
-    a.dq_block = dq_block;
-    e = launch_nf4_gemm(a, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  // dA = dH^T X and dB = scale * dY^T H do not feed the dX GEMM: they run on
+  // the side stream while the GEMM runs on s, taking the SMs its last,
+  // partial wave leaves idle; the call joins them before it returns.
+  if (dX) {
+    std::lock_guard<std::mutex> lock(g_side_mutex);
+    SideStream* ss = side_stream();
+    if (ss) {
+      e = cudaEventRecord(ss->fork, s);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->st, ss->fork, 0);
+      if (e == cudaSuccess) e = launch_dx_gemm(codes, absmax_q, dq_scale, block, dq_block, N, K, dY, M, A, r,
+                                               w.dH16, dX, s);
+      if (e == cudaSuccess) e = launch_coldot(w.dH16, X, M, K, r, 1.0f, 0, dA, ss->st, false);
+      if (e == cudaSuccess) e = launch_coldot(Huse, dY, M, N, r, scale, 1, dB, ss->st, true);
+      if (e == cudaSuccess) e = cudaEventRecord(ss->join, ss->st);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ss->join, 0);
+      return cuda_status(e);
+    }
   }
+  // one stream: dA, dB, then the dX GEMM (programmatic dependent launches:
+  // the GEMM's main loop starts while the adapter kernels finish; only its
+  // LoRA tail reads dH)
+  e = launch_coldot(w.dH16, X, M, K, r, 1.0f, 0, dA, s, true);
+  if (e == cudaSuccess) e = launch_coldot(Huse, dY, M, N, r, scale, 1, dB, s, true);
+  if (e == cudaSuccess && dX)
+    e = launch_dx_gemm(codes, absmax_q, dq_scale, block, dq_block, N, K, dY, M, A, r, w.dH16, dX, s);
   return cuda_status(e);
 }
 

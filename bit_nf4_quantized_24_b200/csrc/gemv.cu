@@ -526,6 +526,7 @@ constexpr int T_ITEM = 16;                    // blocks per work item
 constexpr int T_GU = 4;                       // units per group of code loads (two groups in flight)
 constexpr int T_SLOTS_MAX = 4;                // tiles whose partial sums can wait for the epilogue
 constexpr int T_SMEM_LIMIT = 231424;          // dynamic shared memory cap (227 KB less 1 KB of static)
+constexpr int T_HS_SMS = 8;                   // SMs of the kernel before this one (the Hs cluster)
 
 __host__ __device__ constexpr int tiles_slot_bytes(int nch, int ntile) { return nch * ntile * 4 * 32 * 4; }
 __host__ __device__ constexpr int tiles_smem_bytes(int nch, int ntile, int ts) {
@@ -870,9 +871,16 @@ cudaError_t gemv_tiles_launch(const uint8_t* tiles, const uint16_t* X, int64_t M
   if (ts < 1) return cudaErrorInvalidValue;  // K too large for one slot of partial sums
   cudaError_t e = smem_limit_once<k_gemv_tiles<NTILE, MULTI>>(T_SMEM_LIMIT);
   if (e != cudaSuccess) return e;
-  const int sms = device_sm_count();
+  // The kernel that computes Hs runs on T_HS_SMS SMs while this one starts
+  // (programmatic dependent launch), and a CTA of this kernel cannot share an
+  // SM with it (it holds the whole register file).  Use the fewest CTAs that
+  // keep the largest per-CTA tile count of a launch that avoids those SMs: the
+  // slowest CTA is as fast as with one CTA per SM, and no CTA waits for the
+  // Hs kernel to leave its SM.
+  const int64_t sms = std::max(1, device_sm_count() - T_HS_SMS);
   const int64_t ntiles = (N + G_ROWS - 1) / G_ROWS;
-  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ntiles, sms));
+  const int64_t per_cta = (ntiles + sms - 1) / sms;
+  const unsigned grid = static_cast<unsigned>((ntiles + per_cta - 1) / per_cta);
   return launch_ex(k_gemv_tiles<NTILE, MULTI>, dim3(grid), dim3(T_THREADS), tiles_smem_bytes(nch, NTILE, ts), st,
                    true, tiles, X, int(M), absmax_q, dq_scale, int(N), int(K), Hs, B, r, host_codebook().levels,
                    aidx, na, ts, 1, Y, device_status_ptr());

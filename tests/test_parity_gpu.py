@@ -396,6 +396,7 @@ DECODE_TILES = [
     (16, 520, 3072, 40),   # three items per tile, r not a multiple of 16
     (3, 8, 1024, 24),      # a single half tile
     (2, 4096, 5120, 16),   # more tiles than SMs
+    (12, 64, 28672, 16),   # 28 items per tile: three slots of partial sums fit shared memory
 ]
 
 
