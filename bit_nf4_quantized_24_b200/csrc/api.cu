@@ -151,13 +151,17 @@ BwdWorkspace bwd_layout(void* ws, int64_t M, int64_t N, int64_t K, int r) {
   return w;
 }
 
-// The current device's side stream, created on first use (nullptr if that fails).
-// Call with g_side_mutex held.
-SideStream* side_stream() {
+// The current device's side stream, created on first use (nullptr if that
+// fails, or if `s` is being captured into a CUDA graph before the side stream
+// exists: creating one inside a capture is not allowed everywhere).  Call with
+// g_side_mutex held.
+SideStream* side_stream(cudaStream_t s) {
   const int d = current_device();
   if (d < 0 || d >= kMaxDevices) return nullptr;
   SideStream& ss = g_side[d];
   if (!ss.st) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) return nullptr;
     cudaStream_t st = nullptr;
     cudaEvent_t f = nullptr, j = nullptr;
     if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
@@ -631,7 +635,7 @@ int qlora_linear_bwd_fmt(const uint8_t* codes, const uint8_t* absmax_q, const fl
   // partial wave leaves idle; the call joins them before it returns.
   if (dX) {
     std::lock_guard<std::mutex> lock(g_side_mutex);
-    SideStream* ss = side_stream();
+    SideStream* ss = side_stream(s);
     if (ss) {
       e = cudaEventRecord(ss->fork, s);
       if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->st, ss->fork, 0);

@@ -231,6 +231,12 @@ int qlora_linear_fwd_multi_tiles(const uint8_t* tiles, const uint8_t* absmax_q, 
  *     dB = scale * dY^T H,  H = X A^T   [N, r]
  * dY: bf16 [M, N].  H: bf16 [M, r] from qlora_linear_fwd's H_save, or NULL to
  * recompute it.  dX, dA, dB: bf16 outputs (dX may be NULL to skip it).
+ * With dX, dA and dB are computed on an internal per-device stream that forks
+ * from `stream` after dH and joins it before the call returns (two events), so
+ * they overlap the dX GEMM; every output is ready when the work enqueued on
+ * `stream` is, also inside a CUDA graph captured from `stream` (the internal
+ * stream is created outside any capture; a first call made during a capture
+ * runs all kernels on `stream`).
  * Same shape rules and errors as qlora_linear_fwd. */
 int qlora_linear_bwd(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale,
                      int64_t N, int64_t K, const qlora_bf16_t* X, const qlora_bf16_t* dY,

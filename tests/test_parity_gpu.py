@@ -523,6 +523,51 @@ def test_decode_and_gemm_paths_agree(qb):
     assert relfro(Yd.float().cpu().numpy(), Yg[:16].float().cpu().numpy()) <= 5e-3
 
 
+def test_fwd_bwd_in_cuda_graph(qb):
+    """The backward forks dA and dB onto a side stream and joins it: the same
+    calls captured in a CUDA graph and replayed give the eager results."""
+    M, N, K, r = 1040, 1024, 2048, 16
+    p = wl.draw_small(95, M, N, K, r, 32.0)
+    q = qb.nf4_quantize(p["W"].cuda())
+    X, A, B, dY = p["X"].cuda(), p["A"].cuda(), p["B"].cuda(), p["dY"].cuda()
+    Y0, H0 = qb.qlora_linear_fwd(q, X, A, B, p["scale"])
+    dX0, dA0, dB0 = qb.qlora_linear_bwd(q, X, dY, A, B, p["scale"], H=H0)
+    torch.cuda.synchronize()
+    Y = torch.empty_like(Y0)
+    H = torch.empty_like(H0)
+    dX, dA, dB = torch.empty_like(dX0), torch.empty_like(dA0), torch.empty_like(dB0)
+    wsf = torch.empty(qb.fwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device="cuda")
+    wsb = torch.empty(qb.bwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device="cuda")
+    L = qb.lib()
+    import ctypes
+
+    def step():
+        st = qb._stream()
+        assert L.qlora_linear_fwd(qb._ptr(q.codes), qb._ptr(q.absmax_q), qb._ptr(q.dq_scale), N, K, qb._ptr(X), M,
+                                  qb._ptr(A), qb._ptr(B), r, ctypes.c_float(p["scale"]), qb._ptr(Y), qb._ptr(H),
+                                  qb._ptr(wsf), wsf.numel(), st) == 0
+        assert L.qlora_linear_bwd(qb._ptr(q.codes), qb._ptr(q.absmax_q), qb._ptr(q.dq_scale), N, K, qb._ptr(X),
+                                  qb._ptr(dY), M, qb._ptr(A), qb._ptr(B), r, ctypes.c_float(p["scale"]), qb._ptr(H),
+                                  qb._ptr(dX), qb._ptr(dA), qb._ptr(dB), qb._ptr(wsb), wsb.numel(), st) == 0
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for t in (Y, H, dX, dA, dB):
+        t.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    for got, ref in ((Y, Y0), (H, H0), (dX, dX0), (dA, dA0), (dB, dB0)):
+        assert torch.equal(got, ref)
+    del g
+    assert qb.device_status() == 0
+
+
 def test_argument_errors_on_device(qb):
     q = qb.nf4_quantize(torch.randn(64, 128, device="cuda") * 0.02)
     X = torch.randn(32, 128, device="cuda").bfloat16()
