@@ -354,6 +354,9 @@ __global__ void __launch_bounds__(32 * (NT / 2 + 1)) k_rows(const __grid_constan
         mma_bf16_16816(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
       }
     }
+    // the stage is refilled by TMA (async proxy): order this warp's reads of
+    // it before the release
+    fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(empty0 + 8u * s);
   }
@@ -474,6 +477,9 @@ __global__ void __launch_bounds__(160) k_cols(const __grid_constant__ CUtensorMa
           mma_bf16_16816(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
         }
       }
+      // the stage is refilled by TMA (async proxy): order this warp's reads
+      // of it before the release
+      fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(empty0 + 8u * s);
     }

@@ -424,6 +424,9 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         blocks_mma<NTILE, 1>(acc, in, ca, lane_base, sc);
     }
     if (more) load_next();
+    // the stage is refilled by TMA (async proxy): order this warp's reads of
+    // it before the release
+    fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(empty0 + 8u * slot);
     if (++slot == NS) {

@@ -523,6 +523,33 @@ def test_decode_and_gemm_paths_agree(qb):
     assert relfro(Yd.float().cpu().numpy(), Yg[:16].float().cpu().numpy()) <= 5e-3
 
 
+def test_backward_repeatable_large(qb):
+    """dA and dB come out bit for bit the same on every call, with the dX GEMM
+    (dA, dB on the side stream) and without it, at a shape with thousands of
+    column-kernel CTAs: the TMA rings release a stage only after the
+    consumers' reads of it are ordered before the refill."""
+    M, N, K, r = 4096, 8192, 28672, 64
+    g = wl.generator(97)
+    X = torch.randn(M, K, generator=g).bfloat16().cuda()
+    dY = torch.randn(M, N, generator=g).bfloat16().cuda()
+    A = ((torch.rand(r, K, generator=g) * 2 - 1) / np.sqrt(K)).bfloat16().cuda()
+    B = (torch.randn(N, r, generator=g) * 0.01).bfloat16().cuda()
+    q = qb.nf4_quantize(torch.randn(N, K, generator=g).cuda() * 0.02)
+    _, H = qb.qlora_linear_fwd(q, X[:16].contiguous(), A, B, 0.25)
+    H = (X.float() @ A.float().t()).bfloat16()
+    ref = None
+    for want_dx in (True, False, True, False, True):
+        _, dA, dB = qb.qlora_linear_bwd(q, X, dY, A, B, 0.25, H=H, want_dx=want_dx)
+        torch.cuda.synchronize()
+        if ref is None:
+            ref = (dA.clone(), dB.clone())
+        assert torch.equal(dA, ref[0]) and torch.equal(dB, ref[1])
+    dH = (0.25 * (dY.float() @ B.float())).bfloat16().float()
+    dA_t = dH.t() @ X.float()
+    assert relfro(ref[0].float().cpu().numpy(), dA_t.cpu().numpy()) <= 5e-3
+    assert qb.device_status() == 0
+
+
 def test_fwd_bwd_in_cuda_graph(qb):
     """The backward forks dA and dB onto a side stream and joins it: the same
     calls captured in a CUDA graph and replayed give the eager results."""
