@@ -126,21 +126,6 @@ cudaError_t smem_limit_once(int bytes) {
   if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
   return e;
 }
-// Asks for the largest shared-memory carve-out for kernel KERN on the current
-// device, once per device (so that several CTAs with static shared memory fit
-// an SM).
-template <auto KERN>
-cudaError_t carveout_max_once() {
-  static std::atomic<uint64_t> done{0};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
-  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
-  e = cudaFuncSetAttribute(KERN, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
-  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
-  return e;
-}
 // Streaming multiprocessors of the current device (cached per device).
 int device_sm_count();
 

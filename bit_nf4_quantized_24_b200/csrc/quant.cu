@@ -9,8 +9,6 @@
 // code): t = fl32(w / a_b); code = number of midpoints strictly below t; an
 // all-zero block encodes the zero level; s2 = fl32(max a / 255);
 // q = min(255, rint(fl32(a / s2))).
-#include <algorithm>
-
 #include "internal.h"
 
 namespace qn {
@@ -25,20 +23,17 @@ constexpr int kGroup = 256;  // blocks per double-quant group (and per quantize 
 // spacing is above 1/32) and none lies on a cell edge, so
 // code = base[j] + (t > mid[j]) with base[j] = midpoints below the cell and
 // mid[j] = the midpoint inside it (+inf if none).  rn(64 t) + 64 is read from
-// the low mantissa bits of fl32(64 t + 1.5 * 2^23 + 64); the index is clamped
-// to the last cell so a non-finite t (its block is reported) still reads
-// inside the table.  Each lane reads its own copy of the table (cell j of lane
-// l at [j][l]), so the lookups of a warp never share a bank pair.
+// the low mantissa bits of fl32(64 t + 1.5 * 2^23 + 64); the index is masked to
+// 8 bits so a non-finite t (its block is reported) still reads inside the table.
 struct Cell {
   int base;
   float mid;
 };
-constexpr int kCells = 129;
+constexpr int kCells = 256;
 
-__device__ __forceinline__ int nf4_code(float t, const Cell (*cells)[32], int lane) {
+__device__ __forceinline__ int nf4_code(float t, const Cell* cells) {
   const float f = __fmaf_rn(t, 64.0f, 12582976.0f);
-  const uint32_t j = min(static_cast<uint32_t>(__float_as_int(f) - 0x4B400000), static_cast<uint32_t>(kCells - 1));
-  const Cell c = cells[j][lane];
+  const Cell c = cells[(__float_as_int(f) - 0x4B400000) & (kCells - 1)];
   return c.base + (t > c.mid ? 1 : 0);
 }
 
@@ -101,28 +96,31 @@ __device__ __forceinline__ float4 merged4(const MergeSrc& m, const float* lv, in
                      __fadd_rn(w[2], __fmul_rn(m.s, acc[2])), __fadd_rn(w[3], __fmul_rn(m.s, acc[3])));
 }
 
-// A CTA walks groups of 256 blocks (the double-quant group) with a stride of
-// the grid.  A block of B weights is spread over LP = min(32, B / 4) lanes,
-// F = B / (4 LP) float4s per lane; a warp covers 32 / LP blocks per step, and
-// four steps' loads are issued before any is used, to keep HBM busy.  DQ:
-// double quantization of the group's absmax values (else each block's fp32
-// absmax is stored as is).
+// One CTA per group of 256 blocks (the double-quant group).  A block of B
+// weights is spread over LP = min(32, B / 4) lanes, F = B / (4 LP) float4s per
+// lane; a warp covers 32 / LP blocks per step, and four steps' loads are
+// issued before any is used, to keep HBM busy.  DQ: double quantization of the
+// group's absmax values (else each block's fp32 absmax is stored as is).
 template <int B, bool DQ, bool MERGE>
-__global__ void __launch_bounds__(256) k_quantize(const float* W, MergeSrc msrc, Nf4Levels levels,
+__global__ void __launch_bounds__(256) k_quantize(const float* __restrict__ W, MergeSrc msrc, Nf4Levels levels,
                                                   int64_t nblocks, Nf4Mids mids, uint8_t* __restrict__ codes,
                                                   uint8_t* __restrict__ absmax_q, float* __restrict__ dq_scale,
                                                   int* nonfinite) {
   constexpr int LP = B / 4 < 32 ? B / 4 : 32;
   constexpr int F = B / (4 * LP);
   constexpr int BPW = 32 / LP;  // blocks per warp step
-  __shared__ Cell s_cell[kCells][32];
+  __shared__ Cell s_cell[kCells];
   __shared__ float s_amax[kGroup];
   __shared__ float s_red[8];
   __shared__ float s_lv[16];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int sub = lane / LP, sl = lane % LP;
   if (MERGE && tid < 16) s_lv[tid] = levels.v[tid];
-  if (tid < kCells) {  // cell tid, written to the 32 lane copies (rotated so the stores spread over the banks)
+  const int64_t g = blockIdx.x;
+  const int64_t b0 = g * kGroup;
+  const int64_t rem = nblocks - b0;
+  const int nb = rem < kGroup ? static_cast<int>(rem) : kGroup;
+  {  // cell table (kCells == blockDim.x)
     const float lo = (static_cast<float>(tid) - 64.5f) * 0.015625f, hi = lo + 0.015625f;
     int base = 0;
     float mid = __int_as_float(0x7f800000);
@@ -130,98 +128,92 @@ __global__ void __launch_bounds__(256) k_quantize(const float* W, MergeSrc msrc,
       base += mids.v[i] < lo ? 1 : 0;
       if (mids.v[i] > lo && mids.v[i] < hi) mid = mids.v[i];
     }
-    for (int l = 0; l < 32; ++l) s_cell[tid][(l + tid) & 31] = Cell{base, mid};
+    s_cell[tid] = Cell{base, mid};
   }
   __syncthreads();
 
-  const int64_t ngroups = (nblocks + kGroup - 1) / kGroup;
+  const int nsteps = (nb + BPW - 1) / BPW;
   float nan_probe = 0.0f;  // becomes NaN if any weight is NaN or infinite (x * 0)
-  for (int64_t g = blockIdx.x; g < ngroups; g += gridDim.x) {
-    const int64_t b0 = g * kGroup;
-    const int64_t rem = nblocks - b0;
-    const int nb = rem < kGroup ? static_cast<int>(rem) : kGroup;
-    const int nsteps = (nb + BPW - 1) / BPW;
-    for (int p0 = warp; p0 < nsteps; p0 += 32) {
-      float4 x[4][F];
-      bool ok[4];
+  for (int p0 = warp; p0 < nsteps; p0 += 32) {
+    float4 x[4][F];
+    bool ok[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = BPW * (p0 + 8 * u) + sub;
-        ok[u] = (p0 + 8 * u < nsteps) && (i < nb);
+    for (int u = 0; u < 4; ++u) {
+      const int i = BPW * (p0 + 8 * u) + sub;
+      ok[u] = (p0 + 8 * u < nsteps) && (i < nb);
 #pragma unroll
-        for (int f = 0; f < F; ++f) {
-          if (MERGE)
-            x[u][f] = ok[u] ? merged4(msrc, s_lv, (b0 + i) * B + (f * LP + sl) * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
-          else
-            x[u][f] = ok[u] ? __ldcs(reinterpret_cast<const float4*>(W + (b0 + i) * B) + f * LP + sl)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
+      for (int f = 0; f < F; ++f) {
+        if (MERGE)
+          x[u][f] = ok[u] ? merged4(msrc, s_lv, (b0 + i) * B + (f * LP + sl) * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        else
+          x[u][f] = ok[u] ? __ldcs(reinterpret_cast<const float4*>(W + (b0 + i) * B) + f * LP + sl)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (p0 + 8 * u >= nsteps) break;  // warp-uniform
+      const int i = BPW * (p0 + 8 * u) + sub;
+      float m = 0.0f;
+#pragma unroll
+      for (int f = 0; f < F; ++f) {
+        const float4 v = x[u][f];
+        nan_probe = __fmaf_rn(v.x, 0.0f, __fmaf_rn(v.y, 0.0f, __fmaf_rn(v.z, 0.0f, __fmaf_rn(v.w, 0.0f, nan_probe))));
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (p0 + 8 * u >= nsteps) break;  // warp-uniform
-        const int i = BPW * (p0 + 8 * u) + sub;
-        float m = 0.0f;
+      for (int off = LP / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      if (ok[u]) {
+        const bool fast = m >= 0x1p-100f && m <= 0x1p100f;
+        const float r = fast ? __frcp_rn(m) : 0.0f;
 #pragma unroll
         for (int f = 0; f < F; ++f) {
           const float4 v = x[u][f];
-          nan_probe = __fmaf_rn(v.x, 0.0f, __fmaf_rn(v.y, 0.0f, __fmaf_rn(v.z, 0.0f, __fmaf_rn(v.w, 0.0f, nan_probe))));
-          m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+          uint32_t c;
+          if (m == 0.0f) {
+            c = 0x7777u;  // an all-zero block encodes the zero level
+          } else if (fast) {
+            c = nf4_code(div_by_absmax(v.x, m, r), s_cell) | (nf4_code(div_by_absmax(v.y, m, r), s_cell) << 4) |
+                (nf4_code(div_by_absmax(v.z, m, r), s_cell) << 8) |
+                (nf4_code(div_by_absmax(v.w, m, r), s_cell) << 12);
+          } else {
+            c = nf4_code(__fdiv_rn(v.x, m), s_cell) | (nf4_code(__fdiv_rn(v.y, m), s_cell) << 4) |
+                (nf4_code(__fdiv_rn(v.z, m), s_cell) << 8) | (nf4_code(__fdiv_rn(v.w, m), s_cell) << 12);
+          }
+          reinterpret_cast<uint16_t*>(codes + (b0 + i) * (B / 2))[f * LP + sl] = static_cast<uint16_t>(c);
         }
-#pragma unroll
-        for (int off = LP / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-        if (ok[u]) {
-          const bool fast = m >= 0x1p-100f && m <= 0x1p100f;
-          const float r = fast ? __frcp_rn(m) : 0.0f;
-#pragma unroll
-          for (int f = 0; f < F; ++f) {
-            const float4 v = x[u][f];
-            uint32_t c;
-            if (m == 0.0f) {
-              c = 0x7777u;  // an all-zero block encodes the zero level
-            } else if (fast) {
-              c = nf4_code(div_by_absmax(v.x, m, r), s_cell, lane) |
-                  (nf4_code(div_by_absmax(v.y, m, r), s_cell, lane) << 4) |
-                  (nf4_code(div_by_absmax(v.z, m, r), s_cell, lane) << 8) |
-                  (nf4_code(div_by_absmax(v.w, m, r), s_cell, lane) << 12);
-            } else {
-              c = nf4_code(__fdiv_rn(v.x, m), s_cell, lane) | (nf4_code(__fdiv_rn(v.y, m), s_cell, lane) << 4) |
-                  (nf4_code(__fdiv_rn(v.z, m), s_cell, lane) << 8) |
-                  (nf4_code(__fdiv_rn(v.w, m), s_cell, lane) << 12);
-            }
-            reinterpret_cast<uint16_t*>(codes + (b0 + i) * (B / 2))[f * LP + sl] = static_cast<uint16_t>(c);
-          }
-          if (sl == 0) {
-            if (DQ)
-              s_amax[i] = m;
-            else
-              dq_scale[b0 + i] = m;
-          }
+        if (sl == 0) {
+          if (DQ)
+            s_amax[i] = m;
+          else
+            dq_scale[b0 + i] = m;
         }
       }
     }
-    if (!DQ) continue;
-    __syncthreads();  // the group's absmax values are in s_amax
-
-    // double quantization of the group's absmax values
-    float m = (tid < nb) ? s_amax[tid] : 0.0f;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    if (lane == 0) s_red[warp] = m;
-    __syncthreads();
-    float c2 = s_red[0];
-#pragma unroll
-    for (int w = 1; w < 8; ++w) c2 = fmaxf(c2, s_red[w]);
-    const float s2 = (c2 > 0.0f) ? __fdiv_rn(c2, 255.0f) : 0.0f;
-    if (tid < nb) {
-      uint8_t q = 0;
-      if (s2 != 0.0f) q = static_cast<uint8_t>(fminf(255.0f, rintf(__fdiv_rn(s_amax[tid], s2))));
-      absmax_q[b0 + tid] = q;
-    }
-    if (tid == 0) dq_scale[g] = s2;
-    __syncthreads();  // s_amax and s_red are reused by the next group
   }
   const bool bad = !(nan_probe == 0.0f);
+  if (!DQ) {
+    if (__syncthreads_or(bad) && tid == 0) atomicExch(nonfinite, 1);
+    return;
+  }
+  __syncthreads();
+
+  // double quantization of the group's absmax values
+  float m = (tid < nb) ? s_amax[tid] : 0.0f;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if (lane == 0) s_red[warp] = m;
+  __syncthreads();
+  float c2 = s_red[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) c2 = fmaxf(c2, s_red[w]);
+  const float s2 = (c2 > 0.0f) ? __fdiv_rn(c2, 255.0f) : 0.0f;
+  if (tid < nb) {
+    uint8_t q = 0;
+    if (s2 != 0.0f) q = static_cast<uint8_t>(fminf(255.0f, rintf(__fdiv_rn(s_amax[tid], s2))));
+    absmax_q[b0 + tid] = q;
+  }
+  if (tid == 0) dq_scale[g] = s2;
   if (__syncthreads_or(bad) && tid == 0) atomicExch(nonfinite, 1);
 }
 
@@ -286,17 +278,12 @@ cudaError_t quantize_launch(const float* W, const MergeSrc* merge, int64_t numel
   const int64_t ngroups = (nblocks + kGroup - 1) / kGroup;
   if (ngroups == 0) return cudaSuccess;
   const HostCodebook& cb = host_codebook();
-  // CTAs stride over the groups: six fit an SM (34 KB of shared memory each),
-  // so the per-lane cell table is built once per resident CTA
-  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ngroups, int64_t(6) * device_sm_count()));
-  cudaError_t e = merge ? carveout_max_once<k_quantize<B, DQ, true>>() : carveout_max_once<k_quantize<B, DQ, false>>();
-  if (e != cudaSuccess) return e;
   if (merge)
-    k_quantize<B, DQ, true><<<grid, 256, 0, st>>>(nullptr, *merge, cb.levels, nblocks, cb.mids, codes, absmax_q,
-                                                  dq_scale, nonfinite);
+    k_quantize<B, DQ, true><<<static_cast<unsigned>(ngroups), 256, 0, st>>>(
+        nullptr, *merge, cb.levels, nblocks, cb.mids, codes, absmax_q, dq_scale, nonfinite);
   else
-    k_quantize<B, DQ, false><<<grid, 256, 0, st>>>(W, MergeSrc{}, cb.levels, nblocks, cb.mids, codes, absmax_q,
-                                                   dq_scale, nonfinite);
+    k_quantize<B, DQ, false><<<static_cast<unsigned>(ngroups), 256, 0, st>>>(
+        W, MergeSrc{}, cb.levels, nblocks, cb.mids, codes, absmax_q, dq_scale, nonfinite);
   return cudaGetLastError();
 }
 
