@@ -13,6 +13,9 @@ stream and the per-step times are summed.
 Also reported: the fused dequant-GEMM kernel against the tensor-core roofline
 (events around each launch), the decode GEMV weight stream (70B-shaped up
 projection, 1/4/16 tokens) and nf4_quantize against HBM bandwidth, an
+fwd + bwd of the 7B MLP and 70B decoder-layer projections and the 2048 x 2048
+forward at 128 tokens (with a dense torch bf16 matmul of each forward shape as a
+library ceiling), an
 end-to-end number with host buffers (pinned host -> device copies of X and dY,
 device -> host copies of Y, dX, dA, dB inside the timed region), SM clocks
 sampled through NVML during the timed region, and the CPU oracle timed on the
@@ -517,7 +520,86 @@ def run_extras(qb, wl, dev, pk, flush):
                              "note": "includes the call's stream synchronization (non-finite check)"}
     del Wd, out, W2, X2, Y2
     torch.cuda.empty_cache()
+    res["configs"] = run_configs(qb, wl, dev, pk, timed)
     return res
+
+
+def run_configs(qb, wl, dev, pk, timed):
+    """The other configurations: the 2048 x 2048 forward at 128 tokens
+    (latency-bound, in us), and fwd + bwd of every projection of the 7B MLP and
+    of the 70B decoder layer against the tensor roofline (and the one-time
+    quantize of the layer's seven weights).  Timing inputs of the same shapes
+    and distributions are drawn on the device (parity of these shapes is in
+    the GPU tests).  Beside each projection: a dense torch bf16 matmul of the
+    forward shape on the dequantized weight, as a library ceiling."""
+    import ctypes
+
+    import torch
+    L = qb.lib()
+    P = qb._ptr
+    f32 = ctypes.c_float
+    out = {}
+    g = torch.Generator(device=dev)
+    for name in ("fwd_2048", "mlp_7b", "layer_70b"):
+        w = wl.WORKLOADS[name]
+        g.manual_seed(1000 + w.seed)
+        M, r, s = w.M, w.r, w.scale
+        per, tot_ms, tot_flops, q_ms = {}, 0.0, 0, 0.0
+        for pr in w.projections:
+            N, K = pr.N, pr.K
+            W = torch.randn(N, K, device=dev, generator=g) * w.w_std
+            q_ms += timed(lambda: qb.nf4_quantize(W), n=3)
+            q = qb.nf4_quantize(W)
+            del W
+            X = torch.randn(M, K, device=dev, generator=g).bfloat16()
+            A = ((torch.rand(r, K, device=dev, generator=g) * 2 - 1) / K ** 0.5).bfloat16()
+            B = (torch.randn(N, r, device=dev, generator=g) * w.b_std).bfloat16()
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            H = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
+            wsf = torch.empty(qb.fwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+            if w.backward:
+                dY = torch.randn(M, N, device=dev, generator=g).bfloat16()
+                wsb = torch.empty(qb.bwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+                dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+                dA = torch.empty(r, K, dtype=torch.bfloat16, device=dev)
+                dB = torch.empty(N, r, dtype=torch.bfloat16, device=dev)
+
+                def step():  # as the headline step: H saved by the forward, read by the backward
+                    st = qb._stream()
+                    e = L.qlora_linear_fwd(P(q.codes), P(q.absmax_q), P(q.dq_scale), N, K, P(X), M, P(A), P(B), r,
+                                           f32(s), P(Y), P(H), P(wsf), wsf.numel(), st)
+                    if e == 0:
+                        e = L.qlora_linear_bwd(P(q.codes), P(q.absmax_q), P(q.dq_scale), N, K, P(X), P(dY), M, P(A),
+                                               P(B), r, f32(s), P(H), P(dX), P(dA), P(dB), P(wsb), wsb.numel(), st)
+                    if e:
+                        raise qb.QloraError(e, "configs step")
+                flops = 4 * M * N * K + 6 * M * r * (K + N)
+            else:
+                def step():
+                    e = L.qlora_linear_fwd(P(q.codes), P(q.absmax_q), P(q.dq_scale), N, K, P(X), M, P(A), P(B), r,
+                                           f32(s), P(Y), None, P(wsf), wsf.numel(), qb._stream())
+                    if e:
+                        raise qb.QloraError(e, "configs fwd")
+                flops = 2 * M * N * K + 2 * M * r * (K + N)
+            ms = timed(step, n=10)
+            Wd = qb.nf4_dequantize(q)
+            ms_c = timed(lambda: torch.matmul(X, Wd.t()), n=10)
+            per[pr.name] = {"N": N, "K": K, "ms": round(ms, 4), "tflops": round(flops / ms / 1e9, 1),
+                            "torch_bf16_matmul_fwd_tflops": round(2 * M * N * K / ms_c / 1e9, 1)}
+            tot_ms += ms
+            tot_flops += flops
+            del q, X, A, B, Y, H, wsf, Wd
+            if w.backward:
+                del dY, wsb, dX, dA, dB
+            torch.cuda.empty_cache()
+        entry = {"M": M, "r": r, "pass": "fwd+bwd" if w.backward else "fwd", "ms": round(tot_ms, 4),
+                 "tflops": round(tot_flops / tot_ms / 1e9, 1),
+                 "frac_tensor": round(tot_flops / tot_ms / 1e9 / pk["bf16_tflops"], 4),
+                 "quantize_ms": round(q_ms, 4), "projections": per}
+        if name == "fwd_2048":
+            entry["us"] = round(tot_ms * 1e3, 1)
+        out[name] = entry
+    return out
 
 
 # -------------------------------------------------------- reference arm
