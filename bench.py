@@ -164,25 +164,34 @@ class ClockSampler:
 # -------------------------------------------------------------- CPU oracle
 
 
-def oracle_sample(rows_sample: int | None = None):
+def oracle_prepare():
+    """Inputs of the workload for the CPU oracle: drawn on the host, quantized
+    and dequantized by the oracle (done once, outside any timed region)."""
+    import oracle
+    from bit_nf4_quantized_24_b200 import workloads as wl
+    w = wl.WORKLOADS[WORKLOAD]
+    p = wl.draw_linear(w)
+    N, K = p["N"], p["K"]
+    oc, oa, od, _ = oracle.nf4_quantize(p["W"].numpy())
+    _, Wp = oracle.nf4_dequantize(oc, oa, od, N, K)
+    bits = wl.bf16_bits
+    return {"M": p["M"], "N": N, "K": K, "r": p["r"], "scale": p["scale"], "Wp": Wp,
+            "X": bits(p["X"]), "A": bits(p["A"]), "B": bits(p["B"]), "dY": bits(p["dY"])}
+
+
+def oracle_run(prep, rows_sample: int | None = None):
     """Times the CPU oracle on a bounded sample of the workload: Y and dX for
     `rows_sample` token rows, H, dH, dA, dB in full.  Returns (TFLOP/s, cores,
     sample description, seconds)."""
     import numpy as np
 
     import oracle
-    from bit_nf4_quantized_24_b200 import workloads as wl
-    w = wl.WORKLOADS[WORKLOAD]
-    p = wl.draw_linear(w)
-    M, N, K, r = p["M"], p["N"], p["K"], p["r"]
-    oc, oa, od, _ = oracle.nf4_quantize(p["W"].numpy())
-    _, Wp = oracle.nf4_dequantize(oc, oa, od, N, K)
-    bits = wl.bf16_bits
-    X, A, B, dY = bits(p["X"]), bits(p["A"]), bits(p["B"]), bits(p["dY"])
+    M, N, K, r = prep["M"], prep["N"], prep["K"], prep["r"]
+    X, A, B, dY, Wp = prep["X"], prep["A"], prep["B"], prep["dY"], prep["Wp"]
     rows = np.arange(M, dtype=np.int64) if rows_sample is None else np.linspace(0, M - 1, rows_sample).astype(np.int64)
     t0 = time.perf_counter()
-    oracle.linear_fwd(X, Wp, A, B, p["scale"], rows=rows)
-    oracle.linear_bwd(X, dY, Wp, A, B, p["scale"], rows=rows)
+    oracle.linear_fwd(X, Wp, A, B, prep["scale"], rows=rows)
+    oracle.linear_bwd(X, dY, Wp, A, B, prep["scale"], rows=rows)
     dt = time.perf_counter() - t0
     S = len(rows)
     flops = S * (2 * K * r + 2 * N * K + 2 * N * r)          # forward rows
@@ -192,6 +201,10 @@ def oracle_sample(rows_sample: int | None = None):
     desc = (f"{WORKLOAD} (M={M}, N={N}, K={K}, r={r}): Y and dX for {S} of {M} token rows, "
             f"H, dH, dA, dB in full; one fwd+bwd pass of the fp64 oracle")
     return flops / dt / 1e12, oracle.num_threads(), desc, dt
+
+
+def oracle_sample(rows_sample: int | None = None):
+    return oracle_run(oracle_prepare(), rows_sample)
 
 
 # -------------------------------------------------------------- our arm
@@ -607,18 +620,29 @@ def run_configs(qb, wl, dev, pk, timed):
 
 def run_reference(args, rank, world):
     """The reference arm is the CPU oracle (this method has no runnable
-    reference implementation): it is timed as it stands on the host cores."""
+    reference implementation): it is timed as it stands on the host cores,
+    W untimed and K timed steps, each step one bounded sample of the workload
+    (the row count of a sample shrinks only if the whole run would otherwise
+    take more than about 150 s)."""
     if rank != 0:
         return
-    vals = []
+    prep = oracle_prepare()
+    rows = 512
+    n_total = max(1, args.warmup + args.steps)
+    budget_s = 150.0
     cores = desc = None
-    for _ in range(max(1, args.steps if args.steps <= 3 else 3)):
-        tf, cores, desc, dt = oracle_sample(rows_sample=512)
+    for i in range(args.warmup):
+        _, cores, desc, dt = oracle_run(prep, rows)
+        if i == 0 and dt * n_total > budget_s:
+            rows = max(32, int(rows * budget_s / (dt * n_total)) // 32 * 32)
+    vals = []
+    for _ in range(max(1, args.steps)):
+        tf, cores, desc, dt = oracle_run(prep, rows)
         vals.append(tf)
     v = statistics.median(vals)
     out = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
-           "steps": len(vals), "warmup": 0, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-           "dtype": "f64", "data": "synthetic (seeded; see workloads.py)",
+           "steps": len(vals), "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; see workloads.py)",
            "config": {"workload": f"{WORKLOAD} (bounded sample, see cpu_baseline.sample)"},
            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
