@@ -260,7 +260,9 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             dp.allreduce_adapter_grads(dA, dB)
 
-    launches_per_step = 2 + 6  # fwd: rows, gemm; bwd: rows, gemm, 2x(cols partial + reduce)
+    # our kernels per step (the ncu launch list shows the same): forward k_rows (H) and
+    # k_nf4_gemm; backward k_rows (dH), two k_cols (dA, dB) and k_nf4_gemm (dX)
+    launches_per_step = 2 + 4
 
     for _ in range(args.warmup):
         step()
