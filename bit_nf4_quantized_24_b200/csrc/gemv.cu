@@ -504,7 +504,7 @@ namespace {
 // L = 4g + t of a warp owns bytes 16L .. 16L+15: the code bytes 8t .. 8t+7 of
 // block kb in row 16 tau + g, then the same bytes of row 16 tau + g + 8 (rows
 // past N hold zeros).  The units of a tile follow in kb order, so a tile is
-// one contiguous run of 8 K bytes, a warp reads a unit with one 128-bit load
+// one contiguous run of 8 * K bytes, a warp reads a unit with one 128-bit load
 // per lane, and the bytes land in exactly the registers the lookups of the
 // row-major kernel above build from shared memory.
 //
@@ -547,9 +547,9 @@ __device__ __forceinline__ void prefetch_l1(const void* p) {
 __device__ __forceinline__ uint4 ldg_v4(const void* p) {  // activations and absmax bytes: keep them in L1
   return __ldg(reinterpret_cast<const uint4*>(p));
 }
-// The same load issued only by lanes with `on` set (others get zeros): the
+// The same load issued only by lanes with `on` set (others get zeros); the
 // predicate is explicit so the compiler cannot turn it into a load by every
-// lane, and the L1 returns only the active lanes' bytes.
+// lane.
 __device__ __forceinline__ uint4 ldg_v4_if(const void* p, bool on) {
   uint4 v;
   asm volatile(
@@ -743,9 +743,7 @@ __global__ void __launch_bounds__(T_THREADS, 1)
     return tiles + static_cast<int64_t>(t0 + ti) * tile_bytes + static_cast<int64_t>(ch) * (T_ITEM * T_UNIT) + lane * 16;
   };
   // Lanes of token rows >= M load nothing and hold zeros (those columns are
-  // never stored): the loads return only the bytes of real tokens, which
-  // matters because every byte a load returns costs the same L1 bandwidth
-  // as the table lookups.
+  // never stored).
   const uint16_t* xrow[NTILE];
   bool xon[NTILE];
 #pragma unroll
