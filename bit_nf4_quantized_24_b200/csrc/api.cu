@@ -639,13 +639,14 @@ int qlora_linear_bwd_fmt(const uint8_t* codes, const uint8_t* absmax_q, const fl
     if (ss) {
       e = cudaEventRecord(ss->fork, s);
       if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->st, ss->fork, 0);
-      if (e == cudaSuccess) e = launch_dx_gemm(codes, absmax_q, dq_scale, block, dq_block, N, K, dY, M, A, r,
-                                               w.dH16, dX, s);
+      if (e != cudaSuccess) return cuda_status(e);
+      e = launch_dx_gemm(codes, absmax_q, dq_scale, block, dq_block, N, K, dY, M, A, r, w.dH16, dX, s);
       if (e == cudaSuccess) e = launch_coldot(w.dH16, X, M, K, r, 1.0f, 0, dA, ss->st, false);
       if (e == cudaSuccess) e = launch_coldot(Huse, dY, M, N, r, scale, 1, dB, ss->st, true);
-      if (e == cudaSuccess) e = cudaEventRecord(ss->join, ss->st);
-      if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ss->join, 0);
-      return cuda_status(e);
+      // join on every path, so that nothing of this call stays unordered with `s`
+      cudaError_t j = cudaEventRecord(ss->join, ss->st);
+      if (j == cudaSuccess) j = cudaStreamWaitEvent(s, ss->join, 0);
+      return cuda_status(e != cudaSuccess ? e : j);
     }
   }
   // one stream: dA, dB, then the dX GEMM (programmatic dependent launches:
