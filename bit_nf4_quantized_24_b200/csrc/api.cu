@@ -73,24 +73,9 @@ T* symbol_ptr(T** cache, const void* symbol) {
   return cache[d];
 }
 
-int cuda_status(cudaError_t e) {
-  if (e == cudaSuccess) return QLORA_OK;
-  t_last_cuda_error = static_cast<int>(e);
-  return QLORA_ERR_CUDA;
-}
-
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
-
-// Shape rules shared by the layer entry points.
-int check_layer_shapes(int64_t M, int64_t N, int64_t K, int r) {
-  if (M < 0 || N <= 0 || K <= 0) return QLORA_ERR_ARG;
-  if (r < 8 || r > 64 || r % 8) return r <= 0 ? QLORA_ERR_ARG : QLORA_ERR_UNSUPPORTED;
-  if (K % 64 || N % 8) return QLORA_ERR_SHAPE;
-  if (M > (1 << 24) || N > (1 << 24) || K > (1 << 24) || N * K / 2 > (int64_t(1) << 40)) return QLORA_ERR_SHAPE;
-  return QLORA_OK;
-}
 
 // Scratch of the dropout variants: Xd [M, K] bf16 and a zero [M, r] bf16
 // tail (the dX GEMM then adds no adapter term; k_dx_add_masked does, masked).
@@ -111,12 +96,6 @@ DropWorkspace drop_layout(void* ws, size_t off0, int64_t M, int64_t K, int r) {
   return w;
 }
 
-// The NF4 formats the layer reads: block in {32, 64, 128, 256}, dq_block 256 or 0.
-int check_format(int64_t K, int block, int dq_block) {
-  if ((block != 32 && block != 64 && block != 128 && block != 256) || (dq_block != 256 && dq_block != 0))
-    return QLORA_ERR_UNSUPPORTED;
-  return K % block ? QLORA_ERR_SHAPE : QLORA_OK;
-}
 
 struct FwdWorkspace {
   uint16_t* Hs;  // bf16(scale * X A^T) [M, r]
@@ -179,6 +158,26 @@ SideStream* side_stream(cudaStream_t s) {
 }
 
 }  // namespace
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return QLORA_OK;
+  t_last_cuda_error = static_cast<int>(e);
+  return QLORA_ERR_CUDA;
+}
+
+int check_layer_shapes(int64_t M, int64_t N, int64_t K, int r) {
+  if (M < 0 || N <= 0 || K <= 0) return QLORA_ERR_ARG;
+  if (r < 8 || r > 64 || r % 8) return r <= 0 ? QLORA_ERR_ARG : QLORA_ERR_UNSUPPORTED;
+  if (K % 64 || N % 8) return QLORA_ERR_SHAPE;
+  if (M > (1 << 24) || N > (1 << 24) || K > (1 << 24) || N * K / 2 > (int64_t(1) << 40)) return QLORA_ERR_SHAPE;
+  return QLORA_OK;
+}
+
+int check_format(int64_t K, int block, int dq_block) {
+  if ((block != 32 && block != 64 && block != 128 && block != 256) || (dq_block != 256 && dq_block != 0))
+    return QLORA_ERR_UNSUPPORTED;
+  return K % block ? QLORA_ERR_SHAPE : QLORA_OK;
+}
 
 int* device_status_ptr() { return symbol_ptr(g_status_ptr, &g_device_status); }
 int* device_nonfinite_ptr() { return symbol_ptr(g_nonfinite_ptr, &g_nonfinite); }

@@ -25,6 +25,15 @@ struct HostCodebook {
 };
 const HostCodebook& host_codebook();
 
+// Status of a CUDA runtime result for the C ABI: QLORA_OK, or QLORA_ERR_CUDA
+// after recording the error for qlora_last_cuda_error() on this host thread.
+int cuda_status(cudaError_t e);
+// Shape rules of the layer entry points (M, N, K, r; QLORA_OK or the status
+// to return) and the NF4 formats the layer reads (block in {32, 64, 128, 256},
+// dq_block 256 or 0, K % block == 0).
+int check_layer_shapes(int64_t M, int64_t N, int64_t K, int r);
+int check_format(int64_t K, int block, int dq_block);
+
 // Per-device status word (timeouts of bounded waits) and the non-finite
 // flag of nf4_quantize; both live in file-scope device memory.
 int* device_status_ptr();      // device address of the status word

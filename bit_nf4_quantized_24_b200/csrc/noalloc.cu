@@ -79,11 +79,9 @@ extern "C" int qlora_linear_fwd_noalloc(const uint8_t* codes, const uint8_t* abs
                                         int64_t N, int64_t K, const qlora_bf16_t* X, int64_t M,
                                         const qlora_bf16_t* A, const qlora_bf16_t* B, int r, float scale,
                                         qlora_bf16_t* Y, qlora_bf16_t* H_save, void* stream) {
-  // the same shape and pointer rules as qlora_linear_fwd
-  if (M < 0 || N <= 0 || K <= 0) return QLORA_ERR_ARG;
-  if (r < 8 || r > 64 || r % 8) return r <= 0 ? QLORA_ERR_ARG : QLORA_ERR_UNSUPPORTED;
-  if (K % 64 || N % 8) return QLORA_ERR_SHAPE;
-  if (M > (1 << 24) || N > (1 << 24) || K > (1 << 24)) return QLORA_ERR_SHAPE;
+  // the same shape and pointer rules as qlora_linear_fwd (shared checks)
+  int st = check_layer_shapes(M, N, K, r);
+  if (st) return st;
   if (!codes || !absmax_q || !dq_scale || !A || !B || (M > 0 && (!X || !Y))) return QLORA_ERR_ARG;
   if (!std::isfinite(scale)) return QLORA_ERR_ARG;
   if (M * r > kScratchElems) return QLORA_ERR_WORKSPACE;  // beyond the fixed scratch
@@ -95,9 +93,7 @@ extern "C" int qlora_linear_fwd_noalloc(const uint8_t* codes, const uint8_t* abs
 
   cudaError_t e;
   uint16_t* Hs = scratch_on_current_device(&e);
-  if (!Hs) {
-    return QLORA_ERR_CUDA;
-  }
+  if (!Hs) return cuda_status(e);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   e = launch_rowdot(X, A, M, K, r, scale, Hs, 1.0f, H_save, nullptr, s);
   if (e == cudaSuccess) {
@@ -121,5 +117,5 @@ extern "C" int qlora_linear_fwd_noalloc(const uint8_t* codes, const uint8_t* abs
       e = launch_nf4_gemm(a, s);
     }
   }
-  return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+  return cuda_status(e);
 }

@@ -103,3 +103,35 @@ def test_midpoints_avoid_the_quantizer_cell_edges(L):
     scaled = mids.astype(np.float64) * 128.0
     on_edge = (scaled == np.round(scaled)) & (np.round(scaled) % 2 == 1)
     assert not on_edge.any()
+
+
+def test_cuda_failure_is_reported_by_both_forward_entry_points(L):
+    """Without a usable CUDA device (this test runs only where there is none),
+    the first CUDA call of a forward fails on the host: the workspace entry
+    point and the no-workspace one both return QLORA_ERR_CUDA and record the
+    CUDA error for qlora_last_cuda_error() on the calling thread.  The pointers
+    are never dereferenced (nothing reaches a device)."""
+    import threading
+
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("needs a host without a usable CUDA device")
+    P = ctypes.c_void_p
+    fake, ws = P(0x10000), P(0x20000)
+    res = {}
+
+    def run(name, call):
+        res[name] = (L.qlora_last_cuda_error(), call(), L.qlora_last_cuda_error())
+
+    calls = {
+        "noalloc": lambda: L.qlora_linear_fwd_noalloc(fake, fake, fake, 256, 256, fake, 32, fake, fake, 16,
+                                                      ctypes.c_float(2.0), fake, None, None),
+        "workspace": lambda: L.qlora_linear_fwd(fake, fake, fake, 256, 256, fake, 32, fake, fake, 16,
+                                                ctypes.c_float(2.0), fake, None, ws, 1 << 20, None),
+    }
+    for name, call in calls.items():  # a fresh host thread each: its last error starts at 0
+        t = threading.Thread(target=run, args=(name, call))
+        t.start()
+        t.join()
+        before, status, after = res[name]
+        assert before == 0 and status == -5 and after != 0, (name, res[name])

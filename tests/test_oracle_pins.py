@@ -248,6 +248,27 @@ def test_adapter_parameter_counts_match_pages(oracle):
     assert d * k / count == g["lora_reduction_factor_4096_r16"]
 
 
+def test_adapter_counts_of_the_practice_question_and_bert_tiny(oracle):
+    """quantmemo, Practice 1: a 2048 x 2048 weight at r = 8.  katajob, "What an
+    adapter actually adds": BERT-tiny (hidden 128, 2 layers) with r = 8 on the
+    query and value projections and its 2-class head trainable prints 8,450.
+    The adapter shapes are the ones the oracle's layer accepts."""
+    g = golden()
+
+    def adapter(d, k, r):
+        A = np.zeros((r, k), np.uint16)
+        B = np.zeros((d, r), np.uint16)
+        oracle.linear_fwd(np.zeros((1, k), np.uint16), np.zeros((d, k), np.float32), A, B, 2.0)
+        return A.size + B.size
+
+    c = adapter(2048, 2048, 8)
+    assert c == g["lora_params_2048_r8"]
+    assert round(100 * c / (2048 * 2048), 2) == g["lora_fraction_2048_r8_pct"]
+    per_projection = adapter(128, 128, 8)
+    head = 2 * 128 + 2  # classifier weight [2, 128] and bias [2]
+    assert 2 * 2 * per_projection + head == g["bert_tiny_trainable_params"]
+
+
 def test_forward_equals_merged_weight_product(oracle):
     """Y = X (W' + s B A)^T: the merge identity, with numpy's matmul."""
     p = _small()

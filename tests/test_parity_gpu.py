@@ -3,9 +3,13 @@
 Bars: NF4 codes, absmax codes and double-quant scales bit-exact; dequantized
 bf16 weights bit-exact; Y, dX, dA, dB within a relative Frobenius error of 1e-2
 (the layer's stated tolerance; the expected error is the bf16 rounding of the
-outputs, ~3e-3).  Small cases span several tiles with ragged tails and are
-checked in full; the five workloads are checked at full size on sampled rows of
-Y and dX plus all of dA and dB, with the same launches the benchmark times.
+outputs, ~3e-3), both over the whole tensor and tile by tile: every 256-token x
+256-output tile of Y and dX and every 16 x 16 block of dA and dB must meet it on
+its own (tests/parity_tiles.py), so a fault confined to one tile cannot hide in
+the norm of the rest.  Small cases span several tiles with ragged tails and are
+checked in full; the five workloads are checked at full size on rows sampled
+from every 256-token tile (plus the last, ragged row) of Y and dX and on all of
+dA and dB, with the same launches the benchmark times.
 """
 import math
 
@@ -13,6 +17,7 @@ import numpy as np
 import pytest
 import torch
 
+import parity_tiles as pt
 from bit_nf4_quantized_24_b200 import workloads as wl
 
 pytestmark = pytest.mark.gpu
@@ -65,6 +70,7 @@ def run_fwd_check(qb, oracle, p, rows=None, q=None, Wp=None):
         Yg = Yg[rows]
     e = relfro(Yg, Yref)
     assert e <= TOL, f"Y rel err {e}"
+    pt.assert_tiles("Y", Yg, Yref, rows if rows is not None else np.arange(Yg.shape[0]), TOL)
     Href = oracle.lora_h(bits(p["X"][rows] if rows is not None else p["X"]), bits(p["A"]))
     Hg = H.float().cpu().numpy()
     eh = relfro(Hg[rows] if rows is not None else Hg, Href)
@@ -86,8 +92,12 @@ def run_bwd_check(qb, oracle, p, rows=None, q=None, Wp=None, use_saved_h=True):
     dXg = dX.float().cpu().numpy()
     if rows is not None:
         dXg = dXg[rows]
-    errs = (relfro(dXg, dXr), relfro(dA.float().cpu().numpy(), dAr), relfro(dB.float().cpu().numpy(), dBr))
+    dAg, dBg = dA.float().cpu().numpy(), dB.float().cpu().numpy()
+    errs = (relfro(dXg, dXr), relfro(dAg, dAr), relfro(dBg, dBr))
     assert max(errs) <= TOL, f"dX/dA/dB rel err {errs}"
+    pt.assert_tiles("dX", dXg, dXr, rows if rows is not None else np.arange(dXg.shape[0]), TOL)
+    pt.assert_blocks("dA", dAg, dAr, TOL)
+    pt.assert_blocks("dB", dBg, dBr, TOL)
     return errs
 
 
@@ -613,11 +623,10 @@ def test_argument_errors_on_device(qb):
 # ---------------------------------------------------- workloads, full size
 
 
-def _rows(M, n, seed):
-    g = np.random.default_rng(seed)
-    rows = np.sort(g.choice(M, size=min(n, M), replace=False))
-    rows[0], rows[-1] = 0, M - 1  # first and last (ragged) rows included
-    return np.unique(rows)
+def _rows(M, per_tile, seed):
+    """Rows of every 256-token tile (the GEMM's CTA token tile), plus the first
+    and the last (ragged) row."""
+    return pt.rows_every_tile(M, seed, tile=256, per_tile=per_tile)
 
 
 def test_workload_fwd_2048(qb, oracle):
@@ -628,7 +637,7 @@ def test_workload_fwd_2048(qb, oracle):
 def test_workload_qproj_7b(qb, oracle):
     w = wl.WORKLOADS["qproj_7b"]
     p = wl.draw_linear(w)
-    rows = _rows(p["M"], 48, 1)
+    rows = _rows(p["M"], 3, 1)
     _, q, Wp = run_fwd_check(qb, oracle, p, rows=rows)
     run_bwd_check(qb, oracle, p, rows=rows, q=q, Wp=Wp)
 
@@ -652,7 +661,7 @@ def test_workload_decode_70b_up_tiles(qb, oracle, M):
 def test_workload_mlp_7b(qb, oracle, proj):
     w = wl.WORKLOADS["mlp_7b"]
     p = wl.draw_linear(w, proj)
-    rows = _rows(p["M"], 16, 10 + proj)
+    rows = _rows(p["M"], 1, 10 + proj)
     _, q, Wp = run_fwd_check(qb, oracle, p, rows=rows)
     run_bwd_check(qb, oracle, p, rows=rows, q=q, Wp=Wp)
 
@@ -661,8 +670,22 @@ def test_workload_mlp_7b(qb, oracle, proj):
 def test_workload_layer_70b(qb, oracle, proj):
     w = wl.WORKLOADS["layer_70b"]
     p = wl.draw_linear(w, proj)
-    rows = _rows(p["M"], 8, 20 + proj)
+    rows = _rows(p["M"], 1, 20 + proj)
     _, q, Wp = run_fwd_check(qb, oracle, p, rows=rows)
+    run_bwd_check(qb, oracle, p, rows=rows, q=q, Wp=Wp)
+
+
+def test_workload_qproj_7b_adapter_only(qb, oracle):
+    """The q_proj workload at full size with W = 0: Y and dX are then the LoRA
+    terms alone, so an output tile that drops or misplaces its adapter product
+    fails the tile check outright ("QLoRA: fine-tuning a large model on one
+    GPU", LoRA, stated once: h = W0 x + (alpha/r) B A x)."""
+    w = wl.WORKLOADS["qproj_7b"]
+    p = wl.draw_linear(w)
+    p["W"] = torch.zeros_like(p["W"])
+    rows = _rows(p["M"], 1, 31)
+    _, q, Wp = run_fwd_check(qb, oracle, p, rows=rows)
+    assert not np.any(Wp)
     run_bwd_check(qb, oracle, p, rows=rows, q=q, Wp=Wp)
 
 
