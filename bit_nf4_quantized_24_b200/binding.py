@@ -68,6 +68,7 @@ def lib():
     L.nf4_decode_tiles_bytes.argtypes = [i64, i64, P]
     L.nf4_decode_tiles.argtypes = [P, i64, i64, P, P]
     L.qlora_linear_fwd_tiles.argtypes = [P, P, P, i64, i64, P, i64, P, P, i32, f32, P, P, P, sz, P]
+    L.qlora_linear_fwd_tiles_fmt.argtypes = [P, P, P, i32, i32, i64, i64, P, i64, P, P, i32, f32, P, P, P, sz, P]
     L.qlora_linear_fwd_multi_tiles.argtypes = [P, P, P, i64, i64, P, i64, P, P, i32, i32, P, P, P, P, sz, P]
     L.qlora_linear_fwd_dropout.argtypes = [P, P, P, i64, i64, P, i64, P, P, i32, f32, P, f32, P, P, P, sz, P]
     L.qlora_linear_bwd_dropout.argtypes = [P, P, P, i64, i64, P, P, i64, P, P, i32, f32, P, f32, P, P, P, P, P, sz,
@@ -75,6 +76,7 @@ def lib():
     L.qlora_linear_bwd_fmt.argtypes = [P, P, P, i32, i32, i64, i64, P, P, i64, P, P, i32, f32, P, P, P, P, P, sz,
                                        P]
     L.qlora_device_status.restype = i32
+    L.qlora_test_decode_timeout.argtypes = [P, P, P, i64, i64, P, i64, P, P, i32, f32, P, P, sz, P]
     L.qlora_trace_gemm_events.argtypes = [P, i32]
     L.qlora_trace_gemm_count.restype = i32
     L.qlora_gemm_resident_pairs.argtypes = [i32]
@@ -324,8 +326,8 @@ def nf4_decode_tiles_bytes(N: int, K: int) -> int:
 
 def nf4_decode_tiles(w: NF4Weight, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """The decode-tile copy of w's codes (uint8, nf4_decode_tiles_bytes(N, K)
-    bytes) for qlora_linear_fwd_tiles / qlora_linear_fwd_multi_tiles."""
-    w._layer_format()
+    bytes) for qlora_linear_fwd_tiles / qlora_linear_fwd_multi_tiles (the
+    arrangement of the code bytes does not depend on the format)."""
     nbytes = nf4_decode_tiles_bytes(w.N, w.K)
     if out is None:
         out = torch.empty(nbytes, dtype=torch.uint8, device=w.codes.device)
@@ -338,8 +340,8 @@ def qlora_linear_fwd_tiles(w: NF4Weight, tiles: torch.Tensor, X: torch.Tensor, A
                            scale: float, save_h: bool = True, out: torch.Tensor | None = None,
                            workspace: torch.Tensor | None = None, stream=None):
     """qlora_linear_fwd for M <= 16 tokens reading the decode tiles of w's
-    codes (w supplies absmax_q, dq_scale and the shape).  Returns (Y, H)."""
-    w._layer_format()
+    codes (w supplies absmax_q, dq_scale, the format and the shape; block 64,
+    128 or 256).  Returns (Y, H)."""
     M = X.shape[0]
     r = A.shape[0]
     _req(tiles, torch.uint8, "tiles", (nf4_decode_tiles_bytes(w.N, w.K),))
@@ -351,9 +353,10 @@ def qlora_linear_fwd_tiles(w: NF4Weight, tiles: torch.Tensor, X: torch.Tensor, A
     _req(out, torch.bfloat16, "Y", (M, w.N))
     H = torch.empty(M, r, dtype=torch.bfloat16, device=X.device) if save_h else None
     ws = _workspace(fwd_workspace_bytes(M, w.N, w.K, r), X.device, workspace)
-    _check(lib().qlora_linear_fwd_tiles(_ptr(tiles), _ptr(w.absmax_q), _ptr(w.dq_scale), w.N, w.K, _ptr(X), M,
-                                        _ptr(A), _ptr(B), r, float(scale), _ptr(out), _ptr(H), _ptr(ws), ws.numel(),
-                                        _stream(stream)), "qlora_linear_fwd_tiles")
+    _check(lib().qlora_linear_fwd_tiles_fmt(_ptr(tiles), _ptr(w.absmax_q) if w.absmax_q.numel() else None,
+                                            _ptr(w.dq_scale), w.block, w.dq_block, w.N, w.K, _ptr(X), M, _ptr(A),
+                                            _ptr(B), r, float(scale), _ptr(out), _ptr(H), _ptr(ws), ws.numel(),
+                                            _stream(stream)), "qlora_linear_fwd_tiles")
     return out, H
 
 

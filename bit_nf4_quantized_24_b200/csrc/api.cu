@@ -3,39 +3,49 @@
 #include <climits>
 #include <cstring>
 #include <mutex>
+#include <thread>
+#include <unordered_map>
 
 #include "internal.h"
 #include "qlora_nf4.h"
 
 namespace qn {
 
-// File-scope device words: the status of bounded waits, and nf4_quantize's
-// non-finite flag.  Every device that loads the library holds its own copy.
+// File-scope device words: the status of bounded waits, and a pool of
+// non-finite flags for nf4_quantize / nf4_merge_lora (one per call in flight;
+// a call takes a free slot, clears it, lets the kernel set it and reads it back
+// before it returns).  Every device that loads the library holds its own copy.
+constexpr int kFlagSlots = 64;
 __device__ int g_device_status;
-__device__ int g_nonfinite;
+__device__ int g_nonfinite[kFlagSlots];
 
 namespace {
 
 thread_local int t_last_cuda_error = 0;
-std::mutex g_quantize_mutex;
 
 constexpr int kMaxDevices = 64;
 int* g_status_ptr[kMaxDevices];
 int* g_nonfinite_ptr[kMaxDevices];
 std::mutex g_symbol_mutex;
+std::atomic<uint64_t> g_flag_busy[kMaxDevices];
 
-void** g_trace_events = nullptr;
-int g_trace_pairs = 0;
-int g_trace_count = 0;
+// Tracing of the fused-GEMM launches, per host thread (each thread records
+// the launches it makes).
+thread_local void** t_trace_events = nullptr;
+thread_local int t_trace_pairs = 0;
+thread_local int t_trace_count = 0;
 
-// Per-device side stream of the backward: dA and dB run on it while the dX
-// GEMM runs on the caller's stream (fork and join through two events).  The
-// mutex keeps each call's record/wait pairs together.
+// Side streams of the backward: dA and dB run on a side stream while the dX
+// GEMM runs on the caller's stream (fork and join through two events).  Each
+// caller stream of a device gets its own side stream and events, so the
+// backward calls of independent streams never wait for one another; the
+// mutex guards only the lookup and creation.
 struct SideStream {
   cudaStream_t st = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
 };
-SideStream g_side[kMaxDevices];
+constexpr size_t kMaxSideStreams = 64;  // per device; further caller streams run the backward on one stream
+std::unordered_map<cudaStream_t, SideStream> g_side[kMaxDevices];
 std::mutex g_side_mutex;
 
 int current_device() {
@@ -130,31 +140,79 @@ BwdWorkspace bwd_layout(void* ws, int64_t M, int64_t N, int64_t K, int r) {
   return w;
 }
 
-// The current device's side stream, created on first use (nullptr if that
-// fails, or if `s` is being captured into a CUDA graph before the side stream
-// exists: creating one inside a capture is not allowed everywhere).  Call with
-// g_side_mutex held.
-SideStream* side_stream(cudaStream_t s) {
+// The side stream of caller stream `s` on the current device, created on
+// first use.  Returns false (the backward then runs on `s` alone) if creation
+// fails, if the device already has kMaxSideStreams of them, or if `s` is being
+// captured into a CUDA graph before its side stream exists (creating a stream
+// inside a capture is not allowed everywhere).  The entry, once made, is never
+// changed or removed, so the copy returned stays valid.
+bool side_stream(cudaStream_t s, SideStream* out) {
   const int d = current_device();
-  if (d < 0 || d >= kMaxDevices) return nullptr;
-  SideStream& ss = g_side[d];
-  if (!ss.st) {
-    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-    if (cudaStreamIsCapturing(s, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) return nullptr;
-    cudaStream_t st = nullptr;
-    cudaEvent_t f = nullptr, j = nullptr;
-    if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
-    if (cudaEventCreateWithFlags(&f, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&j, cudaEventDisableTiming) != cudaSuccess) {
-      if (f) cudaEventDestroy(f);
-      cudaStreamDestroy(st);
-      return nullptr;
-    }
-    ss.st = st;
-    ss.fork = f;
-    ss.join = j;
+  if (d < 0 || d >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lock(g_side_mutex);
+  auto& map = g_side[d];
+  auto it = map.find(s);
+  if (it != map.end()) {
+    *out = it->second;
+    return true;
   }
-  return &ss;
+  if (map.size() >= kMaxSideStreams) return false;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) return false;
+  SideStream ss;
+  if (cudaStreamCreateWithFlags(&ss.st, cudaStreamNonBlocking) != cudaSuccess) return false;
+  if (cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
+    if (ss.fork) cudaEventDestroy(ss.fork);
+    cudaStreamDestroy(ss.st);
+    return false;
+  }
+  map.emplace(s, ss);
+  *out = ss;
+  return true;
+}
+
+// A free non-finite flag slot of the current device (its index), held until
+// release_flag.  More than kFlagSlots calls in flight at once on one device
+// wait here for a slot to come free.
+int acquire_flag(int dev) {
+  std::atomic<uint64_t>& busy = g_flag_busy[dev];
+  for (;;) {
+    uint64_t cur = busy.load(std::memory_order_relaxed);
+    while (~cur) {
+      const int slot = __builtin_ctzll(~cur);
+      if (busy.compare_exchange_weak(cur, cur | (uint64_t(1) << slot), std::memory_order_acquire))
+        return slot;
+    }
+    std::this_thread::yield();
+  }
+}
+void release_flag(int dev, int slot) {
+  g_flag_busy[dev].fetch_and(~(uint64_t(1) << slot), std::memory_order_release);
+}
+
+// Runs `launch(flag)` on `s` with a cleared per-call non-finite flag and
+// reports it (synchronizes `s`).
+template <typename F>
+int run_with_nonfinite_flag(cudaStream_t s, F&& launch) {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return cuda_status(cudaErrorInvalidDevice);
+  int* flags = device_nonfinite_ptr();
+  if (!flags) return cuda_status(cudaErrorInvalidSymbol);
+  const int slot = acquire_flag(dev);
+  int* flag = flags + slot;
+  cudaError_t e = cudaMemsetAsync(flag, 0, sizeof(int), s);
+  if (e == cudaSuccess) e = launch(flag);
+  int host_flag = 0;
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&host_flag, flag, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    cudaStreamSynchronize(s);  // nothing of this call may still touch the slot once it is released
+    release_flag(dev, slot);
+    return cuda_status(e);
+  }
+  release_flag(dev, slot);
+  return host_flag ? QLORA_ERR_NONFINITE : QLORA_OK;
 }
 
 }  // namespace
@@ -183,13 +241,13 @@ int* device_status_ptr() { return symbol_ptr(g_status_ptr, &g_device_status); }
 int* device_nonfinite_ptr() { return symbol_ptr(g_nonfinite_ptr, &g_nonfinite); }
 
 void trace_before(cudaStream_t st) {
-  if (g_trace_events && g_trace_count < g_trace_pairs)
-    cudaEventRecord(static_cast<cudaEvent_t>(g_trace_events[2 * g_trace_count]), st);
+  if (t_trace_events && t_trace_count < t_trace_pairs)
+    cudaEventRecord(static_cast<cudaEvent_t>(t_trace_events[2 * t_trace_count]), st);
 }
 void trace_after(cudaStream_t st) {
-  if (g_trace_events && g_trace_count < g_trace_pairs) {
-    cudaEventRecord(static_cast<cudaEvent_t>(g_trace_events[2 * g_trace_count + 1]), st);
-    ++g_trace_count;
+  if (t_trace_events && t_trace_count < t_trace_pairs) {
+    cudaEventRecord(static_cast<cudaEvent_t>(t_trace_events[2 * t_trace_count + 1]), st);
+    ++t_trace_count;
   }
 }
 
@@ -245,16 +303,9 @@ int nf4_quantize(const float* W, int64_t N, int64_t K, int block, int dq_block, 
   if (!W || !codes || (dq_block && !absmax_q) || !dq_scale) return QLORA_ERR_ARG;
   if (!aligned(W, 16) || !aligned(codes, 4)) return QLORA_ERR_SHAPE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  std::lock_guard<std::mutex> lock(g_quantize_mutex);
-  int* flag = device_nonfinite_ptr();
-  if (!flag) return cuda_status(cudaErrorInvalidSymbol);
-  cudaError_t e = cudaMemsetAsync(flag, 0, sizeof(int), s);
-  if (e == cudaSuccess) e = launch_quantize(W, N * K, block, dq_block, codes, absmax_q, dq_scale, flag, s);
-  int host_flag = 0;
-  if (e == cudaSuccess) e = cudaMemcpyAsync(&host_flag, flag, sizeof(int), cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  if (e != cudaSuccess) return cuda_status(e);
-  return host_flag ? QLORA_ERR_NONFINITE : QLORA_OK;
+  return run_with_nonfinite_flag(s, [&](int* flag) {
+    return launch_quantize(W, N * K, block, dq_block, codes, absmax_q, dq_scale, flag, s);
+  });
 }
 
 int nf4_dequantize(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale, int64_t N, int64_t K,
@@ -285,18 +336,10 @@ int nf4_merge_lora(const uint8_t* codes, const uint8_t* absmax_q, const float* d
     return QLORA_ERR_ARG;
   if (!aligned(codes, 4) || !aligned(A, 16) || !aligned(out_codes, 4)) return QLORA_ERR_SHAPE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  std::lock_guard<std::mutex> lock(g_quantize_mutex);
-  int* flag = device_nonfinite_ptr();
-  if (!flag) return cuda_status(cudaErrorInvalidSymbol);
-  cudaError_t e = cudaMemsetAsync(flag, 0, sizeof(int), s);
-  if (e == cudaSuccess)
-    e = launch_merge_quantize(codes, absmax_q, dq_scale, block, dq_block, N, K, A, B, r, scale, out_block,
-                              out_dq_block, out_codes, out_absmax_q, out_dq_scale, flag, s);
-  int host_flag = 0;
-  if (e == cudaSuccess) e = cudaMemcpyAsync(&host_flag, flag, sizeof(int), cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  if (e != cudaSuccess) return cuda_status(e);
-  return host_flag ? QLORA_ERR_NONFINITE : QLORA_OK;
+  return run_with_nonfinite_flag(s, [&](int* flag) {
+    return launch_merge_quantize(codes, absmax_q, dq_scale, block, dq_block, N, K, A, B, r, scale, out_block,
+                                 out_dq_block, out_codes, out_absmax_q, out_dq_scale, flag, s);
+  });
 }
 
 int qlora_linear_fwd_workspace(int64_t M, int64_t N, int64_t K, int r, size_t* bytes) {
@@ -334,10 +377,10 @@ int qlora_linear_fwd_fmt(const uint8_t* codes, const uint8_t* absmax_q, const fl
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < w.bytes) return QLORA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-  cudaError_t e = launch_rowdot(X, A, M, K, r, scale, w.Hs, 1.0f, H_save, nullptr, s);
+  cudaError_t e = launch_rowdot(X, A, M, K, r, scale, w.Hs, 1.0f, H_save, nullptr, s, true);
   if (e != cudaSuccess) return cuda_status(e);
-  if (M <= 16 && block == 64 && dq_block == 256) {  // the decode kernel reads the default format
-    e = launch_gemv(X, M, codes, absmax_q, dq_scale, N, K, w.Hs, B, r, Y, s);
+  if (M <= 16 && block >= 64) {  // the decode kernel (one scale per 64-weight block: not for block 32)
+    e = launch_gemv(X, M, codes, absmax_q, dq_scale, N, K, w.Hs, B, r, Y, s, nullptr, 0, false, block, dq_block);
   } else {
     GemmArgs a{};
     a.mode = 0;
@@ -398,27 +441,38 @@ int nf4_decode_tiles(const uint8_t* codes, int64_t N, int64_t K, uint8_t* tiles,
   return cuda_status(launch_pack_tiles(codes, N, K, tiles, static_cast<cudaStream_t>(stream)));
 }
 
-int qlora_linear_fwd_tiles(const uint8_t* tiles, const uint8_t* absmax_q, const float* dq_scale, int64_t N, int64_t K,
-                           const qlora_bf16_t* X, int64_t M, const qlora_bf16_t* A, const qlora_bf16_t* B, int r,
-                           float scale, qlora_bf16_t* Y, qlora_bf16_t* H_save, void* workspace, size_t workspace_bytes,
-                           void* stream) {
+int qlora_linear_fwd_tiles_fmt(const uint8_t* tiles, const uint8_t* absmax_q, const float* dq_scale, int block,
+                               int dq_block, int64_t N, int64_t K, const qlora_bf16_t* X, int64_t M,
+                               const qlora_bf16_t* A, const qlora_bf16_t* B, int r, float scale, qlora_bf16_t* Y,
+                               qlora_bf16_t* H_save, void* workspace, size_t workspace_bytes, void* stream) {
   int st = check_layer_shapes(M, N, K, r);
   if (st) return st;
+  st = check_format(K, block, dq_block);
+  if (st) return st;
   if (K % 1024) return QLORA_ERR_SHAPE;
-  if (M > 16) return QLORA_ERR_UNSUPPORTED;
-  if (!tiles || !absmax_q || !dq_scale || !A || !B || (M > 0 && (!X || !Y))) return QLORA_ERR_ARG;
+  if (M > 16 || block == 32) return QLORA_ERR_UNSUPPORTED;
+  if (!tiles || (dq_block && !absmax_q) || !dq_scale || !A || !B || (M > 0 && (!X || !Y))) return QLORA_ERR_ARG;
   if (!std::isfinite(scale)) return QLORA_ERR_ARG;
   if (M == 0) return QLORA_OK;
-  const void* ptrs[] = {tiles, absmax_q, X, A, B, Y};
+  const void* ptrs[] = {tiles, X, A, B, Y};
   for (const void* p : ptrs)
     if (!aligned(p, 16)) return QLORA_ERR_SHAPE;
   if (H_save && !aligned(H_save, 16)) return QLORA_ERR_SHAPE;
   FwdWorkspace w = fwd_layout(workspace, M, r);
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < w.bytes) return QLORA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_rowdot(X, A, M, K, r, scale, w.Hs, 1.0f, H_save, nullptr, s);
-  if (e == cudaSuccess) e = launch_gemv_tiles(X, M, tiles, absmax_q, dq_scale, N, K, w.Hs, B, r, Y, s);
+  cudaError_t e = launch_rowdot(X, A, M, K, r, scale, w.Hs, 1.0f, H_save, nullptr, s, true);
+  if (e == cudaSuccess)
+    e = launch_gemv_tiles(X, M, tiles, absmax_q, dq_scale, N, K, w.Hs, B, r, Y, s, nullptr, 0, block, dq_block);
   return cuda_status(e);
+}
+
+int qlora_linear_fwd_tiles(const uint8_t* tiles, const uint8_t* absmax_q, const float* dq_scale, int64_t N, int64_t K,
+                           const qlora_bf16_t* X, int64_t M, const qlora_bf16_t* A, const qlora_bf16_t* B, int r,
+                           float scale, qlora_bf16_t* Y, qlora_bf16_t* H_save, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  return qlora_linear_fwd_tiles_fmt(tiles, absmax_q, dq_scale, 64, 256, N, K, X, M, A, B, r, scale, Y, H_save,
+                                    workspace, workspace_bytes, stream);
 }
 
 int qlora_linear_fwd_multi_tiles(const uint8_t* tiles, const uint8_t* absmax_q, const float* dq_scale, int64_t N,
@@ -473,7 +527,7 @@ int qlora_linear_fwd_dropout(const uint8_t* codes, const uint8_t* absmax_q, cons
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < d.bytes) return QLORA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // H from the dropped-out input; the base product from X itself
-  cudaError_t e = launch_dropout_input(X, keep_mask, keep_scale, M * K, d.Xd, s, false);
+  cudaError_t e = launch_dropout_input(X, keep_mask, keep_scale, M * K, d.Xd, s, true);
   if (e == cudaSuccess) e = launch_rowdot(d.Xd, A, M, K, r, scale, w.Hs, 1.0f, H_save, nullptr, s, true);
   if (e != cudaSuccess) return cuda_status(e);
   if (M <= 16) {
@@ -526,7 +580,7 @@ int qlora_linear_bwd_dropout(const uint8_t* codes, const uint8_t* absmax_q, cons
     return cuda_status(e);
   }
   if (dX) e = cudaMemsetAsync(d.zero_tail, 0, static_cast<size_t>(M) * r * 2, s);
-  if (e == cudaSuccess) e = launch_dropout_input(X, keep_mask, keep_scale, M * K, d.Xd, s, false);
+  if (e == cudaSuccess) e = launch_dropout_input(X, keep_mask, keep_scale, M * K, d.Xd, s, true);
   if (e == cudaSuccess) e = launch_rowdot_qt(dY, B, M, N, r, scale, w.dH16, scale, nullptr, nullptr, s, true);
   const uint16_t* Huse = H;
   if (e == cudaSuccess && !H) {
@@ -622,7 +676,7 @@ int qlora_linear_bwd_fmt(const uint8_t* codes, const uint8_t* absmax_q, const fl
   // dH = scale * dY B  (B [N, r] read in place: its rows are the contraction),
   // then H if the caller did not keep it.  The second is a programmatic
   // dependent launch that waits for the first before touching shared data.
-  e = launch_rowdot_qt(dY, B, M, N, r, scale, w.dH16, scale, nullptr, nullptr, s, false);
+  e = launch_rowdot_qt(dY, B, M, N, r, scale, w.dH16, scale, nullptr, nullptr, s, true);
   const uint16_t* Huse = H;
   if (e == cudaSuccess && !H) {
     e = launch_rowdot(X, A, M, K, r, 1.0f, w.H16, 1.0f, nullptr, nullptr, s, true);
@@ -632,21 +686,18 @@ int qlora_linear_bwd_fmt(const uint8_t* codes, const uint8_t* absmax_q, const fl
   // dA = dH^T X and dB = scale * dY^T H do not feed the dX GEMM: they run on
   // the side stream while the GEMM runs on s, taking the SMs its last,
   // partial wave leaves idle; the call joins them before it returns.
-  if (dX) {
-    std::lock_guard<std::mutex> lock(g_side_mutex);
-    SideStream* ss = side_stream(s);
-    if (ss) {
-      e = cudaEventRecord(ss->fork, s);
-      if (e == cudaSuccess) e = cudaStreamWaitEvent(ss->st, ss->fork, 0);
-      if (e != cudaSuccess) return cuda_status(e);
-      e = launch_dx_gemm(codes, absmax_q, dq_scale, block, dq_block, N, K, dY, M, A, r, w.dH16, dX, s);
-      if (e == cudaSuccess) e = launch_coldot(w.dH16, X, M, K, r, 1.0f, 0, dA, ss->st, false);
-      if (e == cudaSuccess) e = launch_coldot(Huse, dY, M, N, r, scale, 1, dB, ss->st, true);
-      // join on every path, so that nothing of this call stays unordered with `s`
-      cudaError_t j = cudaEventRecord(ss->join, ss->st);
-      if (j == cudaSuccess) j = cudaStreamWaitEvent(s, ss->join, 0);
-      return cuda_status(e != cudaSuccess ? e : j);
-    }
+  SideStream ss;
+  if (dX && side_stream(s, &ss)) {
+    e = cudaEventRecord(ss.fork, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.st, ss.fork, 0);
+    if (e != cudaSuccess) return cuda_status(e);
+    e = launch_dx_gemm(codes, absmax_q, dq_scale, block, dq_block, N, K, dY, M, A, r, w.dH16, dX, s);
+    if (e == cudaSuccess) e = launch_coldot(w.dH16, X, M, K, r, 1.0f, 0, dA, ss.st, false);
+    if (e == cudaSuccess) e = launch_coldot(Huse, dY, M, N, r, scale, 1, dB, ss.st, true);
+    // join on every path, so that nothing of this call stays unordered with `s`
+    cudaError_t j = cudaEventRecord(ss.join, ss.st);
+    if (j == cudaSuccess) j = cudaStreamWaitEvent(s, ss.join, 0);
+    return cuda_status(e != cudaSuccess ? e : j);
   }
   // one stream: dA, dB, then the dX GEMM (programmatic dependent launches:
   // the GEMM's main loop starts while the adapter kernels finish; only its
@@ -666,6 +717,25 @@ int qlora_linear_bwd(const uint8_t* codes, const uint8_t* absmax_q, const float*
                               workspace, workspace_bytes, stream);
 }
 
+int qlora_test_decode_timeout(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale, int64_t N,
+                              int64_t K, const qlora_bf16_t* X, int64_t M, const qlora_bf16_t* A,
+                              const qlora_bf16_t* B, int r, float scale, qlora_bf16_t* Y, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  int st = check_layer_shapes(M, N, K, r);
+  if (st) return st;
+  if (M < 1 || M > 16) return M < 1 ? QLORA_ERR_ARG : QLORA_ERR_UNSUPPORTED;
+  if (!codes || !absmax_q || !dq_scale || !X || !A || !B || !Y || !std::isfinite(scale)) return QLORA_ERR_ARG;
+  const void* ptrs[] = {codes, X, A, B, Y};
+  for (const void* p : ptrs)
+    if (!aligned(p, 16)) return QLORA_ERR_SHAPE;
+  FwdWorkspace w = fwd_layout(workspace, M, r);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < w.bytes) return QLORA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_rowdot(X, A, M, K, r, scale, w.Hs, 1.0f, nullptr, nullptr, s);
+  if (e == cudaSuccess) e = launch_gemv(X, M, codes, absmax_q, dq_scale, N, K, w.Hs, B, r, Y, s, nullptr, 0, true);
+  return cuda_status(e);
+}
+
 int qlora_device_status(void) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_status(e);
@@ -680,13 +750,13 @@ int qlora_device_status(void) {
 
 int qlora_trace_gemm_events(void** events, int n_pairs) {
   if (n_pairs < 0 || (n_pairs > 0 && !events)) return QLORA_ERR_ARG;
-  g_trace_events = n_pairs > 0 ? events : nullptr;
-  g_trace_pairs = n_pairs;
-  g_trace_count = 0;
+  t_trace_events = n_pairs > 0 ? events : nullptr;
+  t_trace_pairs = n_pairs;
+  t_trace_count = 0;
   return QLORA_OK;
 }
 
-int qlora_trace_gemm_count(void) { return g_trace_count; }
+int qlora_trace_gemm_count(void) { return t_trace_count; }
 
 int qlora_gemm_resident_pairs(int mode) {
   if (mode != 0 && mode != 1) return QLORA_ERR_ARG;

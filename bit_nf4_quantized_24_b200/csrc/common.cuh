@@ -139,22 +139,58 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Waits for the phase of `bar` with the given parity to complete.  Gives up
 // when another thread of the CTA has already given up (*abort != 0) or after
-// kWaitLimitNs, in which case it sets *abort and the device status word.
+// limit_ns (default kWaitLimitNs), in which case it sets *abort and the device
+// status word.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort,
-                                             int* status) {
+                                             int* status, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((n & 63u) == 0) {
       if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         *abort = 1;
         atomicExch(status, kDevTimeout);
         return false;
       }
     }
   }
+}
+
+// Waits until the shared-memory counter at `addr` (a count that only grows,
+// e.g. the number of times a buffer was released) reaches `target`, with the
+// bounds of wait_bounded.  Unlike an mbarrier phase parity, a count cannot be
+// mistaken for one two uses older, so a waiter may run any number of uses
+// ahead.  Orders the caller's later memory accesses after the observation.
+__device__ __forceinline__ int ld_volatile_shared(uint32_t addr) {
+  int v;
+  asm volatile("ld.volatile.shared.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ bool wait_count_bounded(uint32_t addr, int target, volatile int* abort, int* status,
+                                                   uint64_t limit_ns = kWaitLimitNs) {
+  if (ld_volatile_shared(addr) < target) {
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t n = 1;; ++n) {
+      if (ld_volatile_shared(addr) >= target) break;
+      if ((n & 63u) == 0) {
+        if (*abort) return false;
+        if (global_timer_ns() - t0 > limit_ns) {
+          *abort = 1;
+          atomicExch(status, kDevTimeout);
+          return false;
+        }
+      }
+    }
+  }
+  __threadfence_block();
+  return true;
+}
+// Publishes a new count (after the caller's earlier memory accesses).
+__device__ __forceinline__ void set_count(uint32_t addr, int value) {
+  __threadfence_block();
+  asm volatile("st.volatile.shared.s32 [%0], %1;" ::"r"(addr), "r"(value) : "memory");
 }
 
 // The same wait with cluster-scope acquire, for barriers that also receive

@@ -97,9 +97,14 @@ cudaError_t launch_rowdot_qt(const uint16_t* P, const uint16_t* Qt, int64_t M, i
                              bool pdl = false);
 
 // ----- decode GEMV (M <= 16): Y = X deq(W)^T + Hs B^T, Hs = bf16(s X A^T)
+// withhold_one_stage: the testing aid of qlora_test_decode_timeout (a 1 ms
+// wait limit and one code stage never copied, so a bounded wait runs out).
+// block in {64, 128, 256} (a 64-weight block lies in one scale block), dq_block
+// 256 or 0 (the fp32 absmax of each block in dq_scale).
 cudaError_t launch_gemv(const uint16_t* X, int64_t M, const uint8_t* codes, const uint8_t* absmax_q,
                         const float* dq_scale, int64_t N, int64_t K, const uint16_t* Hs, const uint16_t* B, int r,
-                        uint16_t* Y, cudaStream_t st, const int32_t* aidx = nullptr, int na = 0);
+                        uint16_t* Y, cudaStream_t st, const int32_t* aidx = nullptr, int na = 0,
+                        bool withhold_one_stage = false, int block = 64, int dq_block = 256);
 // Decode tiles (see gemv.cu): bytes of the tiled copy of an N x K weight's
 // codes, the repacking kernel (K % 1024 == 0), and the decode forward that
 // reads them (M <= 16, default format).
@@ -107,7 +112,8 @@ int64_t decode_tiles_bytes(int64_t N, int64_t K);
 cudaError_t launch_pack_tiles(const uint8_t* codes, int64_t N, int64_t K, uint8_t* tiles, cudaStream_t st);
 cudaError_t launch_gemv_tiles(const uint16_t* X, int64_t M, const uint8_t* tiles, const uint8_t* absmax_q,
                               const float* dq_scale, int64_t N, int64_t K, const uint16_t* Hs, const uint16_t* B,
-                              int r, uint16_t* Y, cudaStream_t st, const int32_t* aidx = nullptr, int na = 0);
+                              int r, uint16_t* Y, cudaStream_t st, const int32_t* aidx = nullptr, int na = 0,
+                              int block = 64, int dq_block = 256);
 // LoRA dropout: Xd = mask ? bf16(fl32(X * keep)) : 0 over n elements (n % 8 == 0,
 // 16-byte aligned); dX += mask * keep * (dH A) (see adapter.cu).
 cudaError_t launch_dropout_input(const uint16_t* X, const uint8_t* mask, float keep, int64_t n, uint16_t* Xd,

@@ -95,7 +95,7 @@ extern "C" int qlora_linear_fwd_noalloc(const uint8_t* codes, const uint8_t* abs
   uint16_t* Hs = scratch_on_current_device(&e);
   if (!Hs) return cuda_status(e);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  e = launch_rowdot(X, A, M, K, r, scale, Hs, 1.0f, H_save, nullptr, s);
+  e = launch_rowdot(X, A, M, K, r, scale, Hs, 1.0f, H_save, nullptr, s, true);
   if (e == cudaSuccess) {
     if (M <= 16) {
       e = launch_gemv(X, M, codes, absmax_q, dq_scale, N, K, Hs, B, r, Y, s);

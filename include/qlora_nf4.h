@@ -103,7 +103,10 @@ int nf4_codebook(float* levels_out);
  * W: device fp32 [N, K]; codes, absmax_q, dq_scale: device outputs sized by
  * nf4_quantized_sizes.  Synchronizes `stream` to report non-finite input:
  * returns QLORA_ERR_NONFINITE if W holds a NaN or an infinity (the outputs are
- * then unspecified).  Other errors: ARG, SHAPE, UNSUPPORTED, CUDA. */
+ * then unspecified).  Calls on different streams or host threads run
+ * independently (each takes its own non-finite flag from a per-device pool of
+ * 64; a 65th concurrent call waits for a flag to come free).
+ * Other errors: ARG, SHAPE, UNSUPPORTED, CUDA. */
 int nf4_quantize(const float* W, int64_t N, int64_t K, int block, int dq_block,
                  uint8_t* codes, uint8_t* absmax_q, float* dq_scale, void* stream);
 
@@ -162,8 +165,10 @@ int qlora_linear_fwd(const uint8_t* codes, const uint8_t* absmax_q, const float*
 /* qlora_linear_fwd for an NF4 weight in any format the codec writes: block
  * in {32, 64, 128, 256}, dq_block 256 or 0 (absmax_q may then be NULL; see
  * the NF4 format above; K % block == 0).  qlora_linear_fwd is this call with
- * block 64, dq_block 256.  The bandwidth-bound decode kernel reads the default
- * format only: other formats run the tensor-core GEMM for every M. */
+ * block 64, dq_block 256.  For M <= 16 the bandwidth-bound decode kernel reads
+ * blocks of 64, 128 and 256 with double quantization on or off (each
+ * 64-weight group of a row then has one scale); block 32 runs the tensor-core
+ * GEMM for every M. */
 int qlora_linear_fwd_fmt(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale,
                          int block, int dq_block, int64_t N, int64_t K,
                          const qlora_bf16_t* X, int64_t M, const qlora_bf16_t* A,
@@ -216,6 +221,16 @@ int qlora_linear_fwd_tiles(const uint8_t* tiles, const uint8_t* absmax_q, const 
                            const qlora_bf16_t* A, const qlora_bf16_t* B, int r, float scale,
                            qlora_bf16_t* Y, qlora_bf16_t* H_save,
                            void* workspace, size_t workspace_bytes, void* stream);
+/* qlora_linear_fwd_tiles for an NF4 weight in block 64, 128 or 256 with
+ * double quantization on (dq_block 256) or off (dq_block 0; absmax_q may then
+ * be NULL); the decode tiles do not depend on the format.  block 32:
+ * QLORA_ERR_UNSUPPORTED.  qlora_linear_fwd_tiles is this call with block 64,
+ * dq_block 256. */
+int qlora_linear_fwd_tiles_fmt(const uint8_t* tiles, const uint8_t* absmax_q, const float* dq_scale,
+                               int block, int dq_block, int64_t N, int64_t K, const qlora_bf16_t* X,
+                               int64_t M, const qlora_bf16_t* A, const qlora_bf16_t* B, int r,
+                               float scale, qlora_bf16_t* Y, qlora_bf16_t* H_save, void* workspace,
+                               size_t workspace_bytes, void* stream);
 int qlora_linear_fwd_multi_tiles(const uint8_t* tiles, const uint8_t* absmax_q, const float* dq_scale,
                                  int64_t N, int64_t K, const qlora_bf16_t* X, int64_t M,
                                  const qlora_bf16_t* A_all, const qlora_bf16_t* B_all, int n_adapters,
@@ -231,12 +246,15 @@ int qlora_linear_fwd_multi_tiles(const uint8_t* tiles, const uint8_t* absmax_q, 
  *     dB = scale * dY^T H,  H = X A^T   [N, r]
  * dY: bf16 [M, N].  H: bf16 [M, r] from qlora_linear_fwd's H_save, or NULL to
  * recompute it.  dX, dA, dB: bf16 outputs (dX may be NULL to skip it).
- * With dX, dA and dB are computed on an internal per-device stream that forks
- * from `stream` after dH and joins it before the call returns (two events), so
- * they overlap the dX GEMM; every output is ready when the work enqueued on
- * `stream` is, also inside a CUDA graph captured from `stream` (the internal
- * stream is created outside any capture; a first call made during a capture
- * runs all kernels on `stream`).
+ * With dX, dA and dB are computed on an internal side stream that forks from
+ * `stream` after dH and joins it before the call returns (two events), so they
+ * overlap the dX GEMM; every output is ready when the work enqueued on
+ * `stream` is, also inside a CUDA graph captured from `stream`.  Each caller
+ * stream gets its own side stream and events (up to 64 caller streams per
+ * device; further ones run all kernels on `stream`), so backward calls on
+ * independent streams do not wait for each other.  A side stream is created
+ * outside any capture: a first call on a stream made during a capture runs all
+ * kernels on `stream`.
  * Same shape rules and errors as qlora_linear_fwd. */
 int qlora_linear_bwd(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale,
                      int64_t N, int64_t K, const qlora_bf16_t* X, const qlora_bf16_t* dY,
@@ -311,15 +329,33 @@ int qlora_linear_fwd_noalloc(const uint8_t* codes, const uint8_t* absmax_q, cons
  * device. */
 int qlora_device_status(void);
 
+/* Testing aid for the bounded device waits (the QLoRA pages have no
+ * counterpart; it exists so that the failure path can be exercised without a
+ * fault).  Runs the row-major decode forward of qlora_linear_fwd (1 <= M <= 16,
+ * the default NF4 format, the same arguments minus H_save) with every wait of
+ * the decode kernel limited to 1 ms and its copy producer told to skip the
+ * copy of its second code stage in every CTA.  The consumers' wait for that
+ * stage runs out; the kernel then lets the copies it did issue land and
+ * returns, leaving Y unspecified and QLORA_ERR_TIMEOUT in the device status
+ * word (qlora_device_status).  No memory outside Y and the workspace is
+ * written, and later calls run normally.
+ * Errors: as qlora_linear_fwd; M > 16: UNSUPPORTED. */
+int qlora_test_decode_timeout(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale,
+                              int64_t N, int64_t K, const qlora_bf16_t* X, int64_t M,
+                              const qlora_bf16_t* A, const qlora_bf16_t* B, int r, float scale,
+                              qlora_bf16_t* Y, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Kernel-level tracing for profiling.  While enabled, each launch of the
  * fused dequant-GEMM kernel (forward or dX) records events[2i] before and
  * events[2i+1] after it on the launching stream, for i = 0, 1, ... up to
  * n_pairs - 1 (later launches are not recorded).  `events` is a host array of
- * cudaEvent_t owned by the caller; n_pairs = 0 disables tracing.  Not
- * thread-safe: set it from one host thread.  Errors: ARG. */
+ * cudaEvent_t owned by the caller; n_pairs = 0 disables tracing.  Tracing is
+ * per host thread: it records the launches made by the thread that set it.
+ * Errors: ARG. */
 int qlora_trace_gemm_events(void** events, int n_pairs);
 
-/* Number of event pairs recorded since the last qlora_trace_gemm_events. */
+/* Number of event pairs recorded on this host thread since its last
+ * qlora_trace_gemm_events. */
 int qlora_trace_gemm_count(void);
 
 /* How many CTA pairs (2-SM clusters) of the fused dequant-GEMM kernel can be

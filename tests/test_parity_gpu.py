@@ -173,19 +173,32 @@ def test_codec_other_formats_bit_exact(qb, oracle, block, dq_block):
     assert np.array_equal(Wd.view(torch.int16).cpu().numpy().view(np.uint16), o16)
 
 
-@pytest.mark.parametrize("block,dq_block", [(32, 256), (128, 0), (256, 256), (64, 0)])
+@pytest.mark.parametrize("block,dq_block", [(32, 256), (128, 0), (256, 256), (64, 0), (128, 256), (256, 0)])
 def test_layer_other_formats(qb, oracle, block, dq_block):
-    """The fused GEMM reads every codec format: forward at a GEMM size and at a
-    decode size (both through the GEMM for non-default formats) and backward,
-    against the oracle's dequantized weight of the same format."""
+    """Every codec format through the layer: the fused GEMM (forward and
+    backward at a GEMM size) and, at a decode size, the row-major decode
+    kernel and the decode-tile kernel (blocks 64 to 256; block 32 keeps the
+    GEMM), against the oracle's dequantized weight of the same format."""
     M, N, K, r = 150, 264, 1024, 16
     p = wl.draw_small(600 + block + dq_block, M, N, K, r, 2.0 * r)
     q, Wp = quantize_both(qb, oracle, p["W"], block, dq_block)
     run_fwd_check(qb, oracle, p, q=q, Wp=Wp)
     run_bwd_check(qb, oracle, p, q=q, Wp=Wp)
-    p2 = dict(p)
-    p2["X"] = p["X"][:5].contiguous()
-    run_fwd_check(qb, oracle, p2, q=q, Wp=Wp)
+    for Md in (5, 12):
+        p2 = dict(p)
+        p2["X"] = p["X"][:Md].contiguous()
+        run_fwd_check(qb, oracle, p2, q=q, Wp=Wp)
+        if block >= 64:
+            T = qb.nf4_decode_tiles(q)
+            Y, _ = qb.qlora_linear_fwd_tiles(q, T, p2["X"].cuda(), p["A"].cuda(), p["B"].cuda(), p["scale"])
+            torch.cuda.synchronize()
+            Yref = oracle.linear_fwd(bits(p2["X"]), Wp, bits(p["A"]), bits(p["B"]), p["scale"])
+            assert relfro(Y.float().cpu().numpy(), Yref) <= TOL
+        else:
+            with pytest.raises(qb.QloraError) as ei:
+                qb.qlora_linear_fwd_tiles(q, qb.nf4_decode_tiles(q), p2["X"].cuda(), p["A"].cuda(), p["B"].cuda(),
+                                          p["scale"])
+            assert ei.value.status == -7
 
 
 @pytest.mark.parametrize("fmt_in,fmt_out,r", [((64, 256), (64, 256), 16), ((32, 0), (128, 256), 8),
@@ -406,7 +419,8 @@ DECODE_TILES = [
     (16, 520, 3072, 40),   # three items per tile, r not a multiple of 16
     (3, 8, 1024, 24),      # a single half tile
     (2, 4096, 5120, 16),   # more tiles than SMs
-    (12, 64, 28672, 16),   # 28 items per tile: three slots of partial sums fit shared memory
+    (12, 64, 28672, 16),   # 56 chunks per row: long chunk sequences per half
+    (5, 40008, 1024, 16),  # more than 14 tiles per CTA: two rounds of tile pairs, odd counts, ragged last tile
 ]
 
 
@@ -601,6 +615,93 @@ def test_fwd_bwd_in_cuda_graph(qb):
     for got, ref in ((Y, Y0), (H, H0), (dX, dX0), (dA, dA0), (dB, dB0)):
         assert torch.equal(got, ref)
     del g
+    assert qb.device_status() == 0
+
+
+def test_backward_on_two_unordered_streams(qb, oracle):
+    """Two backward calls on two streams with no ordering between them (each
+    caller stream has its own side stream for dA and dB): both match the
+    oracle, and a CUDA graph captured on a third stream still works."""
+    cases = []
+    for seed, (M, N, K, r) in ((501, (300, 520, 1024, 16)), (502, (260, 264, 2048, 64))):
+        p = wl.draw_small(seed, M, N, K, r, 2.0 * r, b_std=0.5)
+        q, Wp = quantize_both(qb, oracle, p["W"])
+        cases.append((p, q, Wp))
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = []
+    torch.cuda.synchronize()
+    for (p, q, _), st in zip(cases, streams):
+        with torch.cuda.stream(st):
+            X, A, B, dY = (p[k].cuda(non_blocking=True) for k in ("X", "A", "B", "dY"))
+            outs.append(qb.qlora_linear_bwd(q, X, dY, A, B, p["scale"], stream=st) + (X, A, B, dY))
+    torch.cuda.synchronize()
+    for (p, q, Wp), (dX, dA, dB, *_keep) in zip(cases, outs):
+        dXr, dAr, dBr, _ = oracle.linear_bwd(bits(p["X"]), bits(p["dY"]), Wp, bits(p["A"]), bits(p["B"]),
+                                             p["scale"])
+        errs = (relfro(dX.float().cpu().numpy(), dXr), relfro(dA.float().cpu().numpy(), dAr),
+                relfro(dB.float().cpu().numpy(), dBr))
+        assert max(errs) <= TOL, errs
+    assert qb.device_status() == 0
+
+
+def test_quantize_from_two_threads(qb, oracle):
+    """nf4_quantize from two host threads on two streams at once: each call has
+    its own non-finite flag, so the call with a NaN reports it and the other
+    returns its codes bit-exact."""
+    import threading
+    good = wl.draw_weight(wl.generator(511), 512, 4096, 0.02)
+    bad = wl.draw_weight(wl.generator(512), 512, 4096, 0.02)
+    bad[300, 17] = float("nan")
+    res = {}
+
+    def run(name, W):
+        st = torch.cuda.Stream()
+        with torch.cuda.stream(st):
+            Wd = W.cuda(non_blocking=True)
+            for _ in range(20):
+                try:
+                    res[name] = qb.nf4_quantize(Wd, stream=st)
+                except qb.QloraError as e:
+                    res[name] = e.status
+
+    ts = [threading.Thread(target=run, args=("good", good)), threading.Thread(target=run, args=("bad", bad))]
+    for t in ts:
+        t.start()
+    for t in ts:
+        t.join()
+    assert res["bad"] == -3
+    oc, oa, od, _ = oracle.nf4_quantize(good.numpy())
+    q = res["good"]
+    assert np.array_equal(q.codes.cpu().numpy(), oc) and np.array_equal(q.absmax_q.cpu().numpy(), oa)
+    assert q.dq_scale.cpu().numpy().tobytes() == od.tobytes()
+
+
+def test_bounded_wait_runs_out_and_the_next_call_is_correct(qb, oracle):
+    """The decode kernel's testing aid withholds one code stage per CTA with a
+    1 ms wait limit: the consumers' bounded wait runs out, the kernel drains
+    what it issued and returns, the device status reports QLORA_ERR_TIMEOUT
+    (and is cleared by reading it), and the next normal call on the same
+    buffers matches the oracle."""
+    import ctypes
+    M, N, K, r = 3, 4096, 4096, 16   # every CTA has at least two code stages
+    p = wl.draw_small(520, M, N, K, r, 32.0, with_dy=False)
+    q, Wp = quantize_both(qb, oracle, p["W"])
+    X, A, B = p["X"].cuda(), p["A"].cuda(), p["B"].cuda()
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(qb.fwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device="cuda")
+    assert qb.device_status() == 0
+    L = qb.lib()
+    st = L.qlora_test_decode_timeout(qb._ptr(q.codes), qb._ptr(q.absmax_q), qb._ptr(q.dq_scale), N, K, qb._ptr(X), M,
+                                     qb._ptr(A), qb._ptr(B), r, ctypes.c_float(p["scale"]), qb._ptr(Y), qb._ptr(ws),
+                                     ws.numel(), qb._stream())
+    assert st == 0
+    torch.cuda.synchronize()
+    assert qb.device_status() == -6   # QLORA_ERR_TIMEOUT
+    assert qb.device_status() == 0    # read and cleared
+    Y2, _ = qb.qlora_linear_fwd(q, X, A, B, p["scale"], out=Y, workspace=ws)
+    torch.cuda.synchronize()
+    Yref = oracle.linear_fwd(bits(p["X"]), Wp, bits(p["A"]), bits(p["B"]), p["scale"])
+    assert relfro(Y2.float().cpu().numpy(), Yref) <= TOL
     assert qb.device_status() == 0
 
 
