@@ -159,12 +159,21 @@ __device__ __forceinline__ void blocks_mma(float (&acc)[NTILE][4], const BlockIn
 // already holds that adapter's scaled H); the epilogue then adds the LoRA
 // term per output with FMAs instead of one MMA shared by all tokens.  A
 // token whose index is outside [0, na) gets no LoRA term.
+//
+// Bounded waits.  Every wait gives up after `wait_ns` (or once another warp of
+// the CTA has given up) and records kDevTimeout.  `withhold` >= 0 is a testing
+// aid: the producer then skips the copy of that code stage (no arrival, no
+// copy), so the consumers' wait for it runs out; the producer stops at its next
+// wait, lets the copies it did issue land and returns, the consumers and the
+// epilogue warp leave their loops, and the CTA exits (no cluster, no barrier
+// across the roles after the split).  Normal launches pass -1.
 template <int NTILE, bool MULTI>
 __global__ void __launch_bounds__(G_THREADS, 1)
     k_gemv(const __grid_constant__ CUtensorMap tm_codes, const uint16_t* __restrict__ X, int M,
            const uint8_t* __restrict__ absmax_q, const float* __restrict__ dq_scale, int N, int K,
            const uint16_t* __restrict__ Hs, const uint16_t* __restrict__ Bl, int r, Nf4Levels lv,
-           const int32_t* __restrict__ aidx, int na, uint16_t* __restrict__ Y, int* status) {
+           const int32_t* __restrict__ aidx, int na, uint16_t* __restrict__ Y, int* status,
+           unsigned long long wait_ns, int withhold, int lgs, int dq) {
   using S = GemvSmem<NTILE>;
   constexpr int NS = S::NS;
   pdl_trigger();
@@ -182,6 +191,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     return table + (buf * S::RED_ROWS + row) * 256 + 128 + l * 4;
   };
   const uint32_t full0 = table + S::OFF_BAR, empty0 = full0 + 8u * NS;
+  // rfull: an mbarrier per partial-sum buffer; rempty: a count of the buffer's
+  // uses the epilogue has read (a count cannot be taken for one two uses older)
   const uint32_t rfull0 = empty0 + 8u * NS, rempty0 = rfull0 + 16u;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -200,7 +211,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(rfull0 + 8u * b, G_CW);
-      mbar_init(rempty0 + 8u * b, 1);
+      asm volatile("st.shared.s32 [%0], 0;" ::"r"(rempty0 + 4u * b) : "memory");  // uses of buffer b read
     }
     abort_flag = 0;
     fence_mbar_init();
@@ -220,18 +231,21 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       int issued = 0, s = 0, tile = t0;
       for (int it = 0; it < nit; ++it) {
         const int slot = it % NS;
-        if (!wait_bounded(empty0 + 8u * slot, ((it / NS) & 1) ^ 1, &abort_flag, status)) break;
+        if (!wait_bounded(empty0 + 8u * slot, ((it / NS) & 1) ^ 1, &abort_flag, status, wait_ns)) break;
         const int b0 = s * G_SBLK;
         const int nbox = min(G_SBLK / 4, (KB - b0 + 3) / 4);  // boxes that start inside the row
-        mbar_arrive_expect_tx(full0 + 8u * slot, nbox * G_BOX);
-        for (int bx = 0; bx < nbox; ++bx)
-          tma_load_2d(ring + slot * G_STAGE + bx * G_BOX, &tm_codes, full0 + 8u * slot, (b0 + 4 * bx) * 32,
-                      tile * G_ROWS);
+        if (it != withhold) {
+          mbar_arrive_expect_tx(full0 + 8u * slot, nbox * G_BOX);
+          for (int bx = 0; bx < nbox; ++bx)
+            tma_load_2d(ring + slot * G_STAGE + bx * G_BOX, &tm_codes, full0 + 8u * slot, (b0 + 4 * bx) * 32,
+                        tile * G_ROWS);
+        }
         ++issued;
         if (++s == spt) { s = 0; ++tile; }
       }
-      for (int it = (issued > NS ? issued - NS : 0); it < issued; ++it)  // all copies land before exit
-        wait_drain(full0 + 8u * (it % NS), (it / NS) & 1);
+      // all copies land before exit (the withheld stage has none)
+      for (int it = (issued > NS ? issued - NS : 0); it < issued; ++it)
+        if (it != withhold) wait_drain(full0 + 8u * (it % NS), (it / NS) & 1);
     }
     return;
   }
@@ -263,7 +277,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           lb[k][nt][1] = ld2(Hs, 8 * nt + g, M, j0 + 2 * t + 8);
         }
       }
-      if (!wait_bounded(rfull0 + 8u * buf, (ti >> 1) & 1, &abort_flag, status)) break;
+      if (!wait_bounded(rfull0 + 8u * buf, (ti >> 1) & 1, &abort_flag, status, wait_ns)) break;
       float v[NTILE][4];
 #pragma unroll
       for (int nt = 0; nt < NTILE; ++nt)
@@ -275,7 +289,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           v[nt][c] = sum;
         }
       __syncwarp();
-      if (lane == 0) mbar_arrive(rempty0 + 8u * buf);  // partial sums read: the buffer is free
+      if (lane == 0) set_count(rempty0 + 4u * buf, (ti >> 1) + 1);  // partial sums read: the buffer is free
       if (MULTI) {  // per-token adapters: sum_j Hs[m, j] B_a[n, j] with 8-wide loads
 #pragma unroll
         for (int nt = 0; nt < NTILE; ++nt)
@@ -386,8 +400,14 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     d = 0.f;
     if (ss * G_SBLK + 2 * warp + sq < KB) {
       const int j = sidx + ss * G_SBLK;
-      q = __ldg(absmax_q + j);
-      d = __ldg(dq_scale + (j >> 8));
+      const int blk = j >> lgs;  // the format's block of this 64-weight block
+      if (dq) {
+        q = __ldg(absmax_q + blk);
+        d = __ldg(dq_scale + (blk >> 8));
+      } else {  // the exact fp32 absmax: q * d = 1 * d
+        q = 1u;
+        d = __ldg(dq_scale + blk);
+      }
     }
     if (++ss == spt) {
       ss = 0;
@@ -402,7 +422,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
   int s = 0, ti = 0, slot = 0;
   uint32_t ph = 0;
   for (int it = 0; it < nit; ++it) {
-    if (!wait_bounded(full0 + 8u * slot, ph, &abort_flag, status)) break;
+    if (!wait_bounded(full0 + 8u * slot, ph, &abort_flag, status, wait_ns)) break;
     const bool more = it + 1 < nit;
     const int nvalid = KB - s * G_SBLK - 2 * warp;  // blocks of this warp inside the row
     const uint32_t sbuf = wscale + ((it & 1) << 7);
@@ -435,7 +455,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     }
     if (++s == spt) {  // tile done: hand the partial sums to the epilogue warp
       const int buf = ti & 1;
-      if (!wait_bounded(rempty0 + 8u * buf, ((ti >> 1) & 1) ^ 1, &abort_flag, status)) break;
+      if (!wait_count_bounded(rempty0 + 4u * buf, ti >> 1, &abort_flag, status, wait_ns)) break;
 #pragma unroll
       for (int nt = 0; nt < NTILE; ++nt)
 #pragma unroll
@@ -454,7 +474,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
 template <int NTILE, bool MULTI>
 cudaError_t gemv_launch(const CUtensorMap& tm, const uint16_t* X, int64_t M, const uint8_t* absmax_q,
                         const float* dq_scale, int64_t N, int64_t K, const uint16_t* Hs, const uint16_t* B, int r,
-                        const int32_t* aidx, int na, uint16_t* Y, cudaStream_t st) {
+                        const int32_t* aidx, int na, uint16_t* Y, cudaStream_t st, unsigned long long wait_ns,
+                        int withhold, int lgs, int dq) {
   using S = GemvSmem<NTILE>;
   cudaError_t e = smem_limit_once<k_gemv<NTILE, MULTI>>(S::BYTES);
   if (e != cudaSuccess) return e;
@@ -475,25 +496,36 @@ cudaError_t gemv_launch(const CUtensorMap& tm, const uint16_t* X, int64_t M, con
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, k_gemv<NTILE, MULTI>, tm, static_cast<const uint16_t*>(X), int(M), absmax_q,
                             dq_scale, int(N), int(K), Hs, B, r, host_codebook().levels, aidx, na, Y,
-                            device_status_ptr());
+                            device_status_ptr(), wait_ns, withhold, lgs, dq);
 }
 
 }  // namespace
 
 cudaError_t launch_gemv(const uint16_t* X, int64_t M, const uint8_t* codes, const uint8_t* absmax_q,
                         const float* dq_scale, int64_t N, int64_t K, const uint16_t* Hs, const uint16_t* B, int r,
-                        uint16_t* Y, cudaStream_t st, const int32_t* aidx, int na) {
+                        uint16_t* Y, cudaStream_t st, const int32_t* aidx, int na, bool withhold_one_stage,
+                        int block, int dq_block) {
   if (M == 0 || N == 0) return cudaSuccess;
+  // the testing aid: a 1 ms wait limit and the second code stage of every CTA withheld
+  const unsigned long long wait_ns = withhold_one_stage ? 1000000ull : kWaitLimitNs;
+  const int withhold = withhold_one_stage ? 1 : -1;
+  if (block != 64 && block != 128 && block != 256) return cudaErrorInvalidValue;  // a 64-weight block has one scale
+  const int lgs = block == 64 ? 0 : block == 128 ? 1 : 2;
+  const int dq = dq_block ? 1 : 0;
   if (M > 16 || r > 64 || N * (K / 64) >= (int64_t(1) << 31)) return cudaErrorInvalidValue;  // 32-bit block index
   CUtensorMap tm;
   if (!make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, K / 2, N, K / 2, 128, G_ROWS,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   if (aidx)
-    return M <= 8 ? gemv_launch<1, true>(tm, X, M, absmax_q, dq_scale, N, K, Hs, B, r, aidx, na, Y, st)
-                  : gemv_launch<2, true>(tm, X, M, absmax_q, dq_scale, N, K, Hs, B, r, aidx, na, Y, st);
-  return M <= 8 ? gemv_launch<1, false>(tm, X, M, absmax_q, dq_scale, N, K, Hs, B, r, nullptr, 0, Y, st)
-                : gemv_launch<2, false>(tm, X, M, absmax_q, dq_scale, N, K, Hs, B, r, nullptr, 0, Y, st);
+    return M <= 8 ? gemv_launch<1, true>(tm, X, M, absmax_q, dq_scale, N, K, Hs, B, r, aidx, na, Y, st, wait_ns,
+                                         withhold, lgs, dq)
+                  : gemv_launch<2, true>(tm, X, M, absmax_q, dq_scale, N, K, Hs, B, r, aidx, na, Y, st, wait_ns,
+                                         withhold, lgs, dq);
+  return M <= 8 ? gemv_launch<1, false>(tm, X, M, absmax_q, dq_scale, N, K, Hs, B, r, nullptr, 0, Y, st, wait_ns,
+                                        withhold, lgs, dq)
+                : gemv_launch<2, false>(tm, X, M, absmax_q, dq_scale, N, K, Hs, B, r, nullptr, 0, Y, st, wait_ns,
+                                        withhold, lgs, dq);
 }
 
 namespace {
@@ -547,19 +579,17 @@ __device__ __forceinline__ void prefetch_l1(const void* p) {
 __device__ __forceinline__ uint4 ldg_v4(const void* p) {  // activations and absmax bytes: keep them in L1
   return __ldg(reinterpret_cast<const uint4*>(p));
 }
-// The same load issued only by lanes with `on` set (others get zeros); the
-// predicate is explicit so the compiler cannot turn it into a load by every
-// lane.
-__device__ __forceinline__ uint4 ldg_v4_if(const void* p, bool on) {
-  uint4 v;
+// The same load issued only by lanes with `on` set; the other lanes keep
+// their registers (zeros, set once).  The predicate is explicit so the
+// compiler cannot turn it into a load by every lane.
+__device__ __forceinline__ void ldg_v4_if(const void* p, int on, uint32_t& a, uint32_t& b, uint32_t& c,
+                                          uint32_t& d) {
   asm volatile(
       "{\n\t.reg .pred q;\n\t"
       "setp.ne.b32 q, %5, 0;\n\t"
-      "mov.b32 %0, 0;\n\tmov.b32 %1, 0;\n\tmov.b32 %2, 0;\n\tmov.b32 %3, 0;\n\t"
       "@q ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];\n\t}"
-      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-      : "l"(p), "r"(static_cast<int>(on)));
-  return v;
+      : "+r"(a), "+r"(b), "+r"(c), "+r"(d)
+      : "l"(p), "r"(on));
 }
 
 // fl32(q * d) for the absmax byte at byte position `byte` of `word`: 2^23 + q
@@ -603,12 +633,16 @@ __device__ __forceinline__ void unit_mma(float (&acc)[NTILE][4], const uint4& cw
   }
 }
 
-template <int NTILE, bool MULTI>
+// GEN: a non-default format (blocks of 2^(6 + lgs) weights, double
+// quantization on or off: dq); the scale of each unit is then loaded per unit
+// instead of 16 absmax bytes per item.
+template <int NTILE, bool MULTI, bool GEN>
 __global__ void __launch_bounds__(T_THREADS, 1)
     k_gemv_tiles(const uint8_t* __restrict__ tiles, const uint16_t* __restrict__ X, int M,
                  const uint8_t* __restrict__ absmax_q, const float* __restrict__ dq_scale, int N, int K,
                  const uint16_t* __restrict__ Hs, const uint16_t* __restrict__ Bl, int r, Nf4Levels lv,
-                 const int32_t* __restrict__ aidx, int na, int ts, int pf, uint16_t* __restrict__ Y, int* status) {
+                 const int32_t* __restrict__ aidx, int na, int ts, int pf, uint16_t* __restrict__ Y, int* status,
+                 int lgs, int dq) {
   pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   __shared__ int abort_flag;
@@ -618,8 +652,11 @@ __global__ void __launch_bounds__(T_THREADS, 1)
   const uint32_t table = (raw + 65535u) & ~65535u;
   const uint32_t part0 = table + G_TABLE;
   const uint32_t slot_bytes = tiles_slot_bytes(NCH, NTILE);
-  const uint32_t full0 = part0 + ts * slot_bytes, empty0 = full0 + 8u * ts;
-  if (empty0 + 8u * ts > raw + bytes) {  // cannot happen with the launch's size; never index past it
+  // full: an mbarrier per slot (NCH hand-overs per use); freed: how many uses
+  // of the slot the epilogue has read (a count, so a warp may run any number
+  // of tiles ahead of the epilogue without mistaking an old release for a new one)
+  const uint32_t full0 = part0 + ts * slot_bytes, freed0 = full0 + 8u * ts;
+  if (freed0 + 8u * ts > raw + bytes) {  // cannot happen with the launch's size; never index past it
     if (threadIdx.x == 0) atomicExch(status, kDevTimeout);
     return;
   }
@@ -634,7 +671,7 @@ __global__ void __launch_bounds__(T_THREADS, 1)
   if (tid == 0) {
     for (int s = 0; s < ts; ++s) {
       mbar_init(full0 + 8u * s, NCH);
-      mbar_init(empty0 + 8u * s, 1);
+      asm volatile("st.shared.s32 [%0], 0;" ::"r"(freed0 + 4u * s) : "memory");
     }
     abort_flag = 0;
     fence_mbar_init();
@@ -686,7 +723,7 @@ __global__ void __launch_bounds__(T_THREADS, 1)
 #pragma unroll
           for (int c = 0; c < 4; ++c) v[nt][c] += lds_f32(part_addr(slot, ch, nt, c, lane));
       __syncwarp();
-      if (lane == 0) mbar_arrive(empty0 + 8u * slot);  // partial sums read: the slot is free
+      if (lane == 0) set_count(freed0 + 4u * slot, use + 1);  // partial sums read: the slot is free
       if (MULTI) {
 #pragma unroll
         for (int nt = 0; nt < NTILE; ++nt)
@@ -745,7 +782,7 @@ __global__ void __launch_bounds__(T_THREADS, 1)
   // Lanes of token rows >= M load nothing and hold zeros (those columns are
   // never stored).
   const uint16_t* xrow[NTILE];
-  bool xon[NTILE];
+  int xon[NTILE];
 #pragma unroll
   for (int nt = 0; nt < NTILE; ++nt) {
     xon[nt] = 8 * nt + g < M;
@@ -755,9 +792,8 @@ __global__ void __launch_bounds__(T_THREADS, 1)
 #pragma unroll
     for (int nt = 0; nt < NTILE; ++nt) {
       const uint16_t* p = xrow[nt] + kb * 64;
-      const uint4 lo = ldg_v4_if(p, xon[nt]), hi = ldg_v4_if(p + 8, xon[nt]);
-      in.x[nt][0] = lo.x; in.x[nt][1] = lo.y; in.x[nt][2] = lo.z; in.x[nt][3] = lo.w;
-      in.x[nt][4] = hi.x; in.x[nt][5] = hi.y; in.x[nt][6] = hi.z; in.x[nt][7] = hi.w;
+      ldg_v4_if(p, xon[nt], in.x[nt][0], in.x[nt][1], in.x[nt][2], in.x[nt][3]);
+      ldg_v4_if(p + 8, xon[nt], in.x[nt][4], in.x[nt][5], in.x[nt][6], in.x[nt][7]);
     }
   };
   // the two rows' absmax bytes of item j start at this lane's index (dq group: index >> 8)
@@ -794,9 +830,10 @@ __global__ void __launch_bounds__(T_THREADS, 1)
     // item's lines go to L1 now, so its loads do not wait on L2
     const int kb0 = ch * T_ITEM;
     const int64_t ia = absmax_index(j, 0), ib = absmax_index(j, 1);
-    const uint4 qa = ldg_v4(absmax_q + ia), qb = ldg_v4(absmax_q + ib);
-    const float da = __ldg(dq_scale + (ia >> 8)), db = __ldg(dq_scale + (ib >> 8));
-    if (j + T_CW < nitems) {
+    const uint4 qa = GEN ? make_uint4(0u, 0u, 0u, 0u) : ldg_v4(absmax_q + ia);
+    const uint4 qb = GEN ? make_uint4(0u, 0u, 0u, 0u) : ldg_v4(absmax_q + ib);
+    const float da = GEN ? 0.f : __ldg(dq_scale + (ia >> 8)), db = GEN ? 0.f : __ldg(dq_scale + (ib >> 8));
+    if (!GEN && j + T_CW < nitems) {
       const int64_t pa = absmax_index(j + T_CW, 0), pb = absmax_index(j + T_CW, 1);
       prefetch_l1(absmax_q + pa);
       prefetch_l1(absmax_q + pb);
@@ -806,6 +843,12 @@ __global__ void __launch_bounds__(T_THREADS, 1)
     const float ca = -8388608.0f * da, cb = -8388608.0f * db;
     const uint32_t qaw[4] = {qa.x, qa.y, qa.z, qa.w}, qbw[4] = {qb.x, qb.y, qb.z, qb.w};
     UnitX<NTILE> xin[2];
+#pragma unroll
+    for (int b = 0; b < 2; ++b)
+#pragma unroll
+      for (int nt = 0; nt < NTILE; ++nt)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) xin[b].x[nt][i] = 0u;  // lanes of absent tokens keep zeros
     load_x(xin[0], kb0);
 #pragma unroll
     for (int grp = 0; grp < NG; ++grp) {
@@ -823,14 +866,23 @@ __global__ void __launch_bounds__(T_THREADS, 1)
       for (int u = 0; u < T_GU; ++u) {
         const int uu = T_GU * grp + u;
         if (uu + 1 < T_ITEM) load_x(xin[(uu + 1) & 1], kb0 + uu + 1);
-        const float sa = block_scale(qaw[uu >> 2], uu & 3, da, ca);
-        const float sb = block_scale(qbw[uu >> 2], uu & 3, db, cb);
+        float sa, sb;
+        if (!GEN) {
+          sa = block_scale(qaw[uu >> 2], uu & 3, da, ca);
+          sb = block_scale(qbw[uu >> 2], uu & 3, db, cb);
+        } else {  // the format's blocks of this unit's 64-weight blocks (2^lgs of them per scale)
+          const int64_t ga = (ia + uu) >> lgs, gb = (ib + uu) >> lgs;
+          sa = dq ? __fmul_rn(static_cast<float>(__ldg(absmax_q + ga)), __ldg(dq_scale + (ga >> 8)))
+                  : __ldg(dq_scale + ga);
+          sb = dq ? __fmul_rn(static_cast<float>(__ldg(absmax_q + gb)), __ldg(dq_scale + (gb >> 8)))
+                  : __ldg(dq_scale + gb);
+        }
         unit_mma<NTILE>(acc, cw[grp & 1][u], xin[uu & 1], lane_base, sa, sb);
       }
     }
     // hand the item's partial sums to the epilogue warp
     const int slot = ti % ts, use = ti / ts;
-    if (!wait_bounded(empty0 + 8u * slot, (use & 1) ^ 1, &abort_flag, status)) break;
+    if (!wait_count_bounded(freed0 + 4u * slot, use, &abort_flag, status)) break;
 #pragma unroll
     for (int nt = 0; nt < NTILE; ++nt)
 #pragma unroll
@@ -862,15 +914,15 @@ __global__ void k_pack_tiles(const uint8_t* __restrict__ codes, int N, int K, ui
   reinterpret_cast<uint4*>(tiles)[idx] = make_uint4(a.x, a.y, b.x, b.y);
 }
 
-template <int NTILE, bool MULTI>
-cudaError_t gemv_tiles_launch(const uint8_t* tiles, const uint16_t* X, int64_t M, const uint8_t* absmax_q,
-                              const float* dq_scale, int64_t N, int64_t K, const uint16_t* Hs, const uint16_t* B,
-                              int r, const int32_t* aidx, int na, uint16_t* Y, cudaStream_t st) {
+template <int NTILE, bool MULTI, bool GEN>
+cudaError_t gemv_tiles_launch_t(const uint8_t* tiles, const uint16_t* X, int64_t M, const uint8_t* absmax_q,
+                                const float* dq_scale, int64_t N, int64_t K, const uint16_t* Hs, const uint16_t* B,
+                                int r, const int32_t* aidx, int na, uint16_t* Y, cudaStream_t st, int lgs, int dq) {
   const int nch = static_cast<int>(K / 64 / T_ITEM);
   const int avail = T_SMEM_LIMIT - tiles_smem_bytes(nch, NTILE, 0);
   const int ts = std::min(T_SLOTS_MAX, avail / (tiles_slot_bytes(nch, NTILE) + 16));
   if (ts < 1) return cudaErrorInvalidValue;  // K too large for one slot of partial sums
-  cudaError_t e = smem_limit_once<k_gemv_tiles<NTILE, MULTI>>(T_SMEM_LIMIT);
+  cudaError_t e = smem_limit_once<k_gemv_tiles<NTILE, MULTI, GEN>>(T_SMEM_LIMIT);
   if (e != cudaSuccess) return e;
   // The kernel that computes Hs runs on T_HS_SMS SMs while this one starts
   // (programmatic dependent launch), and a CTA of this kernel cannot share an
@@ -882,9 +934,20 @@ cudaError_t gemv_tiles_launch(const uint8_t* tiles, const uint16_t* X, int64_t M
   const int64_t ntiles = (N + G_ROWS - 1) / G_ROWS;
   const int64_t per_cta = (ntiles + sms - 1) / sms;
   const unsigned grid = static_cast<unsigned>((ntiles + per_cta - 1) / per_cta);
-  return launch_ex(k_gemv_tiles<NTILE, MULTI>, dim3(grid), dim3(T_THREADS), tiles_smem_bytes(nch, NTILE, ts), st,
-                   true, tiles, X, int(M), absmax_q, dq_scale, int(N), int(K), Hs, B, r, host_codebook().levels,
-                   aidx, na, ts, 1, Y, device_status_ptr());
+  return launch_ex(k_gemv_tiles<NTILE, MULTI, GEN>, dim3(grid), dim3(T_THREADS), tiles_smem_bytes(nch, NTILE, ts),
+                   st, true, tiles, X, int(M), absmax_q, dq_scale, int(N), int(K), Hs, B, r, host_codebook().levels,
+                   aidx, na, ts, 1, Y, device_status_ptr(), lgs, dq);
+}
+
+template <int NTILE, bool MULTI>
+cudaError_t gemv_tiles_launch(const uint8_t* tiles, const uint16_t* X, int64_t M, const uint8_t* absmax_q,
+                              const float* dq_scale, int64_t N, int64_t K, const uint16_t* Hs, const uint16_t* B,
+                              int r, const int32_t* aidx, int na, uint16_t* Y, cudaStream_t st, int lgs, int dq) {
+  if (lgs == 0 && dq)
+    return gemv_tiles_launch_t<NTILE, MULTI, false>(tiles, X, M, absmax_q, dq_scale, N, K, Hs, B, r, aidx, na, Y, st,
+                                                    lgs, dq);
+  return gemv_tiles_launch_t<NTILE, MULTI, true>(tiles, X, M, absmax_q, dq_scale, N, K, Hs, B, r, aidx, na, Y, st, lgs,
+                                                 dq);
 }
 
 }  // namespace
@@ -902,14 +965,20 @@ cudaError_t launch_pack_tiles(const uint8_t* codes, int64_t N, int64_t K, uint8_
 
 cudaError_t launch_gemv_tiles(const uint16_t* X, int64_t M, const uint8_t* tiles, const uint8_t* absmax_q,
                               const float* dq_scale, int64_t N, int64_t K, const uint16_t* Hs, const uint16_t* B,
-                              int r, uint16_t* Y, cudaStream_t st, const int32_t* aidx, int na) {
+                              int r, uint16_t* Y, cudaStream_t st, const int32_t* aidx, int na, int block,
+                              int dq_block) {
   if (M == 0 || N == 0) return cudaSuccess;
   if (M > 16 || r > 64 || K % 1024 || N * (K / 64) >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+  if (block != 64 && block != 128 && block != 256) return cudaErrorInvalidValue;  // a 64-weight block has one scale
+  const int lgs = block == 64 ? 0 : block == 128 ? 1 : 2;
+  const int dq = dq_block ? 1 : 0;
   if (aidx)
-    return M <= 8 ? gemv_tiles_launch<1, true>(tiles, X, M, absmax_q, dq_scale, N, K, Hs, B, r, aidx, na, Y, st)
-                  : gemv_tiles_launch<2, true>(tiles, X, M, absmax_q, dq_scale, N, K, Hs, B, r, aidx, na, Y, st);
-  return M <= 8 ? gemv_tiles_launch<1, false>(tiles, X, M, absmax_q, dq_scale, N, K, Hs, B, r, nullptr, 0, Y, st)
-                : gemv_tiles_launch<2, false>(tiles, X, M, absmax_q, dq_scale, N, K, Hs, B, r, nullptr, 0, Y, st);
+    return M <= 8
+               ? gemv_tiles_launch<1, true>(tiles, X, M, absmax_q, dq_scale, N, K, Hs, B, r, aidx, na, Y, st, lgs, dq)
+               : gemv_tiles_launch<2, true>(tiles, X, M, absmax_q, dq_scale, N, K, Hs, B, r, aidx, na, Y, st, lgs, dq);
+  return M <= 8
+             ? gemv_tiles_launch<1, false>(tiles, X, M, absmax_q, dq_scale, N, K, Hs, B, r, nullptr, 0, Y, st, lgs, dq)
+             : gemv_tiles_launch<2, false>(tiles, X, M, absmax_q, dq_scale, N, K, Hs, B, r, nullptr, 0, Y, st, lgs, dq);
 }
 
 }  // namespace qn
