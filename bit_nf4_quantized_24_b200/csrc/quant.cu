@@ -9,6 +9,9 @@
 // code): t = fl32(w / a_b); code = number of midpoints strictly below t; an
 // all-zero block encodes the zero level; s2 = fl32(max a / 255);
 // q = min(255, rint(fl32(a / s2))).
+#include <atomic>
+#include <mutex>
+
 #include "internal.h"
 
 namespace qn {
@@ -31,10 +34,65 @@ struct Cell {
 };
 constexpr int kCells = 256;
 
+// The cell table is a function of the codebook alone: built once on the host
+// (cell j covers [(j - 64.5) / 64, (j - 63.5) / 64), the same fp32 expressions
+// the code below relies on) and copied to each device at its first use.
+__device__ Cell g_cells[kCells];
+
+void build_cells(const Nf4Mids& mids, Cell* out) {
+  for (int j = 0; j < kCells; ++j) {
+    const float lo = (static_cast<float>(j) - 64.5f) * 0.015625f, hi = lo + 0.015625f;
+    int base = 0;
+    float mid = __builtin_huge_valf();
+    for (int i = 0; i < 15; ++i) {
+      base += mids.v[i] < lo ? 1 : 0;
+      if (mids.v[i] > lo && mids.v[i] < hi) mid = mids.v[i];
+    }
+    out[j] = Cell{base, mid};
+  }
+}
+
+// Device address of the cell table on the current device, uploaded the first
+// time it is asked for there (nullptr and the error on failure).
+const Cell* device_cells(cudaError_t* err) {
+  static std::atomic<uint64_t> done{0};
+  static std::mutex mu;
+  static Cell host[kCells];
+  static std::once_flag built;
+  std::call_once(built, [] { build_cells(host_codebook().mids, host); });
+  int dev = 0;
+  *err = cudaGetDevice(&dev);
+  if (*err != cudaSuccess) return nullptr;
+  void* p = nullptr;
+  *err = cudaGetSymbolAddress(&p, g_cells);
+  if (*err != cudaSuccess) return nullptr;
+  const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+  if (!bit || !(done.load(std::memory_order_acquire) & bit)) {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!bit || !(done.load(std::memory_order_acquire) & bit)) {
+      *err = cudaMemcpy(p, host, sizeof(host), cudaMemcpyHostToDevice);
+      if (*err != cudaSuccess) return nullptr;
+      if (bit) done.fetch_or(bit, std::memory_order_release);
+    }
+  }
+  return static_cast<const Cell*>(p);
+}
+
+// The index of t's cell is the low 8 bits of fl32(64 t + 1.5 * 2^23 + 64)
+// (the bias has zeros there), masked so that any t reads inside the table.
 __device__ __forceinline__ int nf4_code(float t, const Cell* cells) {
   const float f = __fmaf_rn(t, 64.0f, 12582976.0f);
-  const Cell c = cells[(__float_as_int(f) - 0x4B400000) & (kCells - 1)];
+  const Cell c = cells[__float_as_int(f) & (kCells - 1)];
   return c.base + (t > c.mid ? 1 : 0);
+}
+
+// max with NaN propagation (IEEE maximum): a NaN operand gives NaN, so the
+// block maximum of |w| is NaN or infinite exactly when the block holds a
+// non-finite weight.
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
 }
 
 // fl32(w / a), correctly rounded, from the block's reciprocal r = fl32(1 / a):
@@ -72,43 +130,61 @@ struct MergeSrc {
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t h) { return __uint_as_float(h << 16); }
 
-// merged values of elements e .. e+3 (one row, one input block); lv: the 16
-// levels in shared memory
-__device__ __forceinline__ float4 merged4(const MergeSrc& m, const float* lv, int64_t e) {
-  const int64_t n = e / m.K, k = e - n * m.K;
-  const uint32_t c = *reinterpret_cast<const uint16_t*>(m.codes + e / 2);
-  const int64_t b = e >> m.lg;
-  const float a = m.dq ? __fmul_rn(static_cast<float>(m.absmax_q[b]), m.dq_scale[b >> 8]) : m.dq_scale[b];
-  float w[4], acc[4] = {0.f, 0.f, 0.f, 0.f};
+// Merged values of the F groups of 4 elements e0 + f * STRIDE + 0..3
+// (f < F; all in one row, one output block; each group inside one input
+// block); lv: the 16 levels in shared memory.  B[n, j] is loaded once per j
+// for all F groups; A[j, k..k+3] with one 8-byte load per group and j.
+template <int F, int STRIDE>
+__device__ __forceinline__ void mergedF(const MergeSrc& m, const float* lv, int64_t e0, float4 (&x)[F]) {
+  const int64_t n = e0 / m.K, k0 = e0 - n * m.K;
+  float acc[F][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) w[i] = __bfloat162float(__float2bfloat16_rn(__fmul_rn(lv[(c >> (4 * i)) & 15u], a)));
-  const uint16_t* arow = m.A + k;
+  for (int f = 0; f < F; ++f) acc[f][0] = acc[f][1] = acc[f][2] = acc[f][3] = 0.f;
+  const uint16_t* arow = m.A + k0;
   const uint16_t* brow = m.B + n * m.r;
   for (int j = 0; j < m.r; ++j) {
-    const float bj = bf16_bits_to_f32(brow[j]);
-    const uint2 a4 = *reinterpret_cast<const uint2*>(arow + static_cast<int64_t>(j) * m.K);
-    acc[0] = __fmaf_rn(bj, bf16_bits_to_f32(a4.x & 0xffffu), acc[0]);
-    acc[1] = __fmaf_rn(bj, bf16_bits_to_f32(a4.x >> 16), acc[1]);
-    acc[2] = __fmaf_rn(bj, bf16_bits_to_f32(a4.y & 0xffffu), acc[2]);
-    acc[3] = __fmaf_rn(bj, bf16_bits_to_f32(a4.y >> 16), acc[3]);
+    const float bj = bf16_bits_to_f32(__ldg(brow + j));
+    const uint16_t* aj = arow + static_cast<int64_t>(j) * m.K;
+#pragma unroll
+    for (int f = 0; f < F; ++f) {
+      const uint2 a4 = __ldg(reinterpret_cast<const uint2*>(aj + f * STRIDE));
+      acc[f][0] = __fmaf_rn(bj, __uint_as_float(a4.x << 16), acc[f][0]);
+      acc[f][1] = __fmaf_rn(bj, __uint_as_float(a4.x & 0xffff0000u), acc[f][1]);
+      acc[f][2] = __fmaf_rn(bj, __uint_as_float(a4.y << 16), acc[f][2]);
+      acc[f][3] = __fmaf_rn(bj, __uint_as_float(a4.y & 0xffff0000u), acc[f][3]);
+    }
   }
-  return make_float4(__fadd_rn(w[0], __fmul_rn(m.s, acc[0])), __fadd_rn(w[1], __fmul_rn(m.s, acc[1])),
-                     __fadd_rn(w[2], __fmul_rn(m.s, acc[2])), __fadd_rn(w[3], __fmul_rn(m.s, acc[3])));
+#pragma unroll
+  for (int f = 0; f < F; ++f) {
+    const int64_t e = e0 + f * STRIDE;
+    const int64_t b = e >> m.lg;  // the input block of this group
+    const float a = m.dq ? __fmul_rn(static_cast<float>(m.absmax_q[b]), m.dq_scale[b >> 8]) : m.dq_scale[b];
+    const uint32_t c = *reinterpret_cast<const uint16_t*>(m.codes + e / 2);
+    float w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = __bfloat162float(__float2bfloat16_rn(__fmul_rn(lv[(c >> (4 * i)) & 15u], a)));
+    x[f] = make_float4(__fadd_rn(w[0], __fmul_rn(m.s, acc[f][0])), __fadd_rn(w[1], __fmul_rn(m.s, acc[f][1])),
+                       __fadd_rn(w[2], __fmul_rn(m.s, acc[f][2])), __fadd_rn(w[3], __fmul_rn(m.s, acc[f][3])));
+  }
 }
 
 // One CTA per group of 256 blocks (the double-quant group).  A block of B
-// weights is spread over LP = min(32, B / 4) lanes, F = B / (4 LP) float4s per
-// lane; a warp covers 32 / LP blocks per step, and four steps' loads are
-// issued before any is used, to keep HBM busy.  DQ: double quantization of the
-// group's absmax values (else each block's fp32 absmax is stored as is).
+// weights is spread over LP = B / 16 lanes with F = 4 float4s (16 weights) per
+// lane, so the block maximum needs log2(LP) shuffles and one reciprocal per 16
+// weights; a warp step covers 32 / LP blocks and each warp issues the loads of
+// U steps before it uses any, to keep HBM busy.  A block whose maximum is not
+// finite (NaN or infinity inside) is reported and not coded.  DQ: double
+// quantization of the group's absmax values (else each block's fp32 absmax is
+// stored as is).
 template <int B, bool DQ, bool MERGE>
 __global__ void __launch_bounds__(256) k_quantize(const float* __restrict__ W, MergeSrc msrc, Nf4Levels levels,
-                                                  int64_t nblocks, Nf4Mids mids, uint8_t* __restrict__ codes,
-                                                  uint8_t* __restrict__ absmax_q, float* __restrict__ dq_scale,
-                                                  int* nonfinite) {
-  constexpr int LP = B / 4 < 32 ? B / 4 : 32;
-  constexpr int F = B / (4 * LP);
-  constexpr int BPW = 32 / LP;  // blocks per warp step
+                                                  int64_t nblocks, const Cell* __restrict__ cells,
+                                                  uint8_t* __restrict__ codes, uint8_t* __restrict__ absmax_q,
+                                                  float* __restrict__ dq_scale, int* nonfinite) {
+  constexpr int F = 4;
+  constexpr int LP = B / (4 * F);  // 2, 4, 8, 16
+  constexpr int BPW = 32 / LP;     // blocks per warp step
+  constexpr int U = 4;             // warp steps whose loads are in flight together
   __shared__ Cell s_cell[kCells];
   __shared__ float s_amax[kGroup];
   __shared__ float s_red[8];
@@ -116,62 +192,60 @@ __global__ void __launch_bounds__(256) k_quantize(const float* __restrict__ W, M
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int sub = lane / LP, sl = lane % LP;
   if (MERGE && tid < 16) s_lv[tid] = levels.v[tid];
+  s_cell[tid] = cells[tid];  // kCells == blockDim.x
   const int64_t g = blockIdx.x;
   const int64_t b0 = g * kGroup;
   const int64_t rem = nblocks - b0;
   const int nb = rem < kGroup ? static_cast<int>(rem) : kGroup;
-  {  // cell table (kCells == blockDim.x)
-    const float lo = (static_cast<float>(tid) - 64.5f) * 0.015625f, hi = lo + 0.015625f;
-    int base = 0;
-    float mid = __int_as_float(0x7f800000);
-    for (int i = 0; i < 15; ++i) {
-      base += mids.v[i] < lo ? 1 : 0;
-      if (mids.v[i] > lo && mids.v[i] < hi) mid = mids.v[i];
-    }
-    s_cell[tid] = Cell{base, mid};
-  }
   __syncthreads();
 
   const int nsteps = (nb + BPW - 1) / BPW;
-  float nan_probe = 0.0f;  // becomes NaN if any weight is NaN or infinite (x * 0)
-  for (int p0 = warp; p0 < nsteps; p0 += 32) {
-    float4 x[4][F];
-    bool ok[4];
+  bool bad = false;
+  for (int p0 = warp; p0 < nsteps; p0 += 8 * U) {  // steps p0, p0 + 8, ..., p0 + 8 (U - 1)
+    float4 x[U][F];
+    bool ok[U];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < U; ++u) {
       const int i = BPW * (p0 + 8 * u) + sub;
       ok[u] = (p0 + 8 * u < nsteps) && (i < nb);
+      if (MERGE) {
+        if (ok[u]) {
+          mergedF<F, 4 * LP>(msrc, s_lv, (b0 + i) * B + sl * 4, x[u]);
+        } else {
 #pragma unroll
-      for (int f = 0; f < F; ++f) {
-        if (MERGE)
-          x[u][f] = ok[u] ? merged4(msrc, s_lv, (b0 + i) * B + (f * LP + sl) * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
-        else
+          for (int f = 0; f < F; ++f) x[u][f] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      } else {
+#pragma unroll
+        for (int f = 0; f < F; ++f)
           x[u][f] = ok[u] ? __ldcs(reinterpret_cast<const float4*>(W + (b0 + i) * B) + f * LP + sl)
                           : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < U; ++u) {
       if (p0 + 8 * u >= nsteps) break;  // warp-uniform
       const int i = BPW * (p0 + 8 * u) + sub;
       float m = 0.0f;
 #pragma unroll
       for (int f = 0; f < F; ++f) {
         const float4 v = x[u][f];
-        nan_probe = __fmaf_rn(v.x, 0.0f, __fmaf_rn(v.y, 0.0f, __fmaf_rn(v.z, 0.0f, __fmaf_rn(v.w, 0.0f, nan_probe))));
-        m = fmaxf(m, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+        m = fmax_nan(m, fmax_nan(fmax_nan(fabsf(v.x), fabsf(v.y)), fmax_nan(fabsf(v.z), fabsf(v.w))));
       }
 #pragma unroll
-      for (int off = LP / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      for (int off = LP / 2; off > 0; off >>= 1) m = fmax_nan(m, __shfl_xor_sync(0xffffffffu, m, off));
       if (ok[u]) {
+        const bool finite = m <= 3.402823466e38f;  // false for NaN and infinity
+        bad |= !finite;
         const bool fast = m >= 0x1p-100f && m <= 0x1p100f;
         const float r = fast ? __frcp_rn(m) : 0.0f;
+        uint16_t* dst = reinterpret_cast<uint16_t*>(codes + (b0 + i) * (B / 2)) + sl;
 #pragma unroll
         for (int f = 0; f < F; ++f) {
           const float4 v = x[u][f];
           uint32_t c;
-          if (m == 0.0f) {
-            c = 0x7777u;  // an all-zero block encodes the zero level
+          if (m == 0.0f || !finite) {
+            c = 0x7777u;  // an all-zero block encodes the zero level (a non-finite one is reported)
           } else if (fast) {
             c = nf4_code(div_by_absmax(v.x, m, r), s_cell) | (nf4_code(div_by_absmax(v.y, m, r), s_cell) << 4) |
                 (nf4_code(div_by_absmax(v.z, m, r), s_cell) << 8) |
@@ -180,7 +254,7 @@ __global__ void __launch_bounds__(256) k_quantize(const float* __restrict__ W, M
             c = nf4_code(__fdiv_rn(v.x, m), s_cell) | (nf4_code(__fdiv_rn(v.y, m), s_cell) << 4) |
                 (nf4_code(__fdiv_rn(v.z, m), s_cell) << 8) | (nf4_code(__fdiv_rn(v.w, m), s_cell) << 12);
           }
-          reinterpret_cast<uint16_t*>(codes + (b0 + i) * (B / 2))[f * LP + sl] = static_cast<uint16_t>(c);
+          dst[f * LP] = static_cast<uint16_t>(c);
         }
         if (sl == 0) {
           if (DQ)
@@ -191,7 +265,6 @@ __global__ void __launch_bounds__(256) k_quantize(const float* __restrict__ W, M
       }
     }
   }
-  const bool bad = !(nan_probe == 0.0f);
   if (!DQ) {
     if (__syncthreads_or(bad) && tid == 0) atomicExch(nonfinite, 1);
     return;
@@ -278,12 +351,15 @@ cudaError_t quantize_launch(const float* W, const MergeSrc* merge, int64_t numel
   const int64_t ngroups = (nblocks + kGroup - 1) / kGroup;
   if (ngroups == 0) return cudaSuccess;
   const HostCodebook& cb = host_codebook();
+  cudaError_t e;
+  const Cell* cells = device_cells(&e);
+  if (!cells) return e;
   if (merge)
     k_quantize<B, DQ, true><<<static_cast<unsigned>(ngroups), 256, 0, st>>>(
-        nullptr, *merge, cb.levels, nblocks, cb.mids, codes, absmax_q, dq_scale, nonfinite);
+        nullptr, *merge, cb.levels, nblocks, cells, codes, absmax_q, dq_scale, nonfinite);
   else
     k_quantize<B, DQ, false><<<static_cast<unsigned>(ngroups), 256, 0, st>>>(
-        W, MergeSrc{}, cb.levels, nblocks, cb.mids, codes, absmax_q, dq_scale, nonfinite);
+        W, MergeSrc{}, cb.levels, nblocks, cells, codes, absmax_q, dq_scale, nonfinite);
   return cudaGetLastError();
 }
 
