@@ -257,14 +257,19 @@ __global__ void __launch_bounds__(256) k_rows_multi(const uint16_t* __restrict__
 
 // ------------------------------------------------------------------ rows
 //
-// out[m, j] = sum_k P[m, k] Q(j, k) for 16 * CW tokens per CTA over the whole
-// contraction.  P is bf16 [M, Kc]; Q is either [R, Kc] (QT = false: A) or
-// [Kc, R] (QT = true: lora_B, read in place for dH = dY B).  CW = NT / 2
-// consumer warps (16 tokens each) run ldmatrix + m16n8k16, the last warp's
-// lane 0 produces: per stage a (16 CW) x 64 tile of P (128-byte swizzle) and
-// the 64-wide slice of Q (as many bytes as the P tile, so Q costs no more L2
-// traffic than P), RW_ST stages in flight.
-constexpr int RW_ST = 8;
+// out[m, j] = sum_k P[m, k] Q(j, k) for 16 * CW tokens per CTA.  P is bf16
+// [M, Kc]; Q is either [R, Kc] (QT = false: A) or [Kc, R] (QT = true: lora_B,
+// read in place for dH = dY B).  CW = NT / 2 consumer warps (16 tokens each)
+// run ldmatrix + m16n8k16, the last warp's lane 0 produces: per stage a
+// (16 CW) x 64 tile of P (128-byte swizzle) and the 64-wide slice of Q (as
+// many bytes as the P tile, so Q costs no more L2 traffic than P), RW_ST
+// stages in flight.  When the token tiles alone do not fill the GPU, the
+// contraction is split too: a cluster of `nsplit` CTAs (consecutive along
+// grid x) shares a token tile, each CTA takes a contiguous range of the
+// 64-wide stages, leaves its fp32 sums in shared memory, and after a cluster
+// barrier each CTA adds one share of the outputs over the cluster's partials
+// in rank order (distributed shared memory): deterministic, no scratch.
+constexpr int RW_ST = 5;
 
 template <int NT>
 struct RowsSmem {
@@ -272,27 +277,64 @@ struct RowsSmem {
   static constexpr int P_BYTES = 16 * CW * 64 * 2;
   static constexpr int Q_BYTES = NT * 8 * 64 * 2;
   static constexpr int OFF_Q = RW_ST * P_BYTES;
-  static constexpr int OFF_BAR = OFF_Q + RW_ST * Q_BYTES;
+  static constexpr int OFF_PART = OFF_Q + RW_ST * Q_BYTES;  // fp32 [16 CW m][NT * 8 j]
+  static constexpr int OFF_BAR = OFF_PART + 16 * CW * NT * 8 * 4;
   static constexpr int BYTES = OFF_BAR + 2 * RW_ST * 8 + 1024;
 };
+
+// The cluster's reduction of k_rows with a split contraction: every thread of
+// every CTA arrives (the producer warp too); then CTA `split` writes outputs
+// [V split / nsplit, V (split + 1) / nsplit) of the tile's V = 16 CW x R, each
+// the sum of the ranks' partials in rank order.
+template <int NT, int CW>
+__device__ __forceinline__ void rows_reduce(uint32_t part, int M, int R, int m0, int split, int nsplit, float sa,
+                                            uint16_t* out16a, float sb, uint16_t* out16b, float* out32) {
+  constexpr int RJ = NT * 8;
+  cluster_sync_all();  // every CTA's partial sums are in its shared memory
+  const int V = 16 * CW * R;
+  const int v0 = static_cast<int>(static_cast<int64_t>(V) * split / nsplit);
+  const int v1 = static_cast<int>(static_cast<int64_t>(V) * (split + 1) / nsplit);
+  for (int v = v0 + static_cast<int>(threadIdx.x); v < v1; v += blockDim.x) {
+    const int ml = v / R, j = v - ml * R;
+    const int m = m0 + ml;
+    const uint32_t off = part + (ml * RJ + j) * 4;
+    float sum = 0.f;
+    for (int rk = 0; rk < nsplit; ++rk) {
+      float x;
+      asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(x) : "r"(mapa_shared(off, rk)) : "memory");
+      sum += x;
+    }
+    if (m >= M) continue;
+    const int64_t o = static_cast<int64_t>(m) * R + j;
+    out16a[o] = static_cast<uint16_t>(bf16x2_bits(sa * sum, 0.f));
+    if (out16b) out16b[o] = static_cast<uint16_t>(bf16x2_bits(sb * sum, 0.f));
+    if (out32) out32[o] = sb * sum;
+  }
+  cluster_sync_all();  // peers keep their shared memory until every read is done
+}
 
 template <int NT, bool QT>
 __global__ void __launch_bounds__(32 * (NT / 2 + 1)) k_rows(const __grid_constant__ CUtensorMap tmP,
                                                             const __grid_constant__ CUtensorMap tmQ, int M, int Kc,
                                                             int R, float sa, uint16_t* __restrict__ out16a, float sb,
                                                             uint16_t* __restrict__ out16b, float* __restrict__ out32,
-                                                            int* status) {
+                                                            int nsplit, int* status) {
   using S = RowsSmem<NT>;
   constexpr int CW = S::CW;
+  constexpr int RJ = NT * 8;  // j extent of the partial buffer
   pdl_trigger();
   pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t full0 = base + S::OFF_BAR, empty0 = full0 + 8u * RW_ST;
+  const uint32_t part = base + S::OFF_PART;
   __shared__ int abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * 16 * CW;
-  const int nk = (Kc + 63) / 64;
+  const int split = nsplit > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int m0 = (blockIdx.x / nsplit) * 16 * CW;
+  const int nk_all = (Kc + 63) / 64;
+  const int it0 = static_cast<int>(static_cast<int64_t>(nk_all) * split / nsplit);
+  const int nk = static_cast<int>(static_cast<int64_t>(nk_all) * (split + 1) / nsplit) - it0;
   if (threadIdx.x == 0) {
     for (int s = 0; s < RW_ST; ++s) {
       mbar_init(full0 + 8u * s, 1);
@@ -310,16 +352,19 @@ __global__ void __launch_bounds__(32 * (NT / 2 + 1)) k_rows(const __grid_constan
         const int s = it % RW_ST;
         if (!wait_bounded(empty0 + 8u * s, ((it / RW_ST) & 1) ^ 1, &abort_flag, status)) break;
         mbar_arrive_expect_tx(full0 + 8u * s, S::P_BYTES + S::Q_BYTES);
-        tma_load_2d(base + s * S::P_BYTES, &tmP, full0 + 8u * s, it * 64, m0);
+        const int kx = (it0 + it) * 64;
+        tma_load_2d(base + s * S::P_BYTES, &tmP, full0 + 8u * s, kx, m0);
         if (QT)
-          tma_load_2d(base + S::OFF_Q + s * S::Q_BYTES, &tmQ, full0 + 8u * s, 0, it * 64);
+          tma_load_2d(base + S::OFF_Q + s * S::Q_BYTES, &tmQ, full0 + 8u * s, 0, kx);
         else
-          tma_load_2d(base + S::OFF_Q + s * S::Q_BYTES, &tmQ, full0 + 8u * s, it * 64, 0);
+          tma_load_2d(base + S::OFF_Q + s * S::Q_BYTES, &tmQ, full0 + 8u * s, kx, 0);
         ++issued;
       }
       for (int it = (issued > RW_ST ? issued - RW_ST : 0); it < issued; ++it)  // all copies land before exit
         wait_drain(full0 + 8u * (it % RW_ST), (it / RW_ST) & 1);
     }
+    __syncwarp();  // lane 0 rejoins the warp before the cluster barriers
+    if (nsplit > 1) rows_reduce<NT, CW>(part, M, R, m0, split, nsplit, sa, out16a, sb, out16b, out32);
     return;
   }
 
@@ -362,6 +407,20 @@ __global__ void __launch_bounds__(32 * (NT / 2 + 1)) k_rows(const __grid_constan
   }
 
   const int g = lane >> 2, t = lane & 3;
+  if (nsplit > 1) {  // this CTA's partial sums part[m_local][j], then the cluster's reduction
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int ml = 16 * warp + g + 8 * h, j = nt * 8 + 2 * t;
+        asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(part + (ml * RJ + j) * 4), "f"(acc[nt][2 * h]),
+                     "f"(acc[nt][2 * h + 1])
+                     : "memory");
+      }
+    __syncwarp();
+    rows_reduce<NT, CW>(part, M, R, m0, split, nsplit, sa, out16a, sb, out16b, out32);
+    return;
+  }
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
@@ -549,9 +608,35 @@ cudaError_t rows_launch(const uint16_t* P, const uint16_t* Q, int64_t M, int64_t
   if (!ok) return cudaErrorInvalidValue;
   cudaError_t e = smem_limit_once<k_rows<NT, QT>>(S::BYTES);
   if (e != cudaSuccess) return e;
-  const unsigned grid = static_cast<unsigned>((M + 16 * S::CW - 1) / (16 * S::CW));
-  return launch_ex(k_rows<NT, QT>, dim3(grid), dim3(32 * (S::CW + 1)), S::BYTES, st, pdl, tmP, tmQ, int(M), int(Kc),
-                   R, sa, out16a, sb, out16b, out32, device_status_ptr());
+  const int64_t tiles = (M + 16 * S::CW - 1) / (16 * S::CW);
+  // split the contraction when the token tiles give fewer than two CTAs per
+  // SM (two fit by shared memory), keeping at least 4 stages per split
+  const int64_t nk = (Kc + 63) / 64;
+  const int64_t want = (2 * device_sm_count()) / std::max<int64_t>(1, tiles);
+  const int nsplit = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({8, want, nk / 4})));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles * nsplit), 1, 1);
+  cfg.blockDim = dim3(32 * (S::CW + 1), 1, 1);
+  cfg.dynamicSmemBytes = S::BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (nsplit > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = static_cast<unsigned>(nsplit);
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, k_rows<NT, QT>, tmP, tmQ, int(M), int(Kc), R, sa, out16a, sb, out16b, out32,
+                            nsplit, device_status_ptr());
 }
 
 template <bool QT>
