@@ -1,26 +1,30 @@
 #!/usr/bin/env python
 """Benchmark of the QLoRA NF4 linear layer on B200.
 
-One step = forward + backward of the Llama-7B-shaped q_proj workload
-(X [4096 tokens, 4096] bf16, W 4096x4096 in NF4 with double quantization,
-LoRA r = 16, alpha = 32): qlora_linear_fwd then qlora_linear_bwd through the
-C ABI, all inputs resident in HBM.  The metric is algorithmic TFLOP/s
-(4MNK + 6Mr(K+N) per step; no gradient for W).  L2 is flushed between timed
-steps (a 256 MB write, then a 256 MB read so that no dirty lines are left to
-be written back inside the timed region); each step is timed with CUDA events on the launching
-stream and the per-step times are summed.
+One step = forward + backward of every projection of a 70B-shaped decoder
+layer (q, o 8192x8192; k, v 1024x8192; gate, up 28672x8192; down 28672 ->
+8192), 4096 tokens, LoRA r = 64, alpha = 16 on all seven, the weights NF4 with
+8-bit double quantization (block 64, groups of 256 blocks): the forwards in
+layer order, then the backwards in reverse order (each reading the H its
+forward saved), through the C ABI, all inputs resident in HBM.  The seven
+weights are quantized once, before any step, with nf4_quantize (timed on its
+own).  The metric is algorithmic TFLOP/s (4MNK + 6Mr(K+N) per projection; no
+gradient for W).  L2 is flushed between timed steps (a 256 MB write, then a
+256 MB read, so that no dirty lines are left to be written back inside the
+timed region); each step is timed with CUDA events on the launching stream and
+the per-step times are summed.
 
 Also reported: the fused dequant-GEMM kernel against the tensor-core roofline
-(events around each launch), the decode GEMV weight stream (70B-shaped up
-projection, 1/4/16 tokens) and nf4_quantize against HBM bandwidth, an
-fwd + bwd of the 7B MLP and 70B decoder-layer projections and the 2048 x 2048
-forward at 128 tokens (with a dense torch bf16 matmul of each forward shape as a
-library ceiling), an
-end-to-end number with host buffers (pinned host -> device copies of X and dY,
-device -> host copies of Y, dX, dA, dB of every step inside the timed region,
-pipelined across steps on copy streams), SM clocks
-sampled through NVML during the timed region, and the CPU oracle timed on the
-host cores on a bounded sample.
+(events around each of its 14 launches per step), the decode GEMV weight stream
+(70B-shaped up projection, 1/4/16 tokens) and the NF4 codec against HBM
+bandwidth, fwd + bwd of the 7B q_proj and MLP projections and the 2048 x 2048
+forward at 128 tokens (with a dense torch bf16 matmul of each forward shape as
+a library ceiling), an end-to-end number with host buffers (pinned host ->
+device copies of every projection's X and dY, device -> host copies of its Y,
+dX, dA, dB, every step, inside the timed region, pipelined across steps on copy
+streams), SM clocks sampled through NVML during the timed region, and the CPU
+oracle timed on the host cores on a bounded sample (the same layer on fewer
+tokens).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -32,6 +36,7 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import hashlib
 import json
 import os
 import statistics
@@ -43,7 +48,25 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "QLoRA linear fwd+bwd TFLOP/s and NF4 weight-stream GB/s on 1 B200; % roofline"
-WORKLOAD = "qproj_7b"
+WORKLOAD = "layer_70b"
+
+# DRAM bytes (read + write) per fused-GEMM launch, mean over the 14 launches of
+# one step of the workload above, from one ncu capture of `bench.py --profile
+# layer` (metrics dram__bytes_read.sum, dram__bytes_write.sum; the summary and
+# command are in profiles/).  Valid only for the kernel source it was taken on
+# (sha256 prefix of gemm_tc.cu); reported as null otherwise.
+GEMM_TRAFFIC = {"gemm_tc_sha16": None, "bytes_per_launch": None}
+
+
+def gemm_traffic():
+    path = os.path.join(ROOT, "bit_nf4_quantized_24_b200", "csrc", "gemm_tc.cu")
+    try:
+        sha = hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    if GEMM_TRAFFIC["gemm_tc_sha16"] != sha:
+        return None
+    return GEMM_TRAFFIC["bytes_per_launch"]
 
 
 class L2Flush:
@@ -64,25 +87,6 @@ class L2Flush:
         torch.sum(self.r, 0, out=self.out)
 
 
-def gemm_traffic():
-    """DRAM bytes (read + write) per fused-GEMM launch, from the committed ncu
-    summary of this workload -- but only while the kernel source is the one the
-    counters were taken on (its sha256 prefix is recorded in the summary)."""
-    import hashlib
-    import re
-    here = os.path.dirname(os.path.abspath(__file__))
-    try:
-        text = open(os.path.join(here, "profiles", "k_nf4_gemm_qproj_7b.md")).read()
-        src = open(os.path.join(here, "bit_nf4_quantized_24_b200", "csrc", "gemm_tc.cu"), "rb").read()
-    except OSError:
-        return None
-    sha = re.search(r"gemm_tc\.cu`, sha256 prefix ([0-9a-f]{16})", text)
-    val = re.search(r"traffic_bytes_per_launch: (\d+)", text)
-    if not sha or not val or hashlib.sha256(src).hexdigest()[:16] != sha.group(1):
-        return None
-    return int(val.group(1))
-
-
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -96,6 +100,11 @@ def peaks():
 
 def step_flops(M, N, K, r):
     return 4 * M * N * K + 6 * M * r * (K + N)
+
+
+def layer_flops(w, M=None):
+    M = w.M if M is None else M
+    return sum(step_flops(M, pr.N, pr.K, w.r) for pr in w.projections)
 
 
 # ------------------------------------------------------------------ clocks
@@ -165,50 +174,125 @@ class ClockSampler:
 # -------------------------------------------------------------- CPU oracle
 
 
-def oracle_prepare():
-    """Inputs of the workload for the CPU oracle: drawn on the host, quantized
-    and dequantized by the oracle (done once, outside any timed region)."""
+def draw_layer_host(w):
+    """The workload's seeded inputs, one dict per projection, on the host."""
+    from bit_nf4_quantized_24_b200 import workloads as wl
+    return [wl.draw_linear(w, i) for i in range(len(w.projections))]
+
+
+def oracle_layer_prepare(w, host=None):
+    """Per projection: the oracle's own NF4 quantization and dequantization of
+    the fp32 weight, and the bf16 bits of X, A, B, dY (done once, untimed)."""
     import oracle
     from bit_nf4_quantized_24_b200 import workloads as wl
-    w = wl.WORKLOADS[WORKLOAD]
-    p = wl.draw_linear(w)
-    N, K = p["N"], p["K"]
-    oc, oa, od, _ = oracle.nf4_quantize(p["W"].numpy())
-    _, Wp = oracle.nf4_dequantize(oc, oa, od, N, K)
+    host = draw_layer_host(w) if host is None else host
     bits = wl.bf16_bits
-    return {"M": p["M"], "N": N, "K": K, "r": p["r"], "scale": p["scale"], "Wp": Wp,
-            "X": bits(p["X"]), "A": bits(p["A"]), "B": bits(p["B"]), "dY": bits(p["dY"])}
+    prep = []
+    for p in host:
+        N, K = p["N"], p["K"]
+        oc, oa, od, _ = oracle.nf4_quantize(p["W"].numpy())
+        _, Wp = oracle.nf4_dequantize(oc, oa, od, N, K)
+        prep.append({"N": N, "K": K, "Wp": Wp, "X": bits(p["X"]), "A": bits(p["A"]), "B": bits(p["B"]),
+                     "dY": bits(p["dY"]), "scale": p["scale"], "name": p["name"]})
+    return prep
 
 
-def oracle_run(prep, rows_sample: int | None = None):
-    """Times the CPU oracle on a bounded sample of the workload: Y and dX for
-    `rows_sample` token rows, H, dH, dA, dB in full.  Returns (TFLOP/s, cores,
+def oracle_layer_run(w, prep, tokens: int):
+    """Times the CPU oracle on a bounded sample of the workload: the same
+    layer (all projections, forward and backward: Y, dX, dA, dB, with H and dH)
+    on `tokens` of its token rows, evenly spaced.  Returns (TFLOP/s, cores,
     sample description, seconds)."""
     import numpy as np
 
     import oracle
-    M, N, K, r = prep["M"], prep["N"], prep["K"], prep["r"]
-    X, A, B, dY, Wp = prep["X"], prep["A"], prep["B"], prep["dY"], prep["Wp"]
-    rows = np.arange(M, dtype=np.int64) if rows_sample is None else np.linspace(0, M - 1, rows_sample).astype(np.int64)
-    t0 = time.perf_counter()
-    oracle.linear_fwd(X, Wp, A, B, prep["scale"], rows=rows)
-    oracle.linear_bwd(X, dY, Wp, A, B, prep["scale"], rows=rows)
-    dt = time.perf_counter() - t0
-    S = len(rows)
-    flops = S * (2 * K * r + 2 * N * K + 2 * N * r)          # forward rows
-    flops += 2 * M * K * r + 2 * M * N * r                    # H, dH
-    flops += S * (2 * N * K + 2 * r * K)                      # dX rows
-    flops += 2 * r * K * M + 2 * N * r * M                    # dA, dB
-    desc = (f"{WORKLOAD} (M={M}, N={N}, K={K}, r={r}): Y and dX for {S} of {M} token rows, "
-            f"H, dH, dA, dB in full; one fwd+bwd pass of the fp64 oracle")
+    M = w.M
+    rows = np.linspace(0, M - 1, tokens).astype(np.int64)
+    dt = 0.0
+    for pp in prep:
+        X, dY = np.ascontiguousarray(pp["X"][rows]), np.ascontiguousarray(pp["dY"][rows])
+        t0 = time.perf_counter()
+        oracle.linear_fwd(X, pp["Wp"], pp["A"], pp["B"], pp["scale"])
+        oracle.linear_bwd(X, dY, pp["Wp"], pp["A"], pp["B"], pp["scale"])
+        dt += time.perf_counter() - t0
+    flops = layer_flops(w, tokens)
+    desc = (f"{w.name}: all {len(prep)} projections, forward and backward (Y, dX, dA, dB) of the fp64 oracle "
+            f"on {tokens} of the {M} tokens (evenly spaced rows), r={w.r}; the weights quantized and "
+            f"dequantized by the oracle beforehand, untimed")
     return flops / dt / 1e12, oracle.num_threads(), desc, dt
 
 
-def oracle_sample(rows_sample: int | None = None):
-    return oracle_run(oracle_prepare(), rows_sample)
-
-
 # -------------------------------------------------------------- our arm
+
+
+class Layer:
+    """Device state of the workload: per projection the NF4 weight, the LoRA
+    adapter and one buffer set (X, dY, Y, H, dX, dA, dB and workspaces); a step
+    runs the forwards in layer order, then the backwards in reverse order,
+    through the C ABI on the current stream."""
+
+    def __init__(self, qb, w, host, dev):
+        import torch
+        self.qb, self.w, self.dev = qb, w, dev
+        self.M, self.r, self.s = w.M, w.r, w.scale
+        self.projs = []
+        for p in host:
+            N, K = p["N"], p["K"]
+            q = qb.nf4_quantize(p["W"].to(dev))
+            self.projs.append({"N": N, "K": K, "q": q, "A": p["A"].to(dev), "B": p["B"].to(dev)})
+        torch.cuda.synchronize()
+
+    def new_set(self, host=None):
+        import torch
+        qb, M, r, dev = self.qb, self.M, self.r, self.dev
+        out = []
+        for i, pr in enumerate(self.projs):
+            N, K = pr["N"], pr["K"]
+            b = {"Y": torch.empty(M, N, dtype=torch.bfloat16, device=dev),
+                 "H": torch.empty(M, r, dtype=torch.bfloat16, device=dev),
+                 "dX": torch.empty(M, K, dtype=torch.bfloat16, device=dev),
+                 "dA": torch.empty(r, K, dtype=torch.bfloat16, device=dev),
+                 "dB": torch.empty(N, r, dtype=torch.bfloat16, device=dev),
+                 "wsf": torch.empty(qb.fwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev),
+                 "wsb": torch.empty(qb.bwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)}
+            if host is not None:
+                b["X"] = host[i]["X"].to(dev)
+                b["dY"] = host[i]["dY"].to(dev)
+            else:
+                b["X"] = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+                b["dY"] = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            out.append(b)
+        return out
+
+    def step(self, bufs, allreduce=None):
+        import ctypes
+        qb = self.qb
+        L, P, f32 = qb.lib(), qb._ptr, ctypes.c_float
+        M, r, s = self.M, self.r, self.s
+        st = qb._stream()
+        for pr, b in zip(self.projs, bufs):
+            q, N, K = pr["q"], pr["N"], pr["K"]
+            e = L.qlora_linear_fwd(P(q.codes), P(q.absmax_q), P(q.dq_scale), N, K, P(b["X"]), M, P(pr["A"]),
+                                   P(pr["B"]), r, f32(s), P(b["Y"]), P(b["H"]), P(b["wsf"]), b["wsf"].numel(), st)
+            if e:
+                raise qb.QloraError(e, "fwd")
+        for pr, b in reversed(list(zip(self.projs, bufs))):
+            q, N, K = pr["q"], pr["N"], pr["K"]
+            e = L.qlora_linear_bwd(P(q.codes), P(q.absmax_q), P(q.dq_scale), N, K, P(b["X"]), P(b["dY"]), M,
+                                   P(pr["A"]), P(pr["B"]), r, f32(s), P(b["H"]), P(b["dX"]), P(b["dA"]),
+                                   P(b["dB"]), P(b["wsb"]), b["wsb"].numel(), st)
+            if e:
+                raise qb.QloraError(e, "bwd")
+            if allreduce is not None:
+                allreduce(b["dA"], b["dB"])
+
+    def gemm_launch_flops(self):
+        """Algorithmic FLOP of each fused-GEMM launch of a step, in launch
+        order: the 7 forwards (2MNK + 2MNr), then the 7 dX GEMMs in reverse
+        projection order (2MNK + 2MKr)."""
+        M, r = self.M, self.r
+        fwd = [2 * M * p["N"] * p["K"] + 2 * M * p["N"] * r for p in self.projs]
+        dx = [2 * M * p["N"] * p["K"] + 2 * M * p["K"] * r for p in reversed(self.projs)]
+        return fwd + dx
 
 
 def run_ours(args, rank, world, local_rank):
@@ -230,52 +314,48 @@ def run_ours(args, rank, world, local_rank):
 
     pk = peaks()
     w = wl.WORKLOADS[WORKLOAD]
-    p = wl.draw_linear(w)
-    M, N, K, r, s = p["M"], p["N"], p["K"], p["r"], p["scale"]
     dev = torch.device("cuda", local_rank)
-    q = qb.nf4_quantize(p["W"].to(dev))
-    X, A, B, dY = (p[k].to(dev) for k in ("X", "A", "B", "dY"))
-    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-    dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
-    dA = torch.empty(r, K, dtype=torch.bfloat16, device=dev)
-    dB = torch.empty(N, r, dtype=torch.bfloat16, device=dev)
-    H = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
-    wsf = torch.empty(qb.fwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
-    wsb = torch.empty(qb.bwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev)
+    host = draw_layer_host(w)
     flush = L2Flush(dev)
-    L = qb.lib()
-    import ctypes
-    f32 = ctypes.c_float
-    P = qb._ptr
 
-    main = {"X": X, "dY": dY, "Y": Y, "dX": dX, "dA": dA, "dB": dB, "H": H, "wsf": wsf, "wsb": wsb}
+    # the one-time quantization of the seven weights (4 B read, 0.516 B written per weight)
+    Wd = [p["W"].to(dev) for p in host]
+    for W in Wd:
+        qb.nf4_quantize(W)
+    torch.cuda.synchronize()
+    flush()
+    q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    q0.record()
+    for W in Wd:
+        qb.nf4_quantize(W)
+    q1.record()
+    torch.cuda.synchronize()
+    quant_ms = q0.elapsed_time(q1)
+    numel = sum(W.numel() for W in Wd)
+    quant_bytes = sum(4 * W.numel() + W.numel() // 2 + W.numel() // 64 + 4 * ((W.numel() // 64 + 255) // 256)
+                      for W in Wd)
+    del Wd
+    torch.cuda.empty_cache()
 
-    def step(b=main):
-        st = qb._stream()
-        e = L.qlora_linear_fwd(P(q.codes), P(q.absmax_q), P(q.dq_scale), N, K, P(b["X"]), M, P(A), P(B), r, f32(s),
-                               P(b["Y"]), P(b["H"]), P(b["wsf"]), b["wsf"].numel(), st)
-        if e:
-            raise qb.QloraError(e, "fwd")
-        e = L.qlora_linear_bwd(P(q.codes), P(q.absmax_q), P(q.dq_scale), N, K, P(b["X"]), P(b["dY"]), M, P(A), P(B),
-                               r, f32(s), P(b["H"]), P(b["dX"]), P(b["dA"]), P(b["dB"]), P(b["wsb"]),
-                               b["wsb"].numel(), st)
-        if e:
-            raise qb.QloraError(e, "bwd")
-        if world > 1:
-            dp.allreduce_adapter_grads(b["dA"], b["dB"])
-
-    # our kernels per step (the ncu launch list shows the same): forward k_rows (H) and
-    # k_nf4_gemm; backward k_rows (dH), two k_cols (dA, dB) and k_nf4_gemm (dX)
-    launches_per_step = 2 + 4
+    layer = Layer(qb, w, host, dev)
+    main = layer.new_set(host)
+    allreduce = dp.allreduce_adapter_grads if world > 1 else None
+    M, r = w.M, w.r
+    flops = layer_flops(w)
+    n_proj = len(w.projections)
+    # our kernels per step (the ncu launch list shows the same): per projection,
+    # forward k_rows (H) and k_nf4_gemm; backward k_rows (dH), two k_cols (dA,
+    # dB) and k_nf4_gemm (dX)
+    launches_per_step = n_proj * (2 + 4)
 
     for _ in range(args.warmup):
-        step()
+        layer.step(main, allreduce)
     torch.cuda.synchronize()
 
     K_steps = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K_steps)]
     sampler = ClockSampler(local_rank)
-    trace = qb.GemmTrace(2 * K_steps)
+    trace = qb.GemmTrace(2 * n_proj * K_steps)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -283,7 +363,7 @@ def run_ours(args, rank, world, local_rank):
         for i in range(K_steps):
             flush()
             ev[i][0].record()
-            step()
+            layer.step(main, allreduce)
             ev[i][1].record()
         torch.cuda.synchronize()
     if world > 1:
@@ -295,39 +375,60 @@ def run_ours(args, rank, world, local_rank):
         t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
-    flops = step_flops(M, N, K, r)
     value = flops * world * K_steps / (total_ms / 1e3) / 1e12
 
-    # dominant kernel: the fused dequant-GEMM, launched twice per step (forward,
-    # dX).  The forward launch has the GPU to itself; the dX launch shares it
-    # with the dA / dB kernels, which the backward runs on a side stream in the
-    # SMs the GEMM's last wave leaves idle, so its event time is not the
-    # kernel's own: the roofline uses the forward launches, dx_ms is reported.
-    fwd_ms = gemm_ms[0::2]
-    bwd_ms = gemm_ms[1::2]
-    gemm_flops_fwd = 2 * M * N * K + 2 * M * N * r
-    fwd_mean = statistics.mean(fwd_ms) if fwd_ms else float("nan")
-    achieved = gemm_flops_fwd / (fwd_mean / 1e3) / 1e12
-    roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": round(achieved / pk["bf16_tflops"], 4), "traffic": gemm_traffic(),
-                "kernel": "k_nf4_gemm (fused NF4 dequant + tcgen05 GEMM), forward launches; the dX launch "
-                          "overlaps the adapter-gradient kernels (dx_ms)",
-                "peak_source": f"{pk['source']} bf16 burst (MEASURED_PEAKS.json)",
-                "fwd_ms": round(fwd_mean, 4) if fwd_ms else None,
-                "dx_ms": round(statistics.mean(bwd_ms), 4) if bwd_ms else None}
+    # dominant kernel: the fused dequant-GEMM, 14 launches per step (7 forwards,
+    # 7 dX).  achieved = algorithmic FLOP of all traced launches / their summed
+    # event durations (= mean FLOP per launch / mean launch duration).  The dX
+    # launches share the GPU with the adapter-gradient kernels of the side
+    # stream, so their event times include that sharing.
+    per_launch = layer.gemm_launch_flops()
+    nl = len(per_launch)
+    cnt = min(len(gemm_ms), nl * K_steps)
+    lf = [per_launch[i % nl] for i in range(cnt)]
+    gt = gemm_ms[:cnt]
+    fwd_idx = [i for i in range(cnt) if i % nl < n_proj]
+    dx_idx = [i for i in range(cnt) if i % nl >= n_proj]
 
-    # End to end through the C ABI with host buffers: every step copies its
-    # inputs X, dY from pinned host memory and reads its results Y, dX, dA, dB
-    # back, as a training loop does; the copies are pipelined across steps
-    # (two device buffer sets; the input copy of step i + 1 and the read-back
-    # of step i - 1 run on their own streams while step i computes).
-    Xh = p["X"].pin_memory()
-    dYh = p["dY"].pin_memory()
-    Yh = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
-    dXh = torch.empty(M, K, dtype=torch.bfloat16).pin_memory()
-    dAh = torch.empty(r, K, dtype=torch.bfloat16).pin_memory()
-    dBh = torch.empty(N, r, dtype=torch.bfloat16).pin_memory()
-    second = {k: torch.empty_like(v) for k, v in main.items()}
+    def rate(idx):
+        t = sum(gt[i] for i in idx)
+        return sum(lf[i] for i in idx) / (t / 1e3) / 1e12 if t > 0 else float("nan")
+
+    achieved = rate(range(cnt))
+    names = [p.name for p in w.projections]
+    per_proj = {}
+    for j, nm in enumerate(names):
+        fi = [i for i in fwd_idx if i % nl == j]
+        di = [i for i in dx_idx if i % nl == nl - 1 - j]
+        per_proj[nm] = {"fwd_ms": round(statistics.mean(gt[i] for i in fi), 4) if fi else None,
+                        "fwd_tflops": round(rate(fi), 1) if fi else None,
+                        "dx_ms": round(statistics.mean(gt[i] for i in di), 4) if di else None,
+                        "dx_tflops": round(rate(di), 1) if di else None}
+    roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": round(achieved / pk["bf16_tflops"], 4),
+                "frac_of_sustained": round(achieved / pk["bf16_tflops_sustained"], 4),
+                "traffic": gemm_traffic(),
+                "kernel": "k_nf4_gemm (fused NF4 dequant + tcgen05 GEMM): all 14 launches of a step, 7 forward and "
+                          "7 dX (the dX launches overlap the adapter-gradient kernels on the side stream)",
+                "peak_source": f"{pk['source']} bf16 burst (MEASURED_PEAKS.json); sustained "
+                               f"{pk['bf16_tflops_sustained']} TFLOP/s quoted beside it",
+                "launches_timed": cnt,
+                "gemm_ms_per_step": round(sum(gt) / K_steps, 4) if cnt else None,
+                "fwd_tflops": round(rate(fwd_idx), 1), "dx_tflops": round(rate(dx_idx), 1),
+                "step_tflops": round(value / world, 2),
+                "step_frac": round(value / world / pk["bf16_tflops"], 4),
+                "step_frac_of_sustained": round(value / world / pk["bf16_tflops_sustained"], 4),
+                "per_projection": per_proj}
+
+    # End to end through the C ABI with host buffers: every step copies each
+    # projection's X and dY from pinned host memory and reads its Y, dX, dA and
+    # dB back, as a training loop does; the copies are pipelined across steps
+    # (two device buffer sets; the input copies of step i + 1 and the
+    # read-backs of step i - 1 run on their own streams while step i computes).
+    hin = [{"X": p["X"].pin_memory(), "dY": p["dY"].pin_memory()} for p in host]
+    hout = [{k: torch.empty(tuple(b[k].shape), dtype=torch.bfloat16).pin_memory() for k in ("Y", "dX", "dA", "dB")}
+            for b in main]
+    second = layer.new_set()
     sets = (main, second)
     comp = torch.cuda.current_stream()
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
@@ -337,30 +438,30 @@ def run_ours(args, rank, world, local_rank):
         if start_event is not None:
             s_in.wait_event(start_event)
         for i in range(n):
-            b, ev = sets[i % 2], evs[i % 2]
+            bs, ev_ = sets[i % 2], evs[i % 2]
             if i >= 2:
-                s_in.wait_event(ev["done"])   # step i - 2 has finished reading this set's inputs
+                s_in.wait_event(ev_["done"])   # step i - 2 has finished reading this set's inputs
             with torch.cuda.stream(s_in):
-                b["X"].copy_(Xh, non_blocking=True)
-                b["dY"].copy_(dYh, non_blocking=True)
-            ev["in"].record(s_in)
-            comp.wait_event(ev["in"])
+                for b, h in zip(bs, hin):
+                    b["X"].copy_(h["X"], non_blocking=True)
+                    b["dY"].copy_(h["dY"], non_blocking=True)
+            ev_["in"].record(s_in)
+            comp.wait_event(ev_["in"])
             if i >= 2:
-                comp.wait_event(ev["out"])    # step i - 2's results have been read back
-            step(b)
-            ev["done"].record(comp)
-            s_out.wait_event(ev["done"])
+                comp.wait_event(ev_["out"])    # step i - 2's results have been read back
+            layer.step(bs, allreduce)
+            ev_["done"].record(comp)
+            s_out.wait_event(ev_["done"])
             with torch.cuda.stream(s_out):
-                Yh.copy_(b["Y"], non_blocking=True)
-                dXh.copy_(b["dX"], non_blocking=True)
-                dAh.copy_(b["dA"], non_blocking=True)
-                dBh.copy_(b["dB"], non_blocking=True)
-            ev["out"].record(s_out)
+                for b, h in zip(bs, hout):
+                    for k in ("Y", "dX", "dA", "dB"):
+                        h[k].copy_(b[k], non_blocking=True)
+            ev_["out"].record(s_out)
         comp.wait_stream(s_out)
 
     e2e_run(2)
     torch.cuda.synchronize()
-    n_e2e = max(3, min(K_steps, 20))
+    n_e2e = max(3, min(K_steps, 10))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
@@ -373,24 +474,34 @@ def run_ours(args, rank, world, local_rank):
         t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
+    h2d = sum(h["X"].numel() * 2 + h["dY"].numel() * 2 for h in hin)
+    d2h = sum(v.numel() * 2 for h in hout for v in h.values())
     e2e = {"value": round(flops * world * n_e2e / (e2e_ms / 1e3) / 1e12, 3), "unit": "TFLOP/s",
-           "h2d_bytes_per_step": Xh.numel() * 2 + dYh.numel() * 2,
-           "d2h_bytes_per_step": (Yh.numel() + dXh.numel() + dAh.numel() + dBh.numel()) * 2,
-           "steps": n_e2e, "copies": "pipelined across steps (two device buffer sets, copy streams)"}
-    del second, sets
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
+           "copies": "pipelined across steps (two device buffer sets, copy streams)"}
+    del second, sets, hin, hout
+    torch.cuda.empty_cache()
 
-    extra = {}
+    extra = {"nf4_quantize_layer": {"weights": numel, "ms": round(quant_ms, 4),
+                                    "gbs": round(quant_bytes / quant_ms / 1e6, 1),
+                                    "frac_hbm": round(quant_bytes / quant_ms / 1e6 / pk["hbm_gbs"], 4),
+                                    "note": "the seven weights of the layer, once before the steps, through "
+                                            "nf4_quantize (each call synchronizes for its non-finite check)"}}
     if not args.no_extras:
-        extra = run_extras(qb, wl, dev, pk, flush)
+        del layer, main
+        torch.cuda.empty_cache()
+        extra.update(run_extras(qb, wl, dev, pk, flush))
 
     status = qb.device_status()
+    proj_desc = ", ".join(f"{p.name} {p.N}x{p.K}" for p in w.projections)
     out = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": K_steps,
         "warmup": args.warmup, "ms_per_step": round(total_ms / K_steps, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; see workloads.py)",
-        "config": {"workload": f"{WORKLOAD}: Llama-7B q_proj fwd+bwd, M=4096 tokens (4x1024), N=K=4096, "
-                               f"NF4 block 64 + 8-bit double quant (group 256), LoRA r=16 alpha=32",
-                   "M": M, "N": N, "K": K, "r": r, "global_batch_tokens": M * world,
+        "config": {"workload": f"{WORKLOAD}: 70B-shaped decoder layer, all 7 projections ({proj_desc}; N x K), "
+                               f"forward then backward, M={M} tokens, NF4 block 64 + 8-bit double quant "
+                               f"(group 256), LoRA r={r} alpha={w.alpha:g} on every projection",
+                   "M": M, "r": r, "global_batch_tokens": M * world, "flop_per_step": flops,
                    "parallelism": f"dp{world} (adapter grads all-reduced)" if world > 1 else "single GPU",
                    "l2": "flushed between timed steps (256 MB write, then 256 MB read: cold and clean)"},
         "roofline": roofline,
@@ -401,7 +512,8 @@ def run_ours(args, rank, world, local_rank):
         "device_status": status,
     }
     if rank == 0 and world == 1 and not args.no_cpu:
-        tf, cores, desc, dt = oracle_sample()
+        prep = oracle_layer_prepare(w, host)
+        tf, cores, desc, dt = oracle_layer_run(w, prep, args.cpu_tokens)
         out["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc,
                                "seconds": round(dt, 2)}
     if rank == 0:
@@ -525,7 +637,7 @@ def run_extras(qb, wl, dev, pk, flush):
             "quantize_gbs": round((4 * numel + cb + ab + db) / ms_q / 1e6, 1),
             "dequantize_gbs": round((cb + ab + db + 2 * numel) / ms_d / 1e6, 1)}
         del qf
-    w2 = wl.WORKLOADS[WORKLOAD]
+    w2 = wl.WORKLOADS["qproj_7b"]
     p2 = wl.draw_linear(w2)
     W2, X2, A2, B2 = p2["W"].to(dev), p2["X"].to(dev), p2["A"].to(dev), p2["B"].to(dev)
     M2, N2, K2, r2 = p2["M"], p2["N"], p2["K"], p2["r"]
@@ -569,9 +681,9 @@ def run_extras(qb, wl, dev, pk, flush):
 
 def run_configs(qb, wl, dev, pk, timed):
     """The other configurations: the 2048 x 2048 forward at 128 tokens
-    (latency-bound, in us), and fwd + bwd of every projection of the 7B MLP and
-    of the 70B decoder layer against the tensor roofline (and the one-time
-    quantize of the layer's seven weights).  Timing inputs of the same shapes
+    (latency-bound, in us), and fwd + bwd of the 7B q_proj and of every
+    projection of the 7B MLP against the tensor roofline (and the one-time
+    quantize of their weights).  Timing inputs of the same shapes
     and distributions are drawn on the device (parity of these shapes is in
     the GPU tests).  Beside each projection: a dense torch bf16 matmul of the
     forward shape on the dequantized weight, as a library ceiling."""
@@ -583,7 +695,7 @@ def run_configs(qb, wl, dev, pk, timed):
     f32 = ctypes.c_float
     out = {}
     g = torch.Generator(device=dev)
-    for name in ("fwd_2048", "mlp_7b", "layer_70b"):
+    for name in ("fwd_2048", "qproj_7b", "mlp_7b"):
         w = wl.WORKLOADS[name]
         g.manual_seed(1000 + w.seed)
         M, r, s = w.M, w.r, w.scale
@@ -650,30 +762,34 @@ def run_configs(qb, wl, dev, pk, timed):
 
 def run_reference(args, rank, world):
     """The reference arm is the CPU oracle (this method has no runnable
-    reference implementation): it is timed as it stands on the host cores,
-    W untimed and K timed steps, each step one bounded sample of the workload
-    (the row count of a sample shrinks only if the whole run would otherwise
-    take more than about 150 s)."""
+    reference implementation): it is timed as it stands on the host cores, W
+    untimed and K timed steps, each step one bounded sample of the workload
+    (the layer's forward and backward on a subset of its tokens; the subset
+    shrinks only if the whole run would otherwise take more than about 150 s).
+    The weights are drawn, quantized and dequantized by the oracle once,
+    untimed."""
     if rank != 0:
         return
-    prep = oracle_prepare()
-    rows = 512
+    from bit_nf4_quantized_24_b200 import workloads as wl
+    w = wl.WORKLOADS[WORKLOAD]
+    prep = oracle_layer_prepare(w)
+    tokens = args.cpu_tokens
     n_total = max(1, args.warmup + args.steps)
     budget_s = 150.0
     cores = desc = None
     for i in range(args.warmup):
-        _, cores, desc, dt = oracle_run(prep, rows)
+        _, cores, desc, dt = oracle_layer_run(w, prep, tokens)
         if i == 0 and dt * n_total > budget_s:
-            rows = max(32, int(rows * budget_s / (dt * n_total)) // 32 * 32)
+            tokens = max(4, int(tokens * budget_s / (dt * n_total)))
     vals = []
     for _ in range(max(1, args.steps)):
-        tf, cores, desc, dt = oracle_run(prep, rows)
+        tf, cores, desc, dt = oracle_layer_run(w, prep, tokens)
         vals.append(tf)
     v = statistics.median(vals)
     out = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
            "steps": len(vals), "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; see workloads.py)",
-           "config": {"workload": f"{WORKLOAD} (bounded sample, see cpu_baseline.sample)"},
+           "config": {"workload": f"{WORKLOAD} (bounded sample, see cpu_baseline.sample)", "tokens": tokens},
            "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
@@ -688,9 +804,19 @@ def run_profile(args):
     from bit_nf4_quantized_24_b200 import workloads as wl
     qbuild.build()
     dev = torch.device("cuda", 0)
+    if args.profile == "layer":  # warmup + steps of the benchmark's layer step (14 GEMM launches each)
+        w = wl.WORKLOADS[WORKLOAD]
+        layer = Layer(qb, w, draw_layer_host(w), dev)
+        bufs = layer.new_set(draw_layer_host(w))
+        for _ in range(args.warmup + args.steps):
+            layer.step(bufs)
+        torch.cuda.synchronize()
+        assert qb.device_status() == 0
+        print(f"profile layer {WORKLOAD} M={w.M} steps={args.warmup + args.steps} done")
+        return
     w = wl.WORKLOADS[args.workload]
     M = args.tokens if args.tokens else None
-    p = wl.draw_linear(w, 0, M=M, with_dy=args.profile in ("bwd", "step"))
+    p = wl.draw_linear(w, args.proj, M=M, with_dy=args.profile in ("bwd", "step"))
     q = qb.nf4_quantize(p["W"].to(dev))
     X, A, B = p["X"].to(dev), p["A"].to(dev), p["B"].to(dev)
     dY = p["dY"].to(dev) if "dY" in p else None
@@ -698,17 +824,18 @@ def run_profile(args):
     for _ in range(args.warmup + args.steps):
         if args.profile == "fwd_tiles":
             qb.qlora_linear_fwd_tiles(q, tiles, X, A, B, p["scale"])
+        H = None
         if args.profile in ("fwd", "step"):
             _, H = qb.qlora_linear_fwd(q, X, A, B, p["scale"])
-        if args.profile in ("bwd", "step"):
-            qb.qlora_linear_bwd(q, X, dY, A, B, p["scale"])
+        if args.profile in ("bwd", "step"):  # "step" reads the H its forward saved, as the benchmark does
+            qb.qlora_linear_bwd(q, X, dY, A, B, p["scale"], H=H)
         if args.profile == "quantize":
             qb.nf4_quantize(p["W"].to(dev))
         if args.profile == "dequantize":
             qb.nf4_dequantize(q)
     torch.cuda.synchronize()
     assert qb.device_status() == 0
-    print(f"profile {args.profile} {args.workload} M={p['M']} N={p['N']} K={p['K']} done")
+    print(f"profile {args.profile} {args.workload}[{args.proj}] M={p['M']} N={p['N']} K={p['K']} done")
 
 
 def main():
@@ -719,10 +846,13 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true", help="skip decode/quantize measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--profile", choices=["fwd", "fwd_tiles", "bwd", "step", "quantize", "dequantize"],
+    ap.add_argument("--cpu-tokens", type=int, default=128,
+                    help="token rows of the layer in the CPU oracle's bounded sample")
+    ap.add_argument("--profile", choices=["layer", "fwd", "fwd_tiles", "bwd", "step", "quantize", "dequantize"],
                     help="run only warmup+steps launches of one entry point (for ncu)")
-    ap.add_argument("--workload", default=WORKLOAD, help="workload for --profile")
+    ap.add_argument("--workload", default="qproj_7b", help="workload for --profile (other than layer)")
     ap.add_argument("--tokens", type=int, default=0, help="token count for --profile (default: the workload's)")
+    ap.add_argument("--proj", type=int, default=0, help="projection index of the workload for --profile")
     args = ap.parse_args()
     if args.profile:
         run_profile(args)
