@@ -440,100 +440,120 @@ __global__ void __launch_bounds__(32 * (NT / 2 + 1)) k_rows(const __grid_constan
 // ------------------------------------------------------------------ cols
 //
 // out = bf16(scale * D), D[c, j] = sum_m P[m, c] G[m, j] (contraction over
-// tokens), written as [R, C] or transposed [C, R].  A cluster of CL_SPLIT CTAs
-// (consecutive along grid x) owns 64 columns c x all R; its CTAs split the
-// tokens into ranges of whole 32-token slabs.  In a CTA, warp 4 lane 0 streams
-// 32-token slabs of P (32 x 64, 128-byte swizzle) and G (32 x NT*8) through
-// CL_ST stages and 4 consumer warps (16 columns each) run ldmatrix.trans +
-// mma.sync.  The CTAs then leave their fp32 partial sums in shared memory and,
-// after a cluster barrier, each CTA adds one share of the outputs over the
-// cluster's partials (distributed shared memory, fixed order) and stores it:
-// no global scratch, no second kernel, deterministic.  Rows past M arrive as
-// zeros from TMA.
-constexpr int CL_ST = 8;
+// tokens), written as [R, C] or transposed [C, R].  A cluster of up to
+// CL_SPLIT_MAX CTAs (consecutive along grid x) owns 64 CB columns c x all R;
+// its CTAs split the tokens into ranges of whole 32-token slabs.  In a CTA,
+// the last warp's lane 0 streams 32-token slabs of P (CB boxes of 32 x 64,
+// 128-byte swizzle) and G (32 x NT*8) through the stages, and the consumer
+// warps (16 MT columns each) run ldmatrix.trans + mma.sync.  CB = 4 (256
+// columns) reads G a quarter as often as CB = 1 and gives each TMA row four
+// boxes; CB = 1 serves narrow outputs, where 256-column tiles would leave
+// SMs idle.  The CTAs then leave their fp32 partial sums in shared memory (the
+// ring, no longer in use) and, after a cluster barrier, each CTA adds one
+// share of the outputs over the cluster's partials (distributed shared memory,
+// fixed order) and stores it: no global scratch, no second kernel,
+// deterministic.  Rows past M and columns past C arrive as zeros from TMA.
 constexpr int CL_SPLIT_MAX = 8;  // portable cluster size
 
-template <int NT>
-struct ColsSmem {
-  static constexpr int P_BYTES = 32 * 64 * 2;
+template <int NT, int CB>
+struct ColsCfg {
+  static constexpr int MT = CB == 1 ? 1 : 2;          // 16-column MMA tiles per consumer warp
+  static constexpr int CWC = CB * 4 / MT;             // consumer warps
+  static constexpr int THREADS = 32 * (CWC + 1);
+  static constexpr int ST = CB == 1 ? 8 : 4;          // ring stages
+  static constexpr int P_BYTES = CB * 32 * 64 * 2;    // CB boxes of 32 tokens x 64 columns
   static constexpr int G_BYTES = 32 * NT * 8 * 2;
-  static constexpr int OFF_G = CL_ST * P_BYTES;
-  static constexpr int OFF_PART = OFF_G + CL_ST * G_BYTES;      // fp32 [64 c][NT * 8 j]
-  static constexpr int OFF_BAR = OFF_PART + 64 * NT * 8 * 4;
-  static constexpr int BYTES = OFF_BAR + 2 * CL_ST * 8 + 1024;
+  static constexpr int OFF_G = ST * P_BYTES;
+  static constexpr int RING = OFF_G + ST * G_BYTES;
+  static constexpr int PART = CB * 64 * NT * 8 * 4;   // fp32 [64 CB c][NT * 8 j], over the ring
+  static constexpr int OFF_BAR = RING > PART ? RING : PART;
+  static constexpr int BYTES = OFF_BAR + 2 * ST * 8 + 1024;
 };
 
-template <int NT>
-__global__ void __launch_bounds__(160) k_cols(const __grid_constant__ CUtensorMap tmP,
-                                              const __grid_constant__ CUtensorMap tmG, int M, int C, int R,
-                                              int rows_per_split, float scale, int transpose,
-                                              uint16_t* __restrict__ out, int* status) {
-  using S = ColsSmem<NT>;
+template <int NT, int CB>
+__global__ void __launch_bounds__(ColsCfg<NT, CB>::THREADS) k_cols(const __grid_constant__ CUtensorMap tmP,
+                                                                  const __grid_constant__ CUtensorMap tmG, int M,
+                                                                  int C, int R, int rows_per_split, float scale,
+                                                                  int transpose, uint16_t* __restrict__ out,
+                                                                  int* status) {
+  using S = ColsCfg<NT, CB>;
   constexpr int RJ = NT * 8;  // j extent of the partial buffer
+  constexpr int MT = S::MT, CWC = S::CWC, ST = S::ST;
   pdl_trigger();
   pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  const uint32_t full0 = base + S::OFF_BAR, empty0 = full0 + 8u * CL_ST;
-  const uint32_t part = base + S::OFF_PART;
+  const uint32_t full0 = base + S::OFF_BAR, empty0 = full0 + 8u * ST;
+  const uint32_t part = base;  // the ring, once every stage is consumed
   __shared__ int abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint32_t nsplit;
   asm("mov.u32 %0, %%cluster_nctarank;" : "=r"(nsplit));
   const int split = static_cast<int>(cluster_ctarank());
-  const int c0 = (blockIdx.x / nsplit) * 64;
+  const int c0 = (blockIdx.x / nsplit) * 64 * CB;
   const int mb0 = split * rows_per_split;
   const int mb1 = min(M, mb0 + rows_per_split);
   const int nslab = mb1 > mb0 ? (mb1 - mb0 + 31) / 32 : 0;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < CL_ST; ++s) {
+    for (int s = 0; s < ST; ++s) {
       mbar_init(full0 + 8u * s, 1);
-      mbar_init(empty0 + 8u * s, 4);
+      mbar_init(empty0 + 8u * s, CWC);
     }
     abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
 
-  if (warp == 4) {
+  float acc[MT][NT][4];
+  if (warp == CWC) {
     if (lane == 0) {
       int issued = 0;
       for (int it = 0; it < nslab; ++it) {
-        const int s = it % CL_ST;
-        if (!wait_bounded(empty0 + 8u * s, ((it / CL_ST) & 1) ^ 1, &abort_flag, status)) break;
+        const int s = it % ST;
+        if (!wait_bounded(empty0 + 8u * s, ((it / ST) & 1) ^ 1, &abort_flag, status)) break;
         mbar_arrive_expect_tx(full0 + 8u * s, S::P_BYTES + S::G_BYTES);
-        tma_load_2d(base + s * S::P_BYTES, &tmP, full0 + 8u * s, c0, mb0 + 32 * it);
+#pragma unroll
+        for (int b = 0; b < CB; ++b)
+          tma_load_2d(base + s * S::P_BYTES + b * 4096, &tmP, full0 + 8u * s, c0 + 64 * b, mb0 + 32 * it);
         tma_load_2d(base + S::OFF_G + s * S::G_BYTES, &tmG, full0 + 8u * s, 0, mb0 + 32 * it);
         ++issued;
       }
-      for (int it = (issued > CL_ST ? issued - CL_ST : 0); it < issued; ++it)
-        wait_drain(full0 + 8u * (it % CL_ST), (it / CL_ST) & 1);
+      for (int it = (issued > ST ? issued - ST : 0); it < issued; ++it)
+        wait_drain(full0 + 8u * (it % ST), (it / ST) & 1);
     }
     __syncwarp();
   } else {
-    float acc[NT][4];
 #pragma unroll
-    for (int i = 0; i < NT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int i = 0; i < NT; ++i) acc[mt][i][0] = acc[mt][i][1] = acc[mt][i][2] = acc[mt][i][3] = 0.f;
     const int q = lane >> 3, l7 = lane & 7;
+    const int cw0 = warp * 16 * MT;                  // first column of this warp in the CTA's tile
+    const uint32_t box_off = (cw0 >> 6) * 4096;     // its box (a warp's columns stay in one box)
+    const int cchunk0 = (cw0 & 63) >> 3;             // first 8-column chunk inside the box
     for (int it = 0; it < nslab; ++it) {
-      const int s = it % CL_ST;
-      if (!wait_bounded(full0 + 8u * s, (it / CL_ST) & 1, &abort_flag, status)) break;
-      const uint32_t pt = base + s * S::P_BYTES;
+      const int s = it % ST;
+      if (!wait_bounded(full0 + 8u * s, (it / ST) & 1, &abort_flag, status)) break;
+      const uint32_t pt = base + s * S::P_BYTES + box_off;
       const uint32_t gt = base + S::OFF_G + s * S::G_BYTES;
 #pragma unroll
       for (int ks = 0; ks < 2; ++ks) {
-        uint32_t a0, a1, a2, a3;  // P^T: (c 0-7, m 0-7), (c 8-15, m 0-7), (c 0-7, m 8-15), (c 8-15, m 8-15)
-        {
-          const int m = 16 * ks + (q >> 1) * 8 + l7, chunk = 2 * warp + (q & 1);
-          ldsm_x4_trans(pt + m * 128 + ((chunk ^ (m & 7)) << 4), a0, a1, a2, a3);
+        uint32_t a[MT][4];  // P^T per 16 columns: (c 0-7, m 0-7), (c 8-15, m 0-7), (c 0-7, m 8-15), (c 8-15, m 8-15)
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          const int m = 16 * ks + (q >> 1) * 8 + l7, chunk = cchunk0 + 2 * mt + (q & 1);
+          ldsm_x4_trans(pt + m * 128 + ((chunk ^ (m & 7)) << 4), a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
         }
 #pragma unroll
         for (int np = 0; np < NT / 2; ++np) {
           uint32_t b0, b1, b2, b3;  // G: (m 0-7, tile 2np), (m 8-15, tile 2np), (m 0-7, tile 2np+1), (m 8-15, ...)
           const int m = 16 * ks + (q & 1) * 8 + l7, j = (2 * np + (q >> 1)) * 8;
           ldsm_x4_trans(narrow_addr<NT>(gt, m, j), b0, b1, b2, b3);
-          mma_bf16_16816(acc[2 * np], a0, a1, a2, a3, b0, b1);
-          mma_bf16_16816(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            mma_bf16_16816(acc[mt][2 * np], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b0, b1);
+            mma_bf16_16816(acc[mt][2 * np + 1], a[mt][0], a[mt][1], a[mt][2], a[mt][3], b2, b3);
+          }
         }
       }
       // the stage is refilled by TMA (async proxy): order this warp's reads
@@ -542,24 +562,30 @@ __global__ void __launch_bounds__(160) k_cols(const __grid_constant__ CUtensorMa
       __syncwarp();
       if (lane == 0) mbar_arrive(empty0 + 8u * s);
     }
-    // this CTA's partial sums: part[c_local][j]
+  }
+  // Every stage is consumed and every copy has landed (the producer drains):
+  // the ring now holds this CTA's partial sums part[c_local][j].
+  __syncthreads();
+  if (warp < CWC) {
     const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int cl = 16 * warp + g + 8 * h, j = nt * 8 + 2 * t;
-        asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(part + (cl * RJ + j) * 4), "f"(acc[nt][2 * h]),
-                     "f"(acc[nt][2 * h + 1])
-                     : "memory");
-      }
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int cl = warp * 16 * MT + mt * 16 + g + 8 * h, j = nt * 8 + 2 * t;
+          asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(part + (cl * RJ + j) * 4), "f"(acc[mt][nt][2 * h]),
+                       "f"(acc[mt][nt][2 * h + 1])
+                       : "memory");
+        }
   }
   cluster_sync_all();  // every CTA's partial sums are in its shared memory
 
-  // This CTA's share of the 64 x R outputs, each the sum of the cluster's
+  // This CTA's share of the 64 CB x R outputs, each the sum of the cluster's
   // partials in rank order.  Consecutive threads take consecutive output
   // addresses (c for [R, C], j for [C, R]).
-  const int V = 64 * R;
+  const int V = 64 * CB * R;
   const int v0 = static_cast<int>((static_cast<int64_t>(V) * split) / nsplit);
   const int v1 = static_cast<int>((static_cast<int64_t>(V) * (split + 1)) / nsplit);
   for (int v = v0 + static_cast<int>(threadIdx.x); v < v1; v += blockDim.x) {
@@ -568,8 +594,8 @@ __global__ void __launch_bounds__(160) k_cols(const __grid_constant__ CUtensorMa
       cl = v / R;
       j = v - cl * R;
     } else {
-      j = v >> 6;
-      cl = v & 63;
+      j = v / (64 * CB);
+      cl = v - j * (64 * CB);
     }
     const int c = c0 + cl;
     if (c >= C) continue;
@@ -649,23 +675,23 @@ cudaError_t rows_dispatch(const uint16_t* P, const uint16_t* Q, int64_t M, int64
   }
 }
 
-template <int NT>
-cudaError_t cols_launch(const uint16_t* G, const uint16_t* P, int64_t M, int64_t C, int R, float scale,
-                        int transpose, uint16_t* out, cudaStream_t st, bool pdl) {
-  using S = ColsSmem<NT>;
+template <int NT, int CB>
+cudaError_t cols_launch_cb(const uint16_t* G, const uint16_t* P, int64_t M, int64_t C, int R, float scale,
+                           int transpose, uint16_t* out, cudaStream_t st, bool pdl) {
+  using S = ColsCfg<NT, CB>;
   CUtensorMap tmP, tmG;
   const auto BF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   bool ok = make_map(&tmP, BF16, P, C, M, C * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
   ok = ok && make_map(&tmG, BF16, G, R, M, R * 2, NT * 8, 32, narrow_swizzle<NT>());
   if (!ok) return cudaErrorInvalidValue;
-  cudaError_t e = smem_limit_once<k_cols<NT>>(S::BYTES);
+  cudaError_t e = smem_limit_once<k_cols<NT, CB>>(S::BYTES);
   if (e != cudaSuccess) return e;
   const int splits = cols_splits(M);
   // token ranges are whole 32-token slabs, so a slab never straddles two splits
   const int rows_per_split = static_cast<int>(((M + splits - 1) / splits + 31) / 32 * 32);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>((C + 63) / 64 * splits), 1, 1);
-  cfg.blockDim = dim3(160, 1, 1);
+  cfg.gridDim = dim3(static_cast<unsigned>((C + 64 * CB - 1) / (64 * CB) * splits), 1, 1);
+  cfg.blockDim = dim3(S::THREADS, 1, 1);
   cfg.dynamicSmemBytes = S::BYTES;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
@@ -677,8 +703,17 @@ cudaError_t cols_launch(const uint16_t* G, const uint16_t* P, int64_t M, int64_t
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, k_cols<NT>, tmP, tmG, int(M), int(C), R, rows_per_split, scale, transpose, out,
+  return cudaLaunchKernelEx(&cfg, k_cols<NT, CB>, tmP, tmG, int(M), int(C), R, rows_per_split, scale, transpose, out,
                             device_status_ptr());
+}
+
+// 256-column tiles when they still give most SMs a CTA, else 64-column tiles.
+template <int NT>
+cudaError_t cols_launch(const uint16_t* G, const uint16_t* P, int64_t M, int64_t C, int R, float scale,
+                        int transpose, uint16_t* out, cudaStream_t st, bool pdl) {
+  if ((C + 255) / 256 * cols_splits(M) >= device_sm_count() * 3 / 4)
+    return cols_launch_cb<NT, 4>(G, P, M, C, R, scale, transpose, out, st, pdl);
+  return cols_launch_cb<NT, 1>(G, P, M, C, R, scale, transpose, out, st, pdl);
 }
 
 }  // namespace

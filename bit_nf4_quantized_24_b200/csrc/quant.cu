@@ -177,14 +177,14 @@ __device__ __forceinline__ void mergedF(const MergeSrc& m, const float* lv, int6
 // quantization of the group's absmax values (else each block's fp32 absmax is
 // stored as is).
 template <int B, bool DQ, bool MERGE>
-__global__ void __launch_bounds__(256) k_quantize(const float* __restrict__ W, MergeSrc msrc, Nf4Levels levels,
+__global__ void __launch_bounds__(256, 3) k_quantize(const float* __restrict__ W, MergeSrc msrc, Nf4Levels levels,
                                                   int64_t nblocks, const Cell* __restrict__ cells,
                                                   uint8_t* __restrict__ codes, uint8_t* __restrict__ absmax_q,
                                                   float* __restrict__ dq_scale, int* nonfinite) {
   constexpr int F = 4;
   constexpr int LP = B / (4 * F);  // 2, 4, 8, 16
   constexpr int BPW = 32 / LP;     // blocks per warp step
-  constexpr int U = 4;             // warp steps whose loads are in flight together
+  constexpr int U = MERGE ? 1 : 2; // warp steps whose loads are in flight together
   __shared__ Cell s_cell[kCells];
   __shared__ float s_amax[kGroup];
   __shared__ float s_red[8];
