@@ -53,9 +53,10 @@ WORKLOAD = "layer_70b"
 # DRAM bytes (read + write) per fused-GEMM launch, mean over the 14 launches of
 # one step of the workload above, from one ncu capture of `bench.py --profile
 # layer` (metrics dram__bytes_read.sum, dram__bytes_write.sum; the summary and
-# command are in profiles/).  Valid only for the kernel source it was taken on
-# (sha256 prefix of gemm_tc.cu); reported as null otherwise.
-GEMM_TRAFFIC = {"gemm_tc_sha16": None, "bytes_per_launch": None}
+# the command are in profiles/layer_70b_step_launch_list.md).  Valid only for
+# the kernel source it was taken on (sha256 prefix of gemm_tc.cu); reported as
+# null otherwise.
+GEMM_TRAFFIC = {"gemm_tc_sha16": "4eff4c321b201d5f", "bytes_per_launch": 474913938}
 
 
 def gemm_traffic():
