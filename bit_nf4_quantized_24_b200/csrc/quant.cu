@@ -290,6 +290,284 @@ __global__ void __launch_bounds__(256, 3) k_quantize(const float* __restrict__ W
   if (__syncthreads_or(bad) && tid == 0) atomicExch(nonfinite, 1);
 }
 
+// Merge into the default output format (blocks of 64 weights, double
+// quantization over groups of 256 blocks) when K % 1024 == 0: a CTA owns
+// MG_ROWS = 16 rows, which hold whole double-quantization groups (16 K / 64 is a
+// multiple of 256), and walks them in chunks of MG_COLS = 256 columns.  Per
+// chunk the adapter's A[:, chunk] is converted to fp32 in shared memory once
+// and serves all 16 rows; B of the 16 rows sits there too, transposed, each
+// value twice.  Two phases per chunk:
+//  * a thread forms 4 rows x 4 columns of sum_j B[n, j] A[j, k] (j in order,
+//    one FMA per exact product, as the general path; a warp covers 16 rows x
+//    32 columns) and the merged values
+//    fl32(w' + fl32(s * sum)), which go to shared memory (a byte of input codes
+//    reads the two levels it selects with one 8-byte shared load);
+//  * the 64 blocks of the chunk are coded with 4 threads per block and 16
+//    weights per thread (k_quantize's layout: two shuffles and one reciprocal
+//    per 16 weights).  Blocks sit 80 words apart in shared memory, so the
+//    16-byte accesses of each quarter-warp fall on distinct banks in both
+//    phases.
+// The arithmetic runs on pairs where it can (the f32x2 FMA, multiply and add
+// of sm_100 round each lane as the scalar instruction does).  The loads of the
+// next chunk are in flight while a chunk is computed: its A slice by cp.async
+// into a second bf16 staging buffer, its input codes and scales in registers.
+// The exact block maxima wait in shared memory until the row range is done,
+// then each group of 256 blocks is double-quantized as k_quantize does.  Same
+// results, bit for bit, as the general path (the merge source of k_quantize).
+constexpr int MG_ROWS = 16, MG_COLS = 256;
+
+constexpr int MG_XP = 80;  // words from one block of merged values to the next
+
+__host__ __device__ constexpr int merge64_smem_bytes(int r, int K) {
+  return r * MG_COLS * 4 + 2 * r * MG_COLS * 2 + r * MG_ROWS * 8 + MG_ROWS * (MG_COLS / 64) * MG_XP * 4 +
+         MG_ROWS * (K / 64) * 4;
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Pairs of fp32 values in one 64-bit register (low half = first value).
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ float lo2(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float hi2(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// Both values rounded to bf16 and back to fp32.
+__device__ __forceinline__ uint64_t bf16_round2(uint64_t v) {
+  uint32_t h;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(hi2(v)), "f"(lo2(v)));
+  return pk2(__uint_as_float(h << 16), __uint_as_float(h & 0xffff0000u));
+}
+
+// Input codes (4 per row) and the input block scale of this thread's 4 rows
+// in one chunk.  Offsets are relative to the CTA's first row (32-bit: a CTA
+// covers 16 K <= 2^20 weights).
+struct MergeIn {
+  uint32_t c[4];
+  float a[4];
+};
+
+struct MergeBase {
+  const uint8_t* codes;     // input codes of the CTA's first row
+  const uint8_t* absmax_q;  // input block scales (codes when dq) of that row
+  const float* dq_scale;    // fp32 scales: per block, or per group of 256 blocks when dq
+  int lg, dq;
+  uint32_t bphase;          // dq: index of the first row's first block inside its group
+};
+
+__device__ __forceinline__ void merge_in_load(const MergeBase& mb, uint32_t e0, uint32_t K, int nrows, int rg,
+                                              MergeIn& in) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    in.c[i] = 0;
+    in.a[i] = 0.f;
+    if (4 * rg + i < nrows) {
+      const uint32_t e = e0 + static_cast<uint32_t>(4 * rg + i) * K;
+      in.c[i] = __ldg(reinterpret_cast<const uint16_t*>(mb.codes + (e >> 1)));
+      const uint32_t b = e >> mb.lg;
+      in.a[i] = mb.dq ? __fmul_rn(static_cast<float>(__ldg(mb.absmax_q + b)), __ldg(mb.dq_scale + ((mb.bphase + b) >> 8)))
+                      : __ldg(mb.dq_scale + b);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256, 4) k_merge64(MergeSrc m, Nf4Levels levels, int64_t N,
+                                                    const Cell* __restrict__ cells, uint8_t* __restrict__ codes,
+                                                    uint8_t* __restrict__ absmax_q, float* __restrict__ dq_scale,
+                                                    int* nonfinite) {
+  extern __shared__ __align__(16) float msm[];
+  __shared__ Cell s_cell[kCells];
+  __shared__ uint64_t s_lv2[256];  // byte of two codes -> {L[low nibble], L[high nibble]}
+  __shared__ float s_red[8];
+  const int K = static_cast<int>(m.K), KB = K / 64, r = m.r, nch = K / MG_COLS;
+  float* As = msm;                                                      // [r][MG_COLS] fp32
+  uint16_t* St = reinterpret_cast<uint16_t*>(As + r * MG_COLS);         // 2 x [r][MG_COLS] bf16 staging
+  float* Bs = reinterpret_cast<float*>(St + 2 * r * MG_COLS);           // [r][MG_ROWS][2]
+  float* Xs = Bs + r * MG_ROWS * 2;                                     // [MG_ROWS * 4 blocks][MG_XP] merged
+  float* ab = Xs + MG_ROWS * (MG_COLS / 64) * MG_XP;                    // [MG_ROWS][KB] exact block maxima
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // columns 4 cg .. 4 cg + 3 of a chunk, rows 4 rg .. 4 rg + 3 (a warp covers 16 rows x 32 columns)
+  const int cg = warp * 8 + (lane & 7), rg = lane >> 3;
+  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * MG_ROWS;
+  const int nrows = static_cast<int>(N - n0 < MG_ROWS ? N - n0 : MG_ROWS);
+  const int a16 = r * MG_COLS / 8;  // 16-byte pieces of one chunk of A
+
+  auto stage = [&](int c) {  // A[:, chunk c] -> staging buffer c & 1
+    uint16_t* dst = St + (c & 1) * r * MG_COLS;
+    for (int i = tid; i < a16; i += 256) {
+      const int j = i / (MG_COLS / 8), k8 = i - j * (MG_COLS / 8);
+      cp_async16(dst + j * MG_COLS + k8 * 8, m.A + static_cast<int64_t>(j) * K + c * MG_COLS + k8 * 8);
+    }
+    cp_async_commit();
+  };
+  stage(0);
+  s_cell[tid] = cells[tid];
+  s_lv2[tid] = pk2(levels.v[tid & 15], levels.v[tid >> 4]);
+  for (int i = tid; i < r * MG_ROWS; i += 256) {
+    const int j = i / MG_ROWS, row = i - j * MG_ROWS;
+    const float b = row < nrows ? bf16_bits_to_f32(m.B[(n0 + row) * r + j]) : 0.f;
+    Bs[2 * i] = b;
+    Bs[2 * i + 1] = b;
+  }
+  const uint64_t s_2 = pk2(m.s, m.s);
+  const uint64_t k64 = pk2(64.0f, 64.0f), kbias = pk2(12582976.0f, 12582976.0f);
+  const int64_t e_cta = n0 * K;  // first weight of the CTA (a multiple of 16384)
+  const int64_t b_cta = e_cta >> m.lg;  // its input block
+  const MergeBase mb{m.codes + e_cta / 2, m.dq ? m.absmax_q + b_cta : nullptr,
+                     m.dq_scale + (m.dq ? b_cta >> 8 : b_cta), m.lg, m.dq, static_cast<uint32_t>(b_cta & 255)};
+  uint8_t* const codes_cta = codes + e_cta / 2;
+  MergeIn cur, nxt;
+  merge_in_load(mb, 4 * cg, K, nrows, rg, cur);
+  bool bad = false;
+  for (int c = 0; c < nch; ++c) {
+    cp_async_wait_all();
+    __syncthreads();  // chunk c staged by all threads; everyone is done with As of chunk c - 1
+    {
+      const uint16_t* src = St + (c & 1) * r * MG_COLS;
+      for (int i = tid; i < a16; i += 256) {
+        const uint4 a = *reinterpret_cast<const uint4*>(src + i * 8);
+        float4* dst = reinterpret_cast<float4*>(As + i * 8);
+        dst[0] = make_float4(__uint_as_float(a.x << 16), __uint_as_float(a.x & 0xffff0000u),
+                             __uint_as_float(a.y << 16), __uint_as_float(a.y & 0xffff0000u));
+        dst[1] = make_float4(__uint_as_float(a.z << 16), __uint_as_float(a.z & 0xffff0000u),
+                             __uint_as_float(a.w << 16), __uint_as_float(a.w & 0xffff0000u));
+      }
+    }
+    if (c + 1 < nch) {
+      stage(c + 1);  // buffer (c + 1) & 1 was last read before the barrier above
+      merge_in_load(mb, (c + 1) * MG_COLS + 4 * cg, K, nrows, rg, nxt);
+    }
+    __syncthreads();  // As holds chunk c
+    uint64_t acc[4][2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = 0;
+#pragma unroll 4
+    for (int j = 0; j < r; ++j) {
+      const ulonglong2 a4 = *reinterpret_cast<const ulonglong2*>(As + j * MG_COLS + 4 * cg);
+      const ulonglong2 b01 = *reinterpret_cast<const ulonglong2*>(Bs + (j * MG_ROWS + 4 * rg) * 2);
+      const ulonglong2 b23 = *reinterpret_cast<const ulonglong2*>(Bs + (j * MG_ROWS + 4 * rg) * 2 + 4);
+      acc[0][0] = fma2(b01.x, a4.x, acc[0][0]);
+      acc[0][1] = fma2(b01.x, a4.y, acc[0][1]);
+      acc[1][0] = fma2(b01.y, a4.x, acc[1][0]);
+      acc[1][1] = fma2(b01.y, a4.y, acc[1][1]);
+      acc[2][0] = fma2(b23.x, a4.x, acc[2][0]);
+      acc[2][1] = fma2(b23.x, a4.y, acc[2][1]);
+      acc[3][0] = fma2(b23.y, a4.x, acc[3][0]);
+      acc[3][1] = fma2(b23.y, a4.y, acc[3][1]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {  // merged values of row 4 rg + i -> Xs
+      const uint64_t a2 = pk2(cur.a[i], cur.a[i]);
+      const uint64_t w01 = bf16_round2(mul2(s_lv2[cur.c[i] & 255u], a2));
+      const uint64_t w23 = bf16_round2(mul2(s_lv2[cur.c[i] >> 8], a2));
+      ulonglong2 x;
+      x.x = add2(w01, mul2(s_2, acc[i][0]));
+      x.y = add2(w23, mul2(s_2, acc[i][1]));
+      *reinterpret_cast<ulonglong2*>(Xs + ((4 * rg + i) * 4 + (cg >> 4)) * MG_XP + (cg & 15) * 4) = x;
+    }
+    __syncthreads();  // Xs holds the chunk's merged values
+    {
+      const int bid = tid >> 2, sl = tid & 3;  // block bid of the chunk: row bid / 4, column block bid % 4
+      const int row = bid >> 2;
+      const float* xb = Xs + bid * MG_XP;
+      ulonglong2 v[4];
+#pragma unroll
+      for (int f = 0; f < 4; ++f) v[f] = *reinterpret_cast<const ulonglong2*>(xb + (f * 4 + sl) * 4);
+      float mx = 0.0f;
+#pragma unroll
+      for (int f = 0; f < 4; ++f)
+        mx = fmax_nan(mx, fmax_nan(fmax_nan(fabsf(lo2(v[f].x)), fabsf(hi2(v[f].x))),
+                                   fmax_nan(fabsf(lo2(v[f].y)), fabsf(hi2(v[f].y)))));
+      mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmax_nan(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      if (row < nrows) {
+        uint16_t* dst = reinterpret_cast<uint16_t*>(codes_cta + ((static_cast<uint32_t>(row) * K + c * MG_COLS) >> 1) +
+                                                    (bid & 3) * 32) + sl;
+        if (__builtin_expect(mx >= 0x1p-100f && mx <= 0x1p100f, 1)) {
+          // div_by_absmax on pairs: q0 = x r, e = fma(q0, -a, x) (= fma(-q0, a, x)), t = fma(e, r, q0)
+          const float rr = __frcp_rn(mx);
+          const uint64_t r2 = pk2(rr, rr), na2 = pk2(-mx, -mx);
+#pragma unroll
+          for (int f = 0; f < 4; ++f) {
+            const uint64_t q01 = mul2(v[f].x, r2), q23 = mul2(v[f].y, r2);
+            const uint64_t t01 = fma2(fma2(q01, na2, v[f].x), r2, q01);
+            const uint64_t t23 = fma2(fma2(q23, na2, v[f].y), r2, q23);
+            const uint64_t f01 = fma2(t01, k64, kbias), f23 = fma2(t23, k64, kbias);
+            const float t[4] = {lo2(t01), hi2(t01), lo2(t23), hi2(t23)};
+            const float g[4] = {lo2(f01), hi2(f01), lo2(f23), hi2(f23)};
+            uint32_t code = 0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const Cell cl = s_cell[__float_as_uint(g[q]) & (kCells - 1)];
+              code |= static_cast<uint32_t>(cl.base + (t[q] > cl.mid ? 1 : 0)) << (4 * q);
+            }
+            dst[f * 4] = static_cast<uint16_t>(code);
+          }
+        } else {
+          const bool finite = mx <= 3.402823466e38f;  // false for NaN and infinity
+          bad |= !finite;
+#pragma unroll
+          for (int f = 0; f < 4; ++f) {
+            const float x[4] = {lo2(v[f].x), hi2(v[f].x), lo2(v[f].y), hi2(v[f].y)};
+            uint32_t code = 0x7777u;
+            if (mx != 0.0f && finite)
+              code = nf4_code(__fdiv_rn(x[0], mx), s_cell) | (nf4_code(__fdiv_rn(x[1], mx), s_cell) << 4) |
+                     (nf4_code(__fdiv_rn(x[2], mx), s_cell) << 8) | (nf4_code(__fdiv_rn(x[3], mx), s_cell) << 12);
+            dst[f * 4] = static_cast<uint16_t>(code);
+          }
+        }
+        if (sl == 0) ab[row * KB + c * (MG_COLS / 64) + (bid & 3)] = mx;
+      }
+    }
+    cur = nxt;
+  }
+  __syncthreads();
+  // double quantization of the row range's groups (256 consecutive blocks each)
+  const int nb = nrows * KB;
+  for (int g0 = 0; g0 < nb; g0 += kGroup) {
+    const int i = g0 + tid;
+    const float v = i < nb ? ab[i] : 0.0f;
+    float mv = v;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mv = fmaxf(mv, __shfl_xor_sync(0xffffffffu, mv, off));
+    if (lane == 0) s_red[warp] = mv;
+    __syncthreads();
+    float c2 = s_red[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) c2 = fmaxf(c2, s_red[w]);
+    const float s2 = (c2 > 0.0f) ? __fdiv_rn(c2, 255.0f) : 0.0f;
+    if (i < nb) {
+      uint8_t q = 0;
+      if (s2 != 0.0f) q = static_cast<uint8_t>(fminf(255.0f, rintf(__fdiv_rn(v, s2))));
+      absmax_q[n0 * KB + i] = q;
+    }
+    if (tid == 0) dq_scale[(n0 * KB + g0) / kGroup] = s2;
+    __syncthreads();  // s_red is reused by the next group
+  }
+  if (__syncthreads_or(bad) && tid == 0) atomicExch(nonfinite, 1);
+}
+
 // One thread expands 64 consecutive weights (one register table per block
 // of B weights it touches: two for B = 32, one otherwise; 32 code bytes in,
 // 128 bytes of bf16 out); a warp's 32 x 64 weights pass through shared memory
@@ -402,6 +680,17 @@ cudaError_t launch_merge_quantize(const uint8_t* codes_in, const uint8_t* absmax
   int lg = 0;
   while ((1 << lg) < block_in) ++lg;
   const MergeSrc m{codes_in, absmax_in, dq_in, lg, dq_block_in ? 1 : 0, A, Bl, r, scale, K};
+  if (block == 64 && dq_block == 256 && K % 1024 == 0 && K <= 65536) {  // the tiled path (default output format)
+    cudaError_t e;
+    const Cell* cells = device_cells(&e);
+    if (!cells) return e;
+    const int smem = merge64_smem_bytes(r, static_cast<int>(K));
+    e = cudaFuncSetAttribute(k_merge64, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = static_cast<unsigned>((N + MG_ROWS - 1) / MG_ROWS);
+    k_merge64<<<grid, 256, smem, st>>>(m, host_codebook().levels, N, cells, codes, absmax_q, dq_scale, nonfinite);
+    return cudaGetLastError();
+  }
   const MergeSrc* mp = &m;
   const int64_t numel = N * K;
   const float* W = nullptr;

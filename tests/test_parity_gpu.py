@@ -221,6 +221,40 @@ def test_merge_lora_bit_exact(qb, oracle, fmt_in, fmt_out, r):
     assert m.dq_scale.cpu().numpy().tobytes() == od.tobytes(), "scales differ"
 
 
+@pytest.mark.parametrize("N,K,fmt_in,r", [(45, 3072, (128, 0), 64), (16, 2048, (64, 256), 1), (3, 1024, (32, 256), 16),
+                                           (40, 1024, (256, 256), 8), (50, 1024, (128, 256), 5)])
+def test_merge_lora_tiled_shapes(qb, oracle, N, K, fmt_in, r):
+    """Merges into the default format with K a multiple of 1024 (the tiled
+    path: 16 rows per CTA, groups of 256 blocks that start inside a row when
+    K / 64 is not a multiple of 256, a ragged last row range) equal the oracle
+    bit for bit; a row whose merged values are all zero codes the zero level."""
+    W = wl.draw_weight(wl.generator(710 + N), N, K, 0.02, 0.02)
+    W[N - 1, :] = 0.0
+    q, _ = quantize_both(qb, oracle, W, *fmt_in)
+    g = wl.generator(810 + r)
+    A = ((torch.rand(r, K, generator=g) * 2 - 1) / np.sqrt(K)).bfloat16()
+    B = (torch.randn(N, r, generator=g) * 0.05).bfloat16()
+    B[N - 1, :] = 0.0
+    m = qb.nf4_merge_lora(q, A.cuda(), B.cuda(), 1.5, 64, 256)
+    oc, oa, od, _ = oracle.nf4_merge_lora(q.codes.cpu().numpy(), q.absmax_q.cpu().numpy(), q.dq_scale.cpu().numpy(),
+                                          N, K, bits(A), bits(B), 1.5, *fmt_in, 64, 256)
+    assert np.array_equal(m.codes.cpu().numpy(), oc), "codes differ"
+    assert np.array_equal(m.absmax_q.cpu().numpy(), oa), "absmax codes differ"
+    assert m.dq_scale.cpu().numpy().tobytes() == od.tobytes(), "scales differ"
+
+
+def test_merge_lora_reports_overflow(qb):
+    """A merge whose values overflow fp32 (a huge scale) is reported as
+    non-finite, as a quantize of such weights is."""
+    N, K, r = 20, 1024, 4
+    q = qb.nf4_quantize(wl.draw_weight(wl.generator(720), N, K, 0.02, 0.0).cuda())
+    A = torch.ones(r, K, dtype=torch.bfloat16, device="cuda")
+    B = torch.ones(N, r, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(qb.QloraError) as ei:
+        qb.nf4_merge_lora(q, A, B, 3.0e38)
+    assert ei.value.status == -3
+
+
 def test_merge_lora_at_decode_scale(qb, oracle):
     """The 70B-shaped up projection merged with its r = 16 adapter: sampled
     rows against the oracle (the merge of a row depends only on that row)."""
