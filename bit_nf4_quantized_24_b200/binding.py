@@ -81,6 +81,7 @@ def lib():
     L.qlora_trace_gemm_count.restype = i32
     L.qlora_gemm_resident_pairs.argtypes = [i32]
     L.qlora_gemm_resident_pairs.restype = i32
+    L.qlora_gemm_split_plan.argtypes = [i32, i64, i64, i64, P, P, P]
     _lib = L
     return L
 
@@ -434,6 +435,15 @@ def qlora_linear_fwd_noalloc(w: NF4Weight, X: torch.Tensor, A: torch.Tensor, B: 
 def gemm_resident_pairs(mode: int = 0) -> int:
     """CTA pairs of the fused GEMM that fit on the current device at once."""
     return lib().qlora_gemm_resident_pairs(mode)
+
+
+def gemm_split_plan(mode: int, M: int, N: int, K: int) -> tuple[int, int, int]:
+    """(pieces per split tile, split tiles, bytes of fp32 partial sums) of the
+    fused GEMM for an M x N x K layer on the current device."""
+    ns, nt, pb = ctypes.c_int(), ctypes.c_int64(), ctypes.c_size_t()
+    _check(lib().qlora_gemm_split_plan(mode, M, N, K, ctypes.byref(ns), ctypes.byref(nt), ctypes.byref(pb)),
+           "qlora_gemm_split_plan")
+    return ns.value, nt.value, pb.value
 
 
 def device_status() -> int:

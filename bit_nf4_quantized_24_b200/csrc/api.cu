@@ -140,6 +140,20 @@ BwdWorkspace bwd_layout(void* ws, int64_t M, int64_t N, int64_t K, int r) {
   return w;
 }
 
+// The fused GEMM's room for the fp32 partial sums of split tiles: whatever
+// the workspace holds past its first `used` bytes (the launch splits only if
+// that is at least the plan's part_bytes).
+void gemm_part(GemmArgs& a, void* ws, size_t used, size_t ws_bytes) {
+  const size_t off = align256(used);
+  if (ws && ws_bytes > off) {
+    a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + off);
+    a.part_bytes = ws_bytes - off;
+  }
+}
+size_t gemm_part_bytes(int mode, int64_t M, int64_t N, int64_t K) {
+  return M > 16 ? align256(gemm_split_plan(mode, M, N, K).part_bytes) : 0;
+}
+
 // The side stream of caller stream `s` on the current device, created on
 // first use.  Returns false (the backward then runs on `s` alone) if creation
 // fails, if the device already has kMaxSideStreams of them, or if `s` is being
@@ -346,7 +360,7 @@ int qlora_linear_fwd_workspace(int64_t M, int64_t N, int64_t K, int r, size_t* b
   if (!bytes) return QLORA_ERR_ARG;
   int st = check_layer_shapes(M, N, K, r);
   if (st) return st;
-  *bytes = fwd_layout(nullptr, M, r).bytes;
+  *bytes = fwd_layout(nullptr, M, r).bytes + gemm_part_bytes(0, M, N, K);
   return QLORA_OK;
 }
 
@@ -354,7 +368,7 @@ int qlora_linear_bwd_workspace(int64_t M, int64_t N, int64_t K, int r, size_t* b
   if (!bytes) return QLORA_ERR_ARG;
   int st = check_layer_shapes(M, N, K, r);
   if (st) return st;
-  *bytes = bwd_layout(nullptr, M, N, K, r).bytes;
+  *bytes = bwd_layout(nullptr, M, N, K, r).bytes + gemm_part_bytes(1, M, N, K);
   return QLORA_OK;
 }
 
@@ -398,6 +412,7 @@ int qlora_linear_fwd_fmt(const uint8_t* codes, const uint8_t* absmax_q, const fl
     a.pdl = true;  // its main loop runs while the H kernel finishes; the LoRA tail waits
     a.block = block;
     a.dq_block = dq_block;
+    gemm_part(a, workspace, w.bytes, workspace_bytes);
     e = launch_nf4_gemm(a, s);
   }
   return cuda_status(e);
@@ -504,7 +519,8 @@ int qlora_linear_dropout_workspace(int64_t M, int64_t N, int64_t K, int r, size_
   int st = check_layer_shapes(M, N, K, r);
   if (st) return st;
   const size_t base = std::max(fwd_layout(nullptr, M, r).bytes, bwd_layout(nullptr, M, N, K, r).bytes);
-  *bytes = drop_layout(nullptr, base, M, K, r).bytes;
+  *bytes = drop_layout(nullptr, base, M, K, r).bytes +
+           std::max(gemm_part_bytes(0, M, N, K), gemm_part_bytes(1, M, N, K));
   return QLORA_OK;
 }
 
@@ -547,6 +563,7 @@ int qlora_linear_fwd_dropout(const uint8_t* codes, const uint8_t* absmax_q, cons
     a.r = r;
     a.out = Y;
     a.pdl = true;
+    gemm_part(a, workspace, d.bytes, workspace_bytes);
     e = launch_nf4_gemm(a, s);
   }
   return cuda_status(e);
@@ -604,6 +621,7 @@ int qlora_linear_bwd_dropout(const uint8_t* codes, const uint8_t* absmax_q, cons
     a.r = r;
     a.out = dX;
     a.pdl = true;
+    gemm_part(a, workspace, d.bytes, workspace_bytes);
     e = launch_nf4_gemm(a, s);
     if (e == cudaSuccess) e = launch_dx_add_masked(dX, w.dH16, A, keep_mask, keep_scale, M, K, r, s, true);
   }
@@ -624,7 +642,7 @@ namespace {
 // tail (dH, A); a programmatic dependent launch (it waits before the tail).
 cudaError_t launch_dx_gemm(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale, int block,
                            int dq_block, int64_t N, int64_t K, const uint16_t* dY, int64_t M, const uint16_t* A, int r,
-                           const uint16_t* dH, uint16_t* dX, cudaStream_t s) {
+                           const uint16_t* dH, uint16_t* dX, void* ws, size_t used, size_t ws_bytes, cudaStream_t s) {
   GemmArgs a{};
   a.mode = 1;
   a.act = dY;
@@ -641,6 +659,7 @@ cudaError_t launch_dx_gemm(const uint8_t* codes, const uint8_t* absmax_q, const 
   a.pdl = true;
   a.block = block;
   a.dq_block = dq_block;
+  gemm_part(a, ws, used, ws_bytes);
   return launch_nf4_gemm(a, s);
 }
 }  // namespace
@@ -691,7 +710,8 @@ int qlora_linear_bwd_fmt(const uint8_t* codes, const uint8_t* absmax_q, const fl
     e = cudaEventRecord(ss.fork, s);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.st, ss.fork, 0);
     if (e != cudaSuccess) return cuda_status(e);
-    e = launch_dx_gemm(codes, absmax_q, dq_scale, block, dq_block, N, K, dY, M, A, r, w.dH16, dX, s);
+    e = launch_dx_gemm(codes, absmax_q, dq_scale, block, dq_block, N, K, dY, M, A, r, w.dH16, dX, workspace, w.bytes,
+                       workspace_bytes, s);
     if (e == cudaSuccess) e = launch_coldot(w.dH16, X, M, K, r, 1.0f, 0, dA, ss.st, false);
     if (e == cudaSuccess) e = launch_coldot(Huse, dY, M, N, r, scale, 1, dB, ss.st, true);
     // join on every path, so that nothing of this call stays unordered with `s`
@@ -705,7 +725,8 @@ int qlora_linear_bwd_fmt(const uint8_t* codes, const uint8_t* absmax_q, const fl
   e = launch_coldot(w.dH16, X, M, K, r, 1.0f, 0, dA, s, true);
   if (e == cudaSuccess) e = launch_coldot(Huse, dY, M, N, r, scale, 1, dB, s, true);
   if (e == cudaSuccess && dX)
-    e = launch_dx_gemm(codes, absmax_q, dq_scale, block, dq_block, N, K, dY, M, A, r, w.dH16, dX, s);
+    e = launch_dx_gemm(codes, absmax_q, dq_scale, block, dq_block, N, K, dY, M, A, r, w.dH16, dX, workspace, w.bytes,
+                       workspace_bytes, s);
   return cuda_status(e);
 }
 
@@ -757,6 +778,17 @@ int qlora_trace_gemm_events(void** events, int n_pairs) {
 }
 
 int qlora_trace_gemm_count(void) { return t_trace_count; }
+
+int qlora_gemm_split_plan(int mode, int64_t M, int64_t N, int64_t K, int* nsplit, int64_t* ntail_tiles,
+                          size_t* partial_bytes) {
+  if ((mode != 0 && mode != 1) || M < 0 || N <= 0 || K <= 0) return QLORA_ERR_ARG;
+  SplitPlan p{};
+  if (M > 16) p = gemm_split_plan(mode, M, N, K);
+  if (nsplit) *nsplit = p.nsplit;
+  if (ntail_tiles) *ntail_tiles = p.nsplit > 1 ? p.ntail : 0;
+  if (partial_bytes) *partial_bytes = p.part_bytes;
+  return QLORA_OK;
+}
 
 int qlora_gemm_resident_pairs(int mode) {
   if (mode != 0 && mode != 1) return QLORA_ERR_ARG;

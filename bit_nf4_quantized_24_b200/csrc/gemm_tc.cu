@@ -32,6 +32,7 @@
 // Every wait is bounded (kWaitLimitNs); on expiry the kernel records
 // kDevTimeout, drains what it issued, frees TMEM and exits.
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "internal.h"
@@ -76,6 +77,14 @@ struct Bars {
   int abort;
 };
 
+// Work items of a launch: whole tiles first, then nsplit pieces of each of
+// the last ntail tiles (the tiles that would otherwise form a partial last
+// wave on the resident CTA pairs).
+struct SplitGrid {
+  int npairs, nout_tiles;  // token pairs and output tiles (tiles = npairs * nout_tiles)
+  int nwhole, ntail, nsplit;
+};
+
 // GEN = false: the default NF4 format (64-weight blocks, double quantization
 // over groups of 256 blocks).  GEN = true: 2^lg-weight blocks (lg = 5..8),
 // double quantization on or off (dq), chosen at run time; a thread's 64
@@ -85,7 +94,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_nf4_gemm(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_codes,
                const __grid_constant__ CUtensorMap tm_tail_a, const __grid_constant__ CUtensorMap tm_tail_b,
                const uint8_t* __restrict__ absmax_q, const float* __restrict__ dq_scale, Nf4Levels lv, int M, int N,
-               int K, int r, int band_pairs, int lg, int dq, __nv_bfloat16* __restrict__ out, int* status) {
+               int K, int r, int band_pairs, int lg, int dq, __nv_bfloat16* __restrict__ out, int* status,
+               SplitGrid sg, float* __restrict__ part) {
   pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -110,19 +120,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int Kc = MODE == 0 ? K : N;
   const int Nout = MODE == 0 ? N : K;
   const int numK = (Kc + BK - 1) / BK;
-  // Pairs are handed out band by band: a band of `band_pairs` token pairs
-  // sweeps every output tile before the next band starts, so the band's
+  // Work item blockIdx.x / 2: items below sg.nwhole are whole tiles (tile L =
+  // item); the rest are pieces of the last sg.ntail tiles, sg.nsplit per tile,
+  // piece z taking the z-th of nsplit contiguous ranges of K stages (the last
+  // piece also the LoRA stage) and leaving fp32 partial sums for the reduction
+  // kernel.  Tiles are handed out band by band: a band of `band_pairs` token
+  // pairs sweeps every output tile before the next band starts, so the band's
   // activations stay in L2 while the weight tiles stream past them.
-  int pair, otile;
+  int pair, otile, zpiece = 0, nsplit = 1, tail_idx = 0;
   {
-    const int npx = gridDim.x >> 1, nout = gridDim.y;
-    const int L = blockIdx.y * npx + (blockIdx.x >> 1);  // launch order of the pair
+    const int item = blockIdx.x >> 1;
+    int L = item;
+    if (item >= sg.nwhole) {
+      const int j = item - sg.nwhole;
+      nsplit = sg.nsplit;
+      tail_idx = j / nsplit;
+      zpiece = j - tail_idx * nsplit;
+      L = sg.nwhole + tail_idx;
+    }
+    const int npx = sg.npairs, nout = sg.nout_tiles;
     const int per_band = band_pairs * nout;
     const int band = L / per_band, rem = L - band * per_band;
     const int in_band = min(band_pairs, npx - band * band_pairs);
     otile = rem / in_band;
     pair = band * band_pairs + (rem - otile * in_band);
   }
+  const int kbeg = (zpiece * numK) / nsplit, kend = ((zpiece + 1) * numK) / nsplit;
+  const int nloc = kend - kbeg;                  // K stages of this item
+  const bool has_tail = zpiece == nsplit - 1;    // it also runs the LoRA stage
+  const int nstage = nloc + (has_tail ? 1 : 0);  // ring iterations
   const int n0 = otile * BN;                            // first output of the pair's tile
   const int nl0 = n0 + BNL * static_cast<int>(rank);    // first output this CTA expands
   const int m0 = (2 * pair + static_cast<int>(rank)) * BM;  // first token of this CTA
@@ -165,19 +191,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       int a_issued = 0, c_issued = 0;
       bool ok = true;
+      // it: the item's ring iteration; the K stage it loads is kbeg + it
       auto issue_codes = [&](int it) {
         const int c = it % CSTAGES;
         if (!(ok = wait_bounded(empty_c(c), ((it / CSTAGES) & 1) ^ 1, abort, status))) return;
         mbar_arrive_expect_tx(full_c(c), C_BYTES);
         if (MODE == 0)
-          tma_load_2d(base + OFF_C + c * C_BYTES, &tm_codes, full_c(c), it * (BK / 2), nl0);
+          tma_load_2d(base + OFF_C + c * C_BYTES, &tm_codes, full_c(c), (kbeg + it) * (BK / 2), nl0);
         else
-          tma_load_2d(base + OFF_C + c * C_BYTES, &tm_codes, full_c(c), nl0 / 2, it * BK);
+          tma_load_2d(base + OFF_C + c * C_BYTES, &tm_codes, full_c(c), nl0 / 2, (kbeg + it) * BK);
         ++c_issued;
       };
-      for (int it = 0; it < CAHEAD && it < numK && ok; ++it) issue_codes(it);
-      for (int it = 0; it < numK && ok; ++it) {
-        if (it + CAHEAD < numK) {
+      for (int it = 0; it < CAHEAD && it < nloc && ok; ++it) issue_codes(it);
+      for (int it = 0; it < nloc && ok; ++it) {
+        if (it + CAHEAD < nloc) {
           issue_codes(it + CAHEAD);
           if (!ok) break;
         }
@@ -185,7 +212,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t ph = (it / STAGES) & 1;
         if (!(ok = wait_bounded(empty(s), ph ^ 1, abort, status))) break;
         mbar_arrive_expect_tx(full_tma(s), A_BYTES);
-        tma_load_2d(base + OFF_A + s * A_BYTES, &tm_act, full_tma(s), it * BK, m0);
+        tma_load_2d(base + OFF_A + s * A_BYTES, &tm_act, full_tma(s), (kbeg + it) * BK, m0);
         ++a_issued;
       }
       // The tail operands come from the previous kernel of the stream, which
@@ -193,8 +220,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // input of this kernel predates it.  Waited for on every path, so that
       // this grid completes only after its predecessor.
       pdl_wait();
-      if (ok) {  // tail stage: LoRA operands
-        const int it = numK, s = it % STAGES;
+      if (ok && has_tail) {  // tail stage: LoRA operands
+        const int it = nloc, s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
         if ((ok = wait_bounded(empty(s), ph ^ 1, abort, status))) {
           mbar_arrive_expect_tx(full_tma(s), A_BYTES + B_BYTES);
@@ -222,10 +249,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       constexpr uint32_t idesc = idesc_bf16(2 * UM, BN, false, MODE == 1);
       bool ok = true;
       int committed = 0;
-      for (int it = 0; it <= numK; ++it) {
+      for (int it = 0; it < nstage; ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
-        const bool tail = (it == numK);
+        const bool tail = (it == nloc);
         // full_deq gathers both CTAs: their tiles landed and their B halves are written
         if (!(ok = wait_bounded_cluster(full_deq(s), ph, abort, status))) break;
         tc_fence_after();
@@ -277,9 +304,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     };
     auto fetch = [&](int it) {
       Scale sc{0u, 0u, 0.0f, 0.0f, false};
-      if (it < numK) {
+      if (it < nloc) {
         int wrow, kcol0;
-        item_of(it, wrow, kcol0);
+        item_of(kbeg + it, wrow, kcol0);
         if (wrow < N && kcol0 < K) {
           if (!GEN) {
             const int64_t blk = static_cast<int64_t>(wrow) * KB + (kcol0 >> 6);
@@ -305,11 +332,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       return sc;
     };
     Scale p0 = fetch(grp), p1 = fetch(grp + DQ_GROUPS);
-    for (int it = grp; it <= numK; it += DQ_GROUPS) {  // it == numK: the tail stage
+    for (int it = grp; it < nstage; it += DQ_GROUPS) {  // it == nloc: the tail stage
       const Scale p2 = fetch(it + 2 * DQ_GROUPS);
       const int s = it % STAGES;
       const uint32_t ph = (it / STAGES) & 1;
-      if (it < numK) {
+      if (it < nloc) {
         const int cs = it % CSTAGES;
         if (!(ok = wait_bounded(full_c(cs), (it / CSTAGES) & 1, abort, status))) break;
         const uint32_t c_s = base + OFF_C + cs * C_BYTES;
@@ -382,7 +409,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                            v);
         tmem_ld_wait();
         const int n = n0 + col;
-        if (m < M && n < Nout) {
+        if (nsplit > 1) {  // a piece of a split tile: fp32 partial sums, the whole CTA tile
+          float4* dst = reinterpret_cast<float4*>(
+              part + ((static_cast<int64_t>(tail_idx) * nsplit + zpiece) * 2 + rank) * (BM * BN) +
+              (h * UM + quad * 32 + lane) * BN + col);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dst[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                 __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+        } else if (m < M && n < Nout) {
           uint4* dst = reinterpret_cast<uint4*>(out + static_cast<int64_t>(m) * Nout + n);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -421,6 +456,50 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+// Sum of the split pieces of the last sg.ntail tiles in piece order (fp32),
+// rounded once to bf16.  Thread: 8 consecutive outputs of one token row.
+// Waits for the GEMM grid (programmatic dependent launch) before reading.
+__global__ void __launch_bounds__(256) k_split_reduce(const float* __restrict__ part, SplitGrid sg, int band_pairs,
+                                                      int M, int Nout, __nv_bfloat16* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
+  const int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int per_tile = 2 * BM * (BN / 8);  // 512 rows x 32 groups of 8 outputs
+  const int t = static_cast<int>(g / per_tile), w = static_cast<int>(g - static_cast<int64_t>(t) * per_tile);
+  if (t >= sg.ntail) return;
+  const int row = w / (BN / 8), c8 = (w - row * (BN / 8)) * 8;  // row of the pair tile, first column
+  const int L = sg.nwhole + t;
+  const int per_band = band_pairs * sg.nout_tiles;
+  const int band = L / per_band, rem = L - band * per_band;
+  const int in_band = min(band_pairs, sg.npairs - band * band_pairs);
+  const int otile = rem / in_band, pair = band * band_pairs + (rem - otile * in_band);
+  const int m = pair * 2 * BM + row, n = otile * BN + c8;
+  if (m >= M || n >= Nout) return;
+  // the partial of piece z: [z][rank = row / 256][row % 256][col]
+  const float* src = part + static_cast<int64_t>(t) * sg.nsplit * 2 * (BM * BN) + (row / BM) * (BM * BN) +
+                     (row % BM) * BN + c8;
+  float4 a = *reinterpret_cast<const float4*>(src), b = *reinterpret_cast<const float4*>(src + 4);
+  for (int z = 1; z < sg.nsplit; ++z) {
+    const float* q = src + static_cast<int64_t>(z) * 2 * (BM * BN);
+    const float4 c = *reinterpret_cast<const float4*>(q), d = *reinterpret_cast<const float4*>(q + 4);
+    a.x += c.x; a.y += c.y; a.z += c.z; a.w += c.w;
+    b.x += d.x; b.y += d.y; b.z += d.z; b.w += d.w;
+  }
+  uint4 o;
+  o.x = bf16x2_bits(a.x, a.y);
+  o.y = bf16x2_bits(a.z, a.w);
+  o.z = bf16x2_bits(b.x, b.y);
+  o.w = bf16x2_bits(b.z, b.w);
+  if (n + 8 <= Nout) {
+    *reinterpret_cast<uint4*>(out + static_cast<int64_t>(m) * Nout + n) = o;
+  } else {  // ragged last columns (Nout % 8 == 0 keeps this branch unused for valid shapes)
+    const uint32_t wv[4] = {o.x, o.y, o.z, o.w};
+    for (int i = 0; i < 8 && n + i < Nout; ++i)
+      reinterpret_cast<uint16_t*>(out)[static_cast<int64_t>(m) * Nout + n + i] =
+          static_cast<uint16_t>(wv[i / 2] >> (16 * (i & 1)));
+  }
+}
+
 // ------------------------------------------------------------ host side
 
 template <int MODE, bool GEN>
@@ -449,12 +528,20 @@ cudaError_t launch_mode(const GemmArgs& a, cudaStream_t st) {
 
   // Token tiles are rounded up to whole pairs: a CTA past the last token
   // feeds zeros (TMA fills out-of-range rows) to its half and stores nothing.
-  const int64_t mt = (a.M + BM - 1) / BM;
-  const int64_t npairs = (mt + 1) / 2;
-  const dim3 grid(static_cast<unsigned>(2 * npairs), static_cast<unsigned>((Nout + BN - 1) / BN));
+  const SplitPlan plan = gemm_split_plan(MODE, a.M, a.N, a.K);
+  const bool split = plan.nsplit > 1 && a.part && a.part_bytes >= plan.part_bytes;
+  SplitGrid sg;
+  sg.npairs = static_cast<int>(plan.npairs);
+  sg.nout_tiles = static_cast<int>(plan.nout_tiles);
+  sg.nwhole = static_cast<int>(split ? plan.nwhole : plan.npairs * plan.nout_tiles);
+  sg.ntail = split ? static_cast<int>(plan.ntail) : 0;
+  sg.nsplit = split ? plan.nsplit : 1;
+  const int64_t items = int64_t(sg.nwhole) + int64_t(sg.ntail) * sg.nsplit;
+  const dim3 grid(static_cast<unsigned>(2 * items), 1, 1);
   // token pairs per band: keep a band's activations (512 tokens x Kc per pair) near 48 MB
   const int64_t pair_bytes = int64_t(2) * BM * Kc * 2;
-  const int band_pairs = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(npairs, (48ll << 20) / pair_bytes)));
+  const int band_pairs =
+      static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(plan.npairs, (48ll << 20) / pair_bytes)));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
@@ -472,8 +559,15 @@ cudaError_t launch_mode(const GemmArgs& a, cudaStream_t st) {
   trace_before(st);
   e = cudaLaunchKernelEx(&cfg, k_nf4_gemm<MODE, GEN>, tm_act, tm_codes, tm_ta, tm_tb, a.absmax_q, a.dq_scale,
                          host_codebook().levels, static_cast<int>(a.M), static_cast<int>(a.N), static_cast<int>(a.K),
-                         a.r, band_pairs, lg, a.dq_block ? 1 : 0, reinterpret_cast<__nv_bfloat16*>(a.out), device_status_ptr());
-  trace_after(st);
+                         a.r, band_pairs, lg, a.dq_block ? 1 : 0, reinterpret_cast<__nv_bfloat16*>(a.out),
+                         device_status_ptr(), sg, split ? a.part : nullptr);
+  if (e == cudaSuccess && split) {
+    const int64_t threads = int64_t(sg.ntail) * 2 * BM * (BN / 8);
+    e = launch_ex(k_split_reduce, dim3(static_cast<unsigned>((threads + 255) / 256)), dim3(256), 0, st, true,
+                  static_cast<const float*>(a.part), sg, band_pairs, static_cast<int>(a.M), static_cast<int>(Nout),
+                  reinterpret_cast<__nv_bfloat16*>(a.out));
+  }
+  trace_after(st);  // the traced interval covers the reduction of split tiles too
   return e;
 }
 
@@ -536,5 +630,51 @@ cudaError_t launch_nf4_gemm(const GemmArgs& a, cudaStream_t st) {
 }
 
 int nf4_gemm_max_active_pairs(int mode) { return mode == 0 ? max_active_pairs<0>() : max_active_pairs<1>(); }
+
+// Resident CTA pairs of the current device (cached per device and mode; 0
+// when unknown, e.g. without a device).
+static int resident_pairs_cached(int mode) {
+  constexpr int kDev = 64;
+  static std::atomic<int> cache[kDev][2];  // 0: not yet asked; -1: unknown
+  int d = -1;
+  if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kDev) {
+    cudaGetLastError();
+    return 0;
+  }
+  int v = cache[d][mode].load(std::memory_order_relaxed);
+  if (v == 0) {
+    v = nf4_gemm_max_active_pairs(mode);
+    if (v <= 0) {
+      cudaGetLastError();
+      v = -1;
+    }
+    cache[d][mode].store(v, std::memory_order_relaxed);
+  }
+  return v > 0 ? v : 0;
+}
+
+SplitPlan gemm_split_plan(int mode, int64_t M, int64_t N, int64_t K) {
+  SplitPlan p{};
+  const int64_t Kc = mode == 0 ? K : N, Nout = mode == 0 ? N : K;
+  p.npairs = ((M + BM - 1) / BM + 1) / 2;
+  p.nout_tiles = (Nout + BN - 1) / BN;
+  const int64_t tiles = p.npairs * p.nout_tiles, numK = (Kc + BK - 1) / BK;
+  p.nwhole = tiles;
+  p.nsplit = 1;
+  const int P = resident_pairs_cached(mode);
+  if (P <= 0 || M <= 0) return p;
+  const int64_t w = tiles % P;  // tiles of the partial last wave
+  if (w == 0) return p;
+  // a piece keeps at least 16 K stages: shorter pieces lose more to the
+  // tile's set-up and epilogue than the split gains (measured on the dX of a
+  // 1024-output projection, 16 stages per tile: split in two it ran 11 % slower)
+  const int64_t S = std::min<int64_t>({P / w, numK / 16, 16});
+  if (S < 2) return p;
+  p.nsplit = static_cast<int>(S);
+  p.ntail = w;
+  p.nwhole = tiles - w;
+  p.part_bytes = static_cast<size_t>(w * S) * 2 * BM * BN * 4;
+  return p;
+}
 
 }  // namespace qn

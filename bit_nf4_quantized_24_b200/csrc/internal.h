@@ -71,8 +71,20 @@ struct GemmArgs {
   bool pdl;       // launched right after another kernel of the layer (programmatic dependent launch)
   int block = 64;       // NF4 format: weights per block (32, 64, 128, 256)
   int dq_block = 256;   // 256: double quantization; 0: fp32 absmax per block in dq_scale
+  float* part = nullptr;  // room for the split tiles' fp32 partial sums (nullable: no split)
+  size_t part_bytes = 0;
 };
 cudaError_t launch_nf4_gemm(const GemmArgs& a, cudaStream_t st);
+// How a launch of the fused GEMM divides its tiles on the current device: the
+// tiles that would form a partial last wave on the resident CTA pairs are
+// split along K into nsplit pieces each (fp32 partial sums, part_bytes of
+// them, summed in piece order by a second kernel).  nsplit = 1: no split.
+struct SplitPlan {
+  int64_t npairs = 0, nout_tiles = 0, nwhole = 0, ntail = 0;
+  int nsplit = 1;
+  size_t part_bytes = 0;
+};
+SplitPlan gemm_split_plan(int mode, int64_t M, int64_t N, int64_t K);
 // CTA pairs of the fused GEMM that fit on the current device at once
 // (negative: the occupancy query failed).
 int nf4_gemm_max_active_pairs(int mode);

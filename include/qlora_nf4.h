@@ -363,6 +363,21 @@ int qlora_trace_gemm_count(void);
  * of 0 means the kernel cannot launch on this device.  Errors: ARG, CUDA. */
 int qlora_gemm_resident_pairs(int mode);
 
+/* How the fused GEMM divides an M x N x K layer's tiles on the current device
+ * (mode 0 = forward: N outputs, contraction K; 1 = dX: K outputs, contraction
+ * N).  Tiles are 512 tokens x 256 outputs, one per CTA pair; when the tiles
+ * leave a partial last wave on the resident pairs, each of those *ntail_tiles
+ * tiles is split along the contraction into *nsplit pieces of at least 16
+ * 64-wide stages, whose fp32 partial sums (*partial_bytes in all) a second
+ * kernel adds in piece order before the one bf16 rounding.  The layer entry
+ * points split only when the caller's workspace holds the partial sums too
+ * (the workspace functions above include them); with a smaller workspace
+ * they run every tile whole.  *nsplit = 1: no split.  Without a device (or
+ * for M <= 16, which runs the decode kernel) the plan is no split.  Any
+ * output pointer may be NULL.  Errors: ARG (mode, negative sizes). */
+int qlora_gemm_split_plan(int mode, int64_t M, int64_t N, int64_t K, int* nsplit, int64_t* ntail_tiles,
+                          size_t* partial_bytes);
+
 #ifdef __cplusplus
 }
 #endif

@@ -11,6 +11,7 @@ checked in full; the five workloads are checked at full size on rows sampled
 from every 256-token tile (plus the last, ragged row) of Y and dX and on all of
 dA and dB, with the same launches the benchmark times.
 """
+import ctypes
 import math
 
 import numpy as np
@@ -99,6 +100,49 @@ def run_bwd_check(qb, oracle, p, rows=None, q=None, Wp=None, use_saved_h=True):
     pt.assert_blocks("dA", dAg, dAr, TOL)
     pt.assert_blocks("dB", dBg, dBr, TOL)
     return errs
+
+
+@pytest.mark.parametrize("M,N,K", [(600, 2048, 2048), (1100, 2048, 3072)])
+def test_split_tiles_match_whole_tiles(qb, oracle, M, N, K):
+    """Shapes whose tiles leave a partial last wave run those tiles split along
+    the contraction (fp32 partial sums added in piece order by a second
+    kernel).  With the workspace the plan asks for, Y and dX match the oracle
+    tile by tile, repeat bit for bit, and agree with a run whose workspace has
+    no room for the partial sums (every tile whole) to fp32 summation order."""
+    r = 16
+    for mode in (0, 1):
+        ns, nt, pb = qb.gemm_split_plan(mode, M, N, K)
+        assert ns >= 2 and nt >= 1 and pb == nt * ns * 512 * 256 * 4, (mode, ns, nt, pb)
+    p = wl.draw_small(1200 + M, M, N, K, r, 2.0 * r)
+    q, Wp = quantize_both(qb, oracle, p["W"])
+    X, A, B, dY = p["X"].cuda(), p["A"].cuda(), p["B"].cuda(), p["dY"].cuda()
+    full_f = torch.empty(qb.fwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device="cuda")
+    small_f = torch.empty(full_f.numel() - qb.gemm_split_plan(0, M, N, K)[2], dtype=torch.uint8, device="cuda")
+    Y1, H = qb.qlora_linear_fwd(q, X, A, B, p["scale"], workspace=full_f)
+    Y2, _ = qb.qlora_linear_fwd(q, X, A, B, p["scale"], workspace=full_f)
+    L, P = qb.lib(), qb._ptr
+    Yw = torch.empty_like(Y1)  # a workspace without room for the partial sums (the binding would enlarge it)
+    assert L.qlora_linear_fwd(P(q.codes), P(q.absmax_q), P(q.dq_scale), N, K, P(X), M, P(A), P(B), r,
+                              ctypes.c_float(p["scale"]), P(Yw), None, P(small_f), small_f.numel(), None) == 0
+    full_b = torch.empty(qb.bwd_workspace_bytes(M, N, K, r), dtype=torch.uint8, device="cuda")
+    small_b = torch.empty(full_b.numel() - qb.gemm_split_plan(1, M, N, K)[2], dtype=torch.uint8, device="cuda")
+    dX1, _, _ = qb.qlora_linear_bwd(q, X, dY, A, B, p["scale"], H=H, workspace=full_b)
+    dX2, _, _ = qb.qlora_linear_bwd(q, X, dY, A, B, p["scale"], H=H, workspace=full_b)
+    dXw, dAw, dBw = torch.empty_like(dX1), torch.empty(r, K, dtype=torch.bfloat16, device="cuda"), \
+        torch.empty(N, r, dtype=torch.bfloat16, device="cuda")
+    assert L.qlora_linear_bwd(P(q.codes), P(q.absmax_q), P(q.dq_scale), N, K, P(X), P(dY), M, P(A), P(B), r,
+                              ctypes.c_float(p["scale"]), P(H), P(dXw), P(dAw), P(dBw), P(small_b), small_b.numel(),
+                              None) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(Y1, Y2) and torch.equal(dX1, dX2), "split tiles are not repeatable"
+    assert relfro(Y1.float().cpu().numpy(), Yw.float().cpu().numpy()) < 2e-3
+    assert relfro(dX1.float().cpu().numpy(), dXw.float().cpu().numpy()) < 2e-3
+    rows = pt.rows_every_tile(M, 1300 + M, per_tile=2)
+    Yref = oracle.linear_fwd(bits(p["X"]), Wp, bits(p["A"]), bits(p["B"]), p["scale"], rows=rows)
+    pt.assert_tiles("Y", Y1.float().cpu().numpy()[rows], Yref, rows, TOL)
+    dXr, _, _, _ = oracle.linear_bwd(bits(p["X"]), bits(p["dY"]), Wp, bits(p["A"]), bits(p["B"]), p["scale"],
+                                     rows=rows)
+    pt.assert_tiles("dX", dX1.float().cpu().numpy()[rows], dXr, rows, TOL)
 
 
 # ------------------------------------------------------------------ codec
