@@ -50,13 +50,14 @@ sys.path.insert(0, ROOT)
 METRIC = "QLoRA linear fwd+bwd TFLOP/s and NF4 weight-stream GB/s on 1 B200; % roofline"
 WORKLOAD = "layer_70b"
 
-# DRAM bytes (read + write) per fused-GEMM launch, mean over the 14 launches of
-# one step of the workload above, from one ncu capture of `bench.py --profile
-# layer` (metrics dram__bytes_read.sum, dram__bytes_write.sum; the summary and
-# the command are in profiles/layer_70b_step_launch_list.md).  Valid only for
-# the kernel source it was taken on (sha256 prefix of gemm_tc.cu); reported as
-# null otherwise.
-GEMM_TRAFFIC = {"gemm_tc_sha16": "4eff4c321b201d5f", "bytes_per_launch": 474913938}
+# DRAM bytes (read + write) per traced fused-GEMM launch (the GEMM kernel plus,
+# where its tiles are split, the reduction kernel of the partial sums), mean
+# over the 14 traced launches of one step of the workload above, from one ncu
+# capture of `bench.py --profile layer` (metrics dram__bytes_read.sum,
+# dram__bytes_write.sum; the summary and the command are in
+# profiles/layer_70b_step_launch_list.md).  Valid only for the kernel source it
+# was taken on (sha256 prefix of gemm_tc.cu); reported as null otherwise.
+GEMM_TRAFFIC = {"gemm_tc_sha16": "fa327ba0a3245d6e", "bytes_per_launch": 508793838}
 
 
 def gemm_traffic():
@@ -346,8 +347,10 @@ def run_ours(args, rank, world, local_rank):
     n_proj = len(w.projections)
     # our kernels per step (the ncu launch list shows the same): per projection,
     # forward k_rows (H) and k_nf4_gemm; backward k_rows (dH), two k_cols (dA,
-    # dB) and k_nf4_gemm (dX)
-    launches_per_step = n_proj * (2 + 4)
+    # dB) and k_nf4_gemm (dX); plus k_split_reduce after each GEMM whose tiles
+    # the split plan divides
+    launches_per_step = n_proj * (2 + 4) + sum(
+        qb.gemm_split_plan(mode, M, pr.N, pr.K)[0] > 1 for pr in w.projections for mode in (0, 1))
 
     for _ in range(args.warmup):
         layer.step(main, allreduce)

@@ -665,10 +665,27 @@ SplitPlan gemm_split_plan(int mode, int64_t M, int64_t N, int64_t K) {
   if (P <= 0 || M <= 0) return p;
   const int64_t w = tiles % P;  // tiles of the partial last wave
   if (w == 0) return p;
-  // a piece keeps at least 16 K stages: shorter pieces lose more to the
-  // tile's set-up and epilogue than the split gains (measured on the dX of a
-  // 1024-output projection, 16 stages per tile: split in two it ran 11 % slower)
-  const int64_t S = std::min<int64_t>({P / w, numK / 16, 16});
+  // Pieces of S-th of a tile run in ceil(w S / P) rounds after the whole
+  // tiles, so the tail takes ceil(w S / P) / S of a tile's numK stages
+  // instead of all of them; each piece costs its fp32 partial sums (1 MB
+  // written, then read back by the reduction), about 0.16 of a stage's time
+  // (a pair runs a 64-deep stage of a 512 x 256 tile in ~1 us at ~1.2 PFLOP/s
+  // over 74 pairs; 1 MB moves in ~0.16 us at ~6.4 TB/s).  S maximises the
+  // saving, and must save at least 5 % of a tile.  A piece keeps at least 16
+  // stages: shorter pieces lose more to the tile's set-up and epilogue than the
+  // split gains (measured on the dX of a 1024-output projection, 16 stages per
+  // tile: split in two it ran 11 % slower).
+  const int64_t smax = std::min<int64_t>(numK / 16, 16);
+  int64_t S = 1;
+  double best = 0.05 * static_cast<double>(numK);
+  for (int64_t c = 2; c <= smax; ++c) {
+    const double rounds = static_cast<double>((w * c + P - 1) / P);
+    const double save = (1.0 - rounds / static_cast<double>(c)) * static_cast<double>(numK) - 0.16 * w * c;
+    if (save > best) {
+      best = save;
+      S = c;
+    }
+  }
   if (S < 2) return p;
   p.nsplit = static_cast<int>(S);
   p.ntail = w;
