@@ -176,6 +176,14 @@ __device__ __forceinline__ void mergedF(const MergeSrc& m, const float* lv, int6
 // finite (NaN or infinity inside) is reported and not coded.  DQ: double
 // quantization of the group's absmax values (else each block's fp32 absmax is
 // stored as is).
+// Bulk copy of `bytes` (a multiple of 16) from global to this CTA's shared
+// memory, completing on the mbarrier at `bar`.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
 template <int B, bool DQ, bool MERGE>
 __global__ void __launch_bounds__(256, 3) k_quantize(const float* __restrict__ W, MergeSrc msrc, Nf4Levels levels,
                                                   int64_t nblocks, const Cell* __restrict__ cells,
@@ -287,6 +295,141 @@ __global__ void __launch_bounds__(256, 3) k_quantize(const float* __restrict__ W
     absmax_q[b0 + tid] = q;
   }
   if (tid == 0) dq_scale[g] = s2;
+  if (__syncthreads_or(bad) && tid == 0) atomicExch(nonfinite, 1);
+}
+
+// The same quantization for fp32 input in blocks of at most 64 weights, with
+// the weights staged in shared memory: a persistent CTA takes groups
+// blockIdx.x, + gridDim.x, ... and streams each as two halves of 128 blocks
+// (32 KB for 64-weight blocks) by bulk copies into two buffers, so the copy of
+// the next half is in flight while a half is coded.  Lanes read their float4s
+// with 16-byte shared loads in an order rotated by block (f ^ (block & ROT))
+// so that the eight lanes of a quarter-warp fall on distinct banks.  Every wait
+// is bounded; on expiry the CTA lets its copies land and leaves.
+template <int B, bool DQ>
+__global__ void __launch_bounds__(256, 3) k_quantize_staged(const float* __restrict__ W, int64_t nblocks,
+                                                         const Cell* __restrict__ cells, uint8_t* __restrict__ codes,
+                                                         uint8_t* __restrict__ absmax_q, float* __restrict__ dq_scale,
+                                                         int* nonfinite, int* status) {
+  constexpr int F = 4;
+  constexpr int LP = B / (4 * F);  // 2 or 4 lanes per block
+  constexpr int BPW = 32 / LP;     // blocks per warp step
+  constexpr int ROT = 8 / LP - 1;  // blocks of a quarter-warp: 8 / LP
+  constexpr int HB = kGroup / 2;   // blocks per half-group (one buffer)
+  constexpr int HV = HB * B / 4;   // float4s per buffer
+  extern __shared__ __align__(128) float4 s_w[];  // two buffers of HV float4s
+  __shared__ Cell s_cell[kCells];
+  __shared__ float s_amax[kGroup];
+  __shared__ float s_red[8];
+  __shared__ __align__(8) uint64_t s_full[2];
+  __shared__ int s_abort;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int sub = lane / LP, sl = lane % LP;
+  const int64_t ngroups = (nblocks + kGroup - 1) / kGroup;
+  const int64_t nh = 2 * ((ngroups - blockIdx.x + gridDim.x - 1) / gridDim.x);  // this CTA's halves
+  const uint32_t full0 = smem_u32(&s_full[0]), w0 = smem_u32(s_w);
+  // first block and block count of the CTA's half h
+  auto half = [&](int64_t h, int64_t& bstart) {
+    bstart = (blockIdx.x + (h >> 1) * static_cast<int64_t>(gridDim.x)) * kGroup + (h & 1) * HB;
+    const int64_t n = nblocks - bstart;
+    return static_cast<int>(n < 0 ? 0 : n < HB ? n : HB);
+  };
+  auto issue = [&](int64_t h) {  // one thread
+    int64_t bs;
+    const uint32_t bytes = static_cast<uint32_t>(half(h, bs)) * B * 4, bar = full0 + 8u * (h & 1);
+    mbar_arrive_expect_tx(bar, bytes);
+    for (uint32_t off = 0; off < bytes; off += 16384u)
+      bulk_g2s(w0 + (h & 1) * HV * 16 + off, reinterpret_cast<const uint8_t*>(W + bs * B) + off,
+               min(16384u, bytes - off), bar);
+  };
+  if (tid == 0) {
+    s_abort = 0;
+    mbar_init(full0, 1);
+    mbar_init(full0 + 8u, 1);
+    fence_mbar_init();
+    if (nh > 0) issue(0);
+    if (nh > 1) issue(1);
+  }
+  s_cell[tid] = cells[tid];  // kCells == blockDim.x
+  __syncthreads();
+  bool bad = false;
+  for (int64_t h = 0; h < nh; ++h) {
+    const uint32_t bar = full0 + 8u * (h & 1), par = static_cast<uint32_t>(h >> 1) & 1u;
+    if (!wait_bounded(bar, par, &s_abort, status)) {
+      wait_drain(bar, par);  // let the copies in flight land before the CTA leaves
+      if (h + 1 < nh) wait_drain(full0 + 8u * ((h + 1) & 1), static_cast<uint32_t>((h + 1) >> 1) & 1u);
+      return;
+    }
+    int64_t bs;
+    const int n = half(h, bs);
+    const float4* buf = s_w + (h & 1) * HV;
+    for (int p = warp; p * BPW < n; p += 8) {
+      const int i = p * BPW + sub;
+      const bool ok = i < n;
+      float4 x[F];
+#pragma unroll
+      for (int f = 0; f < F; ++f)
+        x[f] = ok ? buf[i * (B / 4) + (f ^ (sub & ROT)) * LP + sl] : make_float4(0.f, 0.f, 0.f, 0.f);
+      float m = 0.0f;
+#pragma unroll
+      for (int f = 0; f < F; ++f)
+        m = fmax_nan(m, fmax_nan(fmax_nan(fabsf(x[f].x), fabsf(x[f].y)), fmax_nan(fabsf(x[f].z), fabsf(x[f].w))));
+#pragma unroll
+      for (int off = LP / 2; off > 0; off >>= 1) m = fmax_nan(m, __shfl_xor_sync(0xffffffffu, m, off));
+      if (ok) {
+        const bool finite = m <= 3.402823466e38f;  // false for NaN and infinity
+        bad |= !finite;
+        const bool fast = m >= 0x1p-100f && m <= 0x1p100f;
+        const float r = fast ? __frcp_rn(m) : 0.0f;
+        uint16_t* dst = reinterpret_cast<uint16_t*>(codes + (bs + i) * (B / 2)) + sl;
+#pragma unroll
+        for (int f = 0; f < F; ++f) {
+          const float4 v = x[f];
+          uint32_t c;
+          if (m == 0.0f || !finite) {
+            c = 0x7777u;  // an all-zero block encodes the zero level (a non-finite one is reported)
+          } else if (fast) {
+            c = nf4_code(div_by_absmax(v.x, m, r), s_cell) | (nf4_code(div_by_absmax(v.y, m, r), s_cell) << 4) |
+                (nf4_code(div_by_absmax(v.z, m, r), s_cell) << 8) |
+                (nf4_code(div_by_absmax(v.w, m, r), s_cell) << 12);
+          } else {
+            c = nf4_code(__fdiv_rn(v.x, m), s_cell) | (nf4_code(__fdiv_rn(v.y, m), s_cell) << 4) |
+                (nf4_code(__fdiv_rn(v.z, m), s_cell) << 8) | (nf4_code(__fdiv_rn(v.w, m), s_cell) << 12);
+          }
+          dst[(f ^ (sub & ROT)) * LP] = static_cast<uint16_t>(c);
+        }
+        if (sl == 0) {
+          if (DQ)
+            s_amax[(h & 1) * HB + i] = m;
+          else
+            dq_scale[bs + i] = m;
+        }
+      }
+    }
+    __syncthreads();  // the buffer is read (and this half's maxima are in s_amax)
+    if (tid == 0 && h + 2 < nh) issue(h + 2);
+    if (DQ && (h & 1)) {  // the group is complete: double quantization of its absmax values
+      const int64_t g = blockIdx.x + (h >> 1) * static_cast<int64_t>(gridDim.x);
+      const int64_t gr = nblocks - g * kGroup;
+      const int nbg = static_cast<int>(gr < kGroup ? gr : kGroup);
+      float mg = (tid < nbg) ? s_amax[tid] : 0.0f;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mg = fmaxf(mg, __shfl_xor_sync(0xffffffffu, mg, off));
+      if (lane == 0) s_red[warp] = mg;
+      __syncthreads();
+      float c2 = s_red[0];
+#pragma unroll
+      for (int w = 1; w < 8; ++w) c2 = fmaxf(c2, s_red[w]);
+      const float s2 = (c2 > 0.0f) ? __fdiv_rn(c2, 255.0f) : 0.0f;
+      if (tid < nbg) {
+        uint8_t q = 0;
+        if (s2 != 0.0f) q = static_cast<uint8_t>(fminf(255.0f, rintf(__fdiv_rn(s_amax[tid], s2))));
+        absmax_q[g * kGroup + tid] = q;
+      }
+      if (tid == 0) dq_scale[g] = s2;
+      __syncthreads();  // s_amax and s_red are free for the next group
+    }
+  }
   if (__syncthreads_or(bad) && tid == 0) atomicExch(nonfinite, 1);
 }
 
@@ -422,7 +565,7 @@ __global__ void __launch_bounds__(256, 4) k_merge64(MergeSrc m, Nf4Levels levels
     cp_async_commit();
   };
   stage(0);
-  s_cell[tid] = cells[tid];
+  s_cell[tid] = cells[tid];  // kCells == blockDim.x
   s_lv2[tid] = pk2(levels.v[tid & 15], levels.v[tid >> 4]);
   for (int i = tid; i < r * MG_ROWS; i += 256) {
     const int j = i / MG_ROWS, row = i - j * MG_ROWS;
@@ -632,12 +775,20 @@ cudaError_t quantize_launch(const float* W, const MergeSrc* merge, int64_t numel
   cudaError_t e;
   const Cell* cells = device_cells(&e);
   if (!cells) return e;
-  if (merge)
+  if (merge) {
     k_quantize<B, DQ, true><<<static_cast<unsigned>(ngroups), 256, 0, st>>>(
         nullptr, *merge, cb.levels, nblocks, cells, codes, absmax_q, dq_scale, nonfinite);
-  else
+  } else if (B <= 64) {  // staged: two 128-block buffers, three CTAs per SM, each looping over groups
+    constexpr int smem = kGroup * (B <= 64 ? B : 64) * 4;
+    e = smem_limit_once<k_quantize_staged<B <= 64 ? B : 64, DQ>>(smem);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = std::min<int64_t>(ngroups, 3 * static_cast<int64_t>(device_sm_count()));
+    k_quantize_staged<B <= 64 ? B : 64, DQ><<<static_cast<unsigned>(grid), 256, smem, st>>>(
+        W, nblocks, cells, codes, absmax_q, dq_scale, nonfinite, device_status_ptr());
+  } else {
     k_quantize<B, DQ, false><<<static_cast<unsigned>(ngroups), 256, 0, st>>>(
         W, MergeSrc{}, cb.levels, nblocks, cells, codes, absmax_q, dq_scale, nonfinite);
+  }
   return cudaGetLastError();
 }
 
