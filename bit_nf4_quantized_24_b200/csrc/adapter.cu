@@ -137,6 +137,24 @@ __global__ void __cluster_dims__(RS_CTAS, 1, 1) __launch_bounds__(RS_WARPS * 32)
 // The adapter branch reads dropout(X) (the random draw is an input: mask,
 // 1 = keep, and keep = 1 / (1 - p)):  Xd = mask ? bf16(fl32(x * keep)) : 0.
 // Eight elements per thread (16-byte loads).
+// Xd = mask ? bf16(fl32(x * keep)) : 0 for the eight bf16 values of x, mask
+// bytes mk (nonzero = keep).  One definition for the materialised Xd and for
+// the adapter kernels that apply the mask to their X tiles in shared memory.
+__device__ __forceinline__ uint32_t dropout_pair(uint32_t xw, uint32_t mw, int sh, float keep) {
+  const float lo = ((mw >> sh) & 0xffu) ? __fmul_rn(__uint_as_float(xw << 16), keep) : 0.f;
+  const float hi = ((mw >> (sh + 8)) & 0xffu) ? __fmul_rn(__uint_as_float(xw & 0xffff0000u), keep) : 0.f;
+  return bf16x2_bits(lo, hi);
+}
+__device__ __forceinline__ uint4 dropout8(uint4 x, uint2 mk, float keep) {
+  return make_uint4(dropout_pair(x.x, mk.x, 0, keep), dropout_pair(x.y, mk.x, 16, keep),
+                    dropout_pair(x.z, mk.y, 0, keep), dropout_pair(x.w, mk.y, 16, keep));
+}
+__device__ __forceinline__ uint2 ld_shared_v2(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+
 __global__ void __launch_bounds__(256) k_dropout_input(const uint16_t* __restrict__ X,
                                                        const uint8_t* __restrict__ mask, float keep, int64_t n8,
                                                        uint16_t* __restrict__ Xd) {
@@ -146,17 +164,7 @@ __global__ void __launch_bounds__(256) k_dropout_input(const uint16_t* __restric
   if (i >= n8) return;
   const uint4 x = __ldg(reinterpret_cast<const uint4*>(X) + i);
   const uint2 mk = __ldg(reinterpret_cast<const uint2*>(mask) + i);
-  const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
-  uint32_t o[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint32_t mw = q < 2 ? mk.x : mk.y;
-    const int sh = 16 * (q & 1);
-    const float lo = ((mw >> sh) & 0xffu) ? __fmul_rn(__uint_as_float(xw[q] << 16), keep) : 0.f;
-    const float hi = ((mw >> (sh + 8)) & 0xffu) ? __fmul_rn(__uint_as_float(xw[q] & 0xffff0000u), keep) : 0.f;
-    o[q] = bf16x2_bits(lo, hi);
-  }
-  reinterpret_cast<uint4*>(Xd)[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  reinterpret_cast<uint4*>(Xd)[i] = dropout8(x, mk, keep);
 }
 
 // dX += mask * keep * (dH A): the adapter's part of the input gradient under
@@ -269,17 +277,22 @@ __global__ void __launch_bounds__(256) k_rows_multi(const uint16_t* __restrict__
 // 64-wide stages, leaves its fp32 sums in shared memory, and after a cluster
 // barrier each CTA adds one share of the outputs over the cluster's partials
 // in rank order (distributed shared memory): deterministic, no scratch.
-constexpr int RW_ST = 5;
-
-template <int NT>
+// MASK (LoRA dropout, H = Xd A^T without Xd in memory): each stage also
+// brings the (16 CW) x 64 tile of the keep mask, and each consumer warp turns
+// its 16 rows of the P tile into Xd in place before reading them (4 stages,
+// so that two CTAs still fit an SM).
+template <int NT, bool MASK = false>
 struct RowsSmem {
+  static constexpr int ST = MASK ? 4 : 5;  // stages in flight
   static constexpr int CW = NT / 2;
   static constexpr int P_BYTES = 16 * CW * 64 * 2;
   static constexpr int Q_BYTES = NT * 8 * 64 * 2;
-  static constexpr int OFF_Q = RW_ST * P_BYTES;
-  static constexpr int OFF_PART = OFF_Q + RW_ST * Q_BYTES;  // fp32 [16 CW m][NT * 8 j]
+  static constexpr int M_BYTES = MASK ? 16 * CW * 64 : 0;
+  static constexpr int OFF_Q = ST * P_BYTES;
+  static constexpr int OFF_M = OFF_Q + ST * Q_BYTES;
+  static constexpr int OFF_PART = OFF_M + ST * M_BYTES;  // fp32 [16 CW m][NT * 8 j]
   static constexpr int OFF_BAR = OFF_PART + 16 * CW * NT * 8 * 4;
-  static constexpr int BYTES = OFF_BAR + 2 * RW_ST * 8 + 1024;
+  static constexpr int BYTES = OFF_BAR + 2 * ST * 8 + 1024;
 };
 
 // The cluster's reduction of k_rows with a split contraction: every thread of
@@ -313,13 +326,16 @@ __device__ __forceinline__ void rows_reduce(uint32_t part, int M, int R, int m0,
   cluster_sync_all();  // peers keep their shared memory until every read is done
 }
 
-template <int NT, bool QT>
+template <int NT, bool QT, bool MASK>
 __global__ void __launch_bounds__(32 * (NT / 2 + 1)) k_rows(const __grid_constant__ CUtensorMap tmP,
-                                                            const __grid_constant__ CUtensorMap tmQ, int M, int Kc,
-                                                            int R, float sa, uint16_t* __restrict__ out16a, float sb,
+                                                            const __grid_constant__ CUtensorMap tmQ,
+                                                            const __grid_constant__ CUtensorMap tmM, float keep,
+                                                            int M, int Kc, int R, float sa,
+                                                            uint16_t* __restrict__ out16a, float sb,
                                                             uint16_t* __restrict__ out16b, float* __restrict__ out32,
                                                             int nsplit, int* status) {
-  using S = RowsSmem<NT>;
+  using S = RowsSmem<NT, MASK>;
+  constexpr int RW_ST = S::ST;
   constexpr int CW = S::CW;
   constexpr int RJ = NT * 8;  // j extent of the partial buffer
   pdl_trigger();
@@ -351,9 +367,10 @@ __global__ void __launch_bounds__(32 * (NT / 2 + 1)) k_rows(const __grid_constan
       for (int it = 0; it < nk; ++it) {
         const int s = it % RW_ST;
         if (!wait_bounded(empty0 + 8u * s, ((it / RW_ST) & 1) ^ 1, &abort_flag, status)) break;
-        mbar_arrive_expect_tx(full0 + 8u * s, S::P_BYTES + S::Q_BYTES);
+        mbar_arrive_expect_tx(full0 + 8u * s, S::P_BYTES + S::Q_BYTES + S::M_BYTES);
         const int kx = (it0 + it) * 64;
         tma_load_2d(base + s * S::P_BYTES, &tmP, full0 + 8u * s, kx, m0);
+        if (MASK) tma_load_2d(base + S::OFF_M + s * S::M_BYTES, &tmM, full0 + 8u * s, kx, m0);
         if (QT)
           tma_load_2d(base + S::OFF_Q + s * S::Q_BYTES, &tmQ, full0 + 8u * s, 0, kx);
         else
@@ -377,6 +394,17 @@ __global__ void __launch_bounds__(32 * (NT / 2 + 1)) k_rows(const __grid_constan
     if (!wait_bounded(full0 + 8u * s, (it / RW_ST) & 1, &abort_flag, status)) break;
     const uint32_t pt = base + s * S::P_BYTES;
     const uint32_t qt = base + S::OFF_Q + s * S::Q_BYTES;
+    if (MASK) {  // this warp's 16 rows of the tile become Xd (16-byte chunks, 128-byte swizzle)
+      const uint32_t mt = base + S::OFF_M + s * S::M_BYTES;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int ci = lane + 32 * u, row = 16 * warp + (ci >> 3), lc = ci & 7;
+        const uint32_t xa = pt + row * 128 + ((lc ^ (row & 7)) << 4);
+        const uint4 y = dropout8(ld_shared_v4(xa), ld_shared_v2(mt + row * 64 + lc * 8), keep);
+        st_shared_v4(xa, y.x, y.y, y.z, y.w);
+      }
+      __syncwarp();
+    }
 #pragma unroll
     for (int k16 = 0; k16 < 4; ++k16) {
       // A: (rows 0-7, k 0-7), (rows 8-15, k 0-7), (rows 0-7, k 8-15), (rows 8-15, k 8-15)
@@ -455,28 +483,34 @@ __global__ void __launch_bounds__(32 * (NT / 2 + 1)) k_rows(const __grid_constan
 // deterministic.  Rows past M and columns past C arrive as zeros from TMA.
 constexpr int CL_SPLIT_MAX = 8;  // portable cluster size
 
-template <int NT, int CB>
+// MASK (LoRA dropout, dA = dH^T Xd without Xd in memory): each stage also
+// brings the 32 x 64 CB tile of the keep mask, and each consumer warp turns
+// its columns of the P tile into Xd in place before reading them.
+template <int NT, int CB, bool MASK = false>
 struct ColsCfg {
   static constexpr int MT = CB == 1 ? 1 : 2;          // 16-column MMA tiles per consumer warp
   static constexpr int CWC = CB * 4 / MT;             // consumer warps
   static constexpr int THREADS = 32 * (CWC + 1);
-  static constexpr int ST = CB == 1 ? 8 : 4;          // ring stages
+  static constexpr int ST = CB == 1 ? 8 : MASK ? 3 : 4;  // ring stages (two CTAs fit an SM)
   static constexpr int P_BYTES = CB * 32 * 64 * 2;    // CB boxes of 32 tokens x 64 columns
   static constexpr int G_BYTES = 32 * NT * 8 * 2;
+  static constexpr int M_BYTES = MASK ? 32 * 64 * CB : 0;
   static constexpr int OFF_G = ST * P_BYTES;
-  static constexpr int RING = OFF_G + ST * G_BYTES;
+  static constexpr int OFF_M = OFF_G + ST * G_BYTES;
+  static constexpr int RING = OFF_M + ST * M_BYTES;
   static constexpr int PART = CB * 64 * NT * 8 * 4;   // fp32 [64 CB c][NT * 8 j], over the ring
   static constexpr int OFF_BAR = RING > PART ? RING : PART;
   static constexpr int BYTES = OFF_BAR + 2 * ST * 8 + 1024;
 };
 
-template <int NT, int CB>
-__global__ void __launch_bounds__(ColsCfg<NT, CB>::THREADS) k_cols(const __grid_constant__ CUtensorMap tmP,
-                                                                  const __grid_constant__ CUtensorMap tmG, int M,
-                                                                  int C, int R, int rows_per_split, float scale,
-                                                                  int transpose, uint16_t* __restrict__ out,
-                                                                  int* status) {
-  using S = ColsCfg<NT, CB>;
+template <int NT, int CB, bool MASK>
+__global__ void __launch_bounds__(ColsCfg<NT, CB, MASK>::THREADS) k_cols(const __grid_constant__ CUtensorMap tmP,
+                                                                        const __grid_constant__ CUtensorMap tmG,
+                                                                        const __grid_constant__ CUtensorMap tmM,
+                                                                        float keep, int M, int C, int R,
+                                                                        int rows_per_split, float scale, int transpose,
+                                                                        uint16_t* __restrict__ out, int* status) {
+  using S = ColsCfg<NT, CB, MASK>;
   constexpr int RJ = NT * 8;  // j extent of the partial buffer
   constexpr int MT = S::MT, CWC = S::CWC, ST = S::ST;
   pdl_trigger();
@@ -511,11 +545,12 @@ __global__ void __launch_bounds__(ColsCfg<NT, CB>::THREADS) k_cols(const __grid_
       for (int it = 0; it < nslab; ++it) {
         const int s = it % ST;
         if (!wait_bounded(empty0 + 8u * s, ((it / ST) & 1) ^ 1, &abort_flag, status)) break;
-        mbar_arrive_expect_tx(full0 + 8u * s, S::P_BYTES + S::G_BYTES);
+        mbar_arrive_expect_tx(full0 + 8u * s, S::P_BYTES + S::G_BYTES + S::M_BYTES);
 #pragma unroll
         for (int b = 0; b < CB; ++b)
           tma_load_2d(base + s * S::P_BYTES + b * 4096, &tmP, full0 + 8u * s, c0 + 64 * b, mb0 + 32 * it);
         tma_load_2d(base + S::OFF_G + s * S::G_BYTES, &tmG, full0 + 8u * s, 0, mb0 + 32 * it);
+        if (MASK) tma_load_2d(base + S::OFF_M + s * S::M_BYTES, &tmM, full0 + 8u * s, c0, mb0 + 32 * it);
         ++issued;
       }
       for (int it = (issued > ST ? issued - ST : 0); it < issued; ++it)
@@ -536,6 +571,18 @@ __global__ void __launch_bounds__(ColsCfg<NT, CB>::THREADS) k_cols(const __grid_
       if (!wait_bounded(full0 + 8u * s, (it / ST) & 1, &abort_flag, status)) break;
       const uint32_t pt = base + s * S::P_BYTES + box_off;
       const uint32_t gt = base + S::OFF_G + s * S::G_BYTES;
+      if (MASK) {  // this warp's 16 MT columns of the 32 tokens become Xd (128-byte swizzled box)
+        constexpr int CPR = 2 * MT;  // 16-byte chunks of a token row in this warp's columns
+        const uint32_t mt = base + S::OFF_M + s * S::M_BYTES;
+#pragma unroll
+        for (int u = 0; u < CPR; ++u) {
+          const int ci = lane + 32 * u, row = ci / CPR, cc = ci % CPR, lc = cchunk0 + cc;
+          const uint32_t xa = pt + row * 128 + ((lc ^ (row & 7)) << 4);
+          const uint4 y = dropout8(ld_shared_v4(xa), ld_shared_v2(mt + row * (64 * CB) + cw0 + 8 * cc), keep);
+          st_shared_v4(xa, y.x, y.y, y.z, y.w);
+        }
+        __syncwarp();
+      }
 #pragma unroll
       for (int ks = 0; ks < 2; ++ks) {
         uint32_t a[MT][4];  // P^T per 16 columns: (c 0-7, m 0-7), (c 8-15, m 0-7), (c 0-7, m 8-15), (c 8-15, m 8-15)
@@ -620,19 +667,25 @@ int cols_splits(int64_t M) {
   return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(CL_SPLIT_MAX, (M + 255) / 256)));
 }
 
-template <int NT, bool QT>
+template <int NT, bool QT, bool MASK = false>
 cudaError_t rows_launch(const uint16_t* P, const uint16_t* Q, int64_t M, int64_t Kc, int R, float sa,
-                        uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st, bool pdl) {
-  using S = RowsSmem<NT>;
-  CUtensorMap tmP, tmQ;
+                        uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st, bool pdl,
+                        const uint8_t* mask = nullptr, float keep = 1.0f) {
+  using S = RowsSmem<NT, MASK>;
+  CUtensorMap tmP, tmQ, tmM;
   const auto BF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   bool ok = make_map(&tmP, BF16, P, Kc, M, Kc * 2, 64, 16 * S::CW, CU_TENSOR_MAP_SWIZZLE_128B);
   if (QT)
     ok = ok && make_map(&tmQ, BF16, Q, R, Kc, R * 2, NT * 8, 64, narrow_swizzle<NT>());
   else
     ok = ok && make_map(&tmQ, BF16, Q, Kc, R, Kc * 2, 64, NT * 8, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (MASK)  // keep mask u8 [M, Kc], 64-byte rows of the (16 CW) x 64 tile
+    ok = ok && make_map(&tmM, CU_TENSOR_MAP_DATA_TYPE_UINT8, mask, Kc, M, Kc, 64, 16 * S::CW,
+                        CU_TENSOR_MAP_SWIZZLE_NONE);
+  else
+    tmM = tmP;  // unused
   if (!ok) return cudaErrorInvalidValue;
-  cudaError_t e = smem_limit_once<k_rows<NT, QT>>(S::BYTES);
+  cudaError_t e = smem_limit_once<k_rows<NT, QT, MASK>>(S::BYTES);
   if (e != cudaSuccess) return e;
   const int64_t tiles = (M + 16 * S::CW - 1) / (16 * S::CW);
   // split the contraction when the token tiles give fewer than two CTAs per
@@ -661,8 +714,8 @@ cudaError_t rows_launch(const uint16_t* P, const uint16_t* Q, int64_t M, int64_t
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, k_rows<NT, QT>, tmP, tmQ, int(M), int(Kc), R, sa, out16a, sb, out16b, out32,
-                            nsplit, device_status_ptr());
+  return cudaLaunchKernelEx(&cfg, k_rows<NT, QT, MASK>, tmP, tmQ, tmM, keep, int(M), int(Kc), R, sa, out16a, sb,
+                            out16b, out32, nsplit, device_status_ptr());
 }
 
 template <bool QT>
@@ -675,16 +728,21 @@ cudaError_t rows_dispatch(const uint16_t* P, const uint16_t* Q, int64_t M, int64
   }
 }
 
-template <int NT, int CB>
+template <int NT, int CB, bool MASK = false>
 cudaError_t cols_launch_cb(const uint16_t* G, const uint16_t* P, int64_t M, int64_t C, int R, float scale,
-                           int transpose, uint16_t* out, cudaStream_t st, bool pdl) {
-  using S = ColsCfg<NT, CB>;
-  CUtensorMap tmP, tmG;
+                           int transpose, uint16_t* out, cudaStream_t st, bool pdl, const uint8_t* mask = nullptr,
+                           float keep = 1.0f) {
+  using S = ColsCfg<NT, CB, MASK>;
+  CUtensorMap tmP, tmG, tmM;
   const auto BF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   bool ok = make_map(&tmP, BF16, P, C, M, C * 2, 64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
   ok = ok && make_map(&tmG, BF16, G, R, M, R * 2, NT * 8, 32, narrow_swizzle<NT>());
+  if (MASK)  // keep mask u8 [M, C], the 32 x 64 CB tile
+    ok = ok && make_map(&tmM, CU_TENSOR_MAP_DATA_TYPE_UINT8, mask, C, M, C, 64 * CB, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+  else
+    tmM = tmP;  // unused
   if (!ok) return cudaErrorInvalidValue;
-  cudaError_t e = smem_limit_once<k_cols<NT, CB>>(S::BYTES);
+  cudaError_t e = smem_limit_once<k_cols<NT, CB, MASK>>(S::BYTES);
   if (e != cudaSuccess) return e;
   const int splits = cols_splits(M);
   // token ranges are whole 32-token slabs, so a slab never straddles two splits
@@ -703,17 +761,18 @@ cudaError_t cols_launch_cb(const uint16_t* G, const uint16_t* P, int64_t M, int6
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, k_cols<NT, CB>, tmP, tmG, int(M), int(C), R, rows_per_split, scale, transpose, out,
-                            device_status_ptr());
+  return cudaLaunchKernelEx(&cfg, k_cols<NT, CB, MASK>, tmP, tmG, tmM, keep, int(M), int(C), R, rows_per_split, scale,
+                            transpose, out, device_status_ptr());
 }
 
 // 256-column tiles when they still give most SMs a CTA, else 64-column tiles.
-template <int NT>
+template <int NT, bool MASK = false>
 cudaError_t cols_launch(const uint16_t* G, const uint16_t* P, int64_t M, int64_t C, int R, float scale,
-                        int transpose, uint16_t* out, cudaStream_t st, bool pdl) {
+                        int transpose, uint16_t* out, cudaStream_t st, bool pdl, const uint8_t* mask = nullptr,
+                        float keep = 1.0f) {
   if ((C + 255) / 256 * cols_splits(M) >= device_sm_count() * 3 / 4)
-    return cols_launch_cb<NT, 4>(G, P, M, C, R, scale, transpose, out, st, pdl);
-  return cols_launch_cb<NT, 1>(G, P, M, C, R, scale, transpose, out, st, pdl);
+    return cols_launch_cb<NT, 4, MASK>(G, P, M, C, R, scale, transpose, out, st, pdl, mask, keep);
+  return cols_launch_cb<NT, 1, MASK>(G, P, M, C, R, scale, transpose, out, st, pdl, mask, keep);
 }
 
 }  // namespace
@@ -769,6 +828,27 @@ cudaError_t launch_coldot(const uint16_t* G, const uint16_t* P, int64_t M, int64
     case 2: return cols_launch<2>(G, P, M, C, R, scale, transpose, out, st, pdl);
     case 4: return cols_launch<4>(G, P, M, C, R, scale, transpose, out, st, pdl);
     default: return cols_launch<8>(G, P, M, C, R, scale, transpose, out, st, pdl);
+  }
+}
+
+cudaError_t launch_rowdot_masked(const uint16_t* X, const uint8_t* mask, float keep, const uint16_t* Q, int64_t M,
+                                 int64_t Kc, int R, float sa, uint16_t* out16a, float sb, uint16_t* out16b,
+                                 cudaStream_t st, bool pdl) {
+  if (M <= 16) return cudaErrorInvalidValue;  // the caller materialises Xd for the small kernel
+  switch (nt_for(R)) {
+    case 2: return rows_launch<2, false, true>(X, Q, M, Kc, R, sa, out16a, sb, out16b, nullptr, st, pdl, mask, keep);
+    case 4: return rows_launch<4, false, true>(X, Q, M, Kc, R, sa, out16a, sb, out16b, nullptr, st, pdl, mask, keep);
+    default: return rows_launch<8, false, true>(X, Q, M, Kc, R, sa, out16a, sb, out16b, nullptr, st, pdl, mask, keep);
+  }
+}
+
+cudaError_t launch_coldot_masked(const uint16_t* G, const uint16_t* X, const uint8_t* mask, float keep, int64_t M,
+                                 int64_t C, int R, float scale, uint16_t* out, cudaStream_t st, bool pdl) {
+  if (M == 0) return cudaMemsetAsync(out, 0, sizeof(uint16_t) * static_cast<size_t>(R) * C, st);
+  switch (nt_for(R)) {
+    case 2: return cols_launch<2, true>(G, X, M, C, R, scale, 0, out, st, pdl, mask, keep);
+    case 4: return cols_launch<4, true>(G, X, M, C, R, scale, 0, out, st, pdl, mask, keep);
+    default: return cols_launch<8, true>(G, X, M, C, R, scale, 0, out, st, pdl, mask, keep);
   }
 }
 

@@ -99,7 +99,8 @@ DropWorkspace drop_layout(void* ws, size_t off0, int64_t M, int64_t K, int r) {
   size_t off = (off0 + 255) & ~size_t(255);
   uint8_t* p = static_cast<uint8_t*>(ws);
   w.Xd = p ? reinterpret_cast<uint16_t*>(p + off) : nullptr;
-  off += (static_cast<size_t>(M) * K * 2 + 255) & ~size_t(255);
+  // Xd [M, K] only for M <= 16 (larger M applies the mask inside the adapter kernels)
+  off += M <= 16 ? (static_cast<size_t>(M) * K * 2 + 255) & ~size_t(255) : 0;
   w.zero_tail = p ? reinterpret_cast<uint16_t*>(p + off) : nullptr;
   off += (static_cast<size_t>(M) * r * 2 + 255) & ~size_t(255);
   w.bytes = off;
@@ -542,9 +543,15 @@ int qlora_linear_fwd_dropout(const uint8_t* codes, const uint8_t* absmax_q, cons
   DropWorkspace d = drop_layout(workspace, base, M, K, r);
   if (!workspace || !aligned(workspace, 256) || workspace_bytes < d.bytes) return QLORA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // H from the dropped-out input; the base product from X itself
-  cudaError_t e = launch_dropout_input(X, keep_mask, keep_scale, M * K, d.Xd, s, true);
-  if (e == cudaSuccess) e = launch_rowdot(d.Xd, A, M, K, r, scale, w.Hs, 1.0f, H_save, nullptr, s, true);
+  // H from the dropped-out input (masked inside the H kernel; small M from a
+  // materialised Xd); the base product from X itself
+  cudaError_t e;
+  if (M > 16) {
+    e = launch_rowdot_masked(X, keep_mask, keep_scale, A, M, K, r, scale, w.Hs, 1.0f, H_save, s, true);
+  } else {
+    e = launch_dropout_input(X, keep_mask, keep_scale, M * K, d.Xd, s, true);
+    if (e == cudaSuccess) e = launch_rowdot(d.Xd, A, M, K, r, scale, w.Hs, 1.0f, H_save, nullptr, s, true);
+  }
   if (e != cudaSuccess) return cuda_status(e);
   if (M <= 16) {
     e = launch_gemv(X, M, codes, absmax_q, dq_scale, N, K, w.Hs, B, r, Y, s);
@@ -596,17 +603,24 @@ int qlora_linear_bwd_dropout(const uint8_t* codes, const uint8_t* absmax_q, cons
     if (e == cudaSuccess) e = cudaMemsetAsync(dB, 0, static_cast<size_t>(N) * r * 2, s);
     return cuda_status(e);
   }
+  const bool masked = M > 16;  // the adapter kernels apply the mask; else Xd is materialised
   if (dX) e = cudaMemsetAsync(d.zero_tail, 0, static_cast<size_t>(M) * r * 2, s);
-  if (e == cudaSuccess) e = launch_dropout_input(X, keep_mask, keep_scale, M * K, d.Xd, s, true);
+  if (e == cudaSuccess && !masked) e = launch_dropout_input(X, keep_mask, keep_scale, M * K, d.Xd, s, true);
   if (e == cudaSuccess) e = launch_rowdot_qt(dY, B, M, N, r, scale, w.dH16, scale, nullptr, nullptr, s, true);
   const uint16_t* Huse = H;
   if (e == cudaSuccess && !H) {
-    e = launch_rowdot(d.Xd, A, M, K, r, 1.0f, w.H16, 1.0f, nullptr, nullptr, s, true);
+    e = masked ? launch_rowdot_masked(X, keep_mask, keep_scale, A, M, K, r, 1.0f, w.H16, 1.0f, nullptr, s, true)
+               : launch_rowdot(d.Xd, A, M, K, r, 1.0f, w.H16, 1.0f, nullptr, nullptr, s, true);
     Huse = w.H16;
   }
-  if (e == cudaSuccess) e = launch_coldot(w.dH16, d.Xd, M, K, r, 1.0f, 0, dA, s, true);
-  if (e == cudaSuccess) e = launch_coldot(Huse, dY, M, N, r, scale, 1, dB, s, true);
-  if (e == cudaSuccess && dX) {  // dY deq(W) with a zero adapter tail, then the masked adapter term
+  // dA = dH^T Xd
+  auto run_da = [&](cudaStream_t st, bool pdl) {
+    return masked ? launch_coldot_masked(w.dH16, X, keep_mask, keep_scale, M, K, r, 1.0f, dA, st, pdl)
+                  : launch_coldot(w.dH16, d.Xd, M, K, r, 1.0f, 0, dA, st, pdl);
+  };
+  if (e != cudaSuccess) return cuda_status(e);
+  // dY deq(W) with a zero adapter tail, then the masked adapter term
+  auto run_dx = [&]() {
     GemmArgs a{};
     a.mode = 1;
     a.act = dY;
@@ -622,9 +636,28 @@ int qlora_linear_bwd_dropout(const uint8_t* codes, const uint8_t* absmax_q, cons
     a.out = dX;
     a.pdl = true;
     gemm_part(a, workspace, d.bytes, workspace_bytes);
-    e = launch_nf4_gemm(a, s);
-    if (e == cudaSuccess) e = launch_dx_add_masked(dX, w.dH16, A, keep_mask, keep_scale, M, K, r, s, true);
+    cudaError_t x = launch_nf4_gemm(a, s);
+    if (x == cudaSuccess) x = launch_dx_add_masked(dX, w.dH16, A, keep_mask, keep_scale, M, K, r, s, true);
+    return x;
+  };
+  // dA, dB beside the dX GEMM on the caller stream's side stream, as in the
+  // plain backward (joined before the call returns)
+  SideStream ss;
+  if (dX && side_stream(s, &ss)) {
+    e = cudaEventRecord(ss.fork, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ss.st, ss.fork, 0);
+    if (e != cudaSuccess) return cuda_status(e);
+    e = run_da(ss.st, false);
+    if (e == cudaSuccess) e = launch_coldot(Huse, dY, M, N, r, scale, 1, dB, ss.st, true);
+    if (e == cudaSuccess) e = run_dx();
+    // join on every path, so that nothing of this call stays unordered with `s`
+    cudaError_t j = cudaEventRecord(ss.join, ss.st);
+    if (j == cudaSuccess) j = cudaStreamWaitEvent(s, ss.join, 0);
+    return cuda_status(e != cudaSuccess ? e : j);
   }
+  e = run_da(s, true);
+  if (e == cudaSuccess) e = launch_coldot(Huse, dY, M, N, r, scale, 1, dB, s, true);
+  if (e == cudaSuccess && dX) e = run_dx();
   return cuda_status(e);
 }
 

@@ -128,6 +128,15 @@ cudaError_t launch_gemv_tiles(const uint16_t* X, int64_t M, const uint8_t* tiles
                               int block = 64, int dq_block = 256);
 // LoRA dropout: Xd = mask ? bf16(fl32(X * keep)) : 0 over n elements (n % 8 == 0,
 // 16-byte aligned); dX += mask * keep * (dH A) (see adapter.cu).
+// The adapter products on Xd = mask ? bf16(fl32(X keep)) : 0 without Xd in
+// memory: the kernels apply the mask to their X tiles in shared memory.
+// launch_rowdot_masked: out = sa/sb * Xd Q^T (Q [R, Kc]), M > 16 only.
+// launch_coldot_masked: out[j, c] = bf16(scale * sum_m G[m, j] Xd[m, c]).
+cudaError_t launch_rowdot_masked(const uint16_t* X, const uint8_t* mask, float keep, const uint16_t* Q, int64_t M,
+                                 int64_t Kc, int R, float sa, uint16_t* out16a, float sb, uint16_t* out16b,
+                                 cudaStream_t st, bool pdl);
+cudaError_t launch_coldot_masked(const uint16_t* G, const uint16_t* X, const uint8_t* mask, float keep, int64_t M,
+                                 int64_t C, int R, float scale, uint16_t* out, cudaStream_t st, bool pdl);
 cudaError_t launch_dropout_input(const uint16_t* X, const uint8_t* mask, float keep, int64_t n, uint16_t* Xd,
                                  cudaStream_t st, bool pdl);
 cudaError_t launch_dx_add_masked(uint16_t* dX, const uint16_t* dH, const uint16_t* A, const uint8_t* mask, float keep,

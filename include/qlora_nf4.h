@@ -281,9 +281,11 @@ int qlora_linear_bwd_fmt(const uint8_t* codes, const uint8_t* absmax_q, const fl
  *     Y  = X deq(W)^T + scale * (Xd A^T) B^T
  *     dX = dY deq(W) + keep_mask * keep_scale * (dH A),  dH = scale * dY B
  *     dA = dH^T Xd,  dB = scale * dY^T H,  H = Xd A^T  (H_save / H hold it).
+ * Xd is not stored for M > 16: the H and dA kernels apply the mask to the X
+ * tiles they load (for M <= 16 a small Xd sits in the workspace).
  * workspace: qlora_linear_dropout_workspace bytes (shared by both calls).
  * Shapes, format and errors as qlora_linear_fwd / qlora_linear_bwd; keep_mask
- * 16-byte aligned. */
+ * 16-byte aligned; a nonzero byte keeps. */
 int qlora_linear_dropout_workspace(int64_t M, int64_t N, int64_t K, int r, size_t* bytes);
 int qlora_linear_fwd_dropout(const uint8_t* codes, const uint8_t* absmax_q, const float* dq_scale,
                              int64_t N, int64_t K, const qlora_bf16_t* X, int64_t M,

@@ -379,6 +379,33 @@ def test_lora_dropout(qb, oracle, M):
     assert relfro(dA2.float().cpu().numpy(), rA) <= TOL
 
 
+@pytest.mark.parametrize("M,K", [(2048, 4096), (300, 1024)])
+def test_lora_dropout_mask_inside_the_adapter_kernels(qb, M, K):
+    """For M > 16 the dropout entry points apply the keep mask to the X tiles
+    inside the H and dA kernels instead of writing Xd to memory.  Their H and
+    dA equal, bit for bit, those of the plain layer run on Xd made by torch
+    (bf16(fl32(x * keep)) where kept, else 0), which the oracle tests cover;
+    (2048, 4096) takes the 256-column dA kernel, (300, 1024) the 64-column one."""
+    N, r = 512, 16
+    p = wl.draw_small(1500 + M, M, N, K, r, 32.0, b_std=0.5)
+    q = qb.nf4_quantize(p["W"].cuda())
+    g = torch.Generator().manual_seed(1600 + M)
+    mask = (torch.rand(M, K, generator=g) >= 0.1).to(torch.uint8)
+    keep = float(np.float32(1.0 / 0.9))
+    X, A, B, dY = p["X"].cuda(), p["A"].cuda(), p["B"].cuda(), p["dY"].cuda()
+    mk = mask.cuda()
+    Xd = torch.where(mk.bool(), (X.float() * keep).bfloat16(), torch.zeros_like(X))
+    _, H = qb.qlora_linear_fwd_dropout(q, X, A, B, p["scale"], mk, keep)
+    _, Hp = qb.qlora_linear_fwd(q, Xd, A, B, p["scale"])
+    _, dA, _ = qb.qlora_linear_bwd_dropout(q, X, dY, A, B, p["scale"], mk, keep, H=H, want_dx=False)
+    _, dAp, _ = qb.qlora_linear_bwd(q, Xd, dY, A, B, p["scale"], H=Hp, want_dx=False)
+    _, dA2, _ = qb.qlora_linear_bwd_dropout(q, X, dY, A, B, p["scale"], mk, keep, want_dx=False)  # H recomputed
+    torch.cuda.synchronize()
+    assert torch.equal(H, Hp), "H differs from the materialised-Xd path"
+    assert torch.equal(dA, dAp), "dA differs from the materialised-Xd path"
+    assert torch.equal(dA2, dAp), "dA (H recomputed) differs from the materialised-Xd path"
+
+
 def test_noalloc_entry_reads_default_format_only(qb):
     q = qb.nf4_quantize(torch.randn(64, 256, device="cuda") * 0.02, 128, 0)
     X = torch.randn(32, 256, device="cuda").bfloat16()
