@@ -295,6 +295,23 @@ struct RowsSmem {
   static constexpr int BYTES = OFF_BAR + 2 * ST * 8 + 1024;
 };
 
+// Sum over the cluster's ranks 0 .. n-1 (n <= 8) of the fp32 word at shared
+// address `off` of each rank, in rank order; the remote loads are all issued
+// before the first add.
+__device__ __forceinline__ float cluster_sum_ranks(uint32_t off, int n) {
+  float x[8];
+#pragma unroll
+  for (int rk = 0; rk < 8; ++rk) {
+    x[rk] = 0.f;
+    if (rk < n) asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(x[rk]) : "r"(mapa_shared(off, rk)) : "memory");
+  }
+  float sum = x[0];
+#pragma unroll
+  for (int rk = 1; rk < 8; ++rk)
+    if (rk < n) sum += x[rk];
+  return sum;
+}
+
 // The cluster's reduction of k_rows with a split contraction: every thread of
 // every CTA arrives (the producer warp too); then CTA `split` writes outputs
 // [V split / nsplit, V (split + 1) / nsplit) of the tile's V = 16 CW x R, each
@@ -310,13 +327,7 @@ __device__ __forceinline__ void rows_reduce(uint32_t part, int M, int R, int m0,
   for (int v = v0 + static_cast<int>(threadIdx.x); v < v1; v += blockDim.x) {
     const int ml = v / R, j = v - ml * R;
     const int m = m0 + ml;
-    const uint32_t off = part + (ml * RJ + j) * 4;
-    float sum = 0.f;
-    for (int rk = 0; rk < nsplit; ++rk) {
-      float x;
-      asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(x) : "r"(mapa_shared(off, rk)) : "memory");
-      sum += x;
-    }
+    const float sum = cluster_sum_ranks(part + (ml * RJ + j) * 4, nsplit);
     if (m >= M) continue;
     const int64_t o = static_cast<int64_t>(m) * R + j;
     out16a[o] = static_cast<uint16_t>(bf16x2_bits(sa * sum, 0.f));
@@ -512,6 +523,13 @@ __global__ void __launch_bounds__(ColsCfg<NT, CB, MASK>::THREADS) k_cols(const _
                                                                         uint16_t* __restrict__ out, int* status) {
   using S = ColsCfg<NT, CB, MASK>;
   constexpr int RJ = NT * 8;  // j extent of the partial buffer
+  // The partial sums sit where the cluster's reduction reads them in runs of
+  // consecutive words (a warp's remote loads then form few requests): for the
+  // transposed output (consecutive threads take consecutive j) at
+  // part[cl][j ^ pswz(cl)] (pairs j, j + 1 adjacent, the consumers' paired
+  // stores spread over banks), for the untransposed one (consecutive cl) at
+  // part[j][cl].
+  auto pswz = [](int cl) { return (cl << 1) & (RJ - 1); };
   constexpr int MT = S::MT, CWC = S::CWC, ST = S::ST;
   pdl_trigger();
   pdl_wait();
@@ -622,9 +640,17 @@ __global__ void __launch_bounds__(ColsCfg<NT, CB, MASK>::THREADS) k_cols(const _
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int cl = warp * 16 * MT + mt * 16 + g + 8 * h, j = nt * 8 + 2 * t;
-          asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(part + (cl * RJ + j) * 4), "f"(acc[mt][nt][2 * h]),
-                       "f"(acc[mt][nt][2 * h + 1])
-                       : "memory");
+          if (transpose) {
+            asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(part + (cl * RJ + (j ^ pswz(cl))) * 4),
+                         "f"(acc[mt][nt][2 * h]), "f"(acc[mt][nt][2 * h + 1])
+                         : "memory");
+          } else {
+            asm volatile("st.shared.f32 [%0], %1;" ::"r"(part + (j * (64 * CB) + cl) * 4), "f"(acc[mt][nt][2 * h])
+                         : "memory");
+            asm volatile("st.shared.f32 [%0], %1;" ::"r"(part + ((j + 1) * (64 * CB) + cl) * 4),
+                         "f"(acc[mt][nt][2 * h + 1])
+                         : "memory");
+          }
         }
   }
   cluster_sync_all();  // every CTA's partial sums are in its shared memory
@@ -646,13 +672,8 @@ __global__ void __launch_bounds__(ColsCfg<NT, CB, MASK>::THREADS) k_cols(const _
     }
     const int c = c0 + cl;
     if (c >= C) continue;
-    const uint32_t off = part + (cl * RJ + j) * 4;
-    float sum = 0.f;
-    for (uint32_t rk = 0; rk < nsplit; ++rk) {
-      float x;
-      asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(x) : "r"(mapa_shared(off, rk)) : "memory");
-      sum += x;
-    }
+    const uint32_t off = transpose ? part + (cl * RJ + (j ^ pswz(cl))) * 4 : part + (j * (64 * CB) + cl) * 4;
+    const float sum = cluster_sum_ranks(off, static_cast<int>(nsplit));
     const int64_t o = transpose ? static_cast<int64_t>(c) * R + j : static_cast<int64_t>(j) * C + c;
     out[o] = static_cast<uint16_t>(bf16x2_bits(scale * sum, 0.f));
   }
