@@ -57,7 +57,7 @@ WORKLOAD = "layer_70b"
 # dram__bytes_write.sum; the summary and the command are in
 # profiles/layer_70b_step_launch_list.md).  Valid only for the kernel source it
 # was taken on (sha256 prefix of gemm_tc.cu); reported as null otherwise.
-GEMM_TRAFFIC = {"gemm_tc_sha16": "fa327ba0a3245d6e", "bytes_per_launch": 508793838}
+GEMM_TRAFFIC = {"gemm_tc_sha16": "fa327ba0a3245d6e", "bytes_per_launch": 509335351}
 
 
 def gemm_traffic():
@@ -837,6 +837,8 @@ def run_profile(args):
             qb.nf4_quantize(p["W"].to(dev))
         if args.profile == "dequantize":
             qb.nf4_dequantize(q)
+        if args.profile == "merge":  # the weight merged with its adapter and quantized again
+            qb.nf4_merge_lora(q, A, B, p["scale"])
     torch.cuda.synchronize()
     assert qb.device_status() == 0
     print(f"profile {args.profile} {args.workload}[{args.proj}] M={p['M']} N={p['N']} K={p['K']} done")
@@ -852,7 +854,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--cpu-tokens", type=int, default=128,
                     help="token rows of the layer in the CPU oracle's bounded sample")
-    ap.add_argument("--profile", choices=["layer", "fwd", "fwd_tiles", "bwd", "step", "quantize", "dequantize"],
+    ap.add_argument("--profile", choices=["layer", "fwd", "fwd_tiles", "bwd", "step", "quantize", "dequantize", "merge"],
                     help="run only warmup+steps launches of one entry point (for ncu)")
     ap.add_argument("--workload", default="qproj_7b", help="workload for --profile (other than layer)")
     ap.add_argument("--tokens", type=int, default=0, help="token count for --profile (default: the workload's)")
