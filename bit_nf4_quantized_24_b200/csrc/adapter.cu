@@ -267,10 +267,12 @@ __global__ void __launch_bounds__(256) k_rows_multi(const uint16_t* __restrict__
 //
 // out[m, j] = sum_k P[m, k] Q(j, k) for 16 * CW tokens per CTA.  P is bf16
 // [M, Kc]; Q is either [R, Kc] (QT = false: A) or [Kc, R] (QT = true: lora_B,
-// read in place for dH = dY B).  CW = NT / 2 consumer warps (16 tokens each)
-// run ldmatrix + m16n8k16, the last warp's lane 0 produces: per stage a
+// read in place for dH = dY B).  Two groups of CW = NT / 2 consumer warps (16
+// tokens each) take alternate stages and run ldmatrix + m16n8k16 (the second
+// group doubles the warps that hide the MMA latency), the last warp's lane 0
+// produces: per stage a
 // (16 CW) x 64 tile of P (128-byte swizzle) and the 64-wide slice of Q (as
-// many bytes as the P tile, so Q costs no more L2 traffic than P), RW_ST
+// many bytes as the P tile, so Q costs no more L2 traffic than P), four
 // stages in flight.  When the token tiles alone do not fill the GPU, the
 // contraction is split too: a cluster of `nsplit` CTAs (consecutive along
 // grid x) shares a token tile, each CTA takes a contiguous range of the
@@ -279,11 +281,15 @@ __global__ void __launch_bounds__(256) k_rows_multi(const uint16_t* __restrict__
 // in rank order (distributed shared memory): deterministic, no scratch.
 // MASK (LoRA dropout, H = Xd A^T without Xd in memory): each stage also
 // brings the (16 CW) x 64 tile of the keep mask, and each consumer warp turns
-// its 16 rows of the P tile into Xd in place before reading them (4 stages,
-// so that two CTAs still fit an SM).
+// its 16 rows of the P tile into Xd in place before reading them.
 template <int NT, bool MASK = false>
 struct RowsSmem {
-  static constexpr int ST = MASK ? 4 : 5;  // stages in flight
+  // stages in flight; even, so that every slot of the ring belongs to one
+  // consumer group (stage it goes to slot it % ST and group it % 2): a group
+  // then uses its slots in order and can never wait on a slot two phases
+  // ahead of the one it last released (an mbarrier parity cannot tell those
+  // apart)
+  static constexpr int ST = 4;
   static constexpr int CW = NT / 2;
   static constexpr int P_BYTES = 16 * CW * 64 * 2;
   static constexpr int Q_BYTES = NT * 8 * 64 * 2;
@@ -338,7 +344,7 @@ __device__ __forceinline__ void rows_reduce(uint32_t part, int M, int R, int m0,
 }
 
 template <int NT, bool QT, bool MASK>
-__global__ void __launch_bounds__(32 * (NT / 2 + 1)) k_rows(const __grid_constant__ CUtensorMap tmP,
+__global__ void __launch_bounds__(32 * (NT + 1)) k_rows(const __grid_constant__ CUtensorMap tmP,
                                                             const __grid_constant__ CUtensorMap tmQ,
                                                             const __grid_constant__ CUtensorMap tmM, float keep,
                                                             int M, int Kc, int R, float sa,
@@ -372,7 +378,7 @@ __global__ void __launch_bounds__(32 * (NT / 2 + 1)) k_rows(const __grid_constan
   }
   __syncthreads();
 
-  if (warp == CW) {  // producer
+  if (warp == 2 * CW) {  // producer
     if (lane == 0) {
       int issued = 0;
       for (int it = 0; it < nk; ++it) {
@@ -396,11 +402,14 @@ __global__ void __launch_bounds__(32 * (NT / 2 + 1)) k_rows(const __grid_constan
     return;
   }
 
+  // Two groups of CW consumer warps take alternate stages (group grp the
+  // stages it with it % 2 == grp); warp rw of a group owns rows 16 rw .. +15.
+  const int rw = warp % CW, grp = warp / CW;
   float acc[NT][4];
 #pragma unroll
   for (int i = 0; i < NT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
   const int q = lane >> 3, l7 = lane & 7;
-  for (int it = 0; it < nk; ++it) {
+  for (int it = grp; it < nk; it += 2) {
     const int s = it % RW_ST;
     if (!wait_bounded(full0 + 8u * s, (it / RW_ST) & 1, &abort_flag, status)) break;
     const uint32_t pt = base + s * S::P_BYTES;
@@ -409,7 +418,7 @@ __global__ void __launch_bounds__(32 * (NT / 2 + 1)) k_rows(const __grid_constan
       const uint32_t mt = base + S::OFF_M + s * S::M_BYTES;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int ci = lane + 32 * u, row = 16 * warp + (ci >> 3), lc = ci & 7;
+        const int ci = lane + 32 * u, row = 16 * rw + (ci >> 3), lc = ci & 7;
         const uint32_t xa = pt + row * 128 + ((lc ^ (row & 7)) << 4);
         const uint4 y = dropout8(ld_shared_v4(xa), ld_shared_v2(mt + row * 64 + lc * 8), keep);
         st_shared_v4(xa, y.x, y.y, y.z, y.w);
@@ -421,7 +430,7 @@ __global__ void __launch_bounds__(32 * (NT / 2 + 1)) k_rows(const __grid_constan
       // A: (rows 0-7, k 0-7), (rows 8-15, k 0-7), (rows 0-7, k 8-15), (rows 8-15, k 8-15)
       uint32_t a0, a1, a2, a3;
       {
-        const int row = 16 * warp + l7 + (q & 1) * 8, chunk = 2 * k16 + (q >> 1);
+        const int row = 16 * rw + l7 + (q & 1) * 8, chunk = 2 * k16 + (q >> 1);
         ldsm_x4(pt + row * 128 + ((chunk ^ (row & 7)) << 4), a0, a1, a2, a3);
       }
 #pragma unroll
@@ -446,25 +455,51 @@ __global__ void __launch_bounds__(32 * (NT / 2 + 1)) k_rows(const __grid_constan
   }
 
   const int g = lane >> 2, t = lane & 3;
-  if (nsplit > 1) {  // this CTA's partial sums part[m_local][j], then the cluster's reduction
+  // The groups' sums meet in part[m_local][j]: group 1 leaves its sums there,
+  // group 0 adds them to its own (stage order does not matter for a sum of
+  // disjoint stages, and the pairing is fixed, so the result is deterministic).
+  auto part_addr = [&](int nt, int h) { return part + ((16 * rw + g + 8 * h) * RJ + nt * 8 + 2 * t) * 4; };
+  if (grp == 1) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(part_addr(nt, h)), "f"(acc[nt][2 * h]),
+                     "f"(acc[nt][2 * h + 1])
+                     : "memory");
+  }
+  asm volatile("bar.sync 1, %0;" ::"r"(2 * CW * 32) : "memory");  // the consumer warps only
+  if (grp == 0) {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int ml = 16 * warp + g + 8 * h, j = nt * 8 + 2 * t;
-        asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(part + (ml * RJ + j) * 4), "f"(acc[nt][2 * h]),
-                     "f"(acc[nt][2 * h + 1])
-                     : "memory");
+        float2 o;
+        asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(o.x), "=f"(o.y) : "r"(part_addr(nt, h)) : "memory");
+        acc[nt][2 * h] += o.x;
+        acc[nt][2 * h + 1] += o.y;
       }
+  }
+  if (nsplit > 1) {  // this CTA's sums part[m_local][j], then the cluster's reduction
+    if (grp == 0) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(part_addr(nt, h)), "f"(acc[nt][2 * h]),
+                       "f"(acc[nt][2 * h + 1])
+                       : "memory");
+    }
     __syncwarp();
     rows_reduce<NT, CW>(part, M, R, m0, split, nsplit, sa, out16a, sb, out16b, out32);
     return;
   }
+  if (grp == 1) return;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const int m = m0 + 16 * warp + g + 8 * h;
+      const int m = m0 + 16 * rw + g + 8 * h;
       const int j = nt * 8 + 2 * t;
       if (m >= M || j >= R) continue;
       const float v0 = acc[nt][2 * h], v1 = acc[nt][2 * h + 1];
@@ -716,7 +751,7 @@ cudaError_t rows_launch(const uint16_t* P, const uint16_t* Q, int64_t M, int64_t
   const int nsplit = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({8, want, nk / 4})));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(tiles * nsplit), 1, 1);
-  cfg.blockDim = dim3(32 * (S::CW + 1), 1, 1);
+  cfg.blockDim = dim3(32 * (2 * S::CW + 1), 1, 1);
   cfg.dynamicSmemBytes = S::BYTES;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
