@@ -511,6 +511,186 @@ __global__ void __launch_bounds__(32 * (NT + 1)) k_rows(const __grid_constant__ 
   }
 }
 
+// ---------------------------------------------------- rows on tcgen05, r = 64
+//
+// The same products for r = 64 on the 5th-generation tensor cores: with
+// r = 64 each token row of X (or dY) meets 64 outputs, 64 FLOP per byte
+// streamed, more than mma.sync sustains at HBM speed.  A CTA owns 128 tokens
+// (the UMMA M) and a contiguous range of the 64-wide K stages; warp 0's lane 0
+// streams the 128 x 64 tile of X and the 64 x 64 tile of A (K-major) or of B
+// (QT: [Kc, 64] read in place, MN-major) through an RT_ST-deep TMA ring;
+// warp 1 allocates 64 TMEM columns and its lane 0 issues
+// tcgen05.mma.cta_group::1 (M = 128, N = 64, K = 16, four per stage) and
+// commits each stage's release; warps 2-5 read the 128 x 64 fp32 accumulator
+// back (one TMEM lane quarter each).  When the token tiles do not fill the
+// GPU, the contraction is split over a cluster as in k_rows: the CTAs' fp32
+// sums meet in distributed shared memory and are added in rank order.
+constexpr int RT_BM = 128, RT_N = 64, RT_ST = 6;
+constexpr int RT_P = RT_BM * 64 * 2;                    // X tile, 16 KB
+constexpr int RT_Q = RT_N * 64 * 2;                     // A or B tile, 8 KB
+constexpr int RT_OFF_Q = RT_ST * RT_P;
+constexpr int RT_OFF_PART = RT_OFF_Q + RT_ST * RT_Q;    // fp32 [128][64], 16-byte chunks XOR-swizzled by row
+constexpr int RT_OFF_BAR = RT_OFF_PART + RT_BM * RT_N * 4;
+constexpr int RT_BYTES = RT_OFF_BAR + (2 * RT_ST + 3) * 8 + 1024;
+constexpr int RT_THREADS = 192;
+
+// part[ml][j]: chunk j / 4 of row ml stored at chunk (j / 4) ^ (ml & 15), so that
+// a quarter-warp's 16-byte stores (8 rows, one chunk) and a warp's reads of 32
+// consecutive j of one row both touch distinct banks.
+__device__ __forceinline__ uint32_t rt_part(uint32_t part, int ml, int j) {
+  return part + ml * 256 + ((((j >> 2) ^ (ml & 15))) << 4) + (j & 3) * 4;
+}
+
+__device__ __forceinline__ void rows_tc_reduce(uint32_t part, int M, int m0, int split, int nsplit, float sa,
+                                               uint16_t* out16a, float sb, uint16_t* out16b, float* out32) {
+  cluster_sync_all();  // every CTA's partial sums are in its shared memory
+  const int V = RT_BM * RT_N;
+  const int v0 = V * split / nsplit, v1 = V * (split + 1) / nsplit;
+  for (int v = v0 + static_cast<int>(threadIdx.x); v < v1; v += blockDim.x) {
+    const int ml = v >> 6, j = v & 63, m = m0 + ml;
+    const float sum = cluster_sum_ranks(rt_part(part, ml, j), nsplit);
+    if (m >= M) continue;
+    const int64_t o = static_cast<int64_t>(m) * RT_N + j;
+    out16a[o] = static_cast<uint16_t>(bf16x2_bits(sa * sum, 0.f));
+    if (out16b) out16b[o] = static_cast<uint16_t>(bf16x2_bits(sb * sum, 0.f));
+    if (out32) out32[o] = sb * sum;
+  }
+  cluster_sync_all();  // peers keep their shared memory until every read is done
+}
+
+template <bool QT>
+__global__ void __launch_bounds__(RT_THREADS, 1) k_rows_tc(const __grid_constant__ CUtensorMap tmP,
+                                                          const __grid_constant__ CUtensorMap tmQ, int M, int Kc,
+                                                          float sa, uint16_t* __restrict__ out16a, float sb,
+                                                          uint16_t* __restrict__ out16b, float* __restrict__ out32,
+                                                          int nsplit, int* status) {
+  pdl_trigger();
+  pdl_wait();
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  const uint32_t full0 = base + RT_OFF_BAR, empty0 = full0 + 8u * RT_ST;
+  const uint32_t accum_bar = empty0 + 8u * RT_ST, drain_bar = accum_bar + 8u, tmem_slot = drain_bar + 8u;
+  const uint32_t part = base + RT_OFF_PART;
+  __shared__ int abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = nsplit > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int m0 = (blockIdx.x / nsplit) * RT_BM;
+  const int nk_all = (Kc + 63) / 64;
+  const int it0 = static_cast<int>(static_cast<int64_t>(nk_all) * split / nsplit);
+  const int nk = static_cast<int>(static_cast<int64_t>(nk_all) * (split + 1) / nsplit) - it0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < RT_ST; ++s) {
+      mbar_init(full0 + 8u * s, 1);
+      mbar_init(empty0 + 8u * s, 1);
+    }
+    mbar_init(accum_bar, 1);
+    mbar_init(drain_bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, RT_N);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem_raw + (tmem_slot - raw));
+
+  if (warp == 0) {  // TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int it = 0; it < nk; ++it) {
+        const int s = it % RT_ST;
+        if (!wait_bounded(empty0 + 8u * s, ((it / RT_ST) & 1) ^ 1, &abort_flag, status)) break;
+        mbar_arrive_expect_tx(full0 + 8u * s, RT_P + RT_Q);
+        const int kx = (it0 + it) * 64;
+        tma_load_2d(base + s * RT_P, &tmP, full0 + 8u * s, kx, m0);
+        if (QT)
+          tma_load_2d(base + RT_OFF_Q + s * RT_Q, &tmQ, full0 + 8u * s, 0, kx);
+        else
+          tma_load_2d(base + RT_OFF_Q + s * RT_Q, &tmQ, full0 + 8u * s, kx, 0);
+        ++issued;
+      }
+      for (int it = (issued > RT_ST ? issued - RT_ST : 0); it < issued; ++it)  // all copies land before exit
+        wait_drain(full0 + 8u * (it % RT_ST), (it / RT_ST) & 1);
+    }
+  } else if (warp == 1) {  // MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(RT_BM, RT_N, false, QT);
+      bool ok = true, committed = false;
+      for (int it = 0; it < nk; ++it) {
+        const int s = it % RT_ST;
+        if (!(ok = wait_bounded(full0 + 8u * s, (it / RT_ST) & 1, &abort_flag, status))) break;
+        tc_fence_after();
+        const uint32_t p_s = base + s * RT_P, q_s = base + RT_OFF_Q + s * RT_Q;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t bd = QT ? desc_sw128(q_s + kk * 2048, 8192, 1024) : desc_sw128(q_s + kk * 32, 16, 1024);
+          tc_mma_f16(tmem, desc_sw128(p_s + kk * 32, 16, 1024), bd, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(empty0 + 8u * s);  // the slot is free once these MMAs have read it
+        committed = true;
+      }
+      if (ok) {
+        tc_commit(accum_bar);
+      } else if (committed) {  // MMAs in flight finish before TMEM is freed
+        tc_commit(drain_bar);
+        wait_drain(drain_bar, 0);
+      }
+    }
+  } else {  // warps 2-5: the accumulator back from TMEM (lanes 32 (warp % 4) ..)
+    if (wait_bounded(accum_bar, 0, &abort_flag, status)) {
+      tc_fence_after();
+      const int qd = warp & 3, ml = 32 * qd + lane;
+      uint32_t v[2][32];
+      tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * qd) << 16), v[0]);
+      tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * qd) << 16) + 32u, v[1]);
+      tmem_ld_wait();
+      if (nsplit > 1) {
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          st_shared_v4(rt_part(part, ml, 4 * c), v[c >> 3][(c & 7) * 4], v[c >> 3][(c & 7) * 4 + 1],
+                       v[c >> 3][(c & 7) * 4 + 2], v[c >> 3][(c & 7) * 4 + 3]);
+      } else if (m0 + ml < M) {
+        const int64_t o = static_cast<int64_t>(m0 + ml) * RT_N;
+        auto f = [&](int j) { return __uint_as_float(v[j >> 5][j & 31]); };
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4 a, b;
+          a.x = bf16x2_bits(sa * f(8 * c), sa * f(8 * c + 1));
+          a.y = bf16x2_bits(sa * f(8 * c + 2), sa * f(8 * c + 3));
+          a.z = bf16x2_bits(sa * f(8 * c + 4), sa * f(8 * c + 5));
+          a.w = bf16x2_bits(sa * f(8 * c + 6), sa * f(8 * c + 7));
+          reinterpret_cast<uint4*>(out16a + o)[c] = a;
+          if (out16b) {
+            b.x = bf16x2_bits(sb * f(8 * c), sb * f(8 * c + 1));
+            b.y = bf16x2_bits(sb * f(8 * c + 2), sb * f(8 * c + 3));
+            b.z = bf16x2_bits(sb * f(8 * c + 4), sb * f(8 * c + 5));
+            b.w = bf16x2_bits(sb * f(8 * c + 6), sb * f(8 * c + 7));
+            reinterpret_cast<uint4*>(out16b + o)[c] = b;
+          }
+          if (out32) {
+            reinterpret_cast<float4*>(out32 + o)[2 * c] =
+                make_float4(sb * f(8 * c), sb * f(8 * c + 1), sb * f(8 * c + 2), sb * f(8 * c + 3));
+            reinterpret_cast<float4*>(out32 + o)[2 * c + 1] =
+                make_float4(sb * f(8 * c + 4), sb * f(8 * c + 5), sb * f(8 * c + 6), sb * f(8 * c + 7));
+          }
+        }
+      }
+    }
+  }
+  // every TMEM read is done before the columns are freed
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, RT_N);
+  }
+  if (nsplit > 1) rows_tc_reduce(part, M, m0, split, nsplit, sa, out16a, sb, out16b, out32);
+}
+
 // ------------------------------------------------------------------ cols
 //
 // out = bf16(scale * D), D[c, j] = sum_m P[m, c] G[m, j] (contraction over
@@ -775,8 +955,53 @@ cudaError_t rows_launch(const uint16_t* P, const uint16_t* Q, int64_t M, int64_t
 }
 
 template <bool QT>
+cudaError_t rows_tc_launch(const uint16_t* P, const uint16_t* Q, int64_t M, int64_t Kc, float sa, uint16_t* out16a,
+                           float sb, uint16_t* out16b, float* out32, cudaStream_t st, bool pdl) {
+  CUtensorMap tmP, tmQ;
+  const auto BF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  bool ok = make_map(&tmP, BF16, P, Kc, M, Kc * 2, 64, RT_BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (QT)
+    ok = ok && make_map(&tmQ, BF16, Q, RT_N, Kc, RT_N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  else
+    ok = ok && make_map(&tmQ, BF16, Q, Kc, RT_N, Kc * 2, 64, RT_N, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return cudaErrorInvalidValue;
+  cudaError_t e = smem_limit_once<k_rows_tc<QT>>(RT_BYTES);
+  if (e != cudaSuccess) return e;
+  const int64_t tiles = (M + RT_BM - 1) / RT_BM;
+  // split the contraction over a cluster while the token tiles leave SMs idle
+  // (one CTA per SM), keeping at least 4 stages per split
+  const int64_t nk = (Kc + 63) / 64;
+  const int64_t want = device_sm_count() / std::max<int64_t>(1, tiles);
+  const int nsplit = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({8, want, nk / 4})));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles * nsplit), 1, 1);
+  cfg.blockDim = dim3(RT_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = RT_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (nsplit > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = static_cast<unsigned>(nsplit);
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, k_rows_tc<QT>, tmP, tmQ, int(M), int(Kc), sa, out16a, sb, out16b, out32, nsplit,
+                            device_status_ptr());
+}
+
+template <bool QT>
 cudaError_t rows_dispatch(const uint16_t* P, const uint16_t* Q, int64_t M, int64_t Kc, int R, float sa,
                           uint16_t* out16a, float sb, uint16_t* out16b, float* out32, cudaStream_t st, bool pdl) {
+  if (R == RT_N) return rows_tc_launch<QT>(P, Q, M, Kc, sa, out16a, sb, out16b, out32, st, pdl);
   switch (nt_for(R)) {
     case 2: return rows_launch<2, QT>(P, Q, M, Kc, R, sa, out16a, sb, out16b, out32, st, pdl);
     case 4: return rows_launch<4, QT>(P, Q, M, Kc, R, sa, out16a, sb, out16b, out32, st, pdl);

@@ -444,6 +444,7 @@ SMALL = [
     (128, 256, 128, 16),
     (200, 264, 320, 16),
     (300, 520, 1024, 64),
+    (700, 264, 4160, 64),    # r = 64 on the tensor-core adapter kernels: uneven stage split, ragged last tile
     (257, 1000, 192, 24),
 ]
 
