@@ -518,14 +518,15 @@ __global__ void __launch_bounds__(32 * (NT + 1)) k_rows(const __grid_constant__ 
 // streamed, more than mma.sync sustains at HBM speed.  A CTA owns 128 tokens
 // (the UMMA M) and a contiguous range of the 64-wide K stages; warp 0's lane 0
 // streams the 128 x 64 tile of X and the 64 x 64 tile of A (K-major) or of B
-// (QT: [Kc, 64] read in place, MN-major) through an RT_ST-deep TMA ring;
+// (QT: [Kc, 64] read in place, MN-major) through a 3-deep TMA ring (two CTAs
+// per SM);
 // warp 1 allocates 64 TMEM columns and its lane 0 issues
 // tcgen05.mma.cta_group::1 (M = 128, N = 64, K = 16, four per stage) and
 // commits each stage's release; warps 2-5 read the 128 x 64 fp32 accumulator
 // back (one TMEM lane quarter each).  When the token tiles do not fill the
 // GPU, the contraction is split over a cluster as in k_rows: the CTAs' fp32
 // sums meet in distributed shared memory and are added in rank order.
-constexpr int RT_BM = 128, RT_N = 64, RT_ST = 6;
+constexpr int RT_BM = 128, RT_N = 64, RT_ST = 3;  // two CTAs fit an SM
 constexpr int RT_P = RT_BM * 64 * 2;                    // X tile, 16 KB
 constexpr int RT_Q = RT_N * 64 * 2;                     // A or B tile, 8 KB
 constexpr int RT_OFF_Q = RT_ST * RT_P;
@@ -559,7 +560,7 @@ __device__ __forceinline__ void rows_tc_reduce(uint32_t part, int M, int m0, int
 }
 
 template <bool QT>
-__global__ void __launch_bounds__(RT_THREADS, 1) k_rows_tc(const __grid_constant__ CUtensorMap tmP,
+__global__ void __launch_bounds__(RT_THREADS, 2) k_rows_tc(const __grid_constant__ CUtensorMap tmP,
                                                           const __grid_constant__ CUtensorMap tmQ, int M, int Kc,
                                                           float sa, uint16_t* __restrict__ out16a, float sb,
                                                           uint16_t* __restrict__ out16b, float* __restrict__ out32,
@@ -969,9 +970,9 @@ cudaError_t rows_tc_launch(const uint16_t* P, const uint16_t* Q, int64_t M, int6
   if (e != cudaSuccess) return e;
   const int64_t tiles = (M + RT_BM - 1) / RT_BM;
   // split the contraction over a cluster while the token tiles leave SMs idle
-  // (one CTA per SM), keeping at least 4 stages per split
+  // (two CTAs per SM), keeping at least 4 stages per split
   const int64_t nk = (Kc + 63) / 64;
-  const int64_t want = device_sm_count() / std::max<int64_t>(1, tiles);
+  const int64_t want = 2 * device_sm_count() / std::max<int64_t>(1, tiles);
   const int nsplit = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({8, want, nk / 4})));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(tiles * nsplit), 1, 1);
