@@ -692,6 +692,171 @@ __global__ void __launch_bounds__(RT_THREADS, 2) k_rows_tc(const __grid_constant
   if (nsplit > 1) rows_tc_reduce(part, M, m0, split, nsplit, sa, out16a, sb, out16b, out32);
 }
 
+// ---------------------------------------------------- cols on tcgen05, r = 64
+//
+// dA = dH^T X (out [64, C]) and dB = s dY^T H (transpose: out [C, 64]) for
+// r = 64 on the tensor cores: D[c][j] = sum_m P[m][c] G[m][j] with the
+// columns c as the UMMA M (128 per CTA) and j as N = 64.  Per stage 64 tokens:
+// P arrives as two 64 x 64 boxes (the A operand, MN-major: c contiguous) and
+// G as one 64 x 64 box (the B operand, MN-major: j contiguous).  Roles as in
+// k_rows_tc; the tokens are split over a cluster and the fp32 sums meet in
+// distributed shared memory, laid out so that the reduction reads runs of
+// consecutive words in the output's order: [c][j] (row-swizzled) for the
+// transposed dB, [j][c] for dA.
+constexpr int CT_BN = 128, CT_ST = 3;
+constexpr int CT_P = 64 * CT_BN * 2;                    // 64 tokens x 128 columns, 16 KB
+constexpr int CT_G = 64 * RT_N * 2;                     // 64 tokens x 64, 8 KB
+constexpr int CT_OFF_G = CT_ST * CT_P;
+constexpr int CT_OFF_PART = CT_OFF_G + CT_ST * CT_G;   // fp32, 128 x 64
+constexpr int CT_OFF_BAR = CT_OFF_PART + CT_BN * RT_N * 4;
+constexpr int CT_BYTES = CT_OFF_BAR + (2 * CT_ST + 3) * 8 + 1024;
+
+__global__ void __launch_bounds__(RT_THREADS, 2) k_cols_tc(const __grid_constant__ CUtensorMap tmP,
+                                                          const __grid_constant__ CUtensorMap tmG, int M, int C,
+                                                          float scale, int transpose, uint16_t* __restrict__ out,
+                                                          int nsplit, int* status) {
+  pdl_trigger();
+  pdl_wait();
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  const uint32_t full0 = base + CT_OFF_BAR, empty0 = full0 + 8u * CT_ST;
+  const uint32_t accum_bar = empty0 + 8u * CT_ST, drain_bar = accum_bar + 8u, tmem_slot = drain_bar + 8u;
+  const uint32_t part = base + CT_OFF_PART;
+  __shared__ int abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = nsplit > 1 ? static_cast<int>(cluster_ctarank()) : 0;
+  const int c0 = (blockIdx.x / nsplit) * CT_BN;
+  const int ns_all = (M + 63) / 64;  // 64-token slabs
+  const int it0 = static_cast<int>(static_cast<int64_t>(ns_all) * split / nsplit);
+  const int nk = static_cast<int>(static_cast<int64_t>(ns_all) * (split + 1) / nsplit) - it0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < CT_ST; ++s) {
+      mbar_init(full0 + 8u * s, 1);
+      mbar_init(empty0 + 8u * s, 1);
+    }
+    mbar_init(accum_bar, 1);
+    mbar_init(drain_bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, RT_N);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem_raw + (tmem_slot - raw));
+
+  if (warp == 0) {  // TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int it = 0; it < nk; ++it) {
+        const int s = it % CT_ST;
+        if (!wait_bounded(empty0 + 8u * s, ((it / CT_ST) & 1) ^ 1, &abort_flag, status)) break;
+        mbar_arrive_expect_tx(full0 + 8u * s, CT_P + CT_G);
+        const int m = (it0 + it) * 64;
+        tma_load_2d(base + s * CT_P, &tmP, full0 + 8u * s, c0, m);
+        tma_load_2d(base + s * CT_P + 8192, &tmP, full0 + 8u * s, c0 + 64, m);
+        tma_load_2d(base + CT_OFF_G + s * CT_G, &tmG, full0 + 8u * s, 0, m);
+        ++issued;
+      }
+      for (int it = (issued > CT_ST ? issued - CT_ST : 0); it < issued; ++it)  // all copies land before exit
+        wait_drain(full0 + 8u * (it % CT_ST), (it / CT_ST) & 1);
+    }
+  } else if (warp == 1) {  // MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(CT_BN, RT_N, true, true);
+      bool ok = true, committed = false;
+      for (int it = 0; it < nk; ++it) {
+        const int s = it % CT_ST;
+        if (!(ok = wait_bounded(full0 + 8u * s, (it / CT_ST) & 1, &abort_flag, status))) break;
+        tc_fence_after();
+        const uint32_t p_s = base + s * CT_P, g_s = base + CT_OFF_G + s * CT_G;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)  // 16 tokens per MMA
+          tc_mma_f16(tmem, desc_sw128(p_s + kk * 2048, 8192, 1024), desc_sw128(g_s + kk * 2048, 8192, 1024), idesc,
+                     (it > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(empty0 + 8u * s);
+        committed = true;
+      }
+      if (ok) {
+        tc_commit(accum_bar);
+      } else if (committed) {
+        tc_commit(drain_bar);
+        wait_drain(drain_bar, 0);
+      }
+    }
+  } else {  // warps 2-5: TMEM lane (column) 32 (warp % 4) + lane
+    if (wait_bounded(accum_bar, 0, &abort_flag, status)) {
+      tc_fence_after();
+      const int qd = warp & 3, cl = 32 * qd + lane, c = c0 + cl;
+      uint32_t v[2][32];
+      tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * qd) << 16), v[0]);
+      tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(32 * qd) << 16) + 32u, v[1]);
+      tmem_ld_wait();
+      auto f = [&](int j) { return __uint_as_float(v[j >> 5][j & 31]); };
+      if (nsplit > 1) {
+        if (transpose) {
+#pragma unroll
+          for (int q = 0; q < 16; ++q)
+            st_shared_v4(rt_part(part, cl, 4 * q), v[q >> 3][(q & 7) * 4], v[q >> 3][(q & 7) * 4 + 1],
+                         v[q >> 3][(q & 7) * 4 + 2], v[q >> 3][(q & 7) * 4 + 3]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < RT_N; ++j)
+            asm volatile("st.shared.f32 [%0], %1;" ::"r"(part + (j * CT_BN + cl) * 4), "f"(f(j)) : "memory");
+        }
+      } else if (c < C) {
+        if (transpose) {
+          uint4* dst = reinterpret_cast<uint4*>(out + static_cast<int64_t>(c) * RT_N);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dst[q] = make_uint4(bf16x2_bits(scale * f(8 * q), scale * f(8 * q + 1)),
+                                bf16x2_bits(scale * f(8 * q + 2), scale * f(8 * q + 3)),
+                                bf16x2_bits(scale * f(8 * q + 4), scale * f(8 * q + 5)),
+                                bf16x2_bits(scale * f(8 * q + 6), scale * f(8 * q + 7)));
+        } else {
+#pragma unroll
+          for (int j = 0; j < RT_N; ++j)
+            out[static_cast<int64_t>(j) * C + c] = static_cast<uint16_t>(bf16x2_bits(scale * f(j), 0.f));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, RT_N);
+  }
+  if (nsplit > 1) {
+    cluster_sync_all();  // every CTA's partial sums are in its shared memory
+    const int V = CT_BN * RT_N;
+    const int v0 = V * split / nsplit, v1 = V * (split + 1) / nsplit;
+    for (int v = v0 + static_cast<int>(threadIdx.x); v < v1; v += blockDim.x) {
+      int cl, j;
+      uint32_t off;
+      if (transpose) {
+        cl = v >> 6;
+        j = v & 63;
+        off = rt_part(part, cl, j);
+      } else {
+        j = v >> 7;
+        cl = v & 127;
+        off = part + (j * CT_BN + cl) * 4;
+      }
+      const float sum = cluster_sum_ranks(off, nsplit);
+      const int c = c0 + cl;
+      if (c >= C) continue;
+      const int64_t o = transpose ? static_cast<int64_t>(c) * RT_N + j : static_cast<int64_t>(j) * C + c;
+      out[o] = static_cast<uint16_t>(bf16x2_bits(scale * sum, 0.f));
+    }
+    cluster_sync_all();  // peers keep their shared memory until every read is done
+  }
+}
+
 // ------------------------------------------------------------------ cols
 //
 // out = bf16(scale * D), D[c, j] = sum_m P[m, c] G[m, j] (contraction over
@@ -1103,9 +1268,49 @@ cudaError_t launch_rowdot_qt(const uint16_t* P, const uint16_t* Qt, int64_t M, i
   return rows_dispatch<true>(P, Qt, M, Kc, R, sa, out16a, sb, out16b, out32, st, pdl);
 }
 
+static cudaError_t cols_tc_launch(const uint16_t* G, const uint16_t* P, int64_t M, int64_t C, float scale, int transpose,
+                           uint16_t* out, cudaStream_t st, bool pdl) {
+  CUtensorMap tmP, tmG;
+  const auto BF16 = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  bool ok = make_map(&tmP, BF16, P, C, M, C * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok = ok && make_map(&tmG, BF16, G, RT_N, M, RT_N * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return cudaErrorInvalidValue;
+  cudaError_t e = smem_limit_once<k_cols_tc>(CT_BYTES);
+  if (e != cudaSuccess) return e;
+  const int64_t tiles = (C + CT_BN - 1) / CT_BN, nslab = (M + 63) / 64;
+  // split the tokens over a cluster while the column tiles leave SMs idle
+  // (two CTAs per SM), keeping at least 4 slabs per split
+  const int64_t want = 2 * device_sm_count() / std::max<int64_t>(1, tiles);
+  const int nsplit = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({8, want, nslab / 4})));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles * nsplit), 1, 1);
+  cfg.blockDim = dim3(RT_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = CT_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (nsplit > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = static_cast<unsigned>(nsplit);
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, k_cols_tc, tmP, tmG, int(M), int(C), scale, transpose, out, nsplit,
+                            device_status_ptr());
+}
+
 cudaError_t launch_coldot(const uint16_t* G, const uint16_t* P, int64_t M, int64_t C, int R, float scale,
                           int transpose, uint16_t* out, cudaStream_t st, bool pdl) {
   if (M == 0) return cudaMemsetAsync(out, 0, sizeof(uint16_t) * static_cast<size_t>(R) * C, st);
+  if (R == RT_N) return cols_tc_launch(G, P, M, C, scale, transpose, out, st, pdl);
   switch (nt_for(R)) {
     case 2: return cols_launch<2>(G, P, M, C, R, scale, transpose, out, st, pdl);
     case 4: return cols_launch<4>(G, P, M, C, R, scale, transpose, out, st, pdl);
