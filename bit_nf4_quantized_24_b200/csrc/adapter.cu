@@ -3,10 +3,13 @@
 //   forward     H = X A^T                   (rowdot, contraction over K)
 //   backward    dH = s dY B                 (rowdot over N, B read in place)
 //               dA = dH^T X, dB = s dY^T H  (coldot, contraction over tokens)
-// These are skinny (r <= 64 outputs per token) and bound by reading X or dY
-// once: a single thread streams tiles with TMA through a deep shared-memory
-// ring and the consumer warps run ldmatrix + mma.sync on swizzled tiles
-// (r is too narrow for a full tcgen05 tile).
+// These are skinny (r <= 64 outputs per token) and meant to be bound by
+// reading X or dY once: a single thread streams tiles with TMA through a
+// shared-memory ring.  For r = 64 (64 FLOP per byte streamed) the products
+// run on tcgen05 (k_rows_tc, k_cols_tc: 128 tokens or columns as the UMMA M,
+// r as N, the accumulator in TMEM); for smaller r, and for the dropout's
+// masked inputs, consumer warps run ldmatrix + mma.sync on the swizzled tiles
+// (k_rows, k_cols).
 #include <algorithm>
 
 #include "internal.h"
