@@ -321,6 +321,30 @@ __device__ __forceinline__ float cluster_sum_ranks(uint32_t off, int n) {
   return sum;
 }
 
+// The same for four consecutive fp32 words (16-byte aligned) per rank.
+__device__ __forceinline__ float4 cluster_sum_ranks4(uint32_t off, int n) {
+  float4 x[8];
+#pragma unroll
+  for (int rk = 0; rk < 8; ++rk) {
+    x[rk] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (rk < n)
+      asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                   : "=f"(x[rk].x), "=f"(x[rk].y), "=f"(x[rk].z), "=f"(x[rk].w)
+                   : "r"(mapa_shared(off, rk))
+                   : "memory");
+  }
+  float4 sum = x[0];
+#pragma unroll
+  for (int rk = 1; rk < 8; ++rk)
+    if (rk < n) {
+      sum.x += x[rk].x;
+      sum.y += x[rk].y;
+      sum.z += x[rk].z;
+      sum.w += x[rk].w;
+    }
+  return sum;
+}
+
 // The cluster's reduction of k_rows with a split contraction: every thread of
 // every CTA arrives (the producer warp too); then CTA `split` writes outputs
 // [V split / nsplit, V (split + 1) / nsplit) of the tile's V = 16 CW x R, each
@@ -548,16 +572,20 @@ __device__ __forceinline__ uint32_t rt_part(uint32_t part, int ml, int j) {
 __device__ __forceinline__ void rows_tc_reduce(uint32_t part, int M, int m0, int split, int nsplit, float sa,
                                                uint16_t* out16a, float sb, uint16_t* out16b, float* out32) {
   cluster_sync_all();  // every CTA's partial sums are in its shared memory
-  const int V = RT_BM * RT_N;
-  const int v0 = V * split / nsplit, v1 = V * (split + 1) / nsplit;
+  // four consecutive outputs (one 16-byte chunk of a row) per thread and step
+  const int V4 = RT_BM * RT_N / 4;
+  const int v0 = V4 * split / nsplit, v1 = V4 * (split + 1) / nsplit;
   for (int v = v0 + static_cast<int>(threadIdx.x); v < v1; v += blockDim.x) {
-    const int ml = v >> 6, j = v & 63, m = m0 + ml;
-    const float sum = cluster_sum_ranks(rt_part(part, ml, j), nsplit);
+    const int ml = v >> 4, j = (v & 15) * 4, m = m0 + ml;
+    const float4 sum = cluster_sum_ranks4(rt_part(part, ml, j), nsplit);
     if (m >= M) continue;
     const int64_t o = static_cast<int64_t>(m) * RT_N + j;
-    out16a[o] = static_cast<uint16_t>(bf16x2_bits(sa * sum, 0.f));
-    if (out16b) out16b[o] = static_cast<uint16_t>(bf16x2_bits(sb * sum, 0.f));
-    if (out32) out32[o] = sb * sum;
+    *reinterpret_cast<uint2*>(out16a + o) =
+        make_uint2(bf16x2_bits(sa * sum.x, sa * sum.y), bf16x2_bits(sa * sum.z, sa * sum.w));
+    if (out16b)
+      *reinterpret_cast<uint2*>(out16b + o) =
+          make_uint2(bf16x2_bits(sb * sum.x, sb * sum.y), bf16x2_bits(sb * sum.z, sb * sum.w));
+    if (out32) *reinterpret_cast<float4*>(out32 + o) = make_float4(sb * sum.x, sb * sum.y, sb * sum.z, sb * sum.w);
   }
   cluster_sync_all();  // peers keep their shared memory until every read is done
 }
@@ -836,25 +864,25 @@ __global__ void __launch_bounds__(RT_THREADS, 2) k_cols_tc(const __grid_constant
   }
   if (nsplit > 1) {
     cluster_sync_all();  // every CTA's partial sums are in its shared memory
-    const int V = CT_BN * RT_N;
-    const int v0 = V * split / nsplit, v1 = V * (split + 1) / nsplit;
+    // four consecutive outputs per thread and step: j .. j + 3 of one column (dB)
+    // or columns cl .. cl + 3 of one j (dA)
+    const int V4 = CT_BN * RT_N / 4;
+    const int v0 = V4 * split / nsplit, v1 = V4 * (split + 1) / nsplit;
     for (int v = v0 + static_cast<int>(threadIdx.x); v < v1; v += blockDim.x) {
-      int cl, j;
-      uint32_t off;
       if (transpose) {
-        cl = v >> 6;
-        j = v & 63;
-        off = rt_part(part, cl, j);
+        const int cl = v >> 4, j = (v & 15) * 4, c = c0 + cl;
+        const float4 sum = cluster_sum_ranks4(rt_part(part, cl, j), nsplit);
+        if (c >= C) continue;
+        *reinterpret_cast<uint2*>(out + static_cast<int64_t>(c) * RT_N + j) =
+            make_uint2(bf16x2_bits(scale * sum.x, scale * sum.y), bf16x2_bits(scale * sum.z, scale * sum.w));
       } else {
-        j = v >> 7;
-        cl = v & 127;
-        off = part + (j * CT_BN + cl) * 4;
+        const int j = v >> 5, cl = (v & 31) * 4, c = c0 + cl;
+        const float4 sum = cluster_sum_ranks4(part + (j * CT_BN + cl) * 4, nsplit);
+        const float w[4] = {sum.x, sum.y, sum.z, sum.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (c + q < C) out[static_cast<int64_t>(j) * C + c + q] = static_cast<uint16_t>(bf16x2_bits(scale * w[q], 0.f));
       }
-      const float sum = cluster_sum_ranks(off, nsplit);
-      const int c = c0 + cl;
-      if (c >= C) continue;
-      const int64_t o = transpose ? static_cast<int64_t>(c) * RT_N + j : static_cast<int64_t>(j) * C + c;
-      out[o] = static_cast<uint16_t>(bf16x2_bits(scale * sum, 0.f));
     }
     cluster_sync_all();  // peers keep their shared memory until every read is done
   }
