@@ -57,7 +57,7 @@ WORKLOAD = "layer_70b"
 # dram__bytes_write.sum; the summary and the command are in
 # profiles/layer_70b_step_launch_list.md).  Valid only for the kernel source it
 # was taken on (sha256 prefix of gemm_tc.cu); reported as null otherwise.
-GEMM_TRAFFIC = {"gemm_tc_sha16": "fa327ba0a3245d6e", "bytes_per_launch": 509404818}
+GEMM_TRAFFIC = {"gemm_tc_sha16": "fa327ba0a3245d6e", "bytes_per_launch": 509550610}
 
 
 def gemm_traffic():
