@@ -90,6 +90,23 @@ def test_workspace_sizes_grow_with_shape(L):
     assert qb.bwd_workspace_bytes(4096, 4096, 4096, 16) > qb.bwd_workspace_bytes(128, 2048, 2048, 8)
 
 
+def test_split_plan_without_a_device(L):
+    """The fused GEMM's split plan needs the device's resident CTA pairs:
+    without a device every tile runs whole and the workspace functions add no
+    room for partial sums; bad arguments are rejected."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("checks the host-only answer")
+    for mode in (0, 1):
+        assert qb.gemm_split_plan(mode, 4096, 1024, 8192) == (1, 0, 0)
+    ns, nt, pb = ctypes.c_int(), ctypes.c_int64(), ctypes.c_size_t()
+    assert L.qlora_gemm_split_plan(2, 4096, 1024, 8192, ctypes.byref(ns), ctypes.byref(nt), ctypes.byref(pb)) == -1
+    assert L.qlora_gemm_split_plan(0, -1, 1024, 8192, None, None, None) == -1
+    assert L.qlora_gemm_split_plan(0, 4096, 1024, 8192, None, None, None) == 0  # NULL outputs allowed
+    M, r = 4096, 64
+    assert qb.fwd_workspace_bytes(M, 1024, 8192, r) == M * r * 2  # Hs only
+
+
 def test_midpoints_avoid_the_quantizer_cell_edges(L):
     """The GPU quantizer finds a code from the 1/64-wide cell that holds
     t = w / absmax (cell edges at odd multiples of 1/128) plus one compare with
