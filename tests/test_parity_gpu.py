@@ -598,6 +598,15 @@ def test_backward_small(qb, oracle, M, N, K, r):
     run_bwd_check(qb, oracle, p, use_saved_h=False)
 
 
+@pytest.mark.parametrize("M,N,K,r", [(5, 264, 1024, 64), (16, 1000, 2048, 64), (3, 72, 320, 16)])
+def test_backward_few_tokens(qb, oracle, M, N, K, r):
+    """The backward at decode-sized token counts (one partly filled token tile
+    in every adapter kernel, the GEMM's single token pair)."""
+    p = wl.draw_small(3500 + M + N + K, M, N, K, r, 2.0 * r)
+    run_bwd_check(qb, oracle, p)
+    run_bwd_check(qb, oracle, p, use_saved_h=False)
+
+
 def test_adapter_isolating_cases(qb, oracle):
     """W = 0 makes Y and dX pure LoRA; a large B makes the adapter dominate."""
     M, N, K, r = 150, 320, 256, 16
